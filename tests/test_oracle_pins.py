@@ -1,0 +1,451 @@
+"""Pins of the CPU oracle to things other than itself (no GPU needed).
+
+Each test checks an oracle function against an independent statement of what the
+PACT pages and the mathematics fix: exact-rational enumeration, closed forms,
+invariants, brute force on tiny inputs, a library routine the oracle does not use,
+and finite differences.  A plausible slip anywhere in the oracle (a dropped term, a
+wrong sign or index, a transposed operand, a wrong tie rule) fails one of them.
+"""
+import bisect
+import os
+from fractions import Fraction
+
+import numpy as np
+import pytest
+
+import synth
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+# ---------------------------------------------------------------- helpers (independent)
+def e4m3_table():
+    """All non-negative finite E4M3 values as exact fractions, from the format
+    definition (bias 7, 3 mantissa bits, subnormals at exponent field 0)."""
+    vals = []
+    for b in range(0x7F):
+        e, m = b >> 3, b & 7
+        v = Fraction(m, 512) if e == 0 else (1 + Fraction(m, 8)) * Fraction(2) ** (e - 7)
+        vals.append(v)
+    return vals
+
+
+E4M3 = e4m3_table()
+
+
+def e4m3_rne_exact(v: Fraction) -> int:
+    """Nearest E4M3 byte to the exact rational v, ties to even, saturate at 448."""
+    if v >= 448:
+        return 0x7E
+    i = bisect.bisect_left(E4M3, v)
+    if i < len(E4M3) and E4M3[i] == v:
+        return i
+    lo, hi = i - 1, i
+    dl, dh = v - E4M3[lo], E4M3[hi] - v
+    if dl < dh:
+        return lo
+    if dh < dl:
+        return hi
+    return lo if lo % 2 == 0 else hi
+
+
+def bf16_bits_value(b):
+    return synth.bf16_bits_to_f64(np.asarray(b))
+
+
+def positive_finite_bf16():
+    bits = np.arange(1, 0x7F80, dtype=np.uint16)   # +denormals .. max finite
+    return bits, bf16_bits_value(bits)
+
+
+# ---------------------------------------------------------------------------- format
+def test_golden_format_facts(orc):
+    facts = {}
+    for line in open(os.path.join(GOLDEN, "nvfp4_format.txt")):
+        line = line.strip()
+        if line and not line.startswith("#"):
+            k, *v = line.split()
+            facts[k] = v
+    grid = [float(v) for v in facts["e2m1_magnitudes"]]
+    assert [orc.e2m1_value(c) for c in range(8)] == grid
+    assert [orc.e2m1_value(8 | c) for c in range(8)] == [-g for g in grid]
+    assert orc.e4m3_value(0x7E) == float(facts["e4m3_max"][0])
+    assert orc.e4m3_value(0x01) == float(facts["e4m3_min_subnormal"][0])
+    # storage budget: codes (4 bit) + one 8-bit scale per block of 16 elements
+    rows, cols = 128, 256
+    x = synth.gaussian_bf16(1, (rows, cols))
+    t = orc.quantize(x)
+    bits = 8 * (t.codes.size + t.scales.size) / (rows * cols)
+    assert bits == float(facts["bits_per_element"][0])
+    assert cols // t.scales.shape[1] == int(facts["block_elements"][0])
+
+
+# ------------------------------------------------------------------ P1 scale function
+def test_scale_exhaustive_against_exact_rationals(orc):
+    """Every finite positive BF16 amax: oracle scale byte == E4M3_RNE_sat(amax/6) with
+    exact rational arithmetic (independent enumeration)."""
+    bits, vals = positive_finite_bf16()
+    blocks = np.zeros((bits.size, 16), dtype=np.uint16)
+    blocks[:, 0] = bits
+    t = orc.quantize(blocks)
+    expect = np.array([e4m3_rne_exact(Fraction(float(v)) / 6) for v in vals], dtype=np.uint8)
+    bad = np.nonzero(t.scales[:, 0] != expect)[0]
+    assert bad.size == 0, (bits[bad[:5]], t.scales[bad[:5], 0], expect[bad[:5]])
+
+
+@pytest.mark.parametrize("amax,byte", [
+    (6.0, 0x38),              # scale 1.0
+    (2688.0, 0x7E),           # 448 exactly
+    (1e30, 0x7E),             # saturates
+    (6 * 2.0 ** -9, 0x01),    # smallest subnormal
+    (6 * 2.0 ** -10, 0x00),   # tie between 0 and 2^-9 -> even (0)
+    (6.375, 0x38),            # 1.0625: tie between 1.0 and 1.125 -> even (1.0)
+    (6.0 * 1.1875, 0x3A),     # 1.1875: tie between 1.125 (0x39) and 1.25 (0x3A) -> even
+])
+def test_scale_anchors(orc, amax, byte):
+    x = np.zeros((1, 16), dtype=np.uint16)
+    x[0, 3] = synth.f64_to_bf16_bits(np.array([amax]))[0]
+    if amax < 1e30:
+        assert bf16_bits_value(x[0, 3]) == amax
+    assert orc.quantize(x).scales[0, 0] == byte
+
+
+# -------------------------------------------------------------- P2 element quantizer
+def _expected_mag(x, s):
+    """E2M1 RNE magnitude code of |x|/s by threshold counting: thresholds are the
+    midpoints of the grid, strict where the lower neighbour is the even code."""
+    a = np.abs(x)
+    return ((a > 0.25 * s).astype(int) + (a >= 0.75 * s) + (a > 1.25 * s) + (a >= 1.75 * s)
+            + (a > 2.5 * s) + (a >= 3.5 * s) + (a > 5.0 * s))
+
+
+def test_element_codes_exhaustive(orc):
+    """For every positive E4M3 scale s and every BF16 x with |x| <= 6s (both signs),
+    in blocks [6s, x, ...] that force the scale to s: codes match threshold counting."""
+    bits, vals = positive_finite_bf16()
+    for sb in range(1, 0x7F):
+        s = float(E4M3[sb])
+        six_s = 6.0 * s
+        head = synth.f64_to_bf16_bits(np.array([six_s]))[0]
+        assert bf16_bits_value(head) == six_s
+        sel = vals <= six_s
+        xb = np.concatenate([bits[sel], bits[sel] | np.uint16(0x8000)])
+        xv = bf16_bits_value(xb)
+        pad = (-xb.size) % 15
+        xb = np.concatenate([xb, np.zeros(pad, dtype=np.uint16)])
+        xv = np.concatenate([xv, np.zeros(pad)])
+        blocks = np.empty((xb.size // 15, 16), dtype=np.uint16)
+        blocks[:, 0] = head
+        blocks[:, 1:] = xb.reshape(-1, 15)
+        t = orc.quantize(blocks)
+        assert np.all(t.scales[:, 0] == sb)
+        codes = np.empty((blocks.shape[0], 16), dtype=np.uint8)
+        codes[:, 0::2] = t.codes & 15
+        codes[:, 1::2] = t.codes >> 4
+        got = codes[:, 1:].reshape(-1)
+        exp = _expected_mag(xv, s) | np.where(xb & 0x8000, 8, 0)
+        assert np.array_equal(got, exp.astype(np.uint8)), sb
+        assert np.all(codes[:, 0] == 7)
+
+
+def test_zero_scale_and_signed_zero(orc):
+    x = np.zeros((2, 16), dtype=np.uint16)
+    x[0, :] = 0x8000                     # -0.0 everywhere
+    x[1, 0] = synth.f64_to_bf16_bits(np.array([-1e-4]))[0]   # amax/6 < 2^-10 -> scale 0
+    t = orc.quantize(x)
+    assert list(t.scales[:, 0]) == [0, 0]
+    assert np.all(t.codes[0] == 0x88)
+    assert t.codes[1, 0] == 0x08 and np.all(t.codes[1, 1:] == 0)
+
+
+# ------------------------------------------------------------------ P3 grid round trip
+def test_grid_round_trip(orc):
+    rng = np.random.default_rng(7)
+    n = 4096
+    codes = rng.integers(0, 16, size=(n, 16))
+    codes[np.arange(n), rng.integers(0, 16, size=n)] = rng.choice([7, 15], size=n)
+    sb = rng.integers(1, 0x7F, size=n)
+    grid = np.array([0, .5, 1, 1.5, 2, 3, 4, 6])
+    s = np.array([float(E4M3[b]) for b in sb])
+    v = np.where(codes & 8, -1.0, 1.0) * grid[codes & 7] * s[:, None]
+    xb = synth.f64_to_bf16_bits(v)
+    assert np.array_equal(bf16_bits_value(xb), v)
+    t = orc.quantize(xb)
+    assert np.array_equal(t.scales[:, 0], sb)
+    packed = (codes[:, 0::2] | (codes[:, 1::2] << 4)).astype(np.uint8)
+    assert np.array_equal(t.codes, packed)
+    assert np.array_equal(orc.dequantize(t), v)
+
+
+def test_dequantized_value_is_a_nearest_grid_point(orc):
+    x = synth.gaussian_bf16(3, (64, 256), std=3.0)
+    t = orc.quantize(x)
+    xv = bf16_bits_value(x)
+    d = orc.dequantize(t)
+    s = np.repeat(np.array([[float(E4M3[b]) for b in row] for row in t.scales]), 16, axis=1)
+    grid = np.array([0, .5, 1, 1.5, 2, 3, 4, 6])
+    cand = np.sign(xv)[..., None] * grid * s[..., None]
+    best = np.min(np.abs(xv[..., None] - cand), axis=-1)
+    assert np.all(np.abs(xv - d) <= best)
+    assert np.all(np.abs(d) <= 6 * s)
+
+
+# ------------------------------------------------------------------------ scale layout
+def test_scale_layout_is_a_padded_bijection(orc):
+    for rows, cols in [(128, 64), (300, 320), (1, 64), (257, 1024)]:
+        nb = cols // 16
+        plain = np.arange(rows * nb, dtype=np.int64).reshape(rows, nb) % 251 + 1
+        packed = orc.pack_scales(plain.astype(np.uint8), rows, cols)
+        assert packed.size == ((rows + 127) // 128 * 128) * ((nb + 3) // 4 * 4)
+        offs = {orc.scale_offset(r, c, cols) for r in range(rows) for c in range(nb)}
+        assert len(offs) == rows * nb and max(offs) < packed.size
+        assert np.count_nonzero(packed) == rows * nb          # padding is zero
+        assert np.array_equal(orc.unpack_scales(packed, rows, cols), plain.astype(np.uint8))
+
+
+def test_scale_layout_chunks_are_contiguous_per_128_rows_and_4_blocks(orc):
+    # one 512-byte chunk holds exactly rows 128i..128i+127 x blocks 4j..4j+3
+    cols = 512
+    for i in range(2):
+        for j in range(cols // 64):
+            offs = sorted(orc.scale_offset(r, c, cols) for r in range(128 * i, 128 * i + 128)
+                          for c in range(4 * j, 4 * j + 4))
+            assert offs == list(range(offs[0], offs[0] + 512)) and offs[0] % 512 == 0
+
+
+# -------------------------------------------------------------------------------- GEMM
+def _decode_py(t, r, c):
+    """Independent pure-Python decode of element (r, c) from the format definition."""
+    byte = int(t.codes[r, c // 2])
+    code = (byte >> 4) if c % 2 else (byte & 15)
+    mag = [0, .5, 1, 1.5, 2, 3, 4, 6][code & 7]
+    sb = int(t.scales[r, c // 16])
+    e, m = sb >> 3, sb & 7
+    s = m * 2.0 ** -9 if e == 0 else (1 + m / 8) * 2.0 ** (e - 7)
+    return (-mag if code & 8 else mag) * s
+
+
+def test_brute_force_8x16x16(orc):
+    """P7: 8 x 16 x 16 NVFP4 GEMM by pure-Python loops over decoded elements."""
+    a = orc.quantize(synth.gaussian_bf16(4, (8, 16)))
+    b = orc.quantize(synth.gaussian_bf16(5, (16, 16), std=0.02))
+    got = orc.nvfp4_gemm(a, b)
+    for m in range(8):
+        for n in range(16):
+            ref = sum(_decode_py(a, m, k) * _decode_py(b, n, k) for k in range(16))
+            assert got[m, n] == ref
+
+
+def test_gemm_matches_numpy(orc):
+    """P8: the oracle's triple loop against numpy's float64 matmul (not used by it)."""
+    rng = np.random.default_rng(1)
+    a = rng.standard_normal((67, 96))
+    b = rng.standard_normal((80, 96))
+    np.testing.assert_allclose(orc.gemm_nt(a, b), a @ b.T, rtol=1e-12, atol=1e-12)
+
+
+def test_dgrad_on_grid_is_exact(orc):
+    """P6: dY on the E2M1 grid with a +-6 in every block quantizes to itself, so the
+    dgrad equals dY . deq(Wb)^T exactly (every product and partial sum is exact)."""
+    rng = np.random.default_rng(2)
+    M, N, K = 40, 64, 48
+    codes = rng.integers(0, 16, size=(M, N))
+    codes[:, ::16] = 7
+    grid = np.array([0, .5, 1, 1.5, 2, 3, 4, 6])
+    dy = np.where(codes & 8, -1.0, 1.0) * grid[codes & 7]
+    dyb = synth.f64_to_bf16_bits(dy)
+    w = synth.weight_bf16(0, (N, K))
+    _, wb = orc.weight_cache(w)
+    got = orc.frozen_dgrad(dyb, wb)
+    assert np.array_equal(got, dy @ orc.dequantize(wb).T)
+
+
+def test_lora_zero_B_reduces_to_frozen(orc):
+    """P5 ([LORA]: h = W0 x + B A x with B = 0 is the frozen projection)."""
+    x = synth.gaussian_bf16(1, (32, 64))
+    w = synth.weight_bf16(0, (48, 64))
+    a = synth.gaussian_bf16(20, (16, 64), std=0.02)
+    wf, wb = orc.weight_cache(w)
+    xq = orc.quantize(x)
+    zero_b = np.zeros((48, 16), dtype=np.uint16)
+    assert np.array_equal(orc.frozen_fwd(xq, wf, x, a, zero_b, 2.0), orc.nvfp4_gemm(xq, wf))
+    dy = synth.gaussian_bf16(50, (32, 48))
+    zero_a = np.zeros((16, 64), dtype=np.uint16)
+    b = synth.gaussian_bf16(30, (48, 16), std=0.02)
+    assert np.array_equal(orc.frozen_dgrad(dy, wb, zero_a, b, 2.0),
+                          orc.nvfp4_gemm(orc.quantize(dy), wb))
+
+
+def test_lora_terms_against_finite_differences(orc):
+    """The LoRA forward term, its input gradient and dA/dB: for the loss
+    L = sum(dY * s (X A^T) B^T), dL/dX = s dY B A, dL/dA = s (dY B)^T X,
+    dL/dB = s dY^T (X A^T).  L is linear in each argument, so central differences
+    are exact up to rounding."""
+    rng = np.random.default_rng(3)
+    M, N, K, r, s = 5, 6, 7, 3, 2.0
+    x = rng.standard_normal((M, K))
+    a = rng.standard_normal((r, K))
+    b = rng.standard_normal((N, r))
+    dy = rng.standard_normal((M, N))
+
+    def loss(x_, a_, b_):
+        return float(np.sum(dy * (s * orc.gemm_nt(orc.gemm_nt(x_, a_), b_))))
+
+    da, db, su = orc.lora_bwd_at(dy, x, a, b, s)
+    h = 1e-3
+    for arr, grad in ((a, da), (b, db)):
+        for idx in np.ndindex(arr.shape):
+            e = np.zeros_like(arr)
+            e[idx] = h
+            args_p = [x, a + e, b] if arr is a else [x, a, b + e]
+            args_m = [x, a - e, b] if arr is a else [x, a, b - e]
+            fd = (loss(*args_p) - loss(*args_m)) / (2 * h)
+            assert abs(fd - grad[idx]) <= 1e-9 * (1 + abs(fd))
+    # dL/dX is the LoRA part of frozen_dgrad: s (dY B) A
+    dx = orc.gemm_nt(su, a.T)
+    for idx in np.ndindex(x.shape):
+        e = np.zeros_like(x)
+        e[idx] = h
+        fd = (loss(x + e, a, b) - loss(x - e, a, b)) / (2 * h)
+        assert abs(fd - dx[idx]) <= 1e-9 * (1 + abs(fd))
+
+
+# ---------------------------------------------------------------- weight layout cache
+def test_weight_cache_transpose_exact_on_grid(orc):
+    """W = +-6 with random signs: every block (along K and along N) has amax 6, so
+    Wf and Wb are exact and deq(Wb) must be exactly deq(Wf)^T."""
+    rng = np.random.default_rng(4)
+    N, K = 48, 80
+    w = np.where(rng.random((N, K)) < 0.5, -6.0, 6.0)
+    wf, wb = orc.weight_cache(synth.f64_to_bf16_bits(w))
+    assert wb.rows == K and wb.cols == N
+    assert np.array_equal(orc.dequantize(wf), w)
+    assert np.array_equal(orc.dequantize(wb), w.T)
+
+
+def test_weight_cache_backward_is_requantized_forward(orc):
+    """Wb re-quantizes deq(Wf)^T along N: its error against deq(Wf)^T is bounded by
+    the nearest-grid property, and it never looks at the original W."""
+    w = synth.weight_bf16(6, (64, 96))
+    wf, wb = orc.weight_cache(w)
+    wd_t = orc.dequantize(wf).T
+    wb2 = orc.quantize(orc.f64_to_bf16_exact(wd_t))
+    assert np.array_equal(wb.codes, wb2.codes) and np.array_equal(wb.scales, wb2.scales)
+    w_other = w.copy()
+    w_other[0, 0] ^= 1     # a change below the NVFP4 resolution of W
+    wf2, wb3 = orc.weight_cache(w_other)
+    if np.array_equal(wf2.codes, wf.codes) and np.array_equal(wf2.scales, wf.scales):
+        assert np.array_equal(wb3.codes, wb.codes)
+
+
+# ----------------------------------------------------------------------------- RMSNorm
+def test_rmsnorm_constant_row_closed_form(orc):
+    H, eps = 64, 1e-5
+    gamma = synth.gaussian_bf16(40, (H,), std=0.02, mean=1.0)
+    g = bf16_bits_value(gamma)
+    for c in (0.5, -3.0, 1e-3, 40.0):
+        x = np.full((1, H), synth.f64_to_bf16_bits(np.array([c]))[0], dtype=np.uint16)
+        cv = float(bf16_bits_value(x[0, 0]))
+        y, yq, rstd = orc.rmsnorm_quant(x, gamma, eps)
+        assert rstd[0] == pytest.approx(1.0 / np.sqrt(cv * cv + eps), rel=1e-15)
+        yv = bf16_bits_value(y[0])
+        ref = cv * g / np.sqrt(cv * cv + eps)
+        assert np.all(np.abs(yv - ref) <= 2.0 ** -8 * np.abs(ref))   # one BF16 rounding
+        assert np.array_equal(orc.quantize(y).codes, yq.codes)
+
+
+def test_rmsnorm_output_is_one_bf16_rounding(orc):
+    x = synth.gaussian_bf16(1, (8, 128))
+    gamma = synth.gaussian_bf16(40, (128,), std=0.02, mean=1.0)
+    y, _, rstd = orc.rmsnorm_quant(x, gamma, 1e-5)
+    xv = bf16_bits_value(x)
+    ref = (xv * rstd[:, None]) * bf16_bits_value(gamma)[None, :]
+    yv = bf16_bits_value(y)
+    # nearest BF16: |y - ref| <= half an ULP of y's binade
+    ulp = 2.0 ** (np.floor(np.log2(np.abs(yv))) - 7)
+    assert np.all(np.abs(yv - ref) <= ulp / 2)
+
+
+def test_rmsnorm_bwd_against_finite_differences(orc):
+    rng = np.random.default_rng(5)
+    M, H, eps = 3, 32, 1e-5
+    x = rng.standard_normal((M, H))
+    gamma = synth.gaussian_bf16(41, (H,), std=0.02, mean=1.0)
+    g = bf16_bits_value(gamma)
+    dy = rng.standard_normal((M, H))
+
+    def fwd(xx):
+        r = 1.0 / np.sqrt(np.mean(xx * xx, axis=1, keepdims=True) + eps)
+        return xx * r * g, r[:, 0]
+
+    y, rstd = fwd(x)
+    dx = orc.rmsnorm_bwd_at(dy, y, rstd, gamma)
+    h = 1e-6
+    for idx in np.ndindex(x.shape):
+        e = np.zeros_like(x)
+        e[idx] = h
+        fd = (np.sum(dy * fwd(x + e)[0]) - np.sum(dy * fwd(x - e)[0])) / (2 * h)
+        assert abs(fd - dx[idx]) <= 1e-7 * (1 + abs(fd))
+
+
+# ------------------------------------------------------------------------ SiLU-multiply
+def test_silu_mul_closed_forms(orc):
+    u = synth.gaussian_bf16(5, (4, 16))
+    g0 = np.zeros_like(u)
+    m, mq, gq, uq = orc.silu_mul_quant(g0, u)
+    assert np.all(bf16_bits_value(m) == 0.0)             # silu(0) = 0
+    big = np.full_like(u, synth.f64_to_bf16_bits(np.array([40.0]))[0])
+    m2, *_ = orc.silu_mul_quant(big, u)
+    assert np.array_equal(m2, synth.f64_to_bf16_bits(40.0 * bf16_bits_value(u)))  # silu(40)=40(1-4e-18)
+    # the NVFP4 copies of gate/up are plain quantizations of the BF16 inputs
+    assert np.array_equal(uq.codes, orc.quantize(u).codes)
+    g = synth.gaussian_bf16(4, (4, 16))
+    m3, *_ = orc.silu_mul_quant(g, u)
+    gv, uv = bf16_bits_value(g), bf16_bits_value(u)
+    ref = gv / (1 + np.exp(-gv)) * uv
+    mv = bf16_bits_value(m3)
+    assert np.all(np.abs(mv - ref) <= 2.0 ** -8 * np.abs(ref) + 1e-300)
+
+
+def test_silu_mul_bwd_against_finite_differences(orc):
+    rng = np.random.default_rng(6)
+    g = rng.standard_normal(200) * 3
+    u = rng.standard_normal(200)
+    dm = rng.standard_normal(200)
+    dg, du = orc.silu_mul_bwd_at(dm, g, u)
+    f = lambda gg, uu: gg / (1 + np.exp(-gg)) * uu
+    h = 1e-6
+    fd_g = dm * (f(g + h, u) - f(g - h, u)) / (2 * h)
+    fd_u = dm * (f(g, u + h) - f(g, u - h)) / (2 * h)
+    np.testing.assert_allclose(dg, fd_g, rtol=1e-6, atol=1e-8)
+    np.testing.assert_allclose(du, fd_u, rtol=1e-6, atol=1e-8)
+
+
+def test_silu_mul_bwd_reads_the_quantized_copies(orc):
+    g = synth.gaussian_bf16(4, (2, 32))
+    u = synth.gaussian_bf16(5, (2, 32))
+    _, _, gq, uq = orc.silu_mul_quant(g, u)
+    dm = np.ones((2, 32))
+    dg, du = orc.silu_mul_bwd(dm, gq, uq)
+    dg2, du2 = orc.silu_mul_bwd_at(dm, orc.dequantize(gq), orc.dequantize(uq))
+    assert np.array_equal(dg, dg2) and np.array_equal(du, du2)
+    m = orc.silu_mul_recompute(gq, uq)
+    gh, uh = orc.dequantize(gq), orc.dequantize(uq)
+    ref = gh / (1 + np.exp(-gh)) * uh
+    assert np.all(np.abs(bf16_bits_value(m) - ref) <= 2.0 ** -8 * np.abs(ref) + 1e-300)
+
+
+# ------------------------------------------------------------------------ BF16 rounding
+def test_bf16_rne_ties_and_subnormals(orc):
+    one = 1.0
+    assert orc.bf16_rne(one + 2.0 ** -8) == 0x3F80          # tie -> even (1.0)
+    assert orc.bf16_rne(one + 3 * 2.0 ** -8) == 0x3F82      # tie -> even (1 + 2^-6)
+    assert orc.bf16_rne(one + 2.0 ** -8 + 2.0 ** -40) == 0x3F81
+    assert orc.bf16_rne(-2.0 ** -133) == 0x8001             # smallest subnormal
+    assert orc.bf16_rne(2.0 ** -134) == 0x0000              # tie -> even (0)
+    assert orc.bf16_rne(3 * 2.0 ** -134) == 0x0002
+    # against float32 rounding for values whose float32 conversion is exact
+    rng = np.random.default_rng(8)
+    v = rng.standard_normal(2000).astype(np.float32).astype(np.float64)
+    got = np.array([orc.bf16_rne(float(t)) for t in v], dtype=np.uint16)
+    assert np.array_equal(got, synth.f64_to_bf16_bits(v))
