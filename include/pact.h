@@ -1,0 +1,269 @@
+/*
+ * pact.h -- C ABI of libpact: the NVFP4 data flow through the seven frozen
+ * projections of a LoRA decoder layer (PACT), for NVIDIA B200 (sm_100a).
+ *
+ * What each call computes is defined by the PACT pages:
+ *   [FAQ]    PACT blog summary (simolm.com), section "相关问题" (FAQ), answer on
+ *            NVFP4: 16 E2M1 values share one E4M3 block scale, ~4.5 bit/element.
+ *   [METHOD] same page, section "方法" (method): bullet 1, NVFP4 GEMMs with FP32
+ *            accumulation and BF16 output for the forward and the input gradient of
+ *            the 7 frozen projections; bullet 2, the quantized RMSNorm output is
+ *            reused for backward and SiLU-multiply keeps BF16 in forward while
+ *            saving NVFP4 copies of gate/up; bullet 4, quantization fused into
+ *            RMSNorm and SiLU-multiply, forward and backward weight layouts rebuilt,
+ *            transposed, re-quantized and cached; the paragraph after the bullets,
+ *            LoRA A and B stay BF16.
+ *   [ABS]    PACT abstract (arxiv.science page): the same data flow.
+ *   [LORA]   PEFT explainer (kongchang.com), section "LoRA": h = W0 x + B A x.
+ *
+ * Conventions shared by every call
+ * --------------------------------
+ * Numbers.  NVFP4 quantization of a block of 16 BF16 values x_i:
+ *   scale byte  s = E4M3_RNE(amax / 6), saturating at 448 (never the NaN byte);
+ *   element     c_i = sign(x_i) << 3 | E2M1_RNE(|x_i| / s), saturating at 6, ties to
+ *               the even code, magnitude 0 when s == 0; the sign bit is kept even
+ *               when the magnitude rounds to 0.
+ *   value       E2M1(c_i) * E4M3(s), exact in FP32 and BF16.
+ * Storage (pact_nvfp4_t).  Blocks run along the last dimension ("cols").  codes:
+ *   rows x cols/2 bytes, row-major, element 2j in the low nibble of byte j.
+ *   scales: pact_scale_bytes(rows, cols) bytes in 512-byte tiles of 128 rows x 4
+ *   blocks; tiles are row-tile-major; inside a tile (row r, block c) is at byte
+ *   (r % 32) * 16 + ((r % 128) / 32) * 4 + (c % 4).  Rows pad to 128 with zero bytes.
+ *   No per-tensor second-level scale exists (4 bits + 8/16 bits = 4.5 bit/element).
+ * Shapes.  cols of every NVFP4 tensor is a multiple of 64; rows >= 1 is free.
+ *   Frozen weights are [N x K] (PyTorch [out, in]); N and K are multiples of 64.
+ * Pointers.  Every pointer argument is DEVICE memory unless stated, 16-byte
+ *   aligned; leading dimensions (ld*) are in elements and make each row start
+ *   16-byte aligned.  The caller owns every buffer; libpact never allocates,
+ *   frees or synchronises (except pact_get_device_status, which says so).
+ * Streams.  Every call enqueues asynchronously on `stream` (a cudaStream_t; NULL
+ *   is the legacy default stream) and returns once the work is enqueued.
+ * Errors.  Arguments are checked on the host before anything is enqueued: a bad
+ *   shape returns PACT_ERR_SHAPE, a misaligned pointer or leading dimension
+ *   PACT_ERR_ALIGN, a NULL required pointer PACT_ERR_INVALID_ARG; nothing is
+ *   launched then.  A failed launch returns PACT_ERR_CUDA.  Kernels bound every
+ *   wait; a wait that runs out records PACT_ERR_TIMEOUT in a per-device status
+ *   word read by pact_get_device_status.  pact_last_error() gives the message of
+ *   the last failing call on the calling thread.
+ */
+#ifndef PACT_H
+#define PACT_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define PACT_ABI_VERSION 1
+
+#if defined(__GNUC__)
+#define PACT_API __attribute__((visibility("default")))
+#else
+#define PACT_API
+#endif
+
+typedef struct CUstream_st *pact_stream_t; /* cudaStream_t */
+typedef uint16_t pact_bf16;                /* BF16 bit pattern */
+
+typedef enum {
+    PACT_OK = 0,
+    PACT_ERR_INVALID_ARG = 1,
+    PACT_ERR_SHAPE = 2,
+    PACT_ERR_ALIGN = 3,
+    PACT_ERR_CUDA = 4,
+    PACT_ERR_TIMEOUT = 5,
+    PACT_ERR_UNSUPPORTED = 6
+} pact_status;
+
+/* An NVFP4 tensor [rows x cols], blocks of 16 along cols (layout above).  The
+ * struct itself is host memory; codes and scales point to device memory. */
+typedef struct {
+    void *codes;
+    void *scales;
+    int64_t rows, cols;
+} pact_nvfp4_t;
+
+/* The two cached layouts of one frozen weight W [N x K] ([METHOD] bullet 4):
+ * fwd = q(W) [N x K] along K; bwd = q(deq(fwd)^T) [K x N] along N. */
+typedef struct {
+    pact_nvfp4_t fwd;
+    pact_nvfp4_t bwd;
+} pact_weight_cache_t;
+
+/* The LoRA branch fused into a frozen GEMM ([LORA]; [METHOD]: A, B in BF16).
+ * Several projections that share an input can be concatenated along N (q|k|v,
+ * gate|up): segment i covers output columns [seg_end[i-1], seg_end[i]) and has
+ * its own rank-r adapter.
+ *   Forward  (pact_frozen_gemm_fwd):   act = T [M x nseg*r], T = scale * X A^T as
+ *     written by pact_lora_fwd (segment i uses columns i*r .. i*r+r-1);
+ *     weight = B [N x r] (segments' B stacked along rows); adds act_i . B_i^T.
+ *   Dgrad    (pact_frozen_gemm_dgrad): act = U [M x nseg*r], U = scale * dY B as
+ *     written by pact_lora_bwd_u; weight = A [nseg*r x K] (segments' A stacked
+ *     along rows); adds U . A (one contraction over nseg*r).
+ * r is 16, 32, 48 or 64; nseg*r <= 64; nseg <= 4; every internal boundary
+ * seg_end[0..nseg-2] is a multiple of 256 and seg_end[nseg-1] == N.  act and
+ * weight are row-major with leading dimension ld_act / ld_weight (elements). */
+typedef struct {
+    const pact_bf16 *act;
+    int64_t ld_act;
+    const pact_bf16 *weight;
+    int64_t ld_weight;
+    int r;
+    int nseg;
+    int64_t seg_end[4];
+} pact_lora_t;
+
+/* ---------------------------------------------------------------- sizes */
+/* Bytes of the codes of an NVFP4 [rows x cols] tensor: rows * cols / 2. */
+PACT_API size_t pact_nvfp4_code_bytes(int64_t rows, int64_t cols);
+/* Bytes of its scales: round_up(rows, 128) * round_up(cols / 16, 4). */
+PACT_API size_t pact_scale_bytes(int64_t rows, int64_t cols);
+/* Bytes of the buffer pact_weight_layout_cache fills for W [N x K]: both
+ * layouts, each part 256-byte aligned. */
+PACT_API size_t pact_weight_cache_bytes(int64_t N, int64_t K);
+
+/* ------------------------------------------------------- A2: quantize */
+/* NVFP4 quantization of x [rows x cols] BF16 (row stride ldx) along cols
+ * ([FAQ]; [METHOD] bullet 4: used for the attention output feeding o and for
+ * every upstream gradient before its dgrad).  out->rows/cols must equal
+ * rows/cols; out->codes/scales are written (scale padding included). */
+PACT_API pact_status pact_quantize_nvfp4(const pact_bf16 *x, int64_t ldx, int64_t rows, int64_t cols,
+                                const pact_nvfp4_t *out, pact_stream_t stream);
+
+/* --------------------------------------------- A3: fused RMSNorm + quantize */
+/* [METHOD] bullets 2 and 4.  For each row of x [M x H] (row stride ldx):
+ *   rstd = 1 / sqrt(sum(x^2) / H + eps)            (double)
+ *   y    = BF16_RNE((x * rstd) * gamma)            (exactly rounded)
+ *   yq   = NVFP4(y)                                (the saved copy for backward)
+ * y (the LoRA input of the forward, [M x H] row stride H) and rstd ([M] FP32)
+ * may be NULL.  H is a multiple of 64 and at most 16384. */
+PACT_API pact_status pact_rmsnorm_quant(const pact_bf16 *x, int64_t ldx, const pact_bf16 *gamma, float eps,
+                               int64_t M, int64_t H, const pact_nvfp4_t *yq, pact_bf16 *y,
+                               float *rstd, pact_stream_t stream);
+
+/* ----------------------------------------- A4: fused SiLU-multiply + quantize */
+/* [METHOD] bullet 2.  From BF16 gate g and up u ([M x I], shared row stride
+ * ld_gu; e.g. the two halves of the gate|up GEMM output):
+ *   m  = BF16_RNE(silu(g) * u)   -> m [M x I] (row stride I), the LoRA input of down
+ *   mq = NVFP4(m)                -> the down GEMM operand
+ *   gq = NVFP4(g), uq = NVFP4(u) -> the copies saved for backward (may be NULL)
+ * m may be NULL.  I is a multiple of 64. */
+PACT_API pact_status pact_silu_mul_quant(const pact_bf16 *g, const pact_bf16 *u, int64_t ld_gu, int64_t M,
+                                int64_t I, pact_bf16 *m, const pact_nvfp4_t *mq,
+                                const pact_nvfp4_t *gq, const pact_nvfp4_t *uq,
+                                pact_stream_t stream);
+
+/* ----------------------------------------------- A1: weight layout cache */
+/* [METHOD] bullet 4.  Quantizes W [N x K] (BF16, row stride ldw) along K into the
+ * forward layout and builds the backward layout q(deq(fwd)^T) [K x N] along N.
+ * buf (device, >= pact_weight_cache_bytes(N, K) bytes, 256-byte aligned) receives
+ * both; *out (host struct) is filled with pointers into buf.  Run once per frozen
+ * weight; the result stays valid while buf lives. */
+PACT_API pact_status pact_weight_layout_cache(const pact_bf16 *W, int64_t ldw, int64_t N, int64_t K,
+                                     void *buf, size_t bytes, pact_weight_cache_t *out,
+                                     pact_stream_t stream);
+
+/* ---------------------------------------------------- A5: forward GEMM */
+/* [METHOD] bullet 1 with [LORA]:
+ *   y[M x N] = BF16_RNE( deq(xq) . deq(w->fwd)^T  +  sum_i act_i . B_i^T )
+ * FP32 accumulation in tensor memory.  xq is [M x K], w->fwd [N x K]; y has row
+ * stride ldy.  lora may be NULL (frozen GEMM only). */
+PACT_API pact_status pact_frozen_gemm_fwd(const pact_nvfp4_t *xq, const pact_weight_cache_t *w,
+                                 const pact_lora_t *lora, pact_bf16 *y, int64_t ldy,
+                                 pact_stream_t stream);
+
+/* ------------------------------------------------------ A6: dgrad GEMM */
+/* [METHOD] bullet 1 (input gradient) with [LORA]:
+ *   dx[M x K] (+)= BF16_RNE( deq(dyq) . deq(w->bwd)^T  +  U . A )
+ * dyq is the NVFP4 upstream gradient [M x N] (pact_quantize_nvfp4), w->bwd
+ * [K x N].  With accumulate != 0 the existing dx is added before rounding.
+ * lora may be NULL. */
+PACT_API pact_status pact_frozen_gemm_dgrad(const pact_nvfp4_t *dyq, const pact_weight_cache_t *w,
+                                   const pact_lora_t *lora, pact_bf16 *dx, int64_t lddx,
+                                   int accumulate, pact_stream_t stream);
+
+/* ------------------------------------------------------ A7: LoRA forward */
+/* [LORA]: T[M x R] = BF16_RNE(scale * X . A^T) for X [M x K] (row stride ldx) and
+ * A [R x K] (row stride K; R = nseg*r stacked adapters sharing X).  T has row
+ * stride ldt.  R is a multiple of 16, at most 64. */
+PACT_API pact_status pact_lora_fwd(const pact_bf16 *x, int64_t ldx, int64_t M, int64_t K,
+                          const pact_bf16 *A, int R, float scale, pact_bf16 *T, int64_t ldt,
+                          pact_stream_t stream);
+
+/* --------------------------------------------------- A8: LoRA backward */
+/* [LORA] gradients, BF16 throughout ([METHOD]: adapters stay BF16).
+ * pact_lora_bwd_u: U[:, i*r .. i*r+r-1] = BF16_RNE(scale * dY[:, seg_i] . B[seg_i, :])
+ *   for dY [M x N] (row stride lddy), B [N x r]; U [M x nseg*r] (row stride ldu)
+ *   feeds pact_frozen_gemm_dgrad and pact_lora_bwd. */
+PACT_API pact_status pact_lora_bwd_u(const pact_bf16 *dy, int64_t lddy, int64_t M, int64_t N,
+                            const pact_bf16 *B, int r, int nseg, const int64_t *seg_end,
+                            float scale, pact_bf16 *U, int64_t ldu, pact_stream_t stream);
+
+/* The input X~ the adapter saw, as backward holds it: BF16 x, or the saved NVFP4
+ * copy xq (dequantized on the fly); exactly one is non-NULL. */
+typedef struct {
+    int64_t M, N, K;
+    const pact_bf16 *dy;      /* [M x N] BF16 upstream gradient, row stride lddy */
+    int64_t lddy;
+    const pact_bf16 *x;       /* [M x K] BF16, row stride ldx, or NULL */
+    int64_t ldx;
+    const pact_nvfp4_t *xq;   /* [M x K] NVFP4, or NULL */
+    const pact_bf16 *A;       /* [nseg*r x K] */
+    const pact_bf16 *U;       /* [M x nseg*r] from pact_lora_bwd_u, row stride ldu */
+    int64_t ldu;
+    int r, nseg;
+    int64_t seg_end[4];
+    float scale;
+    pact_bf16 *dA;            /* out [nseg*r x K]:  U^T . X~ */
+    pact_bf16 *dB;            /* out [N x r]: rows seg_i = scale * dY[:, seg_i]^T . (X~ . A_i^T) */
+} pact_lora_bwd_t;
+
+/* Scratch bytes pact_lora_bwd needs for its FP32 partial sums. */
+PACT_API size_t pact_lora_bwd_workspace_bytes(int64_t M, int64_t N, int64_t K, int r, int nseg);
+/* dA and dB of the adapters; workspace (device, >= pact_lora_bwd_workspace_bytes)
+ * is scratch owned by the caller; its contents on entry do not matter. */
+PACT_API pact_status pact_lora_bwd(const pact_lora_bwd_t *args, void *workspace, size_t ws_bytes,
+                          pact_stream_t stream);
+
+/* ------------------------------------- A9: SiLU-multiply backward + quantize */
+/* [METHOD] bullet 2 (backward reads the NVFP4 gate/up copies).  With
+ * g^ = deq(gq), u^ = deq(uq), s = sigmoid(g^) and dm [M x I] (row stride lddm):
+ *   dg = dm * u^ * s * (1 + g^ (1 - s)),  du = dm * g^ * s
+ * written as BF16 into dgu [M x 2I] (dg in columns 0..I-1, du in I..2I-1, row
+ * stride lddgu) and NVFP4-quantized (of the BF16 values) into dguq [M x 2I], the
+ * operand of the gate|up dgrad.  m_re (nullable, [M x I], row stride I) receives
+ * BF16_RNE(silu(g^) * u^), the down projection's LoRA input in backward. */
+PACT_API pact_status pact_silu_mul_bwd_quant(const pact_bf16 *dm, int64_t lddm, const pact_nvfp4_t *gq,
+                                    const pact_nvfp4_t *uq, int64_t M, int64_t I, pact_bf16 *dgu,
+                                    int64_t lddgu, const pact_nvfp4_t *dguq, pact_bf16 *m_re,
+                                    pact_stream_t stream);
+
+/* ------------------------------------------------- A10: RMSNorm backward */
+/* [METHOD] bullet 2 (backward reuses the quantized RMSNorm output).  With
+ * y^ = deq(yq), xn = y^ / gamma, g = gamma * dy (dy [M x H], row stride lddy):
+ *   dx = rstd * (g - xn * mean(g * xn))  (+ dres when dres != NULL, the residual
+ *   stream's gradient), written as BF16 to dx [M x H] (row stride H) and, when
+ *   dxq != NULL, NVFP4-quantized (of the BF16 values) into dxq.
+ * H is a multiple of 64 and at most 16384. */
+PACT_API pact_status pact_rmsnorm_bwd(const pact_bf16 *dy, int64_t lddy, const pact_nvfp4_t *yq,
+                             const float *rstd, const pact_bf16 *gamma, int64_t M, int64_t H,
+                             const pact_bf16 *dres, pact_bf16 *dx, const pact_nvfp4_t *dxq,
+                             pact_stream_t stream);
+
+/* ------------------------------------------------------------ status */
+/* Message of the last failing call on this thread ("" if none). */
+PACT_API const char *pact_last_error(void);
+/* Name of a status code. */
+PACT_API const char *pact_status_string(pact_status s);
+/* Synchronises `stream`, then reads and clears the status word of the current
+ * device: PACT_OK, or PACT_ERR_TIMEOUT if a kernel gave up a bounded wait. */
+PACT_API pact_status pact_get_device_status(pact_stream_t stream);
+/* PACT_ABI_VERSION of the loaded library. */
+PACT_API int pact_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* PACT_H */

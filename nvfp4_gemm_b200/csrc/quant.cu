@@ -1,0 +1,521 @@
+// quant.cu -- HBM-bound kernels of the PACT data flow: NVFP4 quantize, the fused
+// RMSNorm / SiLU-multiply quantizers, their backward kernels and the weight layout
+// cache.  All of them stream BF16 with 16-byte vector accesses (a warp moves 512
+// contiguous bytes per instruction) and quantize with warp-shuffle block maxima.
+#include <math.h>
+
+#include "quant.cuh"
+
+namespace pact {
+
+constexpr int CHUNK = 256;  // columns per warp task
+
+// Rows padded to 128 for the scale layout; padding rows get zero scales.
+__device__ __forceinline__ void zero_pad_scales(const pact_nvfp4_t &t, int64_t row, int64_t c0) {
+    const int lane = threadIdx.x & 31;
+    if ((lane & 7) == 0 && c0 + 8 * lane < t.cols) {
+        const int64_t blk = (c0 >> 4) + (lane >> 1);
+        *reinterpret_cast<uint32_t *>(static_cast<uint8_t *>(t.scales) + scale_offset(row, blk, t.cols)) = 0u;
+    }
+}
+
+// ------------------------------------------------------------------ A2: quantize
+__global__ void __launch_bounds__(256) k_quantize(const pact_bf16 *__restrict__ x, int64_t ldx, int64_t rows,
+                                                  pact_nvfp4_t out) {
+    const int lane = threadIdx.x & 31;
+    const int64_t nchunk = (out.cols + CHUNK - 1) / CHUNK;
+    const int64_t rows_pad = (rows + 127) & ~int64_t(127);
+    const int64_t ntask = rows_pad * nchunk;
+    const int64_t warp0 = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+    const int64_t nwarps = (int64_t)gridDim.x * (blockDim.x >> 5);
+    for (int64_t task = warp0; task < ntask; task += nwarps) {
+        const int64_t row = task / nchunk;
+        const int64_t c0 = (task % nchunk) * CHUNK;
+        if (row >= rows) {
+            zero_pad_scales(out, row, c0);
+            continue;
+        }
+        const bool valid = c0 + 8 * lane < out.cols;
+        float v[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+        if (valid) load8_bf16(x + row * ldx + c0 + 8 * lane, v);
+        uint32_t sb;
+        const uint32_t codes = quant8(v, &sb);
+        store_chunk(out, row, c0, codes, sb, valid);
+    }
+}
+
+static int grid_for(int64_t warp_tasks, int threads) {
+    const int sms = sm_count();
+    const int64_t per_block = threads / 32;
+    int64_t blocks = (warp_tasks + per_block - 1) / per_block;
+    const int64_t cap = (int64_t)sms * 8;
+    if (blocks > cap) blocks = cap;
+    if (blocks < 1) blocks = 1;
+    return (int)blocks;
+}
+
+// ------------------------------------------------------- A3: RMSNorm + quantize
+// One CTA (256 threads) per row; each warp owns chunks w, w+8, ... of the row and
+// keeps them in registers between the reduction and the output pass.
+constexpr int RMS_THREADS = 256;
+constexpr int RMS_MAX_CHUNKS = 8;  // H <= 8 warps x 8 chunks x 256 = 16384
+
+// Chunks of 256 columns each warp holds for a row of H columns: 1, 2, 4 or 8.
+static int rms_nch(int64_t H) {
+    const int64_t per_warp = ((H + CHUNK - 1) / CHUNK + RMS_THREADS / 32 - 1) / (RMS_THREADS / 32);
+    return per_warp <= 1 ? 1 : per_warp <= 2 ? 2 : per_warp <= 4 ? 4 : 8;
+}
+
+// BF16 rounding of y = (x * rstd) * gamma with one correct rounding of the double
+// expression: the FP32 evaluation decides unless it lies within 64 FP32 ulps of a
+// BF16 midpoint (its error is below 4 ulps), in which case the double expression
+// is rounded directly (Ziv, "Fast evaluation of elementary mathematical functions
+// with correctly rounded last bit", ACM TOMS 17(3), 1991).
+__device__ __forceinline__ float rms_out(float x, float g, float r32, double rstd) {
+    const float y = __fmul_rn(__fmul_rn(x, r32), g);
+    const uint32_t lo = __float_as_uint(y) & 0xFFFFu;
+    if (lo - 0x7FC0u <= 0x80u) {
+        const double yd = ((double)x * rstd) * (double)g;
+        return __bfloat162float(__double2bfloat16(yd));
+    }
+    return __bfloat162float(__float2bfloat16_rn(y));
+}
+
+template <int NCH>
+__global__ void __launch_bounds__(RMS_THREADS) k_rmsnorm_quant(const pact_bf16 *__restrict__ x, int64_t ldx,
+                                                               const pact_bf16 *__restrict__ gamma, float eps,
+                                                               int64_t M, int64_t H, pact_nvfp4_t yq,
+                                                               pact_bf16 *__restrict__ y, float *__restrict__ rstd_out) {
+    __shared__ double red[RMS_THREADS / 32];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int64_t row = blockIdx.x;
+    const int64_t nchunk = (H + CHUNK - 1) / CHUNK;
+    if (row >= M) {  // padding rows of the scale layout
+        for (int64_t ch = warp; ch < nchunk; ch += RMS_THREADS / 32) zero_pad_scales(yq, row, ch * CHUNK);
+        return;
+    }
+    float v[NCH][8];
+    double ss = 0.0;
+#pragma unroll
+    for (int k = 0; k < NCH; ++k) {
+        const int64_t c = (warp + (int64_t)k * (RMS_THREADS / 32)) * CHUNK + 8 * lane;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) v[k][i] = 0.0f;
+        if (c < H) {
+            load8_bf16(x + row * ldx + c, v[k]);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) ss = fma((double)v[k][i], (double)v[k][i], ss);
+        }
+    }
+#pragma unroll
+    for (int o = 16; o; o >>= 1) ss += __shfl_xor_sync(0xFFFFFFFFu, ss, o);
+    if (lane == 0) red[warp] = ss;
+    __syncthreads();
+    double tot = 0.0;
+#pragma unroll
+    for (int w = 0; w < RMS_THREADS / 32; ++w) tot += red[w];
+    const double rstd = 1.0 / sqrt(tot / (double)H + (double)eps);
+    const float r32 = (float)rstd;
+    if (threadIdx.x == 0 && rstd_out) rstd_out[row] = r32;
+#pragma unroll
+    for (int k = 0; k < NCH; ++k) {
+        const int64_t c0 = (warp + (int64_t)k * (RMS_THREADS / 32)) * CHUNK;
+        if (c0 >= H) break;  // warp-uniform
+        const int64_t c = c0 + 8 * lane;
+        const bool valid = c < H;
+        float g[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+        if (valid) load8_bf16(gamma + c, g);
+        float o[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) o[i] = valid ? rms_out(v[k][i], g[i], r32, rstd) : 0.0f;
+        if (valid && y) store8_bf16(y + row * H + c, o);
+        uint32_t sb;
+        const uint32_t codes = quant8(o, &sb);
+        store_chunk(yq, row, c0, codes, sb, valid);
+    }
+}
+
+// --------------------------------------------------- A4: SiLU-multiply + quantize
+// m = BF16_RNE(silu(g) * u) with the same FP32-then-check scheme: FP32 error of
+// g / (1 + expf(-g)) * u is a few ulps; near a BF16 midpoint the double expression
+// decides.
+__device__ __forceinline__ float silu_mul_out(float g, float u) {
+    const float m = __fmul_rn(__fdiv_rn(g, __fadd_rn(1.0f, expf(-g))), u);
+    const uint32_t lo = __float_as_uint(m) & 0xFFFFu;
+    if (lo - 0x7FC0u <= 0x80u || !isfinite(m)) {
+        const double gd = (double)g;
+        return __bfloat162float(__double2bfloat16((gd / (1.0 + exp(-gd))) * (double)u));
+    }
+    return __bfloat162float(__float2bfloat16_rn(m));
+}
+
+__global__ void __launch_bounds__(256) k_silu_mul_quant(const pact_bf16 *__restrict__ g, const pact_bf16 *__restrict__ u,
+                                                        int64_t ld_gu, int64_t M, int64_t I,
+                                                        pact_bf16 *__restrict__ m, pact_nvfp4_t mq, pact_nvfp4_t gq,
+                                                        pact_nvfp4_t uq, int has_gq, int has_uq) {
+    const int lane = threadIdx.x & 31;
+    const int64_t nchunk = (I + CHUNK - 1) / CHUNK;
+    const int64_t rows_pad = (M + 127) & ~int64_t(127);
+    const int64_t ntask = rows_pad * nchunk;
+    const int64_t warp0 = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+    const int64_t nwarps = (int64_t)gridDim.x * (blockDim.x >> 5);
+    for (int64_t task = warp0; task < ntask; task += nwarps) {
+        const int64_t row = task / nchunk;
+        const int64_t c0 = (task % nchunk) * CHUNK;
+        if (row >= M) {
+            zero_pad_scales(mq, row, c0);
+            if (has_gq) zero_pad_scales(gq, row, c0);
+            if (has_uq) zero_pad_scales(uq, row, c0);
+            continue;
+        }
+        const int64_t c = c0 + 8 * lane;
+        const bool valid = c < I;
+        float gv[8] = {0, 0, 0, 0, 0, 0, 0, 0}, uv[8] = {0, 0, 0, 0, 0, 0, 0, 0}, mv[8];
+        if (valid) {
+            load8_bf16(g + row * ld_gu + c, gv);
+            load8_bf16(u + row * ld_gu + c, uv);
+        }
+#pragma unroll
+        for (int i = 0; i < 8; ++i) mv[i] = valid ? silu_mul_out(gv[i], uv[i]) : 0.0f;
+        if (valid && m) store8_bf16(m + row * I + c, mv);
+        uint32_t sb;
+        uint32_t codes = quant8(mv, &sb);
+        store_chunk(mq, row, c0, codes, sb, valid);
+        if (has_gq) {
+            codes = quant8(gv, &sb);
+            store_chunk(gq, row, c0, codes, sb, valid);
+        }
+        if (has_uq) {
+            codes = quant8(uv, &sb);
+            store_chunk(uq, row, c0, codes, sb, valid);
+        }
+    }
+}
+
+// ---------------------------------------------- A9: SiLU-multiply backward + quantize
+__global__ void __launch_bounds__(256) k_silu_mul_bwd_quant(const pact_bf16 *__restrict__ dm, int64_t lddm,
+                                                            pact_nvfp4_t gq, pact_nvfp4_t uq, int64_t M, int64_t I,
+                                                            pact_bf16 *__restrict__ dgu, int64_t lddgu,
+                                                            pact_nvfp4_t dguq, pact_bf16 *__restrict__ m_re) {
+    const int lane = threadIdx.x & 31;
+    const int64_t nchunk = (I + CHUNK - 1) / CHUNK;
+    const int64_t rows_pad = (M + 127) & ~int64_t(127);
+    const int64_t ntask = rows_pad * nchunk;
+    const int64_t warp0 = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+    const int64_t nwarps = (int64_t)gridDim.x * (blockDim.x >> 5);
+    for (int64_t task = warp0; task < ntask; task += nwarps) {
+        const int64_t row = task / nchunk;
+        const int64_t c0 = (task % nchunk) * CHUNK;
+        if (row >= M) {
+            zero_pad_scales(dguq, row, c0);
+            zero_pad_scales(dguq, row, c0 + I);
+            continue;
+        }
+        const int64_t c = c0 + 8 * lane;
+        const bool valid = c < I;
+        float d[8] = {0, 0, 0, 0, 0, 0, 0, 0}, gh[8] = {0, 0, 0, 0, 0, 0, 0, 0}, uh[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+        if (valid) {
+            load8_bf16(dm + row * lddm + c, d);
+            load8_nvfp4(gq, row, c, gh);
+            load8_nvfp4(uq, row, c, uh);
+        }
+        float dg[8], du[8], mr[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const float s = 1.0f / (1.0f + expf(-gh[i]));
+            dg[i] = __bfloat162float(__float2bfloat16_rn(d[i] * uh[i] * s * (1.0f + gh[i] * (1.0f - s))));
+            du[i] = __bfloat162float(__float2bfloat16_rn(d[i] * gh[i] * s));
+            mr[i] = valid ? silu_mul_out(gh[i], uh[i]) : 0.0f;
+        }
+        if (valid) {
+            store8_bf16(dgu + row * lddgu + c, dg);
+            store8_bf16(dgu + row * lddgu + I + c, du);
+            if (m_re) store8_bf16(m_re + row * I + c, mr);
+        }
+        uint32_t sb;
+        uint32_t codes = quant8(dg, &sb);
+        store_chunk(dguq, row, c0, codes, sb, valid);
+        codes = quant8(du, &sb);
+        store_chunk(dguq, row, c0 + I, codes, sb, valid);
+    }
+}
+
+// ------------------------------------------------------- A10: RMSNorm backward
+template <int NCH>
+__global__ void __launch_bounds__(RMS_THREADS) k_rmsnorm_bwd(const pact_bf16 *__restrict__ dy, int64_t lddy,
+                                                             pact_nvfp4_t yq, const float *__restrict__ rstd,
+                                                             const pact_bf16 *__restrict__ gamma, int64_t M, int64_t H,
+                                                             const pact_bf16 *__restrict__ dres,
+                                                             pact_bf16 *__restrict__ dx, pact_nvfp4_t dxq, int has_dxq) {
+    __shared__ float red[RMS_THREADS / 32];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int64_t row = blockIdx.x;
+    const int64_t nchunk = (H + CHUNK - 1) / CHUNK;
+    if (row >= M) {
+        if (has_dxq)
+            for (int64_t ch = warp; ch < nchunk; ch += RMS_THREADS / 32) zero_pad_scales(dxq, row, ch * CHUNK);
+        return;
+    }
+    float dv[NCH][8], yv[NCH][8];
+    float dot = 0.0f;
+#pragma unroll
+    for (int k = 0; k < NCH; ++k) {
+        const int64_t c = (warp + (int64_t)k * (RMS_THREADS / 32)) * CHUNK + 8 * lane;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) dv[k][i] = yv[k][i] = 0.0f;
+        if (c < H) {
+            load8_bf16(dy + row * lddy + c, dv[k]);
+            load8_nvfp4(yq, row, c, yv[k]);
+            // (gamma * dy) * (y^ / gamma) == dy * y^
+#pragma unroll
+            for (int i = 0; i < 8; ++i) dot = fmaf(dv[k][i], yv[k][i], dot);
+        }
+    }
+#pragma unroll
+    for (int o = 16; o; o >>= 1) dot += __shfl_xor_sync(0xFFFFFFFFu, dot, o);
+    if (lane == 0) red[warp] = dot;
+    __syncthreads();
+    float tot = 0.0f;
+#pragma unroll
+    for (int w = 0; w < RMS_THREADS / 32; ++w) tot += red[w];
+    const float mean = tot / (float)H;
+    const float r = rstd[row];
+#pragma unroll
+    for (int k = 0; k < NCH; ++k) {
+        const int64_t c0 = (warp + (int64_t)k * (RMS_THREADS / 32)) * CHUNK;
+        if (c0 >= H) break;
+        const int64_t c = c0 + 8 * lane;
+        const bool valid = c < H;
+        float g[8] = {1, 1, 1, 1, 1, 1, 1, 1}, res[8] = {0, 0, 0, 0, 0, 0, 0, 0}, o[8];
+        if (valid) {
+            load8_bf16(gamma + c, g);
+            if (dres) load8_bf16(dres + row * H + c, res);
+        }
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const float val = r * (g[i] * dv[k][i] - (yv[k][i] / g[i]) * mean) + res[i];
+            o[i] = valid ? __bfloat162float(__float2bfloat16_rn(val)) : 0.0f;
+        }
+        if (valid) store8_bf16(dx + row * H + c, o);
+        if (has_dxq) {
+            uint32_t sb;
+            const uint32_t codes = quant8(o, &sb);
+            store_chunk(dxq, row, c0, codes, sb, valid);
+        }
+    }
+}
+
+// ------------------------------------------------------- A1: backward weight layout
+// Wb = q(deq(Wf)^T): a CTA turns a 64 (n) x 64 (k) tile of the forward layout into
+// 64 rows (k) x 4 blocks (n) of the backward layout.  Runs once per frozen weight.
+__global__ void __launch_bounds__(256) k_weight_bwd_layout(pact_nvfp4_t wf, pact_nvfp4_t wb) {
+    __shared__ float tile[64][65];
+    const int64_t n0 = (int64_t)blockIdx.y * 64, k0 = (int64_t)blockIdx.x * 64;
+    const int t = threadIdx.x;
+    // dequantize: thread t -> row n0 + t/4, columns k0 + 16*(t%4) .. +16
+    {
+        const int rn = t >> 2, cb = (t & 3) * 16;
+        const int64_t n = n0 + rn;
+        if (n < wf.rows) {
+            float a[8], b[8];
+            load8_nvfp4(wf, n, k0 + cb, a);
+            load8_nvfp4(wf, n, k0 + cb + 8, b);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                tile[rn][cb + i] = a[i];
+                tile[rn][cb + 8 + i] = b[i];
+            }
+        } else {
+#pragma unroll
+            for (int i = 0; i < 16; ++i) tile[rn][cb + i] = 0.0f;
+        }
+    }
+    __syncthreads();
+    // quantize along n: warp w handles rows k0 + 8w .. 8w+7; per row 64 columns = 8
+    // lanes x 8 values, so one warp instruction covers 4 rows.
+    const int lane = t & 31, warp = t >> 5;
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+        const int rk = warp * 8 + h * 4 + (lane >> 3);
+        const int cn = (lane & 7) * 8;
+        float v[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) v[i] = tile[cn + i][rk];
+        uint32_t sb;
+        const uint32_t codes = quant8(v, &sb);
+        const uint32_t packed = gather_scales4(sb);
+        const int64_t k = k0 + rk, n = n0 + cn;
+        if (k < wb.rows && n < wb.cols) {
+            *reinterpret_cast<uint32_t *>(static_cast<uint8_t *>(wb.codes) + k * (wb.cols >> 1) + (n >> 1)) = codes;
+            if ((lane & 7) == 0)
+                *reinterpret_cast<uint32_t *>(static_cast<uint8_t *>(wb.scales) + scale_offset(k, n >> 4, wb.cols)) =
+                    packed;
+        }
+    }
+}
+
+// Zero scale rows [rows, round_up(rows, 128)) of a tensor (the layout's padding).
+__global__ void k_zero_scale_pad(pact_nvfp4_t t) {
+    const int64_t rows_pad = (t.rows + 127) & ~int64_t(127);
+    const int64_t nblk = t.cols >> 4;
+    const int64_t n = (rows_pad - t.rows) * nblk;
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t r = t.rows + i / nblk, c = i % nblk;
+        static_cast<uint8_t *>(t.scales)[scale_offset(r, c, t.cols)] = 0;
+    }
+}
+
+}  // namespace pact
+
+using namespace pact;
+
+extern "C" {
+
+size_t pact_nvfp4_code_bytes(int64_t rows, int64_t cols) { return (size_t)(rows * (cols / 2)); }
+
+size_t pact_scale_bytes(int64_t rows, int64_t cols) {
+    return (size_t)(((rows + 127) / 128 * 128) * ((cols / 16 + 3) / 4 * 4));
+}
+
+static size_t up256(size_t b) { return (b + 255) & ~(size_t)255; }
+
+size_t pact_weight_cache_bytes(int64_t N, int64_t K) {
+    return up256(pact_nvfp4_code_bytes(N, K)) + up256(pact_scale_bytes(N, K)) + up256(pact_nvfp4_code_bytes(K, N)) +
+           up256(pact_scale_bytes(K, N));
+}
+
+pact_status pact_quantize_nvfp4(const pact_bf16 *x, int64_t ldx, int64_t rows, int64_t cols, const pact_nvfp4_t *out,
+                                pact_stream_t stream) {
+    PACT_CHECK(x && out, PACT_ERR_INVALID_ARG, "pact_quantize_nvfp4: NULL argument");
+    PACT_CHECK(rows >= 1 && cols >= 64 && cols % 64 == 0, PACT_ERR_SHAPE,
+               "pact_quantize_nvfp4: rows >= 1 and cols a positive multiple of 64 required (rows=%lld cols=%lld)",
+               (long long)rows, (long long)cols);
+    PACT_CHECK(ldx >= cols && ldx % 8 == 0 && aligned16(x), PACT_ERR_ALIGN,
+               "pact_quantize_nvfp4: x must be 16-byte aligned with ldx >= cols, ldx %% 8 == 0");
+    pact_status s = check_nvfp4(out, rows, cols, "out");
+    if (s != PACT_OK) return s;
+    const int64_t tasks = ((rows + 127) / 128 * 128) * ((cols + CHUNK - 1) / CHUNK);
+    k_quantize<<<grid_for(tasks, 256), 256, 0, (cudaStream_t)stream>>>(x, ldx, rows, *out);
+    return launch_status("pact_quantize_nvfp4");
+}
+
+pact_status pact_rmsnorm_quant(const pact_bf16 *x, int64_t ldx, const pact_bf16 *gamma, float eps, int64_t M,
+                               int64_t H, const pact_nvfp4_t *yq, pact_bf16 *y, float *rstd, pact_stream_t stream) {
+    PACT_CHECK(x && gamma && yq, PACT_ERR_INVALID_ARG, "pact_rmsnorm_quant: NULL argument");
+    PACT_CHECK(M >= 1 && H >= 64 && H % 64 == 0 && H <= RMS_THREADS / 32 * RMS_MAX_CHUNKS * CHUNK, PACT_ERR_SHAPE,
+               "pact_rmsnorm_quant: M >= 1, H a multiple of 64 in [64, 16384] required (M=%lld H=%lld)",
+               (long long)M, (long long)H);
+    PACT_CHECK(!(eps < 0.0f) && isfinite(eps), PACT_ERR_INVALID_ARG, "pact_rmsnorm_quant: eps must be finite and >= 0");
+    PACT_CHECK(ldx >= H && ldx % 8 == 0 && aligned16(x) && aligned16(gamma) && aligned16(y) && aligned16(rstd),
+               PACT_ERR_ALIGN, "pact_rmsnorm_quant: pointers must be 16-byte aligned, ldx >= H, ldx %% 8 == 0");
+    pact_status s = check_nvfp4(yq, M, H, "yq");
+    if (s != PACT_OK) return s;
+    const int64_t grid = (M + 127) / 128 * 128;
+    PACT_CHECK(grid <= 0x7FFFFFFF, PACT_ERR_SHAPE, "pact_rmsnorm_quant: M too large");
+    cudaStream_t st = (cudaStream_t)stream;
+    switch (rms_nch(H)) {
+        case 1: k_rmsnorm_quant<1><<<(unsigned)grid, RMS_THREADS, 0, st>>>(x, ldx, gamma, eps, M, H, *yq, y, rstd); break;
+        case 2: k_rmsnorm_quant<2><<<(unsigned)grid, RMS_THREADS, 0, st>>>(x, ldx, gamma, eps, M, H, *yq, y, rstd); break;
+        case 4: k_rmsnorm_quant<4><<<(unsigned)grid, RMS_THREADS, 0, st>>>(x, ldx, gamma, eps, M, H, *yq, y, rstd); break;
+        default: k_rmsnorm_quant<8><<<(unsigned)grid, RMS_THREADS, 0, st>>>(x, ldx, gamma, eps, M, H, *yq, y, rstd); break;
+    }
+    return launch_status("pact_rmsnorm_quant");
+}
+
+pact_status pact_silu_mul_quant(const pact_bf16 *g, const pact_bf16 *u, int64_t ld_gu, int64_t M, int64_t I,
+                                pact_bf16 *m, const pact_nvfp4_t *mq, const pact_nvfp4_t *gq, const pact_nvfp4_t *uq,
+                                pact_stream_t stream) {
+    PACT_CHECK(g && u && mq, PACT_ERR_INVALID_ARG, "pact_silu_mul_quant: NULL argument");
+    PACT_CHECK(M >= 1 && I >= 64 && I % 64 == 0, PACT_ERR_SHAPE,
+               "pact_silu_mul_quant: M >= 1 and I a positive multiple of 64 required");
+    PACT_CHECK(ld_gu >= I && ld_gu % 8 == 0 && aligned16(g) && aligned16(u) && aligned16(m), PACT_ERR_ALIGN,
+               "pact_silu_mul_quant: pointers must be 16-byte aligned, ld_gu >= I, ld_gu %% 8 == 0");
+    pact_status s = check_nvfp4(mq, M, I, "mq");
+    if (s == PACT_OK && gq) s = check_nvfp4(gq, M, I, "gq");
+    if (s == PACT_OK && uq) s = check_nvfp4(uq, M, I, "uq");
+    if (s != PACT_OK) return s;
+    pact_nvfp4_t none = {nullptr, nullptr, M, I};
+    const int64_t tasks = ((M + 127) / 128 * 128) * ((I + CHUNK - 1) / CHUNK);
+    k_silu_mul_quant<<<grid_for(tasks, 256), 256, 0, (cudaStream_t)stream>>>(
+        g, u, ld_gu, M, I, m, *mq, gq ? *gq : none, uq ? *uq : none, gq != nullptr, uq != nullptr);
+    return launch_status("pact_silu_mul_quant");
+}
+
+pact_status pact_silu_mul_bwd_quant(const pact_bf16 *dm, int64_t lddm, const pact_nvfp4_t *gq, const pact_nvfp4_t *uq,
+                                    int64_t M, int64_t I, pact_bf16 *dgu, int64_t lddgu, const pact_nvfp4_t *dguq,
+                                    pact_bf16 *m_re, pact_stream_t stream) {
+    PACT_CHECK(dm && gq && uq && dgu && dguq, PACT_ERR_INVALID_ARG, "pact_silu_mul_bwd_quant: NULL argument");
+    PACT_CHECK(M >= 1 && I >= 64 && I % 64 == 0, PACT_ERR_SHAPE,
+               "pact_silu_mul_bwd_quant: M >= 1 and I a positive multiple of 64 required");
+    PACT_CHECK(lddm >= I && lddm % 8 == 0 && lddgu >= 2 * I && lddgu % 8 == 0 && aligned16(dm) && aligned16(dgu) &&
+                   aligned16(m_re),
+               PACT_ERR_ALIGN, "pact_silu_mul_bwd_quant: pointers must be 16-byte aligned, leading dims %% 8 == 0");
+    pact_status s = check_nvfp4(gq, M, I, "gq");
+    if (s == PACT_OK) s = check_nvfp4(uq, M, I, "uq");
+    if (s == PACT_OK) s = check_nvfp4(dguq, M, 2 * I, "dguq");
+    if (s != PACT_OK) return s;
+    const int64_t tasks = ((M + 127) / 128 * 128) * ((I + CHUNK - 1) / CHUNK);
+    k_silu_mul_bwd_quant<<<grid_for(tasks, 256), 256, 0, (cudaStream_t)stream>>>(dm, lddm, *gq, *uq, M, I, dgu, lddgu,
+                                                                                *dguq, m_re);
+    return launch_status("pact_silu_mul_bwd_quant");
+}
+
+pact_status pact_rmsnorm_bwd(const pact_bf16 *dy, int64_t lddy, const pact_nvfp4_t *yq, const float *rstd,
+                             const pact_bf16 *gamma, int64_t M, int64_t H, const pact_bf16 *dres, pact_bf16 *dx,
+                             const pact_nvfp4_t *dxq, pact_stream_t stream) {
+    PACT_CHECK(dy && yq && rstd && gamma && dx, PACT_ERR_INVALID_ARG, "pact_rmsnorm_bwd: NULL argument");
+    PACT_CHECK(M >= 1 && H >= 64 && H % 64 == 0 && H <= RMS_THREADS / 32 * RMS_MAX_CHUNKS * CHUNK, PACT_ERR_SHAPE,
+               "pact_rmsnorm_bwd: M >= 1, H a multiple of 64 in [64, 16384] required");
+    PACT_CHECK(lddy >= H && lddy % 8 == 0 && aligned16(dy) && aligned16(gamma) && aligned16(dx) && aligned16(dres),
+               PACT_ERR_ALIGN, "pact_rmsnorm_bwd: pointers must be 16-byte aligned, lddy %% 8 == 0");
+    pact_status s = check_nvfp4(yq, M, H, "yq");
+    if (s == PACT_OK && dxq) s = check_nvfp4(dxq, M, H, "dxq");
+    if (s != PACT_OK) return s;
+    pact_nvfp4_t none = {nullptr, nullptr, M, H};
+    const int64_t grid = dxq ? (M + 127) / 128 * 128 : M;
+    cudaStream_t st = (cudaStream_t)stream;
+    const pact_nvfp4_t q = dxq ? *dxq : none;
+    const int has = dxq != nullptr;
+    switch (rms_nch(H)) {
+        case 1: k_rmsnorm_bwd<1><<<(unsigned)grid, RMS_THREADS, 0, st>>>(dy, lddy, *yq, rstd, gamma, M, H, dres, dx, q, has); break;
+        case 2: k_rmsnorm_bwd<2><<<(unsigned)grid, RMS_THREADS, 0, st>>>(dy, lddy, *yq, rstd, gamma, M, H, dres, dx, q, has); break;
+        case 4: k_rmsnorm_bwd<4><<<(unsigned)grid, RMS_THREADS, 0, st>>>(dy, lddy, *yq, rstd, gamma, M, H, dres, dx, q, has); break;
+        default: k_rmsnorm_bwd<8><<<(unsigned)grid, RMS_THREADS, 0, st>>>(dy, lddy, *yq, rstd, gamma, M, H, dres, dx, q, has); break;
+    }
+    return launch_status("pact_rmsnorm_bwd");
+}
+
+pact_status pact_weight_layout_cache(const pact_bf16 *W, int64_t ldw, int64_t N, int64_t K, void *buf, size_t bytes,
+                                     pact_weight_cache_t *out, pact_stream_t stream) {
+    PACT_CHECK(W && buf && out, PACT_ERR_INVALID_ARG, "pact_weight_layout_cache: NULL argument");
+    PACT_CHECK(N >= 64 && K >= 64 && N % 64 == 0 && K % 64 == 0, PACT_ERR_SHAPE,
+               "pact_weight_layout_cache: N and K must be positive multiples of 64 (N=%lld K=%lld)", (long long)N,
+               (long long)K);
+    PACT_CHECK(bytes >= pact_weight_cache_bytes(N, K), PACT_ERR_INVALID_ARG,
+               "pact_weight_layout_cache: buffer too small (%zu < %zu)", bytes, pact_weight_cache_bytes(N, K));
+    PACT_CHECK(((uintptr_t)buf & 255) == 0 && aligned16(W) && ldw >= K && ldw % 8 == 0, PACT_ERR_ALIGN,
+               "pact_weight_layout_cache: buf must be 256-byte aligned, W 16-byte aligned with ldw %% 8 == 0");
+    uint8_t *p = static_cast<uint8_t *>(buf);
+    pact_weight_cache_t c;
+    c.fwd.rows = N; c.fwd.cols = K;
+    c.fwd.codes = p; p += up256(pact_nvfp4_code_bytes(N, K));
+    c.fwd.scales = p; p += up256(pact_scale_bytes(N, K));
+    c.bwd.rows = K; c.bwd.cols = N;
+    c.bwd.codes = p; p += up256(pact_nvfp4_code_bytes(K, N));
+    c.bwd.scales = p;
+    pact_status s = pact_quantize_nvfp4(W, ldw, N, K, &c.fwd, stream);
+    if (s != PACT_OK) return s;
+    dim3 grid((unsigned)(K / 64), (unsigned)(N / 64));
+    k_weight_bwd_layout<<<grid, 256, 0, (cudaStream_t)stream>>>(c.fwd, c.bwd);
+    s = launch_status("pact_weight_layout_cache");
+    if (s != PACT_OK) return s;
+    if (K % 128) {
+        k_zero_scale_pad<<<64, 256, 0, (cudaStream_t)stream>>>(c.bwd);
+        s = launch_status("pact_weight_layout_cache");
+        if (s != PACT_OK) return s;
+    }
+    *out = c;
+    return PACT_OK;
+}
+
+}  // extern "C"

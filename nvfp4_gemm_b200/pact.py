@@ -1,0 +1,370 @@
+"""Thin Python binding of libpact (include/pact.h): argument marshalling only.
+
+Every function here has the name of the C entry point it calls.  Outputs the caller
+does not pass are allocated with PyTorch (device memory is PyTorch's job); the
+computation itself always runs in libpact's CUDA kernels.  There is no fallback:
+if libpact.so cannot be loaded, importing this module raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+from typing import Optional, Sequence
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libpact.so")
+
+PACT_OK = 0
+STATUS_NAMES = {0: "PACT_OK", 1: "PACT_ERR_INVALID_ARG", 2: "PACT_ERR_SHAPE", 3: "PACT_ERR_ALIGN",
+                4: "PACT_ERR_CUDA", 5: "PACT_ERR_TIMEOUT", 6: "PACT_ERR_UNSUPPORTED"}
+
+
+class PactError(RuntimeError):
+    def __init__(self, status: int, message: str):
+        super().__init__(f"{STATUS_NAMES.get(status, status)}: {message}")
+        self.status = status
+
+
+class c_nvfp4(ctypes.Structure):
+    _fields_ = [("codes", ctypes.c_void_p), ("scales", ctypes.c_void_p),
+                ("rows", ctypes.c_int64), ("cols", ctypes.c_int64)]
+
+
+class c_weight_cache(ctypes.Structure):
+    _fields_ = [("fwd", c_nvfp4), ("bwd", c_nvfp4)]
+
+
+class c_lora(ctypes.Structure):
+    _fields_ = [("act", ctypes.c_void_p), ("ld_act", ctypes.c_int64), ("weight", ctypes.c_void_p),
+                ("ld_weight", ctypes.c_int64), ("r", ctypes.c_int), ("nseg", ctypes.c_int),
+                ("seg_end", ctypes.c_int64 * 4)]
+
+
+class c_lora_bwd(ctypes.Structure):
+    _fields_ = [("M", ctypes.c_int64), ("N", ctypes.c_int64), ("K", ctypes.c_int64),
+                ("dy", ctypes.c_void_p), ("lddy", ctypes.c_int64),
+                ("x", ctypes.c_void_p), ("ldx", ctypes.c_int64),
+                ("xq", ctypes.POINTER(c_nvfp4)),
+                ("A", ctypes.c_void_p), ("U", ctypes.c_void_p), ("ldu", ctypes.c_int64),
+                ("r", ctypes.c_int), ("nseg", ctypes.c_int), ("seg_end", ctypes.c_int64 * 4),
+                ("scale", ctypes.c_float), ("dA", ctypes.c_void_p), ("dB", ctypes.c_void_p)]
+
+
+def _load() -> ctypes.CDLL:
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"libpact.so is not built ({LIB_PATH}); run nvfp4_gemm_b200/build.py")
+    lib = ctypes.CDLL(LIB_PATH)
+    P, I64, I, F = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_float
+    S = ctypes.c_int
+    NV = ctypes.POINTER(c_nvfp4)
+    sig = {
+        "pact_nvfp4_code_bytes": (ctypes.c_size_t, [I64, I64]),
+        "pact_scale_bytes": (ctypes.c_size_t, [I64, I64]),
+        "pact_weight_cache_bytes": (ctypes.c_size_t, [I64, I64]),
+        "pact_quantize_nvfp4": (S, [P, I64, I64, I64, NV, P]),
+        "pact_rmsnorm_quant": (S, [P, I64, P, F, I64, I64, NV, P, P, P]),
+        "pact_silu_mul_quant": (S, [P, P, I64, I64, I64, P, NV, NV, NV, P]),
+        "pact_weight_layout_cache": (S, [P, I64, I64, I64, P, ctypes.c_size_t, ctypes.POINTER(c_weight_cache), P]),
+        "pact_frozen_gemm_fwd": (S, [NV, ctypes.POINTER(c_weight_cache), ctypes.POINTER(c_lora), P, I64, P]),
+        "pact_frozen_gemm_dgrad": (S, [NV, ctypes.POINTER(c_weight_cache), ctypes.POINTER(c_lora), P, I64, I, P]),
+        "pact_lora_fwd": (S, [P, I64, I64, I64, P, I, F, P, I64, P]),
+        "pact_lora_bwd_u": (S, [P, I64, I64, I64, P, I, I, ctypes.POINTER(I64), F, P, I64, P]),
+        "pact_lora_bwd_workspace_bytes": (ctypes.c_size_t, [I64, I64, I64, I, I]),
+        "pact_lora_bwd": (S, [ctypes.POINTER(c_lora_bwd), P, ctypes.c_size_t, P]),
+        "pact_silu_mul_bwd_quant": (S, [P, I64, NV, NV, I64, I64, P, I64, NV, P, P]),
+        "pact_rmsnorm_bwd": (S, [P, I64, NV, P, P, I64, I64, P, P, NV, P]),
+        "pact_last_error": (ctypes.c_char_p, []),
+        "pact_status_string": (ctypes.c_char_p, [S]),
+        "pact_get_device_status": (S, [P]),
+        "pact_abi_version": (I, []),
+    }
+    for name, (res, args) in sig.items():
+        fn = getattr(lib, name)
+        fn.restype = res
+        fn.argtypes = args
+    return lib
+
+
+_lib = _load()
+lib = _lib
+
+
+def _check(status: int):
+    if status != PACT_OK:
+        raise PactError(status, _lib.pact_last_error().decode())
+
+
+def _stream(stream) -> Optional[int]:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, torch.cuda.Stream):
+        return stream.cuda_stream
+    return int(stream)
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else t.data_ptr()
+
+
+def _bf16(t: torch.Tensor, name: str) -> torch.Tensor:
+    if t.dtype != torch.bfloat16 or not t.is_cuda:
+        raise TypeError(f"{name}: expected a CUDA bfloat16 tensor")
+    if t.dim() == 2 and t.stride(1) != 1:
+        raise ValueError(f"{name}: rows must be contiguous")
+    return t
+
+
+def _ld(t: torch.Tensor) -> int:
+    return t.stride(0) if t.dim() == 2 else t.shape[-1]
+
+
+# ------------------------------------------------------------------- tensor types
+@dataclass
+class NVFP4Tensor:
+    """NVFP4 tensor [rows x cols]: codes (uint8, rows x cols/2) and scales (uint8,
+    tiled layout of pact_scale_bytes(rows, cols) bytes), both on the device."""
+    codes: torch.Tensor
+    scales: torch.Tensor
+    rows: int
+    cols: int
+
+    @staticmethod
+    def empty(rows: int, cols: int, device="cuda") -> "NVFP4Tensor":
+        codes = torch.empty((rows, cols // 2), dtype=torch.uint8, device=device)
+        scales = torch.empty(int(_lib.pact_scale_bytes(rows, cols)), dtype=torch.uint8, device=device)
+        return NVFP4Tensor(codes, scales, rows, cols)
+
+    def c(self) -> c_nvfp4:
+        return c_nvfp4(self.codes.data_ptr(), self.scales.data_ptr(), self.rows, self.cols)
+
+
+@dataclass
+class WeightCache:
+    """The cached forward [N x K] and backward [K x N] NVFP4 layouts of one frozen weight."""
+    buf: torch.Tensor
+    cstruct: c_weight_cache
+    N: int
+    K: int
+
+    @property
+    def fwd(self) -> NVFP4Tensor:
+        return self._view(self.cstruct.fwd)
+
+    @property
+    def bwd(self) -> NVFP4Tensor:
+        return self._view(self.cstruct.bwd)
+
+    def _view(self, s: c_nvfp4) -> NVFP4Tensor:
+        base = self.buf.data_ptr()
+        co = s.codes - base
+        so = s.scales - base
+        nc = int(_lib.pact_nvfp4_code_bytes(s.rows, s.cols))
+        ns = int(_lib.pact_scale_bytes(s.rows, s.cols))
+        return NVFP4Tensor(self.buf[co:co + nc].view(s.rows, s.cols // 2), self.buf[so:so + ns], s.rows, s.cols)
+
+
+def lora_struct(act: torch.Tensor, weight: torch.Tensor, r: int, seg_end: Sequence[int]) -> c_lora:
+    se = (ctypes.c_int64 * 4)(*(list(seg_end) + [0] * (4 - len(seg_end))))
+    return c_lora(act.data_ptr(), _ld(act), weight.data_ptr(), _ld(weight), r, len(seg_end), se)
+
+
+# ------------------------------------------------------------------- entry points
+def pact_nvfp4_code_bytes(rows: int, cols: int) -> int:
+    return int(_lib.pact_nvfp4_code_bytes(rows, cols))
+
+
+def pact_scale_bytes(rows: int, cols: int) -> int:
+    return int(_lib.pact_scale_bytes(rows, cols))
+
+
+def pact_weight_cache_bytes(N: int, K: int) -> int:
+    return int(_lib.pact_weight_cache_bytes(N, K))
+
+
+def pact_quantize_nvfp4(x: torch.Tensor, out: Optional[NVFP4Tensor] = None, stream=None) -> NVFP4Tensor:
+    _bf16(x, "x")
+    rows, cols = x.shape
+    out = out or NVFP4Tensor.empty(rows, cols, x.device)
+    s = out.c()
+    _check(_lib.pact_quantize_nvfp4(x.data_ptr(), _ld(x), rows, cols, ctypes.byref(s), _stream(stream)))
+    return out
+
+
+def pact_rmsnorm_quant(x: torch.Tensor, gamma: torch.Tensor, eps: float, yq: Optional[NVFP4Tensor] = None,
+                       y: Optional[torch.Tensor] = None, rstd: Optional[torch.Tensor] = None,
+                       want_y: bool = True, want_rstd: bool = True, stream=None):
+    _bf16(x, "x")
+    M, H = x.shape
+    yq = yq or NVFP4Tensor.empty(M, H, x.device)
+    if y is None and want_y:
+        y = torch.empty((M, H), dtype=torch.bfloat16, device=x.device)
+    if rstd is None and want_rstd:
+        rstd = torch.empty(M, dtype=torch.float32, device=x.device)
+    s = yq.c()
+    _check(_lib.pact_rmsnorm_quant(x.data_ptr(), _ld(x), gamma.data_ptr(), float(eps), M, H, ctypes.byref(s),
+                                   _ptr(y), _ptr(rstd), _stream(stream)))
+    return yq, y, rstd
+
+
+def pact_silu_mul_quant(g: torch.Tensor, u: torch.Tensor, m: Optional[torch.Tensor] = None,
+                        mq: Optional[NVFP4Tensor] = None, gq: Optional[NVFP4Tensor] = None,
+                        uq: Optional[NVFP4Tensor] = None, want_m: bool = True, want_copies: bool = True,
+                        stream=None):
+    _bf16(g, "g")
+    _bf16(u, "u")
+    if _ld(g) != _ld(u):
+        raise ValueError("g and u must share a row stride")
+    M, I = g.shape
+    if m is None and want_m:
+        m = torch.empty((M, I), dtype=torch.bfloat16, device=g.device)
+    mq = mq or NVFP4Tensor.empty(M, I, g.device)
+    if want_copies:
+        gq = gq or NVFP4Tensor.empty(M, I, g.device)
+        uq = uq or NVFP4Tensor.empty(M, I, g.device)
+    smq, sgq, suq = mq.c(), gq.c() if gq else None, uq.c() if uq else None
+    _check(_lib.pact_silu_mul_quant(g.data_ptr(), u.data_ptr(), _ld(g), M, I, _ptr(m), ctypes.byref(smq),
+                                    ctypes.byref(sgq) if sgq else None, ctypes.byref(suq) if suq else None,
+                                    _stream(stream)))
+    return m, mq, gq, uq
+
+
+def pact_weight_layout_cache(W: torch.Tensor, stream=None) -> WeightCache:
+    _bf16(W, "W")
+    N, K = W.shape
+    nbytes = pact_weight_cache_bytes(N, K)
+    buf = torch.empty(nbytes + 256, dtype=torch.uint8, device=W.device)
+    off = (-buf.data_ptr()) % 256
+    buf = buf[off:off + nbytes]
+    c = c_weight_cache()
+    _check(_lib.pact_weight_layout_cache(W.data_ptr(), _ld(W), N, K, buf.data_ptr(), nbytes, ctypes.byref(c),
+                                         _stream(stream)))
+    return WeightCache(buf, c, N, K)
+
+
+def pact_frozen_gemm_fwd(xq: NVFP4Tensor, w: WeightCache, lora: Optional[c_lora] = None,
+                         y: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    if y is None:
+        y = torch.empty((xq.rows, w.N), dtype=torch.bfloat16, device=xq.codes.device)
+    s = xq.c()
+    _check(_lib.pact_frozen_gemm_fwd(ctypes.byref(s), ctypes.byref(w.cstruct),
+                                     ctypes.byref(lora) if lora is not None else None,
+                                     y.data_ptr(), _ld(y), _stream(stream)))
+    return y
+
+
+def pact_frozen_gemm_dgrad(dyq: NVFP4Tensor, w: WeightCache, lora: Optional[c_lora] = None,
+                           dx: Optional[torch.Tensor] = None, accumulate: bool = False, stream=None) -> torch.Tensor:
+    if dx is None:
+        dx = torch.empty((dyq.rows, w.K), dtype=torch.bfloat16, device=dyq.codes.device)
+    s = dyq.c()
+    _check(_lib.pact_frozen_gemm_dgrad(ctypes.byref(s), ctypes.byref(w.cstruct),
+                                       ctypes.byref(lora) if lora is not None else None,
+                                       dx.data_ptr(), _ld(dx), int(bool(accumulate)), _stream(stream)))
+    return dx
+
+
+def pact_lora_fwd(x: torch.Tensor, A: torch.Tensor, scale: float, T: Optional[torch.Tensor] = None,
+                  stream=None) -> torch.Tensor:
+    _bf16(x, "x")
+    _bf16(A, "A")
+    M, K = x.shape
+    R = A.shape[0]
+    if T is None:
+        T = torch.empty((M, R), dtype=torch.bfloat16, device=x.device)
+    _check(_lib.pact_lora_fwd(x.data_ptr(), _ld(x), M, K, A.data_ptr(), R, float(scale), T.data_ptr(), _ld(T),
+                              _stream(stream)))
+    return T
+
+
+def pact_lora_bwd_u(dy: torch.Tensor, B: torch.Tensor, r: int, seg_end: Sequence[int], scale: float,
+                    U: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    _bf16(dy, "dy")
+    M, N = dy.shape
+    if U is None:
+        U = torch.empty((M, r * len(seg_end)), dtype=torch.bfloat16, device=dy.device)
+    se = (ctypes.c_int64 * 4)(*(list(seg_end) + [0] * (4 - len(seg_end))))
+    _check(_lib.pact_lora_bwd_u(dy.data_ptr(), _ld(dy), M, N, B.data_ptr(), r, len(seg_end), se, float(scale),
+                                U.data_ptr(), _ld(U), _stream(stream)))
+    return U
+
+
+def pact_lora_bwd_workspace_bytes(M: int, N: int, K: int, r: int, nseg: int) -> int:
+    return int(_lib.pact_lora_bwd_workspace_bytes(M, N, K, r, nseg))
+
+
+def pact_lora_bwd(dy: torch.Tensor, A: torch.Tensor, U: torch.Tensor, r: int, seg_end: Sequence[int], scale: float,
+                  x: Optional[torch.Tensor] = None, xq: Optional[NVFP4Tensor] = None,
+                  dA: Optional[torch.Tensor] = None, dB: Optional[torch.Tensor] = None,
+                  workspace: Optional[torch.Tensor] = None, stream=None):
+    _bf16(dy, "dy")
+    M, N = dy.shape
+    K = A.shape[1]
+    nseg = len(seg_end)
+    if dA is None:
+        dA = torch.empty((nseg * r, K), dtype=torch.bfloat16, device=dy.device)
+    if dB is None:
+        dB = torch.empty((N, r), dtype=torch.bfloat16, device=dy.device)
+    need = pact_lora_bwd_workspace_bytes(M, N, K, r, nseg)
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=dy.device)
+    xq_s = xq.c() if xq is not None else None
+    args = c_lora_bwd()
+    args.M, args.N, args.K = M, N, K
+    args.dy, args.lddy = dy.data_ptr(), _ld(dy)
+    args.x, args.ldx = (x.data_ptr(), _ld(x)) if x is not None else (None, 0)
+    args.xq = ctypes.pointer(xq_s) if xq_s is not None else None
+    args.A, args.U, args.ldu = A.data_ptr(), U.data_ptr(), _ld(U)
+    args.r, args.nseg = r, nseg
+    for i in range(4):
+        args.seg_end[i] = seg_end[i] if i < nseg else 0
+    args.scale = float(scale)
+    args.dA, args.dB = dA.data_ptr(), dB.data_ptr()
+    _check(_lib.pact_lora_bwd(ctypes.byref(args), workspace.data_ptr(), workspace.numel(), _stream(stream)))
+    return dA, dB
+
+
+def pact_silu_mul_bwd_quant(dm: torch.Tensor, gq: NVFP4Tensor, uq: NVFP4Tensor, dgu: Optional[torch.Tensor] = None,
+                            dguq: Optional[NVFP4Tensor] = None, m_re: Optional[torch.Tensor] = None,
+                            want_m: bool = False, stream=None):
+    _bf16(dm, "dm")
+    M, I = dm.shape
+    if dgu is None:
+        dgu = torch.empty((M, 2 * I), dtype=torch.bfloat16, device=dm.device)
+    dguq = dguq or NVFP4Tensor.empty(M, 2 * I, dm.device)
+    if m_re is None and want_m:
+        m_re = torch.empty((M, I), dtype=torch.bfloat16, device=dm.device)
+    sg, su, sd = gq.c(), uq.c(), dguq.c()
+    _check(_lib.pact_silu_mul_bwd_quant(dm.data_ptr(), _ld(dm), ctypes.byref(sg), ctypes.byref(su), M, I,
+                                        dgu.data_ptr(), _ld(dgu), ctypes.byref(sd), _ptr(m_re), _stream(stream)))
+    return dgu, dguq, m_re
+
+
+def pact_rmsnorm_bwd(dy: torch.Tensor, yq: NVFP4Tensor, rstd: torch.Tensor, gamma: torch.Tensor,
+                     dres: Optional[torch.Tensor] = None, dx: Optional[torch.Tensor] = None,
+                     dxq: Optional[NVFP4Tensor] = None, want_q: bool = False, stream=None):
+    _bf16(dy, "dy")
+    M, H = dy.shape
+    if dx is None:
+        dx = torch.empty((M, H), dtype=torch.bfloat16, device=dy.device)
+    if dxq is None and want_q:
+        dxq = NVFP4Tensor.empty(M, H, dy.device)
+    sy = yq.c()
+    sq = dxq.c() if dxq is not None else None
+    _check(_lib.pact_rmsnorm_bwd(dy.data_ptr(), _ld(dy), ctypes.byref(sy), rstd.data_ptr(), gamma.data_ptr(), M, H,
+                                 _ptr(dres), dx.data_ptr(), ctypes.byref(sq) if sq else None, _stream(stream)))
+    return dx, dxq
+
+
+def pact_get_device_status(stream=None) -> int:
+    return int(_lib.pact_get_device_status(_stream(stream)))
+
+
+def pact_last_error() -> str:
+    return _lib.pact_last_error().decode()
+
+
+def pact_abi_version() -> int:
+    return int(_lib.pact_abi_version())

@@ -1,0 +1,112 @@
+"""The C ABI without a GPU: libpact.so loads, exports every function include/pact.h
+declares, its size queries agree with the layout definition, and host-side argument
+checks reject bad calls with the documented status before anything is enqueued."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def declared_functions():
+    src = open(os.path.join(ROOT, "include", "pact.h")).read()
+    return sorted(set(re.findall(r"PACT_API\s+[\w\s\*]+?\b(pact_\w+)\s*\(", src)))
+
+
+@pytest.fixture(scope="module")
+def P():
+    import nvfp4_gemm_b200.build as b
+    b.build()
+    import nvfp4_gemm_b200 as p
+    return p
+
+
+def test_every_declared_symbol_is_exported(P):
+    names = declared_functions()
+    assert len(names) >= 18
+    lib = ctypes.CDLL(P.pact.LIB_PATH)
+    missing = [n for n in names if not hasattr(lib, n)]
+    assert not missing, missing
+
+
+def test_abi_version_and_status_names(P):
+    assert P.pact_abi_version() == 1
+    lib = P.pact.lib
+    assert lib.pact_status_string(0) == b"PACT_OK"
+    assert lib.pact_status_string(5) == b"PACT_ERR_TIMEOUT"
+
+
+def test_sizes_match_the_layout(P, orc):
+    for rows, cols in [(1, 64), (128, 64), (300, 320), (2048, 8960), (129, 1536)]:
+        assert P.pact_scale_bytes(rows, cols) == orc.scale_bytes(rows, cols)
+        assert P.pact_nvfp4_code_bytes(rows, cols) == rows * cols // 2
+    up = lambda b: (b + 255) // 256 * 256
+    N, K = 448, 320
+    assert P.pact_weight_cache_bytes(N, K) == (up(N * K // 2) + up(orc.scale_bytes(N, K)) + up(K * N // 2)
+                                               + up(orc.scale_bytes(K, N)))
+
+
+def _nv(rows, cols, codes=0x1000, scales=0x2000):
+    return P_mod().c_nvfp4(codes, scales, rows, cols)
+
+
+def P_mod():
+    import nvfp4_gemm_b200.pact as pm
+    return pm
+
+
+def test_host_checks_reject_bad_arguments(P):
+    lib = P.pact.lib
+    pm = P_mod()
+    good = pm.c_nvfp4(0x1000, 0x2000, 128, 128)
+    # NULL input
+    assert lib.pact_quantize_nvfp4(None, 128, 128, 128, ctypes.byref(good), None) == 1
+    # cols not a multiple of 64
+    bad = pm.c_nvfp4(0x1000, 0x2000, 128, 100)
+    assert lib.pact_quantize_nvfp4(0x3000, 100, 128, 100, ctypes.byref(bad), None) == 2
+    # misaligned input pointer
+    assert lib.pact_quantize_nvfp4(0x3008, 128, 128, 128, ctypes.byref(good), None) == 3
+    # output descriptor of the wrong shape
+    other = pm.c_nvfp4(0x1000, 0x2000, 64, 128)
+    assert lib.pact_quantize_nvfp4(0x3000, 128, 128, 128, ctypes.byref(other), None) == 2
+    assert "shape" in P.pact_last_error()
+    # RMSNorm: H beyond the supported maximum
+    big = pm.c_nvfp4(0x1000, 0x2000, 4, 32768)
+    assert lib.pact_rmsnorm_quant(0x3000, 32768, 0x4000, ctypes.c_float(1e-5), 4, 32768, ctypes.byref(big),
+                                  None, None, None) == 2
+    # weight cache: buffer too small / misaligned
+    wc = pm.c_weight_cache()
+    assert lib.pact_weight_layout_cache(0x3000, 512, 512, 512, 0x10000, 16, ctypes.byref(wc), None) == 1
+    n = P.pact_weight_cache_bytes(512, 512)
+    assert lib.pact_weight_layout_cache(0x3000, 512, 512, 512, 0x10010, n, ctypes.byref(wc), None) == 3
+    # GEMM: output leading dimension not a multiple of 8
+    wcache = pm.c_weight_cache(pm.c_nvfp4(0x1000, 0x2000, 512, 512), pm.c_nvfp4(0x3000, 0x4000, 512, 512))
+    xq = pm.c_nvfp4(0x5000, 0x6000, 256, 512)
+    assert lib.pact_frozen_gemm_fwd(ctypes.byref(xq), ctypes.byref(wcache), None, 0x7000, 516, None) == 3
+    # GEMM: activation K does not match the weight
+    xq2 = pm.c_nvfp4(0x5000, 0x6000, 256, 448)
+    assert lib.pact_frozen_gemm_fwd(ctypes.byref(xq2), ctypes.byref(wcache), None, 0x7000, 512, None) == 2
+    # LoRA: internal segment boundary not a multiple of 256
+    se = (ctypes.c_int64 * 4)(320, 512, 0, 0)
+    lo = pm.c_lora(0x8000, 32, 0x9000, 16, 16, 2, se)
+    assert lib.pact_frozen_gemm_fwd(ctypes.byref(xq), ctypes.byref(wcache), ctypes.byref(lo), 0x7000, 512,
+                                    None) == 2
+    # LoRA rank not supported
+    lo2 = pm.c_lora(0x8000, 32, 0x9000, 16, 8, 1, (ctypes.c_int64 * 4)(512, 0, 0, 0))
+    assert lib.pact_frozen_gemm_fwd(ctypes.byref(xq), ctypes.byref(wcache), ctypes.byref(lo2), 0x7000, 512,
+                                    None) == 2
+    # LoRA backward: workspace too small
+    args = pm.c_lora_bwd()
+    args.M, args.N, args.K = 256, 512, 512
+    args.dy, args.lddy, args.x, args.ldx = 0x1000, 512, 0x2000, 512
+    args.A, args.U, args.ldu, args.r, args.nseg = 0x3000, 0x4000, 16, 16, 1
+    args.seg_end[0] = 512
+    args.dA, args.dB, args.scale = 0x5000, 0x6000, 2.0
+    assert lib.pact_lora_bwd(ctypes.byref(args), 0x10000, 64, None) == 1
+    # both x and xq given
+    xq3 = pm.c_nvfp4(0x5000, 0x6000, 256, 512)
+    args.xq = ctypes.pointer(xq3)
+    need = P.pact_lora_bwd_workspace_bytes(256, 512, 512, 16, 1)
+    assert lib.pact_lora_bwd(ctypes.byref(args), 0x10000, need, None) == 1

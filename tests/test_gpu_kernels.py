@@ -1,0 +1,334 @@
+"""Parity of every libpact kernel with the CPU oracle (needs a B200).
+
+Integer outputs (NVFP4 codes and scales, padding included) must match bit for bit;
+floating-point outputs must satisfy |gpu - oracle| <= 8e-3 |oracle| + 1e-3 rms(oracle).
+Stages are teacher-forced: each kernel is compared with the oracle run on the GPU
+kernel's own inputs.  Sizes span several tiles and ragged tails.
+"""
+import numpy as np
+import pytest
+import torch
+
+import synth
+from tests.util import assert_close, assert_nvfp4_equal, nvfp4_host, to_bits, to_dev, to_f64
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def P():
+    import nvfp4_gemm_b200 as p
+    return p
+
+
+def sync():
+    torch.cuda.synchronize()
+
+
+def status_ok(P):
+    assert P.pact_get_device_status() == 0, P.pact_last_error()
+
+
+# --------------------------------------------------------------------- quantize
+def _positive_bf16():
+    bits = np.arange(1, 0x7F80, dtype=np.uint16)
+    return bits, synth.bf16_bits_to_f64(bits)
+
+
+def test_quantize_all_scales(P, orc):
+    """Every finite positive BF16 amax, as a block [amax, 0, ...]: scale and codes
+    bit-exact (pins the E4M3 decision of the device path exhaustively)."""
+    bits, _ = _positive_bf16()
+    blocks = np.zeros((bits.size, 64), dtype=np.uint16)
+    blocks[:, 0] = bits
+    blocks[:, 17] = bits | 0x8000
+    dev = P.pact_quantize_nvfp4(to_dev(blocks))
+    sync()
+    assert_nvfp4_equal(dev, orc.quantize(blocks), orc, "all scales")
+
+
+def test_quantize_all_elements(P, orc):
+    """Every E4M3 scale s and every BF16 |x| <= 6s, both signs, in blocks that force
+    the scale to s: codes bit-exact, every tie included."""
+    bits, vals = _positive_bf16()
+    rows = []
+    for sb in range(0, 0x7F):
+        s = orc.e4m3_value(sb)
+        head = synth.f64_to_bf16_bits(np.array([6.0 * s]))[0] if sb else np.uint16(0)
+        sel = vals <= 6.0 * s if sb else vals < 6 * 2.0 ** -10
+        xb = np.concatenate([bits[sel], bits[sel] | np.uint16(0x8000), [0x8000]])
+        xb = np.concatenate([xb, np.zeros((-xb.size) % 15, dtype=np.uint16)])
+        blk = np.empty((xb.size // 15, 16), dtype=np.uint16)
+        blk[:, 0] = head
+        blk[:, 1:] = xb.reshape(-1, 15)
+        rows.append(blk)
+    blocks = np.concatenate(rows)
+    blocks = np.concatenate([blocks, np.zeros(((-blocks.shape[0]) % 4, 16), dtype=np.uint16)])
+    x = blocks.reshape(-1, 64)
+    dev = P.pact_quantize_nvfp4(to_dev(x))
+    sync()
+    assert_nvfp4_equal(dev, orc.quantize(x), orc, "all elements")
+
+
+@pytest.mark.parametrize("rows,cols,ld", [(1, 64, 64), (200, 320, 320), (300, 1024, 1088), (128, 256, 256),
+                                          (2048, 2048, 2048)])
+def test_quantize_shapes(P, orc, rows, cols, ld):
+    x = synth.gaussian_bf16(1, (rows, ld), std=2.0)
+    xd = to_dev(x)[:, :cols]
+    dev = P.pact_quantize_nvfp4(xd)
+    sync()
+    assert_nvfp4_equal(dev, orc.quantize(x[:, :cols]), orc, f"quantize {rows}x{cols}")
+
+
+# ------------------------------------------------------------------ weight cache
+@pytest.mark.parametrize("N,K", [(64, 64), (512, 512), (448, 320), (2048, 512), (384, 2048)])
+def test_weight_layout_cache(P, orc, N, K):
+    w = synth.weight_bf16(0, (N, K), outliers=True)
+    wc = P.pact_weight_layout_cache(to_dev(w))
+    sync()
+    wf, wb = orc.weight_cache(w)
+    assert_nvfp4_equal(wc.fwd, wf, orc, "fwd layout")
+    assert_nvfp4_equal(wc.bwd, wb, orc, "bwd layout")
+
+
+# ------------------------------------------------------------------------- GEMM
+def _nvfp4_from_oracle(P, t, orc):
+    """Upload an oracle NVFP4 tensor (codes + packed scales) to the device."""
+    d = P.NVFP4Tensor.empty(t.rows, t.cols)
+    d.codes.copy_(torch.from_numpy(t.codes))
+    d.scales.copy_(torch.from_numpy(orc.pack_scales(t.scales, t.rows, t.cols)))
+    return d
+
+
+@pytest.mark.parametrize("N,K", [(512, 512), (448, 576), (2048, 1024)])
+def test_gemm_one_hot(P, orc, N, K):
+    """X rows 6 e_i (scale 1, code 7): Y row = 6 deq(W_fwd)[:, i] exactly in BF16; the
+    same for dgrad with the backward layout.  Pins indexing, nibble order and the
+    scale layout as the tensor core reads it."""
+    w = synth.weight_bf16(1, (N, K))
+    wc = P.pact_weight_layout_cache(to_dev(w))
+    wf, wb = orc.weight_cache(w)
+    rng = np.random.default_rng(0)
+    M = 256
+    for lay, (rows, cols) in ((wf, (N, K)), (wb, (K, N))):
+        idx = rng.integers(0, cols, size=M)
+        x = np.zeros((M, cols), dtype=np.uint16)
+        x[np.arange(M), idx] = synth.f64_to_bf16_bits(np.array([6.0]))[0]
+        xq = P.pact_quantize_nvfp4(to_dev(x))
+        if lay is wf:
+            y = P.pact_frozen_gemm_fwd(xq, wc)
+        else:
+            y = P.pact_frozen_gemm_dgrad(xq, wc)
+        sync()
+        want = 6.0 * orc.dequantize(lay)[:, idx].T
+        assert np.array_equal(to_f64(y), want)
+
+
+GEMM_SHAPES = [(256, 512, 512), (300, 640, 576), (128, 256, 64), (1, 320, 448), (513, 1024, 2048)]
+
+
+@pytest.mark.parametrize("M,N,K", GEMM_SHAPES)
+def test_gemm_fwd(P, orc, M, N, K):
+    x = synth.gaussian_bf16(1, (M, K))
+    w = synth.weight_bf16(0, (N, K))
+    wc = P.pact_weight_layout_cache(to_dev(w))
+    xq = P.pact_quantize_nvfp4(to_dev(x))
+    y = P.pact_frozen_gemm_fwd(xq, wc)
+    sync()
+    status_ok(P)
+    wf, _ = orc.weight_cache(w)
+    assert_close(to_f64(y), orc.nvfp4_gemm(orc.quantize(x), wf), "fwd")
+
+
+@pytest.mark.parametrize("M,N,K", GEMM_SHAPES)
+def test_gemm_dgrad(P, orc, M, N, K):
+    dy = synth.gaussian_bf16(50, (M, N))
+    w = synth.weight_bf16(0, (N, K))
+    wc = P.pact_weight_layout_cache(to_dev(w))
+    dyq = P.pact_quantize_nvfp4(to_dev(dy))
+    dx = P.pact_frozen_gemm_dgrad(dyq, wc)
+    sync()
+    _, wb = orc.weight_cache(w)
+    assert_close(to_f64(dx), orc.frozen_dgrad(dy, wb), "dgrad")
+
+
+def test_gemm_dgrad_accumulate(P, orc):
+    M, N, K = 256, 512, 768
+    dy = synth.gaussian_bf16(50, (M, N))
+    base = synth.gaussian_bf16(2, (M, K))
+    w = synth.weight_bf16(0, (N, K))
+    wc = P.pact_weight_layout_cache(to_dev(w))
+    dx = to_dev(base)
+    P.pact_frozen_gemm_dgrad(P.pact_quantize_nvfp4(to_dev(dy)), wc, dx=dx, accumulate=True)
+    sync()
+    _, wb = orc.weight_cache(w)
+    assert_close(to_f64(dx), orc.frozen_dgrad(dy, wb) + synth.bf16_bits_to_f64(base), "dgrad accumulate")
+
+
+def _segments(N, parts):
+    ends, acc = [], 0
+    for p_ in parts:
+        acc += p_
+        ends.append(acc)
+    assert acc == N
+    return ends
+
+
+@pytest.mark.parametrize("M,parts,K,r", [(256, [512], 512, 16), (300, [512, 256, 256], 576, 16),
+                                         (200, [256, 320], 256, 32)])
+def test_gemm_fwd_lora(P, orc, M, parts, K, r):
+    N = sum(parts)
+    seg_end = _segments(N, parts)
+    x = synth.gaussian_bf16(1, (M, K))
+    w = synth.weight_bf16(0, (N, K))
+    nseg = len(parts)
+    a = synth.gaussian_bf16(20, (nseg * r, K), std=0.02)
+    b = synth.gaussian_bf16(30, (N, r), std=0.02)
+    s = 2.0
+    wc = P.pact_weight_layout_cache(to_dev(w))
+    xd = to_dev(x)
+    xq = P.pact_quantize_nvfp4(xd)
+    T = P.pact_lora_fwd(xd, to_dev(a), s)
+    bd = to_dev(b)
+    y = P.pact_frozen_gemm_fwd(xq, wc, lora=P.lora_struct(T, bd, r, seg_end))
+    sync()
+    # oracle, teacher-forced on the device's T (its BF16 rounding is the device's)
+    wf, _ = orc.weight_cache(w)
+    ref = orc.nvfp4_gemm(orc.quantize(x), wf)
+    t_dev = to_f64(T)
+    bb = synth.bf16_bits_to_f64(b)
+    lo = 0
+    for i, hi in enumerate(seg_end):
+        ref[:, lo:hi] += orc.gemm_nt(t_dev[:, i * r:(i + 1) * r], bb[lo:hi])
+        lo = hi
+    assert_close(to_f64(y), ref, "fwd + LoRA")
+    # and T itself against the oracle's scale * X A^T
+    assert_close(t_dev, s * orc.lora_t(synth.bf16_bits_to_f64(x), a), "T")
+
+
+@pytest.mark.parametrize("M,N,K,R", [(256, 512, 512, 16), (300, 640, 576, 48), (130, 256, 320, 64)])
+def test_gemm_dgrad_lora(P, orc, M, N, K, R):
+    dy = synth.gaussian_bf16(50, (M, N))
+    w = synth.weight_bf16(0, (N, K))
+    a = synth.gaussian_bf16(20, (R, K), std=0.02)
+    u = synth.gaussian_bf16(31, (M, R), std=0.5)
+    wc = P.pact_weight_layout_cache(to_dev(w))
+    dyq = P.pact_quantize_nvfp4(to_dev(dy))
+    ud, ad = to_dev(u), to_dev(a)
+    dx = P.pact_frozen_gemm_dgrad(dyq, wc, lora=P.lora_struct(ud, ad, R, [K]))
+    sync()
+    _, wb = orc.weight_cache(w)
+    ref = orc.frozen_dgrad(dy, wb) + orc.gemm_nt(synth.bf16_bits_to_f64(u), synth.bf16_bits_to_f64(a).T)
+    assert_close(to_f64(dx), ref, "dgrad + LoRA")
+
+
+# ------------------------------------------------------------------------- LoRA
+@pytest.mark.parametrize("M,parts,r", [(256, [512], 16), (300, [512, 256, 256], 16), (130, [256, 320], 32)])
+def test_lora_bwd(P, orc, M, parts, r):
+    N = sum(parts)
+    seg_end = _segments(N, parts)
+    nseg = len(parts)
+    K = 384
+    dy = synth.gaussian_bf16(50, (M, N))
+    x = synth.gaussian_bf16(1, (M, K))
+    a = synth.gaussian_bf16(20, (nseg * r, K), std=0.02)
+    b = synth.gaussian_bf16(30, (N, r), std=0.02)
+    s = 2.0
+    dyd, xd, ad, bd = to_dev(dy), to_dev(x), to_dev(a), to_dev(b)
+    U = P.pact_lora_bwd_u(dyd, bd, r, seg_end, s)
+    dA, dB = P.pact_lora_bwd(dyd, ad, U, r, seg_end, s, x=xd)
+    xq = P.pact_quantize_nvfp4(xd)
+    dA2, dB2 = P.pact_lora_bwd(dyd, ad, U, r, seg_end, s, xq=xq)
+    sync()
+    dyf, xf = synth.bf16_bits_to_f64(dy), synth.bf16_bits_to_f64(x)
+    af, bf = synth.bf16_bits_to_f64(a), synth.bf16_bits_to_f64(b)
+    u_dev = to_f64(U)
+    lo = 0
+    u_ref = np.zeros((M, nseg * r))
+    for i, hi in enumerate(seg_end):
+        u_ref[:, i * r:(i + 1) * r] = s * orc.gemm_nt(dyf[:, lo:hi], bf[lo:hi].T)
+        lo = hi
+    assert_close(u_dev, u_ref, "U")
+    for xt, gA, gB, what in ((xf, dA, dB, "bf16 x"), (orc.dequantize(orc.quantize(x)), dA2, dB2, "nvfp4 x")):
+        # dA from the device's U (teacher-forced), dB per segment
+        assert_close(to_f64(gA), orc.gemm_nt(u_dev.T, xt.T), f"dA ({what})")
+        db_ref = np.zeros((N, r))
+        lo = 0
+        for i, hi in enumerate(seg_end):
+            _, db_i, _ = orc.lora_bwd_at(dyf[:, lo:hi], xt, af[i * r:(i + 1) * r], bf[lo:hi], s)
+            db_ref[lo:hi] = db_i
+            lo = hi
+        assert_close(to_f64(gB), db_ref, f"dB ({what})")
+
+
+# --------------------------------------------------------------- fused producers
+@pytest.mark.parametrize("M,H", [(64, 512), (257, 2048), (96, 3072), (33, 1536)])
+def test_rmsnorm_quant(P, orc, M, H):
+    x = synth.gaussian_bf16(1, (M, H))
+    g = synth.gaussian_bf16(40, (H,), std=0.02, mean=1.0)
+    yq, y, rstd = P.pact_rmsnorm_quant(to_dev(x), to_dev(g), 1e-5)
+    sync()
+    y_ref, yq_ref, rstd_ref = orc.rmsnorm_quant(x, g, 1e-5)
+    yb = to_bits(y)
+    assert np.array_equal(yb, y_ref), f"y differs at {np.argwhere(yb != y_ref)[:3].tolist()}"
+    assert_nvfp4_equal(yq, yq_ref, orc, "yq")
+    np.testing.assert_allclose(rstd.cpu().numpy(), rstd_ref, rtol=1e-7)
+
+
+@pytest.mark.parametrize("M,I", [(64, 512), (130, 8960), (257, 2048)])
+def test_silu_mul_quant(P, orc, M, I):
+    gu = synth.gaussian_bf16(4, (M, 2 * I), std=2.0)
+    gud = to_dev(gu)
+    m, mq, gq, uq = P.pact_silu_mul_quant(gud[:, :I], gud[:, I:])
+    sync()
+    m_ref, mq_ref, gq_ref, uq_ref = orc.silu_mul_quant(gu[:, :I], gu[:, I:])
+    mb = to_bits(m)
+    assert np.array_equal(mb, m_ref), f"m differs at {np.argwhere(mb != m_ref)[:3].tolist()}"
+    assert_nvfp4_equal(mq, mq_ref, orc, "mq")
+    assert_nvfp4_equal(gq, gq_ref, orc, "gq")
+    assert_nvfp4_equal(uq, uq_ref, orc, "uq")
+
+
+@pytest.mark.parametrize("M,I", [(64, 512), (130, 2048)])
+def test_silu_mul_bwd_quant(P, orc, M, I):
+    gu = synth.gaussian_bf16(4, (M, 2 * I), std=2.0)
+    dm = synth.gaussian_bf16(56, (M, I))
+    _, _, gq, uq = orc.silu_mul_quant(gu[:, :I], gu[:, I:])
+    gqd, uqd = _nvfp4_from_oracle(P, gq, orc), _nvfp4_from_oracle(P, uq, orc)
+    dgu, dguq, m_re = P.pact_silu_mul_bwd_quant(to_dev(dm), gqd, uqd, want_m=True)
+    sync()
+    dg_ref, du_ref = orc.silu_mul_bwd(synth.bf16_bits_to_f64(dm), gq, uq)
+    dgu_dev = to_f64(dgu)
+    assert_close(dgu_dev[:, :I], dg_ref, "dg")
+    assert_close(dgu_dev[:, I:], du_ref, "du")
+    assert_nvfp4_equal(dguq, orc.quantize(to_bits(dgu)), orc, "q(dg|du)")
+    mr = to_bits(m_re)
+    want = orc.silu_mul_recompute(gq, uq)
+    assert np.array_equal(mr, want), f"m~ differs at {np.argwhere(mr != want)[:3].tolist()}"
+
+
+@pytest.mark.parametrize("M,H,with_res", [(64, 512, False), (130, 2048, True), (33, 3072, True)])
+def test_rmsnorm_bwd(P, orc, M, H, with_res):
+    x = synth.gaussian_bf16(1, (M, H))
+    g = synth.gaussian_bf16(40, (H,), std=0.02, mean=1.0)
+    dy = synth.gaussian_bf16(57, (M, H))
+    res = synth.gaussian_bf16(58, (M, H))
+    yq, _, rstd = P.pact_rmsnorm_quant(to_dev(x), to_dev(g), 1e-5)
+    dx, dxq = P.pact_rmsnorm_bwd(to_dev(dy), yq, rstd, to_dev(g), dres=to_dev(res) if with_res else None,
+                                 want_q=True)
+    sync()
+    _, yq_ref, _ = orc.rmsnorm_quant(x, g, 1e-5)
+    ref = orc.rmsnorm_bwd(synth.bf16_bits_to_f64(dy), yq_ref, rstd.cpu().numpy().astype(np.float64), g)
+    if with_res:
+        ref = ref + synth.bf16_bits_to_f64(res)
+    assert_close(to_f64(dx), ref, "dx")
+    assert_nvfp4_equal(dxq, orc.quantize(to_bits(dx)), orc, "q(dx)")
+
+
+# ------------------------------------------------------------- host-side errors
+def test_errors_leave_nothing_enqueued(P):
+    x = torch.zeros((128, 100), dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(P.PactError) as e:
+        P.pact_quantize_nvfp4(x)
+    assert e.value.status == 2
+    status_ok(P)
