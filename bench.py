@@ -1,0 +1,362 @@
+#!/usr/bin/env python
+"""Benchmark of one PACT LoRA decoder layer step on B200.
+
+A step is the forward and backward pass of the NVFP4 data flow through a decoder
+layer's seven frozen projections (fused RMSNorm / SiLU-multiply quantizers, NVFP4
+GEMMs with the fused BF16 LoRA branch, NVFP4 dgrad GEMMs on the cached transposed
+weight layouts, LoRA weight gradients, the backward elementwise kernels), all in
+libpact.  Inputs are seeded synthetic tensors shaped like a Llama-3.2-1B layer
+(H 2048, I 8192, k/v 512, batch 4 x seq 512 tokens), LoRA r 16, alpha 32.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl pact|reference]
+
+prints one JSON line.  --impl reference times the CPU oracle (the plain FP64
+reference implementation) on the host cores on a bounded token sample of the
+same workload.  Multi-GPU runs (torchrun) are data-parallel replicas: each rank
+runs its own layer step on its own tokens and the LoRA gradients are all-reduced
+over NCCL.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+METRIC = "NVFP4 frozen-proj fwd+dgrad TFLOPS & layer tokens/s; % of FP4 tensor peak"
+WORKLOAD = "llama-3.2-1b"
+# nominal dense FP4 / BF16 tensor throughput ratio on B200 (9 / 2.25 PFLOP/s)
+FP4_PER_BF16 = 4.0
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=("pact", "reference"), default="pact")
+    ap.add_argument("--workload", default=WORKLOAD)
+    ap.add_argument("--cpu-tokens", type=int, default=128, help="token sample of the CPU oracle baseline")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        d = json.load(open(path))
+        return {"hbm_gbs": float(d["hbm_gbs"]), "bf16": float(d["bf16_tflops"]),
+                "bf16_sustained": float(d.get("bf16_tflops_sustained", d["bf16_tflops"])), "src": "measured"}
+    except (OSError, KeyError, ValueError):
+        return {"hbm_gbs": 6650.0, "bf16": 1590.0, "bf16_sustained": 1400.0, "src": "fallback"}
+
+
+# ------------------------------------------------------------------ clocks
+class ClockSampler:
+    """nvidia-smi samples (every 200 ms) while the timed region runs."""
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.dev = device_index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.dev), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except OSError:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *a):
+        if self.proc:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+            self.thread.join(timeout=2)
+
+    def summary(self):
+        sm, mx, reasons = [], 0.0, set()
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        for ln in self.lines:
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 8:
+                continue
+            try:
+                sm.append(float(f[0]))
+                mx = max(mx, float(f[1]))
+            except ValueError:
+                continue
+            for n, v in zip(names, f[4:8]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx or None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ------------------------------------------------------------------ CPU oracle
+def oracle_layer(name, inputs):
+    import oracle
+    from oracle.layer import OracleLayer
+    import synth
+    oracle.build()
+    c = synth.LAYERS[name]
+    return OracleLayer(c["H"], c["I"], c["KV"], synth.LORA_R, synth.LORA_ALPHA, synth.RMS_EPS, inputs["w"],
+                       inputs["lora_a"], inputs["lora_b"], inputs["gamma1"], inputs["gamma2"])
+
+
+def oracle_rate(layer, inputs, tokens, min_seconds=10.0, max_steps=20):
+    """Tokens/s of the oracle's layer step on the first `tokens` tokens."""
+    import oracle
+    sl = slice(0, tokens)
+    args = (inputs["h"][sl], inputs["attn"][sl], inputs["d_out"][sl], inputs["d_qkv"][sl])
+    t0 = time.perf_counter()
+    n = 0
+    while True:
+        layer.step(*args)
+        n += 1
+        el = time.perf_counter() - t0
+        if el >= min_seconds or n >= max_steps:
+            break
+    return n * tokens / el, n, el, oracle.num_threads()
+
+
+def reference_arm(a):
+    """--impl reference: the CPU oracle timed on the host cores (rank 0 only)."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    import synth
+    M = synth.tokens(a.workload)
+    inputs = synth.layer_inputs(a.workload)
+    layer = oracle_layer(a.workload, inputs)
+    for _ in range(max(0, min(a.warmup, 1))):
+        layer.step(inputs["h"][:8], inputs["attn"][:8], inputs["d_out"][:8], inputs["d_qkv"][:8])
+    tok = max(8, min(a.cpu_tokens, M))
+    rate, n, el, cores = oracle_rate(layer, inputs, tok, min_seconds=0.0, max_steps=max(1, a.steps))
+    sample = (f"{tok} of {M} tokens per step ({n} steps), one layer fwd+bwd; weight layouts "
+              f"cached before timing")
+    print(json.dumps({
+        "impl": "reference", "metric": METRIC, "value": rate, "unit": "tokens/s", "n_gpus": a.gpus,
+        "steps": n, "warmup": a.warmup, "ms_per_step": 1000.0 * el / n, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": config_block(a.workload, M),
+        "cpu_baseline": {"value": rate, "unit": "tokens/s", "cores": cores, "kind": "oracle", "sample": sample},
+        "e2e": {"value": rate, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }), flush=True)
+
+
+def config_block(name, M):
+    import synth
+    c = synth.LAYERS[name]
+    return {"workload": f"{name} decoder layer fwd+bwd: 7 NVFP4 frozen projections + LoRA",
+            "H": c["H"], "I": c["I"], "kv": c["KV"], "tokens": M, "batch": c["batch"], "seq": c["seq"],
+            "lora_r": synth.LORA_R, "lora_alpha": synth.LORA_ALPHA,
+            "l2": "flushed between timed steps (256 MiB write)", "launch": "per-segment CUDA graphs"}
+
+
+# ------------------------------------------------------------------ GPU arm
+def main():
+    a = parse()
+    if a.impl == "reference":
+        return reference_arm(a)
+
+    import torch
+    import torch.distributed as dist
+
+    import synth
+    import nvfp4_gemm_b200 as P
+    from nvfp4_gemm_b200.layer import LayerShape, PactLayer
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+
+    c = synth.LAYERS[a.workload]
+    M = synth.tokens(a.workload)
+    inputs = synth.layer_inputs(a.workload)
+    d = lambda bits: torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).to(dev)
+    shape = LayerShape(M=M, H=c["H"], I=c["I"], KV=c["KV"], r=synth.LORA_R, alpha=synth.LORA_ALPHA,
+                       eps=synth.RMS_EPS)
+    layer = PactLayer(shape, {k: d(v) for k, v in inputs["w"].items()},
+                      {k: d(v) for k, v in inputs["lora_a"].items()},
+                      {k: d(v) for k, v in inputs["lora_b"].items()}, d(inputs["gamma1"]), d(inputs["gamma2"]))
+    x_in = {k: d(inputs[k]) for k in ("h", "attn", "d_out", "d_qkv")}
+    layer.bind(x_in["h"], x_in["attn"], x_in["d_out"], x_in["d_qkv"])
+    ops = layer.step_ops()
+    launches_per_step = sum(op.kernels for op in ops)
+
+    # segments: each NVFP4 GEMM alone, consecutive other ops together
+    segs = []
+    for op in ops:
+        if op.kind == "gemm" or not segs or segs[-1]["kind"] == "gemm":
+            segs.append({"kind": op.kind, "ops": [op], "flops": op.flops})
+        else:
+            segs[-1]["ops"].append(op)
+    stream = torch.cuda.Stream(device=dev)
+    torch.cuda.synchronize()
+    with torch.cuda.stream(stream):
+        for _ in range(2):           # eager passes: per-device attributes, lazy init
+            layer.step()
+    torch.cuda.synchronize()
+    if P.pact_get_device_status() != 0:
+        raise RuntimeError(P.pact_last_error())
+    for sg in segs:
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            for op in sg["ops"]:
+                op.fn()
+        sg["graph"] = g
+    torch.cuda.synchronize()
+
+    def run_step():
+        for sg in segs:
+            sg["graph"].replay()
+
+    grads = list(layer.grads.values())
+
+    def allreduce_grads():
+        if world > 1:
+            for gt in grads:
+                dist.all_reduce(gt)
+
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    with torch.cuda.stream(stream):
+        for _ in range(a.warmup):
+            flush.zero_()
+            run_step()
+            allreduce_grads()
+    torch.cuda.synchronize()
+
+    K = a.steps
+    ev = lambda: torch.cuda.Event(enable_timing=True)
+    st_ev = [(ev(), ev()) for _ in range(K)]
+    seg_ev = [[(ev(), ev()) for _ in segs] for _ in range(K)]
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        time.sleep(0.25)
+        with torch.cuda.stream(stream):
+            for k in range(K):
+                flush.zero_()
+                st_ev[k][0].record(stream)
+                for i, sg in enumerate(segs):
+                    seg_ev[k][i][0].record(stream)
+                    sg["graph"].replay()
+                    seg_ev[k][i][1].record(stream)
+                allreduce_grads()
+                st_ev[k][1].record(stream)
+        torch.cuda.synchronize()
+        time.sleep(0.25)
+    if world > 1:
+        dist.barrier()
+    step_ms = [s.elapsed_time(e) for s, e in st_ev]
+    total_ms = sum(step_ms)
+    seg_ms = [sum(seg_ev[k][i][0].elapsed_time(seg_ev[k][i][1]) for k in range(K)) / K for i in range(len(segs))]
+    if world > 1:
+        t = torch.tensor([total_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+    ms_per_step = total_ms / K
+    tokens_per_s = M * K * world / (total_ms / 1e3)
+
+    gemm_flops = sum(sg["flops"] for sg in segs if sg["kind"] == "gemm")
+    gemm_ms = sum(t for t, sg in zip(seg_ms, segs) if sg["kind"] == "gemm")
+    gemm_launch_ms = gemm_ms / sum(1 for sg in segs if sg["kind"] == "gemm")
+    tflops = gemm_flops / (gemm_ms / 1e3) / 1e12
+    pk = peaks()
+    fp4_peak = FP4_PER_BF16 * pk["bf16_sustained"]
+
+    # end to end: inputs from pinned host memory, LoRA gradients back to pinned host memory
+    host_in = {k: x_in[k].cpu().pin_memory() for k in x_in}
+    host_out = [gt.cpu().pin_memory() for gt in grads]
+    h2d = sum(t.numel() * t.element_size() for t in host_in.values())
+    d2h = sum(t.numel() * t.element_size() for t in host_out)
+    e2e_ev = [(ev(), ev()) for _ in range(K)]
+    torch.cuda.synchronize()
+    with torch.cuda.stream(stream):
+        for k in range(K):
+            flush.zero_()
+            e2e_ev[k][0].record(stream)
+            for key, t in host_in.items():
+                x_in[key].copy_(t, non_blocking=True)
+            run_step()
+            allreduce_grads()
+            for ho, gt in zip(host_out, grads):
+                ho.copy_(gt, non_blocking=True)
+            e2e_ev[k][1].record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = sum(s.elapsed_time(e) for s, e in e2e_ev)
+    if world > 1:
+        t = torch.tensor([e2e_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    if P.pact_get_device_status() != 0:
+        raise RuntimeError(P.pact_last_error())
+
+    cpu = None
+    if rank == 0 and world == 1 and not a.no_cpu_baseline:
+        ol = oracle_layer(a.workload, inputs)
+        rate, n, el, cores = oracle_rate(ol, inputs, min(a.cpu_tokens, M))
+        cpu = {"value": rate, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+               "sample": f"{min(a.cpu_tokens, M)} of {M} tokens per step ({n} steps, {el:.1f} s), one layer "
+                         f"fwd+bwd on the FP64 CPU oracle; weight layouts cached before timing"}
+
+    if rank == 0:
+        out = {
+            "metric": METRIC, "value": tokens_per_s, "unit": "tokens/s", "n_gpus": world, "steps": K,
+            "warmup": a.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "nvfp4", "data": "synthetic",
+            "config": {**config_block(a.workload, M), "parallelism": f"dp{world}" if world > 1 else "single"},
+            "frozen_proj_tflops": tflops,
+            "frac_fp4_peak": tflops / fp4_peak,
+            "roofline": {"bound": "tensor", "kernel": "k_nvfp4_gemm (frozen fwd + dgrad GEMMs)",
+                         "achieved": tflops, "peak": fp4_peak, "unit": "TFLOP/s", "frac": tflops / fp4_peak,
+                         "traffic": None,
+                         "peak_note": f"{pk['src']} sustained BF16 {pk['bf16_sustained']} TF/s x {FP4_PER_BF16} "
+                                      f"(nominal FP4/BF16 ratio)",
+                         "flops_per_step": gemm_flops, "avg_launch_ms": gemm_launch_ms},
+            "cpu_baseline": cpu,
+            "e2e": {"value": M * K * world / (e2e_ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+                    "d2h_bytes_per_step": d2h},
+            "gpu_launches": launches_per_step * K,
+            "clocks": clk.summary(),
+            "segments_ms": {"+".join(op.name for op in sg["ops"]): round(t, 4) for sg, t in zip(segs, seg_ms)},
+        }
+        print(json.dumps(out), flush=True)
+    for sg in segs:
+        sg["graph"] = None
+    if world > 1:
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

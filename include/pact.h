@@ -96,15 +96,19 @@ typedef struct {
  * Several projections that share an input can be concatenated along N (q|k|v,
  * gate|up): segment i covers output columns [seg_end[i-1], seg_end[i]) and has
  * its own rank-r adapter.
- *   Forward  (pact_frozen_gemm_fwd):   act = T [M x nseg*r], T = scale * X A^T as
- *     written by pact_lora_fwd (segment i uses columns i*r .. i*r+r-1);
- *     weight = B [N x r] (segments' B stacked along rows); adds act_i . B_i^T.
- *   Dgrad    (pact_frozen_gemm_dgrad): act = U [M x nseg*r], U = scale * dY B as
- *     written by pact_lora_bwd_u; weight = A [nseg*r x K] (segments' A stacked
- *     along rows); adds U . A (one contraction over nseg*r).
- * r is 16, 32, 48 or 64; nseg*r <= 64; nseg <= 4; every internal boundary
+ * With R = nseg*r, the activations act are [M x 2R]: an FP32-accurate value held as
+ * the unevaluated sum of two BF16 matrices, hi in columns 0..R-1 and lo in columns
+ * R..2R-1 (lo = BF16(v - hi)), so the BF16 rounding of the small intermediate does
+ * not reach the output.
+ *   Forward  (pact_frozen_gemm_fwd):   act = T, T = scale * X A^T as written by
+ *     pact_lora_fwd (segment i uses columns i*r .. i*r+r-1 of each half);
+ *     weight = B [N x r] (segments' B stacked along rows); adds T_i . B_i^T.
+ *   Dgrad    (pact_frozen_gemm_dgrad): act = U, U = scale * dY B as written by
+ *     pact_lora_bwd_u; weight = A [R x K] (segments' A stacked along rows); adds
+ *     U . A (one contraction over R).
+ * r is 16, 32 or 48; nseg <= 3 and R <= 48; every internal boundary
  * seg_end[0..nseg-2] is a multiple of 256 and seg_end[nseg-1] == N.  act and
- * weight are row-major with leading dimension ld_act / ld_weight (elements). */
+ * weight are row-major with leading dimension ld_act (>= 2R) / ld_weight. */
 typedef struct {
     const pact_bf16 *act;
     int64_t ld_act;
@@ -167,36 +171,39 @@ PACT_API pact_status pact_weight_layout_cache(const pact_bf16 *W, int64_t ldw, i
 
 /* ---------------------------------------------------- A5: forward GEMM */
 /* [METHOD] bullet 1 with [LORA]:
- *   y[M x N] = BF16_RNE( deq(xq) . deq(w->fwd)^T  +  sum_i act_i . B_i^T )
+ *   y[M x N] = BF16_RNE( residual + deq(xq) . deq(w->fwd)^T + sum_i T_i . B_i^T )
  * FP32 accumulation in tensor memory.  xq is [M x K], w->fwd [N x K]; y has row
- * stride ldy.  lora may be NULL (frozen GEMM only). */
+ * stride ldy.  lora may be NULL (frozen GEMM only); residual (BF16 [M x N], row
+ * stride ldr, e.g. the residual stream) may be NULL and may equal y (in place). */
 PACT_API pact_status pact_frozen_gemm_fwd(const pact_nvfp4_t *xq, const pact_weight_cache_t *w,
-                                 const pact_lora_t *lora, pact_bf16 *y, int64_t ldy,
-                                 pact_stream_t stream);
+                                          const pact_lora_t *lora, const pact_bf16 *residual, int64_t ldr,
+                                          pact_bf16 *y, int64_t ldy, pact_stream_t stream);
 
 /* ------------------------------------------------------ A6: dgrad GEMM */
 /* [METHOD] bullet 1 (input gradient) with [LORA]:
- *   dx[M x K] (+)= BF16_RNE( deq(dyq) . deq(w->bwd)^T  +  U . A )
+ *   dx[M x K] = BF16_RNE( residual + deq(dyq) . deq(w->bwd)^T + U . A )
  * dyq is the NVFP4 upstream gradient [M x N] (pact_quantize_nvfp4), w->bwd
- * [K x N].  With accumulate != 0 the existing dx is added before rounding.
- * lora may be NULL. */
+ * [K x N].  lora and residual may be NULL; residual may equal dx (accumulate in
+ * place). */
 PACT_API pact_status pact_frozen_gemm_dgrad(const pact_nvfp4_t *dyq, const pact_weight_cache_t *w,
-                                   const pact_lora_t *lora, pact_bf16 *dx, int64_t lddx,
-                                   int accumulate, pact_stream_t stream);
+                                            const pact_lora_t *lora, const pact_bf16 *residual, int64_t ldr,
+                                            pact_bf16 *dx, int64_t lddx, pact_stream_t stream);
 
 /* ------------------------------------------------------ A7: LoRA forward */
-/* [LORA]: T[M x R] = BF16_RNE(scale * X . A^T) for X [M x K] (row stride ldx) and
- * A [R x K] (row stride K; R = nseg*r stacked adapters sharing X).  T has row
- * stride ldt.  R is a multiple of 16, at most 64. */
+/* [LORA]: T = scale * X . A^T for X [M x K] (row stride ldx) and A [R x K] (row
+ * stride K; R = nseg*r stacked adapters sharing X), FP32-accumulated and written
+ * as hi + lo BF16 halves: T [M x 2R] (row stride ldt >= 2R), hi = BF16_RNE(t) in
+ * columns 0..R-1, lo = BF16_RNE(t - hi) in columns R..2R-1.  R is 16, 32, 48 or 64. */
 PACT_API pact_status pact_lora_fwd(const pact_bf16 *x, int64_t ldx, int64_t M, int64_t K,
                           const pact_bf16 *A, int R, float scale, pact_bf16 *T, int64_t ldt,
                           pact_stream_t stream);
 
 /* --------------------------------------------------- A8: LoRA backward */
 /* [LORA] gradients, BF16 throughout ([METHOD]: adapters stay BF16).
- * pact_lora_bwd_u: U[:, i*r .. i*r+r-1] = BF16_RNE(scale * dY[:, seg_i] . B[seg_i, :])
- *   for dY [M x N] (row stride lddy), B [N x r]; U [M x nseg*r] (row stride ldu)
- *   feeds pact_frozen_gemm_dgrad and pact_lora_bwd. */
+ * pact_lora_bwd_u: U[:, i*r .. i*r+r-1] = scale * dY[:, seg_i] . B[seg_i, :] for dY
+ *   [M x N] (row stride lddy), B [N x r]; written like T as hi + lo BF16 halves,
+ *   U [M x 2*nseg*r] (row stride ldu).  U feeds pact_frozen_gemm_dgrad and
+ *   pact_lora_bwd.  Internal segment ends are multiples of 64. */
 PACT_API pact_status pact_lora_bwd_u(const pact_bf16 *dy, int64_t lddy, int64_t M, int64_t N,
                             const pact_bf16 *B, int r, int nseg, const int64_t *seg_end,
                             float scale, pact_bf16 *U, int64_t ldu, pact_stream_t stream);
@@ -211,12 +218,12 @@ typedef struct {
     int64_t ldx;
     const pact_nvfp4_t *xq;   /* [M x K] NVFP4, or NULL */
     const pact_bf16 *A;       /* [nseg*r x K] */
-    const pact_bf16 *U;       /* [M x nseg*r] from pact_lora_bwd_u, row stride ldu */
+    const pact_bf16 *U;       /* [M x 2*nseg*r] (hi + lo) from pact_lora_bwd_u, row stride ldu */
     int64_t ldu;
     int r, nseg;
     int64_t seg_end[4];
     float scale;
-    pact_bf16 *dA;            /* out [nseg*r x K]:  U^T . X~ */
+    pact_bf16 *dA;            /* out [nseg*r x K]:  (U_hi + U_lo)^T . X~ */
     pact_bf16 *dB;            /* out [N x r]: rows seg_i = scale * dY[:, seg_i]^T . (X~ . A_i^T) */
 } pact_lora_bwd_t;
 

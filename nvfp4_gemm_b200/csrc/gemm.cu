@@ -36,6 +36,9 @@ constexpr int OFF_B = A_BYTES;
 constexpr int OFF_SFA = OFF_B + B_BYTES;
 constexpr int OFF_SFB = OFF_SFA + SFA_BYTES;
 constexpr int STAGE_BYTES = OFF_SFB + SFB_BYTES;  // 55296, a multiple of 1024
+// A LoRA stage holds up to 6 activation chunks (4 KB) and then the weight tile.
+constexpr int OFF_LW = 6 * BM * 32;               // 24576
+static_assert(OFF_LW + 3 * BN * 32 <= STAGE_BYTES && OFF_LW + 4 * 48 * 128 <= STAGE_BYTES, "LoRA stage");
 constexpr int BAR_BYTES = 256;
 constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + BAR_BYTES;
 constexpr int THREADS = 192;
@@ -54,9 +57,10 @@ struct Params {
     const uint8_t *sfb;   // scales of B (rows N, cols K)
     __nv_bfloat16 *out;
     int64_t ldo;
-    int accumulate;
+    const __nv_bfloat16 *res;   // optional residual added in the epilogue (may alias out)
+    int64_t ldr;
     int lora_mode;
-    int lora_steps;       // kind::f16 MMAs (K = 16 each) per tile
+    int lora_steps;       // weight chunks of K = 16 per tile (two MMAs each: hi and lo activations)
     int lora_r;
     int lora_nseg;
     int64_t seg_end[4];
@@ -135,20 +139,25 @@ k_nvfp4_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CU
                 if (p.lora_mode != LORA_NONE) {
                     if (!mbar_wait(&empty[stage], phase ^ 1)) { *abort_flag = 1; break; }
                     uint8_t *st = smem + stage * STAGE_BYTES;
+                    // LoRA stage: 2 * steps activation chunks (hi parts, then lo parts; 128
+                    // rows x 16 BF16 each) and the weight chunks at OFF_LW.
+                    const int R = p.lora_nseg * p.lora_r;
                     if (p.lora_mode == LORA_FWD) {
                         const int xs = lora_segment(p, n0) * p.lora_r;
-                        mbar_arrive_expect_tx(&full[stage], p.lora_steps * (BM * 32 + BN * 32));
+                        mbar_arrive_expect_tx(&full[stage], p.lora_steps * (2 * BM * 32 + BN * 32));
                         for (int c = 0; c < p.lora_steps; ++c) {
                             tma_load_2d(st + c * BM * 32, &tmLa, &full[stage], xs + 16 * c, m0);
-                            tma_load_2d(st + OFF_B + c * BN * 32, &tmLb, &full[stage], 16 * c, n0);
+                            tma_load_2d(st + (p.lora_steps + c) * BM * 32, &tmLa, &full[stage], R + xs + 16 * c, m0);
+                            tma_load_2d(st + OFF_LW + c * BN * 32, &tmLb, &full[stage], 16 * c, n0);
                         }
                     } else {
-                        const int R = p.lora_steps * 16;
-                        mbar_arrive_expect_tx(&full[stage], p.lora_steps * BM * 32 + 4 * R * 128);
-                        for (int c = 0; c < p.lora_steps; ++c)
+                        mbar_arrive_expect_tx(&full[stage], p.lora_steps * 2 * BM * 32 + 4 * R * 128);
+                        for (int c = 0; c < p.lora_steps; ++c) {
                             tma_load_2d(st + c * BM * 32, &tmLa, &full[stage], 16 * c, m0);
+                            tma_load_2d(st + (p.lora_steps + c) * BM * 32, &tmLa, &full[stage], R + 16 * c, m0);
+                        }
                         for (int q = 0; q < 4; ++q)
-                            tma_load_2d(st + OFF_B + q * R * 128, &tmLb, &full[stage], n0 + 64 * q, 0);
+                            tma_load_2d(st + OFF_LW + q * R * 128, &tmLb, &full[stage], n0 + 64 * q, 0);
                     }
                     pending |= 1u << stage;
                     pending_parity = (pending_parity & ~(1u << stage)) | (phase << stage);
@@ -192,14 +201,16 @@ k_nvfp4_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CU
                 tc_fence_after();
                 if (ok && lane == 0) {
                     const uint32_t st = smem_u32(smem + stage * STAGE_BYTES);
-                    const int R = p.lora_steps * 16;
+                    const int R = p.lora_nseg * p.lora_r;
                     for (int c = 0; c < p.lora_steps; ++c) {
-                        const uint64_t ad = smem_desc(st + c * BM * 32, 16, 256, SW_32);
                         const uint64_t bd = (p.lora_mode == LORA_FWD)
-                                                ? smem_desc(st + OFF_B + c * BN * 32, 16, 256, SW_32)
-                                                : smem_desc(st + OFF_B + c * 2048, R * 128, 1024, SW_128);
-                        mma_bf16(tmem + COL_ACC, ad, bd, idesc_lora, accum);
-                        accum = 1;
+                                                ? smem_desc(st + OFF_LW + c * BN * 32, 16, 256, SW_32)
+                                                : smem_desc(st + OFF_LW + c * 2048, R * 128, 1024, SW_128);
+                        for (int h = 0; h < 2; ++h) {  // hi part, then lo part
+                            const uint64_t ad = smem_desc(st + (h * p.lora_steps + c) * BM * 32, 16, 256, SW_32);
+                            mma_bf16(tmem + COL_ACC, ad, bd, idesc_lora, accum);
+                            accum = 1;
+                        }
                     }
                     tc_commit(&empty[stage]);
                 }
@@ -260,13 +271,14 @@ k_nvfp4_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CU
                 if (row < p.M) {
                     __nv_bfloat16 *dst = p.out + (size_t)row * p.ldo + n;
                     uint4 *d4 = reinterpret_cast<uint4 *>(dst);
+                    const uint4 *r4 = p.res ? reinterpret_cast<const uint4 *>(p.res + (size_t)row * p.ldr + n) : nullptr;
 #pragma unroll
                     for (int q = 0; q < 4; ++q) {
                         float f[8];
 #pragma unroll
                         for (int i = 0; i < 8; ++i) f[i] = __uint_as_float(r[8 * q + i]);
-                        if (p.accumulate) {
-                            const uint4 old = d4[q];
+                        if (r4) {
+                            const uint4 old = r4[q];
                             f[0] += bf16lo(old.x); f[1] += bf16hi(old.x); f[2] += bf16lo(old.y); f[3] += bf16hi(old.y);
                             f[4] += bf16lo(old.z); f[5] += bf16hi(old.z); f[6] += bf16lo(old.w); f[7] += bf16hi(old.w);
                         }
@@ -339,10 +351,9 @@ static pact_status ensure_attrs() {
 
 static pact_status check_lora(const pact_lora_t *l, int64_t M, int64_t N, int64_t Kout, bool dgrad, const char *what) {
     PACT_CHECK(l->act && l->weight, PACT_ERR_INVALID_ARG, "%s: LoRA act/weight NULL", what);
-    PACT_CHECK(l->r == 16 || l->r == 32 || l->r == 48 || l->r == 64, PACT_ERR_SHAPE, "%s: LoRA r must be 16/32/48/64",
-               what);
-    PACT_CHECK(l->nseg >= 1 && l->nseg <= 4 && l->nseg * l->r <= 64, PACT_ERR_SHAPE,
-               "%s: LoRA needs 1 <= nseg <= 4 and nseg * r <= 64", what);
+    PACT_CHECK(l->r == 16 || l->r == 32 || l->r == 48, PACT_ERR_SHAPE, "%s: LoRA r must be 16, 32 or 48", what);
+    PACT_CHECK(l->nseg >= 1 && l->nseg <= 3 && l->nseg * l->r <= 48, PACT_ERR_SHAPE,
+               "%s: LoRA needs 1 <= nseg <= 3 and nseg * r <= 48", what);
     const int R = l->nseg * l->r;
     if (!dgrad) {
         int64_t prev = 0;
@@ -352,11 +363,11 @@ static pact_status check_lora(const pact_lora_t *l, int64_t M, int64_t N, int64_
                        "%s: LoRA segment ends must increase, be multiples of 256 and end at N", what);
             prev = e;
         }
-        PACT_CHECK(l->ld_act >= R && l->ld_weight >= l->r, PACT_ERR_SHAPE, "%s: LoRA leading dimensions too small",
-                   what);
+        PACT_CHECK(l->ld_act >= 2 * R && l->ld_weight >= l->r, PACT_ERR_SHAPE,
+                   "%s: LoRA leading dimensions too small", what);
     } else {
-        PACT_CHECK(l->ld_act >= R && l->ld_weight >= Kout, PACT_ERR_SHAPE, "%s: LoRA leading dimensions too small",
-                   what);
+        PACT_CHECK(l->ld_act >= 2 * R && l->ld_weight >= Kout, PACT_ERR_SHAPE,
+                   "%s: LoRA leading dimensions too small", what);
     }
     PACT_CHECK(aligned16(l->act) && aligned16(l->weight) && l->ld_act % 8 == 0 && l->ld_weight % 8 == 0,
                PACT_ERR_ALIGN, "%s: LoRA pointers must be 16-byte aligned with leading dims %% 8 == 0", what);
@@ -366,12 +377,15 @@ static pact_status check_lora(const pact_lora_t *l, int64_t M, int64_t N, int64_
 
 // D[M x N] = deq(a) . deq(b)^T (+ LoRA); a [M x K], b [N x K].
 static pact_status run(const pact_nvfp4_t *a, const pact_nvfp4_t *b, const pact_lora_t *lora, bool dgrad,
-                       pact_bf16 *out, int64_t ldo, int accumulate, cudaStream_t stream, const char *what) {
+                       const pact_bf16 *res, int64_t ldr, pact_bf16 *out, int64_t ldo, cudaStream_t stream,
+                       const char *what) {
     const int64_t M = a->rows, K = a->cols, N = b->rows;
     PACT_CHECK(M <= 0x7FFFFFFF && N <= 0x7FFFFFFF && K <= 0x7FFFFFFF, PACT_ERR_SHAPE, "%s: dimension too large", what);
     PACT_CHECK(out, PACT_ERR_INVALID_ARG, "%s: output NULL", what);
     PACT_CHECK(ldo >= N && ldo % 8 == 0 && aligned16(out), PACT_ERR_ALIGN,
                "%s: output must be 16-byte aligned with ld >= %lld and ld %% 8 == 0", what, (long long)N);
+    PACT_CHECK(!res || (ldr >= N && ldr % 8 == 0 && aligned16(res)), PACT_ERR_ALIGN,
+               "%s: residual must be 16-byte aligned with ld >= %lld and ld %% 8 == 0", what, (long long)N);
     pact_status s = lora ? check_lora(lora, M, N, N, dgrad, what) : PACT_OK;
     if (s != PACT_OK) return s;
     s = ensure_attrs();
@@ -389,7 +403,8 @@ static pact_status run(const pact_nvfp4_t *a, const pact_nvfp4_t *b, const pact_
     p.sfb = static_cast<const uint8_t *>(b->scales);
     p.out = reinterpret_cast<__nv_bfloat16 *>(out);
     p.ldo = ldo;
-    p.accumulate = accumulate ? 1 : 0;
+    p.res = reinterpret_cast<const __nv_bfloat16 *>(res);
+    p.ldr = ldr;
     p.lora_mode = LORA_NONE;
     p.lora_steps = 0; p.lora_r = 0; p.lora_nseg = 1;
     for (int i = 0; i < 4; ++i) p.seg_end[i] = N;
@@ -400,7 +415,7 @@ static pact_status run(const pact_nvfp4_t *a, const pact_nvfp4_t *b, const pact_
         p.lora_r = lora->r;
         p.lora_nseg = lora->nseg;
         for (int i = 0; i < 4; ++i) p.seg_end[i] = i < lora->nseg ? lora->seg_end[i] : N;
-        s = make_map(&tmLa, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, lora->act, R, M, lora->ld_act * 2, 16, BM,
+        s = make_map(&tmLa, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, lora->act, 2 * R, M, lora->ld_act * 2, 16, BM,
                      CU_TENSOR_MAP_SWIZZLE_32B, what);
         if (s != PACT_OK) return s;
         if (!dgrad) {
@@ -430,25 +445,28 @@ using namespace pact;
 extern "C" {
 
 pact_status pact_frozen_gemm_fwd(const pact_nvfp4_t *xq, const pact_weight_cache_t *w, const pact_lora_t *lora,
-                                 pact_bf16 *y, int64_t ldy, pact_stream_t stream) {
+                                 const pact_bf16 *residual, int64_t ldr, pact_bf16 *y, int64_t ldy,
+                                 pact_stream_t stream) {
     PACT_CHECK(xq && w, PACT_ERR_INVALID_ARG, "pact_frozen_gemm_fwd: NULL argument");
     const int64_t N = w->fwd.rows, K = w->fwd.cols;
     pact_status s = check_nvfp4(&w->fwd, N, K, "w->fwd");
     if (s == PACT_OK) s = check_nvfp4(xq, xq->rows, K, "xq");
     if (s != PACT_OK) return s;
     PACT_CHECK(xq->rows >= 1 && N % 64 == 0 && K % 64 == 0, PACT_ERR_SHAPE, "pact_frozen_gemm_fwd: bad shape");
-    return gemm::run(xq, &w->fwd, lora, false, y, ldy, 0, (cudaStream_t)stream, "pact_frozen_gemm_fwd");
+    return gemm::run(xq, &w->fwd, lora, false, residual, ldr, y, ldy, (cudaStream_t)stream, "pact_frozen_gemm_fwd");
 }
 
 pact_status pact_frozen_gemm_dgrad(const pact_nvfp4_t *dyq, const pact_weight_cache_t *w, const pact_lora_t *lora,
-                                   pact_bf16 *dx, int64_t lddx, int accumulate, pact_stream_t stream) {
+                                   const pact_bf16 *residual, int64_t ldr, pact_bf16 *dx, int64_t lddx,
+                                   pact_stream_t stream) {
     PACT_CHECK(dyq && w, PACT_ERR_INVALID_ARG, "pact_frozen_gemm_dgrad: NULL argument");
     const int64_t K = w->bwd.rows, N = w->bwd.cols;
     pact_status s = check_nvfp4(&w->bwd, K, N, "w->bwd");
     if (s == PACT_OK) s = check_nvfp4(dyq, dyq->rows, N, "dyq");
     if (s != PACT_OK) return s;
     PACT_CHECK(dyq->rows >= 1 && N % 64 == 0 && K % 64 == 0, PACT_ERR_SHAPE, "pact_frozen_gemm_dgrad: bad shape");
-    return gemm::run(dyq, &w->bwd, lora, true, dx, lddx, accumulate, (cudaStream_t)stream, "pact_frozen_gemm_dgrad");
+    return gemm::run(dyq, &w->bwd, lora, true, residual, ldr, dx, lddx, (cudaStream_t)stream,
+                     "pact_frozen_gemm_dgrad");
 }
 
 }  // extern "C"

@@ -34,7 +34,7 @@ struct RowArgs {
     int R, r, nseg;
     int64_t seg_end[4];
     float scale;
-    pact_bf16 *out_bf16;  // one of these two
+    pact_bf16 *out_bf16;  // one of these two; BF16 output is hi (columns 0..R-1) + lo (R..2R-1)
     float *out_f32;
     int64_t ldo;
 };
@@ -99,8 +99,15 @@ __global__ void __launch_bounds__(256) k_rows(const RowArgs a) {
         for (int i = 0; i < 8; ++i) {
             const int j = jl + 8 * i;
             if (j < a.R) {
-                if (a.out_f32) a.out_f32[m * a.ldo + j] = acc[i] * a.scale;
-                else a.out_bf16[m * a.ldo + j] = __bfloat16_as_ushort(__float2bfloat16_rn(acc[i] * a.scale));
+                const float v = acc[i] * a.scale;
+                if (a.out_f32) {
+                    a.out_f32[m * a.ldo + j] = v;
+                } else {  // v as the unevaluated sum hi + lo of two BF16 values
+                    const __nv_bfloat16 hi = __float2bfloat16_rn(v);
+                    a.out_bf16[m * a.ldo + j] = __bfloat16_as_ushort(hi);
+                    a.out_bf16[m * a.ldo + a.R + j] =
+                        __bfloat16_as_ushort(__float2bfloat16_rn(v - __bfloat162float(hi)));
+                }
             }
         }
     }
@@ -116,6 +123,7 @@ constexpr int TA = 64, TB = 64, MC = 32, MCHUNK = 256;
 struct OuterArgs {
     const pact_bf16 *p;
     int64_t ldp;
+    int p_split;  // P holds hi (columns 0..A-1) + lo (A..2A-1)
     const pact_bf16 *q;
     const float *qf;
     pact_nvfp4_t qq;
@@ -149,7 +157,15 @@ __global__ void __launch_bounds__(256) k_outer(const OuterArgs o) {
             const int rr = t >> 3, cc = (t & 7) * 8;
             const int64_t m = m0 + rr, a = a0 + cc;
             float v[8] = {0, 0, 0, 0, 0, 0, 0, 0};
-            if (m < mend && a < o.A) load8_bf16(o.p + m * o.ldp + a, v);
+            if (m < mend && a < o.A) {
+                load8_bf16(o.p + m * o.ldp + a, v);
+                if (o.p_split) {
+                    float lo[8];
+                    load8_bf16(o.p + m * o.ldp + o.A + a, lo);
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) v[i] += lo[i];
+                }
+            }
 #pragma unroll
             for (int i = 0; i < 8; ++i) ps[rr][cc + i] = v[i];
         }
@@ -223,7 +239,7 @@ pact_status pact_lora_fwd(const pact_bf16 *x, int64_t ldx, int64_t M, int64_t K,
     PACT_CHECK(x && A && T, PACT_ERR_INVALID_ARG, "pact_lora_fwd: NULL argument");
     PACT_CHECK(M >= 1 && K >= 64 && K % 64 == 0 && R >= 16 && R <= 64 && R % 16 == 0, PACT_ERR_SHAPE,
                "pact_lora_fwd: need M >= 1, K a multiple of 64, R in {16, 32, 48, 64}");
-    PACT_CHECK(ldx >= K && ldx % 8 == 0 && ldt >= R && ldt % 8 == 0 && aligned16(x) && aligned16(A) && aligned16(T),
+    PACT_CHECK(ldx >= K && ldx % 8 == 0 && ldt >= 2 * R && ldt % 8 == 0 && aligned16(x) && aligned16(A) && aligned16(T),
                PACT_ERR_ALIGN, "pact_lora_fwd: pointers 16-byte aligned, leading dims %% 8 == 0");
     RowArgs a = {};
     a.x = x; a.ldx = ldx; a.use_xq = 0; a.M = M; a.K = K;
@@ -246,7 +262,7 @@ pact_status pact_lora_bwd_u(const pact_bf16 *dy, int64_t lddy, int64_t M, int64_
                    "pact_lora_bwd_u: segment ends must increase by multiples of 64 and end at N");
         prev = seg_end[i];
     }
-    PACT_CHECK(lddy >= N && lddy % 8 == 0 && ldu >= nseg * r && ldu % 8 == 0 && aligned16(dy) && aligned16(B) &&
+    PACT_CHECK(lddy >= N && lddy % 8 == 0 && ldu >= 2 * nseg * r && ldu % 8 == 0 && aligned16(dy) && aligned16(B) &&
                    aligned16(U),
                PACT_ERR_ALIGN, "pact_lora_bwd_u: pointers 16-byte aligned, leading dims %% 8 == 0");
     RowArgs a = {};
@@ -281,7 +297,7 @@ pact_status pact_lora_bwd(const pact_lora_bwd_t *g, void *workspace, size_t ws_b
     const int R = nseg * r;
     PACT_CHECK(ws_bytes >= pact_lora_bwd_workspace_bytes(M, N, K, r, nseg), PACT_ERR_INVALID_ARG,
                "pact_lora_bwd: workspace too small");
-    PACT_CHECK(g->lddy >= N && g->lddy % 8 == 0 && g->ldu >= R && g->ldu % 8 == 0 && aligned16(g->dy) &&
+    PACT_CHECK(g->lddy >= N && g->lddy % 8 == 0 && g->ldu >= 2 * R && g->ldu % 8 == 0 && aligned16(g->dy) &&
                    aligned16(g->A) && aligned16(g->U) && aligned16(g->dA) && aligned16(g->dB) && aligned16(workspace) &&
                    (!g->x || (g->ldx >= K && g->ldx % 8 == 0 && aligned16(g->x))),
                PACT_ERR_ALIGN, "pact_lora_bwd: pointers 16-byte aligned, leading dims %% 8 == 0");
@@ -310,7 +326,7 @@ pact_status pact_lora_bwd(const pact_lora_bwd_t *g, void *workspace, size_t ws_b
     const unsigned mchunks = (unsigned)((M + MCHUNK - 1) / MCHUNK);
     // dA = U^T . X~   [R x K]
     OuterArgs o = {};
-    o.p = g->U; o.ldp = g->ldu; o.q = g->x; o.qq = g->xq ? *g->xq : none; o.q_kind = g->xq ? 1 : 0; o.ldq = g->ldx;
+    o.p = g->U; o.ldp = g->ldu; o.p_split = 1; o.q = g->x; o.qq = g->xq ? *g->xq : none; o.q_kind = g->xq ? 1 : 0; o.ldq = g->ldx;
     o.M = M; o.A = R; o.Bn = K; o.segmented = 0; o.ws = wda; o.ldws = K;
     k_outer<<<dim3((unsigned)((R + TA - 1) / TA), (unsigned)((K + TB - 1) / TB), mchunks), 256, 0, st>>>(o);
     // dB = dY^T . T~ (segment-wise)   [N x r]

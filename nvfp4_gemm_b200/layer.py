@@ -1,0 +1,214 @@
+"""One PACT LoRA decoder layer: the NVFP4 data flow through its seven frozen
+projections, forward and backward, composed from libpact calls.
+
+Data flow (PACT blog summary, section "方法" (method); PACT abstract):
+  forward   xq1, x1, rstd1 = RMSNorm+quantize(h)            x1 BF16 feeds LoRA only
+            qkv  = NVFP4 GEMM(xq1, W_qkv) + LoRA(x1)          q|k|v concatenated along N
+            [attention core: not on the NVFP4 path; a synthetic BF16 `attn` stands in]
+            h2   = h + NVFP4 GEMM(q(attn), W_o) + LoRA(attn)  residual fused in the epilogue
+            xq2, x2, rstd2 = RMSNorm+quantize(h2)
+            gu   = NVFP4 GEMM(xq2, W_gu) + LoRA(x2)           gate|up concatenated along N
+            m, mq, gq, uq = SiLU-multiply+quantize(gate, up)  gq, uq saved for backward
+            out  = h2 + NVFP4 GEMM(mq, W_down) + LoRA(m)
+  saved for backward: xq1, rstd1, xq2, rstd2, gq, uq (NVFP4) and attn.
+  backward  the input gradients run the NVFP4 dgrad GEMMs on the cached transposed,
+            re-quantized weight layouts; the LoRA weight gradients read the saved
+            NVFP4 copies (q/k/v, gate/up: xq; down: m~ recomputed from gq, uq) or
+            attn (o).  The attention backward is replaced by a synthetic d(qkv).
+
+Every op writes into buffers allocated once here, so a whole step can be captured
+into CUDA graphs.  Nothing below computes on the host or in PyTorch kernels.
+"""
+from __future__ import annotations
+
+from dataclasses import dataclass, field
+from typing import Callable, Dict, List
+
+import torch
+
+from . import pact as P
+
+
+@dataclass
+class Op:
+    name: str
+    fn: Callable[[], None]
+    kind: str = "other"        # "gemm" for the NVFP4 frozen GEMMs
+    flops: float = 0.0         # algorithmic FLOPs of a GEMM op
+    kernels: int = 1           # libpact kernels one call launches
+
+
+@dataclass
+class LayerShape:
+    M: int
+    H: int
+    I: int
+    KV: int
+    r: int = 16
+    alpha: float = 32.0
+    eps: float = 1e-5
+
+    @property
+    def scale(self) -> float:
+        return self.alpha / self.r
+
+    @property
+    def n_qkv(self) -> int:
+        return self.H + 2 * self.KV
+
+    def frozen_flops(self) -> float:
+        """2 M N K for the forward and the dgrad of the seven frozen projections."""
+        nk = self.n_qkv * self.H + self.H * self.H + 2 * self.I * self.H + self.H * self.I
+        return 2.0 * 2.0 * self.M * nk
+
+
+class PactLayer:
+    """Weights are BF16 device tensors in PyTorch [out, in] layout:
+    w = {q, k, v, o, gate, up, down}; lora_a = {p: [r, in]}, lora_b = {p: [out, r]};
+    gamma1, gamma2: [H].  Frozen weights are cached as NVFP4 forward/backward layouts
+    at construction (once)."""
+
+    def __init__(self, shape: LayerShape, w: Dict[str, torch.Tensor], lora_a: Dict[str, torch.Tensor],
+                 lora_b: Dict[str, torch.Tensor], gamma1: torch.Tensor, gamma2: torch.Tensor):
+        self.s = shape
+        S = shape
+        dev = gamma1.device
+        cat = lambda names, d: torch.cat([d[n] for n in names], 0).contiguous()
+        # frozen weights: concatenated where projections share an input, then cached
+        self.c_qkv = P.pact_weight_layout_cache(cat(("q", "k", "v"), w))
+        self.c_o = P.pact_weight_layout_cache(w["o"].contiguous())
+        self.c_gu = P.pact_weight_layout_cache(cat(("gate", "up"), w))
+        self.c_d = P.pact_weight_layout_cache(w["down"].contiguous())
+        # adapters, stacked like the weights
+        self.a_qkv, self.b_qkv = cat(("q", "k", "v"), lora_a), cat(("q", "k", "v"), lora_b)
+        self.a_o, self.b_o = lora_a["o"].contiguous(), lora_b["o"].contiguous()
+        self.a_gu, self.b_gu = cat(("gate", "up"), lora_a), cat(("gate", "up"), lora_b)
+        self.a_d, self.b_d = lora_a["down"].contiguous(), lora_b["down"].contiguous()
+        self.seg_qkv = [S.H, S.H + S.KV, S.H + 2 * S.KV]
+        self.seg_gu = [S.I, 2 * S.I]
+        self.g1, self.g2 = gamma1, gamma2
+        M, H, I, r = S.M, S.H, S.I, S.r
+        bf = lambda *sh: torch.empty(sh, dtype=torch.bfloat16, device=dev)
+        nv = lambda rows, cols: P.NVFP4Tensor.empty(rows, cols, dev)
+        # forward activations
+        self.xq1, self.x1, self.rstd1 = nv(M, H), bf(M, H), torch.empty(M, dtype=torch.float32, device=dev)
+        self.t_qkv, self.qkv = bf(M, 2 * 3 * r), bf(M, S.n_qkv)
+        self.aq, self.t_o, self.h2 = nv(M, H), bf(M, 2 * r), bf(M, H)
+        self.xq2, self.x2, self.rstd2 = nv(M, H), bf(M, H), torch.empty(M, dtype=torch.float32, device=dev)
+        self.t_gu, self.gu = bf(M, 2 * 2 * r), bf(M, 2 * I)
+        self.m, self.mq, self.gq, self.uq = bf(M, I), nv(M, I), nv(M, I), nv(M, I)
+        self.t_d, self.out = bf(M, 2 * r), bf(M, H)
+        # backward
+        self.u_d, self.doq, self.dm = bf(M, 2 * r), nv(M, H), bf(M, I)
+        self.dgu, self.dguq, self.m_re = bf(M, 2 * I), nv(M, 2 * I), bf(M, I)
+        self.u_gu, self.dx2 = bf(M, 2 * 2 * r), bf(M, H)
+        self.dh2, self.dh2q = bf(M, H), nv(M, H)
+        self.u_o, self.dattn = bf(M, 2 * r), bf(M, H)
+        self.u_qkv, self.dqkvq, self.dx1, self.dh = bf(M, 2 * 3 * r), nv(M, S.n_qkv), bf(M, H), bf(M, H)
+        # LoRA weight gradients (BF16, same stacking as the adapters)
+        self.grads = {
+            "a_qkv": torch.empty_like(self.a_qkv), "b_qkv": torch.empty_like(self.b_qkv),
+            "a_o": torch.empty_like(self.a_o), "b_o": torch.empty_like(self.b_o),
+            "a_gu": torch.empty_like(self.a_gu), "b_gu": torch.empty_like(self.b_gu),
+            "a_d": torch.empty_like(self.a_d), "b_d": torch.empty_like(self.b_d),
+        }
+        ws = max(P.pact_lora_bwd_workspace_bytes(M, S.n_qkv, H, r, 3),
+                 P.pact_lora_bwd_workspace_bytes(M, 2 * I, H, r, 2),
+                 P.pact_lora_bwd_workspace_bytes(M, H, I, r, 1),
+                 P.pact_lora_bwd_workspace_bytes(M, H, H, r, 1))
+        self.ws = torch.empty(ws, dtype=torch.uint8, device=dev)
+        # LoRA descriptors for the fused GEMM epilogue
+        self.l_qkv_f = P.lora_struct(self.t_qkv, self.b_qkv, r, self.seg_qkv)
+        self.l_o_f = P.lora_struct(self.t_o, self.b_o, r, [H])
+        self.l_gu_f = P.lora_struct(self.t_gu, self.b_gu, r, self.seg_gu)
+        self.l_d_f = P.lora_struct(self.t_d, self.b_d, r, [H])
+        self.l_d_b = P.lora_struct(self.u_d, self.a_d, 1 * r, [I])
+        self.l_gu_b = P.lora_struct(self.u_gu, self.a_gu, 2 * r, [H])
+        self.l_o_b = P.lora_struct(self.u_o, self.a_o, r, [H])
+        self.l_qkv_b = P.lora_struct(self.u_qkv, self.a_qkv, 3 * r, [H])
+        self.inputs = None
+
+    # ------------------------------------------------------------------ op lists
+    def bind(self, h: torch.Tensor, attn: torch.Tensor, d_out: torch.Tensor, d_qkv: torch.Tensor):
+        """Attach the step's inputs: layer input h [M, H], the attention-output stand-in
+        attn [M, H], the upstream gradient d_out [M, H] and the attention-backward
+        stand-in d_qkv [M, H + 2 KV].  The op lists read these tensors in place."""
+        self.inputs = (h, attn, d_out, d_qkv)
+
+    def forward_ops(self) -> List[Op]:
+        S, s = self.s, self.s.scale
+        h, attn, _, _ = self.inputs
+        I = S.I
+        gemm = lambda M, N, K: 2.0 * M * N * K
+        return [
+            Op("rmsnorm_quant_1", lambda: P.pact_rmsnorm_quant(h, self.g1, S.eps, self.xq1, self.x1, self.rstd1)),
+            Op("lora_fwd_qkv", lambda: P.pact_lora_fwd(self.x1, self.a_qkv, s, self.t_qkv)),
+            Op("gemm_fwd_qkv", lambda: P.pact_frozen_gemm_fwd(self.xq1, self.c_qkv, self.l_qkv_f, y=self.qkv),
+               "gemm", gemm(S.M, S.n_qkv, S.H)),
+            Op("quantize_attn", lambda: P.pact_quantize_nvfp4(attn, self.aq)),
+            Op("lora_fwd_o", lambda: P.pact_lora_fwd(attn, self.a_o, s, self.t_o)),
+            Op("gemm_fwd_o", lambda: P.pact_frozen_gemm_fwd(self.aq, self.c_o, self.l_o_f, residual=h, y=self.h2),
+               "gemm", gemm(S.M, S.H, S.H)),
+            Op("rmsnorm_quant_2", lambda: P.pact_rmsnorm_quant(self.h2, self.g2, S.eps, self.xq2, self.x2,
+                                                               self.rstd2)),
+            Op("lora_fwd_gu", lambda: P.pact_lora_fwd(self.x2, self.a_gu, s, self.t_gu)),
+            Op("gemm_fwd_gu", lambda: P.pact_frozen_gemm_fwd(self.xq2, self.c_gu, self.l_gu_f, y=self.gu),
+               "gemm", gemm(S.M, 2 * I, S.H)),
+            Op("silu_mul_quant", lambda: P.pact_silu_mul_quant(self.gu[:, :I], self.gu[:, I:], self.m, self.mq,
+                                                               self.gq, self.uq)),
+            Op("lora_fwd_down", lambda: P.pact_lora_fwd(self.m, self.a_d, s, self.t_d)),
+            Op("gemm_fwd_down", lambda: P.pact_frozen_gemm_fwd(self.mq, self.c_d, self.l_d_f, residual=self.h2,
+                                                               y=self.out),
+               "gemm", gemm(S.M, S.H, I)),
+        ]
+
+    def backward_ops(self) -> List[Op]:
+        S, s, r = self.s, self.s.scale, self.s.r
+        H, I = S.H, S.I
+        _, attn, d_out, d_qkv = self.inputs
+        g = self.grads
+        gemm = lambda M, N, K: 2.0 * M * N * K
+        LB = 5  # kernels of one pact_lora_bwd call (plus two memsets)
+        return [
+            # down projection
+            Op("lora_bwd_u_down", lambda: P.pact_lora_bwd_u(d_out, self.b_d, r, [H], s, self.u_d)),
+            Op("quantize_dout", lambda: P.pact_quantize_nvfp4(d_out, self.doq)),
+            Op("gemm_dgrad_down", lambda: P.pact_frozen_gemm_dgrad(self.doq, self.c_d, self.l_d_b, dx=self.dm),
+               "gemm", gemm(S.M, I, H)),
+            Op("silu_mul_bwd_quant", lambda: P.pact_silu_mul_bwd_quant(self.dm, self.gq, self.uq, self.dgu,
+                                                                       self.dguq, self.m_re)),
+            Op("lora_bwd_down", lambda: P.pact_lora_bwd(d_out, self.a_d, self.u_d, r, [H], s, x=self.m_re,
+                                                        dA=g["a_d"], dB=g["b_d"], workspace=self.ws), kernels=LB),
+            # gate|up
+            Op("lora_bwd_u_gu", lambda: P.pact_lora_bwd_u(self.dgu, self.b_gu, r, self.seg_gu, s, self.u_gu)),
+            Op("gemm_dgrad_gu", lambda: P.pact_frozen_gemm_dgrad(self.dguq, self.c_gu, self.l_gu_b, dx=self.dx2),
+               "gemm", gemm(S.M, H, 2 * I)),
+            Op("lora_bwd_gu", lambda: P.pact_lora_bwd(self.dgu, self.a_gu, self.u_gu, r, self.seg_gu, s,
+                                                      xq=self.xq2, dA=g["a_gu"], dB=g["b_gu"], workspace=self.ws),
+               kernels=LB),
+            Op("rmsnorm_bwd_2", lambda: P.pact_rmsnorm_bwd(self.dx2, self.xq2, self.rstd2, self.g2, dres=d_out,
+                                                           dx=self.dh2, dxq=self.dh2q)),
+            # o projection (its output joined the residual stream h2)
+            Op("lora_bwd_u_o", lambda: P.pact_lora_bwd_u(self.dh2, self.b_o, r, [H], s, self.u_o)),
+            Op("gemm_dgrad_o", lambda: P.pact_frozen_gemm_dgrad(self.dh2q, self.c_o, self.l_o_b, dx=self.dattn),
+               "gemm", gemm(S.M, H, H)),
+            Op("lora_bwd_o", lambda: P.pact_lora_bwd(self.dh2, self.a_o, self.u_o, r, [H], s, x=attn,
+                                                     dA=g["a_o"], dB=g["b_o"], workspace=self.ws), kernels=LB),
+            # q|k|v (d_qkv stands in for the attention backward)
+            Op("lora_bwd_u_qkv", lambda: P.pact_lora_bwd_u(d_qkv, self.b_qkv, r, self.seg_qkv, s, self.u_qkv)),
+            Op("quantize_dqkv", lambda: P.pact_quantize_nvfp4(d_qkv, self.dqkvq)),
+            Op("gemm_dgrad_qkv", lambda: P.pact_frozen_gemm_dgrad(self.dqkvq, self.c_qkv, self.l_qkv_b, dx=self.dx1),
+               "gemm", gemm(S.M, H, S.n_qkv)),
+            Op("lora_bwd_qkv", lambda: P.pact_lora_bwd(d_qkv, self.a_qkv, self.u_qkv, r, self.seg_qkv, s,
+                                                       xq=self.xq1, dA=g["a_qkv"], dB=g["b_qkv"],
+                                                       workspace=self.ws), kernels=LB),
+            Op("rmsnorm_bwd_1", lambda: P.pact_rmsnorm_bwd(self.dx1, self.xq1, self.rstd1, self.g1, dres=self.dh2,
+                                                           dx=self.dh)),
+        ]
+
+    def step_ops(self) -> List[Op]:
+        return self.forward_ops() + self.backward_ops()
+
+    def step(self):
+        for op in self.step_ops():
+            op.fn()

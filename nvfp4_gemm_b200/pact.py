@@ -68,8 +68,9 @@ def _load() -> ctypes.CDLL:
         "pact_rmsnorm_quant": (S, [P, I64, P, F, I64, I64, NV, P, P, P]),
         "pact_silu_mul_quant": (S, [P, P, I64, I64, I64, P, NV, NV, NV, P]),
         "pact_weight_layout_cache": (S, [P, I64, I64, I64, P, ctypes.c_size_t, ctypes.POINTER(c_weight_cache), P]),
-        "pact_frozen_gemm_fwd": (S, [NV, ctypes.POINTER(c_weight_cache), ctypes.POINTER(c_lora), P, I64, P]),
-        "pact_frozen_gemm_dgrad": (S, [NV, ctypes.POINTER(c_weight_cache), ctypes.POINTER(c_lora), P, I64, I, P]),
+        "pact_frozen_gemm_fwd": (S, [NV, ctypes.POINTER(c_weight_cache), ctypes.POINTER(c_lora), P, I64, P, I64, P]),
+        "pact_frozen_gemm_dgrad": (S, [NV, ctypes.POINTER(c_weight_cache), ctypes.POINTER(c_lora), P, I64, P, I64,
+                                       P]),
         "pact_lora_fwd": (S, [P, I64, I64, I64, P, I, F, P, I64, P]),
         "pact_lora_bwd_u": (S, [P, I64, I64, I64, P, I, I, ctypes.POINTER(I64), F, P, I64, P]),
         "pact_lora_bwd_workspace_bytes": (ctypes.c_size_t, [I64, I64, I64, I, I]),
@@ -245,24 +246,28 @@ def pact_weight_layout_cache(W: torch.Tensor, stream=None) -> WeightCache:
 
 
 def pact_frozen_gemm_fwd(xq: NVFP4Tensor, w: WeightCache, lora: Optional[c_lora] = None,
-                         y: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+                         residual: Optional[torch.Tensor] = None, y: Optional[torch.Tensor] = None,
+                         stream=None) -> torch.Tensor:
     if y is None:
         y = torch.empty((xq.rows, w.N), dtype=torch.bfloat16, device=xq.codes.device)
     s = xq.c()
     _check(_lib.pact_frozen_gemm_fwd(ctypes.byref(s), ctypes.byref(w.cstruct),
                                      ctypes.byref(lora) if lora is not None else None,
+                                     _ptr(residual), _ld(residual) if residual is not None else 0,
                                      y.data_ptr(), _ld(y), _stream(stream)))
     return y
 
 
 def pact_frozen_gemm_dgrad(dyq: NVFP4Tensor, w: WeightCache, lora: Optional[c_lora] = None,
-                           dx: Optional[torch.Tensor] = None, accumulate: bool = False, stream=None) -> torch.Tensor:
+                           residual: Optional[torch.Tensor] = None, dx: Optional[torch.Tensor] = None,
+                           stream=None) -> torch.Tensor:
     if dx is None:
         dx = torch.empty((dyq.rows, w.K), dtype=torch.bfloat16, device=dyq.codes.device)
     s = dyq.c()
     _check(_lib.pact_frozen_gemm_dgrad(ctypes.byref(s), ctypes.byref(w.cstruct),
                                        ctypes.byref(lora) if lora is not None else None,
-                                       dx.data_ptr(), _ld(dx), int(bool(accumulate)), _stream(stream)))
+                                       _ptr(residual), _ld(residual) if residual is not None else 0,
+                                       dx.data_ptr(), _ld(dx), _stream(stream)))
     return dx
 
 
@@ -273,7 +278,7 @@ def pact_lora_fwd(x: torch.Tensor, A: torch.Tensor, scale: float, T: Optional[to
     M, K = x.shape
     R = A.shape[0]
     if T is None:
-        T = torch.empty((M, R), dtype=torch.bfloat16, device=x.device)
+        T = torch.empty((M, 2 * R), dtype=torch.bfloat16, device=x.device)
     _check(_lib.pact_lora_fwd(x.data_ptr(), _ld(x), M, K, A.data_ptr(), R, float(scale), T.data_ptr(), _ld(T),
                               _stream(stream)))
     return T
@@ -284,7 +289,7 @@ def pact_lora_bwd_u(dy: torch.Tensor, B: torch.Tensor, r: int, seg_end: Sequence
     _bf16(dy, "dy")
     M, N = dy.shape
     if U is None:
-        U = torch.empty((M, r * len(seg_end)), dtype=torch.bfloat16, device=dy.device)
+        U = torch.empty((M, 2 * r * len(seg_end)), dtype=torch.bfloat16, device=dy.device)
     se = (ctypes.c_int64 * 4)(*(list(seg_end) + [0] * (4 - len(seg_end))))
     _check(_lib.pact_lora_bwd_u(dy.data_ptr(), _ld(dy), M, N, B.data_ptr(), r, len(seg_end), se, float(scale),
                                 U.data_ptr(), _ld(U), _stream(stream)))

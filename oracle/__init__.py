@@ -85,6 +85,7 @@ def _load():
             lib.orc_silu_mul_bwd.argtypes = [P, P, P, I, P, P]
             lib.orc_rmsnorm_bwd.argtypes = [P, P, P, P, I, I, P]
             lib.orc_num_threads.restype = ctypes.c_int
+            lib.orc_bf16_rne_array.argtypes = [P, I, P]
             _lib = lib
     return _lib
 
@@ -134,9 +135,10 @@ def bf16_to_f64(bits: np.ndarray) -> np.ndarray:
 
 def f64_to_bf16(v: np.ndarray) -> np.ndarray:
     """Single-rounding RNE float64 -> BF16 bits, element by element (orc_bf16_rne)."""
-    lib = _load()
-    flat = np.asarray(v, dtype=np.float64).ravel()
-    out = np.fromiter((lib.orc_bf16_rne(float(x)) for x in flat), dtype=np.uint16, count=flat.size)
+    flat = _c(np.asarray(v, dtype=np.float64).ravel(), np.float64)
+    out = np.empty(flat.size, dtype=np.uint16)
+    if flat.size:
+        _load().orc_bf16_rne_array(_p(flat), flat.size, _p(out))
     return out.reshape(np.shape(v))
 
 
@@ -147,9 +149,20 @@ class NVFP4:
 
     def __init__(self, codes: np.ndarray, scales: np.ndarray, rows: int, cols: int):
         self.codes, self.scales, self.rows, self.cols = codes, scales, rows, cols
+        self._deq = None
 
     def dequantize(self) -> np.ndarray:
-        return dequantize(self)
+        """Dequantized values (computed once per tensor; the tensor is immutable)."""
+        if self._deq is None:
+            self._deq = dequantize(self)
+            self._deq.flags.writeable = False
+        return self._deq
+
+    def rows_slice(self, rows) -> "NVFP4":
+        """The NVFP4 tensor made of the given rows (blocks run along rows, so a row
+        subset is itself a valid NVFP4 tensor)."""
+        idx = np.asarray(rows)
+        return NVFP4(self.codes[idx], self.scales[idx], len(idx), self.cols)
 
     def packed_scales(self) -> np.ndarray:
         return pack_scales(self.scales, self.rows, self.cols)
@@ -211,7 +224,7 @@ def gemm_nt(a: np.ndarray, b: np.ndarray) -> np.ndarray:
 
 def nvfp4_gemm(aq: NVFP4, bq: NVFP4) -> np.ndarray:
     """[METHOD] NVFP4 GEMM: deq(A) . deq(B)^T, accumulated without rounding."""
-    return gemm_nt(dequantize(aq), dequantize(bq))
+    return gemm_nt(aq.dequantize(), bq.dequantize())
 
 
 def weight_cache(w_bits: np.ndarray):
@@ -219,7 +232,7 @@ def weight_cache(w_bits: np.ndarray):
     Backward: the forward layout is rebuilt (dequantized, exact in BF16), transposed
     to [K x N] and re-quantized along N: Wb = q(deq(Wf)^T)."""
     wf = quantize(w_bits)
-    wd = dequantize(wf)
+    wd = wf.dequantize()
     wd_bits = f64_to_bf16_exact(wd.T)
     wb = quantize(wd_bits)
     return wf, wb

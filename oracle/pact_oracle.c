@@ -281,3 +281,10 @@ void orc_rmsnorm_bwd(const double *dy, const double *yh, const double *rstd,
         }
     }
 }
+
+/* Element-wise orc_bf16_rne over an array (the stage outputs the data flow stores
+ * as BF16: GEMM outputs, gradients). */
+void orc_bf16_rne_array(const double *v, int64_t n, uint16_t *out) {
+#pragma omp parallel for schedule(static)
+    for (int64_t i = 0; i < n; ++i) out[i] = orc_bf16_rne(v[i]);
+}

@@ -121,3 +121,31 @@ def layer_shapes(name: str) -> dict:
 def tokens(name: str) -> int:
     c = LAYERS[name]
     return c["batch"] * c["seq"]
+
+
+def layer_inputs(name: str, M: int = None, r: int = LORA_R) -> dict:
+    """BF16 bit arrays of one decoder layer's weights and one step's inputs:
+    frozen weights W_p ~ N(0, 0.02^2) (with the outlier mask when the workload has
+    one), LoRA A_p [r, in] and B_p [out, r] ~ N(0, 0.02^2), RMSNorm weights
+    gamma_i = 1 + N(0, 0.02^2), layer input h, attention-output stand-in attn,
+    upstream gradient d_out and attention-backward stand-in d_qkv ~ N(0, 1)."""
+    c = LAYERS[name]
+    M = M or tokens(name)
+    shp = layer_shapes(name)
+    w, a, b = {}, {}, {}
+    for p, proj in enumerate(PROJ):
+        N, K = shp[proj]
+        w[proj] = weight_bf16(p, (N, K), outliers=c["outliers"])
+        a[proj] = gaussian_bf16(20 + p, (r, K), std=0.02)
+        b[proj] = gaussian_bf16(30 + p, (N, r), std=0.02)
+    H, KV = c["H"], c["KV"]
+    return {
+        "w": w, "lora_a": a, "lora_b": b,
+        "gamma1": gaussian_bf16(40, (H,), std=0.02, mean=1.0),
+        "gamma2": gaussian_bf16(41, (H,), std=0.02, mean=1.0),
+        "h": gaussian_bf16(1, (M, H)),
+        "attn": gaussian_bf16(60, (M, H)),
+        "d_out": gaussian_bf16(56, (M, H)),
+        "d_qkv": np.concatenate([gaussian_bf16(61, (M, H)), gaussian_bf16(62, (M, KV)),
+                                 gaussian_bf16(63, (M, KV))], axis=1),
+    }

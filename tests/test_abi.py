@@ -84,19 +84,19 @@ def test_host_checks_reject_bad_arguments(P):
     # GEMM: output leading dimension not a multiple of 8
     wcache = pm.c_weight_cache(pm.c_nvfp4(0x1000, 0x2000, 512, 512), pm.c_nvfp4(0x3000, 0x4000, 512, 512))
     xq = pm.c_nvfp4(0x5000, 0x6000, 256, 512)
-    assert lib.pact_frozen_gemm_fwd(ctypes.byref(xq), ctypes.byref(wcache), None, 0x7000, 516, None) == 3
+    assert lib.pact_frozen_gemm_fwd(ctypes.byref(xq), ctypes.byref(wcache), None, None, 0, 0x7000, 516, None) == 3
     # GEMM: activation K does not match the weight
     xq2 = pm.c_nvfp4(0x5000, 0x6000, 256, 448)
-    assert lib.pact_frozen_gemm_fwd(ctypes.byref(xq2), ctypes.byref(wcache), None, 0x7000, 512, None) == 2
+    assert lib.pact_frozen_gemm_fwd(ctypes.byref(xq2), ctypes.byref(wcache), None, None, 0, 0x7000, 512, None) == 2
     # LoRA: internal segment boundary not a multiple of 256
     se = (ctypes.c_int64 * 4)(320, 512, 0, 0)
     lo = pm.c_lora(0x8000, 32, 0x9000, 16, 16, 2, se)
-    assert lib.pact_frozen_gemm_fwd(ctypes.byref(xq), ctypes.byref(wcache), ctypes.byref(lo), 0x7000, 512,
-                                    None) == 2
+    assert lib.pact_frozen_gemm_fwd(ctypes.byref(xq), ctypes.byref(wcache), ctypes.byref(lo), None, 0, 0x7000,
+                                    512, None) == 2
     # LoRA rank not supported
     lo2 = pm.c_lora(0x8000, 32, 0x9000, 16, 8, 1, (ctypes.c_int64 * 4)(512, 0, 0, 0))
-    assert lib.pact_frozen_gemm_fwd(ctypes.byref(xq), ctypes.byref(wcache), ctypes.byref(lo2), 0x7000, 512,
-                                    None) == 2
+    assert lib.pact_frozen_gemm_fwd(ctypes.byref(xq), ctypes.byref(wcache), ctypes.byref(lo2), None, 0,
+                                    0x7000, 512, None) == 2
     # LoRA backward: workspace too small
     args = pm.c_lora_bwd()
     args.M, args.N, args.K = 256, 512, 512

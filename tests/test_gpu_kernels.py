@@ -152,6 +152,18 @@ def test_gemm_dgrad(P, orc, M, N, K):
     assert_close(to_f64(dx), orc.frozen_dgrad(dy, wb), "dgrad")
 
 
+def test_gemm_fwd_residual(P, orc):
+    M, N, K = 300, 768, 512
+    x = synth.gaussian_bf16(1, (M, K))
+    res = synth.gaussian_bf16(2, (M, N))
+    w = synth.weight_bf16(0, (N, K))
+    wc = P.pact_weight_layout_cache(to_dev(w))
+    y = P.pact_frozen_gemm_fwd(P.pact_quantize_nvfp4(to_dev(x)), wc, residual=to_dev(res))
+    sync()
+    wf, _ = orc.weight_cache(w)
+    assert_close(to_f64(y), orc.nvfp4_gemm(orc.quantize(x), wf) + synth.bf16_bits_to_f64(res), "fwd + residual")
+
+
 def test_gemm_dgrad_accumulate(P, orc):
     M, N, K = 256, 512, 768
     dy = synth.gaussian_bf16(50, (M, N))
@@ -159,7 +171,7 @@ def test_gemm_dgrad_accumulate(P, orc):
     w = synth.weight_bf16(0, (N, K))
     wc = P.pact_weight_layout_cache(to_dev(w))
     dx = to_dev(base)
-    P.pact_frozen_gemm_dgrad(P.pact_quantize_nvfp4(to_dev(dy)), wc, dx=dx, accumulate=True)
+    P.pact_frozen_gemm_dgrad(P.pact_quantize_nvfp4(to_dev(dy)), wc, residual=dx, dx=dx)
     sync()
     _, wb = orc.weight_cache(w)
     assert_close(to_f64(dx), orc.frozen_dgrad(dy, wb) + synth.bf16_bits_to_f64(base), "dgrad accumulate")
@@ -175,7 +187,7 @@ def _segments(N, parts):
 
 
 @pytest.mark.parametrize("M,parts,K,r", [(256, [512], 512, 16), (300, [512, 256, 256], 576, 16),
-                                         (200, [256, 320], 256, 32)])
+                                         (200, [256, 320], 256, 16), (130, [768], 320, 48)])
 def test_gemm_fwd_lora(P, orc, M, parts, K, r):
     N = sum(parts)
     seg_end = _segments(N, parts)
@@ -192,10 +204,11 @@ def test_gemm_fwd_lora(P, orc, M, parts, K, r):
     bd = to_dev(b)
     y = P.pact_frozen_gemm_fwd(xq, wc, lora=P.lora_struct(T, bd, r, seg_end))
     sync()
-    # oracle, teacher-forced on the device's T (its BF16 rounding is the device's)
+    # oracle, teacher-forced on the device's T (T = hi + lo)
     wf, _ = orc.weight_cache(w)
     ref = orc.nvfp4_gemm(orc.quantize(x), wf)
-    t_dev = to_f64(T)
+    R = nseg * r
+    t_dev = to_f64(T[:, :R]) + to_f64(T[:, R:])
     bb = synth.bf16_bits_to_f64(b)
     lo = 0
     for i, hi in enumerate(seg_end):
@@ -206,19 +219,20 @@ def test_gemm_fwd_lora(P, orc, M, parts, K, r):
     assert_close(t_dev, s * orc.lora_t(synth.bf16_bits_to_f64(x), a), "T")
 
 
-@pytest.mark.parametrize("M,N,K,R", [(256, 512, 512, 16), (300, 640, 576, 48), (130, 256, 320, 64)])
+@pytest.mark.parametrize("M,N,K,R", [(256, 512, 512, 16), (300, 640, 576, 48), (130, 256, 320, 32)])
 def test_gemm_dgrad_lora(P, orc, M, N, K, R):
     dy = synth.gaussian_bf16(50, (M, N))
     w = synth.weight_bf16(0, (N, K))
     a = synth.gaussian_bf16(20, (R, K), std=0.02)
-    u = synth.gaussian_bf16(31, (M, R), std=0.5)
+    u = np.concatenate([synth.gaussian_bf16(31, (M, R), std=0.5), synth.gaussian_bf16(32, (M, R), std=1e-3)], 1)
     wc = P.pact_weight_layout_cache(to_dev(w))
     dyq = P.pact_quantize_nvfp4(to_dev(dy))
     ud, ad = to_dev(u), to_dev(a)
     dx = P.pact_frozen_gemm_dgrad(dyq, wc, lora=P.lora_struct(ud, ad, R, [K]))
     sync()
     _, wb = orc.weight_cache(w)
-    ref = orc.frozen_dgrad(dy, wb) + orc.gemm_nt(synth.bf16_bits_to_f64(u), synth.bf16_bits_to_f64(a).T)
+    uf = synth.bf16_bits_to_f64(u)
+    ref = orc.frozen_dgrad(dy, wb) + orc.gemm_nt(uf[:, :R] + uf[:, R:], synth.bf16_bits_to_f64(a).T)
     assert_close(to_f64(dx), ref, "dgrad + LoRA")
 
 
@@ -242,7 +256,8 @@ def test_lora_bwd(P, orc, M, parts, r):
     sync()
     dyf, xf = synth.bf16_bits_to_f64(dy), synth.bf16_bits_to_f64(x)
     af, bf = synth.bf16_bits_to_f64(a), synth.bf16_bits_to_f64(b)
-    u_dev = to_f64(U)
+    R = nseg * r
+    u_dev = to_f64(U[:, :R]) + to_f64(U[:, R:])
     lo = 0
     u_ref = np.zeros((M, nseg * r))
     for i, hi in enumerate(seg_end):
@@ -332,3 +347,30 @@ def test_errors_leave_nothing_enqueued(P):
         P.pact_quantize_nvfp4(x)
     assert e.value.status == 2
     status_ok(P)
+
+
+# ------------------------------------------------- one projection, not teacher-forced
+@pytest.mark.parametrize("M,N,K", [(256, 512, 512), (300, 768, 320)])
+def test_projection_end_to_end(P, orc, M, N, K):
+    """Forward, dgrad and dA/dB of one projection with its LoRA branch against the
+    fully independent oracle (no device intermediate fed back)."""
+    r, s = 16, 2.0
+    x = synth.gaussian_bf16(1, (M, K))
+    w = synth.weight_bf16(0, (N, K))
+    a = synth.gaussian_bf16(20, (r, K), std=0.02)
+    b = synth.gaussian_bf16(30, (N, r), std=0.02)
+    dy = synth.gaussian_bf16(50, (M, N))
+    xd, ad, bd, dyd = to_dev(x), to_dev(a), to_dev(b), to_dev(dy)
+    wc = P.pact_weight_layout_cache(to_dev(w))
+    T = P.pact_lora_fwd(xd, ad, s)
+    y = P.pact_frozen_gemm_fwd(P.pact_quantize_nvfp4(xd), wc, lora=P.lora_struct(T, bd, r, [N]))
+    U = P.pact_lora_bwd_u(dyd, bd, r, [N], s)
+    dx = P.pact_frozen_gemm_dgrad(P.pact_quantize_nvfp4(dyd), wc, lora=P.lora_struct(U, ad, r, [K]))
+    dA, dB = P.pact_lora_bwd(dyd, ad, U, r, [N], s, x=xd)
+    sync()
+    wf, wb = orc.weight_cache(w)
+    assert_close(to_f64(y), orc.frozen_fwd(orc.quantize(x), wf, x, a, b, s), "y")
+    assert_close(to_f64(dx), orc.frozen_dgrad(dy, wb, a, b, s), "dx")
+    da, db, _ = orc.lora_bwd(dy, synth.bf16_bits_to_f64(x), a, b, s)
+    assert_close(to_f64(dA), da, "dA")
+    assert_close(to_f64(dB), db, "dB")
