@@ -48,6 +48,10 @@ def parse():
     ap.add_argument("--workload", default=WORKLOAD)
     ap.add_argument("--cpu-tokens", type=int, default=128, help="token sample of the CPU oracle baseline")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--sweep", action="store_true",
+                    help="NVFP4 GEMM shape sweep (N x K x M, forward and dgrad): one JSON line per shape")
+    ap.add_argument("--gemm", type=int, nargs=3, metavar=("N", "K", "M"),
+                    help="time one NVFP4 GEMM shape (forward and dgrad) instead of the layer step")
     return ap.parse_args()
 
 
@@ -178,10 +182,60 @@ def config_block(name, M):
 
 
 # ------------------------------------------------------------------ GPU arm
+def gemm_sweep(a, shapes):
+    """Time NVFP4 frozen GEMMs (forward Y = X W^T and dgrad dX = dY W) per shape;
+    inputs X, dY ~ N(0, 1), W ~ N(0, 0.02^2); L2 flushed before every launch."""
+    import torch
+    import synth
+    import nvfp4_gemm_b200 as P
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    d = lambda bits: torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).to(dev)
+    pk = peaks()
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    ev = lambda: torch.cuda.Event(enable_timing=True)
+    for N, K, M in shapes:
+        w = d(synth.weight_bf16(0, (N, K)))
+        wc = P.pact_weight_layout_cache(w)
+        xq = P.pact_quantize_nvfp4(d(synth.gaussian_bf16(1, (M, K))))
+        dyq = P.pact_quantize_nvfp4(d(synth.gaussian_bf16(50, (M, N))))
+        y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+        dx = torch.empty((M, K), dtype=torch.bfloat16, device=dev)
+        res = {}
+        for kind, fn in (("fwd", lambda: P.pact_frozen_gemm_fwd(xq, wc, y=y)),
+                         ("dgrad", lambda: P.pact_frozen_gemm_dgrad(dyq, wc, dx=dx))):
+            for _ in range(max(3, a.warmup)):
+                fn()
+            times = []
+            for _ in range(a.steps):
+                flush.zero_()
+                e0, e1 = ev(), ev()
+                e0.record()
+                fn()
+                e1.record()
+                times.append((e0, e1))
+            torch.cuda.synchronize()
+            ms = sorted(s_.elapsed_time(e_) for s_, e_ in times)
+            med = ms[len(ms) // 2]
+            tf = 2.0 * M * N * K / (med / 1e3) / 1e12
+            res[kind] = {"median_ms": med, "tflops": tf, "frac_fp4_peak": tf / (FP4_PER_BF16 * pk["bf16"])}
+        if P.pact_get_device_status() != 0:
+            raise RuntimeError(P.pact_last_error())
+        print(json.dumps({"gemm": {"N": N, "K": K, "M": M}, **res,
+                          "peak_note": f"{pk['src']} burst BF16 {pk['bf16']} TF/s x {FP4_PER_BF16}"}), flush=True)
+        del w, wc, xq, dyq, y, dx
+        torch.cuda.empty_cache()
+
+
 def main():
     a = parse()
     if a.impl == "reference":
         return reference_arm(a)
+    if a.gemm:
+        return gemm_sweep(a, [tuple(a.gemm)])
+    if a.sweep:
+        import synth
+        return gemm_sweep(a, [(n, k, m) for (n, k) in synth.SWEEP_NK for m in synth.SWEEP_M])
 
     import torch
     import torch.distributed as dist
