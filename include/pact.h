@@ -193,20 +193,28 @@ PACT_API pact_status pact_frozen_gemm_dgrad(const pact_nvfp4_t *dyq, const pact_
 /* [LORA]: T = scale * X . A^T for X [M x K] (row stride ldx) and A [R x K] (row
  * stride K; R = nseg*r stacked adapters sharing X), FP32-accumulated and written
  * as hi + lo BF16 halves: T [M x 2R] (row stride ldt >= 2R), hi = BF16_RNE(t) in
- * columns 0..R-1, lo = BF16_RNE(t - hi) in columns R..2R-1.  R is 16, 32, 48 or 64. */
+ * columns 0..R-1, lo = BF16_RNE(t - hi) in columns R..2R-1.  R is 16, 32, 48 or 64.
+ * workspace (device, 16-byte aligned, >= pact_lora_fwd_workspace_bytes(M, K, R))
+ * is caller-owned scratch for FP32 partial sums; its contents on entry do not
+ * matter and calls that share it must not overlap on the GPU. */
+PACT_API size_t pact_lora_fwd_workspace_bytes(int64_t M, int64_t K, int R);
 PACT_API pact_status pact_lora_fwd(const pact_bf16 *x, int64_t ldx, int64_t M, int64_t K,
-                          const pact_bf16 *A, int R, float scale, pact_bf16 *T, int64_t ldt,
-                          pact_stream_t stream);
+                                   const pact_bf16 *A, int R, float scale, pact_bf16 *T, int64_t ldt,
+                                   void *workspace, size_t ws_bytes, pact_stream_t stream);
 
 /* --------------------------------------------------- A8: LoRA backward */
 /* [LORA] gradients, BF16 throughout ([METHOD]: adapters stay BF16).
  * pact_lora_bwd_u: U[:, i*r .. i*r+r-1] = scale * dY[:, seg_i] . B[seg_i, :] for dY
  *   [M x N] (row stride lddy), B [N x r]; written like T as hi + lo BF16 halves,
  *   U [M x 2*nseg*r] (row stride ldu).  U feeds pact_frozen_gemm_dgrad and
- *   pact_lora_bwd.  Internal segment ends are multiples of 64. */
+ *   pact_lora_bwd.  Segment ends are multiples of 64, the last equals N; r is 16,
+ *   32, 48 or 64, nseg <= 3, nseg*r <= 64.  workspace as for pact_lora_fwd, at
+ *   least pact_lora_bwd_u_workspace_bytes(M, N, r, nseg) bytes. */
+PACT_API size_t pact_lora_bwd_u_workspace_bytes(int64_t M, int64_t N, int r, int nseg);
 PACT_API pact_status pact_lora_bwd_u(const pact_bf16 *dy, int64_t lddy, int64_t M, int64_t N,
-                            const pact_bf16 *B, int r, int nseg, const int64_t *seg_end,
-                            float scale, pact_bf16 *U, int64_t ldu, pact_stream_t stream);
+                                     const pact_bf16 *B, int r, int nseg, const int64_t *seg_end,
+                                     float scale, pact_bf16 *U, int64_t ldu, void *workspace,
+                                     size_t ws_bytes, pact_stream_t stream);
 
 /* The input X~ the adapter saw, as backward holds it: BF16 x, or the saved NVFP4
  * copy xq (dequantized on the fly); exactly one is non-NULL. */
@@ -227,10 +235,11 @@ typedef struct {
     pact_bf16 *dB;            /* out [N x r]: rows seg_i = scale * dY[:, seg_i]^T . (X~ . A_i^T) */
 } pact_lora_bwd_t;
 
-/* Scratch bytes pact_lora_bwd needs for its FP32 partial sums. */
+/* Scratch bytes pact_lora_bwd needs (X~ as BF16, T~ = X~ A^T, FP32 partial sums). */
 PACT_API size_t pact_lora_bwd_workspace_bytes(int64_t M, int64_t N, int64_t K, int r, int nseg);
-/* dA and dB of the adapters; workspace (device, >= pact_lora_bwd_workspace_bytes)
- * is scratch owned by the caller; its contents on entry do not matter. */
+/* dA and dB of the adapters; workspace (device, 256-byte aligned, >=
+ * pact_lora_bwd_workspace_bytes) is scratch owned by the caller; its contents on
+ * entry do not matter and calls that share it must not overlap on the GPU. */
 PACT_API pact_status pact_lora_bwd(const pact_lora_bwd_t *args, void *workspace, size_t ws_bytes,
                           pact_stream_t stream);
 

@@ -2,281 +2,413 @@
 // section "LoRA": h = W0 x + B A x; [METHOD]: PACT blog summary, section "方法",
 // paragraph after the bullets: A and B stay BF16 and are never quantized).
 //
-// The products are skinny (rank 16 per adapter): X . A^T, dY . B (contraction over the
-// feature dimension, R <= 64 outputs per row) and U^T . X, dY^T . T (contraction over
-// the tokens).  These kernels run them on the CUDA cores with FP32 accumulation and
-// shared-memory tiles; the token contractions are split over token chunks and reduced
-// with FP32 atomics into caller-provided scratch.
+// The products are skinny (rank 16 per adapter) and bound by HBM:
+//   T    = X . A^T           [M x R]   contraction over features   (forward)
+//   U_i  = dY_i . B_i        [M x r]   contraction over segment i's outputs
+//   dB_i = dY_i^T . T~_i     [N_i x r] contraction over tokens
+//   dA^T = X~^T . U          [K x R]   contraction over tokens
+// One tcgen05 kernel runs them all: a 128-row output tile times up to 64 columns,
+// BF16 x BF16 -> FP32 in tensor memory (kind::f16), operands staged by TMA with the
+// 128-byte swizzle either K-major or MN-major (the transposed products read the
+// activations in place).  The contraction is split over CTAs so that enough SMs
+// stream the activations; each split writes its FP32 partial tile to caller scratch
+// and a finalize kernel sums the partials in a fixed order (deterministic), scales
+// and rounds.
 #include "quant.cuh"
 
 namespace pact {
-namespace lora {
+namespace lmma {
 
-// ------------------------------------------------------------ row products
-// out[m, j] = scale * sum_k X[m, k] * W(j, k) for j < R, where W(j, k) is
-//   Wt = false: W[j * ldw + k]       (A [R x K] row-major)
-//   Wt = true : W[k * ldw + j_src]   (B [N x r] row-major, used transposed) with
-//               segment-wise contraction: column j belongs to segment j / r and sums
-//               k over that segment's feature range only.
-// X is BF16 (row stride ldx) or NVFP4 (xq, dequantized on load).
-constexpr int RT = 32;   // rows per CTA
-constexpr int KC = 64;   // contraction chunk
+constexpr int BM = 128;        // output rows per CTA (MMA M)
+constexpr int BK = 64;         // contraction elements per stage (128 bytes of BF16)
+constexpr int STAGES = 4;
+constexpr int THREADS = 192;
+constexpr int A_BYTES = BM * BK * 2;     // 16384
+constexpr int B_BYTES = 64 * BK * 2;     // 8192 per B part
+constexpr int STAGE_BYTES = A_BYTES + 2 * B_BYTES;
+constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + 256;
+constexpr uint32_t TMEM_COLS = 64;
 
-struct RowArgs {
-    const pact_bf16 *x;
-    int64_t ldx;
-    pact_nvfp4_t xq;
-    int use_xq;
-    int64_t M, K;
-    const pact_bf16 *w;
-    int64_t ldw;
-    int wt;       // W used transposed (B)
-    int R, r, nseg;
-    int64_t seg_end[4];
-    float scale;
-    pact_bf16 *out_bf16;  // one of these two; BF16 output is hi (columns 0..R-1) + lo (R..2R-1)
-    float *out_f32;
-    int64_t ldo;
+// One output block: rows [row_begin, row_end) of the output, contraction
+// [k_begin, k_end); b_coord positions the B operand (its row for a K-major B, its
+// column for an MN-major B); out_col is the column of the block in the output.
+struct Prob {
+    int row_begin, row_end, k_begin, k_end, b_coord, out_col;
 };
 
-__global__ void __launch_bounds__(256) k_rows(const RowArgs a) {
-    __shared__ float xs[RT][KC + 1];
-    __shared__ float ws[64][KC + 1];
-    const int t = threadIdx.x;
-    const int64_t m0 = (int64_t)blockIdx.x * RT;
-    const int row = t >> 3;          // 0..31
-    const int jl = t & 7;            // j = jl + 8 i
-    float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
-    // With Wt, the contraction of segment s runs over [seg_begin(s), seg_end[s]);
-    // chunk loop covers [0, K) and masks per output column.
-    for (int64_t k0 = 0; k0 < a.K; k0 += KC) {
-        // X chunk: 32 rows x 64 columns; thread t loads 8 values of row t/8
-        {
-            const int rr = t >> 3, cc = (t & 7) * 8;
-            const int64_t m = m0 + rr, k = k0 + cc;
-            float v[8] = {0, 0, 0, 0, 0, 0, 0, 0};
-            if (m < a.M && k < a.K) {
-                if (a.use_xq) load8_nvfp4(a.xq, m, k, v);
-                else load8_bf16(a.x + m * a.ldx + k, v);
-            }
-#pragma unroll
-            for (int i = 0; i < 8; ++i) xs[rr][cc + i] = v[i];
+struct Params {
+    int n_mma;          // MMA N (16..64, multiple of 16)
+    int n_valid;        // output columns per block
+    int nprob;
+    Prob prob[3];
+    int splits, k_per_split;
+    int b_split;        // B holds hi + lo halves: second tile at column b_coord + b_lo_off
+    int b_lo_off;
+    float *ws;          // partials [split][row][ws_ld]
+    int64_t ws_ld, ws_split_stride;
+};
+
+template <bool A_MN, bool B_MN>
+__global__ void __launch_bounds__(THREADS, 1)
+k_lora_mma(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, const Params p) {
+    const Prob pr = p.prob[blockIdx.z];
+    const int row0 = pr.row_begin + blockIdx.x * BM;
+    if (row0 >= pr.row_end) return;  // block-uniform, before any shared state
+    const int kb = pr.k_begin + blockIdx.y * p.k_per_split;
+    const int ke = min(pr.k_end, kb + p.k_per_split);
+    const int ktiles = ke > kb ? (ke - kb + BK - 1) / BK : 0;
+    float *part = p.ws + (size_t)blockIdx.y * p.ws_split_stride;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+    if (ktiles == 0) {  // empty split: its partial is zero
+        for (int i = threadIdx.x; i < BM * p.n_valid; i += THREADS) {
+            const int r = row0 + i / p.n_valid;
+            if (r < pr.row_end) part[(size_t)r * p.ws_ld + pr.out_col + i % p.n_valid] = 0.0f;
         }
-        // W chunk: R rows x 64 columns
-        for (int idx = t; idx < a.R * (KC / 8); idx += 256) {
-            const int j = idx / (KC / 8), cc = (idx % (KC / 8)) * 8;
-            const int64_t k = k0 + cc;
-            float v[8] = {0, 0, 0, 0, 0, 0, 0, 0};
-            if (k < a.K) {
-                if (!a.wt) {
-                    load8_bf16(a.w + (int64_t)j * a.ldw + k, v);
+        return;
+    }
+
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw = smem_u32(smem_raw);
+    uint8_t *smem = smem_raw + (((raw + 1023) & ~1023u) - raw);
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + STAGES * STAGE_BYTES);
+    uint64_t *full = bars, *empty = bars + STAGES, *acc_full = bars + 2 * STAGES;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 2 * STAGES + 1);
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
+        }
+        mbar_init(acc_full, 1);
+        fence_barrier_init();
+        prefetch_tensormap(&tmA);
+        prefetch_tensormap(&tmB);
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_slot, TMEM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    const int nparts = p.b_split ? 2 : 1;
+    const uint32_t b_bytes = B_MN ? (uint32_t)B_BYTES : (uint32_t)p.n_mma * BK * 2;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            uint32_t stage = 0, phase = 0, pending = 0, pending_parity = 0;
+            for (int kt = 0; kt < ktiles; ++kt) {
+                if (!mbar_wait(&empty[stage], phase ^ 1)) break;
+                uint8_t *st = smem + stage * STAGE_BYTES;
+                const int k = kb + kt * BK;
+                mbar_arrive_expect_tx(&full[stage], A_BYTES + nparts * b_bytes);
+                if (A_MN) {
+                    tma_load_2d(st, &tmA, &full[stage], row0, k);
+                    tma_load_2d(st + A_BYTES / 2, &tmA, &full[stage], row0 + 64, k);
                 } else {
-                    const int s = j / a.r, js = j % a.r;
-                    const int64_t lo = s ? a.seg_end[s - 1] : 0, hi = a.seg_end[s];
-#pragma unroll
-                    for (int i = 0; i < 8; ++i) {
-                        const int64_t kk = k + i;
-                        v[i] = (kk >= lo && kk < hi) ? bf16lo(a.w[kk * a.ldw + js]) : 0.0f;
+                    tma_load_2d(st, &tmA, &full[stage], k, row0);
+                }
+                for (int h = 0; h < nparts; ++h) {
+                    uint8_t *bd = st + A_BYTES + h * B_BYTES;
+                    if (B_MN) tma_load_2d(bd, &tmB, &full[stage], pr.b_coord + h * p.b_lo_off, k);
+                    else tma_load_2d(bd, &tmB, &full[stage], k, pr.b_coord);
+                }
+                pending |= 1u << stage;
+                pending_parity = (pending_parity & ~(1u << stage)) | (phase << stage);
+                if (++stage == STAGES) { stage = 0; phase ^= 1; }
+            }
+            // copies land before the CTA may leave
+            for (int s = 0; s < STAGES; ++s)
+                if (pending & (1u << s)) mbar_wait(&full[s], (pending_parity >> s) & 1u);
+        }
+    } else if (warp == 1) {
+        const uint32_t idesc = idesc_bf16(BM, p.n_mma, A_MN, B_MN);
+        uint32_t stage = 0, phase = 0, accum = 0;
+        for (int kt = 0; kt < ktiles; ++kt) {
+            const bool ok = mbar_wait(&full[stage], phase);
+            tc_fence_after();
+            if (!ok) break;
+            if (lane == 0) {
+                const uint32_t st = smem_u32(smem + stage * STAGE_BYTES);
+                for (int s = 0; s < BK / 16; ++s) {
+                    const uint64_t ad = A_MN ? smem_desc(st + s * 2048, A_BYTES / 2, 1024, SW_128)
+                                             : smem_desc(st + s * 32, 16, 1024, SW_128);
+                    for (int h = 0; h < nparts; ++h) {
+                        const uint32_t b0 = st + A_BYTES + h * B_BYTES;
+                        const uint64_t bd = B_MN ? smem_desc(b0 + s * 2048, B_BYTES, 1024, SW_128)
+                                                 : smem_desc(b0 + s * 32, 16, 1024, SW_128);
+                        mma_bf16(tmem, ad, bd, idesc, accum);
+                        accum = 1;
                     }
                 }
+                tc_commit(&empty[stage]);
             }
-#pragma unroll
-            for (int i = 0; i < 8; ++i) ws[j][cc + i] = v[i];
+            __syncwarp();
+            if (++stage == STAGES) { stage = 0; phase ^= 1; }
         }
-        __syncthreads();
-#pragma unroll 8
-        for (int k = 0; k < KC; ++k) {
-            const float xv = xs[row][k];
+        // the epilogue waits for this; it also orders every MMA before the dealloc
+        if (lane == 0) tc_commit(acc_full);
+        __syncwarp();
+    } else {
+        const int sub = warp & 3;
+        const bool ok = mbar_wait(acc_full, 0);
+        tc_fence_after();
+        const int r = row0 + sub * 32 + lane;
+        for (int c = 0; c < p.n_mma / 16; ++c) {
+            uint32_t v[16];
+            tmem_ld_32x32b_x16(tmem + ((uint32_t)(sub * 32) << 16) + c * 16, v);
+            tmem_ld_wait();
+            if (ok && r < pr.row_end) {
+                float *dst = part + (size_t)r * p.ws_ld + pr.out_col + c * 16;
 #pragma unroll
-            for (int i = 0; i < 8; ++i)
-                if (jl + 8 * i < a.R) acc[i] = fmaf(xv, ws[jl + 8 * i][k], acc[i]);
-        }
-        __syncthreads();
-    }
-    const int64_t m = m0 + row;
-    if (m < a.M) {
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            const int j = jl + 8 * i;
-            if (j < a.R) {
-                const float v = acc[i] * a.scale;
-                if (a.out_f32) {
-                    a.out_f32[m * a.ldo + j] = v;
-                } else {  // v as the unevaluated sum hi + lo of two BF16 values
-                    const __nv_bfloat16 hi = __float2bfloat16_rn(v);
-                    a.out_bf16[m * a.ldo + j] = __bfloat16_as_ushort(hi);
-                    a.out_bf16[m * a.ldo + a.R + j] =
-                        __bfloat16_as_ushort(__float2bfloat16_rn(v - __bfloat162float(hi)));
-                }
+                for (int j = 0; j < 16; ++j)
+                    if (c * 16 + j < p.n_valid) dst[j] = __uint_as_float(v[j]);
             }
         }
     }
-}
-
-// ------------------------------------------------------------ token contractions
-// ws[a, b] += sum_{m in chunk} P[m, a] * Q[m, qcol(a) + b], a < A, b < Bn.
-//   P: BF16 [M x A] (row stride ldp).
-//   Q: BF16 (ldq) or NVFP4 (qq) or FP32 (qf, ldq); qcol(a) = seg(a) * r when
-//      segmented (dB), else 0.
-constexpr int TA = 64, TB = 64, MC = 32, MCHUNK = 256;
-
-struct OuterArgs {
-    const pact_bf16 *p;
-    int64_t ldp;
-    int p_split;  // P holds hi (columns 0..A-1) + lo (A..2A-1)
-    const pact_bf16 *q;
-    const float *qf;
-    pact_nvfp4_t qq;
-    int q_kind;  // 0 bf16, 1 nvfp4, 2 fp32
-    int64_t ldq;
-    int64_t M, A, Bn;
-    int segmented, r, nseg;
-    int64_t seg_end[4];
-    float *ws;
-    int64_t ldws;
-};
-
-__global__ void __launch_bounds__(256) k_outer(const OuterArgs o) {
-    __shared__ float ps[MC][TA + 1];
-    __shared__ float qs[MC][TB + 1];
-    const int t = threadIdx.x;
-    const int64_t a0 = (int64_t)blockIdx.x * TA, b0 = (int64_t)blockIdx.y * TB;
-    const int64_t mbeg = (int64_t)blockIdx.z * MCHUNK;
-    const int64_t mend = min(o.M, mbeg + MCHUNK);
-    int64_t qoff = 0;
-    if (o.segmented) {
-        int s = 0;
-        for (int i = 0; i + 1 < o.nseg; ++i) s += (a0 >= o.seg_end[i]) ? 1 : 0;
-        qoff = (int64_t)s * o.r;
-    }
-    const int ta = (t >> 4) * 4, tb = (t & 15) * 4;  // 4 x 4 outputs per thread
-    float acc[4][4] = {};
-    for (int64_t m0 = mbeg; m0 < mend; m0 += MC) {
-        // P tile: MC rows x TA columns (8 per thread load)
-        {
-            const int rr = t >> 3, cc = (t & 7) * 8;
-            const int64_t m = m0 + rr, a = a0 + cc;
-            float v[8] = {0, 0, 0, 0, 0, 0, 0, 0};
-            if (m < mend && a < o.A) {
-                load8_bf16(o.p + m * o.ldp + a, v);
-                if (o.p_split) {
-                    float lo[8];
-                    load8_bf16(o.p + m * o.ldp + o.A + a, lo);
-#pragma unroll
-                    for (int i = 0; i < 8; ++i) v[i] += lo[i];
-                }
-            }
-#pragma unroll
-            for (int i = 0; i < 8; ++i) ps[rr][cc + i] = v[i];
-        }
-        {
-            const int rr = t >> 3, cc = (t & 7) * 8;
-            const int64_t m = m0 + rr, b = b0 + cc;
-            float v[8] = {0, 0, 0, 0, 0, 0, 0, 0};
-            if (m < mend && b < o.Bn) {
-                if (o.q_kind == 0) load8_bf16(o.q + m * o.ldq + qoff + b, v);
-                else if (o.q_kind == 1) load8_nvfp4(o.qq, m, qoff + b, v);
-                else {
-                    const float4 *s4 = reinterpret_cast<const float4 *>(o.qf + m * o.ldq + qoff + b);
-                    const float4 x0 = s4[0], x1 = s4[1];
-                    v[0] = x0.x; v[1] = x0.y; v[2] = x0.z; v[3] = x0.w;
-                    v[4] = x1.x; v[5] = x1.y; v[6] = x1.z; v[7] = x1.w;
-                }
-            }
-#pragma unroll
-            for (int i = 0; i < 8; ++i) qs[rr][cc + i] = v[i];
-        }
-        __syncthreads();
-#pragma unroll 4
-        for (int mm = 0; mm < MC; ++mm) {
-            float pv[4], qv[4];
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                pv[i] = ps[mm][ta + i];
-                qv[i] = qs[mm][tb + i];
-            }
-#pragma unroll
-            for (int i = 0; i < 4; ++i)
-#pragma unroll
-                for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(pv[i], qv[j], acc[i][j]);
-        }
-        __syncthreads();
-    }
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        const int64_t a = a0 + ta + i;
-        if (a >= o.A) continue;
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            const int64_t b = b0 + tb + j;
-            if (b < o.Bn) atomicAdd(&o.ws[a * o.ldws + b], acc[i][j]);
-        }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, TMEM_COLS);
     }
 }
 
-// dst (row stride ldd) = BF16(scale * src), src FP32 [rows x cols] row-major.
-__global__ void k_finalize(const float *__restrict__ src, int64_t rows, int64_t cols, float scale,
-                           pact_bf16 *__restrict__ dst, int64_t ldd) {
+// out = scale * sum_s ws[s][row][col] for rows x cols, written as
+//   mode 0: hi + lo BF16 halves (hi at out[row * ldo + col], lo at col + lo_off)
+//   mode 1: BF16
+//   mode 2: BF16 transposed (out[col * ldo + row])
+__global__ void k_finalize(const float *__restrict__ ws, int splits, int64_t split_stride, int64_t ws_ld, int64_t rows,
+                           int64_t cols, float scale, int mode, pact_bf16 *__restrict__ out, int64_t ldo,
+                           int64_t lo_off) {
     const int64_t n = rows * cols;
     for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x) {
-        const int64_t r = i / cols, c = i % cols;
-        dst[r * ldd + c] = __bfloat16_as_ushort(__float2bfloat16_rn(src[i] * scale));
+        const int64_t r = mode == 2 ? i % rows : i / cols, c = mode == 2 ? i / rows : i % cols;
+        float acc = 0.0f;
+        for (int s = 0; s < splits; ++s) acc += ws[s * split_stride + r * ws_ld + c];
+        acc *= scale;
+        const __nv_bfloat16 hi = __float2bfloat16_rn(acc);
+        if (mode == 2) {
+            out[c * ldo + r] = __bfloat16_as_ushort(hi);
+        } else {
+            out[r * ldo + c] = __bfloat16_as_ushort(hi);
+            if (mode == 0)
+                out[r * ldo + c + lo_off] = __bfloat16_as_ushort(__float2bfloat16_rn(acc - __bfloat162float(hi)));
+        }
     }
 }
 
-}  // namespace lora
+// NVFP4 -> BF16 (exact): the backward's view of a saved activation copy.
+__global__ void k_dequantize(pact_nvfp4_t t, pact_bf16 *__restrict__ out) {
+    const int64_t per_row = t.cols / 8;
+    const int64_t n8 = t.rows * per_row;
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n8; i += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t r = i / per_row, c = (i % per_row) * 8;
+        float v[8];
+        load8_nvfp4(t, r, c, v);
+        store8_bf16(out + r * t.cols + c, v);
+    }
+}
+
+// ---------------------------------------------------------------- host side
+typedef CUresult (*EncodeTiled)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+// 2-D tiled map over a BF16 row-major matrix: `inner` elements per row (row stride
+// `ld` elements), `outer` rows, 128-byte swizzle.
+static pact_status map_bf16(CUtensorMap *m, const void *base, uint64_t inner, uint64_t outer, uint64_t ld,
+                            uint32_t box_inner, uint32_t box_outer, const char *what) {
+    static EncodeTiled enc = nullptr;
+    if (!enc) {
+        void *fp = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &fp, 12000, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            enc = reinterpret_cast<EncodeTiled>(fp);
+    }
+    if (!enc) return fail(PACT_ERR_CUDA, "%s: cuTensorMapEncodeTiled unavailable", what);
+    const cuuint64_t dims[2] = {inner, outer};
+    const cuuint64_t strides[1] = {ld * 2};
+    const cuuint32_t box[2] = {box_inner, box_outer};
+    const cuuint32_t es[2] = {1, 1};
+    CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box, es,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(PACT_ERR_CUDA, "%s: cuTensorMapEncodeTiled failed (%d)", what, (int)r);
+    return PACT_OK;
+}
+
+template <bool A_MN, bool B_MN>
+static pact_status launch_mma(const CUtensorMap &ta, const CUtensorMap &tb, const Params &p, int row_tiles,
+                              cudaStream_t st, const char *what) {
+    static bool done[64] = {false};
+    const int d = current_device();
+    if (d >= 0 && d < 64 && !done[d]) {
+        cudaError_t e =
+            cudaFuncSetAttribute(k_lora_mma<A_MN, B_MN>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+        if (e != cudaSuccess) return fail(PACT_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+        done[d] = true;
+    }
+    dim3 grid((unsigned)row_tiles, (unsigned)p.splits, (unsigned)p.nprob);
+    k_lora_mma<A_MN, B_MN><<<grid, THREADS, SMEM_BYTES, st>>>(ta, tb, p);
+    return launch_status(what);
+}
+
+// Split a contraction of length `len` over CTAs so that `blocks` output blocks x
+// splits covers the SMs, with at least 4 stages (256 elements) per split.
+static void choose_split(int64_t len, int64_t blocks, int *splits, int *kps) {
+    int64_t s = (sm_count() + blocks - 1) / (blocks > 0 ? blocks : 1);
+    const int64_t max_s = (len + 4 * BK - 1) / (4 * BK);
+    if (s > max_s) s = max_s;
+    if (s < 1) s = 1;
+    int64_t k = (len + s - 1) / s;
+    k = (k + BK - 1) / BK * BK;
+    *splits = (int)((len + k - 1) / k);
+    *kps = (int)k;
+}
+
+static int finalize_grid(int64_t n) {
+    const int64_t g = (n + 255) / 256;
+    const int64_t cap = (int64_t)sm_count() * 8;
+    return (int)(g < 1 ? 1 : (g > cap ? cap : g));
+}
+
+static size_t round256(size_t b) { return (b + 255) & ~(size_t)255; }
+
+// Bytes of FP32 partials for rows x cols outputs split `splits` ways.
+static size_t partial_bytes(int64_t rows, int64_t cols, int splits) {
+    return round256((size_t)(rows * cols * 4) * (size_t)splits);
+}
+
+// scale * X . A^T for X [M x K] (map tx) and A [R x K], written hi/lo into out
+// (row stride ldo, lo at column R); ws holds the partials.
+static pact_status rows_times_a(const CUtensorMap &tx, int64_t M, int64_t K, const pact_bf16 *A, int R, float scale,
+                                pact_bf16 *out, int64_t ldo, float *ws, cudaStream_t st, const char *what) {
+    CUtensorMap tb;
+    pact_status s = map_bf16(&tb, A, K, R, K, 64, R, what);
+    if (s != PACT_OK) return s;
+    Params p = {};
+    p.n_mma = R;
+    p.n_valid = R;
+    p.nprob = 1;
+    p.prob[0] = Prob{0, (int)M, 0, (int)K, 0, 0};
+    const int tiles = (int)((M + BM - 1) / BM);
+    choose_split(K, tiles, &p.splits, &p.k_per_split);
+    p.ws = ws;
+    p.ws_ld = R;
+    p.ws_split_stride = M * R;
+    s = launch_mma<false, false>(tx, tb, p, tiles, st, what);
+    if (s != PACT_OK) return s;
+    k_finalize<<<finalize_grid(M * R), 256, 0, st>>>(ws, p.splits, M * R, R, M, R, scale, 0, out, ldo, R);
+    return launch_status(what);
+}
+
+static pact_status check_segments(int64_t N, int nseg, const int64_t *seg_end, const char *what) {
+    int64_t prev = 0;
+    for (int i = 0; i < nseg; ++i) {
+        PACT_CHECK(seg_end[i] > prev && seg_end[i] % 64 == 0 && (i + 1 < nseg || seg_end[i] == N), PACT_ERR_SHAPE,
+                   "%s: segment ends must increase by multiples of 64 and end at N", what);
+        prev = seg_end[i];
+    }
+    return PACT_OK;
+}
+
+}  // namespace lmma
 }  // namespace pact
 
 using namespace pact;
-using namespace pact::lora;
-
-static size_t lora_up256(size_t b) { return (b + 255) & ~(size_t)255; }
+using namespace pact::lmma;
 
 extern "C" {
 
+static int splits_of(int64_t len, int64_t blocks) {
+    int s, k;
+    choose_split(len, blocks, &s, &k);
+    return s;
+}
+
+size_t pact_lora_fwd_workspace_bytes(int64_t M, int64_t K, int R) {
+    return partial_bytes(M, R, splits_of(K, (M + BM - 1) / BM));
+}
+
 pact_status pact_lora_fwd(const pact_bf16 *x, int64_t ldx, int64_t M, int64_t K, const pact_bf16 *A, int R,
-                          float scale, pact_bf16 *T, int64_t ldt, pact_stream_t stream) {
-    PACT_CHECK(x && A && T, PACT_ERR_INVALID_ARG, "pact_lora_fwd: NULL argument");
-    PACT_CHECK(M >= 1 && K >= 64 && K % 64 == 0 && R >= 16 && R <= 64 && R % 16 == 0, PACT_ERR_SHAPE,
-               "pact_lora_fwd: need M >= 1, K a multiple of 64, R in {16, 32, 48, 64}");
-    PACT_CHECK(ldx >= K && ldx % 8 == 0 && ldt >= 2 * R && ldt % 8 == 0 && aligned16(x) && aligned16(A) && aligned16(T),
+                          float scale, pact_bf16 *T, int64_t ldt, void *workspace, size_t ws_bytes,
+                          pact_stream_t stream) {
+    PACT_CHECK(x && A && T && workspace, PACT_ERR_INVALID_ARG, "pact_lora_fwd: NULL argument");
+    PACT_CHECK(M >= 1 && M <= 0x7FFFFFFF && K >= 64 && K % 64 == 0 && K <= 0x7FFFFFFF && R >= 16 && R <= 64 &&
+                   R % 16 == 0,
+               PACT_ERR_SHAPE, "pact_lora_fwd: need M >= 1, K a multiple of 64, R in {16, 32, 48, 64}");
+    PACT_CHECK(ldx >= K && ldx % 8 == 0 && ldt >= 2 * R && ldt % 8 == 0 && aligned16(x) && aligned16(A) &&
+                   aligned16(T) && aligned16(workspace),
                PACT_ERR_ALIGN, "pact_lora_fwd: pointers 16-byte aligned, leading dims %% 8 == 0");
-    RowArgs a = {};
-    a.x = x; a.ldx = ldx; a.use_xq = 0; a.M = M; a.K = K;
-    a.w = A; a.ldw = K; a.wt = 0; a.R = R; a.r = R; a.nseg = 1; a.seg_end[0] = K;
-    a.scale = scale; a.out_bf16 = T; a.out_f32 = nullptr; a.ldo = ldt;
-    k_rows<<<(unsigned)((M + RT - 1) / RT), 256, 0, (cudaStream_t)stream>>>(a);
-    return launch_status("pact_lora_fwd");
+    PACT_CHECK(ws_bytes >= pact_lora_fwd_workspace_bytes(M, K, R), PACT_ERR_INVALID_ARG,
+               "pact_lora_fwd: workspace too small (%zu < %zu)", ws_bytes, pact_lora_fwd_workspace_bytes(M, K, R));
+    CUtensorMap tx;
+    pact_status s = map_bf16(&tx, x, K, M, ldx, 64, BM, "pact_lora_fwd");
+    if (s != PACT_OK) return s;
+    return rows_times_a(tx, M, K, A, R, scale, T, ldt, static_cast<float *>(workspace), (cudaStream_t)stream,
+                        "pact_lora_fwd");
+}
+
+// Upper bound over segmentations: one segment may span all N outputs.
+size_t pact_lora_bwd_u_workspace_bytes(int64_t M, int64_t N, int r, int nseg) {
+    return partial_bytes(M, (int64_t)r * nseg, splits_of(N, (M + BM - 1) / BM));
 }
 
 pact_status pact_lora_bwd_u(const pact_bf16 *dy, int64_t lddy, int64_t M, int64_t N, const pact_bf16 *B, int r,
                             int nseg, const int64_t *seg_end, float scale, pact_bf16 *U, int64_t ldu,
-                            pact_stream_t stream) {
-    PACT_CHECK(dy && B && U && seg_end, PACT_ERR_INVALID_ARG, "pact_lora_bwd_u: NULL argument");
-    PACT_CHECK(M >= 1 && N >= 64 && N % 64 == 0 && (r == 16 || r == 32 || r == 48 || r == 64) && nseg >= 1 &&
-                   nseg <= 4 && nseg * r <= 64,
-               PACT_ERR_SHAPE, "pact_lora_bwd_u: bad shape");
-    int64_t prev = 0;
+                            void *workspace, size_t ws_bytes, pact_stream_t stream) {
+    PACT_CHECK(dy && B && U && seg_end && workspace, PACT_ERR_INVALID_ARG, "pact_lora_bwd_u: NULL argument");
+    PACT_CHECK(M >= 1 && M <= 0x7FFFFFFF && N >= 64 && N % 64 == 0 && N <= 0x7FFFFFFF &&
+                   (r == 16 || r == 32 || r == 48 || r == 64) && nseg >= 1 && nseg <= 3 && nseg * r <= 64,
+               PACT_ERR_SHAPE, "pact_lora_bwd_u: bad shape (r in {16,32,48,64}, nseg <= 3, nseg*r <= 64)");
+    pact_status s = check_segments(N, nseg, seg_end, "pact_lora_bwd_u");
+    if (s != PACT_OK) return s;
+    const int R = nseg * r;
+    PACT_CHECK(lddy >= N && lddy % 8 == 0 && ldu >= 2 * R && ldu % 8 == 0 && aligned16(dy) && aligned16(B) &&
+                   aligned16(U) && aligned16(workspace),
+               PACT_ERR_ALIGN, "pact_lora_bwd_u: pointers 16-byte aligned, leading dims %% 8 == 0");
+    PACT_CHECK(ws_bytes >= pact_lora_bwd_u_workspace_bytes(M, N, r, nseg), PACT_ERR_INVALID_ARG,
+               "pact_lora_bwd_u: workspace too small");
+    cudaStream_t st = (cudaStream_t)stream;
+    CUtensorMap ta, tb;
+    s = map_bf16(&ta, dy, N, M, lddy, 64, BM, "pact_lora_bwd_u");
+    if (s == PACT_OK) s = map_bf16(&tb, B, r, N, r, 64, 64, "pact_lora_bwd_u");  // B^T, MN-major
+    if (s != PACT_OK) return s;
+    Params p = {};
+    p.n_mma = 64;
+    p.n_valid = r;
+    p.nprob = nseg;
+    int64_t longest = 0, prev = 0;
     for (int i = 0; i < nseg; ++i) {
-        PACT_CHECK(seg_end[i] > prev && seg_end[i] % 64 == 0 && (i + 1 < nseg || seg_end[i] == N), PACT_ERR_SHAPE,
-                   "pact_lora_bwd_u: segment ends must increase by multiples of 64 and end at N");
+        p.prob[i] = Prob{0, (int)M, (int)prev, (int)seg_end[i], 0, i * r};
+        if (seg_end[i] - prev > longest) longest = seg_end[i] - prev;
         prev = seg_end[i];
     }
-    PACT_CHECK(lddy >= N && lddy % 8 == 0 && ldu >= 2 * nseg * r && ldu % 8 == 0 && aligned16(dy) && aligned16(B) &&
-                   aligned16(U),
-               PACT_ERR_ALIGN, "pact_lora_bwd_u: pointers 16-byte aligned, leading dims %% 8 == 0");
-    RowArgs a = {};
-    a.x = dy; a.ldx = lddy; a.use_xq = 0; a.M = M; a.K = N;
-    a.w = B; a.ldw = r; a.wt = 1; a.R = nseg * r; a.r = r; a.nseg = nseg;
-    for (int i = 0; i < 4; ++i) a.seg_end[i] = i < nseg ? seg_end[i] : N;
-    a.scale = scale; a.out_bf16 = U; a.out_f32 = nullptr; a.ldo = ldu;
-    k_rows<<<(unsigned)((M + RT - 1) / RT), 256, 0, (cudaStream_t)stream>>>(a);
+    const int tiles = (int)((M + BM - 1) / BM);
+    choose_split(longest, (int64_t)tiles * nseg, &p.splits, &p.k_per_split);
+    float *ws = static_cast<float *>(workspace);
+    p.ws = ws;
+    p.ws_ld = R;
+    p.ws_split_stride = M * R;
+    s = launch_mma<false, true>(ta, tb, p, tiles, st, "pact_lora_bwd_u");
+    if (s != PACT_OK) return s;
+    k_finalize<<<finalize_grid(M * R), 256, 0, st>>>(ws, p.splits, M * R, R, M, R, scale, 0, U, ldu, R);
     return launch_status("pact_lora_bwd_u");
 }
 
+// Upper bound over segmentations: the dB output blocks number at least N / 128.
 size_t pact_lora_bwd_workspace_bytes(int64_t M, int64_t N, int64_t K, int r, int nseg) {
     const int64_t R = (int64_t)r * nseg;
-    return lora_up256((size_t)(M * R * 4)) + lora_up256((size_t)(R * K * 4)) + lora_up256((size_t)(N * r * 4));
+    return round256((size_t)(M * K * 2))                                     /* X~ as BF16 */
+           + partial_bytes(M, R, splits_of(K, (M + BM - 1) / BM))         /* T~ partials */
+           + round256((size_t)(M * 2 * R * 2))                               /* T~ hi/lo */
+           + partial_bytes(N, r, splits_of(M, (N + BM - 1) / BM))         /* dB partials */
+           + partial_bytes(K, R, splits_of(M, (K + BM - 1) / BM));        /* dA^T partials */
 }
 
 pact_status pact_lora_bwd(const pact_lora_bwd_t *g, void *workspace, size_t ws_bytes, pact_stream_t stream) {
@@ -285,59 +417,101 @@ pact_status pact_lora_bwd(const pact_lora_bwd_t *g, void *workspace, size_t ws_b
                PACT_ERR_INVALID_ARG, "pact_lora_bwd: dy, A, U, dA, dB and exactly one of x / xq are required");
     const int64_t M = g->M, N = g->N, K = g->K;
     const int r = g->r, nseg = g->nseg;
-    PACT_CHECK(M >= 1 && N >= 64 && N % 64 == 0 && K >= 64 && K % 64 == 0 &&
-                   (r == 16 || r == 32 || r == 48 || r == 64) && nseg >= 1 && nseg <= 4 && nseg * r <= 64,
+    PACT_CHECK(M >= 1 && M <= 0x7FFFFFFF && N >= 64 && N % 64 == 0 && N <= 0x7FFFFFFF && K >= 64 && K % 64 == 0 &&
+                   K <= 0x7FFFFFFF && (r == 16 || r == 32 || r == 48 || r == 64) && nseg >= 1 && nseg <= 3 &&
+                   nseg * r <= 64,
                PACT_ERR_SHAPE, "pact_lora_bwd: bad shape");
-    int64_t prev = 0;
-    for (int i = 0; i < nseg; ++i) {
-        PACT_CHECK(g->seg_end[i] > prev && g->seg_end[i] % 64 == 0 && (i + 1 < nseg || g->seg_end[i] == N),
-                   PACT_ERR_SHAPE, "pact_lora_bwd: segment ends must increase by multiples of 64 and end at N");
-        prev = g->seg_end[i];
-    }
+    pact_status s = check_segments(N, nseg, g->seg_end, "pact_lora_bwd");
+    if (s != PACT_OK) return s;
     const int R = nseg * r;
     PACT_CHECK(ws_bytes >= pact_lora_bwd_workspace_bytes(M, N, K, r, nseg), PACT_ERR_INVALID_ARG,
                "pact_lora_bwd: workspace too small");
     PACT_CHECK(g->lddy >= N && g->lddy % 8 == 0 && g->ldu >= 2 * R && g->ldu % 8 == 0 && aligned16(g->dy) &&
-                   aligned16(g->A) && aligned16(g->U) && aligned16(g->dA) && aligned16(g->dB) && aligned16(workspace) &&
-                   (!g->x || (g->ldx >= K && g->ldx % 8 == 0 && aligned16(g->x))),
-               PACT_ERR_ALIGN, "pact_lora_bwd: pointers 16-byte aligned, leading dims %% 8 == 0");
+                   aligned16(g->A) && aligned16(g->U) && aligned16(g->dA) && aligned16(g->dB) &&
+                   ((uintptr_t)workspace & 255) == 0 && (!g->x || (g->ldx >= K && g->ldx % 8 == 0 && aligned16(g->x))),
+               PACT_ERR_ALIGN, "pact_lora_bwd: pointers 16-byte aligned (workspace 256), leading dims %% 8 == 0");
     if (g->xq) {
-        pact_status s = check_nvfp4(g->xq, M, K, "xq");
+        s = check_nvfp4(g->xq, M, K, "xq");
         if (s != PACT_OK) return s;
     }
     cudaStream_t st = (cudaStream_t)stream;
     uint8_t *w8 = static_cast<uint8_t *>(workspace);
-    float *tt = reinterpret_cast<float *>(w8);
-    float *wda = reinterpret_cast<float *>(w8 + lora_up256((size_t)(M * R * 4)));
-    float *wdb = reinterpret_cast<float *>(w8 + lora_up256((size_t)(M * R * 4)) + lora_up256((size_t)(R * K * 4)));
-    pact_nvfp4_t none = {nullptr, nullptr, M, K};
+    pact_bf16 *xt = reinterpret_cast<pact_bf16 *>(w8);
+    w8 += round256((size_t)(M * K * 2));
+    float *ws_t = reinterpret_cast<float *>(w8);
+    w8 += partial_bytes(M, R, splits_of(K, (M + BM - 1) / BM));
+    pact_bf16 *tt = reinterpret_cast<pact_bf16 *>(w8);
+    w8 += round256((size_t)(M * 2 * R * 2));
+    float *ws_db = reinterpret_cast<float *>(w8);
+    w8 += partial_bytes(N, r, splits_of(M, (N + BM - 1) / BM));
+    float *ws_da = reinterpret_cast<float *>(w8);
 
-    // T~ = X~ . A^T (FP32, unscaled)
-    RowArgs a = {};
-    a.x = g->x; a.ldx = g->ldx; a.xq = g->xq ? *g->xq : none; a.use_xq = g->xq != nullptr;
-    a.M = M; a.K = K; a.w = g->A; a.ldw = K; a.wt = 0; a.R = R; a.r = R; a.nseg = 1; a.seg_end[0] = K;
-    a.scale = 1.0f; a.out_bf16 = nullptr; a.out_f32 = tt; a.ldo = R;
-    k_rows<<<(unsigned)((M + RT - 1) / RT), 256, 0, st>>>(a);
-    pact_status s = launch_status("pact_lora_bwd");
+    // X~ as BF16
+    const pact_bf16 *x = g->x;
+    int64_t ldx = g->ldx;
+    if (g->xq) {
+        k_dequantize<<<finalize_grid(M * K / 8), 256, 0, st>>>(*g->xq, xt);
+        s = launch_status("pact_lora_bwd");
+        if (s != PACT_OK) return s;
+        x = xt;
+        ldx = K;
+    }
+    // T~ = X~ . A^T (unscaled), hi/lo
+    CUtensorMap tx;
+    s = map_bf16(&tx, x, K, M, ldx, 64, BM, "pact_lora_bwd");
+    if (s == PACT_OK) s = rows_times_a(tx, M, K, g->A, R, 1.0f, tt, 2 * R, ws_t, st, "pact_lora_bwd");
     if (s != PACT_OK) return s;
-    if (cudaMemsetAsync(wda, 0, (size_t)(R * K * 4) , st) != cudaSuccess ||
-        cudaMemsetAsync(wdb, 0, (size_t)(N * r * 4), st) != cudaSuccess)
-        return fail(PACT_ERR_CUDA, "pact_lora_bwd: memset failed");
-    const unsigned mchunks = (unsigned)((M + MCHUNK - 1) / MCHUNK);
-    // dA = U^T . X~   [R x K]
-    OuterArgs o = {};
-    o.p = g->U; o.ldp = g->ldu; o.p_split = 1; o.q = g->x; o.qq = g->xq ? *g->xq : none; o.q_kind = g->xq ? 1 : 0; o.ldq = g->ldx;
-    o.M = M; o.A = R; o.Bn = K; o.segmented = 0; o.ws = wda; o.ldws = K;
-    k_outer<<<dim3((unsigned)((R + TA - 1) / TA), (unsigned)((K + TB - 1) / TB), mchunks), 256, 0, st>>>(o);
-    // dB = dY^T . T~ (segment-wise)   [N x r]
-    OuterArgs b = {};
-    b.p = g->dy; b.ldp = g->lddy; b.qf = tt; b.q_kind = 2; b.ldq = R;
-    b.M = M; b.A = N; b.Bn = r; b.segmented = 1; b.r = r; b.nseg = nseg;
-    for (int i = 0; i < 4; ++i) b.seg_end[i] = i < nseg ? g->seg_end[i] : N;
-    b.ws = wdb; b.ldws = r;
-    k_outer<<<dim3((unsigned)((N + TA - 1) / TA), (unsigned)((r + TB - 1) / TB), mchunks), 256, 0, st>>>(b);
-    k_finalize<<<256, 256, 0, st>>>(wda, R, K, 1.0f, g->dA, K);
-    k_finalize<<<256, 256, 0, st>>>(wdb, N, r, g->scale, g->dB, r);
+    // dB_i = scale * dY_i^T . T~_i: output rows are the outputs n of segment i,
+    // contraction over the tokens
+    {
+        CUtensorMap ta, tb;
+        s = map_bf16(&ta, g->dy, N, M, g->lddy, 64, 64, "pact_lora_bwd");                // dY^T, MN-major
+        if (s == PACT_OK) s = map_bf16(&tb, tt, 2 * R, M, 2 * R, 64, 64, "pact_lora_bwd");  // T~^T, MN-major
+        if (s != PACT_OK) return s;
+        Params p = {};
+        p.n_mma = 64;
+        p.n_valid = r;
+        p.nprob = nseg;
+        int64_t widest = 0, blocks = 0, prev = 0;
+        for (int i = 0; i < nseg; ++i) {
+            p.prob[i] = Prob{(int)prev, (int)g->seg_end[i], 0, (int)M, i * r, 0};
+            const int64_t w = g->seg_end[i] - prev;
+            if (w > widest) widest = w;
+            blocks += (w + BM - 1) / BM;
+            prev = g->seg_end[i];
+        }
+        p.b_split = 1;
+        p.b_lo_off = R;
+        choose_split(M, blocks, &p.splits, &p.k_per_split);
+        p.ws = ws_db;
+        p.ws_ld = r;
+        p.ws_split_stride = N * r;
+        s = launch_mma<true, true>(ta, tb, p, (int)((widest + BM - 1) / BM), st, "pact_lora_bwd");
+        if (s != PACT_OK) return s;
+        k_finalize<<<finalize_grid(N * r), 256, 0, st>>>(ws_db, p.splits, N * r, r, N, r, g->scale, 1, g->dB, r, 0);
+        s = launch_status("pact_lora_bwd");
+        if (s != PACT_OK) return s;
+    }
+    // dA^T = X~^T . U  [K x R], U = hi + lo
+    CUtensorMap ta, tb;
+    s = map_bf16(&ta, x, K, M, ldx, 64, 64, "pact_lora_bwd");                   // X~^T, MN-major
+    if (s == PACT_OK) s = map_bf16(&tb, g->U, 2 * R, M, g->ldu, 64, 64, "pact_lora_bwd");  // U^T, MN-major
+    if (s != PACT_OK) return s;
+    Params p = {};
+    p.n_mma = 64;
+    p.n_valid = R;
+    p.nprob = 1;
+    p.prob[0] = Prob{0, (int)K, 0, (int)M, 0, 0};
+    p.b_split = 1;
+    p.b_lo_off = R;
+    const int tiles = (int)((K + BM - 1) / BM);
+    choose_split(M, tiles, &p.splits, &p.k_per_split);
+    p.ws = ws_da;
+    p.ws_ld = R;
+    p.ws_split_stride = K * R;
+    s = launch_mma<true, true>(ta, tb, p, tiles, st, "pact_lora_bwd");
+    if (s != PACT_OK) return s;
+    k_finalize<<<finalize_grid(K * R), 256, 0, st>>>(ws_da, p.splits, K * R, R, K, R, 1.0f, 2, g->dA, K, 0);
     return launch_status("pact_lora_bwd");
 }
 

@@ -112,11 +112,18 @@ class PactLayer:
             "a_gu": torch.empty_like(self.a_gu), "b_gu": torch.empty_like(self.b_gu),
             "a_d": torch.empty_like(self.a_d), "b_d": torch.empty_like(self.b_d),
         }
+        # one scratch buffer shared by the LoRA calls (they run in order on one stream)
         ws = max(P.pact_lora_bwd_workspace_bytes(M, S.n_qkv, H, r, 3),
                  P.pact_lora_bwd_workspace_bytes(M, 2 * I, H, r, 2),
                  P.pact_lora_bwd_workspace_bytes(M, H, I, r, 1),
-                 P.pact_lora_bwd_workspace_bytes(M, H, H, r, 1))
-        self.ws = torch.empty(ws, dtype=torch.uint8, device=dev)
+                 P.pact_lora_bwd_workspace_bytes(M, H, H, r, 1),
+                 P.pact_lora_fwd_workspace_bytes(M, I, 3 * r),
+                 P.pact_lora_fwd_workspace_bytes(M, H, 3 * r),
+                 P.pact_lora_bwd_u_workspace_bytes(M, 2 * I, r, 2),
+                 P.pact_lora_bwd_u_workspace_bytes(M, S.n_qkv, r, 3))
+        raw = torch.empty(ws + 256, dtype=torch.uint8, device=dev)
+        off = (-raw.data_ptr()) % 256
+        self.ws = raw[off:off + ws]
         # LoRA descriptors for the fused GEMM epilogue
         self.l_qkv_f = P.lora_struct(self.t_qkv, self.b_qkv, r, self.seg_qkv)
         self.l_o_f = P.lora_struct(self.t_o, self.b_o, r, [H])
@@ -142,21 +149,21 @@ class PactLayer:
         gemm = lambda M, N, K: 2.0 * M * N * K
         return [
             Op("rmsnorm_quant_1", lambda: P.pact_rmsnorm_quant(h, self.g1, S.eps, self.xq1, self.x1, self.rstd1)),
-            Op("lora_fwd_qkv", lambda: P.pact_lora_fwd(self.x1, self.a_qkv, s, self.t_qkv)),
+            Op("lora_fwd_qkv", lambda: P.pact_lora_fwd(self.x1, self.a_qkv, s, self.t_qkv, self.ws), kernels=2),
             Op("gemm_fwd_qkv", lambda: P.pact_frozen_gemm_fwd(self.xq1, self.c_qkv, self.l_qkv_f, y=self.qkv),
                "gemm", gemm(S.M, S.n_qkv, S.H)),
             Op("quantize_attn", lambda: P.pact_quantize_nvfp4(attn, self.aq)),
-            Op("lora_fwd_o", lambda: P.pact_lora_fwd(attn, self.a_o, s, self.t_o)),
+            Op("lora_fwd_o", lambda: P.pact_lora_fwd(attn, self.a_o, s, self.t_o, self.ws), kernels=2),
             Op("gemm_fwd_o", lambda: P.pact_frozen_gemm_fwd(self.aq, self.c_o, self.l_o_f, residual=h, y=self.h2),
                "gemm", gemm(S.M, S.H, S.H)),
             Op("rmsnorm_quant_2", lambda: P.pact_rmsnorm_quant(self.h2, self.g2, S.eps, self.xq2, self.x2,
                                                                self.rstd2)),
-            Op("lora_fwd_gu", lambda: P.pact_lora_fwd(self.x2, self.a_gu, s, self.t_gu)),
+            Op("lora_fwd_gu", lambda: P.pact_lora_fwd(self.x2, self.a_gu, s, self.t_gu, self.ws), kernels=2),
             Op("gemm_fwd_gu", lambda: P.pact_frozen_gemm_fwd(self.xq2, self.c_gu, self.l_gu_f, y=self.gu),
                "gemm", gemm(S.M, 2 * I, S.H)),
             Op("silu_mul_quant", lambda: P.pact_silu_mul_quant(self.gu[:, :I], self.gu[:, I:], self.m, self.mq,
                                                                self.gq, self.uq)),
-            Op("lora_fwd_down", lambda: P.pact_lora_fwd(self.m, self.a_d, s, self.t_d)),
+            Op("lora_fwd_down", lambda: P.pact_lora_fwd(self.m, self.a_d, s, self.t_d, self.ws), kernels=2),
             Op("gemm_fwd_down", lambda: P.pact_frozen_gemm_fwd(self.mq, self.c_d, self.l_d_f, residual=self.h2,
                                                                y=self.out),
                "gemm", gemm(S.M, S.H, I)),
@@ -168,19 +175,19 @@ class PactLayer:
         _, attn, d_out, d_qkv = self.inputs
         g = self.grads
         gemm = lambda M, N, K: 2.0 * M * N * K
-        LB = 5  # kernels of one pact_lora_bwd call (plus two memsets)
+        LB = 7  # kernels of one pact_lora_bwd call reading an NVFP4 copy (6 with BF16 input)
         return [
             # down projection
-            Op("lora_bwd_u_down", lambda: P.pact_lora_bwd_u(d_out, self.b_d, r, [H], s, self.u_d)),
+            Op("lora_bwd_u_down", lambda: P.pact_lora_bwd_u(d_out, self.b_d, r, [H], s, self.u_d, self.ws), kernels=2),
             Op("quantize_dout", lambda: P.pact_quantize_nvfp4(d_out, self.doq)),
             Op("gemm_dgrad_down", lambda: P.pact_frozen_gemm_dgrad(self.doq, self.c_d, self.l_d_b, dx=self.dm),
                "gemm", gemm(S.M, I, H)),
             Op("silu_mul_bwd_quant", lambda: P.pact_silu_mul_bwd_quant(self.dm, self.gq, self.uq, self.dgu,
                                                                        self.dguq, self.m_re)),
             Op("lora_bwd_down", lambda: P.pact_lora_bwd(d_out, self.a_d, self.u_d, r, [H], s, x=self.m_re,
-                                                        dA=g["a_d"], dB=g["b_d"], workspace=self.ws), kernels=LB),
+                                                        dA=g["a_d"], dB=g["b_d"], workspace=self.ws), kernels=LB - 1),
             # gate|up
-            Op("lora_bwd_u_gu", lambda: P.pact_lora_bwd_u(self.dgu, self.b_gu, r, self.seg_gu, s, self.u_gu)),
+            Op("lora_bwd_u_gu", lambda: P.pact_lora_bwd_u(self.dgu, self.b_gu, r, self.seg_gu, s, self.u_gu, self.ws), kernels=2),
             Op("gemm_dgrad_gu", lambda: P.pact_frozen_gemm_dgrad(self.dguq, self.c_gu, self.l_gu_b, dx=self.dx2),
                "gemm", gemm(S.M, H, 2 * I)),
             Op("lora_bwd_gu", lambda: P.pact_lora_bwd(self.dgu, self.a_gu, self.u_gu, r, self.seg_gu, s,
@@ -189,13 +196,13 @@ class PactLayer:
             Op("rmsnorm_bwd_2", lambda: P.pact_rmsnorm_bwd(self.dx2, self.xq2, self.rstd2, self.g2, dres=d_out,
                                                            dx=self.dh2, dxq=self.dh2q)),
             # o projection (its output joined the residual stream h2)
-            Op("lora_bwd_u_o", lambda: P.pact_lora_bwd_u(self.dh2, self.b_o, r, [H], s, self.u_o)),
+            Op("lora_bwd_u_o", lambda: P.pact_lora_bwd_u(self.dh2, self.b_o, r, [H], s, self.u_o, self.ws), kernels=2),
             Op("gemm_dgrad_o", lambda: P.pact_frozen_gemm_dgrad(self.dh2q, self.c_o, self.l_o_b, dx=self.dattn),
                "gemm", gemm(S.M, H, H)),
             Op("lora_bwd_o", lambda: P.pact_lora_bwd(self.dh2, self.a_o, self.u_o, r, [H], s, x=attn,
-                                                     dA=g["a_o"], dB=g["b_o"], workspace=self.ws), kernels=LB),
+                                                     dA=g["a_o"], dB=g["b_o"], workspace=self.ws), kernels=LB - 1),
             # q|k|v (d_qkv stands in for the attention backward)
-            Op("lora_bwd_u_qkv", lambda: P.pact_lora_bwd_u(d_qkv, self.b_qkv, r, self.seg_qkv, s, self.u_qkv)),
+            Op("lora_bwd_u_qkv", lambda: P.pact_lora_bwd_u(d_qkv, self.b_qkv, r, self.seg_qkv, s, self.u_qkv, self.ws), kernels=2),
             Op("quantize_dqkv", lambda: P.pact_quantize_nvfp4(d_qkv, self.dqkvq)),
             Op("gemm_dgrad_qkv", lambda: P.pact_frozen_gemm_dgrad(self.dqkvq, self.c_qkv, self.l_qkv_b, dx=self.dx1),
                "gemm", gemm(S.M, H, S.n_qkv)),

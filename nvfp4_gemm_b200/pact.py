@@ -71,8 +71,10 @@ def _load() -> ctypes.CDLL:
         "pact_frozen_gemm_fwd": (S, [NV, ctypes.POINTER(c_weight_cache), ctypes.POINTER(c_lora), P, I64, P, I64, P]),
         "pact_frozen_gemm_dgrad": (S, [NV, ctypes.POINTER(c_weight_cache), ctypes.POINTER(c_lora), P, I64, P, I64,
                                        P]),
-        "pact_lora_fwd": (S, [P, I64, I64, I64, P, I, F, P, I64, P]),
-        "pact_lora_bwd_u": (S, [P, I64, I64, I64, P, I, I, ctypes.POINTER(I64), F, P, I64, P]),
+        "pact_lora_fwd_workspace_bytes": (ctypes.c_size_t, [I64, I64, I]),
+        "pact_lora_fwd": (S, [P, I64, I64, I64, P, I, F, P, I64, P, ctypes.c_size_t, P]),
+        "pact_lora_bwd_u_workspace_bytes": (ctypes.c_size_t, [I64, I64, I, I]),
+        "pact_lora_bwd_u": (S, [P, I64, I64, I64, P, I, I, ctypes.POINTER(I64), F, P, I64, P, ctypes.c_size_t, P]),
         "pact_lora_bwd_workspace_bytes": (ctypes.c_size_t, [I64, I64, I64, I, I]),
         "pact_lora_bwd": (S, [ctypes.POINTER(c_lora_bwd), P, ctypes.c_size_t, P]),
         "pact_silu_mul_bwd_quant": (S, [P, I64, NV, NV, I64, I64, P, I64, NV, P, P]),
@@ -271,28 +273,45 @@ def pact_frozen_gemm_dgrad(dyq: NVFP4Tensor, w: WeightCache, lora: Optional[c_lo
     return dx
 
 
+def _workspace(ws: Optional[torch.Tensor], need: int, device) -> torch.Tensor:
+    if ws is None:
+        ws = torch.empty(need, dtype=torch.uint8, device=device)
+    return ws
+
+
+def pact_lora_fwd_workspace_bytes(M: int, K: int, R: int) -> int:
+    return int(_lib.pact_lora_fwd_workspace_bytes(M, K, R))
+
+
 def pact_lora_fwd(x: torch.Tensor, A: torch.Tensor, scale: float, T: Optional[torch.Tensor] = None,
-                  stream=None) -> torch.Tensor:
+                  workspace: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
     _bf16(x, "x")
     _bf16(A, "A")
     M, K = x.shape
     R = A.shape[0]
     if T is None:
         T = torch.empty((M, 2 * R), dtype=torch.bfloat16, device=x.device)
+    ws = _workspace(workspace, pact_lora_fwd_workspace_bytes(M, K, R), x.device)
     _check(_lib.pact_lora_fwd(x.data_ptr(), _ld(x), M, K, A.data_ptr(), R, float(scale), T.data_ptr(), _ld(T),
-                              _stream(stream)))
+                              ws.data_ptr(), ws.numel(), _stream(stream)))
     return T
 
 
+def pact_lora_bwd_u_workspace_bytes(M: int, N: int, r: int, nseg: int) -> int:
+    return int(_lib.pact_lora_bwd_u_workspace_bytes(M, N, r, nseg))
+
+
 def pact_lora_bwd_u(dy: torch.Tensor, B: torch.Tensor, r: int, seg_end: Sequence[int], scale: float,
-                    U: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+                    U: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None,
+                    stream=None) -> torch.Tensor:
     _bf16(dy, "dy")
     M, N = dy.shape
     if U is None:
         U = torch.empty((M, 2 * r * len(seg_end)), dtype=torch.bfloat16, device=dy.device)
     se = (ctypes.c_int64 * 4)(*(list(seg_end) + [0] * (4 - len(seg_end))))
+    ws = _workspace(workspace, pact_lora_bwd_u_workspace_bytes(M, N, r, len(seg_end)), dy.device)
     _check(_lib.pact_lora_bwd_u(dy.data_ptr(), _ld(dy), M, N, B.data_ptr(), r, len(seg_end), se, float(scale),
-                                U.data_ptr(), _ld(U), _stream(stream)))
+                                U.data_ptr(), _ld(U), ws.data_ptr(), ws.numel(), _stream(stream)))
     return U
 
 
@@ -314,7 +333,9 @@ def pact_lora_bwd(dy: torch.Tensor, A: torch.Tensor, U: torch.Tensor, r: int, se
         dB = torch.empty((N, r), dtype=torch.bfloat16, device=dy.device)
     need = pact_lora_bwd_workspace_bytes(M, N, K, r, nseg)
     if workspace is None:
-        workspace = torch.empty(need, dtype=torch.uint8, device=dy.device)
+        workspace = torch.empty(need + 256, dtype=torch.uint8, device=dy.device)
+        off = (-workspace.data_ptr()) % 256
+        workspace = workspace[off:off + need]
     xq_s = xq.c() if xq is not None else None
     args = c_lora_bwd()
     args.M, args.N, args.K = M, N, K
