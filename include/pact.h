@@ -202,6 +202,22 @@ PACT_API pact_status pact_lora_fwd(const pact_bf16 *x, int64_t ldx, int64_t M, i
                                    const pact_bf16 *A, int R, float scale, pact_bf16 *T, int64_t ldt,
                                    void *workspace, size_t ws_bytes, pact_stream_t stream);
 
+/* pact_lora_fwd without a workspace argument.  The pages have no counterpart of
+ * this call: it exists for callers that cannot allocate device memory where they
+ * call the library (plain C callers without a device allocator, code that must not
+ * call cudaMalloc because it may synchronise the device or because the device
+ * memory budget is fixed at start-up).  Same arguments and results as
+ * pact_lora_fwd; the scratch is an 8 MiB array inside the library's device code
+ * that every GPU loading the library holds until the process exits.  Shapes whose
+ * scratch (pact_lora_fwd_workspace_bytes) exceeds 8 MiB return PACT_ERR_SHAPE.
+ * The first call on a device looks up the array's device address (a CUDA runtime
+ * query, once per device); make that first call before any stream capture.  All
+ * calls on a device share the array, so calls that overlap on the GPU (different
+ * streams) race.  It allocates nothing. */
+PACT_API pact_status pact_lora_fwd_noalloc(const pact_bf16 *x, int64_t ldx, int64_t M, int64_t K,
+                                           const pact_bf16 *A, int R, float scale, pact_bf16 *T,
+                                           int64_t ldt, pact_stream_t stream);
+
 /* --------------------------------------------------- A8: LoRA backward */
 /* [LORA] gradients, BF16 throughout ([METHOD]: adapters stay BF16).
  * pact_lora_bwd_u: U[:, i*r .. i*r+r-1] = scale * dY[:, seg_i] . B[seg_i, :] for dY

@@ -516,3 +516,68 @@ pact_status pact_lora_bwd(const pact_lora_bwd_t *g, void *workspace, size_t ws_b
 }
 
 }  // extern "C"
+
+// ----------------------------------------------------------------------------
+// Allocation-free LoRA forward.
+//
+// Some callers cannot hand this library a workspace: plain C programs that have no
+// device allocator of their own, and code that must not call cudaMalloc at the
+// point of use (cudaMalloc may synchronise the device, and services that fix
+// their device-memory budget at start-up forbid allocation afterwards).  For them,
+// pact_lora_fwd_noalloc runs the same kernels as pact_lora_fwd with its scratch
+// (the FP32 partial sums) in a fixed array that lives in this library's device
+// code.  Every GPU that loads the library holds the array until the process
+// exits.  All calls on a device share it and it keeps the last call's contents
+// (each call overwrites every partial it reads, so nothing needs clearing), so two
+// calls that overlap on the GPU (different streams) race on it.
+// ----------------------------------------------------------------------------
+namespace pact {
+namespace lmma {
+
+constexpr size_t NOALLOC_SCRATCH_BYTES = 8u << 20;  // 8 MiB
+static __device__ __align__(256) unsigned char g_noalloc_scratch[NOALLOC_SCRATCH_BYTES];
+
+// Device address of g_noalloc_scratch for the current device.  The symbol's host
+// name is only a stand-in, so the address is looked up once per device (with that
+// device current) and kept.
+static pact_status noalloc_scratch(void **out) {
+    static void *addr[64] = {nullptr};
+    const int d = current_device();
+    if (d < 0 || d >= 64) return fail(PACT_ERR_UNSUPPORTED, "pact_lora_fwd_noalloc: device index %d unsupported", d);
+    if (!addr[d]) {
+        void *p = nullptr;
+        const cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+        if (e != cudaSuccess || !p)
+            return fail(PACT_ERR_CUDA, "pact_lora_fwd_noalloc: cudaGetSymbolAddress failed: %s", cudaGetErrorString(e));
+        addr[d] = p;
+    }
+    *out = addr[d];
+    return PACT_OK;
+}
+
+}  // namespace lmma
+}  // namespace pact
+
+extern "C" pact_status pact_lora_fwd_noalloc(const pact_bf16 *x, int64_t ldx, int64_t M, int64_t K,
+                                             const pact_bf16 *A, int R, float scale, pact_bf16 *T, int64_t ldt,
+                                             pact_stream_t stream) {
+    PACT_CHECK(x && A && T, PACT_ERR_INVALID_ARG, "pact_lora_fwd_noalloc: NULL argument");
+    PACT_CHECK(M >= 1 && M <= 0x7FFFFFFF && K >= 64 && K % 64 == 0 && K <= 0x7FFFFFFF && R >= 16 && R <= 64 &&
+                   R % 16 == 0,
+               PACT_ERR_SHAPE, "pact_lora_fwd_noalloc: need M >= 1, K a multiple of 64, R in {16, 32, 48, 64}");
+    PACT_CHECK(ldx >= K && ldx % 8 == 0 && ldt >= 2 * R && ldt % 8 == 0 && aligned16(x) && aligned16(A) && aligned16(T),
+               PACT_ERR_ALIGN, "pact_lora_fwd_noalloc: pointers 16-byte aligned, leading dims %% 8 == 0");
+    const size_t need = pact_lora_fwd_workspace_bytes(M, K, R);
+    PACT_CHECK(need <= NOALLOC_SCRATCH_BYTES, PACT_ERR_SHAPE,
+               "pact_lora_fwd_noalloc: this shape needs %zu bytes of scratch, more than the built-in %zu bytes; "
+               "use pact_lora_fwd with a workspace",
+               need, (size_t)NOALLOC_SCRATCH_BYTES);
+    void *scratch = nullptr;
+    pact_status s = noalloc_scratch(&scratch);
+    if (s != PACT_OK) return s;
+    CUtensorMap tx;
+    s = map_bf16(&tx, x, K, M, ldx, 64, BM, "pact_lora_fwd_noalloc");
+    if (s != PACT_OK) return s;
+    return rows_times_a(tx, M, K, A, R, scale, T, ldt, static_cast<float *>(scratch), (cudaStream_t)stream,
+                        "pact_lora_fwd_noalloc");
+}

@@ -73,6 +73,7 @@ def _load() -> ctypes.CDLL:
                                        P]),
         "pact_lora_fwd_workspace_bytes": (ctypes.c_size_t, [I64, I64, I]),
         "pact_lora_fwd": (S, [P, I64, I64, I64, P, I, F, P, I64, P, ctypes.c_size_t, P]),
+        "pact_lora_fwd_noalloc": (S, [P, I64, I64, I64, P, I, F, P, I64, P]),
         "pact_lora_bwd_u_workspace_bytes": (ctypes.c_size_t, [I64, I64, I, I]),
         "pact_lora_bwd_u": (S, [P, I64, I64, I64, P, I, I, ctypes.POINTER(I64), F, P, I64, P, ctypes.c_size_t, P]),
         "pact_lora_bwd_workspace_bytes": (ctypes.c_size_t, [I64, I64, I64, I, I]),
@@ -294,6 +295,20 @@ def pact_lora_fwd(x: torch.Tensor, A: torch.Tensor, scale: float, T: Optional[to
     ws = _workspace(workspace, pact_lora_fwd_workspace_bytes(M, K, R), x.device)
     _check(_lib.pact_lora_fwd(x.data_ptr(), _ld(x), M, K, A.data_ptr(), R, float(scale), T.data_ptr(), _ld(T),
                               ws.data_ptr(), ws.numel(), _stream(stream)))
+    return T
+
+
+def pact_lora_fwd_noalloc(x: torch.Tensor, A: torch.Tensor, scale: float, T: Optional[torch.Tensor] = None,
+                          stream=None) -> torch.Tensor:
+    """pact_lora_fwd without a workspace: the library's built-in device scratch is used."""
+    _bf16(x, "x")
+    _bf16(A, "A")
+    M, K = x.shape
+    R = A.shape[0]
+    if T is None:
+        T = torch.empty((M, 2 * R), dtype=torch.bfloat16, device=x.device)
+    _check(_lib.pact_lora_fwd_noalloc(x.data_ptr(), _ld(x), M, K, A.data_ptr(), R, float(scale), T.data_ptr(), _ld(T),
+                                      _stream(stream)))
     return T
 
 
