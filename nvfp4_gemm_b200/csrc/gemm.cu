@@ -304,6 +304,263 @@ k_nvfp4_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CU
     }
 }
 
+
+// ---------------------------------------------------------------------------------
+// CTA-pair variant: a cluster of 2 CTAs computes a 256 x 256 tile with 2-SM MMAs
+// (tcgen05 cta_group::2).  CTA r of the pair holds rows 128r..128r+127 of A and of
+// the accumulator, and rows 128r..128r+127 of the B tile; the MMA reads both halves
+// of A and B across the pair, so each SM streams half as much B per unit of work
+// as the single-CTA kernel.  Every scale tile arrives by TMA; the leader (rank 0)
+// arms its full barrier for both CTAs' bytes, the peer's loads complete on it, and
+// the leader issues the scale copies and MMAs for the pair and multicasts its
+// commits to both CTAs' barriers.
+// ---------------------------------------------------------------------------------
+namespace pair {
+
+constexpr int BM = 128;               // rows per CTA; the pair tile has 256
+constexpr int BN = 256;               // columns of the pair tile; each CTA loads 128 rows of B
+constexpr int BK = 256;
+constexpr int KSTEP = 64;
+constexpr int STAGES = 5;
+constexpr int A_BYTES = BM * BK / 2;          // 16384
+constexpr int B_BYTES = (BN / 2) * BK / 2;    // 16384
+constexpr int OFF_B = A_BYTES;
+constexpr int OFF_SFA = OFF_B + B_BYTES;      // 4 chunks of 512 (this CTA's rows)
+constexpr int OFF_SFB = OFF_SFA + 2048;       // 2 row groups x 4 chunks (all 256 columns)
+constexpr int STAGE_BYTES = OFF_SFB + 4096;   // 38912 = 38 KiB
+constexpr int LOAD_BYTES = STAGE_BYTES;       // bytes one CTA's loads deliver per k stage
+constexpr int OFF_LW = 6 * BM * 32;           // LoRA weight chunks follow 6 activation chunks
+constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + 256;
+constexpr int THREADS = 192;
+constexpr uint32_t TMEM_COLS = 512;
+constexpr uint32_t COL_ACC = 0, COL_SFA = 256, COL_SFB = 272;
+static_assert(OFF_LW + 3 * BM * 32 <= STAGE_BYTES && OFF_LW + 2 * 48 * 128 <= STAGE_BYTES, "LoRA stage");
+
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
+k_nvfp4_gemm_pair(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                  const __grid_constant__ CUtensorMap tmSFA, const __grid_constant__ CUtensorMap tmSFB,
+                  const __grid_constant__ CUtensorMap tmLa, const __grid_constant__ CUtensorMap tmLb,
+                  const Params p) {
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw = smem_u32(smem_raw);
+    uint8_t *smem = smem_raw + (((raw + 1023) & ~1023u) - raw);
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + STAGES * STAGE_BYTES);
+    uint64_t *full = bars;                       // [STAGES], used in the leader
+    uint64_t *empty = bars + STAGES;             // [STAGES]
+    uint64_t *acc_full = bars + 2 * STAGES;      // leader MMA -> both epilogues
+    uint64_t *acc_empty = bars + 2 * STAGES + 1; // both epilogues -> leader MMA
+    uint64_t *drained = bars + 2 * STAGES + 2;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 2 * STAGES + 3);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint32_t rank = cluster_ctarank();
+    const bool leader = rank == 0;
+    const int mpairs = (p.M + 2 * BM - 1) / (2 * BM), ntiles = (p.N + BN - 1) / BN;
+    const int total = mpairs * ntiles;
+    const int cluster = blockIdx.x >> 1, nclusters = gridDim.x >> 1;
+    const int ktiles = (p.K + BK - 1) / BK;
+    const int kgroups = p.K / 64;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
+        }
+        mbar_init(acc_full, 1);
+        mbar_init(acc_empty, 8);
+        mbar_init(drained, 1);
+        fence_barrier_init();
+    }
+    if (warp == 0 && lane == 0) {
+        prefetch_tensormap(&tmA);
+        prefetch_tensormap(&tmB);
+        prefetch_tensormap(&tmSFA);
+        prefetch_tensormap(&tmSFB);
+        if (p.lora_mode != LORA_NONE) {
+            prefetch_tensormap(&tmLa);
+            prefetch_tensormap(&tmLb);
+        }
+    }
+    if (warp == 1) {
+        tmem_alloc_pair(tmem_slot, TMEM_COLS);
+        tmem_relinquish_pair();
+    }
+    tc_fence_before();
+    __syncthreads();
+    cluster_sync();  // the peer's barriers exist before anything addresses them
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    const uint32_t full_leader = mapa_shared(smem_u32(full), 0);
+    const uint32_t acc_empty_leader = mapa_shared(smem_u32(acc_empty), 0);
+
+    if (warp == 0) {
+        // ------------------------------------------------------------ producer (both CTAs)
+        if (lane == 0) {
+            uint32_t stage = 0, phase = 0;
+            bool ok = true;
+            for (int t = cluster; ok && t < total; t += nclusters) {
+                const int mp = t % mpairs, nt = t / mpairs;
+                const int m0 = mp * 2 * BM + (int)rank * BM;     // this CTA's rows
+                const int n0 = nt * BN, nb = n0 + (int)rank * (BN / 2);
+                if (p.lora_mode != LORA_NONE) {
+                    if (!(ok = mbar_wait(&empty[stage], phase ^ 1))) break;
+                    const uint32_t st = smem_u32(smem + stage * STAGE_BYTES);
+                    const uint32_t fb = full_leader + 8 * stage;
+                    const int R = p.lora_nseg * p.lora_r;
+                    if (p.lora_mode == LORA_FWD) {
+                        if (leader) mbar_arrive_expect_tx(&full[stage], 2 * p.lora_steps * (2 * BM * 32 + BM * 32));
+                        const int xs = lora_segment(p, n0) * p.lora_r;
+                        for (int c = 0; c < p.lora_steps; ++c) {
+                            tma_load_2d_pair(st + c * BM * 32, &tmLa, fb, xs + 16 * c, m0);
+                            tma_load_2d_pair(st + (p.lora_steps + c) * BM * 32, &tmLa, fb, R + xs + 16 * c, m0);
+                            tma_load_2d_pair(st + OFF_LW + c * BM * 32, &tmLb, fb, 16 * c, nb);
+                        }
+                    } else {
+                        if (leader) mbar_arrive_expect_tx(&full[stage], 2 * (p.lora_steps * 2 * BM * 32 + 2 * R * 128));
+                        for (int c = 0; c < p.lora_steps; ++c) {
+                            tma_load_2d_pair(st + c * BM * 32, &tmLa, fb, 16 * c, m0);
+                            tma_load_2d_pair(st + (p.lora_steps + c) * BM * 32, &tmLa, fb, R + 16 * c, m0);
+                        }
+                        for (int q = 0; q < 2; ++q) tma_load_2d_pair(st + OFF_LW + q * R * 128, &tmLb, fb, nb + 64 * q, 0);
+                    }
+                    if (++stage == STAGES) { stage = 0; phase ^= 1; }
+                }
+                const int ga = m0 / 128, gb = n0 / 128;
+                for (int kt = 0; kt < ktiles; ++kt) {
+                    if (!(ok = mbar_wait(&empty[stage], phase ^ 1))) break;
+                    const uint32_t st = smem_u32(smem + stage * STAGE_BYTES);
+                    const uint32_t fb = full_leader + 8 * stage;
+                    if (leader) mbar_arrive_expect_tx(&full[stage], 2 * LOAD_BYTES);
+                    tma_load_2d_pair(st, &tmA, fb, kt * (BK / 2), m0);
+                    tma_load_2d_pair(st + OFF_B, &tmB, fb, kt * (BK / 2), nb);
+                    // scale chunks: 512 bytes = two 256-byte rows of the scale map
+                    tma_load_2d_pair(st + OFF_SFA, &tmSFA, fb, 0, 2 * (ga * kgroups + kt * 4));
+                    tma_load_2d_pair(st + OFF_SFB, &tmSFB, fb, 0, 2 * (gb * kgroups + kt * 4));
+                    tma_load_2d_pair(st + OFF_SFB + 2048, &tmSFB, fb, 0, 2 * ((gb + 1) * kgroups + kt * 4));
+                    if (++stage == STAGES) { stage = 0; phase ^= 1; }
+                }
+            }
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------------------ MMA issuer (leader)
+        if (leader) {
+            const uint32_t idesc = idesc_nvf4(2 * BM, BN);
+            const uint32_t idesc_lora = idesc_bf16(2 * BM, BN, false, p.lora_mode == LORA_DGRAD);
+            uint32_t stage = 0, phase = 0, acc_phase = 0;
+            for (int t = cluster; t < total; t += nclusters) {
+                bool ok = mbar_wait(acc_empty, acc_phase ^ 1);
+                tc_fence_after();
+                uint32_t accum = 0;
+                if (ok && p.lora_mode != LORA_NONE) {
+                    ok = mbar_wait(&full[stage], phase);
+                    tc_fence_after();
+                    if (ok && lane == 0) {
+                        const uint32_t st = smem_u32(smem + stage * STAGE_BYTES);
+                        const int R = p.lora_nseg * p.lora_r;
+                        for (int c = 0; c < p.lora_steps; ++c) {
+                            const uint64_t bd = (p.lora_mode == LORA_FWD)
+                                                    ? smem_desc(st + OFF_LW + c * BM * 32, 16, 256, SW_32)
+                                                    : smem_desc(st + OFF_LW + c * 2048, R * 128, 1024, SW_128);
+                            for (int h = 0; h < 2; ++h) {
+                                const uint64_t ad = smem_desc(st + (h * p.lora_steps + c) * BM * 32, 16, 256, SW_32);
+                                mma_bf16_pair(tmem + COL_ACC, ad, bd, idesc_lora, accum);
+                                accum = 1;
+                            }
+                        }
+                        tc_commit_pair(&empty[stage], 3);
+                    }
+                    accum = 1;
+                    __syncwarp();
+                    if (++stage == STAGES) { stage = 0; phase ^= 1; }
+                }
+                for (int kt = 0; ok && kt < ktiles; ++kt) {
+                    ok = mbar_wait(&full[stage], phase);
+                    tc_fence_after();
+                    if (ok && lane == 0) {
+                        const int nk = min(BK / KSTEP, (p.K - kt * BK) / KSTEP);
+                        const uint32_t st = smem_u32(smem + stage * STAGE_BYTES);
+                        for (int s = 0; s < nk; ++s) {
+                            tmem_cp_pair_32x128b_x4(tmem + COL_SFA + 4 * s,
+                                                    smem_desc(st + OFF_SFA + s * 512, 0, 128, SW_NONE));
+                            for (int g = 0; g < 2; ++g)
+                                tmem_cp_pair_32x128b_x4(tmem + COL_SFB + 8 * s + 4 * g,
+                                                        smem_desc(st + OFF_SFB + g * 2048 + s * 512, 0, 128, SW_NONE));
+                        }
+                        for (int s = 0; s < nk; ++s) {
+                            const uint64_t ad = smem_desc(st + s * 32, 16, 1024, SW_128);
+                            const uint64_t bd = smem_desc(st + OFF_B + s * 32, 16, 1024, SW_128);
+                            mma_nvf4_pair(tmem + COL_ACC, ad, bd, idesc, tmem + COL_SFA + 4 * s, tmem + COL_SFB + 8 * s,
+                                          accum);
+                            accum = 1;
+                        }
+                        tc_commit_pair(&empty[stage], 3);
+                    }
+                    accum = 1;
+                    __syncwarp();
+                    if (++stage == STAGES) { stage = 0; phase ^= 1; }
+                }
+                if (!ok) break;
+                if (lane == 0) tc_commit_pair(acc_full, 3);
+                __syncwarp();
+                acc_phase ^= 1;
+            }
+            if (lane == 0) tc_commit_pair(drained, 1);
+            mbar_wait(drained, 0);
+        }
+    } else {
+        // ------------------------------------------------------------ epilogue (both CTAs)
+        const int sub = warp & 3;
+        uint32_t acc_phase = 0;
+        for (int t = cluster; t < total; t += nclusters) {
+            const int mp = t % mpairs, nt = t / mpairs;
+            if (!mbar_wait(acc_full, acc_phase)) break;
+            tc_fence_after();
+            const int row = mp * 2 * BM + (int)rank * BM + sub * 32 + lane;
+            for (int c = 0; c < BN / 32; ++c) {
+                const int n = nt * BN + c * 32;
+                if (n >= p.N) break;
+                uint32_t r[32];
+                tmem_ld_32x32b_x32(tmem + ((uint32_t)(sub * 32) << 16) + COL_ACC + c * 32, r);
+                tmem_ld_wait();
+                if (row < p.M) {
+                    uint4 *d4 = reinterpret_cast<uint4 *>(p.out + (size_t)row * p.ldo + n);
+                    const uint4 *r4 = p.res ? reinterpret_cast<const uint4 *>(p.res + (size_t)row * p.ldr + n) : nullptr;
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        float f[8];
+#pragma unroll
+                        for (int i = 0; i < 8; ++i) f[i] = __uint_as_float(r[8 * q + i]);
+                        if (r4) {
+                            const uint4 old = r4[q];
+                            f[0] += bf16lo(old.x); f[1] += bf16hi(old.x); f[2] += bf16lo(old.y); f[3] += bf16hi(old.y);
+                            f[4] += bf16lo(old.z); f[5] += bf16hi(old.z); f[6] += bf16lo(old.w); f[7] += bf16hi(old.w);
+                        }
+                        uint4 v;
+                        v.x = pack_bf16x2(f[0], f[1]); v.y = pack_bf16x2(f[2], f[3]);
+                        v.z = pack_bf16x2(f[4], f[5]); v.w = pack_bf16x2(f[6], f[7]);
+                        d4[q] = v;
+                    }
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive_remote(acc_empty_leader);
+            acc_phase ^= 1;
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    cluster_sync();  // every MMA of the pair has completed and both epilogues are done
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc_pair(tmem, TMEM_COLS);
+    }
+    cluster_sync();
+}
+
+}  // namespace pair
+
 // ------------------------------------------------------------------ host side
 typedef CUresult (*EncodeTiled)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
                                 const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
@@ -343,7 +600,8 @@ static pact_status ensure_attrs() {
     static bool done[64] = {false};
     const int d = current_device();
     if (d >= 0 && d < 64 && done[d]) return PACT_OK;
-    cudaError_t e = cudaFuncSetAttribute(k_nvfp4_gemm, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+    cudaError_t e =
+        cudaFuncSetAttribute(pair::k_nvfp4_gemm_pair, cudaFuncAttributeMaxDynamicSharedMemorySize, pair::SMEM_BYTES);
     if (e != cudaSuccess) return fail(PACT_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));
     if (d >= 0 && d < 64) done[d] = true;
     return PACT_OK;
@@ -390,12 +648,22 @@ static pact_status run(const pact_nvfp4_t *a, const pact_nvfp4_t *b, const pact_
     if (s != PACT_OK) return s;
     s = ensure_attrs();
     if (s != PACT_OK) return s;
-    CUtensorMap tmA, tmB, tmLa, tmLb;
-    s = make_map(&tmA, CU_TENSOR_MAP_DATA_TYPE_UINT8, a->codes, K / 2, M, K / 2, 128, BM,
+    CUtensorMap tmA, tmB, tmSFA, tmSFB, tmLa, tmLb;
+    // operand tiles: 128 rows x 128 bytes (256 FP4 values), 128-byte swizzle
+    s = make_map(&tmA, CU_TENSOR_MAP_DATA_TYPE_UINT8, a->codes, K / 2, M, K / 2, 128, 128,
                  CU_TENSOR_MAP_SWIZZLE_128B, what);
     if (s == PACT_OK)
-        s = make_map(&tmB, CU_TENSOR_MAP_DATA_TYPE_UINT8, b->codes, K / 2, N, K / 2, 128, BN,
+        s = make_map(&tmB, CU_TENSOR_MAP_DATA_TYPE_UINT8, b->codes, K / 2, N, K / 2, 128, 128,
                      CU_TENSOR_MAP_SWIZZLE_128B, what);
+    // scale tiles: each 512-byte chunk (128 rows x 4 blocks) is two 256-byte rows of
+    // a [2 * chunks x 256] byte matrix; one box is 4 chunks
+    const uint64_t chunks_a = (uint64_t)((M + 127) / 128) * (K / 64), chunks_b = (uint64_t)((N + 127) / 128) * (K / 64);
+    if (s == PACT_OK)
+        s = make_map(&tmSFA, CU_TENSOR_MAP_DATA_TYPE_UINT8, a->scales, 256, 2 * chunks_a, 256, 256, 8,
+                     CU_TENSOR_MAP_SWIZZLE_NONE, what);
+    if (s == PACT_OK)
+        s = make_map(&tmSFB, CU_TENSOR_MAP_DATA_TYPE_UINT8, b->scales, 256, 2 * chunks_b, 256, 256, 8,
+                     CU_TENSOR_MAP_SWIZZLE_NONE, what);
     if (s != PACT_OK) return s;
     Params p;
     p.M = (int)M; p.N = (int)N; p.K = (int)K;
@@ -415,14 +683,14 @@ static pact_status run(const pact_nvfp4_t *a, const pact_nvfp4_t *b, const pact_
         p.lora_r = lora->r;
         p.lora_nseg = lora->nseg;
         for (int i = 0; i < 4; ++i) p.seg_end[i] = i < lora->nseg ? lora->seg_end[i] : N;
-        s = make_map(&tmLa, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, lora->act, 2 * R, M, lora->ld_act * 2, 16, BM,
+        s = make_map(&tmLa, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, lora->act, 2 * R, M, lora->ld_act * 2, 16, 128,
                      CU_TENSOR_MAP_SWIZZLE_32B, what);
         if (s != PACT_OK) return s;
         if (!dgrad) {
             p.lora_mode = LORA_FWD;
             p.lora_steps = lora->r / 16;
             s = make_map(&tmLb, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, lora->weight, lora->r, N, lora->ld_weight * 2, 16,
-                         BN, CU_TENSOR_MAP_SWIZZLE_32B, what);
+                         128, CU_TENSOR_MAP_SWIZZLE_32B, what);
         } else {
             p.lora_mode = LORA_DGRAD;
             p.lora_steps = R / 16;
@@ -431,9 +699,10 @@ static pact_status run(const pact_nvfp4_t *a, const pact_nvfp4_t *b, const pact_
         }
         if (s != PACT_OK) return s;
     }
-    const int tiles = (int)(((M + BM - 1) / BM) * ((N + BN - 1) / BN));
-    const int grid = tiles < sm_count() ? tiles : sm_count();
-    k_nvfp4_gemm<<<grid, THREADS, SMEM_BYTES, stream>>>(tmA, tmB, tmLa, tmLb, p);
+    const int pairs = (int)(((M + 255) / 256) * ((N + 255) / 256));
+    const int clusters = pairs < sm_count() / 2 ? pairs : sm_count() / 2;
+    pair::k_nvfp4_gemm_pair<<<2 * clusters, pair::THREADS, pair::SMEM_BYTES, stream>>>(tmA, tmB, tmSFA, tmSFB, tmLa,
+                                                                                        tmLb, p);
     return launch_status(what);
 }
 

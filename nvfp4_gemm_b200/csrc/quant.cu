@@ -136,18 +136,25 @@ __global__ void __launch_bounds__(RMS_THREADS) k_rmsnorm_quant(const pact_bf16 *
 }
 
 // --------------------------------------------------- A4: SiLU-multiply + quantize
-// m = BF16_RNE(silu(g) * u) with the same FP32-then-check scheme: FP32 error of
-// g / (1 + expf(-g)) * u is a few ulps; near a BF16 midpoint the double expression
-// decides.
-__device__ __forceinline__ float silu_mul_out(float g, float u) {
-    const float m = __fmul_rn(__fdiv_rn(g, __fadd_rn(1.0f, expf(-g))), u);
+// m = BF16_RNE(silu(g) * u), exactly rounded.  The FP32 evaluation with the fast
+// exponential and division has a relative error of at most (5 + 1.16 |g|) FP32
+// ulps (CUDA's documented bounds for __expf and __fdividef plus three roundings),
+// i.e. at most 2 * (5 + 1.16 * 40) < 110 ulps of the result for |g| <= 40; it
+// decides unless it lies within 256 ulps of a BF16 midpoint, and the double
+// expression decides otherwise and for |g| > 40 (Ziv's method, as above).
+__device__ __forceinline__ float sigmoid_fast(float g) { return __fdividef(1.0f, 1.0f + __expf(-g)); }
+
+__device__ __forceinline__ float silu_mul_round(float g, float u, float s) {
+    const float m = __fmul_rn(__fmul_rn(g, s), u);
     const uint32_t lo = __float_as_uint(m) & 0xFFFFu;
-    if (lo - 0x7FC0u <= 0x80u || !isfinite(m)) {
+    if (lo - 0x7F00u <= 0x200u || !(fabsf(g) <= 40.0f) || !isfinite(m)) {
         const double gd = (double)g;
         return __bfloat162float(__double2bfloat16((gd / (1.0 + exp(-gd))) * (double)u));
     }
     return __bfloat162float(__float2bfloat16_rn(m));
 }
+
+__device__ __forceinline__ float silu_mul_out(float g, float u) { return silu_mul_round(g, u, sigmoid_fast(g)); }
 
 __global__ void __launch_bounds__(256) k_silu_mul_quant(const pact_bf16 *__restrict__ g, const pact_bf16 *__restrict__ u,
                                                         int64_t ld_gu, int64_t M, int64_t I,
@@ -222,10 +229,10 @@ __global__ void __launch_bounds__(256) k_silu_mul_bwd_quant(const pact_bf16 *__r
         float dg[8], du[8], mr[8];
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
-            const float s = 1.0f / (1.0f + expf(-gh[i]));
+            const float s = sigmoid_fast(gh[i]);
             dg[i] = __bfloat162float(__float2bfloat16_rn(d[i] * uh[i] * s * (1.0f + gh[i] * (1.0f - s))));
             du[i] = __bfloat162float(__float2bfloat16_rn(d[i] * gh[i] * s));
-            mr[i] = valid ? silu_mul_out(gh[i], uh[i]) : 0.0f;
+            mr[i] = valid ? silu_mul_round(gh[i], uh[i], s) : 0.0f;
         }
         if (valid) {
             store8_bf16(dgu + row * lddgu + c, dg);
@@ -293,7 +300,7 @@ __global__ void __launch_bounds__(RMS_THREADS) k_rmsnorm_bwd(const pact_bf16 *__
         }
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
-            const float val = r * (g[i] * dv[k][i] - (yv[k][i] / g[i]) * mean) + res[i];
+            const float val = r * (g[i] * dv[k][i] - __fdividef(yv[k][i], g[i]) * mean) + res[i];
             o[i] = valid ? __bfloat162float(__float2bfloat16_rn(val)) : 0.0f;
         }
         if (valid) store8_bf16(dx + row * H + c, o);
