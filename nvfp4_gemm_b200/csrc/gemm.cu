@@ -8,57 +8,72 @@
 // One kernel serves both directions: D[M x N] = deq(A)[M x K] . deq(B)[N x K]^T with
 // A, B NVFP4 and K-major (forward: A = q(x), B = W_fwd; dgrad: A = q(dY), B = W_bwd).
 //
-// Design (sm_100a):
-//  * persistent CTAs, one per SM, 128 x 256 output tiles, static round-robin schedule;
-//  * warp 0 issues TMA (operand tiles, 128-byte swizzle) and bulk copies (scale
-//    tiles, already in the 512-byte layout the tensor core reads) into a 4-stage
-//    shared-memory ring guarded by mbarriers;
-//  * warp 1 moves each stage's scales shared -> tensor memory (tcgen05.cp) and issues
-//    tcgen05.mma kind::mxf4nvf4 (E2M1 x E2M1, UE4M3 scale per 16) into a 128 x 256
-//    FP32 accumulator in tensor memory; the LoRA term is one or more kind::f16 MMAs
-//    into the same accumulator before the NVFP4 K loop;
-//  * warps 2-5 drain the accumulator (tcgen05.ld), round to BF16 and store.
+// Design (sm_100a), one cluster of 2 CTAs (a CTA pair on two SMs) per 256 x 256
+// output tile, persistent over tiles:
+//  * 2-SM MMAs (tcgen05 cta_group::2, kind::mxf4nvf4, scale_vec::4X, K = 64 per
+//    instruction): CTA r of the pair holds rows 128r..128r+127 of A, of the B tile
+//    and of the FP32 accumulator (128 lanes x 256 columns of its tensor memory); the
+//    leader (rank 0) issues every MMA for the pair.  Each SM streams 38 KiB per
+//    K = 256 stage, 30% less than a single-CTA 128 x 256 tile needs, which keeps
+//    the L2 -> shared-memory stream below what the tensor core consumes.
+//  * warp 0 (both CTAs): TMA producer into a 4-stage ring.  Operand tiles complete
+//    on the leader's `full` barrier (armed by the leader for both CTAs' bytes); the
+//    CTA's own scale tiles complete on its local `sf_full` barrier.
+//  * warps 2-5 (both CTAs): scale writers.  Each moves the stage's scale tiles from
+//    shared memory into a per-stage slot of its own sub-partition's tensor memory
+//    with tcgen05.st and arrives on the leader's `full` barrier of the stage, which
+//    therefore completes only when operands and scales of both CTAs are in place.
+//    Writing scales from registers keeps them out of the tensor core's instruction
+//    stream; tcgen05.cp copies there serialise with the MMAs and cost more than
+//    the MMAs themselves.
+//  * warp 1, lane 0 (leader): one barrier wait per stage, then the LoRA MMAs
+//    (kind::f16) or 4 NVFP4 MMAs, committed to both CTAs' `empty` barriers.
+//  * warps 6-21 (both CTAs): epilogue, four warps per tensor-memory sub-partition,
+//    64 columns each.  A warp loads its 32 x 64 block of the accumulator into
+//    registers and releases the accumulator at once, so the pair's next tile starts
+//    while the warp adds the residual (prefetched by TMA into the warp's 4 KiB
+//    shared-memory slab), rounds to BF16 into the slab and writes it with one TMA
+//    store, which also clips the ragged edges of the output.
 #include "common.cuh"
 
 namespace pact {
 namespace gemm {
 
-constexpr int BM = 128;             // rows per tile (MMA M)
-constexpr int BN = 256;             // columns per tile (MMA N)
-constexpr int BK = 256;             // FP4 elements per stage = 128 bytes per row
-constexpr int KSTEP = 64;           // FP4 elements per MMA
+constexpr int BM = 128;               // rows per CTA; the pair tile has 256
+constexpr int BN = 256;               // columns of the pair tile; each CTA loads 128 rows of B
+constexpr int BK = 256;               // FP4 elements per stage = 128 bytes per row
+constexpr int KSTEP = 64;             // FP4 elements per MMA
 constexpr int STAGES = 4;
-constexpr int A_BYTES = BM * BK / 2;        // 16384
-constexpr int B_BYTES = BN * BK / 2;        // 32768
-constexpr int SFA_BYTES = BM * BK / 16;     // 2048: 4 chunks of 512
-constexpr int SFB_BYTES = BN * BK / 16;     // 4096: 2 row groups x 4 chunks
+constexpr int A_BYTES = BM * BK / 2;          // 16384
+constexpr int B_BYTES = (BN / 2) * BK / 2;    // 16384
 constexpr int OFF_B = A_BYTES;
-constexpr int OFF_SFA = OFF_B + B_BYTES;
-constexpr int OFF_SFB = OFF_SFA + SFA_BYTES;
-constexpr int STAGE_BYTES = OFF_SFB + SFB_BYTES;  // 55296, a multiple of 1024
-// A LoRA stage holds up to 6 activation chunks (4 KB) and then the weight tile.
-constexpr int OFF_LW = 6 * BM * 32;               // 24576
-static_assert(OFF_LW + 3 * BN * 32 <= STAGE_BYTES && OFF_LW + 4 * 48 * 128 <= STAGE_BYTES, "LoRA stage");
-constexpr int BAR_BYTES = 256;
-constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + BAR_BYTES;
-constexpr int THREADS = 192;
+constexpr int OFF_SFA = OFF_B + B_BYTES;      // 4 chunks of 512 (this CTA's rows)
+constexpr int OFF_SFB = OFF_SFA + 2048;       // 2 row groups x 4 chunks (all 256 columns)
+constexpr int SF_BYTES = 2048 + 4096;
+constexpr int STAGE_BYTES = OFF_SFB + 4096;   // 38912 = 38 KiB
+constexpr int OFF_LW = 6 * BM * 32;           // LoRA weight chunks follow 6 activation chunks
+static_assert(OFF_LW + 3 * BM * 32 <= STAGE_BYTES && OFF_LW + 2 * 48 * 128 <= STAGE_BYTES, "LoRA stage");
+constexpr int SCALE_WARPS = 4;
+constexpr int EPI_WARPS = 16;
+constexpr int SLAB_BYTES = 32 * 128;          // 32 rows x 64 BF16 columns, 128-byte swizzle
+constexpr int OFF_SLABS = STAGES * STAGE_BYTES;
+constexpr int OFF_BARS = OFF_SLABS + EPI_WARPS * SLAB_BYTES;
+constexpr int SMEM_BYTES = 1024 + OFF_BARS + 512;
+constexpr int THREADS = 32 * (2 + SCALE_WARPS + EPI_WARPS);  // 704
+static_assert(SMEM_BYTES <= 232448, "shared memory");
 
 // tensor memory columns
 constexpr uint32_t TMEM_COLS = 512;
-constexpr uint32_t COL_ACC = 0;     // 256 FP32 columns
-constexpr uint32_t COL_SFA = 256;   // 4 columns per MMA x 4 MMAs
-constexpr uint32_t COL_SFB = 272;   // 8 columns per MMA x 4 MMAs
+constexpr uint32_t COL_ACC = 0;        // 256 FP32 columns
+constexpr uint32_t COL_SF = 256;       // per stage: 16 columns of A scales, then 32 of B scales
+constexpr uint32_t SF_COLS = 48;
+static_assert(COL_SF + STAGES * SF_COLS <= TMEM_COLS, "tensor memory");
 
 enum LoraMode : int { LORA_NONE = 0, LORA_FWD = 1, LORA_DGRAD = 2 };
 
 struct Params {
     int M, N, K;
-    const uint8_t *sfa;   // scales of A (rows M, cols K)
-    const uint8_t *sfb;   // scales of B (rows N, cols K)
-    __nv_bfloat16 *out;
-    int64_t ldo;
-    const __nv_bfloat16 *res;   // optional residual added in the epilogue (may alias out)
-    int64_t ldr;
+    int has_res;          // add the residual (map tmR; may alias the output) in the epilogue
     int lora_mode;
     int lora_steps;       // weight chunks of K = 16 per tile (two MMAs each: hi and lo activations)
     int lora_r;
@@ -66,291 +81,41 @@ struct Params {
     int64_t seg_end[4];
 };
 
-struct Tile {
-    int mt, nt;
-};
-
-__device__ __forceinline__ Tile tile_of(int t, int mtiles) { return Tile{t % mtiles, t / mtiles}; }
-
 __device__ __forceinline__ int lora_segment(const Params &p, int n0) {
     int s = 0;
-    for (int i = 0; i + 1 < p.lora_nseg; ++i) s += (n0 >= p.seg_end[i]) ? 1 : 0;
+#pragma unroll
+    for (int i = 0; i < 3; ++i) s += (i + 1 < p.lora_nseg && n0 >= p.seg_end[i]) ? 1 : 0;
     return s;
 }
 
-__global__ void __launch_bounds__(THREADS, 1)
-k_nvfp4_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-             const __grid_constant__ CUtensorMap tmLa, const __grid_constant__ CUtensorMap tmLb, const Params p) {
-    extern __shared__ uint8_t smem_raw[];
-    const uint32_t raw = smem_u32(smem_raw);
-    uint8_t *smem = smem_raw + (((raw + 1023) & ~1023u) - raw);
-    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + STAGES * STAGE_BYTES);
-    uint64_t *full = bars;                     // [STAGES]
-    uint64_t *empty = bars + STAGES;           // [STAGES]
-    uint64_t *acc_full = bars + 2 * STAGES;    // MMA -> epilogue
-    uint64_t *acc_empty = bars + 2 * STAGES + 1;  // epilogue -> MMA
-    uint64_t *drained = bars + 2 * STAGES + 2;    // MMA warp: all its tcgen05 work done
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 2 * STAGES + 3);
-    volatile uint32_t *abort_flag = tmem_slot + 1;
-
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int mtiles = (p.M + BM - 1) / BM, ntiles = (p.N + BN - 1) / BN;
-    const int ntile_total = mtiles * ntiles;
-    const int ktiles = (p.K + BK - 1) / BK;
-    const int kgroups = p.K / 64;  // scale chunks per 128-row group
-
-    if (threadIdx.x == 0) {
-        for (int s = 0; s < STAGES; ++s) {
-            mbar_init(&full[s], 1);
-            mbar_init(&empty[s], 1);
-        }
-        mbar_init(acc_full, 1);
-        mbar_init(acc_empty, 4);
-        mbar_init(drained, 1);
-        *abort_flag = 0;
-        fence_barrier_init();
+// Every stage of the ring is used in the same order by all roles: per tile, one LoRA
+// stage (when the GEMM carries a LoRA term) and then ktiles K stages.
+struct Ring {
+    uint32_t stage = 0, phase = 0;
+    __device__ __forceinline__ void next() {
+        if (++stage == STAGES) { stage = 0; phase ^= 1; }
     }
-    if (warp == 0 && lane == 0) {
-        prefetch_tensormap(&tmA);
-        prefetch_tensormap(&tmB);
-        if (p.lora_mode != LORA_NONE) {
-            prefetch_tensormap(&tmLa);
-            prefetch_tensormap(&tmLb);
-        }
-    }
-    if (warp == 1) {
-        tmem_alloc(tmem_slot, TMEM_COLS);
-        tmem_relinquish();
-    }
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
-    const uint32_t tmem = *tmem_slot;
+};
 
-    if (warp == 0) {
-        // ------------------------------------------------------------ producer
-        if (lane == 0) {
-            uint32_t stage = 0, phase = 0;
-            uint32_t pending = 0;          // stages with a load issued
-            uint32_t pending_parity = 0;   // full-barrier parity of each stage's last load
-            for (int t = blockIdx.x; t < ntile_total && !*abort_flag; t += gridDim.x) {
-                const Tile tl = tile_of(t, mtiles);
-                const int m0 = tl.mt * BM, n0 = tl.nt * BN;
-                if (p.lora_mode != LORA_NONE) {
-                    if (!mbar_wait(&empty[stage], phase ^ 1)) { *abort_flag = 1; break; }
-                    uint8_t *st = smem + stage * STAGE_BYTES;
-                    // LoRA stage: 2 * steps activation chunks (hi parts, then lo parts; 128
-                    // rows x 16 BF16 each) and the weight chunks at OFF_LW.
-                    const int R = p.lora_nseg * p.lora_r;
-                    if (p.lora_mode == LORA_FWD) {
-                        const int xs = lora_segment(p, n0) * p.lora_r;
-                        mbar_arrive_expect_tx(&full[stage], p.lora_steps * (2 * BM * 32 + BN * 32));
-                        for (int c = 0; c < p.lora_steps; ++c) {
-                            tma_load_2d(st + c * BM * 32, &tmLa, &full[stage], xs + 16 * c, m0);
-                            tma_load_2d(st + (p.lora_steps + c) * BM * 32, &tmLa, &full[stage], R + xs + 16 * c, m0);
-                            tma_load_2d(st + OFF_LW + c * BN * 32, &tmLb, &full[stage], 16 * c, n0);
-                        }
-                    } else {
-                        mbar_arrive_expect_tx(&full[stage], p.lora_steps * 2 * BM * 32 + 4 * R * 128);
-                        for (int c = 0; c < p.lora_steps; ++c) {
-                            tma_load_2d(st + c * BM * 32, &tmLa, &full[stage], 16 * c, m0);
-                            tma_load_2d(st + (p.lora_steps + c) * BM * 32, &tmLa, &full[stage], R + 16 * c, m0);
-                        }
-                        for (int q = 0; q < 4; ++q)
-                            tma_load_2d(st + OFF_LW + q * R * 128, &tmLb, &full[stage], n0 + 64 * q, 0);
-                    }
-                    pending |= 1u << stage;
-                    pending_parity = (pending_parity & ~(1u << stage)) | (phase << stage);
-                    if (++stage == STAGES) { stage = 0; phase ^= 1; }
-                }
-                const int g0 = n0 / 128;                           // first 128-row group of B
-                const int ngroups = (p.N - n0) > 128 ? 2 : 1;      // groups of B inside the padded rows
-                for (int kt = 0; kt < ktiles; ++kt) {
-                    if (!mbar_wait(&empty[stage], phase ^ 1)) { *abort_flag = 1; break; }
-                    uint8_t *st = smem + stage * STAGE_BYTES;
-                    const int nk = min(BK / KSTEP, (p.K - kt * BK) / KSTEP);
-                    mbar_arrive_expect_tx(&full[stage], A_BYTES + B_BYTES + nk * 512 * (1 + ngroups));
-                    tma_load_2d(st, &tmA, &full[stage], kt * (BK / 2), m0);
-                    tma_load_2d(st + OFF_B, &tmB, &full[stage], kt * (BK / 2), n0);
-                    bulk_load(st + OFF_SFA, p.sfa + ((size_t)tl.mt * kgroups + kt * 4) * 512, nk * 512, &full[stage]);
-                    for (int g = 0; g < ngroups; ++g)
-                        bulk_load(st + OFF_SFB + g * 2048, p.sfb + ((size_t)(g0 + g) * kgroups + kt * 4) * 512,
-                                  nk * 512, &full[stage]);
-                    pending |= 1u << stage;
-                    pending_parity = (pending_parity & ~(1u << stage)) | (phase << stage);
-                    if (++stage == STAGES) { stage = 0; phase ^= 1; }
-                }
-            }
-            // Every issued copy must land before the CTA may leave (its shared memory is
-            // the destination).  In a normal run they all have; after an abort, wait for
-            // them (bounded).
-            for (int s = 0; s < STAGES; ++s)
-                if (pending & (1u << s)) mbar_wait(&full[s], (pending_parity >> s) & 1u);
-        }
-    } else if (warp == 1) {
-        // ------------------------------------------------------------ MMA issuer
-        const uint32_t idesc = idesc_nvf4(BM, BN);
-        const uint32_t idesc_lora = idesc_bf16(BM, BN, false, p.lora_mode == LORA_DGRAD);
-        uint32_t stage = 0, phase = 0, acc_phase = 0;
-        for (int t = blockIdx.x; t < ntile_total; t += gridDim.x) {
-            bool ok = mbar_wait(acc_empty, acc_phase ^ 1);
-            tc_fence_after();
-            uint32_t accum = 0;
-            if (ok && p.lora_mode != LORA_NONE) {
-                ok = mbar_wait(&full[stage], phase);
-                tc_fence_after();
-                if (ok && lane == 0) {
-                    const uint32_t st = smem_u32(smem + stage * STAGE_BYTES);
-                    const int R = p.lora_nseg * p.lora_r;
-                    for (int c = 0; c < p.lora_steps; ++c) {
-                        const uint64_t bd = (p.lora_mode == LORA_FWD)
-                                                ? smem_desc(st + OFF_LW + c * BN * 32, 16, 256, SW_32)
-                                                : smem_desc(st + OFF_LW + c * 2048, R * 128, 1024, SW_128);
-                        for (int h = 0; h < 2; ++h) {  // hi part, then lo part
-                            const uint64_t ad = smem_desc(st + (h * p.lora_steps + c) * BM * 32, 16, 256, SW_32);
-                            mma_bf16(tmem + COL_ACC, ad, bd, idesc_lora, accum);
-                            accum = 1;
-                        }
-                    }
-                    tc_commit(&empty[stage]);
-                }
-                accum = 1;
-                __syncwarp();
-                if (++stage == STAGES) { stage = 0; phase ^= 1; }
-            }
-            for (int kt = 0; ok && kt < ktiles; ++kt) {
-                ok = mbar_wait(&full[stage], phase);
-                tc_fence_after();
-                if (ok && lane == 0) {
-                    const int nk = min(BK / KSTEP, (p.K - kt * BK) / KSTEP);
-                    const int n0 = (t / mtiles) * BN;
-                    const int ngroups = (p.N - n0) > 128 ? 2 : 1;
-                    const uint32_t st = smem_u32(smem + stage * STAGE_BYTES);
-                    for (int s = 0; s < nk; ++s) {
-                        tmem_cp_32x128b_x4(tmem + COL_SFA + 4 * s, smem_desc(st + OFF_SFA + s * 512, 0, 128, SW_NONE));
-                        for (int g = 0; g < ngroups; ++g)
-                            tmem_cp_32x128b_x4(tmem + COL_SFB + 8 * s + 4 * g,
-                                               smem_desc(st + OFF_SFB + g * 2048 + s * 512, 0, 128, SW_NONE));
-                    }
-                    for (int s = 0; s < nk; ++s) {
-                        const uint64_t ad = smem_desc(st + s * 32, 16, 1024, SW_128);
-                        const uint64_t bd = smem_desc(st + OFF_B + s * 32, 16, 1024, SW_128);
-                        mma_nvf4(tmem + COL_ACC, ad, bd, idesc, tmem + COL_SFA + 4 * s, tmem + COL_SFB + 8 * s, accum);
-                        accum = 1;
-                    }
-                    tc_commit(&empty[stage]);
-                }
-                accum = 1;
-                __syncwarp();
-                if (++stage == STAGES) { stage = 0; phase ^= 1; }
-            }
-            if (!ok) { *abort_flag = 1; break; }
-            if (lane == 0) tc_commit(acc_full);
-            __syncwarp();
-            acc_phase ^= 1;
-        }
-        // tensor memory is released below only after every MMA and copy issued here
-        // has completed
-        if (lane == 0) tc_commit(drained);
-        mbar_wait(drained, 0);
-    } else {
-        // ------------------------------------------------------------ epilogue
-        const int sub = warp & 3;  // tensor-memory sub-partition this warp may read
-        uint32_t acc_phase = 0;
-        for (int t = blockIdx.x; t < ntile_total; t += gridDim.x) {
-            const Tile tl = tile_of(t, mtiles);
-            if (!mbar_wait(acc_full, acc_phase)) { *abort_flag = 1; break; }
-            tc_fence_after();
-            const int row = tl.mt * BM + sub * 32 + lane;
-            for (int c = 0; c < BN / 32; ++c) {
-                const int n = tl.nt * BN + c * 32;
-                if (n >= p.N) break;
-                uint32_t r[32];
-                tmem_ld_32x32b_x32(tmem + ((uint32_t)(sub * 32) << 16) + COL_ACC + c * 32, r);
-                tmem_ld_wait();
-                if (row < p.M) {
-                    __nv_bfloat16 *dst = p.out + (size_t)row * p.ldo + n;
-                    uint4 *d4 = reinterpret_cast<uint4 *>(dst);
-                    const uint4 *r4 = p.res ? reinterpret_cast<const uint4 *>(p.res + (size_t)row * p.ldr + n) : nullptr;
-#pragma unroll
-                    for (int q = 0; q < 4; ++q) {
-                        float f[8];
-#pragma unroll
-                        for (int i = 0; i < 8; ++i) f[i] = __uint_as_float(r[8 * q + i]);
-                        if (r4) {
-                            const uint4 old = r4[q];
-                            f[0] += bf16lo(old.x); f[1] += bf16hi(old.x); f[2] += bf16lo(old.y); f[3] += bf16hi(old.y);
-                            f[4] += bf16lo(old.z); f[5] += bf16hi(old.z); f[6] += bf16lo(old.w); f[7] += bf16hi(old.w);
-                        }
-                        uint4 v;
-                        v.x = pack_bf16x2(f[0], f[1]); v.y = pack_bf16x2(f[2], f[3]);
-                        v.z = pack_bf16x2(f[4], f[5]); v.w = pack_bf16x2(f[6], f[7]);
-                        d4[q] = v;
-                    }
-                }
-            }
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(acc_empty);
-            acc_phase ^= 1;
-        }
-    }
-
-    tc_fence_before();
-    __syncthreads();
-    if (warp == 1) {
-        tc_fence_after();
-        tmem_dealloc(tmem, TMEM_COLS);
-    }
-}
-
-
-// ---------------------------------------------------------------------------------
-// CTA-pair variant: a cluster of 2 CTAs computes a 256 x 256 tile with 2-SM MMAs
-// (tcgen05 cta_group::2).  CTA r of the pair holds rows 128r..128r+127 of A and of
-// the accumulator, and rows 128r..128r+127 of the B tile; the MMA reads both halves
-// of A and B across the pair, so each SM streams half as much B per unit of work
-// as the single-CTA kernel.  Every scale tile arrives by TMA; the leader (rank 0)
-// arms its full barrier for both CTAs' bytes, the peer's loads complete on it, and
-// the leader issues the scale copies and MMAs for the pair and multicasts its
-// commits to both CTAs' barriers.
-// ---------------------------------------------------------------------------------
-namespace pair {
-
-constexpr int BM = 128;               // rows per CTA; the pair tile has 256
-constexpr int BN = 256;               // columns of the pair tile; each CTA loads 128 rows of B
-constexpr int BK = 256;
-constexpr int KSTEP = 64;
-constexpr int STAGES = 5;
-constexpr int A_BYTES = BM * BK / 2;          // 16384
-constexpr int B_BYTES = (BN / 2) * BK / 2;    // 16384
-constexpr int OFF_B = A_BYTES;
-constexpr int OFF_SFA = OFF_B + B_BYTES;      // 4 chunks of 512 (this CTA's rows)
-constexpr int OFF_SFB = OFF_SFA + 2048;       // 2 row groups x 4 chunks (all 256 columns)
-constexpr int STAGE_BYTES = OFF_SFB + 4096;   // 38912 = 38 KiB
-constexpr int LOAD_BYTES = STAGE_BYTES;       // bytes one CTA's loads deliver per k stage
-constexpr int OFF_LW = 6 * BM * 32;           // LoRA weight chunks follow 6 activation chunks
-constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + 256;
-constexpr int THREADS = 192;
-constexpr uint32_t TMEM_COLS = 512;
-constexpr uint32_t COL_ACC = 0, COL_SFA = 256, COL_SFB = 272;
-static_assert(OFF_LW + 3 * BM * 32 <= STAGE_BYTES && OFF_LW + 2 * 48 * 128 <= STAGE_BYTES, "LoRA stage");
+__device__ __forceinline__ bool warp_all(bool ok) { return __all_sync(0xffffffffu, ok); }
 
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
-k_nvfp4_gemm_pair(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                  const __grid_constant__ CUtensorMap tmSFA, const __grid_constant__ CUtensorMap tmSFB,
-                  const __grid_constant__ CUtensorMap tmLa, const __grid_constant__ CUtensorMap tmLb,
-                  const Params p) {
+k_nvfp4_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+             const __grid_constant__ CUtensorMap tmSFA, const __grid_constant__ CUtensorMap tmSFB,
+             const __grid_constant__ CUtensorMap tmLa, const __grid_constant__ CUtensorMap tmLb,
+             const __grid_constant__ CUtensorMap tmD, const __grid_constant__ CUtensorMap tmR, const Params p) {
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = smem_u32(smem_raw);
     uint8_t *smem = smem_raw + (((raw + 1023) & ~1023u) - raw);
-    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + STAGES * STAGE_BYTES);
-    uint64_t *full = bars;                       // [STAGES], used in the leader
-    uint64_t *empty = bars + STAGES;             // [STAGES]
-    uint64_t *acc_full = bars + 2 * STAGES;      // leader MMA -> both epilogues
-    uint64_t *acc_empty = bars + 2 * STAGES + 1; // both epilogues -> leader MMA
-    uint64_t *drained = bars + 2 * STAGES + 2;
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 2 * STAGES + 3);
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + OFF_BARS);
+    uint64_t *full = bars;                        // [STAGES] leader: operands and scales of both CTAs
+    uint64_t *sf_full = bars + STAGES;            // [STAGES] local: this CTA's scale tiles in shared memory
+    uint64_t *empty = bars + 2 * STAGES;          // [STAGES] local: the pair's MMAs are done with the stage
+    uint64_t *acc_full = bars + 3 * STAGES;       // local: accumulator complete
+    uint64_t *acc_empty = acc_full + 1;           // leader: all epilogue warps of both CTAs have read it
+    uint64_t *drained = acc_full + 2;             // leader: every tcgen05 operation has completed
+    uint64_t *res_full = acc_full + 3;            // [EPI_WARPS] local: residual block in the warp's slab
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(res_full + EPI_WARPS);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const uint32_t rank = cluster_ctarank();
@@ -360,15 +125,19 @@ k_nvfp4_gemm_pair(const __grid_constant__ CUtensorMap tmA, const __grid_constant
     const int cluster = blockIdx.x >> 1, nclusters = gridDim.x >> 1;
     const int ktiles = (p.K + BK - 1) / BK;
     const int kgroups = p.K / 64;
+    const bool lora = p.lora_mode != LORA_NONE;
+    const int nsteps = ktiles + (lora ? 1 : 0);   // ring stages per tile
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
-            mbar_init(&full[s], 1);
+            mbar_init(&full[s], 1 + 2 * SCALE_WARPS);
+            mbar_init(&sf_full[s], 1);
             mbar_init(&empty[s], 1);
         }
         mbar_init(acc_full, 1);
-        mbar_init(acc_empty, 8);
+        mbar_init(acc_empty, 2 * EPI_WARPS);
         mbar_init(drained, 1);
+        for (int w = 0; w < EPI_WARPS; ++w) mbar_init(&res_full[w], 1);
         fence_barrier_init();
     }
     if (warp == 0 && lane == 0) {
@@ -376,7 +145,9 @@ k_nvfp4_gemm_pair(const __grid_constant__ CUtensorMap tmA, const __grid_constant
         prefetch_tensormap(&tmB);
         prefetch_tensormap(&tmSFA);
         prefetch_tensormap(&tmSFB);
-        if (p.lora_mode != LORA_NONE) {
+        prefetch_tensormap(&tmD);
+        if (p.has_res) prefetch_tensormap(&tmR);
+        if (lora) {
             prefetch_tensormap(&tmLa);
             prefetch_tensormap(&tmLb);
         }
@@ -390,25 +161,24 @@ k_nvfp4_gemm_pair(const __grid_constant__ CUtensorMap tmA, const __grid_constant
     cluster_sync();  // the peer's barriers exist before anything addresses them
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-    const uint32_t full_leader = mapa_shared(smem_u32(full), 0);
-    const uint32_t acc_empty_leader = mapa_shared(smem_u32(acc_empty), 0);
 
     if (warp == 0) {
         // ------------------------------------------------------------ producer (both CTAs)
         if (lane == 0) {
-            uint32_t stage = 0, phase = 0;
+            const uint32_t full_leader = mapa_shared(smem_u32(full), 0);
+            Ring rg;
             bool ok = true;
             for (int t = cluster; ok && t < total; t += nclusters) {
                 const int mp = t % mpairs, nt = t / mpairs;
                 const int m0 = mp * 2 * BM + (int)rank * BM;     // this CTA's rows
                 const int n0 = nt * BN, nb = n0 + (int)rank * (BN / 2);
-                if (p.lora_mode != LORA_NONE) {
-                    if (!(ok = mbar_wait(&empty[stage], phase ^ 1))) break;
-                    const uint32_t st = smem_u32(smem + stage * STAGE_BYTES);
-                    const uint32_t fb = full_leader + 8 * stage;
+                if (lora) {
+                    if (!(ok = mbar_wait(&empty[rg.stage], rg.phase ^ 1))) break;
+                    const uint32_t st = smem_u32(smem + rg.stage * STAGE_BYTES);
+                    const uint32_t fb = full_leader + 8 * rg.stage;
                     const int R = p.lora_nseg * p.lora_r;
                     if (p.lora_mode == LORA_FWD) {
-                        if (leader) mbar_arrive_expect_tx(&full[stage], 2 * p.lora_steps * (2 * BM * 32 + BM * 32));
+                        if (leader) mbar_arrive_expect_tx(&full[rg.stage], 2 * p.lora_steps * (2 * BM * 32 + BM * 32));
                         const int xs = lora_segment(p, n0) * p.lora_r;
                         for (int c = 0; c < p.lora_steps; ++c) {
                             tma_load_2d_pair(st + c * BM * 32, &tmLa, fb, xs + 16 * c, m0);
@@ -416,137 +186,211 @@ k_nvfp4_gemm_pair(const __grid_constant__ CUtensorMap tmA, const __grid_constant
                             tma_load_2d_pair(st + OFF_LW + c * BM * 32, &tmLb, fb, 16 * c, nb);
                         }
                     } else {
-                        if (leader) mbar_arrive_expect_tx(&full[stage], 2 * (p.lora_steps * 2 * BM * 32 + 2 * R * 128));
+                        if (leader) mbar_arrive_expect_tx(&full[rg.stage], 2 * (p.lora_steps * 2 * BM * 32 + 2 * R * 128));
                         for (int c = 0; c < p.lora_steps; ++c) {
                             tma_load_2d_pair(st + c * BM * 32, &tmLa, fb, 16 * c, m0);
                             tma_load_2d_pair(st + (p.lora_steps + c) * BM * 32, &tmLa, fb, R + 16 * c, m0);
                         }
                         for (int q = 0; q < 2; ++q) tma_load_2d_pair(st + OFF_LW + q * R * 128, &tmLb, fb, nb + 64 * q, 0);
                     }
-                    if (++stage == STAGES) { stage = 0; phase ^= 1; }
+                    mbar_arrive(&sf_full[rg.stage]);  // a LoRA stage carries no scales
+                    rg.next();
                 }
                 const int ga = m0 / 128, gb = n0 / 128;
                 for (int kt = 0; kt < ktiles; ++kt) {
-                    if (!(ok = mbar_wait(&empty[stage], phase ^ 1))) break;
-                    const uint32_t st = smem_u32(smem + stage * STAGE_BYTES);
-                    const uint32_t fb = full_leader + 8 * stage;
-                    if (leader) mbar_arrive_expect_tx(&full[stage], 2 * LOAD_BYTES);
+                    if (!(ok = mbar_wait(&empty[rg.stage], rg.phase ^ 1))) break;
+                    uint8_t *stp = smem + rg.stage * STAGE_BYTES;
+                    const uint32_t st = smem_u32(stp);
+                    const uint32_t fb = full_leader + 8 * rg.stage;
+                    if (leader) mbar_arrive_expect_tx(&full[rg.stage], 2 * (A_BYTES + B_BYTES));
                     tma_load_2d_pair(st, &tmA, fb, kt * (BK / 2), m0);
                     tma_load_2d_pair(st + OFF_B, &tmB, fb, kt * (BK / 2), nb);
-                    // scale chunks: 512 bytes = two 256-byte rows of the scale map
-                    tma_load_2d_pair(st + OFF_SFA, &tmSFA, fb, 0, 2 * (ga * kgroups + kt * 4));
-                    tma_load_2d_pair(st + OFF_SFB, &tmSFB, fb, 0, 2 * (gb * kgroups + kt * 4));
-                    tma_load_2d_pair(st + OFF_SFB + 2048, &tmSFB, fb, 0, 2 * ((gb + 1) * kgroups + kt * 4));
-                    if (++stage == STAGES) { stage = 0; phase ^= 1; }
+                    // scale chunks: 512 bytes = two 256-byte rows of the scale map; one box
+                    // is the 4 chunks of this K stage
+                    mbar_arrive_expect_tx(&sf_full[rg.stage], SF_BYTES);
+                    tma_load_2d(stp + OFF_SFA, &tmSFA, &sf_full[rg.stage], 0, 2 * (ga * kgroups + kt * 4));
+                    tma_load_2d(stp + OFF_SFB, &tmSFB, &sf_full[rg.stage], 0, 2 * (gb * kgroups + kt * 4));
+                    tma_load_2d(stp + OFF_SFB + 2048, &tmSFB, &sf_full[rg.stage], 0,
+                                2 * ((gb + 1) * kgroups + kt * 4));
+                    rg.next();
                 }
             }
         }
     } else if (warp == 1) {
-        // ------------------------------------------------------------ MMA issuer (leader)
-        if (leader) {
+        // ------------------------------------------------------------ MMA issuer (leader, one thread)
+        if (leader && lane == 0) {
             const uint32_t idesc = idesc_nvf4(2 * BM, BN);
             const uint32_t idesc_lora = idesc_bf16(2 * BM, BN, false, p.lora_mode == LORA_DGRAD);
-            uint32_t stage = 0, phase = 0, acc_phase = 0;
-            for (int t = cluster; t < total; t += nclusters) {
-                bool ok = mbar_wait(acc_empty, acc_phase ^ 1);
+            // operand descriptors of stage 0, K step 0; a stage / K step adds its byte
+            // offset / 16 to the start-address field (addresses stay below 256 KiB)
+            const uint64_t adesc0 = smem_desc(smem_u32(smem), 16, 1024, SW_128);
+            const uint64_t bdesc0 = smem_desc(smem_u32(smem) + OFF_B, 16, 1024, SW_128);
+            Ring rg;
+            uint32_t acc_phase = 0;
+            bool ok = true;
+            for (int t = cluster; ok && t < total; t += nclusters) {
+                ok = mbar_wait(acc_empty, acc_phase ^ 1);
                 tc_fence_after();
                 uint32_t accum = 0;
-                if (ok && p.lora_mode != LORA_NONE) {
-                    ok = mbar_wait(&full[stage], phase);
+                for (int i = 0; ok && i < nsteps; ++i) {
+                    if (!(ok = mbar_wait(&full[rg.stage], rg.phase))) break;
                     tc_fence_after();
-                    if (ok && lane == 0) {
-                        const uint32_t st = smem_u32(smem + stage * STAGE_BYTES);
+                    const uint32_t st = smem_u32(smem + rg.stage * STAGE_BYTES);
+                    if (lora && i == 0) {
                         const int R = p.lora_nseg * p.lora_r;
                         for (int c = 0; c < p.lora_steps; ++c) {
                             const uint64_t bd = (p.lora_mode == LORA_FWD)
                                                     ? smem_desc(st + OFF_LW + c * BM * 32, 16, 256, SW_32)
                                                     : smem_desc(st + OFF_LW + c * 2048, R * 128, 1024, SW_128);
-                            for (int h = 0; h < 2; ++h) {
+                            for (int h = 0; h < 2; ++h) {  // hi part, then lo part
                                 const uint64_t ad = smem_desc(st + (h * p.lora_steps + c) * BM * 32, 16, 256, SW_32);
                                 mma_bf16_pair(tmem + COL_ACC, ad, bd, idesc_lora, accum);
                                 accum = 1;
                             }
                         }
-                        tc_commit_pair(&empty[stage], 3);
-                    }
-                    accum = 1;
-                    __syncwarp();
-                    if (++stage == STAGES) { stage = 0; phase ^= 1; }
-                }
-                for (int kt = 0; ok && kt < ktiles; ++kt) {
-                    ok = mbar_wait(&full[stage], phase);
-                    tc_fence_after();
-                    if (ok && lane == 0) {
+                    } else {
+                        const int kt = i - (lora ? 1 : 0);
                         const int nk = min(BK / KSTEP, (p.K - kt * BK) / KSTEP);
-                        const uint32_t st = smem_u32(smem + stage * STAGE_BYTES);
-                        for (int s = 0; s < nk; ++s) {
-                            tmem_cp_pair_32x128b_x4(tmem + COL_SFA + 4 * s,
-                                                    smem_desc(st + OFF_SFA + s * 512, 0, 128, SW_NONE));
-                            for (int g = 0; g < 2; ++g)
-                                tmem_cp_pair_32x128b_x4(tmem + COL_SFB + 8 * s + 4 * g,
-                                                        smem_desc(st + OFF_SFB + g * 2048 + s * 512, 0, 128, SW_NONE));
+                        const uint32_t sf = tmem + COL_SF + rg.stage * SF_COLS;
+                        const uint64_t ad = adesc0 + (uint64_t)((rg.stage * STAGE_BYTES) >> 4);
+                        const uint64_t bd = bdesc0 + (uint64_t)((rg.stage * STAGE_BYTES) >> 4);
+                        if (nk == BK / KSTEP) {
+#pragma unroll
+                            for (int s = 0; s < BK / KSTEP; ++s) {
+                                mma_nvf4_pair(tmem + COL_ACC, ad + 2 * s, bd + 2 * s, idesc, sf + 4 * s, sf + 16 + 8 * s,
+                                              accum);
+                                accum = 1;
+                            }
+                        } else {
+                            for (int s = 0; s < nk; ++s) {
+                                mma_nvf4_pair(tmem + COL_ACC, ad + 2 * s, bd + 2 * s, idesc, sf + 4 * s, sf + 16 + 8 * s,
+                                              accum);
+                                accum = 1;
+                            }
                         }
-                        for (int s = 0; s < nk; ++s) {
-                            const uint64_t ad = smem_desc(st + s * 32, 16, 1024, SW_128);
-                            const uint64_t bd = smem_desc(st + OFF_B + s * 32, 16, 1024, SW_128);
-                            mma_nvf4_pair(tmem + COL_ACC, ad, bd, idesc, tmem + COL_SFA + 4 * s, tmem + COL_SFB + 8 * s,
-                                          accum);
-                            accum = 1;
-                        }
-                        tc_commit_pair(&empty[stage], 3);
                     }
-                    accum = 1;
-                    __syncwarp();
-                    if (++stage == STAGES) { stage = 0; phase ^= 1; }
+                    tc_commit_pair(&empty[rg.stage], 3);
+                    rg.next();
                 }
                 if (!ok) break;
-                if (lane == 0) tc_commit_pair(acc_full, 3);
-                __syncwarp();
+                tc_commit_pair(acc_full, 3);
                 acc_phase ^= 1;
             }
-            if (lane == 0) tc_commit_pair(drained, 1);
+            // tensor memory is released below only after every MMA issued here has completed
+            tc_commit_pair(drained, 1);
             mbar_wait(drained, 0);
+        }
+        __syncwarp();
+    } else if (warp < 2 + SCALE_WARPS) {
+        // ------------------------------------------------------------ scale writers (both CTAs)
+        const int sub = warp & 3;  // tensor-memory sub-partition this warp may access
+        const uint32_t full_leader = mapa_shared(smem_u32(full), 0);
+        const uint32_t lane_base = tmem + ((uint32_t)(sub * 32) << 16);
+        Ring rg;
+        bool ok = true;
+        for (int t = cluster; ok && t < total; t += nclusters) {
+            for (int i = 0; i < nsteps; ++i) {
+                if (!(ok = warp_all(mbar_wait(&sf_full[rg.stage], rg.phase)))) break;
+                if (!(lora && i == 0)) {
+                    // Lane j takes the 16 bytes of row j of every 512-byte chunk: the
+                    // chunk's 4 scale columns for lanes j of each sub-partition, the
+                    // layout the block-scaled MMA reads.
+                    const uint8_t *src = smem + rg.stage * STAGE_BYTES + OFF_SFA + lane * 16;
+                    uint32_t v[48];
+#pragma unroll
+                    for (int c = 0; c < 12; ++c) {  // A chunks 0-3, then B: step s, group g at 4 + 2s + g
+                        const int off = c < 4 ? c * 512 : 2048 + ((c - 4) & 1) * 2048 + ((c - 4) >> 1) * 512;
+                        const uint4 q = *reinterpret_cast<const uint4 *>(src + off);
+                        v[4 * c] = q.x; v[4 * c + 1] = q.y; v[4 * c + 2] = q.z; v[4 * c + 3] = q.w;
+                    }
+                    const uint32_t col = lane_base + COL_SF + rg.stage * SF_COLS;
+                    tmem_st_32x32b_x32(col, v);
+                    tmem_st_32x32b_x16(col + 32, v + 32);
+                    tmem_st_wait();
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive_remote_relaxed(full_leader + 8 * rg.stage);
+                rg.next();
+            }
         }
     } else {
         // ------------------------------------------------------------ epilogue (both CTAs)
-        const int sub = warp & 3;
-        uint32_t acc_phase = 0;
-        for (int t = cluster; t < total; t += nclusters) {
-            const int mp = t % mpairs, nt = t / mpairs;
-            if (!mbar_wait(acc_full, acc_phase)) break;
+        const int ew = warp - 2 - SCALE_WARPS;   // 0..15
+        const int sub = warp & 3;                // tensor-memory sub-partition this warp may read
+        const int quarter = ew >> 2;             // columns 64*quarter .. 64*quarter+63 of the tile
+        const uint32_t acc_empty_leader = mapa_shared(smem_u32(acc_empty), 0);
+        const uint32_t taddr = tmem + ((uint32_t)(sub * 32) << 16) + COL_ACC + quarter * 64;
+        uint8_t *slab_p = smem + OFF_SLABS + ew * SLAB_BYTES;
+        const uint32_t slab = smem_u32(slab_p);
+        // this warp's 32 x 64 block of tile t: first row and column
+        auto block_y = [&](int t) { return (t % mpairs) * 2 * BM + (int)rank * BM + sub * 32; };
+        auto block_x = [&](int t) { return (t / mpairs) * BN + quarter * 64; };
+        auto inside = [&](int t) { return block_y(t) < p.M && block_x(t) < p.N; };
+        auto load_residual = [&](int t) {  // lane 0; the slab is free
+            mbar_arrive_expect_tx(&res_full[ew], SLAB_BYTES);
+            tma_load_2d(slab_p, &tmR, &res_full[ew], block_x(t), block_y(t));
+        };
+        uint32_t acc_phase = 0, res_phase = 0;
+        if (p.has_res && lane == 0 && cluster < total && inside(cluster)) load_residual(cluster);
+        bool ok = true;
+        for (int t = cluster; ok && t < total; t += nclusters) {
+            bool got = false;
+            if (lane == 0) got = mbar_wait_sleep(acc_full, acc_phase);
+            if (!(ok = __shfl_sync(0xffffffffu, got, 0))) break;
             tc_fence_after();
-            const int row = mp * 2 * BM + (int)rank * BM + sub * 32 + lane;
-            for (int c = 0; c < BN / 32; ++c) {
-                const int n = nt * BN + c * 32;
-                if (n >= p.N) break;
-                uint32_t r[32];
-                tmem_ld_32x32b_x32(tmem + ((uint32_t)(sub * 32) << 16) + COL_ACC + c * 32, r);
-                tmem_ld_wait();
-                if (row < p.M) {
-                    uint4 *d4 = reinterpret_cast<uint4 *>(p.out + (size_t)row * p.ldo + n);
-                    const uint4 *r4 = p.res ? reinterpret_cast<const uint4 *>(p.res + (size_t)row * p.ldr + n) : nullptr;
-#pragma unroll
-                    for (int q = 0; q < 4; ++q) {
-                        float f[8];
-#pragma unroll
-                        for (int i = 0; i < 8; ++i) f[i] = __uint_as_float(r[8 * q + i]);
-                        if (r4) {
-                            const uint4 old = r4[q];
-                            f[0] += bf16lo(old.x); f[1] += bf16hi(old.x); f[2] += bf16lo(old.y); f[3] += bf16hi(old.y);
-                            f[4] += bf16lo(old.z); f[5] += bf16hi(old.z); f[6] += bf16lo(old.w); f[7] += bf16hi(old.w);
-                        }
-                        uint4 v;
-                        v.x = pack_bf16x2(f[0], f[1]); v.y = pack_bf16x2(f[2], f[3]);
-                        v.z = pack_bf16x2(f[4], f[5]); v.w = pack_bf16x2(f[6], f[7]);
-                        d4[q] = v;
-                    }
-                }
-            }
+            uint32_t r[64];
+            tmem_ld_32x32b_x32(taddr, *reinterpret_cast<uint32_t(*)[32]>(r));
+            tmem_ld_32x32b_x32(taddr + 32, *reinterpret_cast<uint32_t(*)[32]>(r + 32));
+            tmem_ld_wait();
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive_remote(acc_empty_leader);
+            if (lane == 0) mbar_arrive_remote_relaxed(acc_empty_leader);  // the pair may reuse the accumulator
             acc_phase ^= 1;
+            if (inside(t)) {
+                if (p.has_res) {
+                    if (lane == 0) got = mbar_wait_sleep(&res_full[ew], res_phase);
+                    if (!(ok = __shfl_sync(0xffffffffu, got, 0))) break;
+                    res_phase ^= 1;
+                } else {
+                    if (lane == 0) bulk_wait_read_all();  // the previous block's store has read the slab
+                    __syncwarp();
+                }
+                // row `lane` of the block: 8 pieces of 16 bytes, 128-byte swizzle
+#pragma unroll
+                for (int q = 0; q < 8; ++q) {
+                    const uint32_t a = slab + lane * 128 + ((q ^ (lane & 7)) << 4);
+                    float f[8];
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) f[i] = __uint_as_float(r[8 * q + i]);
+                    if (p.has_res) {
+                        uint32_t o0, o1, o2, o3;
+                        asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                                     : "=r"(o0), "=r"(o1), "=r"(o2), "=r"(o3)
+                                     : "r"(a));
+                        f[0] += bf16lo(o0); f[1] += bf16hi(o0); f[2] += bf16lo(o1); f[3] += bf16hi(o1);
+                        f[4] += bf16lo(o2); f[5] += bf16hi(o2); f[6] += bf16lo(o3); f[7] += bf16hi(o3);
+                    }
+                    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(a), "r"(pack_bf16x2(f[0], f[1])),
+                                 "r"(pack_bf16x2(f[2], f[3])), "r"(pack_bf16x2(f[4], f[5])),
+                                 "r"(pack_bf16x2(f[6], f[7]))
+                                 : "memory");
+                }
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) {
+                    tma_store_2d(&tmD, slab, block_x(t), block_y(t));
+                    bulk_commit_group();
+                }
+            }
+            if (lane == 0 && p.has_res && t + nclusters < total && inside(t + nclusters)) {
+                bulk_wait_read_all();
+                load_residual(t + nclusters);
+            }
+            __syncwarp();
         }
+        if (lane == 0) bulk_wait_all();
+        __syncwarp();
     }
 
     tc_fence_before();
@@ -558,8 +402,6 @@ k_nvfp4_gemm_pair(const __grid_constant__ CUtensorMap tmA, const __grid_constant
     }
     cluster_sync();
 }
-
-}  // namespace pair
 
 // ------------------------------------------------------------------ host side
 typedef CUresult (*EncodeTiled)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
@@ -601,7 +443,7 @@ static pact_status ensure_attrs() {
     const int d = current_device();
     if (d >= 0 && d < 64 && done[d]) return PACT_OK;
     cudaError_t e =
-        cudaFuncSetAttribute(pair::k_nvfp4_gemm_pair, cudaFuncAttributeMaxDynamicSharedMemorySize, pair::SMEM_BYTES);
+        cudaFuncSetAttribute(k_nvfp4_gemm, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
     if (e != cudaSuccess) return fail(PACT_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));
     if (d >= 0 && d < 64) done[d] = true;
     return PACT_OK;
@@ -648,7 +490,7 @@ static pact_status run(const pact_nvfp4_t *a, const pact_nvfp4_t *b, const pact_
     if (s != PACT_OK) return s;
     s = ensure_attrs();
     if (s != PACT_OK) return s;
-    CUtensorMap tmA, tmB, tmSFA, tmSFB, tmLa, tmLb;
+    CUtensorMap tmA, tmB, tmSFA, tmSFB, tmLa, tmLb, tmD, tmR;
     // operand tiles: 128 rows x 128 bytes (256 FP4 values), 128-byte swizzle
     s = make_map(&tmA, CU_TENSOR_MAP_DATA_TYPE_UINT8, a->codes, K / 2, M, K / 2, 128, 128,
                  CU_TENSOR_MAP_SWIZZLE_128B, what);
@@ -664,15 +506,18 @@ static pact_status run(const pact_nvfp4_t *a, const pact_nvfp4_t *b, const pact_
     if (s == PACT_OK)
         s = make_map(&tmSFB, CU_TENSOR_MAP_DATA_TYPE_UINT8, b->scales, 256, 2 * chunks_b, 256, 256, 8,
                      CU_TENSOR_MAP_SWIZZLE_NONE, what);
+    // output (and residual) blocks: 32 rows x 64 BF16 columns, 128-byte swizzle
+    if (s == PACT_OK)
+        s = make_map(&tmD, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, out, N, M, ldo * 2, 64, 32, CU_TENSOR_MAP_SWIZZLE_128B,
+                     what);
+    tmR = tmD;
+    if (s == PACT_OK && res)
+        s = make_map(&tmR, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, res, N, M, ldr * 2, 64, 32, CU_TENSOR_MAP_SWIZZLE_128B,
+                     what);
     if (s != PACT_OK) return s;
     Params p;
     p.M = (int)M; p.N = (int)N; p.K = (int)K;
-    p.sfa = static_cast<const uint8_t *>(a->scales);
-    p.sfb = static_cast<const uint8_t *>(b->scales);
-    p.out = reinterpret_cast<__nv_bfloat16 *>(out);
-    p.ldo = ldo;
-    p.res = reinterpret_cast<const __nv_bfloat16 *>(res);
-    p.ldr = ldr;
+    p.has_res = res != nullptr;
     p.lora_mode = LORA_NONE;
     p.lora_steps = 0; p.lora_r = 0; p.lora_nseg = 1;
     for (int i = 0; i < 4; ++i) p.seg_end[i] = N;
@@ -701,8 +546,7 @@ static pact_status run(const pact_nvfp4_t *a, const pact_nvfp4_t *b, const pact_
     }
     const int pairs = (int)(((M + 255) / 256) * ((N + 255) / 256));
     const int clusters = pairs < sm_count() / 2 ? pairs : sm_count() / 2;
-    pair::k_nvfp4_gemm_pair<<<2 * clusters, pair::THREADS, pair::SMEM_BYTES, stream>>>(tmA, tmB, tmSFA, tmSFB, tmLa,
-                                                                                        tmLb, p);
+    k_nvfp4_gemm<<<2 * clusters, THREADS, SMEM_BYTES, stream>>>(tmA, tmB, tmSFA, tmSFB, tmLa, tmLb, tmD, tmR, p);
     return launch_status(what);
 }
 
