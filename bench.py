@@ -52,6 +52,9 @@ def parse():
                     help="NVFP4 GEMM shape sweep (N x K x M, forward and dgrad): one JSON line per shape")
     ap.add_argument("--gemm", type=int, nargs=3, metavar=("N", "K", "M"),
                     help="time one NVFP4 GEMM shape (forward and dgrad) instead of the layer step")
+    ap.add_argument("--ops", action="store_true",
+                    help="time each op of the layer step alone: one JSON line per op with its roofline")
+    ap.add_argument("--only", default=None, help="with --ops: time only the ops whose name contains this")
     return ap.parse_args()
 
 
@@ -178,13 +181,89 @@ def config_block(name, M):
     return {"workload": f"{name} decoder layer fwd+bwd: 7 NVFP4 frozen projections + LoRA",
             "H": c["H"], "I": c["I"], "kv": c["KV"], "tokens": M, "batch": c["batch"], "seq": c["seq"],
             "lora_r": synth.LORA_R, "lora_alpha": synth.LORA_ALPHA,
-            "l2": "flushed between timed steps (256 MiB write)", "launch": "per-segment CUDA graphs"}
+            "l2": "flushed between timed steps (256 MiB write)", "launch": "one CUDA graph per step"}
 
 
 # ------------------------------------------------------------------ GPU arm
+def make_layer(name, dev):
+    """The layer of workload `name` on device `dev` with its seeded synthetic inputs bound."""
+    import torch
+    import synth
+    from nvfp4_gemm_b200.layer import LayerShape, PactLayer
+    c = synth.LAYERS[name]
+    M = synth.tokens(name)
+    inputs = synth.layer_inputs(name)
+    d = lambda bits: torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).to(dev)
+    shape = LayerShape(M=M, H=c["H"], I=c["I"], KV=c["KV"], r=synth.LORA_R, alpha=synth.LORA_ALPHA,
+                       eps=synth.RMS_EPS)
+    layer = PactLayer(shape, {k: d(v) for k, v in inputs["w"].items()},
+                      {k: d(v) for k, v in inputs["lora_a"].items()},
+                      {k: d(v) for k, v in inputs["lora_b"].items()}, d(inputs["gamma1"]), d(inputs["gamma2"]))
+    x_in = {k: d(inputs[k]) for k in ("h", "attn", "d_out", "d_qkv")}
+    layer.bind(x_in["h"], x_in["attn"], x_in["d_out"], x_in["d_qkv"])
+    return inputs, layer, x_in
+
+
+def device_ms(fn, stream, flush, reps=8, samples=5):
+    """Device time of one call of `fn` with a cold L2 and without launch overhead:
+    (graph of reps x [flush, fn] - graph of reps x [flush]) / reps, each graph timed
+    `samples` times with CUDA events on `stream`."""
+    import torch
+    graphs = []
+    for with_op in (True, False):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            for _ in range(reps):
+                flush.zero_()
+                if with_op:
+                    fn()
+        graphs.append(g)
+    out = []
+    with torch.cuda.stream(stream):
+        for g in graphs:
+            g.replay()
+            tt = []
+            for _ in range(samples):
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record(stream)
+                g.replay()
+                e1.record(stream)
+                tt.append((e0, e1))
+            torch.cuda.synchronize()
+            out.append(sum(x.elapsed_time(y) for x, y in tt) / samples)
+    return max(out[0] - out[1], 1e-6) / reps
+
+
+def op_table(a, layer, dev):
+    """Each op of the step alone (device time per call, cold L2, no launch overhead),
+    its algorithmic bytes / FLOPs and the fraction of the measured peak."""
+    import torch
+    import nvfp4_gemm_b200 as P
+    pk = peaks()
+    stream = torch.cuda.Stream(device=dev)
+    with torch.cuda.stream(stream):
+        layer.step()          # every op once: per-device attributes, lazy init
+    torch.cuda.synchronize()
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    for op in layer.step_ops():
+        if a.only and a.only not in op.name:
+            continue
+        ms = device_ms(op.fn, stream, flush, reps=8, samples=max(3, a.steps))
+        row = {"op": op.name, "kind": op.kind, "kernels": op.kernels, "us": round(ms * 1e3, 2),
+               "bytes": op.bytes, "GBps": round(op.bytes / (ms / 1e3) / 1e9, 1),
+               "frac_hbm": round(op.bytes / (ms / 1e3) / 1e9 / pk["hbm_gbs"], 3)}
+        if op.kind == "gemm":
+            tf = op.flops / (ms / 1e3) / 1e12
+            row.update({"tflops": round(tf, 1), "frac_fp4_peak": round(tf / (FP4_PER_BF16 * pk["bf16"]), 3)})
+        print(json.dumps(row), flush=True)
+    if P.pact_get_device_status() != 0:
+        raise RuntimeError(P.pact_last_error())
+
+
 def gemm_sweep(a, shapes):
     """Time NVFP4 frozen GEMMs (forward Y = X W^T and dgrad dX = dY W) per shape;
-    inputs X, dY ~ N(0, 1), W ~ N(0, 0.02^2); L2 flushed before every launch."""
+    inputs X, dY ~ N(0, 1), W ~ N(0, 0.02^2); device time per launch with a cold L2
+    and without launch overhead."""
     import torch
     import synth
     import nvfp4_gemm_b200 as P
@@ -193,7 +272,7 @@ def gemm_sweep(a, shapes):
     d = lambda bits: torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).to(dev)
     pk = peaks()
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
-    ev = lambda: torch.cuda.Event(enable_timing=True)
+    stream = torch.cuda.Stream(device=dev)
     for N, K, M in shapes:
         w = d(synth.weight_bf16(0, (N, K)))
         wc = P.pact_weight_layout_cache(w)
@@ -206,25 +285,9 @@ def gemm_sweep(a, shapes):
                          ("dgrad", lambda: P.pact_frozen_gemm_dgrad(dyq, wc, dx=dx))):
             for _ in range(max(3, a.warmup)):
                 fn()
-            # one launch per CUDA graph, so the events time the kernel and not the
-            # host-side argument checks and tensor-map encoding
-            g = torch.cuda.CUDAGraph()
-            with torch.cuda.graph(g):
-                fn()
-            g.replay()
-            times = []
-            for _ in range(a.steps):
-                flush.zero_()
-                e0, e1 = ev(), ev()
-                e0.record()
-                g.replay()
-                e1.record()
-                times.append((e0, e1))
-            torch.cuda.synchronize()
-            ms = sorted(s_.elapsed_time(e_) for s_, e_ in times)
-            med = ms[len(ms) // 2]
+            med = device_ms(fn, stream, flush, reps=8, samples=max(3, a.steps))
             tf = 2.0 * M * N * K / (med / 1e3) / 1e12
-            res[kind] = {"median_ms": med, "tflops": tf, "frac_fp4_peak": tf / (FP4_PER_BF16 * pk["bf16"])}
+            res[kind] = {"ms": med, "tflops": tf, "frac_fp4_peak": tf / (FP4_PER_BF16 * pk["bf16"])}
         if P.pact_get_device_status() != 0:
             raise RuntimeError(P.pact_last_error())
         print(json.dumps({"gemm": {"N": N, "K": K, "M": M}, **res,
@@ -248,7 +311,6 @@ def main():
 
     import synth
     import nvfp4_gemm_b200 as P
-    from nvfp4_gemm_b200.layer import LayerShape, PactLayer
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -259,17 +321,10 @@ def main():
         import datetime
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
 
-    c = synth.LAYERS[a.workload]
     M = synth.tokens(a.workload)
-    inputs = synth.layer_inputs(a.workload)
-    d = lambda bits: torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).to(dev)
-    shape = LayerShape(M=M, H=c["H"], I=c["I"], KV=c["KV"], r=synth.LORA_R, alpha=synth.LORA_ALPHA,
-                       eps=synth.RMS_EPS)
-    layer = PactLayer(shape, {k: d(v) for k, v in inputs["w"].items()},
-                      {k: d(v) for k, v in inputs["lora_a"].items()},
-                      {k: d(v) for k, v in inputs["lora_b"].items()}, d(inputs["gamma1"]), d(inputs["gamma2"]))
-    x_in = {k: d(inputs[k]) for k in ("h", "attn", "d_out", "d_qkv")}
-    layer.bind(x_in["h"], x_in["attn"], x_in["d_out"], x_in["d_qkv"])
+    inputs, layer, x_in = make_layer(a.workload, dev)
+    if a.ops:
+        return op_table(a, layer, dev)
     ops = layer.step_ops()
     launches_per_step = sum(op.kernels for op in ops)
 
@@ -288,6 +343,12 @@ def main():
     torch.cuda.synchronize()
     if P.pact_get_device_status() != 0:
         raise RuntimeError(P.pact_last_error())
+    # the timed step: every op of the step in one CUDA graph (kernels back to back);
+    # per-segment graphs give the breakdown in a separate pass after the timed region
+    step_graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(step_graph, stream=stream):
+        for op in ops:
+            op.fn()
     for sg in segs:
         g = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g, stream=stream):
@@ -297,8 +358,7 @@ def main():
     torch.cuda.synchronize()
 
     def run_step():
-        for sg in segs:
-            sg["graph"].replay()
+        step_graph.replay()
 
     grads = list(layer.grads.values())
 
@@ -318,7 +378,6 @@ def main():
     K = a.steps
     ev = lambda: torch.cuda.Event(enable_timing=True)
     st_ev = [(ev(), ev()) for _ in range(K)]
-    seg_ev = [[(ev(), ev()) for _ in segs] for _ in range(K)]
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
@@ -328,10 +387,7 @@ def main():
             for k in range(K):
                 flush.zero_()
                 st_ev[k][0].record(stream)
-                for i, sg in enumerate(segs):
-                    seg_ev[k][i][0].record(stream)
-                    sg["graph"].replay()
-                    seg_ev[k][i][1].record(stream)
+                run_step()
                 allreduce_grads()
                 st_ev[k][1].record(stream)
         torch.cuda.synchronize()
@@ -340,6 +396,16 @@ def main():
         dist.barrier()
     step_ms = [s.elapsed_time(e) for s, e in st_ev]
     total_ms = sum(step_ms)
+    # breakdown (not the timed number): each segment's graph alone, after a flush
+    seg_ev = [[(ev(), ev()) for _ in segs] for _ in range(K)]
+    with torch.cuda.stream(stream):
+        for k in range(K):
+            for i, sg in enumerate(segs):
+                flush.zero_()
+                seg_ev[k][i][0].record(stream)
+                sg["graph"].replay()
+                seg_ev[k][i][1].record(stream)
+    torch.cuda.synchronize()
     seg_ms = [sum(seg_ev[k][i][0].elapsed_time(seg_ev[k][i][1]) for k in range(K)) / K for i in range(len(segs))]
     if world > 1:
         t = torch.tensor([total_ms], device=dev)
@@ -348,12 +414,14 @@ def main():
     ms_per_step = total_ms / K
     tokens_per_s = M * K * world / (total_ms / 1e3)
 
-    gemm_flops = sum(sg["flops"] for sg in segs if sg["kind"] == "gemm")
-    gemm_ms = sum(t for t, sg in zip(seg_ms, segs) if sg["kind"] == "gemm")
-    gemm_launch_ms = gemm_ms / sum(1 for sg in segs if sg["kind"] == "gemm")
+    # the dominant kernel (the NVFP4 GEMM): device time per launch, cold L2, no launch overhead
+    gemm_ops = [op for op in ops if op.kind == "gemm"]
+    gemm_flops = sum(op.flops for op in gemm_ops)
+    gemm_ms = sum(device_ms(op.fn, stream, flush) for op in gemm_ops)
+    gemm_launch_ms = gemm_ms / len(gemm_ops)
     tflops = gemm_flops / (gemm_ms / 1e3) / 1e12
     pk = peaks()
-    fp4_peak = FP4_PER_BF16 * pk["bf16_sustained"]
+    fp4_peak = FP4_PER_BF16 * pk["bf16"]   # the GEMM is timed alone: burst peak
 
     # end to end: inputs from pinned host memory, LoRA gradients back to pinned host memory
     host_in = {k: x_in[k].cpu().pin_memory() for k in x_in}
@@ -401,8 +469,8 @@ def main():
             "roofline": {"bound": "tensor", "kernel": "k_nvfp4_gemm (frozen fwd + dgrad GEMMs)",
                          "achieved": tflops, "peak": fp4_peak, "unit": "TFLOP/s", "frac": tflops / fp4_peak,
                          "traffic": None,
-                         "peak_note": f"{pk['src']} sustained BF16 {pk['bf16_sustained']} TF/s x {FP4_PER_BF16} "
-                                      f"(nominal FP4/BF16 ratio)",
+                         "peak_note": f"{pk['src']} burst BF16 {pk['bf16']} TF/s x {FP4_PER_BF16} "
+                                      f"(nominal FP4/BF16 ratio); GEMM launches timed alone, cold L2",
                          "flops_per_step": gemm_flops, "avg_launch_ms": gemm_launch_ms},
             "cpu_baseline": cpu,
             "e2e": {"value": M * K * world / (e2e_ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
@@ -414,6 +482,7 @@ def main():
         print(json.dumps(out), flush=True)
     for sg in segs:
         sg["graph"] = None
+    step_graph = None
     if world > 1:
         dist.destroy_process_group()
 

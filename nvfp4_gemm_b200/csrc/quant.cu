@@ -25,12 +25,11 @@ __global__ void __launch_bounds__(256) k_quantize(const pact_bf16 *__restrict__ 
     const int lane = threadIdx.x & 31;
     const int64_t nchunk = (out.cols + CHUNK - 1) / CHUNK;
     const int64_t rows_pad = (rows + 127) & ~int64_t(127);
-    const int64_t ntask = rows_pad * nchunk;
     const int64_t warp0 = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
     const int64_t nwarps = (int64_t)gridDim.x * (blockDim.x >> 5);
-    for (int64_t task = warp0; task < ntask; task += nwarps) {
-        const int64_t row = task / nchunk;
-        const int64_t c0 = (task % nchunk) * CHUNK;
+    for (TaskIter it(warp0, nchunk, nwarps); it.row < rows_pad; it.next()) {
+        const int64_t row = it.row;
+        const int64_t c0 = it.chunk * CHUNK;
         if (row >= rows) {
             zero_pad_scales(out, row, c0);
             continue;
@@ -55,15 +54,28 @@ static int grid_for(int64_t warp_tasks, int threads) {
 }
 
 // ------------------------------------------------------- A3: RMSNorm + quantize
-// One CTA (256 threads) per row; each warp owns chunks w, w+8, ... of the row and
-// keeps them in registers between the reduction and the output pass.
+// A group of WPR warps owns a row (256 / 32 / WPR rows per 256-thread CTA); warp w of
+// the group holds chunks w, w + WPR, ... of the row as packed BF16 between the
+// reduction and the output pass.  One warp per row when H <= 2048, so the row's
+// loads are all in flight at once and the reduction needs no block barrier.
 constexpr int RMS_THREADS = 256;
+constexpr int RMS_WARPS = RMS_THREADS / 32;
 constexpr int RMS_MAX_CHUNKS = 8;  // H <= 8 warps x 8 chunks x 256 = 16384
 
-// Chunks of 256 columns each warp holds for a row of H columns: 1, 2, 4 or 8.
+// Warps per row for H columns: the fewest (1, 2, 4 or 8) whose chunks fit in 8 each.
+static int rms_wpr(int64_t H) {
+    const int64_t chunks = (H + CHUNK - 1) / CHUNK;
+    return chunks <= 8 ? 1 : chunks <= 16 ? 2 : chunks <= 32 ? 4 : 8;
+}
+// Chunks each warp holds: 1, 2, 4 or 8.
 static int rms_nch(int64_t H) {
-    const int64_t per_warp = ((H + CHUNK - 1) / CHUNK + RMS_THREADS / 32 - 1) / (RMS_THREADS / 32);
+    const int64_t per_warp = ((H + CHUNK - 1) / CHUNK + rms_wpr(H) - 1) / rms_wpr(H);
     return per_warp <= 1 ? 1 : per_warp <= 2 ? 2 : per_warp <= 4 ? 4 : 8;
+}
+
+__device__ __forceinline__ void unpack8_bf16(const uint4 &u, float (&v)[8]) {
+    v[0] = bf16lo(u.x); v[1] = bf16hi(u.x); v[2] = bf16lo(u.y); v[3] = bf16hi(u.y);
+    v[4] = bf16lo(u.z); v[5] = bf16hi(u.z); v[6] = bf16lo(u.w); v[7] = bf16hi(u.w);
 }
 
 // BF16 rounding of y = (x * rstd) * gamma with one correct rounding of the double
@@ -81,53 +93,58 @@ __device__ __forceinline__ float rms_out(float x, float g, float r32, double rst
     return __bfloat162float(__float2bfloat16_rn(y));
 }
 
-template <int NCH>
-__global__ void __launch_bounds__(RMS_THREADS) k_rmsnorm_quant(const pact_bf16 *__restrict__ x, int64_t ldx,
+template <int NCH, int WPR>
+__global__ void __launch_bounds__(RMS_THREADS, 2) k_rmsnorm_quant(const pact_bf16 *__restrict__ x, int64_t ldx,
                                                                const pact_bf16 *__restrict__ gamma, float eps,
                                                                int64_t M, int64_t H, pact_nvfp4_t yq,
                                                                pact_bf16 *__restrict__ y, float *__restrict__ rstd_out) {
-    __shared__ double red[RMS_THREADS / 32];
+    __shared__ double red[RMS_WARPS];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const int64_t row = blockIdx.x;
-    const int64_t nchunk = (H + CHUNK - 1) / CHUNK;
-    if (row >= M) {  // padding rows of the scale layout
-        for (int64_t ch = warp; ch < nchunk; ch += RMS_THREADS / 32) zero_pad_scales(yq, row, ch * CHUNK);
-        return;
-    }
-    float v[NCH][8];
+    const int wr = warp % WPR;                                       // warp within the row group
+    const int64_t row = (int64_t)blockIdx.x * (RMS_WARPS / WPR) + warp / WPR;
+    const bool real = row < M;                                       // else a padding row of the scale layout
+    uint4 xv[NCH];
     double ss = 0.0;
 #pragma unroll
     for (int k = 0; k < NCH; ++k) {
-        const int64_t c = (warp + (int64_t)k * (RMS_THREADS / 32)) * CHUNK + 8 * lane;
+        const int64_t c = (wr + (int64_t)k * WPR) * CHUNK + 8 * lane;
+        xv[k] = make_uint4(0, 0, 0, 0);
+        if (real && c < H) xv[k] = *reinterpret_cast<const uint4 *>(x + row * ldx + c);
+    }
 #pragma unroll
-        for (int i = 0; i < 8; ++i) v[k][i] = 0.0f;
-        if (c < H) {
-            load8_bf16(x + row * ldx + c, v[k]);
+    for (int k = 0; k < NCH; ++k) {
+        float v[8];
+        unpack8_bf16(xv[k], v);
 #pragma unroll
-            for (int i = 0; i < 8; ++i) ss = fma((double)v[k][i], (double)v[k][i], ss);
-        }
+        for (int i = 0; i < 8; ++i) ss = fma((double)v[i], (double)v[i], ss);
     }
 #pragma unroll
     for (int o = 16; o; o >>= 1) ss += __shfl_xor_sync(0xFFFFFFFFu, ss, o);
-    if (lane == 0) red[warp] = ss;
-    __syncthreads();
-    double tot = 0.0;
+    if (WPR > 1) {
+        if (lane == 0) red[warp] = ss;
+        __syncthreads();
+        ss = 0.0;
 #pragma unroll
-    for (int w = 0; w < RMS_THREADS / 32; ++w) tot += red[w];
-    const double rstd = 1.0 / sqrt(tot / (double)H + (double)eps);
+        for (int w = 0; w < WPR; ++w) ss += red[warp - wr + w];
+    }
+    const double rstd = 1.0 / sqrt(ss / (double)H + (double)eps);
     const float r32 = (float)rstd;
-    if (threadIdx.x == 0 && rstd_out) rstd_out[row] = r32;
+    if (real && wr == 0 && lane == 0 && rstd_out) rstd_out[row] = r32;
 #pragma unroll
     for (int k = 0; k < NCH; ++k) {
-        const int64_t c0 = (warp + (int64_t)k * (RMS_THREADS / 32)) * CHUNK;
+        const int64_t c0 = (wr + (int64_t)k * WPR) * CHUNK;
         if (c0 >= H) break;  // warp-uniform
+        if (!real) {
+            zero_pad_scales(yq, row, c0);
+            continue;
+        }
         const int64_t c = c0 + 8 * lane;
         const bool valid = c < H;
-        float g[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+        float v[8], g[8] = {0, 0, 0, 0, 0, 0, 0, 0}, o[8];
+        unpack8_bf16(xv[k], v);
         if (valid) load8_bf16(gamma + c, g);
-        float o[8];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) o[i] = valid ? rms_out(v[k][i], g[i], r32, rstd) : 0.0f;
+        for (int i = 0; i < 8; ++i) o[i] = valid ? rms_out(v[i], g[i], r32, rstd) : 0.0f;
         if (valid && y) store8_bf16(y + row * H + c, o);
         uint32_t sb;
         const uint32_t codes = quant8(o, &sb);
@@ -163,12 +180,11 @@ __global__ void __launch_bounds__(256) k_silu_mul_quant(const pact_bf16 *__restr
     const int lane = threadIdx.x & 31;
     const int64_t nchunk = (I + CHUNK - 1) / CHUNK;
     const int64_t rows_pad = (M + 127) & ~int64_t(127);
-    const int64_t ntask = rows_pad * nchunk;
     const int64_t warp0 = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
     const int64_t nwarps = (int64_t)gridDim.x * (blockDim.x >> 5);
-    for (int64_t task = warp0; task < ntask; task += nwarps) {
-        const int64_t row = task / nchunk;
-        const int64_t c0 = (task % nchunk) * CHUNK;
+    for (TaskIter it(warp0, nchunk, nwarps); it.row < rows_pad; it.next()) {
+        const int64_t row = it.row;
+        const int64_t c0 = it.chunk * CHUNK;
         if (row >= M) {
             zero_pad_scales(mq, row, c0);
             if (has_gq) zero_pad_scales(gq, row, c0);
@@ -207,12 +223,11 @@ __global__ void __launch_bounds__(256) k_silu_mul_bwd_quant(const pact_bf16 *__r
     const int lane = threadIdx.x & 31;
     const int64_t nchunk = (I + CHUNK - 1) / CHUNK;
     const int64_t rows_pad = (M + 127) & ~int64_t(127);
-    const int64_t ntask = rows_pad * nchunk;
     const int64_t warp0 = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
     const int64_t nwarps = (int64_t)gridDim.x * (blockDim.x >> 5);
-    for (int64_t task = warp0; task < ntask; task += nwarps) {
-        const int64_t row = task / nchunk;
-        const int64_t c0 = (task % nchunk) * CHUNK;
+    for (TaskIter it(warp0, nchunk, nwarps); it.row < rows_pad; it.next()) {
+        const int64_t row = it.row;
+        const int64_t c0 = it.chunk * CHUNK;
         if (row >= M) {
             zero_pad_scales(dguq, row, c0);
             zero_pad_scales(dguq, row, c0 + I);
@@ -223,8 +238,12 @@ __global__ void __launch_bounds__(256) k_silu_mul_bwd_quant(const pact_bf16 *__r
         float d[8] = {0, 0, 0, 0, 0, 0, 0, 0}, gh[8] = {0, 0, 0, 0, 0, 0, 0, 0}, uh[8] = {0, 0, 0, 0, 0, 0, 0, 0};
         if (valid) {
             load8_bf16(dm + row * lddm + c, d);
-            load8_nvfp4(gq, row, c, gh);
-            load8_nvfp4(uq, row, c, uh);
+            // gq and uq share their shape: one code offset, one scale offset
+            const int64_t co = row * (I >> 1) + (c >> 1), so = scale_offset(row, c >> 4, I);
+            dequant8(*reinterpret_cast<const uint32_t *>(static_cast<const uint8_t *>(gq.codes) + co),
+                     static_cast<const uint8_t *>(gq.scales)[so], gh);
+            dequant8(*reinterpret_cast<const uint32_t *>(static_cast<const uint8_t *>(uq.codes) + co),
+                     static_cast<const uint8_t *>(uq.scales)[so], uh);
         }
         float dg[8], du[8], mr[8];
 #pragma unroll
@@ -248,59 +267,75 @@ __global__ void __launch_bounds__(256) k_silu_mul_bwd_quant(const pact_bf16 *__r
 }
 
 // ------------------------------------------------------- A10: RMSNorm backward
-template <int NCH>
-__global__ void __launch_bounds__(RMS_THREADS) k_rmsnorm_bwd(const pact_bf16 *__restrict__ dy, int64_t lddy,
+// Same row groups as the forward; dy stays packed BF16 and y^ stays NVFP4 (codes and
+// scale byte) in registers between the reduction and the output pass.
+template <int NCH, int WPR>
+__global__ void __launch_bounds__(RMS_THREADS, 2) k_rmsnorm_bwd(const pact_bf16 *__restrict__ dy, int64_t lddy,
                                                              pact_nvfp4_t yq, const float *__restrict__ rstd,
                                                              const pact_bf16 *__restrict__ gamma, int64_t M, int64_t H,
                                                              const pact_bf16 *__restrict__ dres,
                                                              pact_bf16 *__restrict__ dx, pact_nvfp4_t dxq, int has_dxq) {
-    __shared__ float red[RMS_THREADS / 32];
+    __shared__ float red[RMS_WARPS];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const int64_t row = blockIdx.x;
-    const int64_t nchunk = (H + CHUNK - 1) / CHUNK;
-    if (row >= M) {
-        if (has_dxq)
-            for (int64_t ch = warp; ch < nchunk; ch += RMS_THREADS / 32) zero_pad_scales(dxq, row, ch * CHUNK);
-        return;
-    }
-    float dv[NCH][8], yv[NCH][8];
+    const int wr = warp % WPR;
+    const int64_t row = (int64_t)blockIdx.x * (RMS_WARPS / WPR) + warp / WPR;
+    const bool real = row < M;
+    uint4 dv[NCH];
+    uint32_t yc[NCH], ys[NCH];
     float dot = 0.0f;
 #pragma unroll
     for (int k = 0; k < NCH; ++k) {
-        const int64_t c = (warp + (int64_t)k * (RMS_THREADS / 32)) * CHUNK + 8 * lane;
-#pragma unroll
-        for (int i = 0; i < 8; ++i) dv[k][i] = yv[k][i] = 0.0f;
-        if (c < H) {
-            load8_bf16(dy + row * lddy + c, dv[k]);
-            load8_nvfp4(yq, row, c, yv[k]);
-            // (gamma * dy) * (y^ / gamma) == dy * y^
-#pragma unroll
-            for (int i = 0; i < 8; ++i) dot = fmaf(dv[k][i], yv[k][i], dot);
+        const int64_t c = (wr + (int64_t)k * WPR) * CHUNK + 8 * lane;
+        dv[k] = make_uint4(0, 0, 0, 0);
+        yc[k] = 0;
+        ys[k] = 0;
+        if (real && c < H) {
+            dv[k] = *reinterpret_cast<const uint4 *>(dy + row * lddy + c);
+            yc[k] = *reinterpret_cast<const uint32_t *>(static_cast<const uint8_t *>(yq.codes) + row * (H >> 1) +
+                                                         (c >> 1));
+            ys[k] = static_cast<const uint8_t *>(yq.scales)[scale_offset(row, c >> 4, H)];
         }
     }
 #pragma unroll
-    for (int o = 16; o; o >>= 1) dot += __shfl_xor_sync(0xFFFFFFFFu, dot, o);
-    if (lane == 0) red[warp] = dot;
-    __syncthreads();
-    float tot = 0.0f;
+    for (int k = 0; k < NCH; ++k) {
+        float d[8], yv[8];
+        unpack8_bf16(dv[k], d);
+        dequant8(yc[k], ys[k], yv);
+        // (gamma * dy) * (y^ / gamma) == dy * y^
 #pragma unroll
-    for (int w = 0; w < RMS_THREADS / 32; ++w) tot += red[w];
-    const float mean = tot / (float)H;
-    const float r = rstd[row];
+        for (int i = 0; i < 8; ++i) dot = fmaf(d[i], yv[i], dot);
+    }
+#pragma unroll
+    for (int o = 16; o; o >>= 1) dot += __shfl_xor_sync(0xFFFFFFFFu, dot, o);
+    if (WPR > 1) {
+        if (lane == 0) red[warp] = dot;
+        __syncthreads();
+        dot = 0.0f;
+#pragma unroll
+        for (int w = 0; w < WPR; ++w) dot += red[warp - wr + w];
+    }
+    const float mean = dot / (float)H;
+    const float r = real ? rstd[row] : 0.0f;
 #pragma unroll
     for (int k = 0; k < NCH; ++k) {
-        const int64_t c0 = (warp + (int64_t)k * (RMS_THREADS / 32)) * CHUNK;
+        const int64_t c0 = (wr + (int64_t)k * WPR) * CHUNK;
         if (c0 >= H) break;
+        if (!real) {
+            if (has_dxq) zero_pad_scales(dxq, row, c0);
+            continue;
+        }
         const int64_t c = c0 + 8 * lane;
         const bool valid = c < H;
-        float g[8] = {1, 1, 1, 1, 1, 1, 1, 1}, res[8] = {0, 0, 0, 0, 0, 0, 0, 0}, o[8];
+        float d[8], yv[8], g[8] = {1, 1, 1, 1, 1, 1, 1, 1}, res[8] = {0, 0, 0, 0, 0, 0, 0, 0}, o[8];
+        unpack8_bf16(dv[k], d);
+        dequant8(yc[k], ys[k], yv);
         if (valid) {
             load8_bf16(gamma + c, g);
             if (dres) load8_bf16(dres + row * H + c, res);
         }
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
-            const float val = r * (g[i] * dv[k][i] - __fdividef(yv[k][i], g[i]) * mean) + res[i];
+            const float val = r * (g[i] * d[i] - __fdividef(yv[i], g[i]) * mean) + res[i];
             o[i] = valid ? __bfloat162float(__float2bfloat16_rn(val)) : 0.0f;
         }
         if (valid) store8_bf16(dx + row * H + c, o);
@@ -409,7 +444,7 @@ pact_status pact_quantize_nvfp4(const pact_bf16 *x, int64_t ldx, int64_t rows, i
 pact_status pact_rmsnorm_quant(const pact_bf16 *x, int64_t ldx, const pact_bf16 *gamma, float eps, int64_t M,
                                int64_t H, const pact_nvfp4_t *yq, pact_bf16 *y, float *rstd, pact_stream_t stream) {
     PACT_CHECK(x && gamma && yq, PACT_ERR_INVALID_ARG, "pact_rmsnorm_quant: NULL argument");
-    PACT_CHECK(M >= 1 && H >= 64 && H % 64 == 0 && H <= RMS_THREADS / 32 * RMS_MAX_CHUNKS * CHUNK, PACT_ERR_SHAPE,
+    PACT_CHECK(M >= 1 && H >= 64 && H % 64 == 0 && H <= RMS_WARPS * RMS_MAX_CHUNKS * CHUNK, PACT_ERR_SHAPE,
                "pact_rmsnorm_quant: M >= 1, H a multiple of 64 in [64, 16384] required (M=%lld H=%lld)",
                (long long)M, (long long)H);
     PACT_CHECK(!(eps < 0.0f) && isfinite(eps), PACT_ERR_INVALID_ARG, "pact_rmsnorm_quant: eps must be finite and >= 0");
@@ -417,15 +452,27 @@ pact_status pact_rmsnorm_quant(const pact_bf16 *x, int64_t ldx, const pact_bf16 
                PACT_ERR_ALIGN, "pact_rmsnorm_quant: pointers must be 16-byte aligned, ldx >= H, ldx %% 8 == 0");
     pact_status s = check_nvfp4(yq, M, H, "yq");
     if (s != PACT_OK) return s;
-    const int64_t grid = (M + 127) / 128 * 128;
-    PACT_CHECK(grid <= 0x7FFFFFFF, PACT_ERR_SHAPE, "pact_rmsnorm_quant: M too large");
+    const int64_t rows_pad = (M + 127) / 128 * 128;
+    PACT_CHECK(rows_pad <= 0x7FFFFFFF, PACT_ERR_SHAPE, "pact_rmsnorm_quant: M too large");
     cudaStream_t st = (cudaStream_t)stream;
-    switch (rms_nch(H)) {
-        case 1: k_rmsnorm_quant<1><<<(unsigned)grid, RMS_THREADS, 0, st>>>(x, ldx, gamma, eps, M, H, *yq, y, rstd); break;
-        case 2: k_rmsnorm_quant<2><<<(unsigned)grid, RMS_THREADS, 0, st>>>(x, ldx, gamma, eps, M, H, *yq, y, rstd); break;
-        case 4: k_rmsnorm_quant<4><<<(unsigned)grid, RMS_THREADS, 0, st>>>(x, ldx, gamma, eps, M, H, *yq, y, rstd); break;
-        default: k_rmsnorm_quant<8><<<(unsigned)grid, RMS_THREADS, 0, st>>>(x, ldx, gamma, eps, M, H, *yq, y, rstd); break;
+    const int wpr = rms_wpr(H), nch = rms_nch(H);
+    const unsigned grid = (unsigned)(rows_pad / (RMS_WARPS / wpr));
+#define PACT_RMS_FWD(NC, WP) k_rmsnorm_quant<NC, WP><<<grid, RMS_THREADS, 0, st>>>(x, ldx, gamma, eps, M, H, *yq, y, rstd)
+    if (wpr == 1) {
+        switch (nch) {
+            case 1: PACT_RMS_FWD(1, 1); break;
+            case 2: PACT_RMS_FWD(2, 1); break;
+            case 4: PACT_RMS_FWD(4, 1); break;
+            default: PACT_RMS_FWD(8, 1); break;
+        }
+    } else if (wpr == 2) {
+        PACT_RMS_FWD(8, 2);
+    } else if (wpr == 4) {
+        PACT_RMS_FWD(8, 4);
+    } else {
+        PACT_RMS_FWD(8, 8);
     }
+#undef PACT_RMS_FWD
     return launch_status("pact_rmsnorm_quant");
 }
 
@@ -471,7 +518,7 @@ pact_status pact_rmsnorm_bwd(const pact_bf16 *dy, int64_t lddy, const pact_nvfp4
                              const pact_bf16 *gamma, int64_t M, int64_t H, const pact_bf16 *dres, pact_bf16 *dx,
                              const pact_nvfp4_t *dxq, pact_stream_t stream) {
     PACT_CHECK(dy && yq && rstd && gamma && dx, PACT_ERR_INVALID_ARG, "pact_rmsnorm_bwd: NULL argument");
-    PACT_CHECK(M >= 1 && H >= 64 && H % 64 == 0 && H <= RMS_THREADS / 32 * RMS_MAX_CHUNKS * CHUNK, PACT_ERR_SHAPE,
+    PACT_CHECK(M >= 1 && H >= 64 && H % 64 == 0 && H <= RMS_WARPS * RMS_MAX_CHUNKS * CHUNK, PACT_ERR_SHAPE,
                "pact_rmsnorm_bwd: M >= 1, H a multiple of 64 in [64, 16384] required");
     PACT_CHECK(lddy >= H && lddy % 8 == 0 && aligned16(dy) && aligned16(gamma) && aligned16(dx) && aligned16(dres),
                PACT_ERR_ALIGN, "pact_rmsnorm_bwd: pointers must be 16-byte aligned, lddy %% 8 == 0");
@@ -479,16 +526,30 @@ pact_status pact_rmsnorm_bwd(const pact_bf16 *dy, int64_t lddy, const pact_nvfp4
     if (s == PACT_OK && dxq) s = check_nvfp4(dxq, M, H, "dxq");
     if (s != PACT_OK) return s;
     pact_nvfp4_t none = {nullptr, nullptr, M, H};
-    const int64_t grid = dxq ? (M + 127) / 128 * 128 : M;
+    const int64_t rows = dxq ? (M + 127) / 128 * 128 : M;
     cudaStream_t st = (cudaStream_t)stream;
     const pact_nvfp4_t q = dxq ? *dxq : none;
     const int has = dxq != nullptr;
-    switch (rms_nch(H)) {
-        case 1: k_rmsnorm_bwd<1><<<(unsigned)grid, RMS_THREADS, 0, st>>>(dy, lddy, *yq, rstd, gamma, M, H, dres, dx, q, has); break;
-        case 2: k_rmsnorm_bwd<2><<<(unsigned)grid, RMS_THREADS, 0, st>>>(dy, lddy, *yq, rstd, gamma, M, H, dres, dx, q, has); break;
-        case 4: k_rmsnorm_bwd<4><<<(unsigned)grid, RMS_THREADS, 0, st>>>(dy, lddy, *yq, rstd, gamma, M, H, dres, dx, q, has); break;
-        default: k_rmsnorm_bwd<8><<<(unsigned)grid, RMS_THREADS, 0, st>>>(dy, lddy, *yq, rstd, gamma, M, H, dres, dx, q, has); break;
+    const int wpr = rms_wpr(H), nch = rms_nch(H);
+    const int64_t per_cta = RMS_WARPS / wpr;
+    const unsigned grid = (unsigned)((rows + per_cta - 1) / per_cta);
+#define PACT_RMS_BWD(NC, WP) \
+    k_rmsnorm_bwd<NC, WP><<<grid, RMS_THREADS, 0, st>>>(dy, lddy, *yq, rstd, gamma, M, H, dres, dx, q, has)
+    if (wpr == 1) {
+        switch (nch) {
+            case 1: PACT_RMS_BWD(1, 1); break;
+            case 2: PACT_RMS_BWD(2, 1); break;
+            case 4: PACT_RMS_BWD(4, 1); break;
+            default: PACT_RMS_BWD(8, 1); break;
+        }
+    } else if (wpr == 2) {
+        PACT_RMS_BWD(8, 2);
+    } else if (wpr == 4) {
+        PACT_RMS_BWD(8, 4);
+    } else {
+        PACT_RMS_BWD(8, 8);
     }
+#undef PACT_RMS_BWD
     return launch_status("pact_rmsnorm_bwd");
 }
 

@@ -6,6 +6,8 @@
 // Work split: a warp owns 256 consecutive columns of one row; lane j holds the 8
 // values [8j, 8j+8) of that chunk, so the 16-value block b lives in lanes 2b, 2b+1.
 #pragma once
+#include <cuda_fp16.h>
+
 #include "common.cuh"
 
 namespace pact {
@@ -22,13 +24,15 @@ __device__ __forceinline__ float e4m3_to_float(uint32_t b) {
     return e ? __uint_as_float(((e + 120u) << 23) | (m << 20)) : (float)m * 0.001953125f;
 }
 
-// E2M1 code (4 bits incl. sign) -> float, exact.
-__device__ __forceinline__ float e2m1_to_float(uint32_t c) {
-    // magnitudes 0, .5, 1, 1.5, 2, 3, 4, 6 as float bit patterns
-    const uint32_t e = c & 7u;
-    const uint32_t bits = (e == 0) ? 0u : (e == 1) ? 0x3F000000u : (e == 2) ? 0x3F800000u : (e == 3) ? 0x3FC00000u
-                        : (e == 4) ? 0x40000000u : (e == 5) ? 0x40400000u : (e == 6) ? 0x40800000u : 0x40C00000u;
-    return __uint_as_float(bits | ((c & 8u) << 28));
+// One byte of two E2M1 codes (element 0 in the low nibble) -> two FP16 values
+// (element 0 in the low half), exact: hardware conversion.
+__device__ __forceinline__ uint32_t e2m1x2_to_f16x2(uint32_t byte) {
+    uint32_t r;
+    asm("{\n\t.reg .b8 t;\n\t.reg .b16 w;\n\tcvt.u16.u32 w, %1;\n\tcvt.u8.u16 t, w;\n\t"
+        "cvt.rn.f16x2.e2m1x2 %0, t;\n\t}"
+        : "=r"(r)
+        : "r"(byte));
+    return r;
 }
 
 // |x| / s as the correctly rounded FP32 quotient would decide it, from the correctly
@@ -124,13 +128,46 @@ __device__ __forceinline__ void store8_bf16(pact_bf16 *p, const float (&v)[8]) {
     *reinterpret_cast<uint4 *>(p) = u;
 }
 
+// Dequantize 8 NVFP4 values: 4 code bytes (element 0 in the low nibble of byte 0)
+// and their block's scale byte.  Exact: E2M1 pairs convert to FP16 in hardware, the
+// product with the E4M3 scale has at most 6 significant bits and lies in
+// [2^-10, 2688], so it is exact in FP16, and FP16 widens to FP32 exactly.
+__device__ __forceinline__ void dequant8(uint32_t codes, uint32_t sbyte, float (&v)[8]) {
+    const __half sh = __float2half_rn(e4m3_to_float(sbyte));  // exact: E4M3 values are FP16 values
+    const __half2 s2 = __half2half2(sh);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const uint32_t h = e2m1x2_to_f16x2((codes >> (8 * i)) & 0xFFu);
+        const __half2 p = __hmul2(*reinterpret_cast<const __half2 *>(&h), s2);
+        const float2 f = __half22float2(p);
+        v[2 * i] = f.x;
+        v[2 * i + 1] = f.y;
+    }
+}
+
 // Dequantize the 8 values [c, c+8) of row `row` (c a multiple of 8).
 __device__ __forceinline__ void load8_nvfp4(const pact_nvfp4_t &t, int64_t row, int64_t c, float (&v)[8]) {
     const uint32_t codes =
         *reinterpret_cast<const uint32_t *>(static_cast<const uint8_t *>(t.codes) + row * (t.cols >> 1) + (c >> 1));
-    const float s = e4m3_to_float(static_cast<const uint8_t *>(t.scales)[scale_offset(row, c >> 4, t.cols)]);
-#pragma unroll
-    for (int i = 0; i < 8; ++i) v[i] = e2m1_to_float((codes >> (4 * i)) & 15u) * s;
+    dequant8(codes, static_cast<const uint8_t *>(t.scales)[scale_offset(row, c >> 4, t.cols)], v);
 }
+
+// Row-major (row, 256-column chunk) tasks visited by a grid-stride loop without a
+// division per task: the stride is split once into whole rows and a chunk remainder.
+struct TaskIter {
+    int64_t row;
+    int64_t chunk, nchunk, drow, dchunk;
+    __device__ __forceinline__ TaskIter(int64_t start, int64_t nchunk_, int64_t stride)
+        : row(start / nchunk_), chunk(start % nchunk_), nchunk(nchunk_), drow(stride / nchunk_),
+          dchunk(stride % nchunk_) {}
+    __device__ __forceinline__ void next() {
+        row += drow;
+        chunk += dchunk;
+        if (chunk >= nchunk) {
+            chunk -= nchunk;
+            ++row;
+        }
+    }
+};
 
 }  // namespace pact

@@ -36,6 +36,7 @@ class Op:
     kind: str = "other"        # "gemm" for the NVFP4 frozen GEMMs
     flops: float = 0.0         # algorithmic FLOPs of a GEMM op
     kernels: int = 1           # libpact kernels one call launches
+    bytes: float = 0.0         # algorithmic HBM bytes of one call (each input read once, each output written once)
 
 
 @dataclass
@@ -55,6 +56,10 @@ class LayerShape:
     @property
     def n_qkv(self) -> int:
         return self.H + 2 * self.KV
+
+    def nv(self, rows: int, cols: int) -> float:
+        """Bytes of an NVFP4 tensor: codes plus one scale byte per 16 values."""
+        return rows * cols / 2 + rows * cols / 16
 
     def frozen_flops(self) -> float:
         """2 M N K for the forward and the dgrad of the seven frozen projections."""
@@ -145,28 +150,40 @@ class PactLayer:
     def forward_ops(self) -> List[Op]:
         S, s = self.s, self.s.scale
         h, attn, _, _ = self.inputs
-        I = S.I
+        M, H, I, r = S.M, S.H, S.I, S.r
         gemm = lambda M, N, K: 2.0 * M * N * K
+        # NVFP4 GEMM: activation codes + weight codes in, BF16 output and the LoRA term's
+        # hi|lo activations [M x 2R] and B chunk [N x R] in (residual added by the caller)
+        gbytes = lambda N, K, R: S.nv(M, K) + S.nv(N, K) + 2 * M * N + 2 * M * 2 * R + 2 * N * R
+        # LoRA forward T = s x A^T as hi|lo: x [M x K] and A [R x K] in, T [M x 2R] out
+        lora_fwd = lambda K, R: 2 * M * K + 2 * R * K + 2 * M * 2 * R
         return [
-            Op("rmsnorm_quant_1", lambda: P.pact_rmsnorm_quant(h, self.g1, S.eps, self.xq1, self.x1, self.rstd1)),
-            Op("lora_fwd_qkv", lambda: P.pact_lora_fwd(self.x1, self.a_qkv, s, self.t_qkv, self.ws), kernels=2),
+            Op("rmsnorm_quant_1", lambda: P.pact_rmsnorm_quant(h, self.g1, S.eps, self.xq1, self.x1, self.rstd1),
+               bytes=2 * M * H + 2 * H + S.nv(M, H) + 2 * M * H + 4 * M),
+            Op("lora_fwd_qkv", lambda: P.pact_lora_fwd(self.x1, self.a_qkv, s, self.t_qkv, self.ws), kernels=2,
+               bytes=lora_fwd(H, 3 * r)),
             Op("gemm_fwd_qkv", lambda: P.pact_frozen_gemm_fwd(self.xq1, self.c_qkv, self.l_qkv_f, y=self.qkv),
-               "gemm", gemm(S.M, S.n_qkv, S.H)),
-            Op("quantize_attn", lambda: P.pact_quantize_nvfp4(attn, self.aq)),
-            Op("lora_fwd_o", lambda: P.pact_lora_fwd(attn, self.a_o, s, self.t_o, self.ws), kernels=2),
+               "gemm", gemm(S.M, S.n_qkv, S.H), bytes=gbytes(S.n_qkv, H, 3 * r)),
+            Op("quantize_attn", lambda: P.pact_quantize_nvfp4(attn, self.aq), bytes=2 * M * H + S.nv(M, H)),
+            Op("lora_fwd_o", lambda: P.pact_lora_fwd(attn, self.a_o, s, self.t_o, self.ws), kernels=2,
+               bytes=lora_fwd(H, r)),
             Op("gemm_fwd_o", lambda: P.pact_frozen_gemm_fwd(self.aq, self.c_o, self.l_o_f, residual=h, y=self.h2),
-               "gemm", gemm(S.M, S.H, S.H)),
+               "gemm", gemm(S.M, S.H, S.H), bytes=gbytes(H, H, r) + 2 * M * H),
             Op("rmsnorm_quant_2", lambda: P.pact_rmsnorm_quant(self.h2, self.g2, S.eps, self.xq2, self.x2,
-                                                               self.rstd2)),
-            Op("lora_fwd_gu", lambda: P.pact_lora_fwd(self.x2, self.a_gu, s, self.t_gu, self.ws), kernels=2),
+                                                               self.rstd2),
+               bytes=2 * M * H + 2 * H + S.nv(M, H) + 2 * M * H + 4 * M),
+            Op("lora_fwd_gu", lambda: P.pact_lora_fwd(self.x2, self.a_gu, s, self.t_gu, self.ws), kernels=2,
+               bytes=lora_fwd(H, 2 * r)),
             Op("gemm_fwd_gu", lambda: P.pact_frozen_gemm_fwd(self.xq2, self.c_gu, self.l_gu_f, y=self.gu),
-               "gemm", gemm(S.M, 2 * I, S.H)),
+               "gemm", gemm(S.M, 2 * I, S.H), bytes=gbytes(2 * I, H, 2 * r)),
             Op("silu_mul_quant", lambda: P.pact_silu_mul_quant(self.gu[:, :I], self.gu[:, I:], self.m, self.mq,
-                                                               self.gq, self.uq)),
-            Op("lora_fwd_down", lambda: P.pact_lora_fwd(self.m, self.a_d, s, self.t_d, self.ws), kernels=2),
+                                                               self.gq, self.uq),
+               bytes=4 * M * I + 2 * M * I + 3 * S.nv(M, I)),
+            Op("lora_fwd_down", lambda: P.pact_lora_fwd(self.m, self.a_d, s, self.t_d, self.ws), kernels=2,
+               bytes=lora_fwd(I, r)),
             Op("gemm_fwd_down", lambda: P.pact_frozen_gemm_fwd(self.mq, self.c_d, self.l_d_f, residual=self.h2,
                                                                y=self.out),
-               "gemm", gemm(S.M, S.H, I)),
+               "gemm", gemm(S.M, S.H, I), bytes=gbytes(H, I, r) + 2 * M * H),
         ]
 
     def backward_ops(self) -> List[Op]:
@@ -174,43 +191,59 @@ class PactLayer:
         H, I = S.H, S.I
         _, attn, d_out, d_qkv = self.inputs
         g = self.grads
+        M = S.M
         gemm = lambda M, N, K: 2.0 * M * N * K
+        gbytes = lambda N, K, R: S.nv(M, K) + S.nv(N, K) + 2 * M * N + 2 * M * 2 * R + 2 * K * R
+        # U = s dY B as hi|lo: dY [M x N] and B [N x R] in, U [M x 2R] out
+        lora_u = lambda N, R: 2 * M * N + 2 * N * R + 2 * M * 2 * R
+        # dA, dB: dY [M x N], the saved input (x_bytes), U [M x 2R] and A [R x K] in; dA, dB out
+        lora_bwd = lambda N, x_bytes, K, R: 2 * M * N + x_bytes + 2 * M * 2 * R + 2 * R * K + 2 * R * K + 2 * N * R
         LB = 7  # kernels of one pact_lora_bwd call reading an NVFP4 copy (6 with BF16 input)
         return [
             # down projection
-            Op("lora_bwd_u_down", lambda: P.pact_lora_bwd_u(d_out, self.b_d, r, [H], s, self.u_d, self.ws), kernels=2),
-            Op("quantize_dout", lambda: P.pact_quantize_nvfp4(d_out, self.doq)),
+            Op("lora_bwd_u_down", lambda: P.pact_lora_bwd_u(d_out, self.b_d, r, [H], s, self.u_d, self.ws), kernels=2,
+               bytes=lora_u(H, r)),
+            Op("quantize_dout", lambda: P.pact_quantize_nvfp4(d_out, self.doq), bytes=2 * M * H + S.nv(M, H)),
             Op("gemm_dgrad_down", lambda: P.pact_frozen_gemm_dgrad(self.doq, self.c_d, self.l_d_b, dx=self.dm),
-               "gemm", gemm(S.M, I, H)),
+               "gemm", gemm(S.M, I, H), bytes=gbytes(I, H, r)),
             Op("silu_mul_bwd_quant", lambda: P.pact_silu_mul_bwd_quant(self.dm, self.gq, self.uq, self.dgu,
-                                                                       self.dguq, self.m_re)),
+                                                                       self.dguq, self.m_re),
+               bytes=2 * M * I + 2 * S.nv(M, I) + 4 * M * I + S.nv(M, 2 * I) + 2 * M * I),
             Op("lora_bwd_down", lambda: P.pact_lora_bwd(d_out, self.a_d, self.u_d, r, [H], s, x=self.m_re,
-                                                        dA=g["a_d"], dB=g["b_d"], workspace=self.ws), kernels=LB - 1),
+                                                        dA=g["a_d"], dB=g["b_d"], workspace=self.ws), kernels=LB - 1,
+               bytes=lora_bwd(H, 2 * M * I, I, r)),
             # gate|up
-            Op("lora_bwd_u_gu", lambda: P.pact_lora_bwd_u(self.dgu, self.b_gu, r, self.seg_gu, s, self.u_gu, self.ws), kernels=2),
+            Op("lora_bwd_u_gu", lambda: P.pact_lora_bwd_u(self.dgu, self.b_gu, r, self.seg_gu, s, self.u_gu, self.ws), kernels=2,
+               bytes=lora_u(2 * I, 2 * r)),
             Op("gemm_dgrad_gu", lambda: P.pact_frozen_gemm_dgrad(self.dguq, self.c_gu, self.l_gu_b, dx=self.dx2),
-               "gemm", gemm(S.M, H, 2 * I)),
+               "gemm", gemm(S.M, H, 2 * I), bytes=gbytes(H, 2 * I, 2 * r)),
             Op("lora_bwd_gu", lambda: P.pact_lora_bwd(self.dgu, self.a_gu, self.u_gu, r, self.seg_gu, s,
                                                       xq=self.xq2, dA=g["a_gu"], dB=g["b_gu"], workspace=self.ws),
-               kernels=LB),
+               kernels=LB, bytes=lora_bwd(2 * I, S.nv(M, H), H, 2 * r)),
             Op("rmsnorm_bwd_2", lambda: P.pact_rmsnorm_bwd(self.dx2, self.xq2, self.rstd2, self.g2, dres=d_out,
-                                                           dx=self.dh2, dxq=self.dh2q)),
+                                                           dx=self.dh2, dxq=self.dh2q),
+               bytes=2 * M * H + S.nv(M, H) + 4 * M + 2 * H + 2 * M * H + 2 * M * H + S.nv(M, H)),
             # o projection (its output joined the residual stream h2)
-            Op("lora_bwd_u_o", lambda: P.pact_lora_bwd_u(self.dh2, self.b_o, r, [H], s, self.u_o, self.ws), kernels=2),
+            Op("lora_bwd_u_o", lambda: P.pact_lora_bwd_u(self.dh2, self.b_o, r, [H], s, self.u_o, self.ws), kernels=2,
+               bytes=lora_u(H, r)),
             Op("gemm_dgrad_o", lambda: P.pact_frozen_gemm_dgrad(self.dh2q, self.c_o, self.l_o_b, dx=self.dattn),
-               "gemm", gemm(S.M, H, H)),
+               "gemm", gemm(S.M, H, H), bytes=gbytes(H, H, r)),
             Op("lora_bwd_o", lambda: P.pact_lora_bwd(self.dh2, self.a_o, self.u_o, r, [H], s, x=attn,
-                                                     dA=g["a_o"], dB=g["b_o"], workspace=self.ws), kernels=LB - 1),
+                                                     dA=g["a_o"], dB=g["b_o"], workspace=self.ws), kernels=LB - 1,
+               bytes=lora_bwd(H, 2 * M * H, H, r)),
             # q|k|v (d_qkv stands in for the attention backward)
-            Op("lora_bwd_u_qkv", lambda: P.pact_lora_bwd_u(d_qkv, self.b_qkv, r, self.seg_qkv, s, self.u_qkv, self.ws), kernels=2),
-            Op("quantize_dqkv", lambda: P.pact_quantize_nvfp4(d_qkv, self.dqkvq)),
+            Op("lora_bwd_u_qkv", lambda: P.pact_lora_bwd_u(d_qkv, self.b_qkv, r, self.seg_qkv, s, self.u_qkv, self.ws), kernels=2,
+               bytes=lora_u(S.n_qkv, 3 * r)),
+            Op("quantize_dqkv", lambda: P.pact_quantize_nvfp4(d_qkv, self.dqkvq), bytes=2 * M * S.n_qkv + S.nv(M, S.n_qkv)),
             Op("gemm_dgrad_qkv", lambda: P.pact_frozen_gemm_dgrad(self.dqkvq, self.c_qkv, self.l_qkv_b, dx=self.dx1),
-               "gemm", gemm(S.M, H, S.n_qkv)),
+               "gemm", gemm(S.M, H, S.n_qkv), bytes=gbytes(H, S.n_qkv, 3 * r)),
             Op("lora_bwd_qkv", lambda: P.pact_lora_bwd(d_qkv, self.a_qkv, self.u_qkv, r, self.seg_qkv, s,
                                                        xq=self.xq1, dA=g["a_qkv"], dB=g["b_qkv"],
-                                                       workspace=self.ws), kernels=LB),
+                                                       workspace=self.ws), kernels=LB,
+               bytes=lora_bwd(S.n_qkv, S.nv(M, H), H, 3 * r)),
             Op("rmsnorm_bwd_1", lambda: P.pact_rmsnorm_bwd(self.dx1, self.xq1, self.rstd1, self.g1, dres=self.dh2,
-                                                           dx=self.dh)),
+                                                           dx=self.dh),
+               bytes=2 * M * H + S.nv(M, H) + 4 * M + 2 * H + 2 * M * H + 2 * M * H),
         ]
 
     def step_ops(self) -> List[Op]:
