@@ -181,7 +181,7 @@ def config_block(name, M):
     return {"workload": f"{name} decoder layer fwd+bwd: 7 NVFP4 frozen projections + LoRA",
             "H": c["H"], "I": c["I"], "kv": c["KV"], "tokens": M, "batch": c["batch"], "seq": c["seq"],
             "lora_r": synth.LORA_R, "lora_alpha": synth.LORA_ALPHA,
-            "l2": "flushed between timed steps (256 MiB write)", "launch": "one CUDA graph per step"}
+            "l2": "flushed between timed steps (256 MiB write)", "launch": "one CUDA graph per step (LoRA weight gradients on a parallel branch)"}
 
 
 # ------------------------------------------------------------------ GPU arm
@@ -345,10 +345,10 @@ def main():
         raise RuntimeError(P.pact_last_error())
     # the timed step: every op of the step in one CUDA graph (kernels back to back);
     # per-segment graphs give the breakdown in a separate pass after the timed region
+    side = torch.cuda.Stream(device=dev)
     step_graph = torch.cuda.CUDAGraph()
     with torch.cuda.graph(step_graph, stream=stream):
-        for op in ops:
-            op.fn()
+        layer.step_concurrent(side)   # LoRA weight-gradient leaves on a parallel branch
     for sg in segs:
         g = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g, stream=stream):

@@ -37,6 +37,7 @@ class Op:
     flops: float = 0.0         # algorithmic FLOPs of a GEMM op
     kernels: int = 1           # libpact kernels one call launches
     bytes: float = 0.0         # algorithmic HBM bytes of one call (each input read once, each output written once)
+    side: bool = False         # a leaf (LoRA weight gradients): may run beside the rest of the step
 
 
 @dataclass
@@ -126,9 +127,15 @@ class PactLayer:
                  P.pact_lora_fwd_workspace_bytes(M, H, 3 * r),
                  P.pact_lora_bwd_u_workspace_bytes(M, 2 * I, r, 2),
                  P.pact_lora_bwd_u_workspace_bytes(M, S.n_qkv, r, 3))
-        raw = torch.empty(ws + 256, dtype=torch.uint8, device=dev)
-        off = (-raw.data_ptr()) % 256
-        self.ws = raw[off:off + ws]
+        self.ws = self._scratch(ws, dev)
+        # the LoRA weight-gradient calls are leaves of the step and may run on a second
+        # stream beside the rest of it: each gets scratch of its own
+        self.ws_leaf = {
+            "down": self._scratch(P.pact_lora_bwd_workspace_bytes(M, H, I, r, 1), dev),
+            "gu": self._scratch(P.pact_lora_bwd_workspace_bytes(M, 2 * I, H, r, 2), dev),
+            "o": self._scratch(P.pact_lora_bwd_workspace_bytes(M, H, H, r, 1), dev),
+            "qkv": self._scratch(P.pact_lora_bwd_workspace_bytes(M, S.n_qkv, H, r, 3), dev),
+        }
         # LoRA descriptors for the fused GEMM epilogue
         self.l_qkv_f = P.lora_struct(self.t_qkv, self.b_qkv, r, self.seg_qkv)
         self.l_o_f = P.lora_struct(self.t_o, self.b_o, r, [H])
@@ -139,6 +146,12 @@ class PactLayer:
         self.l_o_b = P.lora_struct(self.u_o, self.a_o, r, [H])
         self.l_qkv_b = P.lora_struct(self.u_qkv, self.a_qkv, 3 * r, [H])
         self.inputs = None
+
+    @staticmethod
+    def _scratch(nbytes: int, dev) -> torch.Tensor:
+        raw = torch.empty(nbytes + 256, dtype=torch.uint8, device=dev)
+        off = (-raw.data_ptr()) % 256
+        return raw[off:off + nbytes]
 
     # ------------------------------------------------------------------ op lists
     def bind(self, h: torch.Tensor, attn: torch.Tensor, d_out: torch.Tensor, d_qkv: torch.Tensor):
@@ -210,7 +223,8 @@ class PactLayer:
                                                                        self.dguq, self.m_re),
                bytes=2 * M * I + 2 * S.nv(M, I) + 4 * M * I + S.nv(M, 2 * I) + 2 * M * I),
             Op("lora_bwd_down", lambda: P.pact_lora_bwd(d_out, self.a_d, self.u_d, r, [H], s, x=self.m_re,
-                                                        dA=g["a_d"], dB=g["b_d"], workspace=self.ws), kernels=LB - 1,
+                                                        dA=g["a_d"], dB=g["b_d"], workspace=self.ws_leaf["down"]),
+               kernels=LB - 1, side=True,
                bytes=lora_bwd(H, 2 * M * I, I, r)),
             # gate|up
             Op("lora_bwd_u_gu", lambda: P.pact_lora_bwd_u(self.dgu, self.b_gu, r, self.seg_gu, s, self.u_gu, self.ws), kernels=2,
@@ -218,8 +232,9 @@ class PactLayer:
             Op("gemm_dgrad_gu", lambda: P.pact_frozen_gemm_dgrad(self.dguq, self.c_gu, self.l_gu_b, dx=self.dx2),
                "gemm", gemm(S.M, H, 2 * I), bytes=gbytes(H, 2 * I, 2 * r)),
             Op("lora_bwd_gu", lambda: P.pact_lora_bwd(self.dgu, self.a_gu, self.u_gu, r, self.seg_gu, s,
-                                                      xq=self.xq2, dA=g["a_gu"], dB=g["b_gu"], workspace=self.ws),
-               kernels=LB, bytes=lora_bwd(2 * I, S.nv(M, H), H, 2 * r)),
+                                                      xq=self.xq2, dA=g["a_gu"], dB=g["b_gu"],
+                                                      workspace=self.ws_leaf["gu"]),
+               kernels=LB, side=True, bytes=lora_bwd(2 * I, S.nv(M, H), H, 2 * r)),
             Op("rmsnorm_bwd_2", lambda: P.pact_rmsnorm_bwd(self.dx2, self.xq2, self.rstd2, self.g2, dres=d_out,
                                                            dx=self.dh2, dxq=self.dh2q),
                bytes=2 * M * H + S.nv(M, H) + 4 * M + 2 * H + 2 * M * H + 2 * M * H + S.nv(M, H)),
@@ -229,7 +244,8 @@ class PactLayer:
             Op("gemm_dgrad_o", lambda: P.pact_frozen_gemm_dgrad(self.dh2q, self.c_o, self.l_o_b, dx=self.dattn),
                "gemm", gemm(S.M, H, H), bytes=gbytes(H, H, r)),
             Op("lora_bwd_o", lambda: P.pact_lora_bwd(self.dh2, self.a_o, self.u_o, r, [H], s, x=attn,
-                                                     dA=g["a_o"], dB=g["b_o"], workspace=self.ws), kernels=LB - 1,
+                                                     dA=g["a_o"], dB=g["b_o"], workspace=self.ws_leaf["o"]),
+               kernels=LB - 1, side=True,
                bytes=lora_bwd(H, 2 * M * H, H, r)),
             # q|k|v (d_qkv stands in for the attention backward)
             Op("lora_bwd_u_qkv", lambda: P.pact_lora_bwd_u(d_qkv, self.b_qkv, r, self.seg_qkv, s, self.u_qkv, self.ws), kernels=2,
@@ -239,7 +255,7 @@ class PactLayer:
                "gemm", gemm(S.M, H, S.n_qkv), bytes=gbytes(H, S.n_qkv, 3 * r)),
             Op("lora_bwd_qkv", lambda: P.pact_lora_bwd(d_qkv, self.a_qkv, self.u_qkv, r, self.seg_qkv, s,
                                                        xq=self.xq1, dA=g["a_qkv"], dB=g["b_qkv"],
-                                                       workspace=self.ws), kernels=LB,
+                                                       workspace=self.ws_leaf["qkv"]), kernels=LB, side=True,
                bytes=lora_bwd(S.n_qkv, S.nv(M, H), H, 3 * r)),
             Op("rmsnorm_bwd_1", lambda: P.pact_rmsnorm_bwd(self.dx1, self.xq1, self.rstd1, self.g1, dres=self.dh2,
                                                            dx=self.dh),
@@ -252,3 +268,22 @@ class PactLayer:
     def step(self):
         for op in self.step_ops():
             op.fn()
+
+    def step_concurrent(self, side: torch.cuda.Stream):
+        """The step with its leaf ops (LoRA weight gradients) on the stream `side`, each
+        ordered after everything issued before it on the current stream; the current
+        stream waits for `side` at the end.  Same results as step(); under CUDA graph
+        capture the leaves become a parallel branch of the graph."""
+        main = torch.cuda.current_stream()
+        for op in self.step_ops():
+            if op.side:
+                ready = torch.cuda.Event()
+                ready.record(main)
+                side.wait_event(ready)
+                with torch.cuda.stream(side):
+                    op.fn()
+            else:
+                op.fn()
+        done = torch.cuda.Event()
+        done.record(side)
+        main.wait_event(done)

@@ -6,9 +6,10 @@ error downstream.  NVFP4 codes/scales and BF16 values the method rounds exactly
 must satisfy |gpu - oracle| <= 8e-3 |oracle| + 1e-3 rms(oracle).
 
 The full-size case runs the bench's workload (Llama-3.2-1B layer, 2048 tokens) in
-the same launch configuration bench.py times (the same op list, captured into the
-same per-segment CUDA graphs); the frozen GEMM outputs are checked on sampled rows
-the oracle computes one by one, everything else in full."""
+the launch configuration bench.py times (the same op list captured into one CUDA
+graph, the LoRA weight gradients on a parallel branch); the frozen GEMM outputs are
+checked on sampled rows the oracle computes one by one, everything else in full,
+and the graph's results must equal an eager sequential step bit for bit."""
 import numpy as np
 import pytest
 import torch
@@ -42,26 +43,13 @@ def run_layer(name, M, graphs):
     if graphs:
         L.step()                       # eager pass first (lazy per-device setup)
         torch.cuda.synchronize()
-        segs, cur = [], []
-        for op in ops:
-            if op.kind == "gemm":
-                if cur:
-                    segs.append(cur)
-                segs.append([op])
-                cur = []
-            else:
-                cur.append(op)
-        if cur:
-            segs.append(cur)
-        s = torch.cuda.Stream()
-        gs = []
-        for sg in segs:
-            g = torch.cuda.CUDAGraph()
-            with torch.cuda.graph(g, stream=s):
-                for op in sg:
-                    op.fn()
-            gs.append(g)
-        for g in gs:
+        # bench.py's timed configuration: the whole step in one CUDA graph, the LoRA
+        # weight-gradient leaves on a parallel branch
+        s, side = torch.cuda.Stream(), torch.cuda.Stream()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=s):
+            L.step_concurrent(side)
+        for _ in range(2):
             g.replay()
     else:
         L.step()
@@ -221,6 +209,15 @@ def test_layer_small_all_rows(orc, small_layer, graphs):
 def test_layer_llama1b_full_size(orc):
     """The bench workload itself, in the bench's launch configuration."""
     L, inp = run_layer("llama-3.2-1b", synth.tokens("llama-3.2-1b"), graphs=True)
+    # the concurrent graph step and an eager sequential step agree bit for bit
+    snap = {k: v.clone() for k, v in L.grads.items()}
+    outs = {"out": L.out.clone(), "dh": L.dh.clone(), "dattn": L.dattn.clone()}
+    L.step()
+    torch.cuda.synchronize()
+    for k, v in snap.items():
+        assert torch.equal(v, L.grads[k]), f"LoRA gradient {k}: concurrent graph step != eager step"
+    for k, v in outs.items():
+        assert torch.equal(v, getattr(L, k)), f"{k}: concurrent graph step != eager step"
     rows = np.sort(np.random.default_rng(11).choice(L.s.M, size=48, replace=False))
     rows[-1] = L.s.M - 1
     check_layer(L, inp, orc, rows=rows)
