@@ -19,6 +19,12 @@ __device__ __forceinline__ void zero_pad_scales(const pact_nvfp4_t &t, int64_t r
     }
 }
 
+// 8 packed BF16 values -> floats (element 0 in the low half of .x).
+__device__ __forceinline__ void unpack8_bf16(const uint4 &u, float (&v)[8]) {
+    v[0] = bf16lo(u.x); v[1] = bf16hi(u.x); v[2] = bf16lo(u.y); v[3] = bf16hi(u.y);
+    v[4] = bf16lo(u.z); v[5] = bf16hi(u.z); v[6] = bf16lo(u.w); v[7] = bf16hi(u.w);
+}
+
 // ------------------------------------------------------------------ A2: quantize
 __global__ void __launch_bounds__(256) k_quantize(const pact_bf16 *__restrict__ x, int64_t ldx, int64_t rows,
                                                   pact_nvfp4_t out) {
@@ -27,19 +33,32 @@ __global__ void __launch_bounds__(256) k_quantize(const pact_bf16 *__restrict__ 
     const int64_t rows_pad = (rows + 127) & ~int64_t(127);
     const int64_t warp0 = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
     const int64_t nwarps = (int64_t)gridDim.x * (blockDim.x >> 5);
-    for (TaskIter it(warp0, nchunk, nwarps); it.row < rows_pad; it.next()) {
+    auto load = [&](const TaskIter &t) {
+        const int64_t c = t.chunk * CHUNK + 8 * lane;
+        return (t.row < rows && c < out.cols) ? *reinterpret_cast<const uint4 *>(x + t.row * ldx + c)
+                                              : make_uint4(0, 0, 0, 0);
+    };
+    TaskIter it(warp0, nchunk, nwarps);
+    uint4 cur = make_uint4(0, 0, 0, 0);
+    if (it.row < rows_pad) cur = load(it);
+    while (it.row < rows_pad) {    // software-pipelined: the next task's load is in flight
+        TaskIter nx = it;
+        nx.next();
+        const uint4 nxt = nx.row < rows_pad ? load(nx) : make_uint4(0, 0, 0, 0);
         const int64_t row = it.row;
         const int64_t c0 = it.chunk * CHUNK;
         if (row >= rows) {
             zero_pad_scales(out, row, c0);
-            continue;
+        } else {
+            const bool valid = c0 + 8 * lane < out.cols;
+            float v[8];
+            unpack8_bf16(cur, v);
+            uint32_t sb;
+            const uint32_t codes = quant8(v, &sb);
+            store_chunk(out, row, c0, codes, sb, valid);
         }
-        const bool valid = c0 + 8 * lane < out.cols;
-        float v[8] = {0, 0, 0, 0, 0, 0, 0, 0};
-        if (valid) load8_bf16(x + row * ldx + c0 + 8 * lane, v);
-        uint32_t sb;
-        const uint32_t codes = quant8(v, &sb);
-        store_chunk(out, row, c0, codes, sb, valid);
+        it = nx;
+        cur = nxt;
     }
 }
 
@@ -71,11 +90,6 @@ static int rms_wpr(int64_t H) {
 static int rms_nch(int64_t H) {
     const int64_t per_warp = ((H + CHUNK - 1) / CHUNK + rms_wpr(H) - 1) / rms_wpr(H);
     return per_warp <= 1 ? 1 : per_warp <= 2 ? 2 : per_warp <= 4 ? 4 : 8;
-}
-
-__device__ __forceinline__ void unpack8_bf16(const uint4 &u, float (&v)[8]) {
-    v[0] = bf16lo(u.x); v[1] = bf16hi(u.x); v[2] = bf16lo(u.y); v[3] = bf16hi(u.y);
-    v[4] = bf16lo(u.z); v[5] = bf16hi(u.z); v[6] = bf16lo(u.w); v[7] = bf16hi(u.w);
 }
 
 // BF16 rounding of y = (x * rstd) * gamma with one correct rounding of the double
@@ -156,15 +170,19 @@ __global__ void __launch_bounds__(RMS_THREADS, 2) k_rmsnorm_quant(const pact_bf1
 // m = BF16_RNE(silu(g) * u), exactly rounded.  The FP32 evaluation with the fast
 // exponential and division has a relative error of at most (5 + 1.16 |g|) FP32
 // ulps (CUDA's documented bounds for __expf and __fdividef plus three roundings),
-// i.e. at most 2 * (5 + 1.16 * 40) < 110 ulps of the result for |g| <= 40; it
-// decides unless it lies within 256 ulps of a BF16 midpoint, and the double
-// expression decides otherwise and for |g| > 40 (Ziv's method, as above).
+// i.e. at most 2 (5 + 1.16 |g|) = 10 + 2.32 |g| ulps of the result; it decides
+// unless it lies within 12 + 3 |g| ulps of a BF16 midpoint (at most 132 for
+// |g| <= 40), and the double expression decides otherwise and for |g| > 40 (Ziv's
+// method, as above).  The margin grows with |g| so that the double path stays rare.
 __device__ __forceinline__ float sigmoid_fast(float g) { return __fdividef(1.0f, 1.0f + __expf(-g)); }
 
 __device__ __forceinline__ float silu_mul_round(float g, float u, float s) {
     const float m = __fmul_rn(__fmul_rn(g, s), u);
     const uint32_t lo = __float_as_uint(m) & 0xFFFFu;
-    if (lo - 0x7F00u <= 0x200u || !(fabsf(g) <= 40.0f) || !isfinite(m)) {
+    const float ag = fabsf(g);
+    const uint32_t margin = 12u + (uint32_t)(3.0f * fminf(ag, 40.0f));
+    const uint32_t dist = lo >= 0x8000u ? lo - 0x8000u : 0x8000u - lo;
+    if (dist <= margin || !(ag <= 40.0f) || !isfinite(m)) {
         const double gd = (double)g;
         return __bfloat162float(__double2bfloat16((gd / (1.0 + exp(-gd))) * (double)u));
     }
@@ -173,6 +191,8 @@ __device__ __forceinline__ float silu_mul_round(float g, float u, float s) {
 
 __device__ __forceinline__ float silu_mul_out(float g, float u) { return silu_mul_round(g, u, sigmoid_fast(g)); }
 
+// The task loops below are software-pipelined: a warp loads the next task's inputs
+// before it computes the current one, so two tasks' loads are in flight per warp.
 __global__ void __launch_bounds__(256) k_silu_mul_quant(const pact_bf16 *__restrict__ g, const pact_bf16 *__restrict__ u,
                                                         int64_t ld_gu, int64_t M, int64_t I,
                                                         pact_bf16 *__restrict__ m, pact_nvfp4_t mq, pact_nvfp4_t gq,
@@ -182,36 +202,52 @@ __global__ void __launch_bounds__(256) k_silu_mul_quant(const pact_bf16 *__restr
     const int64_t rows_pad = (M + 127) & ~int64_t(127);
     const int64_t warp0 = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
     const int64_t nwarps = (int64_t)gridDim.x * (blockDim.x >> 5);
-    for (TaskIter it(warp0, nchunk, nwarps); it.row < rows_pad; it.next()) {
+    auto load = [&](const TaskIter &t, uint4 &gr, uint4 &ur) {
+        const int64_t c = t.chunk * CHUNK + 8 * lane;
+        gr = ur = make_uint4(0, 0, 0, 0);
+        if (t.row < M && c < I) {
+            gr = *reinterpret_cast<const uint4 *>(g + t.row * ld_gu + c);
+            ur = *reinterpret_cast<const uint4 *>(u + t.row * ld_gu + c);
+        }
+    };
+    TaskIter it(warp0, nchunk, nwarps);
+    uint4 gr, ur;
+    if (it.row < rows_pad) load(it, gr, ur);
+    while (it.row < rows_pad) {
+        TaskIter nx = it;
+        nx.next();
+        uint4 gn = make_uint4(0, 0, 0, 0), un = make_uint4(0, 0, 0, 0);
+        if (nx.row < rows_pad) load(nx, gn, un);
         const int64_t row = it.row;
         const int64_t c0 = it.chunk * CHUNK;
         if (row >= M) {
             zero_pad_scales(mq, row, c0);
             if (has_gq) zero_pad_scales(gq, row, c0);
             if (has_uq) zero_pad_scales(uq, row, c0);
-            continue;
-        }
-        const int64_t c = c0 + 8 * lane;
-        const bool valid = c < I;
-        float gv[8] = {0, 0, 0, 0, 0, 0, 0, 0}, uv[8] = {0, 0, 0, 0, 0, 0, 0, 0}, mv[8];
-        if (valid) {
-            load8_bf16(g + row * ld_gu + c, gv);
-            load8_bf16(u + row * ld_gu + c, uv);
-        }
+        } else {
+            const int64_t c = c0 + 8 * lane;
+            const bool valid = c < I;
+            float gv[8], uv[8], mv[8];
+            unpack8_bf16(gr, gv);
+            unpack8_bf16(ur, uv);
 #pragma unroll
-        for (int i = 0; i < 8; ++i) mv[i] = valid ? silu_mul_out(gv[i], uv[i]) : 0.0f;
-        if (valid && m) store8_bf16(m + row * I + c, mv);
-        uint32_t sb;
-        uint32_t codes = quant8(mv, &sb);
-        store_chunk(mq, row, c0, codes, sb, valid);
-        if (has_gq) {
-            codes = quant8(gv, &sb);
-            store_chunk(gq, row, c0, codes, sb, valid);
+            for (int i = 0; i < 8; ++i) mv[i] = valid ? silu_mul_out(gv[i], uv[i]) : 0.0f;
+            if (valid && m) store8_bf16(m + row * I + c, mv);
+            uint32_t sb;
+            uint32_t codes = quant8(mv, &sb);
+            store_chunk(mq, row, c0, codes, sb, valid);
+            if (has_gq) {
+                codes = quant8(gv, &sb);
+                store_chunk(gq, row, c0, codes, sb, valid);
+            }
+            if (has_uq) {
+                codes = quant8(uv, &sb);
+                store_chunk(uq, row, c0, codes, sb, valid);
+            }
         }
-        if (has_uq) {
-            codes = quant8(uv, &sb);
-            store_chunk(uq, row, c0, codes, sb, valid);
-        }
+        it = nx;
+        gr = gn;
+        ur = un;
     }
 }
 
@@ -225,44 +261,67 @@ __global__ void __launch_bounds__(256) k_silu_mul_bwd_quant(const pact_bf16 *__r
     const int64_t rows_pad = (M + 127) & ~int64_t(127);
     const int64_t warp0 = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
     const int64_t nwarps = (int64_t)gridDim.x * (blockDim.x >> 5);
-    for (TaskIter it(warp0, nchunk, nwarps); it.row < rows_pad; it.next()) {
+    struct In {
+        uint4 d;
+        uint32_t gc, uc, gs, us;
+    };
+    auto load = [&](const TaskIter &t, In &v) {
+        const int64_t c = t.chunk * CHUNK + 8 * lane;
+        v.d = make_uint4(0, 0, 0, 0);
+        v.gc = v.uc = v.gs = v.us = 0;
+        if (t.row < M && c < I) {
+            v.d = *reinterpret_cast<const uint4 *>(dm + t.row * lddm + c);
+            // gq and uq share their shape: one code offset, one scale offset
+            const int64_t co = t.row * (I >> 1) + (c >> 1), so = scale_offset(t.row, c >> 4, I);
+            v.gc = *reinterpret_cast<const uint32_t *>(static_cast<const uint8_t *>(gq.codes) + co);
+            v.uc = *reinterpret_cast<const uint32_t *>(static_cast<const uint8_t *>(uq.codes) + co);
+            v.gs = static_cast<const uint8_t *>(gq.scales)[so];
+            v.us = static_cast<const uint8_t *>(uq.scales)[so];
+        }
+    };
+    TaskIter it(warp0, nchunk, nwarps);
+    In cur;
+    if (it.row < rows_pad) load(it, cur);
+    while (it.row < rows_pad) {
+        TaskIter nx = it;
+        nx.next();
+        In nxt;
+        nxt.d = make_uint4(0, 0, 0, 0);
+        nxt.gc = nxt.uc = nxt.gs = nxt.us = 0;
+        if (nx.row < rows_pad) load(nx, nxt);
         const int64_t row = it.row;
         const int64_t c0 = it.chunk * CHUNK;
         if (row >= M) {
             zero_pad_scales(dguq, row, c0);
             zero_pad_scales(dguq, row, c0 + I);
-            continue;
-        }
-        const int64_t c = c0 + 8 * lane;
-        const bool valid = c < I;
-        float d[8] = {0, 0, 0, 0, 0, 0, 0, 0}, gh[8] = {0, 0, 0, 0, 0, 0, 0, 0}, uh[8] = {0, 0, 0, 0, 0, 0, 0, 0};
-        if (valid) {
-            load8_bf16(dm + row * lddm + c, d);
-            // gq and uq share their shape: one code offset, one scale offset
-            const int64_t co = row * (I >> 1) + (c >> 1), so = scale_offset(row, c >> 4, I);
-            dequant8(*reinterpret_cast<const uint32_t *>(static_cast<const uint8_t *>(gq.codes) + co),
-                     static_cast<const uint8_t *>(gq.scales)[so], gh);
-            dequant8(*reinterpret_cast<const uint32_t *>(static_cast<const uint8_t *>(uq.codes) + co),
-                     static_cast<const uint8_t *>(uq.scales)[so], uh);
-        }
-        float dg[8], du[8], mr[8];
+        } else {
+            const int64_t c = c0 + 8 * lane;
+            const bool valid = c < I;
+            float d[8], gh[8], uh[8];
+            unpack8_bf16(cur.d, d);
+            dequant8(cur.gc, cur.gs, gh);
+            dequant8(cur.uc, cur.us, uh);
+            float dg[8], du[8], mr[8];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            const float s = sigmoid_fast(gh[i]);
-            dg[i] = __bfloat162float(__float2bfloat16_rn(d[i] * uh[i] * s * (1.0f + gh[i] * (1.0f - s))));
-            du[i] = __bfloat162float(__float2bfloat16_rn(d[i] * gh[i] * s));
-            mr[i] = valid ? silu_mul_round(gh[i], uh[i], s) : 0.0f;
+            for (int i = 0; i < 8; ++i) {
+                const float sg = sigmoid_fast(gh[i]);
+                dg[i] = __bfloat162float(__float2bfloat16_rn(d[i] * uh[i] * sg * (1.0f + gh[i] * (1.0f - sg))));
+                du[i] = __bfloat162float(__float2bfloat16_rn(d[i] * gh[i] * sg));
+                mr[i] = valid ? silu_mul_round(gh[i], uh[i], sg) : 0.0f;
+            }
+            if (valid) {
+                store8_bf16(dgu + row * lddgu + c, dg);
+                store8_bf16(dgu + row * lddgu + I + c, du);
+                if (m_re) store8_bf16(m_re + row * I + c, mr);
+            }
+            uint32_t sb;
+            uint32_t codes = quant8(dg, &sb);
+            store_chunk(dguq, row, c0, codes, sb, valid);
+            codes = quant8(du, &sb);
+            store_chunk(dguq, row, c0 + I, codes, sb, valid);
         }
-        if (valid) {
-            store8_bf16(dgu + row * lddgu + c, dg);
-            store8_bf16(dgu + row * lddgu + I + c, du);
-            if (m_re) store8_bf16(m_re + row * I + c, mr);
-        }
-        uint32_t sb;
-        uint32_t codes = quant8(dg, &sb);
-        store_chunk(dguq, row, c0, codes, sb, valid);
-        codes = quant8(du, &sb);
-        store_chunk(dguq, row, c0 + I, codes, sb, valid);
+        it = nx;
+        cur = nxt;
     }
 }
 

@@ -35,8 +35,8 @@ __device__ __forceinline__ uint32_t e2m1x2_to_f16x2(uint32_t byte) {
     return r;
 }
 
-// |x| / s as the correctly rounded FP32 quotient would decide it, from the correctly
-// rounded reciprocal r = 1/s: one product and one residual correction (Markstein,
+// x / s as the correctly rounded FP32 quotient would decide it (for either sign of
+// x: every step is symmetric in sign), from the correctly rounded reciprocal r = 1/s: one product and one residual correction (Markstein,
 // "Computation of elementary functions on the IBM RISC System/6000 processor",
 // IBM J. Res. Dev. 34(1), 1990).  For BF16 |x| and E4M3 s this reproduces every
 // rounding decision of the exact quotient (checked over all pairs by the tests).
@@ -44,15 +44,6 @@ __device__ __forceinline__ float quotient(float a, float s, float r) {
     float q0 = __fmul_rn(a, r);
     float e = __fmaf_rn(-q0, s, a);
     return __fmaf_rn(e, r, q0);
-}
-
-// Two non-negative values -> one byte of two E2M1 magnitude codes (lo in bits 0..3).
-__device__ __forceinline__ uint32_t e2m1x2(float lo, float hi) {
-    uint16_t r;
-    asm("{\n\t.reg .b8 t;\n\tcvt.rn.satfinite.e2m1x2.f32 t, %1, %2;\n\tcvt.u16.u8 %0, t;\n\t}"
-        : "=h"(r)
-        : "f"(hi), "f"(lo));
-    return r & 0xFFu;
 }
 
 // amax -> E4M3 scale byte: RNE(amax / 6) with saturation.  The product with the
@@ -67,7 +58,9 @@ __device__ __forceinline__ uint32_t scale_byte(float amax) {
 // Quantize the 8 values of this lane (v[0] is the lowest column); the partner lane
 // (lane ^ 1) holds the other half of the block.  All 32 lanes must call this.
 // Returns the 4 code bytes (element 0 in the low nibble of byte 0); *sb gets the
-// block's scale byte (identical in both lanes of the pair).
+// block's scale byte (identical in both lanes of the pair).  The quotients keep the
+// sign of x (a -0 quotient of a -0 input included), and the hardware conversion
+// rounds the magnitude and keeps the sign bit.
 __device__ __forceinline__ uint32_t quant8(const float (&v)[8], uint32_t *sb) {
     float amax = 0.0f;
 #pragma unroll
@@ -76,14 +69,18 @@ __device__ __forceinline__ uint32_t quant8(const float (&v)[8], uint32_t *sb) {
     const uint32_t b = scale_byte(amax);
     const float s = e4m3_to_float(b);
     const float r = b ? __frcp_rn(s) : 0.0f;
-    uint32_t out = 0;
+    float q[8];
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        const float x0 = v[2 * i], x1 = v[2 * i + 1];
-        uint32_t byte = e2m1x2(quotient(fabsf(x0), s, r), quotient(fabsf(x1), s, r));
-        byte |= ((__float_as_uint(x0) >> 31) << 3) | ((__float_as_uint(x1) >> 31) << 7);
-        out |= byte << (8 * i);
-    }
+    for (int i = 0; i < 8; ++i) q[i] = copysignf(quotient(v[i], s, r), v[i]);
+    uint32_t out;
+    asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b0, %2, %1;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b1, %4, %3;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b2, %6, %5;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b3, %8, %7;\n\t"
+        "mov.b32 %0, {b0, b1, b2, b3};\n\t}"
+        : "=r"(out)
+        : "f"(q[0]), "f"(q[1]), "f"(q[2]), "f"(q[3]), "f"(q[4]), "f"(q[5]), "f"(q[6]), "f"(q[7]));
     *sb = b;
     return out;
 }
