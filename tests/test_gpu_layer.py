@@ -206,6 +206,16 @@ def test_layer_small_all_rows(orc, small_layer, graphs):
     check_layer(L, inp, orc, rows=None)
 
 
+@pytest.mark.parametrize("name", ["qwen2.5-1.5b", "llama-3.2-3b"])
+def test_layer_full_size(orc, name):
+    """The other two layer workloads (Qwen2.5-1.5B at 2048 tokens; Llama-3.2-3B at
+    8192 tokens with 1% x20 weight outliers) in the bench's launch configuration."""
+    L, inp = run_layer(name, synth.tokens(name), graphs=True)
+    rows = np.sort(np.random.default_rng(12).choice(L.s.M, size=32, replace=False))
+    rows[-1] = L.s.M - 1
+    check_layer(L, inp, orc, rows=rows)
+
+
 def test_layer_llama1b_full_size(orc):
     """The bench workload itself, in the bench's launch configuration."""
     L, inp = run_layer("llama-3.2-1b", synth.tokens("llama-3.2-1b"), graphs=True)
