@@ -123,6 +123,53 @@ class ClockSampler:
                 "reasons": sorted(reasons), "samples": len(sm)}
 
 
+# ------------------------------------------------------------------ data-parallel replicas
+class Replicas:
+    """The host side of a multi-GPU run: one process per GPU (torchrun's RANK,
+    WORLD_SIZE, LOCAL_RANK), each a full replica of the layer step on its own
+    tokens.  The only exchange is the sum of the LoRA weight gradients; timings are
+    reduced to their maximum over ranks; rank 0 alone prints.  `backend` is "nccl"
+    on GPUs ("gloo" runs the same logic on CPU tensors)."""
+
+    def __init__(self, backend: str = "nccl", device=None, timeout_s: float = 120.0):
+        import datetime
+        import torch.distributed as dist
+        self.dist = dist
+        self.world = int(os.environ.get("WORLD_SIZE", "1"))
+        self.rank = int(os.environ.get("RANK", "0"))
+        self.device = device
+        if self.world > 1 and not dist.is_initialized():
+            kw = {"device_id": device} if backend == "nccl" and device is not None else {}
+            dist.init_process_group(backend, timeout=datetime.timedelta(seconds=timeout_s), **kw)
+
+    def allreduce_grads(self, grads):
+        """Sum each gradient tensor over the ranks, in place (same order on every rank)."""
+        if self.world > 1:
+            for g in grads:
+                self.dist.all_reduce(g)
+
+    def max_over_ranks(self, value: float) -> float:
+        if self.world == 1:
+            return value
+        import torch
+        t = torch.tensor([value], dtype=torch.float64, device=self.device if self.device is not None else "cpu")
+        self.dist.all_reduce(t, op=self.dist.ReduceOp.MAX)
+        return float(t.item())
+
+    def barrier(self):
+        if self.world > 1:
+            self.dist.barrier()
+
+    def emit(self, line: dict):
+        """Print the JSON line on rank 0 only."""
+        if self.rank == 0:
+            print(json.dumps(line), flush=True)
+
+    def close(self):
+        if self.world > 1 and self.dist.is_initialized():
+            self.dist.destroy_process_group()
+
+
 # ------------------------------------------------------------------ CPU oracle
 def oracle_layer(name, inputs):
     import oracle
@@ -307,19 +354,15 @@ def main():
         return gemm_sweep(a, [(n, k, m) for (n, k) in synth.SWEEP_NK for m in synth.SWEEP_M])
 
     import torch
-    import torch.distributed as dist
 
     import synth
     import nvfp4_gemm_b200 as P
 
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
-    if world > 1:
-        import datetime
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+    rep = Replicas("nccl", dev)
+    world, rank = rep.world, rep.rank
 
     M = synth.tokens(a.workload)
     inputs, layer, x_in = make_layer(a.workload, dev)
@@ -363,9 +406,7 @@ def main():
     grads = list(layer.grads.values())
 
     def allreduce_grads():
-        if world > 1:
-            for gt in grads:
-                dist.all_reduce(gt)
+        rep.allreduce_grads(grads)
 
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
     with torch.cuda.stream(stream):
@@ -378,8 +419,7 @@ def main():
     K = a.steps
     ev = lambda: torch.cuda.Event(enable_timing=True)
     st_ev = [(ev(), ev()) for _ in range(K)]
-    if world > 1:
-        dist.barrier()
+    rep.barrier()
     torch.cuda.synchronize()
     with ClockSampler(local) as clk:
         time.sleep(0.25)
@@ -392,8 +432,7 @@ def main():
                 st_ev[k][1].record(stream)
         torch.cuda.synchronize()
         time.sleep(0.25)
-    if world > 1:
-        dist.barrier()
+    rep.barrier()
     step_ms = [s.elapsed_time(e) for s, e in st_ev]
     total_ms = sum(step_ms)
     # breakdown (not the timed number): each segment's graph alone, after a flush
@@ -407,10 +446,7 @@ def main():
                 seg_ev[k][i][1].record(stream)
     torch.cuda.synchronize()
     seg_ms = [sum(seg_ev[k][i][0].elapsed_time(seg_ev[k][i][1]) for k in range(K)) / K for i in range(len(segs))]
-    if world > 1:
-        t = torch.tensor([total_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = rep.max_over_ranks(total_ms)
     ms_per_step = total_ms / K
     tokens_per_s = M * K * world / (total_ms / 1e3)
 
@@ -443,10 +479,7 @@ def main():
             e2e_ev[k][1].record(stream)
     torch.cuda.synchronize()
     e2e_ms = sum(s.elapsed_time(e) for s, e in e2e_ev)
-    if world > 1:
-        t = torch.tensor([e2e_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
+    e2e_ms = rep.max_over_ranks(e2e_ms)
     if P.pact_get_device_status() != 0:
         raise RuntimeError(P.pact_last_error())
 
@@ -458,33 +491,31 @@ def main():
                "sample": f"{min(a.cpu_tokens, M)} of {M} tokens per step ({n} steps, {el:.1f} s), one layer "
                          f"fwd+bwd on the FP64 CPU oracle; weight layouts cached before timing"}
 
-    if rank == 0:
-        out = {
-            "metric": METRIC, "value": tokens_per_s, "unit": "tokens/s", "n_gpus": world, "steps": K,
-            "warmup": a.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "nvfp4", "data": "synthetic",
-            "config": {**config_block(a.workload, M), "parallelism": f"dp{world}" if world > 1 else "single"},
-            "frozen_proj_tflops": tflops,
-            "frac_fp4_peak": tflops / fp4_peak,
-            "roofline": {"bound": "tensor", "kernel": "k_nvfp4_gemm (frozen fwd + dgrad GEMMs)",
-                         "achieved": tflops, "peak": fp4_peak, "unit": "TFLOP/s", "frac": tflops / fp4_peak,
-                         "traffic": None,
-                         "peak_note": f"{pk['src']} burst BF16 {pk['bf16']} TF/s x {FP4_PER_BF16} "
-                                      f"(nominal FP4/BF16 ratio); GEMM launches timed alone, cold L2",
-                         "flops_per_step": gemm_flops, "avg_launch_ms": gemm_launch_ms},
-            "cpu_baseline": cpu,
-            "e2e": {"value": M * K * world / (e2e_ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
-                    "d2h_bytes_per_step": d2h},
-            "gpu_launches": launches_per_step * K,
-            "clocks": clk.summary(),
-            "segments_ms": {"+".join(op.name for op in sg["ops"]): round(t, 4) for sg, t in zip(segs, seg_ms)},
-        }
-        print(json.dumps(out), flush=True)
+    out = {
+        "metric": METRIC, "value": tokens_per_s, "unit": "tokens/s", "n_gpus": world, "steps": K,
+        "warmup": a.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "nvfp4", "data": "synthetic",
+        "config": {**config_block(a.workload, M), "parallelism": f"dp{world}" if world > 1 else "single"},
+        "frozen_proj_tflops": tflops,
+        "frac_fp4_peak": tflops / fp4_peak,
+        "roofline": {"bound": "tensor", "kernel": "k_nvfp4_gemm (frozen fwd + dgrad GEMMs)",
+                     "achieved": tflops, "peak": fp4_peak, "unit": "TFLOP/s", "frac": tflops / fp4_peak,
+                     "traffic": None,
+                     "peak_note": f"{pk['src']} burst BF16 {pk['bf16']} TF/s x {FP4_PER_BF16} "
+                                  f"(nominal FP4/BF16 ratio); GEMM launches timed alone, cold L2",
+                     "flops_per_step": gemm_flops, "avg_launch_ms": gemm_launch_ms},
+        "cpu_baseline": cpu,
+        "e2e": {"value": M * K * world / (e2e_ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h},
+        "gpu_launches": launches_per_step * K,
+        "clocks": clk.summary(),
+        "segments_ms": {"+".join(op.name for op in sg["ops"]): round(t, 4) for sg, t in zip(segs, seg_ms)},
+    }
+    rep.emit(out)
     for sg in segs:
         sg["graph"] = None
-    step_graph = None
-    if world > 1:
-        dist.destroy_process_group()
+    step_graph = None   # release every graph before the process group
+    rep.close()
 
 
 if __name__ == "__main__":
