@@ -32,11 +32,38 @@ enum : uint32_t { STATUS_TIMEOUT = 1u };
 // Validate an NVFP4 descriptor of the given shape.
 pact_status check_nvfp4(const pact_nvfp4_t *t, int64_t rows, int64_t cols, const char *name);
 
+// Launch with programmatic stream serialization: the kernel may be scheduled while
+// the previous kernel on the stream drains; it runs its prologue and then waits in
+// pdl_wait() (griddepcontrol.wait) for that kernel's completion before it touches
+// global memory.  Every libpact kernel calls pdl_wait() before its first global
+// access, so the order of results is that of plain stream order.
+template <typename... KArgs, typename... Args>
+pact_status launch_dep(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                       const char *what, Args &&...args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
+    if (e != cudaSuccess) return fail(PACT_ERR_CUDA, "%s: launch failed: %s", what, cudaGetErrorString(e));
+    return launch_status(what);
+}
+
 // ------------------------------------------------------------------ device side
 // Per-device status word (the library is built as one translation unit).
 __device__ uint32_t g_status = 0;
 
 __device__ __forceinline__ void record_timeout() { atomicOr(&g_status, STATUS_TIMEOUT); }
+
+// Wait for the kernels this one depends on (programmatic dependent launch); a no-op
+// when the kernel was launched without such a dependency.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 
 __device__ __forceinline__ uint64_t globaltimer() {
     uint64_t t;

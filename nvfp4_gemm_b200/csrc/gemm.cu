@@ -160,6 +160,7 @@ k_nvfp4_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CU
     __syncthreads();
     cluster_sync();  // the peer's barriers exist before anything addresses them
     tc_fence_after();
+    pdl_wait();      // inputs of the previous kernel are complete from here on
     const uint32_t tmem = *tmem_slot;
 
     if (warp == 0) {
@@ -546,8 +547,8 @@ static pact_status run(const pact_nvfp4_t *a, const pact_nvfp4_t *b, const pact_
     }
     const int pairs = (int)(((M + 255) / 256) * ((N + 255) / 256));
     const int clusters = pairs < sm_count() / 2 ? pairs : sm_count() / 2;
-    k_nvfp4_gemm<<<2 * clusters, THREADS, SMEM_BYTES, stream>>>(tmA, tmB, tmSFA, tmSFB, tmLa, tmLb, tmD, tmR, p);
-    return launch_status(what);
+    return launch_dep(k_nvfp4_gemm, dim3(2 * clusters), dim3(THREADS), SMEM_BYTES, stream, what, tmA, tmB, tmSFA, tmSFB,
+                      tmLa, tmLb, tmD, tmR, p);
 }
 
 }  // namespace gemm

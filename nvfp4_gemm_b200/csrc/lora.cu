@@ -61,6 +61,7 @@ k_lora_mma(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUte
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
     if (ktiles == 0) {  // empty split: its partial is zero
+        pdl_wait();
         for (int i = threadIdx.x; i < BM * p.n_valid; i += THREADS) {
             const int r = row0 + i / p.n_valid;
             if (r < pr.row_end) part[(size_t)r * p.ws_ld + pr.out_col + i % p.n_valid] = 0.0f;
@@ -92,6 +93,7 @@ k_lora_mma(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUte
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
+    pdl_wait();   // inputs of the previous kernel are complete from here on
     const uint32_t tmem = *tmem_slot;
     const int nparts = p.b_split ? 2 : 1;
     const uint32_t b_bytes = B_MN ? (uint32_t)B_BYTES : (uint32_t)p.n_mma * BK * 2;
@@ -183,6 +185,7 @@ k_lora_mma(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUte
 __global__ void k_finalize(const float *__restrict__ ws, int splits, int64_t split_stride, int64_t ws_ld, int64_t rows,
                            int64_t cols, float scale, int mode, pact_bf16 *__restrict__ out, int64_t ldo,
                            int64_t lo_off) {
+    pdl_wait();
     const int64_t n = rows * cols;
     for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x) {
         const int64_t r = mode == 2 ? i % rows : i / cols, c = mode == 2 ? i / rows : i % cols;
@@ -202,6 +205,7 @@ __global__ void k_finalize(const float *__restrict__ ws, int splits, int64_t spl
 
 // NVFP4 -> BF16 (exact): the backward's view of a saved activation copy.
 __global__ void k_dequantize(pact_nvfp4_t t, pact_bf16 *__restrict__ out) {
+    pdl_wait();
     const int64_t per_row = t.cols / 8;
     const int64_t n8 = t.rows * per_row;
     for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n8; i += (int64_t)gridDim.x * blockDim.x) {
@@ -254,8 +258,7 @@ static pact_status launch_mma(const CUtensorMap &ta, const CUtensorMap &tb, cons
         done[d] = true;
     }
     dim3 grid((unsigned)row_tiles, (unsigned)p.splits, (unsigned)p.nprob);
-    k_lora_mma<A_MN, B_MN><<<grid, THREADS, SMEM_BYTES, st>>>(ta, tb, p);
-    return launch_status(what);
+    return launch_dep(k_lora_mma<A_MN, B_MN>, grid, dim3(THREADS), SMEM_BYTES, st, what, ta, tb, p);
 }
 
 // Split a contraction of length `len` over CTAs so that `blocks` output blocks x
@@ -303,8 +306,8 @@ static pact_status rows_times_a(const CUtensorMap &tx, int64_t M, int64_t K, con
     p.ws_split_stride = M * R;
     s = launch_mma<false, false>(tx, tb, p, tiles, st, what);
     if (s != PACT_OK) return s;
-    k_finalize<<<finalize_grid(M * R), 256, 0, st>>>(ws, p.splits, M * R, R, M, R, scale, 0, out, ldo, R);
-    return launch_status(what);
+    return launch_dep(k_finalize, dim3(finalize_grid(M * R)), dim3(256), 0, st, what, (const float *)ws, p.splits,
+                      (int64_t)(M * R), (int64_t)R, (int64_t)M, (int64_t)R, scale, 0, out, ldo, (int64_t)R);
 }
 
 static pact_status check_segments(int64_t N, int nseg, const int64_t *seg_end, const char *what) {
@@ -397,8 +400,8 @@ pact_status pact_lora_bwd_u(const pact_bf16 *dy, int64_t lddy, int64_t M, int64_
     p.ws_split_stride = M * R;
     s = launch_mma<false, true>(ta, tb, p, tiles, st, "pact_lora_bwd_u");
     if (s != PACT_OK) return s;
-    k_finalize<<<finalize_grid(M * R), 256, 0, st>>>(ws, p.splits, M * R, R, M, R, scale, 0, U, ldu, R);
-    return launch_status("pact_lora_bwd_u");
+    return launch_dep(k_finalize, dim3(finalize_grid(M * R)), dim3(256), 0, st, "pact_lora_bwd_u", (const float *)ws,
+                      p.splits, (int64_t)(M * R), (int64_t)R, (int64_t)M, (int64_t)R, scale, 0, U, ldu, (int64_t)R);
 }
 
 // Upper bound over segmentations: the dB output blocks number at least N / 128.
@@ -450,8 +453,7 @@ pact_status pact_lora_bwd(const pact_lora_bwd_t *g, void *workspace, size_t ws_b
     const pact_bf16 *x = g->x;
     int64_t ldx = g->ldx;
     if (g->xq) {
-        k_dequantize<<<finalize_grid(M * K / 8), 256, 0, st>>>(*g->xq, xt);
-        s = launch_status("pact_lora_bwd");
+        s = launch_dep(k_dequantize, dim3(finalize_grid(M * K / 8)), dim3(256), 0, st, "pact_lora_bwd", *g->xq, xt);
         if (s != PACT_OK) return s;
         x = xt;
         ldx = K;
@@ -488,8 +490,9 @@ pact_status pact_lora_bwd(const pact_lora_bwd_t *g, void *workspace, size_t ws_b
         p.ws_split_stride = N * r;
         s = launch_mma<true, true>(ta, tb, p, (int)((widest + BM - 1) / BM), st, "pact_lora_bwd");
         if (s != PACT_OK) return s;
-        k_finalize<<<finalize_grid(N * r), 256, 0, st>>>(ws_db, p.splits, N * r, r, N, r, g->scale, 1, g->dB, r, 0);
-        s = launch_status("pact_lora_bwd");
+        s = launch_dep(k_finalize, dim3(finalize_grid(N * r)), dim3(256), 0, st, "pact_lora_bwd", (const float *)ws_db,
+                       p.splits, (int64_t)(N * r), (int64_t)r, (int64_t)N, (int64_t)r, g->scale, 1, g->dB, (int64_t)r,
+                       (int64_t)0);
         if (s != PACT_OK) return s;
     }
     // dA^T = X~^T . U  [K x R], U = hi + lo
@@ -511,8 +514,8 @@ pact_status pact_lora_bwd(const pact_lora_bwd_t *g, void *workspace, size_t ws_b
     p.ws_split_stride = K * R;
     s = launch_mma<true, true>(ta, tb, p, tiles, st, "pact_lora_bwd");
     if (s != PACT_OK) return s;
-    k_finalize<<<finalize_grid(K * R), 256, 0, st>>>(ws_da, p.splits, K * R, R, K, R, 1.0f, 2, g->dA, K, 0);
-    return launch_status("pact_lora_bwd");
+    return launch_dep(k_finalize, dim3(finalize_grid(K * R)), dim3(256), 0, st, "pact_lora_bwd", (const float *)ws_da,
+                      p.splits, (int64_t)(K * R), (int64_t)R, (int64_t)K, (int64_t)R, 1.0f, 2, g->dA, K, (int64_t)0);
 }
 
 }  // extern "C"

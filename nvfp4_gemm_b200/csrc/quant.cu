@@ -28,6 +28,7 @@ __device__ __forceinline__ void unpack8_bf16(const uint4 &u, float (&v)[8]) {
 // ------------------------------------------------------------------ A2: quantize
 __global__ void __launch_bounds__(256) k_quantize(const pact_bf16 *__restrict__ x, int64_t ldx, int64_t rows,
                                                   pact_nvfp4_t out) {
+    pdl_wait();
     const int lane = threadIdx.x & 31;
     const int64_t nchunk = (out.cols + CHUNK - 1) / CHUNK;
     const int64_t rows_pad = (rows + 127) & ~int64_t(127);
@@ -112,6 +113,7 @@ __global__ void __launch_bounds__(RMS_THREADS, 2) k_rmsnorm_quant(const pact_bf1
                                                                const pact_bf16 *__restrict__ gamma, float eps,
                                                                int64_t M, int64_t H, pact_nvfp4_t yq,
                                                                pact_bf16 *__restrict__ y, float *__restrict__ rstd_out) {
+    pdl_wait();
     __shared__ double red[RMS_WARPS];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int wr = warp % WPR;                                       // warp within the row group
@@ -197,6 +199,7 @@ __global__ void __launch_bounds__(256) k_silu_mul_quant(const pact_bf16 *__restr
                                                         int64_t ld_gu, int64_t M, int64_t I,
                                                         pact_bf16 *__restrict__ m, pact_nvfp4_t mq, pact_nvfp4_t gq,
                                                         pact_nvfp4_t uq, int has_gq, int has_uq) {
+    pdl_wait();
     const int lane = threadIdx.x & 31;
     const int64_t nchunk = (I + CHUNK - 1) / CHUNK;
     const int64_t rows_pad = (M + 127) & ~int64_t(127);
@@ -256,6 +259,7 @@ __global__ void __launch_bounds__(256) k_silu_mul_bwd_quant(const pact_bf16 *__r
                                                             pact_nvfp4_t gq, pact_nvfp4_t uq, int64_t M, int64_t I,
                                                             pact_bf16 *__restrict__ dgu, int64_t lddgu,
                                                             pact_nvfp4_t dguq, pact_bf16 *__restrict__ m_re) {
+    pdl_wait();
     const int lane = threadIdx.x & 31;
     const int64_t nchunk = (I + CHUNK - 1) / CHUNK;
     const int64_t rows_pad = (M + 127) & ~int64_t(127);
@@ -334,6 +338,7 @@ __global__ void __launch_bounds__(RMS_THREADS, 2) k_rmsnorm_bwd(const pact_bf16 
                                                              const pact_bf16 *__restrict__ gamma, int64_t M, int64_t H,
                                                              const pact_bf16 *__restrict__ dres,
                                                              pact_bf16 *__restrict__ dx, pact_nvfp4_t dxq, int has_dxq) {
+    pdl_wait();
     __shared__ float red[RMS_WARPS];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int wr = warp % WPR;
@@ -410,6 +415,7 @@ __global__ void __launch_bounds__(RMS_THREADS, 2) k_rmsnorm_bwd(const pact_bf16 
 // Wb = q(deq(Wf)^T): a CTA turns a 64 (n) x 64 (k) tile of the forward layout into
 // 64 rows (k) x 4 blocks (n) of the backward layout.  Runs once per frozen weight.
 __global__ void __launch_bounds__(256) k_weight_bwd_layout(pact_nvfp4_t wf, pact_nvfp4_t wb) {
+    pdl_wait();
     __shared__ float tile[64][65];
     const int64_t n0 = (int64_t)blockIdx.y * 64, k0 = (int64_t)blockIdx.x * 64;
     const int t = threadIdx.x;
@@ -457,6 +463,7 @@ __global__ void __launch_bounds__(256) k_weight_bwd_layout(pact_nvfp4_t wf, pact
 
 // Zero scale rows [rows, round_up(rows, 128)) of a tensor (the layout's padding).
 __global__ void k_zero_scale_pad(pact_nvfp4_t t) {
+    pdl_wait();
     const int64_t rows_pad = (t.rows + 127) & ~int64_t(127);
     const int64_t nblk = t.cols >> 4;
     const int64_t n = (rows_pad - t.rows) * nblk;
@@ -496,8 +503,8 @@ pact_status pact_quantize_nvfp4(const pact_bf16 *x, int64_t ldx, int64_t rows, i
     pact_status s = check_nvfp4(out, rows, cols, "out");
     if (s != PACT_OK) return s;
     const int64_t tasks = ((rows + 127) / 128 * 128) * ((cols + CHUNK - 1) / CHUNK);
-    k_quantize<<<grid_for(tasks, 256), 256, 0, (cudaStream_t)stream>>>(x, ldx, rows, *out);
-    return launch_status("pact_quantize_nvfp4");
+    return launch_dep(k_quantize, dim3(grid_for(tasks, 256)), dim3(256), 0, (cudaStream_t)stream, "pact_quantize_nvfp4",
+                      x, ldx, rows, *out);
 }
 
 pact_status pact_rmsnorm_quant(const pact_bf16 *x, int64_t ldx, const pact_bf16 *gamma, float eps, int64_t M,
@@ -516,7 +523,9 @@ pact_status pact_rmsnorm_quant(const pact_bf16 *x, int64_t ldx, const pact_bf16 
     cudaStream_t st = (cudaStream_t)stream;
     const int wpr = rms_wpr(H), nch = rms_nch(H);
     const unsigned grid = (unsigned)(rows_pad / (RMS_WARPS / wpr));
-#define PACT_RMS_FWD(NC, WP) k_rmsnorm_quant<NC, WP><<<grid, RMS_THREADS, 0, st>>>(x, ldx, gamma, eps, M, H, *yq, y, rstd)
+#define PACT_RMS_FWD(NC, WP) \
+    s = launch_dep(k_rmsnorm_quant<NC, WP>, dim3(grid), dim3(RMS_THREADS), 0, st, "pact_rmsnorm_quant", x, ldx, gamma, eps, \
+                   M, H, *yq, y, rstd)
     if (wpr == 1) {
         switch (nch) {
             case 1: PACT_RMS_FWD(1, 1); break;
@@ -532,7 +541,7 @@ pact_status pact_rmsnorm_quant(const pact_bf16 *x, int64_t ldx, const pact_bf16 
         PACT_RMS_FWD(8, 8);
     }
 #undef PACT_RMS_FWD
-    return launch_status("pact_rmsnorm_quant");
+    return s;
 }
 
 pact_status pact_silu_mul_quant(const pact_bf16 *g, const pact_bf16 *u, int64_t ld_gu, int64_t M, int64_t I,
@@ -549,9 +558,9 @@ pact_status pact_silu_mul_quant(const pact_bf16 *g, const pact_bf16 *u, int64_t 
     if (s != PACT_OK) return s;
     pact_nvfp4_t none = {nullptr, nullptr, M, I};
     const int64_t tasks = ((M + 127) / 128 * 128) * ((I + CHUNK - 1) / CHUNK);
-    k_silu_mul_quant<<<grid_for(tasks, 256), 256, 0, (cudaStream_t)stream>>>(
-        g, u, ld_gu, M, I, m, *mq, gq ? *gq : none, uq ? *uq : none, gq != nullptr, uq != nullptr);
-    return launch_status("pact_silu_mul_quant");
+    return launch_dep(k_silu_mul_quant, dim3(grid_for(tasks, 256)), dim3(256), 0, (cudaStream_t)stream,
+                      "pact_silu_mul_quant", g, u, ld_gu, M, I, m, *mq, gq ? *gq : none, uq ? *uq : none,
+                      (int)(gq != nullptr), (int)(uq != nullptr));
 }
 
 pact_status pact_silu_mul_bwd_quant(const pact_bf16 *dm, int64_t lddm, const pact_nvfp4_t *gq, const pact_nvfp4_t *uq,
@@ -568,9 +577,8 @@ pact_status pact_silu_mul_bwd_quant(const pact_bf16 *dm, int64_t lddm, const pac
     if (s == PACT_OK) s = check_nvfp4(dguq, M, 2 * I, "dguq");
     if (s != PACT_OK) return s;
     const int64_t tasks = ((M + 127) / 128 * 128) * ((I + CHUNK - 1) / CHUNK);
-    k_silu_mul_bwd_quant<<<grid_for(tasks, 256), 256, 0, (cudaStream_t)stream>>>(dm, lddm, *gq, *uq, M, I, dgu, lddgu,
-                                                                                *dguq, m_re);
-    return launch_status("pact_silu_mul_bwd_quant");
+    return launch_dep(k_silu_mul_bwd_quant, dim3(grid_for(tasks, 256)), dim3(256), 0, (cudaStream_t)stream,
+                      "pact_silu_mul_bwd_quant", dm, lddm, *gq, *uq, M, I, dgu, lddgu, *dguq, m_re);
 }
 
 pact_status pact_rmsnorm_bwd(const pact_bf16 *dy, int64_t lddy, const pact_nvfp4_t *yq, const float *rstd,
@@ -593,7 +601,8 @@ pact_status pact_rmsnorm_bwd(const pact_bf16 *dy, int64_t lddy, const pact_nvfp4
     const int64_t per_cta = RMS_WARPS / wpr;
     const unsigned grid = (unsigned)((rows + per_cta - 1) / per_cta);
 #define PACT_RMS_BWD(NC, WP) \
-    k_rmsnorm_bwd<NC, WP><<<grid, RMS_THREADS, 0, st>>>(dy, lddy, *yq, rstd, gamma, M, H, dres, dx, q, has)
+    s = launch_dep(k_rmsnorm_bwd<NC, WP>, dim3(grid), dim3(RMS_THREADS), 0, st, "pact_rmsnorm_bwd", dy, lddy, *yq, rstd, \
+                   gamma, M, H, dres, dx, q, has)
     if (wpr == 1) {
         switch (nch) {
             case 1: PACT_RMS_BWD(1, 1); break;
@@ -609,7 +618,7 @@ pact_status pact_rmsnorm_bwd(const pact_bf16 *dy, int64_t lddy, const pact_nvfp4
         PACT_RMS_BWD(8, 8);
     }
 #undef PACT_RMS_BWD
-    return launch_status("pact_rmsnorm_bwd");
+    return s;
 }
 
 pact_status pact_weight_layout_cache(const pact_bf16 *W, int64_t ldw, int64_t N, int64_t K, void *buf, size_t bytes,
@@ -633,12 +642,11 @@ pact_status pact_weight_layout_cache(const pact_bf16 *W, int64_t ldw, int64_t N,
     pact_status s = pact_quantize_nvfp4(W, ldw, N, K, &c.fwd, stream);
     if (s != PACT_OK) return s;
     dim3 grid((unsigned)(K / 64), (unsigned)(N / 64));
-    k_weight_bwd_layout<<<grid, 256, 0, (cudaStream_t)stream>>>(c.fwd, c.bwd);
-    s = launch_status("pact_weight_layout_cache");
+    s = launch_dep(k_weight_bwd_layout, grid, dim3(256), 0, (cudaStream_t)stream, "pact_weight_layout_cache", c.fwd,
+                   c.bwd);
     if (s != PACT_OK) return s;
     if (K % 128) {
-        k_zero_scale_pad<<<64, 256, 0, (cudaStream_t)stream>>>(c.bwd);
-        s = launch_status("pact_weight_layout_cache");
+        s = launch_dep(k_zero_scale_pad, dim3(64), dim3(256), 0, (cudaStream_t)stream, "pact_weight_layout_cache", c.bwd);
         if (s != PACT_OK) return s;
     }
     *out = c;
