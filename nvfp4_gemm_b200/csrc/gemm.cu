@@ -16,13 +16,17 @@
 //    leader (rank 0) issues every MMA for the pair.  Each SM streams 38 KiB per
 //    K = 256 stage, 30% less than a single-CTA 128 x 256 tile needs, which keeps
 //    the L2 -> shared-memory stream below what the tensor core consumes.
-//  * warp 0 (both CTAs): TMA producer into a 4-stage ring.  Operand tiles complete
-//    on the leader's `full` barrier (armed by the leader for both CTAs' bytes); the
-//    CTA's own scale tiles complete on its local `sf_full` barrier.
+//  * warp 0 (both CTAs): TMA producer of the operand tiles into a 4-stage ring; they
+//    complete on the leader's `full` barrier (armed by the leader for both CTAs'
+//    bytes).
+//  * warp 22 (both CTAs): scale-tile producer.  It refills a stage's scale tiles
+//    (local `sf_full` barrier) as soon as the scale writers have read the previous
+//    ones (`sf_empty`), ahead of the operand tiles.
 //  * warps 2-5 (both CTAs): scale writers.  Each moves the stage's scale tiles from
 //    shared memory into a per-stage slot of its own sub-partition's tensor memory
-//    with tcgen05.st and arrives on the leader's `full` barrier of the stage, which
-//    therefore completes only when operands and scales of both CTAs are in place.
+//    with tcgen05.st (once the slot's previous MMAs are done) and arrives on the
+//    leader's `full` barrier of the stage, which therefore completes only when
+//    operands and scales of both CTAs are in place.
 //    Writing scales from registers keeps them out of the tensor core's instruction
 //    stream; tcgen05.cp copies there serialise with the MMAs and cost more than
 //    the MMAs themselves.
@@ -59,7 +63,8 @@ constexpr int SLAB_BYTES = 32 * 128;          // 32 rows x 64 BF16 columns, 128-
 constexpr int OFF_SLABS = STAGES * STAGE_BYTES;
 constexpr int OFF_BARS = OFF_SLABS + EPI_WARPS * SLAB_BYTES;
 constexpr int SMEM_BYTES = 1024 + OFF_BARS + 512;
-constexpr int THREADS = 32 * (2 + SCALE_WARPS + EPI_WARPS);  // 704
+constexpr int SF_WARP = 2 + SCALE_WARPS + EPI_WARPS;          // 22: scale-tile producer
+constexpr int THREADS = 32 * (SF_WARP + 1);                   // 736
 static_assert(SMEM_BYTES <= 232448, "shared memory");
 
 // tensor memory columns
@@ -111,7 +116,8 @@ k_nvfp4_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CU
     uint64_t *full = bars;                        // [STAGES] leader: operands and scales of both CTAs
     uint64_t *sf_full = bars + STAGES;            // [STAGES] local: this CTA's scale tiles in shared memory
     uint64_t *empty = bars + 2 * STAGES;          // [STAGES] local: the pair's MMAs are done with the stage
-    uint64_t *acc_full = bars + 3 * STAGES;       // local: accumulator complete
+    uint64_t *sf_empty = bars + 3 * STAGES;       // [STAGES] local: the scale writers have read the scale tiles
+    uint64_t *acc_full = bars + 4 * STAGES;       // local: accumulator complete
     uint64_t *acc_empty = acc_full + 1;           // leader: all epilogue warps of both CTAs have read it
     uint64_t *drained = acc_full + 2;             // leader: every tcgen05 operation has completed
     uint64_t *res_full = acc_full + 3;            // [EPI_WARPS] local: residual block in the warp's slab
@@ -133,6 +139,7 @@ k_nvfp4_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CU
             mbar_init(&full[s], 1 + 2 * SCALE_WARPS);
             mbar_init(&sf_full[s], 1);
             mbar_init(&empty[s], 1);
+            mbar_init(&sf_empty[s], SCALE_WARPS);
         }
         mbar_init(acc_full, 1);
         mbar_init(acc_empty, 2 * EPI_WARPS);
@@ -194,25 +201,15 @@ k_nvfp4_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CU
                         }
                         for (int q = 0; q < 2; ++q) tma_load_2d_pair(st + OFF_LW + q * R * 128, &tmLb, fb, nb + 64 * q, 0);
                     }
-                    mbar_arrive(&sf_full[rg.stage]);  // a LoRA stage carries no scales
                     rg.next();
                 }
-                const int ga = m0 / 128, gb = n0 / 128;
                 for (int kt = 0; kt < ktiles; ++kt) {
                     if (!(ok = mbar_wait(&empty[rg.stage], rg.phase ^ 1))) break;
-                    uint8_t *stp = smem + rg.stage * STAGE_BYTES;
-                    const uint32_t st = smem_u32(stp);
+                    const uint32_t st = smem_u32(smem + rg.stage * STAGE_BYTES);
                     const uint32_t fb = full_leader + 8 * rg.stage;
                     if (leader) mbar_arrive_expect_tx(&full[rg.stage], 2 * (A_BYTES + B_BYTES));
                     tma_load_2d_pair(st, &tmA, fb, kt * (BK / 2), m0);
                     tma_load_2d_pair(st + OFF_B, &tmB, fb, kt * (BK / 2), nb);
-                    // scale chunks: 512 bytes = two 256-byte rows of the scale map; one box
-                    // is the 4 chunks of this K stage
-                    mbar_arrive_expect_tx(&sf_full[rg.stage], SF_BYTES);
-                    tma_load_2d(stp + OFF_SFA, &tmSFA, &sf_full[rg.stage], 0, 2 * (ga * kgroups + kt * 4));
-                    tma_load_2d(stp + OFF_SFB, &tmSFB, &sf_full[rg.stage], 0, 2 * (gb * kgroups + kt * 4));
-                    tma_load_2d(stp + OFF_SFB + 2048, &tmSFB, &sf_full[rg.stage], 0,
-                                2 * ((gb + 1) * kgroups + kt * 4));
                     rg.next();
                 }
             }
@@ -291,30 +288,79 @@ k_nvfp4_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CU
         bool ok = true;
         for (int t = cluster; ok && t < total; t += nclusters) {
             for (int i = 0; i < nsteps; ++i) {
+                const bool lstep = lora && i == 0;   // a LoRA stage carries no scales
                 if (!(ok = warp_all(mbar_wait(&sf_full[rg.stage], rg.phase)))) break;
-                if (!(lora && i == 0)) {
+                uint32_t v[48];
+                if (!lstep) {
                     // Lane j takes the 16 bytes of row j of every 512-byte chunk: the
                     // chunk's 4 scale columns for lanes j of each sub-partition, the
                     // layout the block-scaled MMA reads.
                     const uint8_t *src = smem + rg.stage * STAGE_BYTES + OFF_SFA + lane * 16;
-                    uint32_t v[48];
 #pragma unroll
                     for (int c = 0; c < 12; ++c) {  // A chunks 0-3, then B: step s, group g at 4 + 2s + g
                         const int off = c < 4 ? c * 512 : 2048 + ((c - 4) & 1) * 2048 + ((c - 4) >> 1) * 512;
                         const uint4 q = *reinterpret_cast<const uint4 *>(src + off);
                         v[4 * c] = q.x; v[4 * c + 1] = q.y; v[4 * c + 2] = q.z; v[4 * c + 3] = q.w;
                     }
+                }
+                // the tensor-memory slot is free once the pair's MMAs of its previous use
+                // are done
+                if (!(ok = warp_all(mbar_wait(&empty[rg.stage], rg.phase ^ 1)))) break;
+                if (!lstep) {
                     const uint32_t col = lane_base + COL_SF + rg.stage * SF_COLS;
                     tmem_st_32x32b_x32(col, v);
                     tmem_st_32x32b_x16(col + 32, v + 32);
                     tmem_st_wait();
                 }
+                // The scale tiles may be refilled now: their values have been consumed,
+                // and releasing them only after the previous use's MMAs are done keeps
+                // the producer within one phase of every barrier it waits on.
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&sf_empty[rg.stage]);
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive_remote_relaxed(full_leader + 8 * rg.stage);
                 rg.next();
             }
         }
+    } else if (warp == SF_WARP) {
+        // ------------------------------------------------------------ scale-tile producer (both CTAs)
+        // Refills a stage's scale tiles as soon as the scale writers have consumed the
+        // previous ones (one use earlier than the operand tiles, which wait for that
+        // use's MMAs): the TMA latency of the scales leaves the chain MMA done ->
+        // refill -> scales in tensor memory -> MMA.  After a LoRA stage (whose weight
+        // chunks overlap the scale region) it also waits for that stage's MMAs.
+        if (lane == 0) {
+            Ring rg;
+            uint32_t lora_prev = 0;   // bit s: the previous use of stage s was a LoRA stage
+            bool ok = true;
+            for (int t = cluster; ok && t < total; t += nclusters) {
+                const int mp = t % mpairs, nt = t / mpairs;
+                const int ga = (mp * 2 * BM + (int)rank * BM) / 128, gb = (nt * BN) / 128;
+                for (int i = 0; ok && i < nsteps; ++i) {
+                    const uint32_t sb = 1u << rg.stage;
+                    if (!(ok = mbar_wait(&sf_empty[rg.stage], rg.phase ^ 1))) break;
+                    if ((lora_prev & sb) && !(ok = mbar_wait(&empty[rg.stage], rg.phase ^ 1))) break;
+                    if (lora && i == 0) {
+                        mbar_arrive(&sf_full[rg.stage]);
+                        lora_prev |= sb;
+                    } else {
+                        const int kt = i - (lora ? 1 : 0);
+                        uint8_t *stp = smem + rg.stage * STAGE_BYTES;
+                        // scale chunks: 512 bytes = two 256-byte rows of the scale map; one
+                        // box is the 4 chunks of this K stage
+                        mbar_arrive_expect_tx(&sf_full[rg.stage], SF_BYTES);
+                        tma_load_2d(stp + OFF_SFA, &tmSFA, &sf_full[rg.stage], 0, 2 * (ga * kgroups + kt * 4));
+                        tma_load_2d(stp + OFF_SFB, &tmSFB, &sf_full[rg.stage], 0, 2 * (gb * kgroups + kt * 4));
+                        tma_load_2d(stp + OFF_SFB + 2048, &tmSFB, &sf_full[rg.stage], 0,
+                                    2 * ((gb + 1) * kgroups + kt * 4));
+                        lora_prev &= ~sb;
+                    }
+                    rg.next();
+                }
+            }
+        }
+        __syncwarp();
     } else {
         // ------------------------------------------------------------ epilogue (both CTAs)
         const int ew = warp - 2 - SCALE_WARPS;   // 0..15
