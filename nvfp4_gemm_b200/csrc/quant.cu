@@ -172,19 +172,17 @@ __global__ void __launch_bounds__(RMS_THREADS, 2) k_rmsnorm_quant(const pact_bf1
 // m = BF16_RNE(silu(g) * u), exactly rounded.  The FP32 evaluation with the fast
 // exponential and division has a relative error of at most (5 + 1.16 |g|) FP32
 // ulps (CUDA's documented bounds for __expf and __fdividef plus three roundings),
-// i.e. at most 2 (5 + 1.16 |g|) = 10 + 2.32 |g| ulps of the result; it decides
-// unless it lies within 12 + 3 |g| ulps of a BF16 midpoint (at most 132 for
-// |g| <= 40), and the double expression decides otherwise and for |g| > 40 (Ziv's
-// method, as above).  The margin grows with |g| so that the double path stays rare.
+// i.e. at most 2 (5 + 1.16 |g|) = 10 + 2.32 |g| ulps of the result, under 19.3
+// for |g| <= 4.  It decides unless it lies within 24 ulps of a BF16 midpoint, and
+// the double expression decides otherwise and for |g| > 4 (Ziv's method, as
+// above).  Gate activations beyond 4 in magnitude are rare, so the double path
+// stays rare, and the margin is one constant (no conversion per element).
 __device__ __forceinline__ float sigmoid_fast(float g) { return __fdividef(1.0f, 1.0f + __expf(-g)); }
 
 __device__ __forceinline__ float silu_mul_round(float g, float u, float s) {
     const float m = __fmul_rn(__fmul_rn(g, s), u);
-    const uint32_t lo = __float_as_uint(m) & 0xFFFFu;
-    const float ag = fabsf(g);
-    const uint32_t margin = 12u + (uint32_t)(3.0f * fminf(ag, 40.0f));
-    const uint32_t dist = lo >= 0x8000u ? lo - 0x8000u : 0x8000u - lo;
-    if (dist <= margin || !(ag <= 40.0f) || !isfinite(m)) {
+    const int lo = (int)(__float_as_uint(m) & 0xFFFFu);
+    if (abs(lo - 0x8000) <= 24 || !(fabsf(g) <= 4.0f) || !isfinite(m)) {
         const double gd = (double)g;
         return __bfloat162float(__double2bfloat16((gd / (1.0 + exp(-gd))) * (double)u));
     }
