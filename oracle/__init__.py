@@ -238,6 +238,43 @@ def weight_cache(w_bits: np.ndarray):
     return wf, wb
 
 
+# Two-level variant of the weight layouts (a reading; the pages give a single E4M3
+# block scale, [FAQ]).  Weights drawn like N(0, 0.02^2) have block amax / 6 below
+# E4M3's smallest normal (2^-6), so their block scales are subnormal and carry two or
+# three significant bits.  The variant puts a per-tensor power of two 2^e in front:
+# the cached codes and scales are those of W * 2^-e, with e the smallest integer
+# for which the largest block scale does not saturate, and every product with the
+# cached weight is multiplied back by 2^e.  A power of two keeps the scaling exact.
+E2M1_MAX = 6.0
+E4M3_MAX = 448.0
+
+
+def two_level_exponent(amax: float) -> int:
+    """The smallest integer e with amax <= 6 * 448 * 2^e (0 when amax is 0), by
+    stepping e one at a time against exact powers of two."""
+    top = E2M1_MAX * E4M3_MAX
+    if not amax > 0.0:
+        return 0
+    e = 0
+    while amax > top * 2.0 ** e:
+        e += 1
+    while amax <= top * 2.0 ** (e - 1):
+        e -= 1
+    return e
+
+
+def weight_cache_two_level(w_bits: np.ndarray):
+    """(e, Wf, Wb): e = two_level_exponent(max |W|); Wf, Wb = weight_cache(W * 2^-e).
+    The scaled values are exact in BF16 wherever they can matter: a value scaled
+    below BF16's normal range sits in a block whose codes it cannot change (its
+    quotient by the block scale rounds to a signed zero, or the block scale itself is
+    zero), and rounding keeps its sign."""
+    w = bf16_to_f64(w_bits)
+    e = two_level_exponent(float(np.max(np.abs(w))) if w.size else 0.0)
+    wf, wb = weight_cache(f64_to_bf16(w * 2.0 ** -e))
+    return e, wf, wb
+
+
 def f64_to_bf16_exact(v: np.ndarray) -> np.ndarray:
     """Bits of float64 values that are exactly representable in BF16 (asserted)."""
     f = np.ascontiguousarray(v, dtype=np.float32)
@@ -322,20 +359,21 @@ def lora_t(x: np.ndarray, a_bits: np.ndarray) -> np.ndarray:
     return gemm_nt(x, bf16_to_f64(a_bits))
 
 
-def frozen_fwd(xq: NVFP4, wf: NVFP4, x_bits=None, a_bits=None, b_bits=None, scale=0.0):
+def frozen_fwd(xq: NVFP4, wf: NVFP4, x_bits=None, a_bits=None, b_bits=None, scale=0.0, gexp=0):
     """[METHOD]+[LORA] forward of one frozen projection with its LoRA branch:
-    Y = deq(Xq) . deq(Wf)^T + scale * (X . A^T) . B^T, with BF16 X, A, B; float64."""
-    y = nvfp4_gemm(xq, wf)
+    Y = 2^gexp deq(Xq) . deq(Wf)^T + scale * (X . A^T) . B^T, with BF16 X, A, B;
+    float64 (gexp: the exponent of a two-level weight cache, else 0)."""
+    y = 2.0 ** gexp * nvfp4_gemm(xq, wf)
     if a_bits is not None:
         t = lora_t(bf16_to_f64(x_bits), a_bits)
         y = y + scale * gemm_nt(t, bf16_to_f64(b_bits))
     return y
 
 
-def frozen_dgrad(dy_bits: np.ndarray, wb: NVFP4, a_bits=None, b_bits=None, scale=0.0):
+def frozen_dgrad(dy_bits: np.ndarray, wb: NVFP4, a_bits=None, b_bits=None, scale=0.0, gexp=0):
     """[METHOD]+[LORA] input gradient of one projection:
-    dX = deq(q(dY)) . deq(Wb)^T + scale * (dY . B) . A, dY BF16; float64."""
-    dx = nvfp4_gemm(quantize(dy_bits), wb)
+    dX = 2^gexp deq(q(dY)) . deq(Wb)^T + scale * (dY . B) . A, dY BF16; float64."""
+    dx = 2.0 ** gexp * nvfp4_gemm(quantize(dy_bits), wb)
     if a_bits is not None:
         dy = bf16_to_f64(dy_bits)
         u = gemm_nt(dy, bf16_to_f64(b_bits).T)          # dY . B        [M x r]

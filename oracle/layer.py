@@ -16,7 +16,7 @@ from __future__ import annotations
 import numpy as np
 
 from . import (bf16_to_f64, f64_to_bf16, gemm_nt, nvfp4_gemm, quantize, rmsnorm_bwd, rmsnorm_quant,
-               silu_mul_bwd, silu_mul_quant, silu_mul_recompute, weight_cache)
+               silu_mul_bwd, silu_mul_quant, silu_mul_recompute, weight_cache, weight_cache_two_level)
 
 
 def _segments(seg_end):
@@ -57,15 +57,21 @@ def lora_grads(dy, xt, a, b, r, seg_end, scale):
 
 class OracleLayer:
     """w, lora_a, lora_b: dicts of BF16 bit arrays keyed q, k, v, o, gate, up, down
-    (PyTorch [out, in] layout); gamma1, gamma2: BF16 bits [H]."""
+    (PyTorch [out, in] layout); gamma1, gamma2: BF16 bits [H].  two_level: cache the
+    weights in the two-level variant (weight_cache_two_level), one exponent per
+    concatenated group."""
 
-    def __init__(self, H, I, KV, r, alpha, eps, w, lora_a, lora_b, gamma1, gamma2):
+    def __init__(self, H, I, KV, r, alpha, eps, w, lora_a, lora_b, gamma1, gamma2, two_level=False):
         self.H, self.I, self.KV, self.r, self.eps = H, I, KV, r, eps
         self.scale = alpha / r
         cat = lambda names, d: np.concatenate([d[n] for n in names], 0)
-        self.wf, self.wb = {}, {}
+        self.wf, self.wb, self.gexp = {}, {}, {}
         for key, names in (("qkv", ("q", "k", "v")), ("o", ("o",)), ("gu", ("gate", "up")), ("d", ("down",))):
-            self.wf[key], self.wb[key] = weight_cache(cat(names, w))
+            if two_level:
+                self.gexp[key], self.wf[key], self.wb[key] = weight_cache_two_level(cat(names, w))
+            else:
+                self.gexp[key] = 0
+                self.wf[key], self.wb[key] = weight_cache(cat(names, w))
             self.wf[key].dequantize()
             self.wb[key].dequantize()
         f = bf16_to_f64
@@ -76,6 +82,10 @@ class OracleLayer:
         self.seg = {"qkv": [H, H + KV, H + 2 * KV], "o": [H], "gu": [I, 2 * I], "d": [H]}
         self.g1, self.g2 = gamma1, gamma2
 
+    def _g(self, key, aq, cache):
+        """The frozen product with group `key`'s cached layout, times its 2^e."""
+        return 2.0 ** self.gexp[key] * nvfp4_gemm(aq, cache[key])
+
     def step(self, h, attn, d_out, d_qkv):
         """One forward + backward over the given tokens (BF16 bit arrays).  Returns the
         stage outputs (BF16 bits or float64 where the path keeps higher precision)."""
@@ -84,35 +94,35 @@ class OracleLayer:
         o = {}
         # ---------------- forward
         y1, xq1, rstd1 = rmsnorm_quant(h, self.g1, self.eps)
-        qkv = nvfp4_gemm(xq1, self.wf["qkv"]) + lora_fwd_term(f(y1), self.a["qkv"], self.b["qkv"], r,
+        qkv = self._g("qkv", xq1, self.wf) + lora_fwd_term(f(y1), self.a["qkv"], self.b["qkv"], r,
                                                                 self.seg["qkv"], s)
         o["qkv"] = q(qkv)
         aq = quantize(attn)
-        o["h2"] = h2 = q(f(h) + nvfp4_gemm(aq, self.wf["o"]) + lora_fwd_term(f(attn), self.a["o"], self.b["o"], r,
+        o["h2"] = h2 = q(f(h) + self._g("o", aq, self.wf) + lora_fwd_term(f(attn), self.a["o"], self.b["o"], r,
                                                                              self.seg["o"], s))
         y2, xq2, rstd2 = rmsnorm_quant(h2, self.g2, self.eps)
-        o["gu"] = gu = q(nvfp4_gemm(xq2, self.wf["gu"]) + lora_fwd_term(f(y2), self.a["gu"], self.b["gu"], r,
+        o["gu"] = gu = q(self._g("gu", xq2, self.wf) + lora_fwd_term(f(y2), self.a["gu"], self.b["gu"], r,
                                                                          self.seg["gu"], s))
         m, mq, gq, uq = silu_mul_quant(gu[:, :I], gu[:, I:])
-        o["out"] = q(f(h2) + nvfp4_gemm(mq, self.wf["d"]) + lora_fwd_term(f(m), self.a["d"], self.b["d"], r,
+        o["out"] = q(f(h2) + self._g("d", mq, self.wf) + lora_fwd_term(f(m), self.a["d"], self.b["d"], r,
                                                                            self.seg["d"], s))
         # ---------------- backward
         dof = f(d_out)
-        o["dm"] = dm = q(nvfp4_gemm(quantize(d_out), self.wb["d"]) +
+        o["dm"] = dm = q(self._g("d", quantize(d_out), self.wb) +
                          lora_dgrad_term(dof, self.a["d"], self.b["d"], r, self.seg["d"], s))
         dg, du = silu_mul_bwd(f(dm), gq, uq)
         o["dgu"] = dgu = q(np.concatenate([dg, du], 1))
         m_re = silu_mul_recompute(gq, uq)
         o["dA_d"], o["dB_d"] = lora_grads(dof, f(m_re), self.a["d"], self.b["d"], r, self.seg["d"], s)
-        o["dx2"] = dx2 = q(nvfp4_gemm(quantize(dgu), self.wb["gu"]) +
+        o["dx2"] = dx2 = q(self._g("gu", quantize(dgu), self.wb) +
                            lora_dgrad_term(f(dgu), self.a["gu"], self.b["gu"], r, self.seg["gu"], s))
         o["dA_gu"], o["dB_gu"] = lora_grads(f(dgu), xq2.dequantize(), self.a["gu"], self.b["gu"], r,
                                             self.seg["gu"], s)
         o["dh2"] = dh2 = q(rmsnorm_bwd(f(dx2), xq2, rstd2, self.g2) + dof)
-        o["dattn"] = q(nvfp4_gemm(quantize(dh2), self.wb["o"]) +
+        o["dattn"] = q(self._g("o", quantize(dh2), self.wb) +
                        lora_dgrad_term(f(dh2), self.a["o"], self.b["o"], r, self.seg["o"], s))
         o["dA_o"], o["dB_o"] = lora_grads(f(dh2), f(attn), self.a["o"], self.b["o"], r, self.seg["o"], s)
-        o["dx1"] = dx1 = q(nvfp4_gemm(quantize(d_qkv), self.wb["qkv"]) +
+        o["dx1"] = dx1 = q(self._g("qkv", quantize(d_qkv), self.wb) +
                            lora_dgrad_term(f(d_qkv), self.a["qkv"], self.b["qkv"], r, self.seg["qkv"], s))
         o["dA_qkv"], o["dB_qkv"] = lora_grads(f(d_qkv), xq1.dequantize(), self.a["qkv"], self.b["qkv"], r,
                                               self.seg["qkv"], s)
