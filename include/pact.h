@@ -29,7 +29,10 @@
  *   scales: pact_scale_bytes(rows, cols) bytes in 512-byte tiles of 128 rows x 4
  *   blocks; tiles are row-tile-major; inside a tile (row r, block c) is at byte
  *   (r % 32) * 16 + ((r % 128) / 32) * 4 + (c % 4).  Rows pad to 128 with zero bytes.
- *   No per-tensor second-level scale exists (4 bits + 8/16 bits = 4.5 bit/element).
+ *   The activations carry no per-tensor second-level scale (4 bits + 8/16 bits =
+ *   4.5 bit/element).  Frozen weights may optionally carry one power of two per
+ *   tensor (the two-level variant, pact_weight_layout_cache_scaled): a variant
+ *   beyond the pages, for weights whose block scales would be subnormal E4M3.
  * Shapes.  cols of every NVFP4 tensor is a multiple of 64; rows >= 1 is free.
  *   Frozen weights are [N x K] (PyTorch [out, in]); N and K are multiples of 64.
  * Pointers.  Every pointer argument is DEVICE memory unless stated, 16-byte
@@ -56,7 +59,7 @@
 extern "C" {
 #endif
 
-#define PACT_ABI_VERSION 1
+#define PACT_ABI_VERSION 2
 
 #if defined(__GNUC__)
 #define PACT_API __attribute__((visibility("default")))
@@ -86,10 +89,13 @@ typedef struct {
 } pact_nvfp4_t;
 
 /* The two cached layouts of one frozen weight W [N x K] ([METHOD] bullet 4):
- * fwd = q(W) [N x K] along K; bwd = q(deq(fwd)^T) [K x N] along N. */
+ * fwd = q(W * 2^-gexp) [N x K] along K; bwd = q(deq(fwd)^T) [K x N] along N.
+ * The weight the GEMMs use is 2^gexp * deq(layout); gexp is 0 for the plain
+ * (one-level) layouts and a tensor exponent for the two-level variant. */
 typedef struct {
     pact_nvfp4_t fwd;
     pact_nvfp4_t bwd;
+    int32_t gexp;
 } pact_weight_cache_t;
 
 /* The LoRA branch fused into a frozen GEMM ([LORA]; [METHOD]: A, B in BF16).
@@ -169,22 +175,48 @@ PACT_API pact_status pact_weight_layout_cache(const pact_bf16 *W, int64_t ldw, i
                                      void *buf, size_t bytes, pact_weight_cache_t *out,
                                      pact_stream_t stream);
 
+/* Two-level variant (beyond the pages: they give one E4M3 scale per block, [FAQ]).
+ * Weights like N(0, 0.02^2) have block amax / 6 below E4M3's smallest normal
+ * value 2^-6, so one-level block scales are subnormal with 2-3 significant bits.
+ * Here a per-tensor power of two 2^gexp stands in front of the block scales:
+ *   pact_absmax_bf16        *amax = max |x| over x [rows x cols] (row stride ldx),
+ *                           written to device memory (amax: one float); finite x.
+ *   pact_two_level_exponent (host, no GPU) the smallest integer e with
+ *                           amax <= 6 * 448 * 2^e (0 for amax <= 0 or not finite),
+ *                           so the largest block scale of W * 2^-e does not saturate.
+ *   pact_weight_layout_cache_scaled  as pact_weight_layout_cache for W * 2^-gexp
+ *                           (each product formed exactly in FP32; |gexp| <= 100,
+ *                           else PACT_ERR_INVALID_ARG); out->gexp = gexp.
+ * The caller reads *amax back to the host (libpact does not synchronise) and passes
+ * the exponent on.  Products with a cache of exponent g are scaled by 2^g in the
+ * GEMM epilogues (see pact_frozen_gemm_fwd); a power of two keeps that exact. */
+PACT_API pact_status pact_absmax_bf16(const pact_bf16 *x, int64_t ldx, int64_t rows, int64_t cols, float *amax,
+                                      pact_stream_t stream);
+PACT_API int pact_two_level_exponent(float amax);
+PACT_API pact_status pact_weight_layout_cache_scaled(const pact_bf16 *W, int64_t ldw, int64_t N, int64_t K,
+                                                     int gexp, void *buf, size_t bytes, pact_weight_cache_t *out,
+                                                     pact_stream_t stream);
+
 /* ---------------------------------------------------- A5: forward GEMM */
 /* [METHOD] bullet 1 with [LORA]:
- *   y[M x N] = BF16_RNE( residual + deq(xq) . deq(w->fwd)^T + sum_i T_i . B_i^T )
- * FP32 accumulation in tensor memory.  xq is [M x K], w->fwd [N x K]; y has row
- * stride ldy.  lora may be NULL (frozen GEMM only); residual (BF16 [M x N], row
- * stride ldr, e.g. the residual stream) may be NULL and may equal y (in place). */
+ *   y[M x N] = BF16_RNE( residual + 2^g (deq(xq) . deq(w->fwd)^T + sum_i T_i . B_i^T) )
+ * with g = w->gexp (0 for one-level layouts).  FP32 accumulation in tensor memory;
+ * the LoRA term shares the accumulator, so for g != 0 the caller passes T computed
+ * with scale * 2^-g (pact_lora_fwd's scale argument), which keeps it exact.  xq is
+ * [M x K], w->fwd [N x K]; y has row stride ldy.  lora may be NULL (frozen GEMM
+ * only); residual (BF16 [M x N], row stride ldr, e.g. the residual stream) may be
+ * NULL and may equal y (in place). */
 PACT_API pact_status pact_frozen_gemm_fwd(const pact_nvfp4_t *xq, const pact_weight_cache_t *w,
                                           const pact_lora_t *lora, const pact_bf16 *residual, int64_t ldr,
                                           pact_bf16 *y, int64_t ldy, pact_stream_t stream);
 
 /* ------------------------------------------------------ A6: dgrad GEMM */
 /* [METHOD] bullet 1 (input gradient) with [LORA]:
- *   dx[M x K] = BF16_RNE( residual + deq(dyq) . deq(w->bwd)^T + U . A )
- * dyq is the NVFP4 upstream gradient [M x N] (pact_quantize_nvfp4), w->bwd
- * [K x N].  lora and residual may be NULL; residual may equal dx (accumulate in
- * place). */
+ *   dx[M x K] = BF16_RNE( residual + 2^g (deq(dyq) . deq(w->bwd)^T + U . A) )
+ * with g = w->gexp; for g != 0, U comes from pact_lora_bwd_u with scale * 2^-g
+ * (and pact_lora_bwd then takes u_gexp = g).  dyq is the NVFP4 upstream gradient
+ * [M x N] (pact_quantize_nvfp4), w->bwd [K x N].  lora and residual may be NULL;
+ * residual may equal dx (accumulate in place). */
 PACT_API pact_status pact_frozen_gemm_dgrad(const pact_nvfp4_t *dyq, const pact_weight_cache_t *w,
                                             const pact_lora_t *lora, const pact_bf16 *residual, int64_t ldr,
                                             pact_bf16 *dx, int64_t lddx, pact_stream_t stream);
@@ -247,7 +279,8 @@ typedef struct {
     int r, nseg;
     int64_t seg_end[4];
     float scale;
-    pact_bf16 *dA;            /* out [nseg*r x K]:  (U_hi + U_lo)^T . X~ */
+    int u_gexp;               /* U holds 2^-u_gexp times the gradient factor (0 usually) */
+    pact_bf16 *dA;            /* out [nseg*r x K]:  2^u_gexp (U_hi + U_lo)^T . X~ */
     pact_bf16 *dB;            /* out [N x r]: rows seg_i = scale * dY[:, seg_i]^T . (X~ . A_i^T) */
 } pact_lora_bwd_t;
 

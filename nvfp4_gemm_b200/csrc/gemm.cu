@@ -38,6 +38,7 @@
 //    while the warp adds the residual (prefetched by TMA into the warp's 4 KiB
 //    shared-memory slab), rounds to BF16 into the slab and writes it with one TMA
 //    store, which also clips the ragged edges of the output.
+#include <cmath>
 #include "common.cuh"
 
 namespace pact {
@@ -84,6 +85,7 @@ struct Params {
     int lora_r;
     int lora_nseg;
     int64_t seg_end[4];
+    float out_scale;      // 2^gexp of the weight cache: scales the accumulator (exact)
 };
 
 __device__ __forceinline__ int lora_segment(const Params &p, int n0) {
@@ -409,7 +411,7 @@ k_nvfp4_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CU
                     const uint32_t a = slab + lane * 128 + ((q ^ (lane & 7)) << 4);
                     float f[8];
 #pragma unroll
-                    for (int i = 0; i < 8; ++i) f[i] = __uint_as_float(r[8 * q + i]);
+                    for (int i = 0; i < 8; ++i) f[i] = __uint_as_float(r[8 * q + i]) * p.out_scale;
                     if (p.has_res) {
                         uint32_t o0, o1, o2, o3;
                         asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
@@ -523,10 +525,11 @@ static pact_status check_lora(const pact_lora_t *l, int64_t M, int64_t N, int64_
 }
 
 // D[M x N] = deq(a) . deq(b)^T (+ LoRA); a [M x K], b [N x K].
-static pact_status run(const pact_nvfp4_t *a, const pact_nvfp4_t *b, const pact_lora_t *lora, bool dgrad,
+static pact_status run(const pact_nvfp4_t *a, const pact_nvfp4_t *b, int gexp, const pact_lora_t *lora, bool dgrad,
                        const pact_bf16 *res, int64_t ldr, pact_bf16 *out, int64_t ldo, cudaStream_t stream,
                        const char *what) {
     const int64_t M = a->rows, K = a->cols, N = b->rows;
+    PACT_CHECK(gexp >= -100 && gexp <= 100, PACT_ERR_INVALID_ARG, "%s: w->gexp out of range (%d)", what, gexp);
     PACT_CHECK(M <= 0x7FFFFFFF && N <= 0x7FFFFFFF && K <= 0x7FFFFFFF, PACT_ERR_SHAPE, "%s: dimension too large", what);
     PACT_CHECK(out, PACT_ERR_INVALID_ARG, "%s: output NULL", what);
     PACT_CHECK(ldo >= N && ldo % 8 == 0 && aligned16(out), PACT_ERR_ALIGN,
@@ -565,6 +568,7 @@ static pact_status run(const pact_nvfp4_t *a, const pact_nvfp4_t *b, const pact_
     Params p;
     p.M = (int)M; p.N = (int)N; p.K = (int)K;
     p.has_res = res != nullptr;
+    p.out_scale = std::ldexp(1.0f, gexp);
     p.lora_mode = LORA_NONE;
     p.lora_steps = 0; p.lora_r = 0; p.lora_nseg = 1;
     for (int i = 0; i < 4; ++i) p.seg_end[i] = N;
@@ -613,7 +617,7 @@ pact_status pact_frozen_gemm_fwd(const pact_nvfp4_t *xq, const pact_weight_cache
     if (s == PACT_OK) s = check_nvfp4(xq, xq->rows, K, "xq");
     if (s != PACT_OK) return s;
     PACT_CHECK(xq->rows >= 1 && N % 64 == 0 && K % 64 == 0, PACT_ERR_SHAPE, "pact_frozen_gemm_fwd: bad shape");
-    return gemm::run(xq, &w->fwd, lora, false, residual, ldr, y, ldy, (cudaStream_t)stream, "pact_frozen_gemm_fwd");
+    return gemm::run(xq, &w->fwd, w->gexp, lora, false, residual, ldr, y, ldy, (cudaStream_t)stream, "pact_frozen_gemm_fwd");
 }
 
 pact_status pact_frozen_gemm_dgrad(const pact_nvfp4_t *dyq, const pact_weight_cache_t *w, const pact_lora_t *lora,
@@ -625,7 +629,7 @@ pact_status pact_frozen_gemm_dgrad(const pact_nvfp4_t *dyq, const pact_weight_ca
     if (s == PACT_OK) s = check_nvfp4(dyq, dyq->rows, N, "dyq");
     if (s != PACT_OK) return s;
     PACT_CHECK(dyq->rows >= 1 && N % 64 == 0 && K % 64 == 0, PACT_ERR_SHAPE, "pact_frozen_gemm_dgrad: bad shape");
-    return gemm::run(dyq, &w->bwd, lora, true, residual, ldr, dx, lddx, (cudaStream_t)stream,
+    return gemm::run(dyq, &w->bwd, w->gexp, lora, true, residual, ldr, dx, lddx, (cudaStream_t)stream,
                      "pact_frozen_gemm_dgrad");
 }
 

@@ -14,6 +14,8 @@
 // stream the activations; each split writes its FP32 partial tile to caller scratch
 // and a finalize kernel sums the partials in a fixed order (deterministic), scales
 // and rounds.
+#include <cmath>
+
 #include "quant.cuh"
 
 namespace pact {
@@ -424,6 +426,7 @@ pact_status pact_lora_bwd(const pact_lora_bwd_t *g, void *workspace, size_t ws_b
                    K <= 0x7FFFFFFF && (r == 16 || r == 32 || r == 48 || r == 64) && nseg >= 1 && nseg <= 3 &&
                    nseg * r <= 64,
                PACT_ERR_SHAPE, "pact_lora_bwd: bad shape");
+    PACT_CHECK(g->u_gexp >= -100 && g->u_gexp <= 100, PACT_ERR_INVALID_ARG, "pact_lora_bwd: |u_gexp| <= 100 required");
     pact_status s = check_segments(N, nseg, g->seg_end, "pact_lora_bwd");
     if (s != PACT_OK) return s;
     const int R = nseg * r;
@@ -515,7 +518,8 @@ pact_status pact_lora_bwd(const pact_lora_bwd_t *g, void *workspace, size_t ws_b
     s = launch_mma<true, true>(ta, tb, p, tiles, st, "pact_lora_bwd");
     if (s != PACT_OK) return s;
     return launch_dep(k_finalize, dim3(finalize_grid(K * R)), dim3(256), 0, st, "pact_lora_bwd", (const float *)ws_da,
-                      p.splits, (int64_t)(K * R), (int64_t)R, (int64_t)K, (int64_t)R, 1.0f, 2, g->dA, K, (int64_t)0);
+                      p.splits, (int64_t)(K * R), (int64_t)R, (int64_t)K, (int64_t)R, std::ldexp(1.0f, g->u_gexp), 2,
+                      g->dA, K, (int64_t)0);
 }
 
 }  // extern "C"

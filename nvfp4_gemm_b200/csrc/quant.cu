@@ -4,6 +4,8 @@
 // contiguous bytes per instruction) and quantize with warp-shuffle block maxima.
 #include <math.h>
 
+#include <cmath>
+
 #include "quant.cuh"
 
 namespace pact {
@@ -26,8 +28,10 @@ __device__ __forceinline__ void unpack8_bf16(const uint4 &u, float (&v)[8]) {
 }
 
 // ------------------------------------------------------------------ A2: quantize
+// prescale: a power of two the values are multiplied by first (exact in FP32); 1
+// for every quantization on the step path, 2^-gexp for two-level weight layouts.
 __global__ void __launch_bounds__(256) k_quantize(const pact_bf16 *__restrict__ x, int64_t ldx, int64_t rows,
-                                                  pact_nvfp4_t out) {
+                                                  pact_nvfp4_t out, float prescale) {
     pdl_wait();
     const int lane = threadIdx.x & 31;
     const int64_t nchunk = (out.cols + CHUNK - 1) / CHUNK;
@@ -54,6 +58,10 @@ __global__ void __launch_bounds__(256) k_quantize(const pact_bf16 *__restrict__ 
             const bool valid = c0 + 8 * lane < out.cols;
             float v[8];
             unpack8_bf16(cur, v);
+            if (prescale != 1.0f) {   // uniform over the launch
+#pragma unroll
+                for (int i = 0; i < 8; ++i) v[i] *= prescale;
+            }
             uint32_t sb;
             const uint32_t codes = quant8(v, &sb);
             store_chunk(out, row, c0, codes, sb, valid);
@@ -61,6 +69,27 @@ __global__ void __launch_bounds__(256) k_quantize(const pact_bf16 *__restrict__ 
         it = nx;
         cur = nxt;
     }
+}
+
+// max |x| over a [rows x cols] BF16 tensor into *amax (zeroed before the launch).
+// Non-negative floats order like their bit patterns, so an unsigned atomicMax of
+// the bits is a float max.
+__global__ void __launch_bounds__(256) k_absmax_bf16(const pact_bf16 *__restrict__ x, int64_t ldx, int64_t rows,
+                                                     int64_t cols, unsigned *__restrict__ amax) {
+    pdl_wait();
+    const int64_t per_row = cols / 8;
+    const int64_t n8 = rows * per_row;
+    float m = 0.0f;
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n8; i += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t r = i / per_row, c = (i % per_row) * 8;
+        float v[8];
+        unpack8_bf16(*reinterpret_cast<const uint4 *>(x + r * ldx + c), v);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) m = fmaxf(m, fabsf(v[j]));
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
+    if ((threadIdx.x & 31) == 0) atomicMax(amax, __float_as_uint(m));
 }
 
 static int grid_for(int64_t warp_tasks, int threads) {
@@ -502,7 +531,33 @@ pact_status pact_quantize_nvfp4(const pact_bf16 *x, int64_t ldx, int64_t rows, i
     if (s != PACT_OK) return s;
     const int64_t tasks = ((rows + 127) / 128 * 128) * ((cols + CHUNK - 1) / CHUNK);
     return launch_dep(k_quantize, dim3(grid_for(tasks, 256)), dim3(256), 0, (cudaStream_t)stream, "pact_quantize_nvfp4",
-                      x, ldx, rows, *out);
+                      x, ldx, rows, *out, 1.0f);
+}
+
+pact_status pact_absmax_bf16(const pact_bf16 *x, int64_t ldx, int64_t rows, int64_t cols, float *amax,
+                             pact_stream_t stream) {
+    PACT_CHECK(x && amax, PACT_ERR_INVALID_ARG, "pact_absmax_bf16: NULL argument");
+    PACT_CHECK(rows >= 1 && cols >= 8 && cols % 8 == 0, PACT_ERR_SHAPE,
+               "pact_absmax_bf16: rows >= 1 and cols a positive multiple of 8 required (rows=%lld cols=%lld)",
+               (long long)rows, (long long)cols);
+    PACT_CHECK(ldx >= cols && ldx % 8 == 0 && aligned16(x) && ((uintptr_t)amax & 3) == 0, PACT_ERR_ALIGN,
+               "pact_absmax_bf16: x 16-byte aligned with ldx >= cols, ldx %% 8 == 0; amax 4-byte aligned");
+    const cudaError_t e = cudaMemsetAsync(amax, 0, sizeof(float), (cudaStream_t)stream);
+    PACT_CHECK(e == cudaSuccess, PACT_ERR_CUDA, "pact_absmax_bf16: %s", cudaGetErrorString(e));
+    const int64_t threads = rows * (cols / 8);
+    return launch_dep(k_absmax_bf16, dim3(grid_for((threads + 31) / 32, 256)), dim3(256), 0, (cudaStream_t)stream,
+                      "pact_absmax_bf16", x, ldx, rows, cols, reinterpret_cast<unsigned *>(amax));
+}
+
+int pact_two_level_exponent(float amax) {
+    // smallest e with amax <= 2688 * 2^e; 2688 * 2^e is exact in double for every e
+    // reached here (|e| < 200), so each comparison is exact
+    if (!(amax > 0.0f) || !std::isfinite(amax)) return 0;
+    const double a = (double)amax;
+    int e = std::ilogb(a) - std::ilogb(2688.0);
+    while (a > std::ldexp(2688.0, e)) ++e;
+    while (a <= std::ldexp(2688.0, e - 1)) --e;
+    return e;
 }
 
 pact_status pact_rmsnorm_quant(const pact_bf16 *x, int64_t ldx, const pact_bf16 *gamma, float eps, int64_t M,
@@ -621,7 +676,15 @@ pact_status pact_rmsnorm_bwd(const pact_bf16 *dy, int64_t lddy, const pact_nvfp4
 
 pact_status pact_weight_layout_cache(const pact_bf16 *W, int64_t ldw, int64_t N, int64_t K, void *buf, size_t bytes,
                                      pact_weight_cache_t *out, pact_stream_t stream) {
+    return pact_weight_layout_cache_scaled(W, ldw, N, K, 0, buf, bytes, out, stream);
+}
+
+pact_status pact_weight_layout_cache_scaled(const pact_bf16 *W, int64_t ldw, int64_t N, int64_t K, int gexp,
+                                            void *buf, size_t bytes, pact_weight_cache_t *out,
+                                            pact_stream_t stream) {
     PACT_CHECK(W && buf && out, PACT_ERR_INVALID_ARG, "pact_weight_layout_cache: NULL argument");
+    PACT_CHECK(gexp >= -100 && gexp <= 100, PACT_ERR_INVALID_ARG,
+               "pact_weight_layout_cache_scaled: |gexp| <= 100 required (gexp=%d)", gexp);
     PACT_CHECK(N >= 64 && K >= 64 && N % 64 == 0 && K % 64 == 0, PACT_ERR_SHAPE,
                "pact_weight_layout_cache: N and K must be positive multiples of 64 (N=%lld K=%lld)", (long long)N,
                (long long)K);
@@ -637,7 +700,10 @@ pact_status pact_weight_layout_cache(const pact_bf16 *W, int64_t ldw, int64_t N,
     c.bwd.rows = K; c.bwd.cols = N;
     c.bwd.codes = p; p += up256(pact_nvfp4_code_bytes(K, N));
     c.bwd.scales = p;
-    pact_status s = pact_quantize_nvfp4(W, ldw, N, K, &c.fwd, stream);
+    c.gexp = gexp;
+    const int64_t tasks = ((N + 127) / 128 * 128) * ((K + CHUNK - 1) / CHUNK);
+    pact_status s = launch_dep(k_quantize, dim3(grid_for(tasks, 256)), dim3(256), 0, (cudaStream_t)stream,
+                               "pact_weight_layout_cache", W, ldw, N, c.fwd, std::ldexp(1.0f, -gexp));
     if (s != PACT_OK) return s;
     dim3 grid((unsigned)(K / 64), (unsigned)(N / 64));
     s = launch_dep(k_weight_bwd_layout, grid, dim3(256), 0, (cudaStream_t)stream, "pact_weight_layout_cache", c.fwd,

@@ -72,19 +72,28 @@ class PactLayer:
     """Weights are BF16 device tensors in PyTorch [out, in] layout:
     w = {q, k, v, o, gate, up, down}; lora_a = {p: [r, in]}, lora_b = {p: [out, r]};
     gamma1, gamma2: [H].  Frozen weights are cached as NVFP4 forward/backward layouts
-    at construction (once)."""
+    at construction (once); two_level selects the variant with a power of two per
+    cached group (pact_weight_layout_cache_scaled)."""
 
     def __init__(self, shape: LayerShape, w: Dict[str, torch.Tensor], lora_a: Dict[str, torch.Tensor],
-                 lora_b: Dict[str, torch.Tensor], gamma1: torch.Tensor, gamma2: torch.Tensor):
+                 lora_b: Dict[str, torch.Tensor], gamma1: torch.Tensor, gamma2: torch.Tensor,
+                 two_level: bool = False):
         self.s = shape
+        self.two_level = two_level
         S = shape
         dev = gamma1.device
         cat = lambda names, d: torch.cat([d[n] for n in names], 0).contiguous()
         # frozen weights: concatenated where projections share an input, then cached
-        self.c_qkv = P.pact_weight_layout_cache(cat(("q", "k", "v"), w))
-        self.c_o = P.pact_weight_layout_cache(w["o"].contiguous())
-        self.c_gu = P.pact_weight_layout_cache(cat(("gate", "up"), w))
-        self.c_d = P.pact_weight_layout_cache(w["down"].contiguous())
+        cache = lambda t: P.pact_weight_layout_cache(t, two_level=two_level)
+        self.c_qkv = cache(cat(("q", "k", "v"), w))
+        self.c_o = cache(w["o"].contiguous())
+        self.c_gu = cache(cat(("gate", "up"), w))
+        self.c_d = cache(w["down"].contiguous())
+        # a group cached with exponent g scales its whole GEMM accumulator by 2^g, so
+        # its LoRA activations (T, U) are computed with scale * 2^-g (exact) and the
+        # dA contraction over U is scaled back by 2^g
+        self.gexp = {"qkv": self.c_qkv.gexp, "o": self.c_o.gexp, "gu": self.c_gu.gexp, "d": self.c_d.gexp}
+        self.sc = {k: shape.scale * 2.0 ** -g for k, g in self.gexp.items()}
         # adapters, stacked like the weights
         self.a_qkv, self.b_qkv = cat(("q", "k", "v"), lora_a), cat(("q", "k", "v"), lora_b)
         self.a_o, self.b_o = lora_a["o"].contiguous(), lora_b["o"].contiguous()
@@ -173,26 +182,26 @@ class PactLayer:
         return [
             Op("rmsnorm_quant_1", lambda: P.pact_rmsnorm_quant(h, self.g1, S.eps, self.xq1, self.x1, self.rstd1),
                bytes=2 * M * H + 2 * H + S.nv(M, H) + 2 * M * H + 4 * M),
-            Op("lora_fwd_qkv", lambda: P.pact_lora_fwd(self.x1, self.a_qkv, s, self.t_qkv, self.ws), kernels=2,
+            Op("lora_fwd_qkv", lambda: P.pact_lora_fwd(self.x1, self.a_qkv, self.sc["qkv"], self.t_qkv, self.ws), kernels=2,
                bytes=lora_fwd(H, 3 * r)),
             Op("gemm_fwd_qkv", lambda: P.pact_frozen_gemm_fwd(self.xq1, self.c_qkv, self.l_qkv_f, y=self.qkv),
                "gemm", gemm(S.M, S.n_qkv, S.H), bytes=gbytes(S.n_qkv, H, 3 * r)),
             Op("quantize_attn", lambda: P.pact_quantize_nvfp4(attn, self.aq), bytes=2 * M * H + S.nv(M, H)),
-            Op("lora_fwd_o", lambda: P.pact_lora_fwd(attn, self.a_o, s, self.t_o, self.ws), kernels=2,
+            Op("lora_fwd_o", lambda: P.pact_lora_fwd(attn, self.a_o, self.sc["o"], self.t_o, self.ws), kernels=2,
                bytes=lora_fwd(H, r)),
             Op("gemm_fwd_o", lambda: P.pact_frozen_gemm_fwd(self.aq, self.c_o, self.l_o_f, residual=h, y=self.h2),
                "gemm", gemm(S.M, S.H, S.H), bytes=gbytes(H, H, r) + 2 * M * H),
             Op("rmsnorm_quant_2", lambda: P.pact_rmsnorm_quant(self.h2, self.g2, S.eps, self.xq2, self.x2,
                                                                self.rstd2),
                bytes=2 * M * H + 2 * H + S.nv(M, H) + 2 * M * H + 4 * M),
-            Op("lora_fwd_gu", lambda: P.pact_lora_fwd(self.x2, self.a_gu, s, self.t_gu, self.ws), kernels=2,
+            Op("lora_fwd_gu", lambda: P.pact_lora_fwd(self.x2, self.a_gu, self.sc["gu"], self.t_gu, self.ws), kernels=2,
                bytes=lora_fwd(H, 2 * r)),
             Op("gemm_fwd_gu", lambda: P.pact_frozen_gemm_fwd(self.xq2, self.c_gu, self.l_gu_f, y=self.gu),
                "gemm", gemm(S.M, 2 * I, S.H), bytes=gbytes(2 * I, H, 2 * r)),
             Op("silu_mul_quant", lambda: P.pact_silu_mul_quant(self.gu[:, :I], self.gu[:, I:], self.m, self.mq,
                                                                self.gq, self.uq),
                bytes=4 * M * I + 2 * M * I + 3 * S.nv(M, I)),
-            Op("lora_fwd_down", lambda: P.pact_lora_fwd(self.m, self.a_d, s, self.t_d, self.ws), kernels=2,
+            Op("lora_fwd_down", lambda: P.pact_lora_fwd(self.m, self.a_d, self.sc["d"], self.t_d, self.ws), kernels=2,
                bytes=lora_fwd(I, r)),
             Op("gemm_fwd_down", lambda: P.pact_frozen_gemm_fwd(self.mq, self.c_d, self.l_d_f, residual=self.h2,
                                                                y=self.out),
@@ -214,7 +223,7 @@ class PactLayer:
         LB = 7  # kernels of one pact_lora_bwd call reading an NVFP4 copy (6 with BF16 input)
         return [
             # down projection
-            Op("lora_bwd_u_down", lambda: P.pact_lora_bwd_u(d_out, self.b_d, r, [H], s, self.u_d, self.ws), kernels=2,
+            Op("lora_bwd_u_down", lambda: P.pact_lora_bwd_u(d_out, self.b_d, r, [H], self.sc["d"], self.u_d, self.ws), kernels=2,
                bytes=lora_u(H, r)),
             Op("quantize_dout", lambda: P.pact_quantize_nvfp4(d_out, self.doq), bytes=2 * M * H + S.nv(M, H)),
             Op("gemm_dgrad_down", lambda: P.pact_frozen_gemm_dgrad(self.doq, self.c_d, self.l_d_b, dx=self.dm),
@@ -223,39 +232,42 @@ class PactLayer:
                                                                        self.dguq, self.m_re),
                bytes=2 * M * I + 2 * S.nv(M, I) + 4 * M * I + S.nv(M, 2 * I) + 2 * M * I),
             Op("lora_bwd_down", lambda: P.pact_lora_bwd(d_out, self.a_d, self.u_d, r, [H], s, x=self.m_re,
-                                                        dA=g["a_d"], dB=g["b_d"], workspace=self.ws_leaf["down"]),
+                                                        dA=g["a_d"], dB=g["b_d"], workspace=self.ws_leaf["down"],
+                                                        u_gexp=self.gexp["d"]),
                kernels=LB - 1, side=True,
                bytes=lora_bwd(H, 2 * M * I, I, r)),
             # gate|up
-            Op("lora_bwd_u_gu", lambda: P.pact_lora_bwd_u(self.dgu, self.b_gu, r, self.seg_gu, s, self.u_gu, self.ws), kernels=2,
+            Op("lora_bwd_u_gu", lambda: P.pact_lora_bwd_u(self.dgu, self.b_gu, r, self.seg_gu, self.sc["gu"], self.u_gu, self.ws), kernels=2,
                bytes=lora_u(2 * I, 2 * r)),
             Op("gemm_dgrad_gu", lambda: P.pact_frozen_gemm_dgrad(self.dguq, self.c_gu, self.l_gu_b, dx=self.dx2),
                "gemm", gemm(S.M, H, 2 * I), bytes=gbytes(H, 2 * I, 2 * r)),
             Op("lora_bwd_gu", lambda: P.pact_lora_bwd(self.dgu, self.a_gu, self.u_gu, r, self.seg_gu, s,
                                                       xq=self.xq2, dA=g["a_gu"], dB=g["b_gu"],
-                                                      workspace=self.ws_leaf["gu"]),
+                                                      workspace=self.ws_leaf["gu"], u_gexp=self.gexp["gu"]),
                kernels=LB, side=True, bytes=lora_bwd(2 * I, S.nv(M, H), H, 2 * r)),
             Op("rmsnorm_bwd_2", lambda: P.pact_rmsnorm_bwd(self.dx2, self.xq2, self.rstd2, self.g2, dres=d_out,
                                                            dx=self.dh2, dxq=self.dh2q),
                bytes=2 * M * H + S.nv(M, H) + 4 * M + 2 * H + 2 * M * H + 2 * M * H + S.nv(M, H)),
             # o projection (its output joined the residual stream h2)
-            Op("lora_bwd_u_o", lambda: P.pact_lora_bwd_u(self.dh2, self.b_o, r, [H], s, self.u_o, self.ws), kernels=2,
+            Op("lora_bwd_u_o", lambda: P.pact_lora_bwd_u(self.dh2, self.b_o, r, [H], self.sc["o"], self.u_o, self.ws), kernels=2,
                bytes=lora_u(H, r)),
             Op("gemm_dgrad_o", lambda: P.pact_frozen_gemm_dgrad(self.dh2q, self.c_o, self.l_o_b, dx=self.dattn),
                "gemm", gemm(S.M, H, H), bytes=gbytes(H, H, r)),
             Op("lora_bwd_o", lambda: P.pact_lora_bwd(self.dh2, self.a_o, self.u_o, r, [H], s, x=attn,
-                                                     dA=g["a_o"], dB=g["b_o"], workspace=self.ws_leaf["o"]),
+                                                     dA=g["a_o"], dB=g["b_o"], workspace=self.ws_leaf["o"],
+                                                     u_gexp=self.gexp["o"]),
                kernels=LB - 1, side=True,
                bytes=lora_bwd(H, 2 * M * H, H, r)),
             # q|k|v (d_qkv stands in for the attention backward)
-            Op("lora_bwd_u_qkv", lambda: P.pact_lora_bwd_u(d_qkv, self.b_qkv, r, self.seg_qkv, s, self.u_qkv, self.ws), kernels=2,
+            Op("lora_bwd_u_qkv", lambda: P.pact_lora_bwd_u(d_qkv, self.b_qkv, r, self.seg_qkv, self.sc["qkv"], self.u_qkv, self.ws), kernels=2,
                bytes=lora_u(S.n_qkv, 3 * r)),
             Op("quantize_dqkv", lambda: P.pact_quantize_nvfp4(d_qkv, self.dqkvq), bytes=2 * M * S.n_qkv + S.nv(M, S.n_qkv)),
             Op("gemm_dgrad_qkv", lambda: P.pact_frozen_gemm_dgrad(self.dqkvq, self.c_qkv, self.l_qkv_b, dx=self.dx1),
                "gemm", gemm(S.M, H, S.n_qkv), bytes=gbytes(H, S.n_qkv, 3 * r)),
             Op("lora_bwd_qkv", lambda: P.pact_lora_bwd(d_qkv, self.a_qkv, self.u_qkv, r, self.seg_qkv, s,
                                                        xq=self.xq1, dA=g["a_qkv"], dB=g["b_qkv"],
-                                                       workspace=self.ws_leaf["qkv"]), kernels=LB, side=True,
+                                                       workspace=self.ws_leaf["qkv"], u_gexp=self.gexp["qkv"]),
+               kernels=LB, side=True,
                bytes=lora_bwd(S.n_qkv, S.nv(M, H), H, 3 * r)),
             Op("rmsnorm_bwd_1", lambda: P.pact_rmsnorm_bwd(self.dx1, self.xq1, self.rstd1, self.g1, dres=self.dh2,
                                                            dx=self.dh),

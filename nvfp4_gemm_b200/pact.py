@@ -34,7 +34,7 @@ class c_nvfp4(ctypes.Structure):
 
 
 class c_weight_cache(ctypes.Structure):
-    _fields_ = [("fwd", c_nvfp4), ("bwd", c_nvfp4)]
+    _fields_ = [("fwd", c_nvfp4), ("bwd", c_nvfp4), ("gexp", ctypes.c_int32)]
 
 
 class c_lora(ctypes.Structure):
@@ -50,7 +50,8 @@ class c_lora_bwd(ctypes.Structure):
                 ("xq", ctypes.POINTER(c_nvfp4)),
                 ("A", ctypes.c_void_p), ("U", ctypes.c_void_p), ("ldu", ctypes.c_int64),
                 ("r", ctypes.c_int), ("nseg", ctypes.c_int), ("seg_end", ctypes.c_int64 * 4),
-                ("scale", ctypes.c_float), ("dA", ctypes.c_void_p), ("dB", ctypes.c_void_p)]
+                ("scale", ctypes.c_float), ("u_gexp", ctypes.c_int), ("dA", ctypes.c_void_p),
+                ("dB", ctypes.c_void_p)]
 
 
 def _load() -> ctypes.CDLL:
@@ -68,6 +69,10 @@ def _load() -> ctypes.CDLL:
         "pact_rmsnorm_quant": (S, [P, I64, P, F, I64, I64, NV, P, P, P]),
         "pact_silu_mul_quant": (S, [P, P, I64, I64, I64, P, NV, NV, NV, P]),
         "pact_weight_layout_cache": (S, [P, I64, I64, I64, P, ctypes.c_size_t, ctypes.POINTER(c_weight_cache), P]),
+        "pact_weight_layout_cache_scaled": (S, [P, I64, I64, I64, I, P, ctypes.c_size_t,
+                                                ctypes.POINTER(c_weight_cache), P]),
+        "pact_absmax_bf16": (S, [P, I64, I64, I64, P, P]),
+        "pact_two_level_exponent": (I, [F]),
         "pact_frozen_gemm_fwd": (S, [NV, ctypes.POINTER(c_weight_cache), ctypes.POINTER(c_lora), P, I64, P, I64, P]),
         "pact_frozen_gemm_dgrad": (S, [NV, ctypes.POINTER(c_weight_cache), ctypes.POINTER(c_lora), P, I64, P, I64,
                                        P]),
@@ -154,6 +159,11 @@ class WeightCache:
     K: int
 
     @property
+    def gexp(self) -> int:
+        """The tensor exponent of a two-level cache (0 for the one-level layouts)."""
+        return int(self.cstruct.gexp)
+
+    @property
     def fwd(self) -> NVFP4Tensor:
         return self._view(self.cstruct.fwd)
 
@@ -235,16 +245,37 @@ def pact_silu_mul_quant(g: torch.Tensor, u: torch.Tensor, m: Optional[torch.Tens
     return m, mq, gq, uq
 
 
-def pact_weight_layout_cache(W: torch.Tensor, stream=None) -> WeightCache:
+def pact_absmax_bf16(x: torch.Tensor, out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """max |x| of a 2-D BF16 tensor, as a one-element FP32 device tensor."""
+    _bf16(x, "x")
+    if out is None:
+        out = torch.empty(1, dtype=torch.float32, device=x.device)
+    _check(_lib.pact_absmax_bf16(x.data_ptr(), _ld(x), x.shape[0], x.shape[1], out.data_ptr(), _stream(stream)))
+    return out
+
+
+def pact_two_level_exponent(amax: float) -> int:
+    return int(_lib.pact_two_level_exponent(ctypes.c_float(amax)))
+
+
+def pact_weight_layout_cache(W: torch.Tensor, stream=None, two_level: bool = False) -> WeightCache:
+    """The cached layouts of W.  two_level: the variant with a per-tensor power of two
+    (its exponent comes from pact_absmax_bf16 on the device; reading that one float
+    back makes this call wait for the stream, once per frozen weight)."""
     _bf16(W, "W")
     N, K = W.shape
     nbytes = pact_weight_cache_bytes(N, K)
     buf = torch.empty(nbytes + 256, dtype=torch.uint8, device=W.device)
     off = (-buf.data_ptr()) % 256
     buf = buf[off:off + nbytes]
+    gexp = 0
+    if two_level:
+        amax = pact_absmax_bf16(W, stream=stream)
+        torch.cuda.synchronize(W.device)       # the kernel may run on a caller's stream
+        gexp = pact_two_level_exponent(float(amax.cpu()))
     c = c_weight_cache()
-    _check(_lib.pact_weight_layout_cache(W.data_ptr(), _ld(W), N, K, buf.data_ptr(), nbytes, ctypes.byref(c),
-                                         _stream(stream)))
+    _check(_lib.pact_weight_layout_cache_scaled(W.data_ptr(), _ld(W), N, K, gexp, buf.data_ptr(), nbytes,
+                                                ctypes.byref(c), _stream(stream)))
     return WeightCache(buf, c, N, K)
 
 
@@ -337,7 +368,7 @@ def pact_lora_bwd_workspace_bytes(M: int, N: int, K: int, r: int, nseg: int) -> 
 def pact_lora_bwd(dy: torch.Tensor, A: torch.Tensor, U: torch.Tensor, r: int, seg_end: Sequence[int], scale: float,
                   x: Optional[torch.Tensor] = None, xq: Optional[NVFP4Tensor] = None,
                   dA: Optional[torch.Tensor] = None, dB: Optional[torch.Tensor] = None,
-                  workspace: Optional[torch.Tensor] = None, stream=None):
+                  workspace: Optional[torch.Tensor] = None, stream=None, u_gexp: int = 0):
     _bf16(dy, "dy")
     M, N = dy.shape
     K = A.shape[1]
@@ -362,6 +393,7 @@ def pact_lora_bwd(dy: torch.Tensor, A: torch.Tensor, U: torch.Tensor, r: int, se
     for i in range(4):
         args.seg_end[i] = seg_end[i] if i < nseg else 0
     args.scale = float(scale)
+    args.u_gexp = int(u_gexp)
     args.dA, args.dB = dA.data_ptr(), dB.data_ptr()
     _check(_lib.pact_lora_bwd(ctypes.byref(args), workspace.data_ptr(), workspace.numel(), _stream(stream)))
     return dA, dB

@@ -17,7 +17,11 @@ def declared_functions():
 
 @pytest.fixture(scope="module")
 def P():
-    import nvfp4_gemm_b200.build as b
+    # the build script is loaded by path so that a stale library is not loaded first
+    import importlib.util
+    spec = importlib.util.spec_from_file_location("_pact_build", os.path.join(ROOT, "nvfp4_gemm_b200", "build.py"))
+    b = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(b)
     b.build()
     import nvfp4_gemm_b200 as p
     return p
@@ -32,7 +36,7 @@ def test_every_declared_symbol_is_exported(P):
 
 
 def test_abi_version_and_status_names(P):
-    assert P.pact_abi_version() == 1
+    assert P.pact_abi_version() == 2
     lib = P.pact.lib
     assert lib.pact_status_string(0) == b"PACT_OK"
     assert lib.pact_status_string(5) == b"PACT_ERR_TIMEOUT"
@@ -110,3 +114,29 @@ def test_host_checks_reject_bad_arguments(P):
     args.xq = ctypes.pointer(xq3)
     need = P.pact_lora_bwd_workspace_bytes(256, 512, 512, 16, 1)
     assert lib.pact_lora_bwd(ctypes.byref(args), 0x10000, need, None) == 1
+
+
+def test_two_level_exponent_host_function(P, orc):
+    """pact_two_level_exponent (host code, no GPU) against the oracle's definition."""
+    import numpy as np
+    rng = np.random.default_rng(31)
+    vals = [0.0, -1.0, float("inf"), float("nan"), 2688.0, 1344.0, 6.0, 0.1, 2.0 ** -140, 3.0e38]
+    vals += [float(np.float32(v)) for v in np.exp(rng.uniform(-90, 88, 300))]
+    for v in vals:
+        want = orc.two_level_exponent(v) if np.isfinite(v) else 0
+        assert P.pact_two_level_exponent(v) == want, v
+
+
+def test_two_level_host_checks(P):
+    lib = P.pact.lib
+    pm = P_mod()
+    wc = pm.c_weight_cache()
+    n = P.pact_weight_cache_bytes(512, 512)
+    assert lib.pact_weight_layout_cache_scaled(0x3000, 512, 512, 512, 101, 0x10000, n, ctypes.byref(wc), None) == 1
+    assert lib.pact_absmax_bf16(None, 512, 512, 512, 0x2000, None) == 1
+    assert lib.pact_absmax_bf16(0x3000, 512, 512, 100, 0x2000, None) == 2
+    assert lib.pact_absmax_bf16(0x3008, 512, 512, 512, 0x2000, None) == 3
+    # GEMM with a cache exponent out of range
+    wcache = pm.c_weight_cache(pm.c_nvfp4(0x1000, 0x2000, 512, 512), pm.c_nvfp4(0x3000, 0x4000, 512, 512), 200)
+    xq = pm.c_nvfp4(0x5000, 0x6000, 256, 512)
+    assert lib.pact_frozen_gemm_fwd(ctypes.byref(xq), ctypes.byref(wcache), None, None, 0, 0x7000, 512, None) == 1

@@ -28,7 +28,7 @@ def _bits(t):
     return to_bits(t)
 
 
-def run_layer(name, M, graphs):
+def run_layer(name, M, graphs, two_level=False):
     import nvfp4_gemm_b200 as P
     from nvfp4_gemm_b200.layer import LayerShape, PactLayer
     c = synth.LAYERS[name]
@@ -37,7 +37,8 @@ def run_layer(name, M, graphs):
     d = lambda b: torch.from_numpy(np.ascontiguousarray(b).view(np.int16)).view(torch.bfloat16).to(dev)
     shape = LayerShape(M=M, H=c["H"], I=c["I"], KV=c["KV"])
     L = PactLayer(shape, {k: d(v) for k, v in inp["w"].items()}, {k: d(v) for k, v in inp["lora_a"].items()},
-                  {k: d(v) for k, v in inp["lora_b"].items()}, d(inp["gamma1"]), d(inp["gamma2"]))
+                  {k: d(v) for k, v in inp["lora_b"].items()}, d(inp["gamma1"]), d(inp["gamma2"]),
+                  two_level=two_level)
     L.bind(d(inp["h"]), d(inp["attn"]), d(inp["d_out"]), d(inp["d_qkv"]))
     ops = L.step_ops()
     if graphs:
@@ -59,15 +60,24 @@ def run_layer(name, M, graphs):
 
 
 def check_layer(L, inp, orc, rows):
-    """Teacher-forced stage checks; GEMM outputs on `rows` (None = all rows)."""
+    """Teacher-forced stage checks; GEMM outputs on `rows` (None = all rows).  With a
+    two-level layer, group k's GEMM outputs are 2^g (frozen + LoRA activations . W),
+    its T and U carry s 2^-g and dA is scaled back by 2^g (g = L.gexp[k])."""
     S = L.s
     H, I, KV, r, s = S.H, S.I, S.KV, S.r, S.scale
     f = synth.bf16_bits_to_f64
     sel = slice(None) if rows is None else rows
     cat = lambda names, dct: np.concatenate([dct[n] for n in names], 0)
-    wf, wb = {}, {}
+    wf, wb, ge = {}, {}, {}
     for key, names in (("qkv", ("q", "k", "v")), ("o", ("o",)), ("gu", ("gate", "up")), ("d", ("down",))):
-        wf[key], wb[key] = orc.weight_cache(cat(names, inp["w"]))
+        if L.two_level:
+            ge[key], wf[key], wb[key] = orc.weight_cache_two_level(cat(names, inp["w"]))
+        else:
+            ge[key] = 0
+            wf[key], wb[key] = orc.weight_cache(cat(names, inp["w"]))
+    assert ge == L.gexp
+    p2 = {k: 2.0 ** g for k, g in ge.items()}
+    sc = {k: s / p2[k] for k in ge}
     A = {"qkv": f(cat(("q", "k", "v"), inp["lora_a"])), "o": f(inp["lora_a"]["o"]),
          "gu": f(cat(("gate", "up"), inp["lora_a"])), "d": f(inp["lora_a"]["down"])}
     B = {"qkv": f(cat(("q", "k", "v"), inp["lora_b"])), "o": f(inp["lora_b"]["o"]),
@@ -99,7 +109,7 @@ def check_layer(L, inp, orc, rows):
 
     def lora_grads_tf(dy_bits, xt, u_dev, key, gA, gB, what):
         dy = f(dy_bits)
-        assert_close(to_f64(gA), orc.gemm_nt(u_dev.T, xt.T), f"dA {what}")
+        assert_close(to_f64(gA), p2[key] * orc.gemm_nt(u_dev.T, xt.T), f"dA {what}")
         db = np.zeros_like(B[key])
         lo = 0
         for i, hi in enumerate(seg[key]):
@@ -112,7 +122,7 @@ def check_layer(L, inp, orc, rows):
         out = np.zeros((dy.shape[0], len(seg[key]) * r))
         lo = 0
         for i, hi in enumerate(seg[key]):
-            out[:, i * r:(i + 1) * r] = s * orc.gemm_nt(dy[:, lo:hi], B[key][lo:hi].T)
+            out[:, i * r:(i + 1) * r] = sc[key] * orc.gemm_nt(dy[:, lo:hi], B[key][lo:hi].T)
             lo = hi
         return out
 
@@ -123,20 +133,21 @@ def check_layer(L, inp, orc, rows):
     nv_equal(L.xq1, xq1, "xq1")
     np.testing.assert_allclose(L.rstd1.cpu().numpy(), rstd1, rtol=1e-7)
     t_qkv = hilo(L.t_qkv)
-    assert_close(t_qkv, s * orc.gemm_nt(f(y1), A["qkv"]), "T qkv")
-    assert_close(to_f64(L.qkv)[sel], gemm_rows(xq1, wf["qkv"]) + lora_rows(t_qkv, "qkv", True), "qkv")
+    assert_close(t_qkv, sc["qkv"] * orc.gemm_nt(f(y1), A["qkv"]), "T qkv")
+    assert_close(to_f64(L.qkv)[sel], p2["qkv"] * (gemm_rows(xq1, wf["qkv"]) + lora_rows(t_qkv, "qkv", True)), "qkv")
     aq = orc.quantize(attn)
     nv_equal(L.aq, aq, "q(attn)")
     t_o = hilo(L.t_o)
-    assert_close(t_o, s * orc.gemm_nt(f(attn), A["o"]), "T o")
-    assert_close(to_f64(L.h2)[sel], f(h)[sel] + gemm_rows(aq, wf["o"]) + lora_rows(t_o, "o", True), "h2")
+    assert_close(t_o, sc["o"] * orc.gemm_nt(f(attn), A["o"]), "T o")
+    assert_close(to_f64(L.h2)[sel], f(h)[sel] + p2["o"] * (gemm_rows(aq, wf["o"]) + lora_rows(t_o, "o", True)),
+                 "h2")
     h2 = _bits(L.h2)
     y2, xq2, rstd2 = orc.rmsnorm_quant(h2, inp["gamma2"], S.eps)
     assert np.array_equal(_bits(L.x2), y2), "x2"
     nv_equal(L.xq2, xq2, "xq2")
     t_gu = hilo(L.t_gu)
-    assert_close(t_gu, s * orc.gemm_nt(f(y2), A["gu"]), "T gu")
-    assert_close(to_f64(L.gu)[sel], gemm_rows(xq2, wf["gu"]) + lora_rows(t_gu, "gu", True), "gate|up")
+    assert_close(t_gu, sc["gu"] * orc.gemm_nt(f(y2), A["gu"]), "T gu")
+    assert_close(to_f64(L.gu)[sel], p2["gu"] * (gemm_rows(xq2, wf["gu"]) + lora_rows(t_gu, "gu", True)), "gate|up")
     gu = _bits(L.gu)
     m, mq, gq, uq = orc.silu_mul_quant(gu[:, :I], gu[:, I:])
     assert np.array_equal(_bits(L.m), m), "m"
@@ -144,14 +155,15 @@ def check_layer(L, inp, orc, rows):
     nv_equal(L.gq, gq, "gq")
     nv_equal(L.uq, uq, "uq")
     t_d = hilo(L.t_d)
-    assert_close(t_d, s * orc.gemm_nt(f(m), A["d"]), "T down")
-    assert_close(to_f64(L.out)[sel], f(h2)[sel] + gemm_rows(mq, wf["d"]) + lora_rows(t_d, "d", True), "out")
+    assert_close(t_d, sc["d"] * orc.gemm_nt(f(m), A["d"]), "T down")
+    assert_close(to_f64(L.out)[sel], f(h2)[sel] + p2["d"] * (gemm_rows(mq, wf["d"]) + lora_rows(t_d, "d", True)),
+                 "out")
     # ---- backward: down
     u_d = hilo(L.u_d)
     assert_close(u_d, u_ref(d_out, "d"), "U down")
     doq = orc.quantize(d_out)
     nv_equal(L.doq, doq, "q(d_out)")
-    assert_close(to_f64(L.dm)[sel], gemm_rows(doq, wb["d"]) + lora_rows(u_d, "d", False), "dm")
+    assert_close(to_f64(L.dm)[sel], p2["d"] * (gemm_rows(doq, wb["d"]) + lora_rows(u_d, "d", False)), "dm")
     dm = _bits(L.dm)
     dg, du = orc.silu_mul_bwd(f(dm), gq, uq)
     dgu_dev = to_f64(L.dgu)
@@ -166,7 +178,7 @@ def check_layer(L, inp, orc, rows):
     # gate|up
     u_gu = hilo(L.u_gu)
     assert_close(u_gu, u_ref(dgu, "gu"), "U gate|up")
-    assert_close(to_f64(L.dx2)[sel], gemm_rows(dguq, wb["gu"]) + lora_rows(u_gu, "gu", False), "dx2")
+    assert_close(to_f64(L.dx2)[sel], p2["gu"] * (gemm_rows(dguq, wb["gu"]) + lora_rows(u_gu, "gu", False)), "dx2")
     lora_grads_tf(dgu, xq2.dequantize(), u_gu, "gu", L.grads["a_gu"], L.grads["b_gu"], "gate|up")
     dx2 = _bits(L.dx2)
     dh2_ref = orc.rmsnorm_bwd(f(dx2), xq2, L.rstd2.cpu().numpy().astype(np.float64), inp["gamma2"]) + f(d_out)
@@ -177,14 +189,15 @@ def check_layer(L, inp, orc, rows):
     # o
     u_o = hilo(L.u_o)
     assert_close(u_o, u_ref(dh2, "o"), "U o")
-    assert_close(to_f64(L.dattn)[sel], gemm_rows(dh2q, wb["o"]) + lora_rows(u_o, "o", False), "d attn")
+    assert_close(to_f64(L.dattn)[sel], p2["o"] * (gemm_rows(dh2q, wb["o"]) + lora_rows(u_o, "o", False)), "d attn")
     lora_grads_tf(dh2, f(attn), u_o, "o", L.grads["a_o"], L.grads["b_o"], "o")
     # q|k|v
     u_qkv = hilo(L.u_qkv)
     assert_close(u_qkv, u_ref(d_qkv, "qkv"), "U qkv")
     dqkvq = orc.quantize(d_qkv)
     nv_equal(L.dqkvq, dqkvq, "q(d_qkv)")
-    assert_close(to_f64(L.dx1)[sel], gemm_rows(dqkvq, wb["qkv"]) + lora_rows(u_qkv, "qkv", False), "dx1")
+    assert_close(to_f64(L.dx1)[sel], p2["qkv"] * (gemm_rows(dqkvq, wb["qkv"]) + lora_rows(u_qkv, "qkv", False)),
+                 "dx1")
     lora_grads_tf(d_qkv, xq1.dequantize(), u_qkv, "qkv", L.grads["a_qkv"], L.grads["b_qkv"], "qkv")
     dh_ref = orc.rmsnorm_bwd(f(_bits(L.dx1)), xq1, L.rstd1.cpu().numpy().astype(np.float64),
                              inp["gamma1"]) + f(dh2)
@@ -203,6 +216,14 @@ def small_layer(monkeypatch):
 @pytest.mark.parametrize("graphs", [False, True])
 def test_layer_small_all_rows(orc, small_layer, graphs):
     L, inp = run_layer(small_layer, 300, graphs)
+    check_layer(L, inp, orc, rows=None)
+
+
+def test_layer_small_two_level(orc, small_layer):
+    """The two-level weight layouts through the whole layer (weights with 1% x20
+    outliers), in the bench's launch configuration, all rows."""
+    L, inp = run_layer(small_layer, 300, graphs=True, two_level=True)
+    assert all(g < 0 for g in L.gexp.values())
     check_layer(L, inp, orc, rows=None)
 
 
