@@ -55,6 +55,8 @@ def parse():
     ap.add_argument("--ops", action="store_true",
                     help="time each op of the layer step alone: one JSON line per op with its roofline")
     ap.add_argument("--only", default=None, help="with --ops: time only the ops whose name contains this")
+    ap.add_argument("--two-level", action="store_true",
+                    help="cache the frozen weights in the two-level variant (a power of two per tensor)")
     return ap.parse_args()
 
 
@@ -171,14 +173,34 @@ class Replicas:
 
 
 # ------------------------------------------------------------------ CPU oracle
-def oracle_layer(name, inputs):
+# DRAM bytes (read + write) per k_nvfp4_gemm launch, mean over the 8 GEMMs of the
+# Llama-3.2-1B layer step, from one ncu capture of the step's first eager pass (cold
+# L2).  Valid only for the GEMM source it was taken on: reported as null once
+# csrc/gemm.cu or csrc/common.cuh differ from these hashes.
+GEMM_TRAFFIC = {"workload": "llama-3.2-1b", "bytes_per_launch": 17724416,
+                "sha256_16": {"gemm.cu": "fe1bc968079a405c", "common.cuh": "774f32b5d22d6330"}}
+
+
+def gemm_traffic(workload):
+    import hashlib
+    if workload != GEMM_TRAFFIC["workload"]:
+        return None
+    csrc = os.path.join(os.path.dirname(os.path.abspath(__file__)), "nvfp4_gemm_b200", "csrc")
+    for name, h in GEMM_TRAFFIC["sha256_16"].items():
+        with open(os.path.join(csrc, name), "rb") as f:
+            if hashlib.sha256(f.read()).hexdigest()[:16] != h:
+                return None
+    return GEMM_TRAFFIC["bytes_per_launch"]
+
+
+def oracle_layer(name, inputs, two_level=False):
     import oracle
     from oracle.layer import OracleLayer
     import synth
     oracle.build()
     c = synth.LAYERS[name]
     return OracleLayer(c["H"], c["I"], c["KV"], synth.LORA_R, synth.LORA_ALPHA, synth.RMS_EPS, inputs["w"],
-                       inputs["lora_a"], inputs["lora_b"], inputs["gamma1"], inputs["gamma2"])
+                       inputs["lora_a"], inputs["lora_b"], inputs["gamma1"], inputs["gamma2"], two_level=two_level)
 
 
 def oracle_rate(layer, inputs, tokens, min_seconds=10.0, max_steps=20):
@@ -205,7 +227,7 @@ def reference_arm(a):
     import synth
     M = synth.tokens(a.workload)
     inputs = synth.layer_inputs(a.workload)
-    layer = oracle_layer(a.workload, inputs)
+    layer = oracle_layer(a.workload, inputs, a.two_level)
     for _ in range(max(0, min(a.warmup, 1))):
         layer.step(inputs["h"][:8], inputs["attn"][:8], inputs["d_out"][:8], inputs["d_qkv"][:8])
     tok = max(8, min(a.cpu_tokens, M))
@@ -232,7 +254,7 @@ def config_block(name, M):
 
 
 # ------------------------------------------------------------------ GPU arm
-def make_layer(name, dev):
+def make_layer(name, dev, two_level=False):
     """The layer of workload `name` on device `dev` with its seeded synthetic inputs bound."""
     import torch
     import synth
@@ -245,7 +267,8 @@ def make_layer(name, dev):
                        eps=synth.RMS_EPS)
     layer = PactLayer(shape, {k: d(v) for k, v in inputs["w"].items()},
                       {k: d(v) for k, v in inputs["lora_a"].items()},
-                      {k: d(v) for k, v in inputs["lora_b"].items()}, d(inputs["gamma1"]), d(inputs["gamma2"]))
+                      {k: d(v) for k, v in inputs["lora_b"].items()}, d(inputs["gamma1"]), d(inputs["gamma2"]),
+                      two_level=two_level)
     x_in = {k: d(inputs[k]) for k in ("h", "attn", "d_out", "d_qkv")}
     layer.bind(x_in["h"], x_in["attn"], x_in["d_out"], x_in["d_qkv"])
     return inputs, layer, x_in
@@ -365,7 +388,7 @@ def main():
     world, rank = rep.world, rep.rank
 
     M = synth.tokens(a.workload)
-    inputs, layer, x_in = make_layer(a.workload, dev)
+    inputs, layer, x_in = make_layer(a.workload, dev, a.two_level)
     if a.ops:
         return op_table(a, layer, dev)
     ops = layer.step_ops()
@@ -521,7 +544,7 @@ def main():
 
     cpu = None
     if rank == 0 and world == 1 and not a.no_cpu_baseline:
-        ol = oracle_layer(a.workload, inputs)
+        ol = oracle_layer(a.workload, inputs, a.two_level)
         rate, n, el, cores = oracle_rate(ol, inputs, min(a.cpu_tokens, M))
         cpu = {"value": rate, "unit": "tokens/s", "cores": cores, "kind": "oracle",
                "sample": f"{min(a.cpu_tokens, M)} of {M} tokens per step ({n} steps, {el:.1f} s), one layer "
@@ -531,12 +554,15 @@ def main():
         "metric": METRIC, "value": tokens_per_s, "unit": "tokens/s", "n_gpus": world, "steps": K,
         "warmup": a.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "nvfp4", "data": "synthetic",
-        "config": {**config_block(a.workload, M), "parallelism": f"dp{world}" if world > 1 else "single"},
+        "config": {**config_block(a.workload, M), "parallelism": f"dp{world}" if world > 1 else "single",
+                   **({"weights": "two-level layouts (a power of two per cached tensor)"} if a.two_level else {})},
         "frozen_proj_tflops": tflops,
         "frac_fp4_peak": tflops / fp4_peak,
         "roofline": {"bound": "tensor", "kernel": "k_nvfp4_gemm (frozen fwd + dgrad GEMMs)",
                      "achieved": tflops, "peak": fp4_peak, "unit": "TFLOP/s", "frac": tflops / fp4_peak,
-                     "traffic": None,
+                     "traffic": gemm_traffic(a.workload),
+                     "traffic_note": "DRAM read+write bytes per launch, mean over the 8 layer GEMMs, one ncu "
+                                     "capture with cold L2 (outputs stay in L2); null when the GEMM source changed",
                      "peak_note": f"{pk['src']} burst BF16 {pk['bf16']} TF/s x {FP4_PER_BF16} "
                                   f"(nominal FP4/BF16 ratio); GEMM launches timed alone, cold L2",
                      "flops_per_step": gemm_flops, "avg_launch_ms": gemm_launch_ms},
