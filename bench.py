@@ -193,6 +193,15 @@ def gemm_traffic(workload):
     return GEMM_TRAFFIC["bytes_per_launch"]
 
 
+def bf16_lora_saved_bytes(M, H, I, r):
+    """Activation bytes a plain BF16 LoRA layer of the same scope (attention core
+    excluded) keeps for its backward under autograd: the RMSNorm inputs h and h2 (BF16)
+    and their rstd (FP32); the adapters' inputs x_norm1 (shared by q, k, v), attn,
+    x_norm2 (shared by gate, up) and m; gate and up for the SiLU-multiply backward;
+    the rank-r intermediates A x of the seven adapters (BF16)."""
+    return 2 * 2 * M * H + 2 * 4 * M + 3 * 2 * M * H + 2 * M * I + 2 * 2 * M * I + 7 * 2 * M * r
+
+
 def oracle_layer(name, inputs, two_level=False):
     import oracle
     from oracle.layer import OracleLayer
@@ -571,6 +580,12 @@ def main():
                 "d2h_bytes_per_step": d2h,
                 "note": "inputs copied from pinned host memory every step, the next step's copy overlapping the "
                         "current step; LoRA gradients read back every step"},
+        "saved_activation_bytes": {
+            "pact": layer.saved_bytes(), "bf16_lora_model": bf16_lora_saved_bytes(M, layer.s.H, layer.s.I, layer.s.r),
+            "note": "bytes held from forward to backward per layer (the NVFP4 copies, rstd, attn) against an "
+                    "autograd count for a BF16 LoRA layer of the same scope"},
+        "weight_bytes": {"pact_cached_layouts": layer.weight_cache_bytes(),
+                         "bf16": 2 * int(layer.s.frozen_flops() / (4.0 * M))},
         "gpu_launches": launches_per_step * K,
         "clocks": clk.summary(),
         "segments_ms": {"+".join(op.name for op in sg["ops"]): round(t, 4) for sg, t in zip(segs, seg_ms)},

@@ -210,8 +210,8 @@ __device__ __forceinline__ float sigmoid_fast(float g) { return __fdividef(1.0f,
 
 __device__ __forceinline__ float silu_mul_round(float g, float u, float s) {
     const float m = __fmul_rn(__fmul_rn(g, s), u);
-    const int lo = (int)(__float_as_uint(m) & 0xFFFFu);
-    if (abs(lo - 0x8000) <= 24 || !(fabsf(g) <= 4.0f) || !isfinite(m)) {
+    // |low 16 bits - 0x8000| <= 24, as one unsigned range test
+    if ((__float_as_uint(m) & 0xFFFFu) - 0x7FE8u <= 48u || !(fabsf(g) <= 4.0f) || !isfinite(m)) {
         const double gd = (double)g;
         return __bfloat162float(__double2bfloat16((gd / (1.0 + exp(-gd))) * (double)u));
     }
@@ -263,16 +263,17 @@ __global__ void __launch_bounds__(256) k_silu_mul_quant(const pact_bf16 *__restr
 #pragma unroll
             for (int i = 0; i < 8; ++i) mv[i] = valid ? silu_mul_out(gv[i], uv[i]) : 0.0f;
             if (valid && m) store8_bf16(m + row * I + c, mv);
+            const ChunkAt at = chunk_at(row, c0, I);   // mq, gq and uq share their shape
             uint32_t sb;
             uint32_t codes = quant8(mv, &sb);
-            store_chunk(mq, row, c0, codes, sb, valid);
+            store_chunk_at(mq, at, codes, sb, valid);
             if (has_gq) {
                 codes = quant8(gv, &sb);
-                store_chunk(gq, row, c0, codes, sb, valid);
+                store_chunk_at(gq, at, codes, sb, valid);
             }
             if (has_uq) {
                 codes = quant8(uv, &sb);
-                store_chunk(uq, row, c0, codes, sb, valid);
+                store_chunk_at(uq, at, codes, sb, valid);
             }
         }
         it = nx;
@@ -345,11 +346,15 @@ __global__ void __launch_bounds__(256) k_silu_mul_bwd_quant(const pact_bf16 *__r
                 store8_bf16(dgu + row * lddgu + I + c, du);
                 if (m_re) store8_bf16(m_re + row * I + c, mr);
             }
+            // du's chunk sits I columns to the right: I / 2 code bytes, and I / 64 whole
+            // scale tiles (I is a multiple of 64)
+            const ChunkAt at = chunk_at(row, c0, 2 * I);
+            const ChunkAt at_u = {at.code_off + (I >> 1), at.scale_off + (I >> 6) * 512};
             uint32_t sb;
             uint32_t codes = quant8(dg, &sb);
-            store_chunk(dguq, row, c0, codes, sb, valid);
+            store_chunk_at(dguq, at, codes, sb, valid);
             codes = quant8(du, &sb);
-            store_chunk(dguq, row, c0 + I, codes, sb, valid);
+            store_chunk_at(dguq, at_u, codes, sb, valid);
         }
         it = nx;
         cur = nxt;

@@ -98,18 +98,27 @@ __device__ __forceinline__ uint32_t gather_scales4(uint32_t sb) {
 // chunk starting at column c0 of row `row`.  `valid` is false for lanes whose 8
 // columns lie past the end of the row (cols is a multiple of 64, so validity is
 // uniform over each group of 8 lanes).
-__device__ __forceinline__ void store_chunk(const pact_nvfp4_t &t, int64_t row, int64_t c0, uint32_t codes,
-                                            uint32_t sb, bool valid) {
+// Byte offsets of this lane's 4 code bytes and (lanes 8q) of its scale word inside
+// a tensor with `cols` columns; tensors of one shape share them.
+struct ChunkAt {
+    int64_t code_off, scale_off;
+};
+__device__ __forceinline__ ChunkAt chunk_at(int64_t row, int64_t c0, int64_t cols) {
+    const int lane = threadIdx.x & 31;
+    return {row * (cols >> 1) + ((c0 + 8 * lane) >> 1), scale_offset(row, (c0 >> 4) + (lane >> 1), cols)};
+}
+__device__ __forceinline__ void store_chunk_at(const pact_nvfp4_t &t, const ChunkAt &at, uint32_t codes, uint32_t sb,
+                                               bool valid) {
     const int lane = threadIdx.x & 31;
     const uint32_t packed = gather_scales4(sb);
     if (valid) {
-        uint8_t *cp = static_cast<uint8_t *>(t.codes) + row * (t.cols >> 1) + ((c0 + 8 * lane) >> 1);
-        *reinterpret_cast<uint32_t *>(cp) = codes;
-        if ((lane & 7) == 0) {
-            const int64_t blk = (c0 >> 4) + (lane >> 1);
-            *reinterpret_cast<uint32_t *>(static_cast<uint8_t *>(t.scales) + scale_offset(row, blk, t.cols)) = packed;
-        }
+        *reinterpret_cast<uint32_t *>(static_cast<uint8_t *>(t.codes) + at.code_off) = codes;
+        if ((lane & 7) == 0) *reinterpret_cast<uint32_t *>(static_cast<uint8_t *>(t.scales) + at.scale_off) = packed;
     }
+}
+__device__ __forceinline__ void store_chunk(const pact_nvfp4_t &t, int64_t row, int64_t c0, uint32_t codes,
+                                            uint32_t sb, bool valid) {
+    store_chunk_at(t, chunk_at(row, c0, t.cols), codes, sb, valid);
 }
 
 // Load 8 BF16 values (16 bytes) as floats.

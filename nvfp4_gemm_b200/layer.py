@@ -274,6 +274,26 @@ class PactLayer:
                bytes=2 * M * H + S.nv(M, H) + 4 * M + 2 * H + 2 * M * H + 2 * M * H),
         ]
 
+    def saved_for_backward(self) -> Dict[str, torch.Tensor]:
+        """The device tensors the forward leaves for the backward, i.e. the activation
+        memory a layer holds between its forward and its backward: the NVFP4 copies
+        (codes and padded scales) of both RMSNorm outputs and of gate and up, the two
+        rstd vectors, and the attention output the o adapter's gradient reads.  The
+        BF16 RMSNorm outputs, m and T are dead once the forward has used them."""
+        _, attn, _, _ = self.inputs
+        out = {"rstd1": self.rstd1, "rstd2": self.rstd2, "attn": attn}
+        for name in ("xq1", "xq2", "gq", "uq"):
+            t = getattr(self, name)
+            out[name + ".codes"], out[name + ".scales"] = t.codes, t.scales
+        return out
+
+    def saved_bytes(self) -> int:
+        return sum(t.numel() * t.element_size() for t in self.saved_for_backward().values())
+
+    def weight_cache_bytes(self) -> int:
+        """Device bytes of the four cached weight groups (both layouts each)."""
+        return sum(c.buf.numel() for c in (self.c_qkv, self.c_o, self.c_gu, self.c_d))
+
     def step_ops(self) -> List[Op]:
         return self.forward_ops() + self.backward_ops()
 

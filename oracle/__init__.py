@@ -398,3 +398,14 @@ def lora_bwd_at(dy: np.ndarray, xt: np.ndarray, a: np.ndarray, b: np.ndarray, sc
     db = scale * gemm_nt(dy.T, t.T)
     da = scale * gemm_nt(u.T, xt.T)
     return da, db, scale * u
+
+
+# ------------------------------------------------------------- saved activations
+def saved_bytes_pact(M: int, H: int, I: int) -> int:
+    """Bytes a PACT layer of M tokens holds from its forward for its backward
+    ([METHOD] bullet 2: the quantized RMSNorm outputs are reused, gate and up are kept
+    as NVFP4 copies; the o adapter reads the BF16 attention output): NVFP4 [M x H]
+    twice and [M x I] twice (codes plus padded scales), two FP32 rstd vectors of M,
+    and the BF16 attention output [M x H]."""
+    nv = lambda rows, cols: rows * cols // 2 + scale_bytes(rows, cols)
+    return 2 * nv(M, H) + 2 * nv(M, I) + 2 * 4 * M + 2 * M * H

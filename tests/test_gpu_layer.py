@@ -217,6 +217,7 @@ def small_layer(monkeypatch):
 def test_layer_small_all_rows(orc, small_layer, graphs):
     L, inp = run_layer(small_layer, 300, graphs)
     check_layer(L, inp, orc, rows=None)
+    assert L.saved_bytes() == orc.saved_bytes_pact(300, L.s.H, L.s.I)
 
 
 def test_layer_small_two_level(orc, small_layer):
@@ -232,6 +233,7 @@ def test_layer_full_size(orc, name):
     """The other two layer workloads (Qwen2.5-1.5B at 2048 tokens; Llama-3.2-3B at
     8192 tokens with 1% x20 weight outliers) in the bench's launch configuration."""
     L, inp = run_layer(name, synth.tokens(name), graphs=True)
+    assert L.saved_bytes() == orc.saved_bytes_pact(L.s.M, L.s.H, L.s.I)
     rows = np.sort(np.random.default_rng(12).choice(L.s.M, size=32, replace=False))
     rows[-1] = L.s.M - 1
     check_layer(L, inp, orc, rows=rows)

@@ -548,3 +548,11 @@ def test_two_level_gemm_scales_the_frozen_product_only(orc):
     lora_d = 2.0 * (bf16_bits_value(dy) @ bf16_bits_value(b)) @ bf16_bits_value(a)
     ref_d = 2.0 ** e * (orc.dequantize(orc.quantize(dy)) @ orc.dequantize(wb).T) + lora_d
     np.testing.assert_allclose(dx, ref_d, rtol=1e-12, atol=1e-12)
+
+
+def test_saved_bytes_pact_hand_count(orc):
+    """M = 200 tokens, H = 64, I = 192, counted by hand: codes M*H/2 = 6400; scales
+    pad rows to 256 and blocks to a multiple of 4: 256 * 4 = 1024 (H) and 256 * 12 =
+    3072 (I); codes M*I/2 = 19200; rstd 2 * 800; attn 2 * 200 * 64 = 25600."""
+    want = 2 * (6400 + 1024) + 2 * (19200 + 3072) + 1600 + 25600
+    assert orc.saved_bytes_pact(200, 64, 192) == want
