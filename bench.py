@@ -193,6 +193,26 @@ def gemm_traffic(workload):
     return GEMM_TRAFFIC["bytes_per_launch"]
 
 
+def gpu_local_cpus(dev):
+    """The CPUs NVML lists as local to the GPU (its NUMA node), within this process's
+    allowed set; empty when NVML cannot tell."""
+    import torch
+    try:
+        import pynvml
+        props = torch.cuda.get_device_properties(dev)
+        pynvml.nvmlInit()
+        try:
+            h = pynvml.nvmlDeviceGetHandleByPciBusId(
+                f"{props.pci_domain_id:08x}:{props.pci_bus_id:02x}:{props.pci_device_id:02x}.0")
+            words = pynvml.nvmlDeviceGetCpuAffinity(h, (os.cpu_count() + 63) // 64)
+        finally:
+            pynvml.nvmlShutdown()
+        cpus = {64 * i + b for i, w in enumerate(words) for b in range(64) if (int(w) >> b) & 1}
+        return cpus & os.sched_getaffinity(0)
+    except Exception:
+        return set()
+
+
 def bf16_lora_saved_bytes(M, H, I, r):
     """Activation bytes a plain BF16 LoRA layer of the same scope (attention core
     excluded) keeps for its backward under autograd: the RMSNorm inputs h and h2 (BF16)
@@ -499,7 +519,16 @@ def main():
     # all K steps, from the first copy to the last gradient read-back.
     keys = ("h", "attn", "d_out", "d_qkv")
     sizes = [x_in[k].numel() for k in keys]          # multiples of 8: every view is 16-byte aligned
-    host_flat = torch.empty(sum(sizes), dtype=torch.bfloat16).pin_memory()
+    # pinned buffers on the GPU's NUMA node: allocated and first touched by this thread
+    # while it runs on the GPU's local CPUs (the previous CPU set comes back after)
+    allowed, local_cpus = os.sched_getaffinity(0), gpu_local_cpus(dev)
+    if local_cpus:
+        os.sched_setaffinity(0, local_cpus)
+    try:
+        host_flat = torch.empty(sum(sizes), dtype=torch.bfloat16, pin_memory=True)
+        host_out = [torch.empty(gt.shape, dtype=gt.dtype, pin_memory=True) for gt in grads]
+    finally:
+        os.sched_setaffinity(0, allowed)
     dev_flat = [torch.empty(sum(sizes), dtype=torch.bfloat16, device=dev) for _ in range(2)]
 
     def views(flat):
@@ -511,7 +540,6 @@ def main():
 
     for k, v in views(host_flat).items():
         v.copy_(x_in[k].cpu())
-    host_out = [gt.cpu().pin_memory() for gt in grads]
     h2d = host_flat.numel() * host_flat.element_size()
     d2h = sum(t.numel() * t.element_size() for t in host_out)
     graphs = []
@@ -579,7 +607,9 @@ def main():
         "e2e": {"value": M * K * world / (e2e_ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h,
                 "note": "inputs copied from pinned host memory every step, the next step's copy overlapping the "
-                        "current step; LoRA gradients read back every step"},
+                        "current step; LoRA gradients read back every step",
+                "host_buffers": (f"pinned on the GPU's NUMA node ({len(local_cpus)} local CPUs)" if local_cpus
+                                 else "pinned; the GPU's NUMA node unknown")},
         "saved_activation_bytes": {
             "pact": layer.saved_bytes(), "bf16_lora_model": bf16_lora_saved_bytes(M, layer.s.H, layer.s.I, layer.s.r),
             "note": "bytes held from forward to backward per layer (the NVFP4 copies, rstd, attn) against an "
