@@ -201,17 +201,20 @@ __global__ void __launch_bounds__(RMS_THREADS, 2) k_rmsnorm_quant(const pact_bf1
 // m = BF16_RNE(silu(g) * u), exactly rounded.  The FP32 evaluation with the fast
 // exponential and division has a relative error of at most (5 + 1.16 |g|) FP32
 // ulps (CUDA's documented bounds for __expf and __fdividef plus three roundings),
-// i.e. at most 2 (5 + 1.16 |g|) = 10 + 2.32 |g| ulps of the result, under 19.3
-// for |g| <= 4.  It decides unless it lies within 24 ulps of a BF16 midpoint, and
-// the double expression decides otherwise and for |g| > 4 (Ziv's method, as
-// above).  Gate activations beyond 4 in magnitude are rare, so the double path
-// stays rare, and the margin is one constant (no conversion per element).
+// i.e. at most 2 (5 + 1.16 |g|) = 10 + 2.32 |g| ulps of the result: under 19.3 for
+// |g| <= 4 and under 47.2 for |g| <= 16.  It decides unless it lies within 24 (resp.
+// 48) ulps of a BF16 midpoint, and the double expression decides otherwise and for
+// |g| > 16 (Ziv's method, as above).  Two margins keep the double path rare both for
+// gate activations of unit scale and for the wider ones of outlier weights, without
+// a float-to-integer conversion per element.
 __device__ __forceinline__ float sigmoid_fast(float g) { return __fdividef(1.0f, 1.0f + __expf(-g)); }
 
 __device__ __forceinline__ float silu_mul_round(float g, float u, float s) {
     const float m = __fmul_rn(__fmul_rn(g, s), u);
-    // |low 16 bits - 0x8000| <= 24, as one unsigned range test
-    if ((__float_as_uint(m) & 0xFFFFu) - 0x7FE8u <= 48u || !(fabsf(g) <= 4.0f) || !isfinite(m)) {
+    // |low 16 bits - 0x8000| <= margin, as one unsigned range test
+    const float ag = fabsf(g);
+    const uint32_t margin = ag <= 4.0f ? 24u : 48u;
+    if ((__float_as_uint(m) & 0xFFFFu) + margin - 0x8000u <= 2u * margin || !(ag <= 16.0f) || !isfinite(m)) {
         const double gd = (double)g;
         return __bfloat162float(__double2bfloat16((gd / (1.0 + exp(-gd))) * (double)u));
     }

@@ -290,9 +290,10 @@ def test_rmsnorm_quant(P, orc, M, H):
     np.testing.assert_allclose(rstd.cpu().numpy(), rstd_ref, rtol=1e-7)
 
 
-@pytest.mark.parametrize("M,I", [(64, 512), (130, 8960), (257, 2048)])
-def test_silu_mul_quant(P, orc, M, I):
-    gu = synth.gaussian_bf16(4, (M, 2 * I), std=2.0)
+@pytest.mark.parametrize("M,I,std", [(64, 512, 2.0), (130, 8960, 2.0), (257, 2048, 2.0), (96, 2048, 9.0)])
+def test_silu_mul_quant(P, orc, M, I, std):
+    # std 2 reaches both margins of the rounding check; std 9 also |g| > 16 (FP64 path)
+    gu = synth.gaussian_bf16(4, (M, 2 * I), std=std)
     gud = to_dev(gu)
     m, mq, gq, uq = P.pact_silu_mul_quant(gud[:, :I], gud[:, I:])
     sync()
@@ -304,9 +305,9 @@ def test_silu_mul_quant(P, orc, M, I):
     assert_nvfp4_equal(uq, uq_ref, orc, "uq")
 
 
-@pytest.mark.parametrize("M,I", [(64, 512), (130, 2048)])
-def test_silu_mul_bwd_quant(P, orc, M, I):
-    gu = synth.gaussian_bf16(4, (M, 2 * I), std=2.0)
+@pytest.mark.parametrize("M,I,std", [(64, 512, 2.0), (130, 2048, 2.0), (96, 1024, 9.0)])
+def test_silu_mul_bwd_quant(P, orc, M, I, std):
+    gu = synth.gaussian_bf16(4, (M, 2 * I), std=std)
     dm = synth.gaussian_bf16(56, (M, I))
     _, _, gq, uq = orc.silu_mul_quant(gu[:, :I], gu[:, I:])
     gqd, uqd = _nvfp4_from_oracle(P, gq, orc), _nvfp4_from_oracle(P, uq, orc)
