@@ -265,8 +265,11 @@ static pact_status launch_mma(const CUtensorMap &ta, const CUtensorMap &tb, cons
 
 // Split a contraction of length `len` over CTAs so that `blocks` output blocks x
 // splits covers the SMs, with at least 4 stages (256 elements) per split.
+// Splits of the contraction so that blocks x splits CTAs fill the SMs in ONE wave
+// (a CTA takes a whole SM: 132 KB of shared memory), each split at least 4 stages
+// long.  Rounding the split count up instead left a nearly empty second wave.
 static void choose_split(int64_t len, int64_t blocks, int *splits, int *kps) {
-    int64_t s = (sm_count() + blocks - 1) / (blocks > 0 ? blocks : 1);
+    int64_t s = sm_count() / (blocks > 0 ? blocks : 1);
     const int64_t max_s = (len + 4 * BK - 1) / (4 * BK);
     if (s > max_s) s = max_s;
     if (s < 1) s = 1;
