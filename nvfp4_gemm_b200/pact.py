@@ -268,14 +268,16 @@ def pact_weight_layout_cache(W: torch.Tensor, stream=None, two_level: bool = Fal
     buf = torch.empty(nbytes + 256, dtype=torch.uint8, device=W.device)
     off = (-buf.data_ptr()) % 256
     buf = buf[off:off + nbytes]
-    gexp = 0
+    c = c_weight_cache()
     if two_level:
         amax = pact_absmax_bf16(W, stream=stream)
         torch.cuda.synchronize(W.device)       # the kernel may run on a caller's stream
         gexp = pact_two_level_exponent(float(amax.cpu()))
-    c = c_weight_cache()
-    _check(_lib.pact_weight_layout_cache_scaled(W.data_ptr(), _ld(W), N, K, gexp, buf.data_ptr(), nbytes,
-                                                ctypes.byref(c), _stream(stream)))
+        _check(_lib.pact_weight_layout_cache_scaled(W.data_ptr(), _ld(W), N, K, gexp, buf.data_ptr(), nbytes,
+                                                    ctypes.byref(c), _stream(stream)))
+    else:
+        _check(_lib.pact_weight_layout_cache(W.data_ptr(), _ld(W), N, K, buf.data_ptr(), nbytes, ctypes.byref(c),
+                                             _stream(stream)))
     return WeightCache(buf, c, N, K)
 
 
