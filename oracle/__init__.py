@@ -72,6 +72,8 @@ def _load():
             lib.orc_e2m1_rne_mag.argtypes = [D]
             lib.orc_e2m1_rne_mag.restype = ctypes.c_uint8
             lib.orc_quantize.argtypes = [P, I, I, I, P, P]
+            lib.orc_e2m1_codes_f64.argtypes = [P, P, I, P]
+            lib.orc_e4m3_scales_f64.argtypes = [P, I, P]
             lib.orc_dequantize.argtypes = [P, P, I, I, P]
             lib.orc_scale_bytes.argtypes = [I, I]
             lib.orc_scale_bytes.restype = I

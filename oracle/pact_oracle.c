@@ -117,6 +117,23 @@ uint8_t orc_e2m1_rne_mag(double q) {
     return (uint8_t)best;
 }
 
+/* Element codes of real (double) values against given block scale bytes, as the
+ * GPTQ calibration needs them (its working weights are not BF16):
+ *   code_i = signbit(x_i) << 3 | E2M1_RNE_sat(|x_i| / E4M3(s_i)), magnitude 0 if s_i == 0. */
+void orc_e2m1_codes_f64(const double *x, const uint8_t *sbytes, int64_t n, uint8_t *codes) {
+    for (int64_t i = 0; i < n; ++i) {
+        double s = orc_e4m3_value(sbytes[i]);
+        uint8_t sign = signbit(x[i]) ? 8 : 0;
+        uint8_t mag = (s == 0.0) ? 0 : orc_e2m1_rne_mag(fabs(x[i]) / s);
+        codes[i] = sign | mag;
+    }
+}
+
+/* Scale bytes of block maxima: E4M3_RNE_sat(amax_i / 6). */
+void orc_e4m3_scales_f64(const double *amax, int64_t n, uint8_t *out) {
+    for (int64_t i = 0; i < n; ++i) out[i] = orc_e4m3_rne_sat(amax[i] / 6.0);
+}
+
 /* ------------------------------------------------------------ NVFP4 block quantizer */
 
 /* Quantize one block of 16 BF16 values [FAQ]:
