@@ -140,3 +140,31 @@ def test_two_level_host_checks(P):
     wcache = pm.c_weight_cache(pm.c_nvfp4(0x1000, 0x2000, 512, 512), pm.c_nvfp4(0x3000, 0x4000, 512, 512), 200)
     xq = pm.c_nvfp4(0x5000, 0x6000, 256, 512)
     assert lib.pact_frozen_gemm_fwd(ctypes.byref(xq), ctypes.byref(wcache), None, None, 0, 0x7000, 512, None) == 1
+
+
+def test_plain_c_program_links_and_calls_the_host_functions(P, tmp_path):
+    """A C99 program includes pact.h, links libpact.so and calls the calls that need no
+    GPU: the ABI version, the size queries, the two-level exponent and a rejected
+    argument check."""
+    import subprocess
+    src = tmp_path / "abi.c"
+    src.write_text(r'''
+#include <stdio.h>
+#include "pact.h"
+int main(void) {
+    pact_nvfp4_t t = {0, 0, 128, 100};
+    if (pact_abi_version() != PACT_ABI_VERSION) return 1;
+    if (pact_nvfp4_code_bytes(128, 64) != 4096) return 2;
+    if (pact_scale_bytes(200, 64) != 1024) return 3;
+    if (pact_two_level_exponent(2688.0f) != 0 || pact_two_level_exponent(0.1f) != -14) return 4;
+    if (pact_quantize_nvfp4((const pact_bf16 *)0x3000, 100, 128, 100, &t, 0) != PACT_ERR_SHAPE) return 5;
+    printf("ok\n");
+    return 0;
+}
+''')
+    exe = tmp_path / "abi"
+    lib_dir = os.path.dirname(P.pact.LIB_PATH)
+    subprocess.check_call(["gcc", "-std=c99", "-Wall", "-Werror", "-I", os.path.join(ROOT, "include"), str(src),
+                           "-L", lib_dir, "-lpact", f"-Wl,-rpath,{lib_dir}", "-o", str(exe)])
+    out = subprocess.run([str(exe)], capture_output=True, text=True)
+    assert out.returncode == 0 and out.stdout.strip() == "ok", (out.returncode, out.stdout, out.stderr)
