@@ -15,8 +15,9 @@ from __future__ import annotations
 
 import numpy as np
 
-from . import (bf16_to_f64, f64_to_bf16, gemm_nt, nvfp4_gemm, quantize, rmsnorm_bwd, rmsnorm_quant,
-               silu_mul_bwd, silu_mul_quant, silu_mul_recompute, weight_cache, weight_cache_two_level)
+from . import (bf16_to_f64, f64_to_bf16, frozen_dgrad, frozen_fwd, gemm_nt, lora_bwd, nvfp4_gemm, quantize,
+               rmsnorm_bwd, rmsnorm_quant, silu_mul_bwd, silu_mul_quant, silu_mul_recompute, weight_cache,
+               weight_cache_two_level)
 
 
 def _segments(seg_end):
@@ -55,11 +56,32 @@ def lora_grads(dy, xt, a, b, r, seg_end, scale):
     return da, db
 
 
+class OracleProjection:
+    """One frozen projection with its LoRA branch (w [N x K], A [r x K], B [N x r],
+    BF16 bits), forward and backward on X and dY:
+      Y = deq(q(X)) deq(Wf)^T + s (X A^T) B^T,  dX = deq(q(dY)) deq(Wb)^T + s (dY B) A,
+      dA = s (dY B)^T X~,  dB = s dY^T (X~ A^T),  X~ = deq(q(X)) the saved NVFP4 copy."""
+
+    input_keys = ("x", "dy")
+
+    def __init__(self, w, a, b, r, alpha):
+        self.wf, self.wb = weight_cache(w)
+        self.a, self.b, self.r, self.scale = a, b, r, alpha / r
+
+    def step(self, x, dy):
+        xq = quantize(x)
+        da, db, _ = lora_bwd(dy, xq.dequantize(), self.a, self.b, self.scale)
+        return {"y": f64_to_bf16(frozen_fwd(xq, self.wf, x, self.a, self.b, self.scale)),
+                "dx": f64_to_bf16(frozen_dgrad(dy, self.wb, self.a, self.b, self.scale)), "dA": da, "dB": db}
+
+
 class OracleLayer:
     """w, lora_a, lora_b: dicts of BF16 bit arrays keyed q, k, v, o, gate, up, down
     (PyTorch [out, in] layout); gamma1, gamma2: BF16 bits [H].  two_level: cache the
     weights in the two-level variant (weight_cache_two_level), one exponent per
     concatenated group."""
+
+    input_keys = ("h", "attn", "d_out", "d_qkv")
 
     def __init__(self, H, I, KV, r, alpha, eps, w, lora_a, lora_b, gamma1, gamma2, two_level=False):
         self.H, self.I, self.KV, self.r, self.eps = H, I, KV, r, eps

@@ -29,10 +29,11 @@ _M2 = np.uint64(0x94D049BB133111EB)
 PROJ = ("q", "k", "v", "o", "gate", "up", "down")
 
 
-def _splitmix64(seed: int, n: int) -> np.ndarray:
-    """n outputs of splitmix64 started at state ``seed`` (counter form)."""
+def _splitmix64(seed: int, n: int, offset: int = 0) -> np.ndarray:
+    """Outputs offset+1 .. offset+n of splitmix64 started at state ``seed`` (counter
+    form: output i is the finaliser of seed + i * golden)."""
     with np.errstate(over="ignore"):
-        i = np.arange(1, n + 1, dtype=np.uint64)
+        i = np.arange(offset + 1, offset + n + 1, dtype=np.uint64)
         z = np.uint64(seed & 0xFFFFFFFFFFFFFFFF) + i * _GOLDEN
         z = (z ^ (z >> np.uint64(30))) * _M1
         z = (z ^ (z >> np.uint64(27))) * _M2
@@ -40,16 +41,19 @@ def _splitmix64(seed: int, n: int) -> np.ndarray:
     return z
 
 
-def uniform(tensor_id: int, n: int) -> np.ndarray:
-    """n float64 uniforms in (0, 1) from the stream of ``tensor_id``."""
-    z = _splitmix64(SEED_BASE + tensor_id, n)
+def uniform(tensor_id: int, n: int, offset: int = 0) -> np.ndarray:
+    """Uniforms offset .. offset+n-1 in (0, 1) of the stream of ``tensor_id`` (float64)."""
+    z = _splitmix64(SEED_BASE + tensor_id, n, offset)
     return ((z >> np.uint64(11)).astype(np.float64) + 0.5) * (2.0 ** -53)
 
 
-def normal(tensor_id: int, n: int) -> np.ndarray:
-    """n float64 standard normals (Box-Muller over consecutive uniform pairs)."""
+def normal(tensor_id: int, n: int, offset: int = 0) -> np.ndarray:
+    """Standard normals offset .. offset+n-1 of the stream of ``tensor_id`` (float64;
+    Box-Muller over consecutive uniform pairs, normal 2j and 2j+1 from uniforms 2j
+    and 2j+1; ``offset`` must be even)."""
+    assert offset % 2 == 0
     m = (n + 1) // 2
-    u = uniform(tensor_id, 2 * m)
+    u = uniform(tensor_id, 2 * m, offset)
     r = np.sqrt(-2.0 * np.log(u[0::2]))
     t = 2.0 * np.pi * u[1::2]
     out = np.empty(2 * m, dtype=np.float64)
@@ -71,10 +75,28 @@ def bf16_bits_to_f64(b: np.ndarray) -> np.ndarray:
     return (np.asarray(b, dtype=np.uint16).astype(np.uint32) << 16).view(np.float32).astype(np.float64)
 
 
+_CHUNK = 1 << 22   # elements generated at a time (bounds the float64 temporaries)
+
+
 def gaussian_bf16(tensor_id: int, shape, std: float = 1.0, mean: float = 0.0) -> np.ndarray:
     """BF16 bit pattern (uint16 array of ``shape``) of mean + std * N(0, 1)."""
     n = int(np.prod(shape))
-    return f64_to_bf16_bits(mean + std * normal(tensor_id, n)).reshape(shape)
+    out = np.empty(n, dtype=np.uint16)
+
+    def fill(o):
+        k = min(_CHUNK, n - o)
+        out[o:o + k] = f64_to_bf16_bits(mean + std * normal(tensor_id, k, o))
+
+    starts = range(0, n, _CHUNK)
+    if len(starts) > 1:   # chunks are independent (counter-based stream): numpy releases the GIL
+        from concurrent.futures import ThreadPoolExecutor
+        import os
+        with ThreadPoolExecutor(max_workers=min(len(starts), os.cpu_count() or 1, 16)) as ex:
+            list(ex.map(fill, starts))
+    else:
+        for o in starts:
+            fill(o)
+    return out.reshape(shape)
 
 
 def weight_bf16(p: int, shape, outliers: bool = False) -> np.ndarray:
@@ -102,6 +124,17 @@ RMS_EPS = 1e-5
 
 # single projection + LoRA: X[256x512], W[512x512]
 SINGLE = dict(M=256, N=512, K=512)
+
+
+def single_inputs(r: int = LORA_R) -> dict:
+    """BF16 bit arrays of the single-projection workload: X [M x K] ~ N(0, 1) (tensor
+    id 1), W [N x K] ~ N(0, 0.02^2) (the q weight's stream, id 10), LoRA A [r x K] and
+    B [N x r] ~ N(0, 0.02^2) (ids 20, 30), upstream gradient dY [M x N] ~ N(0, 1)
+    (id 50)."""
+    M, N, K = SINGLE["M"], SINGLE["N"], SINGLE["K"]
+    return {"w": weight_bf16(0, (N, K)), "lora_a": gaussian_bf16(20, (r, K), std=0.02),
+            "lora_b": gaussian_bf16(30, (N, r), std=0.02), "x": gaussian_bf16(1, (M, K)),
+            "dy": gaussian_bf16(50, (M, N))}
 
 # NVFP4 GEMM sweep: (N, K) x M
 SWEEP_NK = [(2048, 2048), (512, 2048), (8192, 2048), (2048, 8192), (8960, 1536), (8192, 3072)]

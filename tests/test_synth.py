@@ -32,3 +32,18 @@ def test_bf16_tensors_are_rounded_values_of_the_stream():
     ref = 2.0 * synth.normal(4, 128).reshape(8, 16)
     assert np.all(np.abs(v - ref) <= 2.0 ** -8 * np.abs(ref))       # one BF16 rounding
     assert np.array_equal(synth.f64_to_bf16_bits(v), g)               # BF16 values round-trip
+
+
+def test_stream_offsets_continue_the_stream():
+    """A stream started at an (even) offset is the same stream's continuation, so
+    tensors generated in chunks equal tensors generated at once."""
+    full = synth.normal(5, 1000)
+    assert np.array_equal(synth.normal(5, 300, offset=700), full[700:])
+    assert np.array_equal(synth.uniform(5, 10, offset=20), synth.uniform(5, 30)[20:])
+    old = synth._CHUNK
+    try:
+        synth._CHUNK = 64                       # force many chunks, one of them ragged
+        chunked = synth.gaussian_bf16(6, (9, 50), std=0.5, mean=1.0)
+    finally:
+        synth._CHUNK = old
+    assert np.array_equal(chunked, synth.f64_to_bf16_bits(1.0 + 0.5 * synth.normal(6, 450)).reshape(9, 50))
