@@ -5,14 +5,16 @@ A step is the forward and backward pass of the NVFP4 data flow through a decoder
 layer's seven frozen projections (fused RMSNorm / SiLU-multiply quantizers, NVFP4
 GEMMs with the fused BF16 LoRA branch, NVFP4 dgrad GEMMs on the cached transposed
 weight layouts, LoRA weight gradients, the backward elementwise kernels), all in
-libpact.  Inputs are seeded synthetic tensors shaped like a Llama-3.2-1B layer
-(H 2048, I 8192, k/v 512, batch 4 x seq 512 tokens), LoRA r 16, alpha 32.
+libpact.  Inputs are seeded synthetic tensors shaped like a Llama-3.2-3B layer
+(H 3072, I 8192, k/v 1024, batch 4 x seq 2048 = 8192 tokens, weights with 1% outliers
+x20), LoRA r 16, alpha 32; --workload picks the Llama-3.2-1B or Qwen2.5-1.5B layer, or
+`single` (one 512 x 512 projection with LoRA on X[256 x 512]).
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl pact|reference]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl pact|reference] [--workload W]
 
 prints one JSON line.  --impl reference times the CPU oracle (the plain FP64
 reference implementation) on the host cores on a bounded token sample of the
-same workload.  Multi-GPU runs (torchrun) are data-parallel replicas: each rank
+same workload, for exactly --steps steps.  Multi-GPU runs (torchrun) are data-parallel replicas: each rank
 runs its own layer step on its own tokens and the LoRA gradients are all-reduced
 over NCCL.
 """
@@ -34,7 +36,7 @@ if ROOT not in sys.path:
 import numpy as np  # noqa: E402
 
 METRIC = "NVFP4 frozen-proj fwd+dgrad TFLOPS & layer tokens/s; % of FP4 tensor peak"
-WORKLOAD = "llama-3.2-1b"
+WORKLOAD = "llama-3.2-3b"
 # nominal dense FP4 / BF16 tensor throughput ratio on B200 (9 / 2.25 PFLOP/s)
 FP4_PER_BF16 = 4.0
 
@@ -45,8 +47,8 @@ def parse():
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=("pact", "reference"), default="pact")
-    ap.add_argument("--workload", default=WORKLOAD)
-    ap.add_argument("--cpu-tokens", type=int, default=128, help="token sample of the CPU oracle baseline")
+    ap.add_argument("--workload", default=WORKLOAD, choices=("llama-3.2-3b", "llama-3.2-1b", "qwen2.5-1.5b", "single"))
+    ap.add_argument("--cpu-tokens", type=int, default=64, help="token sample of the CPU oracle baseline")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--sweep", action="store_true",
                     help="NVFP4 GEMM shape sweep (N x K x M, forward and dgrad): one JSON line per shape")
@@ -55,6 +57,10 @@ def parse():
     ap.add_argument("--ops", action="store_true",
                     help="time each op of the layer step alone: one JSON line per op with its roofline")
     ap.add_argument("--only", default=None, help="with --ops: time only the ops whose name contains this")
+    ap.add_argument("--gptq", action="store_true",
+                    help="time the NVFP4-adapted GPTQ calibration of each weight group of the layer (one JSON line "
+                         "per group)")
+    ap.add_argument("--calib-tokens", type=int, default=512, help="calibration tokens for --gptq")
     ap.add_argument("--two-level", action="store_true",
                     help="cache the frozen weights in the two-level variant (a power of two per tensor)")
     return ap.parse_args()
@@ -129,9 +135,11 @@ class ClockSampler:
 class Replicas:
     """The host side of a multi-GPU run: one process per GPU (torchrun's RANK,
     WORLD_SIZE, LOCAL_RANK), each a full replica of the layer step on its own
-    tokens.  The only exchange is the sum of the LoRA weight gradients; timings are
-    reduced to their maximum over ranks; rank 0 alone prints.  `backend` is "nccl"
-    on GPUs ("gloo" runs the same logic on CPU tensors)."""
+    tokens.  The only exchange is the sum of the LoRA weight gradients: each rank's
+    backward writes them unrounded in FP32 into one flat buffer, one all-reduce sums
+    the buffer, and the sum is rounded to BF16 once.  Timings are reduced to their
+    maximum over ranks; rank 0 alone prints.  `backend` is "nccl" on GPUs ("gloo"
+    runs the same logic on CPU tensors)."""
 
     def __init__(self, backend: str = "nccl", device=None, timeout_s: float = 120.0):
         import datetime
@@ -144,11 +152,14 @@ class Replicas:
             kw = {"device_id": device} if backend == "nccl" and device is not None else {}
             dist.init_process_group(backend, timeout=datetime.timedelta(seconds=timeout_s), **kw)
 
-    def allreduce_grads(self, grads):
-        """Sum each gradient tensor over the ranks, in place (same order on every rank)."""
+    def allreduce_bucket(self, bucket):
+        """Sum one flat FP32 gradient buffer over the ranks, in place, in one collective
+        (every rank calls it at the same point of every step)."""
+        import torch
+        if bucket.dtype != torch.float32 or not bucket.is_contiguous() or bucket.dim() != 1:
+            raise TypeError("the gradient bucket is one flat contiguous float32 tensor")
         if self.world > 1:
-            for g in grads:
-                self.dist.all_reduce(g)
+            self.dist.all_reduce(bucket)
 
     def max_over_ranks(self, value: float) -> float:
         if self.world == 1:
@@ -173,24 +184,27 @@ class Replicas:
 
 
 # ------------------------------------------------------------------ CPU oracle
-# DRAM bytes (read + write) per k_nvfp4_gemm launch, mean over the 8 GEMMs of the
-# Llama-3.2-1B layer step, from one ncu capture of the step's first eager pass (cold
-# L2).  Valid only for the GEMM source it was taken on: reported as null once
-# csrc/gemm.cu or csrc/common.cuh differ from these hashes.
-GEMM_TRAFFIC = {"workload": "llama-3.2-1b", "bytes_per_launch": 17724416,
-                "sha256_16": {"gemm.cu": "fe1bc968079a405c", "common.cuh": "774f32b5d22d6330"}}
+# DRAM bytes (read + write) per k_nvfp4_gemm launch, mean over the GEMMs of one layer
+# step, from one ncu capture of the step's first eager pass (cold L2), per workload.
+# Valid only for the GEMM source it was taken on: reported as null once csrc/gemm.cu
+# or csrc/common.cuh differ from the recorded hashes.
+GEMM_TRAFFIC = {
+    "llama-3.2-1b": {"bytes_per_launch": 17724416,
+                     "sha256_16": {"gemm.cu": "fe1bc968079a405c", "common.cuh": "774f32b5d22d6330"}},
+}
 
 
 def gemm_traffic(workload):
     import hashlib
-    if workload != GEMM_TRAFFIC["workload"]:
+    rec = GEMM_TRAFFIC.get(workload)
+    if rec is None:
         return None
     csrc = os.path.join(os.path.dirname(os.path.abspath(__file__)), "nvfp4_gemm_b200", "csrc")
-    for name, h in GEMM_TRAFFIC["sha256_16"].items():
+    for name, h in rec["sha256_16"].items():
         with open(os.path.join(csrc, name), "rb") as f:
             if hashlib.sha256(f.read()).hexdigest()[:16] != h:
                 return None
-    return GEMM_TRAFFIC["bytes_per_launch"]
+    return rec["bytes_per_launch"]
 
 
 def gpu_local_cpus(dev):
@@ -222,30 +236,87 @@ def bf16_lora_saved_bytes(M, H, I, r):
     return 2 * 2 * M * H + 2 * 4 * M + 3 * 2 * M * H + 2 * M * I + 2 * 2 * M * I + 7 * 2 * M * r
 
 
+def bf16_lora_saved_bytes_measured(name, dev, M=None):
+    """Bytes PyTorch autograd actually keeps for the backward of a plain BF16 LoRA
+    decoder layer of the same scope as the PACT layer (RMSNorm, the seven projections
+    with frozen BF16 weights and trainable BF16 adapters, SiLU-multiply, both
+    residuals; the attention core excluded, its output a given BF16 tensor), counted
+    with saved-tensor hooks during the forward: every saved activation storage once,
+    the weights and adapters (parameters, not activations) excluded.  A comparison
+    model in PyTorch ops, not part of the PACT path."""
+    import torch
+    import torch.nn.functional as F
+    import synth
+    c = synth.LAYERS[name]
+    M = M or synth.tokens(name)
+    H, I, r = c["H"], c["I"], synth.LORA_R
+    s = synth.LORA_ALPHA / r
+    gen = torch.Generator(device=dev).manual_seed(0)
+    rnd = lambda *sh, std=1.0: (torch.randn(sh, device=dev, generator=gen) * std).to(torch.bfloat16)
+    shapes = synth.layer_shapes(name)
+    W = {p: rnd(*shapes[p], std=0.02) for p in synth.PROJ}
+    A = {p: rnd(r, shapes[p][1], std=0.02).requires_grad_() for p in synth.PROJ}
+    B = {p: rnd(shapes[p][0], r, std=0.02).requires_grad_() for p in synth.PROJ}
+    g1, g2 = (1 + rnd(H, std=0.02)), (1 + rnd(H, std=0.02))
+    params = {t.untyped_storage().data_ptr() for d in (W, A, B) for t in d.values()} | {
+        g1.untyped_storage().data_ptr(), g2.untyped_storage().data_ptr()}
+    seen = {}
+
+    def pack(t):
+        st = t.untyped_storage()
+        if st.data_ptr() not in params:
+            seen[st.data_ptr()] = st.nbytes()
+        return t
+
+    h, attn = rnd(M, H).requires_grad_(), rnd(M, H).requires_grad_()
+    lin = lambda x, p: F.linear(x, W[p]) + s * F.linear(F.linear(x, A[p]), B[p])
+    with torch.autograd.graph.saved_tensors_hooks(pack, lambda t: t):
+        x1 = F.rms_norm(h, (H,), g1, synth.RMS_EPS)
+        q, k, v = lin(x1, "q"), lin(x1, "k"), lin(x1, "v")
+        h2 = h + lin(attn, "o")
+        x2 = F.rms_norm(h2, (H,), g2, synth.RMS_EPS)
+        m = F.silu(lin(x2, "gate")) * lin(x2, "up")
+        out = h2 + lin(m, "down")
+    del q, k, v, out
+    return int(sum(seen.values()))
+
+
 def oracle_layer(name, inputs, two_level=False):
     import oracle
-    from oracle.layer import OracleLayer
+    from oracle.layer import OracleLayer, OracleProjection
     import synth
     oracle.build()
+    if name == "single":
+        return OracleProjection(inputs["w"], inputs["lora_a"], inputs["lora_b"], synth.LORA_R, synth.LORA_ALPHA)
     c = synth.LAYERS[name]
     return OracleLayer(c["H"], c["I"], c["KV"], synth.LORA_R, synth.LORA_ALPHA, synth.RMS_EPS, inputs["w"],
                        inputs["lora_a"], inputs["lora_b"], inputs["gamma1"], inputs["gamma2"], two_level=two_level)
 
 
-def oracle_rate(layer, inputs, tokens, min_seconds=10.0, max_steps=20):
-    """Tokens/s of the oracle's layer step on the first `tokens` tokens."""
+def oracle_rate(layer, inputs, tokens, min_seconds=10.0, max_steps=20, exact_steps=None):
+    """Tokens/s of the oracle's step on the first `tokens` tokens: steps until
+    `min_seconds` have passed or `max_steps` ran, or exactly `exact_steps` steps."""
     import oracle
     sl = slice(0, tokens)
-    args = (inputs["h"][sl], inputs["attn"][sl], inputs["d_out"][sl], inputs["d_qkv"][sl])
+    args = tuple(inputs[k][sl] for k in layer.input_keys)
     t0 = time.perf_counter()
     n = 0
     while True:
         layer.step(*args)
         n += 1
         el = time.perf_counter() - t0
-        if el >= min_seconds or n >= max_steps:
+        if exact_steps is not None:
+            if n >= exact_steps:
+                break
+        elif el >= min_seconds or n >= max_steps:
             break
     return n * tokens / el, n, el, oracle.num_threads()
+
+
+def cpu_sample_tokens(a, M):
+    """Tokens per oracle step: the whole single-projection workload (256 tokens, well
+    under a second), else a sample of --cpu-tokens of the layer's tokens."""
+    return M if a.workload == "single" else max(8, min(a.cpu_tokens, M))
 
 
 def reference_arm(a):
@@ -254,15 +325,15 @@ def reference_arm(a):
     if rank != 0:
         return
     import synth
-    M = synth.tokens(a.workload)
-    inputs = synth.layer_inputs(a.workload)
+    M = workload_tokens(a.workload)
+    inputs = workload_inputs(a.workload)
     layer = oracle_layer(a.workload, inputs, a.two_level)
-    for _ in range(max(0, min(a.warmup, 1))):
-        layer.step(inputs["h"][:8], inputs["attn"][:8], inputs["d_out"][:8], inputs["d_qkv"][:8])
-    tok = max(8, min(a.cpu_tokens, M))
-    rate, n, el, cores = oracle_rate(layer, inputs, tok, min_seconds=0.0, max_steps=max(1, a.steps))
-    sample = (f"{tok} of {M} tokens per step ({n} steps), one layer fwd+bwd; weight layouts "
-              f"cached before timing")
+    for _ in range(a.warmup):      # small untimed passes
+        layer.step(*(inputs[k][:8] for k in layer.input_keys))
+    tok = cpu_sample_tokens(a, M)
+    rate, n, el, cores = oracle_rate(layer, inputs, tok, exact_steps=max(1, a.steps))
+    sample = (f"{tok} of {M} tokens per step ({n} steps, {el:.1f} s), one "
+              f"{'projection' if a.workload == 'single' else 'layer'} fwd+bwd; weight layouts cached before timing")
     print(json.dumps({
         "impl": "reference", "metric": METRIC, "value": rate, "unit": "tokens/s", "n_gpus": a.gpus,
         "steps": n, "warmup": a.warmup, "ms_per_step": 1000.0 * el / n, "higher_is_better": True,
@@ -273,8 +344,24 @@ def reference_arm(a):
     }), flush=True)
 
 
+def workload_tokens(name):
+    import synth
+    return synth.SINGLE["M"] if name == "single" else synth.tokens(name)
+
+
+def workload_inputs(name):
+    import synth
+    return synth.single_inputs() if name == "single" else synth.layer_inputs(name)
+
+
 def config_block(name, M):
     import synth
+    if name == "single":
+        c = synth.SINGLE
+        return {"workload": "single frozen projection + LoRA fwd+bwd (X[256x512], W[512x512], r 16, alpha 32)",
+                "M": c["M"], "N": c["N"], "K": c["K"], "tokens": M, "lora_r": synth.LORA_R,
+                "lora_alpha": synth.LORA_ALPHA, "l2": "flushed between timed steps (256 MiB write)",
+                "launch": "one CUDA graph per step (LoRA weight gradients on a parallel branch)"}
     c = synth.LAYERS[name]
     return {"workload": f"{name} decoder layer fwd+bwd: 7 NVFP4 frozen projections + LoRA",
             "H": c["H"], "I": c["I"], "kv": c["KV"], "tokens": M, "batch": c["batch"], "seq": c["seq"],
@@ -283,23 +370,31 @@ def config_block(name, M):
 
 
 # ------------------------------------------------------------------ GPU arm
-def make_layer(name, dev, two_level=False):
-    """The layer of workload `name` on device `dev` with its seeded synthetic inputs bound."""
+def make_layer(name, dev, two_level=False, grad_fp32=False):
+    """The layer (or the single projection) of workload `name` on device `dev` with its
+    seeded synthetic inputs bound."""
     import torch
     import synth
-    from nvfp4_gemm_b200.layer import LayerShape, PactLayer
+    from nvfp4_gemm_b200.layer import LayerShape, PactLayer, PactProjection
+    d = lambda bits: torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).to(dev)
+    if name == "single":
+        inputs = synth.single_inputs()
+        layer = PactProjection(d(inputs["w"]), d(inputs["lora_a"]), d(inputs["lora_b"]), synth.SINGLE["M"],
+                               synth.LORA_R, synth.LORA_ALPHA)
+        x_in = {k: d(inputs[k]) for k in layer.input_keys}
+        layer.bind(*(x_in[k] for k in layer.input_keys))
+        return inputs, layer, x_in
     c = synth.LAYERS[name]
     M = synth.tokens(name)
     inputs = synth.layer_inputs(name)
-    d = lambda bits: torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).to(dev)
     shape = LayerShape(M=M, H=c["H"], I=c["I"], KV=c["KV"], r=synth.LORA_R, alpha=synth.LORA_ALPHA,
                        eps=synth.RMS_EPS)
     layer = PactLayer(shape, {k: d(v) for k, v in inputs["w"].items()},
                       {k: d(v) for k, v in inputs["lora_a"].items()},
                       {k: d(v) for k, v in inputs["lora_b"].items()}, d(inputs["gamma1"]), d(inputs["gamma2"]),
-                      two_level=two_level)
-    x_in = {k: d(inputs[k]) for k in ("h", "attn", "d_out", "d_qkv")}
-    layer.bind(x_in["h"], x_in["attn"], x_in["d_out"], x_in["d_qkv"])
+                      two_level=two_level, grad_fp32=grad_fp32)
+    x_in = {k: d(inputs[k]) for k in layer.input_keys}
+    layer.bind(*(x_in[k] for k in layer.input_keys))
     return inputs, layer, x_in
 
 
@@ -395,10 +490,84 @@ def gemm_sweep(a, shapes):
         torch.cuda.empty_cache()
 
 
+def saved_block(name, layer, dev, M):
+    """Activation bytes held from forward to backward: the PACT path's, against what
+    autograd keeps for a plain BF16 LoRA layer of the same scope (measured with
+    saved-tensor hooks) and the hand count of the same tensors."""
+    if name == "single":
+        return {"pact": layer.saved_bytes(), "note": "the NVFP4 copy of X"}
+    import torch
+    out = {"pact": layer.saved_bytes(),
+           "bf16_lora_autograd": bf16_lora_saved_bytes_measured(name, dev, M),
+           "bf16_lora_model": bf16_lora_saved_bytes(M, layer.s.H, layer.s.I, layer.s.r),
+           "note": "bytes held from forward to backward per layer (PACT: the NVFP4 copies, rstd, attn) against "
+                   "PyTorch autograd's saved tensors for a BF16 LoRA layer of the same scope (measured) and a hand "
+                   "count of the tensors that layer needs"}
+    torch.cuda.empty_cache()
+    return out
+
+
+def gptq_bench(a):
+    """NVFP4-adapted GPTQ calibration of the workload's four weight groups (q|k|v, o,
+    gate|up, down) on seeded synthetic calibration activations ~N(0, 1): device time
+    per group (CUDA events on the launching stream), the FP64 work it implies, and
+    the oracle on a sample of rows (GPTQ's rows are independent once H is fixed),
+    scaled to the group."""
+    import torch
+    import synth
+    import nvfp4_gemm_b200 as P
+    from oracle import gptq as ogptq
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    c = synth.LAYERS[a.workload]
+    shp = synth.layer_shapes(a.workload)
+    d = lambda bits: torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).to(dev)
+    stream = torch.cuda.Stream(device=dev)
+    for key, group in (("qkv", ("q", "k", "v")), ("o", ("o",)), ("gu", ("gate", "up")), ("d", ("down",))):
+        w = np.concatenate([synth.weight_bf16(synth.PROJ.index(p), shp[p], outliers=c["outliers"]) for p in group], 0)
+        N, K = w.shape
+        x = synth.gaussian_bf16(91, (a.calib_tokens, K))
+        wd, xd = d(w), d(x)
+        out = P.NVFP4Tensor.empty(N, K, dev)
+        need = P.pact_gptq_workspace_bytes(N, K, a.calib_tokens)
+        raw = torch.empty(need + 256, dtype=torch.uint8, device=dev)
+        off = (-raw.data_ptr()) % 256
+        ws = raw[off:off + need]
+        with torch.cuda.stream(stream):
+            P.pact_gptq_nvfp4(wd, xd, 0.01, out=out, workspace=ws, stream=stream)   # warm-up
+            torch.cuda.synchronize()
+            times = []
+            for _ in range(max(1, a.steps)):
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record(stream)
+                P.pact_gptq_nvfp4(wd, xd, 0.01, out=out, workspace=ws, stream=stream)
+                e1.record(stream)
+                torch.cuda.synchronize()
+                times.append(e0.elapsed_time(e1))
+        if P.pact_get_device_status() != 0:
+            raise RuntimeError(P.pact_last_error())
+        ms = statistics.median(times)
+        n = a.calib_tokens
+        flop = 2.0 * n * K * K + 2.0 * K ** 3 / 3.0 + 1.0 * N * K * K
+        rows = 8
+        t0 = time.perf_counter()
+        ogptq.gptq_nvfp4(w[:rows], x)
+        cpu_s = time.perf_counter() - t0
+        print(json.dumps({"gptq": {"workload": a.workload, "group": key, "N": N, "K": K, "calib_tokens": n},
+                          "ms": ms, "fp64_flop": flop, "fp64_tflops": flop / (ms / 1e3) / 1e12,
+                          "oracle_s_for_8_rows": cpu_s,
+                          "note": "FP64 work: H (2 n K^2), the factorisation and triangular inverse (2 K^3 / 3), "
+                                  "the column pass (N K^2 / 2 multiply-subtract pairs)"}), flush=True)
+        del wd, xd, out, raw, ws
+        torch.cuda.empty_cache()
+
+
 def main():
     a = parse()
     if a.impl == "reference":
         return reference_arm(a)
+    if a.gptq:
+        return gptq_bench(a)
     if a.gemm:
         return gemm_sweep(a, [tuple(a.gemm)])
     if a.sweep:
@@ -416,8 +585,8 @@ def main():
     rep = Replicas("nccl", dev)
     world, rank = rep.world, rep.rank
 
-    M = synth.tokens(a.workload)
-    inputs, layer, x_in = make_layer(a.workload, dev, a.two_level)
+    M = workload_tokens(a.workload)
+    inputs, layer, x_in = make_layer(a.workload, dev, a.two_level, grad_fp32=world > 1)
     if a.ops:
         return op_table(a, layer, dev)
     ops = layer.step_ops()
@@ -458,7 +627,10 @@ def main():
     grads = list(layer.grads.values())
 
     def allreduce_grads():
-        rep.allreduce_grads(grads)
+        """Replicas: sum the FP32 gradient buffer over the ranks, then round it once."""
+        if world > 1:
+            rep.allreduce_bucket(layer.grad_bucket)
+            layer.round_grads()
 
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
     with torch.cuda.stream(stream):
@@ -517,7 +689,7 @@ def main():
     # PCIe rate); the copy of step k+1 runs on a copy stream while step k computes
     # (two device input sets, one captured step graph each).  The timed region spans
     # all K steps, from the first copy to the last gradient read-back.
-    keys = ("h", "attn", "d_out", "d_qkv")
+    keys = layer.input_keys
     sizes = [x_in[k].numel() for k in keys]          # multiples of 8: every view is 16-byte aligned
     # pinned buffers on the GPU's NUMA node: allocated and first touched by this thread
     # while it runs on the GPU's local CPUs (the previous CPU set comes back after)
@@ -545,12 +717,12 @@ def main():
     graphs = []
     for flat in dev_flat:
         sv = views(flat)
-        layer.bind(sv["h"], sv["attn"], sv["d_out"], sv["d_qkv"])
+        layer.bind(*(sv[k] for k in keys))
         g = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g, stream=stream):
             layer.step_concurrent(side)
         graphs.append(g)
-    layer.bind(x_in["h"], x_in["attn"], x_in["d_out"], x_in["d_qkv"])
+    layer.bind(*(x_in[k] for k in keys))
     copier = torch.cuda.Stream(device=dev)
     loaded = [torch.cuda.Event() for _ in range(K)]
     consumed = [torch.cuda.Event() for _ in range(K)]
@@ -582,10 +754,12 @@ def main():
     cpu = None
     if rank == 0 and world == 1 and not a.no_cpu_baseline:
         ol = oracle_layer(a.workload, inputs, a.two_level)
-        rate, n, el, cores = oracle_rate(ol, inputs, min(a.cpu_tokens, M))
+        tok = cpu_sample_tokens(a, M)
+        rate, n, el, cores = oracle_rate(ol, inputs, tok)
         cpu = {"value": rate, "unit": "tokens/s", "cores": cores, "kind": "oracle",
-               "sample": f"{min(a.cpu_tokens, M)} of {M} tokens per step ({n} steps, {el:.1f} s), one layer "
-                         f"fwd+bwd on the FP64 CPU oracle; weight layouts cached before timing"}
+               "sample": f"{tok} of {M} tokens per step ({n} steps, {el:.1f} s), one "
+                         f"{'projection' if a.workload == 'single' else 'layer'} fwd+bwd on the FP64 CPU oracle; "
+                         f"weight layouts cached before timing"}
 
     out = {
         "metric": METRIC, "value": tokens_per_s, "unit": "tokens/s", "n_gpus": world, "steps": K,
@@ -610,12 +784,8 @@ def main():
                         "current step; LoRA gradients read back every step",
                 "host_buffers": (f"pinned on the GPU's NUMA node ({len(local_cpus)} local CPUs)" if local_cpus
                                  else "pinned; the GPU's NUMA node unknown")},
-        "saved_activation_bytes": {
-            "pact": layer.saved_bytes(), "bf16_lora_model": bf16_lora_saved_bytes(M, layer.s.H, layer.s.I, layer.s.r),
-            "note": "bytes held from forward to backward per layer (the NVFP4 copies, rstd, attn) against an "
-                    "autograd count for a BF16 LoRA layer of the same scope"},
-        "weight_bytes": {"pact_cached_layouts": layer.weight_cache_bytes(),
-                         "bf16": 2 * int(layer.s.frozen_flops() / (4.0 * M))},
+        "saved_activation_bytes": saved_block(a.workload, layer, dev, M),
+        "weight_bytes": {"pact_cached_layouts": layer.weight_cache_bytes(), "bf16": layer.bf16_weight_bytes()},
         "gpu_launches": launches_per_step * K,
         "clocks": clk.summary(),
         "segments_ms": {"+".join(op.name for op in sg["ops"]): round(t, 4) for sg, t in zip(segs, seg_ms)},

@@ -59,7 +59,7 @@
 extern "C" {
 #endif
 
-#define PACT_ABI_VERSION 2
+#define PACT_ABI_VERSION 3
 
 #if defined(__GNUC__)
 #define PACT_API __attribute__((visibility("default")))
@@ -225,7 +225,9 @@ PACT_API pact_status pact_frozen_gemm_dgrad(const pact_nvfp4_t *dyq, const pact_
 /* [LORA]: T = scale * X . A^T for X [M x K] (row stride ldx) and A [R x K] (row
  * stride K; R = nseg*r stacked adapters sharing X), FP32-accumulated and written
  * as hi + lo BF16 halves: T [M x 2R] (row stride ldt >= 2R), hi = BF16_RNE(t) in
- * columns 0..R-1, lo = BF16_RNE(t - hi) in columns R..2R-1.  R is 16, 32, 48 or 64.
+ * columns 0..R-1, lo = BF16_RNE(t - hi) in columns R..2R-1.  R is 16, 32, 48 or 64;
+ * the LoRA term fused into pact_frozen_gemm_fwd takes at most 48 columns (nseg*r <=
+ * 48), so a T with R = 64 serves callers that use it outside that GEMM.
  * workspace (device, 16-byte aligned, >= pact_lora_fwd_workspace_bytes(M, K, R))
  * is caller-owned scratch for FP32 partial sums; its contents on entry do not
  * matter and calls that share it must not overlap on the GPU. */
@@ -243,9 +245,13 @@ PACT_API pact_status pact_lora_fwd(const pact_bf16 *x, int64_t ldx, int64_t M, i
  * that every GPU loading the library holds until the process exits.  Shapes whose
  * scratch (pact_lora_fwd_workspace_bytes) exceeds 8 MiB return PACT_ERR_SHAPE.
  * The first call on a device looks up the array's device address (a CUDA runtime
- * query, once per device); make that first call before any stream capture.  All
- * calls on a device share the array, so calls that overlap on the GPU (different
- * streams) race.  It allocates nothing. */
+ * query, once per device, under a lock, so first calls from several host threads
+ * are safe); make that first call before any stream capture.  The address is kept
+ * for the life of the process: after cudaDeviceReset on a device this call must not
+ * be used there again.  All calls on a device share the array, so calls that
+ * overlap on the GPU (different streams) race.  A call whose kernel gave up a
+ * bounded wait leaves NaN in T (never a previous call's values); as after every
+ * call, pact_get_device_status reports it.  It allocates nothing. */
 PACT_API pact_status pact_lora_fwd_noalloc(const pact_bf16 *x, int64_t ldx, int64_t M, int64_t K,
                                            const pact_bf16 *A, int R, float scale, pact_bf16 *T,
                                            int64_t ldt, pact_stream_t stream);
@@ -280,17 +286,55 @@ typedef struct {
     int64_t seg_end[4];
     float scale;
     int u_gexp;               /* U holds 2^-u_gexp times the gradient factor (0 usually) */
-    pact_bf16 *dA;            /* out [nseg*r x K]:  2^u_gexp (U_hi + U_lo)^T . X~ */
-    pact_bf16 *dB;            /* out [N x r]: rows seg_i = scale * dY[:, seg_i]^T . (X~ . A_i^T) */
+    void *dA;                 /* out [nseg*r x K]:  2^u_gexp (U_hi + U_lo)^T . X~ */
+    void *dB;                 /* out [N x r]: rows seg_i = scale * dY[:, seg_i]^T . (X~ . A_i^T) */
+    int grads_fp32;           /* 0: dA, dB are BF16 (pact_bf16 *); 1: FP32 (float *), unrounded,
+                                 e.g. to be summed over data-parallel replicas before one
+                                 rounding (pact_round_bf16) */
 } pact_lora_bwd_t;
 
-/* Scratch bytes pact_lora_bwd needs (X~ as BF16, T~ = X~ A^T, FP32 partial sums). */
+/* Scratch bytes pact_lora_bwd needs (T~ = X~ A^T and FP32 partial sums; an NVFP4
+ * X~ is decoded inside the MMA kernel, no BF16 copy of it is made). */
 PACT_API size_t pact_lora_bwd_workspace_bytes(int64_t M, int64_t N, int64_t K, int r, int nseg);
 /* dA and dB of the adapters; workspace (device, 256-byte aligned, >=
  * pact_lora_bwd_workspace_bytes) is scratch owned by the caller; its contents on
  * entry do not matter and calls that share it must not overlap on the GPU. */
 PACT_API pact_status pact_lora_bwd(const pact_lora_bwd_t *args, void *workspace, size_t ws_bytes,
                           pact_stream_t stream);
+
+/* -------------------------------------- N1: NVFP4-adapted GPTQ calibration */
+/* [METHOD] bullet 3 and the abstract: the frozen weights are calibrated offline with
+ * GPTQ adapted to NVFP4, the statistics taken from the reconstructed NVFP4 inputs.
+ * For W [N x K] (BF16, row stride ldw) and calibration inputs X [n x K] (BF16, row
+ * stride ldx), with X~ = deq(q(X)) and H = 2 X~^T X~ / n:
+ *   a column of H with H[i, i] = 0 gets H[i, i] = 1 and zero weights;
+ *   H += damp * mean(diag H) * I;  U = the upper Cholesky factor of H^-1;
+ *   for j = 0 .. K-1: at a 16-column block start, the block's scale byte is
+ *   E4M3_RNE_sat(max |w| / 6) of its current weights; code_j = RNE onto the E2M1
+ *   grid of w_j / scale (sign kept); err = (w_j - q_j) / U[j, j];
+ *   W[:, j+1:] -= err U[j, j+1:].
+ * All of it in FP64 (GPTQ: Frantar et al., 2022).  The codes and scales go to `out`
+ * (NVFP4 [N x K], the forward weight layout); pact_weight_layout_cache_from_nvfp4
+ * turns it into a weight cache.  N <= 2^20, K a multiple of 64 up to 32768, n <= 2^24.
+ * workspace: device, 256-byte aligned, >= pact_gptq_workspace_bytes(N, K, n) bytes
+ * (about 8 (n K + 4 K^2 + N K) bytes).  pivot_error (device int, may be NULL) gets 1
+ * if the damped H was not positive definite (the result is then meaningless), else 0. */
+PACT_API size_t pact_gptq_workspace_bytes(int64_t N, int64_t K, int64_t n);
+PACT_API pact_status pact_gptq_nvfp4(const pact_bf16 *W, int64_t ldw, int64_t N, int64_t K,
+                                     const pact_bf16 *X, int64_t ldx, int64_t n, double damp,
+                                     void *workspace, size_t ws_bytes, const pact_nvfp4_t *out,
+                                     int *pivot_error, pact_stream_t stream);
+/* A1 from a given forward layout (e.g. a calibrated one): copies wf [N x K] into the
+ * cache's forward part and builds the backward part q(deq(wf)^T); gexp as for
+ * pact_weight_layout_cache_scaled (0 for one-level layouts).  buf as for
+ * pact_weight_layout_cache. */
+PACT_API pact_status pact_weight_layout_cache_from_nvfp4(const pact_nvfp4_t *wf, int gexp, void *buf,
+                                                         size_t bytes, pact_weight_cache_t *out,
+                                                         pact_stream_t stream);
+
+/* y[i] = BF16_RNE(x[i]) for n FP32 values (device, 16-byte aligned): the one rounding of
+ * gradients kept in FP32 (pact_lora_bwd with grads_fp32) after they were summed. */
+PACT_API pact_status pact_round_bf16(const float *x, pact_bf16 *y, int64_t n, pact_stream_t stream);
 
 /* ------------------------------------- A9: SiLU-multiply backward + quantize */
 /* [METHOD] bullet 2 (backward reads the NVFP4 gate/up copies).  With
@@ -327,6 +371,16 @@ PACT_API const char *pact_status_string(pact_status s);
 PACT_API pact_status pact_get_device_status(pact_stream_t stream);
 /* PACT_ABI_VERSION of the loaded library. */
 PACT_API int pact_abi_version(void);
+/* Self-test of the failure path (the pages have no counterpart; it tests the
+ * library's bounded waits): one kernel thread waits on an mbarrier that nothing
+ * completes, through the same bounded wait every libpact kernel uses, with a limit
+ * of limit_cycles SM clock cycles (1e3 .. 4e9).  The wait runs out, the kernel
+ * records PACT_ERR_TIMEOUT in the device status word (read and cleared by
+ * pact_get_device_status) and returns; nothing asynchronous is left in flight and
+ * the context stays usable.  waited_cycles (device, 8-byte aligned, may be NULL)
+ * receives the cycles the wait took. */
+PACT_API pact_status pact_selftest_wait_timeout(int64_t limit_cycles, unsigned long long *waited_cycles,
+                                                pact_stream_t stream);
 
 #ifdef __cplusplus
 }

@@ -61,9 +61,33 @@ pact_status check_nvfp4(const pact_nvfp4_t *t, int64_t rows, int64_t cols, const
     return PACT_OK;
 }
 
+// Self-test of the failure path: one thread waits, with the given limit, on an
+// mbarrier that nothing arrives on, through the same bounded wait every kernel uses.
+// The wait runs out, records the timeout in the status word and the kernel returns;
+// nothing asynchronous (no copy, no tensor-core operation) is outstanding.
+__global__ void k_wait_selftest(long long limit_cycles, unsigned long long *waited_cycles) {
+    __shared__ uint64_t bar;
+    pdl_wait();
+    if (threadIdx.x != 0) return;
+    mbar_init(&bar, 1);
+    fence_barrier_init();
+    const long long t0 = clock64();
+    const bool ok = mbar_wait(&bar, 0, limit_cycles);
+    if (waited_cycles) *waited_cycles = ok ? 0ull : (unsigned long long)(clock64() - t0);
+}
+
 }  // namespace pact
 
 extern "C" {
+
+pact_status pact_selftest_wait_timeout(int64_t limit_cycles, unsigned long long *waited_cycles,
+                                       pact_stream_t stream) {
+    PACT_CHECK(limit_cycles >= 1000 && limit_cycles <= 4000000000ll, PACT_ERR_INVALID_ARG,
+               "pact_selftest_wait_timeout: limit must be in [1e3, 4e9] cycles (got %lld)", (long long)limit_cycles);
+    PACT_CHECK(((uintptr_t)waited_cycles & 7) == 0, PACT_ERR_ALIGN, "pact_selftest_wait_timeout: waited_cycles 8-byte aligned");
+    return pact::launch_dep(pact::k_wait_selftest, dim3(1), dim3(32), 0, (cudaStream_t)stream,
+                            "pact_selftest_wait_timeout", (long long)limit_cycles, waited_cycles);
+}
 
 const char *pact_last_error(void) { return pact::t_error; }
 

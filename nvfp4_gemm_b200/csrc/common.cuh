@@ -105,13 +105,13 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
 // false (and records a timeout) after about WAIT_LIMIT_CYCLES SM clock cycles
 // (the cycle counter is cheap to read, unlike the global timer).
 constexpr long long WAIT_LIMIT_CYCLES = 8000000000ll;  // ~4 s at 2 GHz
-__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity) {
+__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, long long limit = WAIT_LIMIT_CYCLES) {
     if (mbar_try_wait(bar, parity)) return true;
     const long long t0 = clock64();
     while (true) {
         for (int i = 0; i < 256; ++i)
             if (mbar_try_wait(bar, parity)) return true;
-        if (clock64() - t0 > WAIT_LIMIT_CYCLES) {
+        if (clock64() - t0 > limit) {
             record_timeout();
             return false;
         }
@@ -391,6 +391,9 @@ __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, bool a_mn, bool 
     return (1u << 4) | (1u << 7) | (1u << 10) | ((a_mn ? 1u : 0u) << 15) | ((b_mn ? 1u : 0u) << 16) |
            ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
 }
+
+// True in every lane when `ok` is true in every lane of the warp.
+__device__ __forceinline__ bool warp_all(bool ok) { return __all_sync(0xffffffffu, ok); }
 
 // ---- small numeric helpers
 __device__ __forceinline__ float bf16lo(uint32_t v) { return __uint_as_float(v << 16); }

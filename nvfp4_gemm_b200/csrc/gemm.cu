@@ -86,7 +86,22 @@ struct Params {
     int lora_nseg;
     int64_t seg_end[4];
     float out_scale;      // 2^gexp of the weight cache: scales the accumulator (exact)
+    int n_fast;           // tile order: 1 = N tiles fastest (A streamed once), 0 = M tiles fastest
 };
+
+// Pair-tile coordinates of persistent tile index t.  Consecutive indices run at the
+// same time on neighbouring clusters, so the operand whose tile they share stays in
+// L2 while the other one streams: with N fastest each row block of A is read once
+// and shared by the clusters working across N; with M fastest the same holds for B.
+__device__ __forceinline__ void tile_coords(const Params &p, int t, int mpairs, int ntiles, int &mp, int &nt) {
+    if (p.n_fast) {
+        nt = t % ntiles;
+        mp = t / ntiles;
+    } else {
+        mp = t % mpairs;
+        nt = t / mpairs;
+    }
+}
 
 __device__ __forceinline__ int lora_segment(const Params &p, int n0) {
     int s = 0;
@@ -103,8 +118,6 @@ struct Ring {
         if (++stage == STAGES) { stage = 0; phase ^= 1; }
     }
 };
-
-__device__ __forceinline__ bool warp_all(bool ok) { return __all_sync(0xffffffffu, ok); }
 
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
 k_nvfp4_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
@@ -179,7 +192,8 @@ k_nvfp4_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CU
             Ring rg;
             bool ok = true;
             for (int t = cluster; ok && t < total; t += nclusters) {
-                const int mp = t % mpairs, nt = t / mpairs;
+                int mp, nt;
+                tile_coords(p, t, mpairs, ntiles, mp, nt);
                 const int m0 = mp * 2 * BM + (int)rank * BM;     // this CTA's rows
                 const int n0 = nt * BN, nb = n0 + (int)rank * (BN / 2);
                 if (lora) {
@@ -337,7 +351,8 @@ k_nvfp4_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CU
             uint32_t lora_prev = 0;   // bit s: the previous use of stage s was a LoRA stage
             bool ok = true;
             for (int t = cluster; ok && t < total; t += nclusters) {
-                const int mp = t % mpairs, nt = t / mpairs;
+                int mp, nt;
+                tile_coords(p, t, mpairs, ntiles, mp, nt);
                 const int ga = (mp * 2 * BM + (int)rank * BM) / 128, gb = (nt * BN) / 128;
                 for (int i = 0; ok && i < nsteps; ++i) {
                     const uint32_t sb = 1u << rg.stage;
@@ -373,8 +388,16 @@ k_nvfp4_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CU
         uint8_t *slab_p = smem + OFF_SLABS + ew * SLAB_BYTES;
         const uint32_t slab = smem_u32(slab_p);
         // this warp's 32 x 64 block of tile t: first row and column
-        auto block_y = [&](int t) { return (t % mpairs) * 2 * BM + (int)rank * BM + sub * 32; };
-        auto block_x = [&](int t) { return (t / mpairs) * BN + quarter * 64; };
+        auto block_y = [&](int t) {
+            int mp, nt;
+            tile_coords(p, t, mpairs, ntiles, mp, nt);
+            return mp * 2 * BM + (int)rank * BM + sub * 32;
+        };
+        auto block_x = [&](int t) {
+            int mp, nt;
+            tile_coords(p, t, mpairs, ntiles, mp, nt);
+            return nt * BN + quarter * 64;
+        };
         auto inside = [&](int t) { return block_y(t) < p.M && block_x(t) < p.N; };
         auto load_residual = [&](int t) {  // lane 0; the slab is free
             mbar_arrive_expect_tx(&res_full[ew], SLAB_BYTES);
@@ -569,6 +592,8 @@ static pact_status run(const pact_nvfp4_t *a, const pact_nvfp4_t *b, int gexp, c
     p.M = (int)M; p.N = (int)N; p.K = (int)K;
     p.has_res = res != nullptr;
     p.out_scale = std::ldexp(1.0f, gexp);
+    // stream the larger operand once: A (M x K) when M > N, else B (N x K)
+    p.n_fast = M > N ? 1 : 0;
     p.lora_mode = LORA_NONE;
     p.lora_steps = 0; p.lora_r = 0; p.lora_nseg = 1;
     for (int i = 0; i < 4; ++i) p.seg_end[i] = N;

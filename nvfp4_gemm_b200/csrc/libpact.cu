@@ -4,3 +4,4 @@
 #include "quant.cu"
 #include "gemm.cu"
 #include "lora.cu"
+#include "gptq.cu"

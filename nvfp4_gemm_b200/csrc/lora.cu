@@ -15,6 +15,7 @@
 // and a finalize kernel sums the partials in a fixed order (deterministic), scales
 // and rounds.
 #include <cmath>
+#include <mutex>
 
 #include "quant.cuh"
 
@@ -27,8 +28,16 @@ constexpr int STAGES = 4;
 constexpr int THREADS = 192;
 constexpr int A_BYTES = BM * BK * 2;     // 16384
 constexpr int B_BYTES = 64 * BK * 2;     // 8192 per B part
-constexpr int STAGE_BYTES = A_BYTES + 2 * B_BYTES;
-constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + 256;
+// NVFP4 A operand: per stage, the codes of the A tile (128 x 64 values, 4 KiB) and
+// up to two 512-byte scale chunks land in a staging area, and the four epilogue
+// warps decode them into the BF16 operand buffer before the MMA reads it
+constexpr int RAW_CODE_BYTES = BM * BK / 2;                      // 4096
+constexpr int RAW_BYTES = RAW_CODE_BYTES + 1024;
+constexpr int OPER_BYTES = A_BYTES + 2 * B_BYTES;                // 32768
+template <bool A_FP4>
+__host__ __device__ constexpr int stage_bytes() { return OPER_BYTES + (A_FP4 ? RAW_BYTES : 0); }   // multiples of 1024
+template <bool A_FP4>
+__host__ __device__ constexpr int smem_bytes() { return 1024 + STAGES * stage_bytes<A_FP4>() + 256; }
 constexpr uint32_t TMEM_COLS = 64;
 
 // One output block: rows [row_begin, row_end) of the output, contraction
@@ -48,11 +57,78 @@ struct Params {
     int b_lo_off;
     float *ws;          // partials [split][row][ws_ld]
     int64_t ws_ld, ws_split_stride;
+    // NVFP4 A operand (A_FP4): scale bytes of the tensor, its rows and columns
+    // (K-major A: the tensor is [output rows x contraction]; MN-major: [contraction x
+    // output rows])
+    const uint8_t *a_scales;
+    int64_t a_rows, a_cols;
 };
 
-template <bool A_MN, bool B_MN>
+// 8 E2M1 codes (element 0 in the low nibble) times their E4M3 block scale, as 8
+// BF16 values (element 0 in the low half of .x).  Exact: E2M1 pairs convert to
+// FP16 in hardware, the product with the scale has at most 6 significant bits in
+// [2^-10, 2688] (exact in FP16 and in BF16), and FP16 -> FP32 -> BF16 is exact.
+__device__ __forceinline__ uint4 decode8_bf16(uint32_t codes, uint32_t sbyte) {
+    const __half2 s2 = __half2half2(__float2half_rn(e4m3_to_float(sbyte)));
+    uint32_t o[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const uint32_t h = e2m1x2_to_f16x2((codes >> (8 * i)) & 0xFFu);
+        const float2 f = __half22float2(__hmul2(*reinterpret_cast<const __half2 *>(&h), s2));
+        o[i] = pack_bf16x2(f.x, f.y);
+    }
+    return make_uint4(o[0], o[1], o[2], o[3]);
+}
+
+// Decode one stage's NVFP4 A tile from the staging area into the BF16 operand
+// buffer, laid out exactly as the TMA load of the BF16 tile with the 128-byte swizzle
+// would lay it out (row q of 64 values at q * 128 bytes, its 16-byte chunk c at
+// position c ^ (q % 8)).  128 threads, one 64-value row each.
+//  K-major (A_MN = false): operand rows are the tensor's rows row0 .. row0 + 127,
+//    the 64 values are columns k .. k + 63; codes staged as [128 rows x 32 bytes],
+//    one scale chunk (rows of group row0 / 128, blocks k / 16 .. + 3).
+//  MN-major (A_MN = true): operand rows are the tensor's columns row0 .. row0 + 127
+//    (two 64-wide halves), the contraction runs over its rows k .. k + 63; codes
+//    staged as [64 rows x 64 bytes], two scale chunks (one per half).
+template <bool A_MN>
+__device__ __forceinline__ void decode_stage(const uint8_t *raw, uint8_t *oper, const Params &p, int row0, int k,
+                                             int tid) {
+    int q, half;            // operand row within its 64-value-wide (half) tile, half index
+    const uint8_t *codes;
+    uint32_t sc;
+    bool valid;
+    if (!A_MN) {
+        q = tid;
+        half = 0;
+        codes = raw + q * 32;
+        sc = *reinterpret_cast<const uint32_t *>(raw + RAW_CODE_BYTES + (q & 31) * 16 + (q >> 5) * 4);
+        valid = row0 + q < p.a_rows;
+    } else {
+        q = tid & 63;
+        half = tid >> 6;
+        codes = raw + q * 64 + half * 32;
+        const int rr = (k & 127) + q;   // row within the scale group
+        sc = *reinterpret_cast<const uint32_t *>(raw + RAW_CODE_BYTES + half * 512 + (rr & 31) * 16 +
+                                                 ((rr >> 5) & 3) * 4);
+        valid = (k + q < p.a_rows) && (row0 + 64 * half < p.a_cols);
+    }
+    const uint4 c0 = *reinterpret_cast<const uint4 *>(codes);
+    const uint4 c1 = *reinterpret_cast<const uint4 *>(codes + 16);
+    const uint32_t w[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+    const uint32_t base = smem_u32(oper) + half * (A_BYTES / 2) + q * 128;
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+        const uint4 v = valid ? decode8_bf16(w[c], (sc >> (8 * (c >> 1))) & 0xFFu) : make_uint4(0, 0, 0, 0);
+        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(base + ((c ^ (q & 7)) << 4)), "r"(v.x),
+                     "r"(v.y), "r"(v.z), "r"(v.w)
+                     : "memory");
+    }
+}
+
+template <bool A_MN, bool B_MN, bool A_FP4>
 __global__ void __launch_bounds__(THREADS, 1)
 k_lora_mma(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, const Params p) {
+    constexpr int STAGE_BYTES = stage_bytes<A_FP4>();
     const Prob pr = p.prob[blockIdx.z];
     const int row0 = pr.row_begin + blockIdx.x * BM;
     if (row0 >= pr.row_end) return;  // block-uniform, before any shared state
@@ -76,12 +152,15 @@ k_lora_mma(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUte
     uint8_t *smem = smem_raw + (((raw + 1023) & ~1023u) - raw);
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + STAGES * STAGE_BYTES);
     uint64_t *full = bars, *empty = bars + STAGES, *acc_full = bars + 2 * STAGES;
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 2 * STAGES + 1);
+    uint64_t *raw_full = bars + 2 * STAGES + 1;   // [STAGES], A_FP4 only
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 3 * STAGES + 1);
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
-            mbar_init(&full[s], 1);
+            // A_FP4: the producer's arrival (B bytes) and the four decoding warps'
+            mbar_init(&full[s], A_FP4 ? 5 : 1);
             mbar_init(&empty[s], 1);
+            mbar_init(&raw_full[s], 1);
         }
         mbar_init(acc_full, 1);
         fence_barrier_init();
@@ -102,17 +181,40 @@ k_lora_mma(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUte
 
     if (warp == 0) {
         if (lane == 0) {
-            uint32_t stage = 0, phase = 0, pending = 0, pending_parity = 0;
+            uint32_t stage = 0, phase = 0, pending = 0, pending_parity = 0, raw_pending = 0;
             for (int kt = 0; kt < ktiles; ++kt) {
                 if (!mbar_wait(&empty[stage], phase ^ 1)) break;
                 uint8_t *st = smem + stage * STAGE_BYTES;
                 const int k = kb + kt * BK;
-                mbar_arrive_expect_tx(&full[stage], A_BYTES + nparts * b_bytes);
-                if (A_MN) {
-                    tma_load_2d(st, &tmA, &full[stage], row0, k);
-                    tma_load_2d(st + A_BYTES / 2, &tmA, &full[stage], row0 + 64, k);
+                if (A_FP4) {
+                    // codes box and the scale chunk(s) of this stage's A tile
+                    uint8_t *rw = st + OPER_BYTES;
+                    const int64_t chunks_per_group = p.a_cols / 64;
+                    if (!A_MN) {
+                        mbar_arrive_expect_tx(&raw_full[stage], RAW_CODE_BYTES + 512);
+                        tma_load_2d(rw, &tmA, &raw_full[stage], k / 2, row0);
+                        bulk_load(rw + RAW_CODE_BYTES,
+                                  p.a_scales + ((int64_t)(row0 / 128) * chunks_per_group + k / 64) * 512, 512,
+                                  &raw_full[stage]);
+                    } else {
+                        // the second half's chunk exists only while its columns do
+                        const uint32_t sbytes = (row0 / 64 + 1 < chunks_per_group) ? 1024u : 512u;
+                        mbar_arrive_expect_tx(&raw_full[stage], RAW_CODE_BYTES + sbytes);
+                        tma_load_2d(rw, &tmA, &raw_full[stage], row0 / 2, k);
+                        bulk_load(rw + RAW_CODE_BYTES,
+                                  p.a_scales + ((int64_t)(k / 128) * chunks_per_group + row0 / 64) * 512, sbytes,
+                                  &raw_full[stage]);
+                    }
+                    raw_pending |= 1u << stage;
+                    mbar_arrive_expect_tx(&full[stage], nparts * b_bytes);
                 } else {
-                    tma_load_2d(st, &tmA, &full[stage], k, row0);
+                    mbar_arrive_expect_tx(&full[stage], A_BYTES + nparts * b_bytes);
+                    if (A_MN) {
+                        tma_load_2d(st, &tmA, &full[stage], row0, k);
+                        tma_load_2d(st + A_BYTES / 2, &tmA, &full[stage], row0 + 64, k);
+                    } else {
+                        tma_load_2d(st, &tmA, &full[stage], k, row0);
+                    }
                 }
                 for (int h = 0; h < nparts; ++h) {
                     uint8_t *bd = st + A_BYTES + h * B_BYTES;
@@ -123,9 +225,15 @@ k_lora_mma(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUte
                 pending_parity = (pending_parity & ~(1u << stage)) | (phase << stage);
                 if (++stage == STAGES) { stage = 0; phase ^= 1; }
             }
-            // copies land before the CTA may leave
-            for (int s = 0; s < STAGES; ++s)
-                if (pending & (1u << s)) mbar_wait(&full[s], (pending_parity >> s) & 1u);
+            // copies land before the CTA may leave: the operand copies of the last use
+            // of each stage complete `full` (with the decoders' arrivals), the staged
+            // NVFP4 copies complete `raw_full`
+            for (int s = 0; s < STAGES; ++s) {
+                if (!(pending & (1u << s))) continue;
+                const uint32_t par = (pending_parity >> s) & 1u;
+                if (A_FP4 && (raw_pending & (1u << s))) mbar_wait(&raw_full[s], par);
+                mbar_wait(&full[s], par);
+            }
         }
     } else if (warp == 1) {
         const uint32_t idesc = idesc_bf16(BM, p.n_mma, A_MN, B_MN);
@@ -156,19 +264,38 @@ k_lora_mma(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUte
         if (lane == 0) tc_commit(acc_full);
         __syncwarp();
     } else {
+        bool ok = true;
+        if (A_FP4) {
+            // decode each stage's NVFP4 A tile into the BF16 operand buffer, then
+            // announce it on the stage's `full` barrier (after a proxy fence: the
+            // tensor core reads shared memory through the async proxy)
+            const int tid = threadIdx.x - 64;
+            uint32_t stage = 0, phase = 0;
+            for (int kt = 0; kt < ktiles; ++kt) {
+                if (!(ok = warp_all(mbar_wait(&raw_full[stage], phase)))) break;
+                uint8_t *st = smem + stage * STAGE_BYTES;
+                decode_stage<A_MN>(st + OPER_BYTES, st, p, row0, kb + kt * BK, tid);
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&full[stage]);
+                if (++stage == STAGES) { stage = 0; phase ^= 1; }
+            }
+        }
         const int sub = warp & 3;
-        const bool ok = mbar_wait(acc_full, 0);
+        ok = mbar_wait(acc_full, 0) && ok;
         tc_fence_after();
         const int r = row0 + sub * 32 + lane;
         for (int c = 0; c < p.n_mma / 16; ++c) {
             uint32_t v[16];
             tmem_ld_32x32b_x16(tmem + ((uint32_t)(sub * 32) << 16) + c * 16, v);
             tmem_ld_wait();
-            if (ok && r < pr.row_end) {
+            if (r < pr.row_end) {
+                // a wait that gave up leaves NaN partials, so the result is NaN rather
+                // than whatever the scratch held before
                 float *dst = part + (size_t)r * p.ws_ld + pr.out_col + c * 16;
 #pragma unroll
                 for (int j = 0; j < 16; ++j)
-                    if (c * 16 + j < p.n_valid) dst[j] = __uint_as_float(v[j]);
+                    if (c * 16 + j < p.n_valid) dst[j] = ok ? __uint_as_float(v[j]) : __int_as_float(0x7fc00000);
             }
         }
     }
@@ -184,49 +311,60 @@ k_lora_mma(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUte
 //   mode 0: hi + lo BF16 halves (hi at out[row * ldo + col], lo at col + lo_off)
 //   mode 1: BF16
 //   mode 2: BF16 transposed (out[col * ldo + row])
-__global__ void k_finalize(const float *__restrict__ ws, int splits, int64_t split_stride, int64_t ws_ld, int64_t rows,
-                           int64_t cols, float scale, int mode, pact_bf16 *__restrict__ out, int64_t ldo,
-                           int64_t lo_off) {
+//   mode 3, 4: as modes 1, 2 in FP32 (out32)
+// The partials are summed in split order (deterministic).  One launch serves one or
+// two such jobs (the index space of the second follows the first's).
+struct FinJob {
+    const float *ws;
+    int splits;
+    int64_t split_stride, ws_ld, rows, cols;
+    float scale;
+    int mode;
+    pact_bf16 *out;
+    int64_t ldo, lo_off;
+    float *out32;
+};
+
+__global__ void k_finalize(const FinJob j0, const FinJob j1, int njobs) {
     pdl_wait();
-    const int64_t n = rows * cols;
+    const int64_t n0 = j0.rows * j0.cols;
+    const int64_t n = n0 + (njobs > 1 ? j1.rows * j1.cols : 0);
     for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x) {
-        const int64_t r = mode == 2 ? i % rows : i / cols, c = mode == 2 ? i / rows : i % cols;
+        const bool second = i >= n0;
+        const FinJob &j = second ? j1 : j0;
+        const int64_t ii = second ? i - n0 : i;
+        const bool tr = j.mode == 2 || j.mode == 4;
+        const int64_t r = tr ? ii % j.rows : ii / j.cols, c = tr ? ii / j.rows : ii % j.cols;
         float acc = 0.0f;
-        for (int s = 0; s < splits; ++s) acc += ws[s * split_stride + r * ws_ld + c];
-        acc *= scale;
+        for (int s = 0; s < j.splits; ++s) acc += j.ws[s * j.split_stride + r * j.ws_ld + c];
+        acc *= j.scale;
+        if (j.mode >= 3) {
+            j.out32[tr ? c * j.ldo + r : r * j.ldo + c] = acc;
+            continue;
+        }
         const __nv_bfloat16 hi = __float2bfloat16_rn(acc);
-        if (mode == 2) {
-            out[c * ldo + r] = __bfloat16_as_ushort(hi);
+        if (j.mode == 2) {
+            j.out[c * j.ldo + r] = __bfloat16_as_ushort(hi);
         } else {
-            out[r * ldo + c] = __bfloat16_as_ushort(hi);
-            if (mode == 0)
-                out[r * ldo + c + lo_off] = __bfloat16_as_ushort(__float2bfloat16_rn(acc - __bfloat162float(hi)));
+            j.out[r * j.ldo + c] = __bfloat16_as_ushort(hi);
+            if (j.mode == 0)
+                j.out[r * j.ldo + c + j.lo_off] = __bfloat16_as_ushort(__float2bfloat16_rn(acc - __bfloat162float(hi)));
         }
     }
 }
 
-// NVFP4 -> BF16 (exact): the backward's view of a saved activation copy.
-__global__ void k_dequantize(pact_nvfp4_t t, pact_bf16 *__restrict__ out) {
-    pdl_wait();
-    const int64_t per_row = t.cols / 8;
-    const int64_t n8 = t.rows * per_row;
-    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n8; i += (int64_t)gridDim.x * blockDim.x) {
-        const int64_t r = i / per_row, c = (i % per_row) * 8;
-        float v[8];
-        load8_nvfp4(t, r, c, v);
-        store8_bf16(out + r * t.cols + c, v);
-    }
-}
-
 // ---------------------------------------------------------------- host side
+static int finalize_grid(int64_t n);
+
 typedef CUresult (*EncodeTiled)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
                                 const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
                                 CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 
-// 2-D tiled map over a BF16 row-major matrix: `inner` elements per row (row stride
-// `ld` elements), `outer` rows, 128-byte swizzle.
-static pact_status map_bf16(CUtensorMap *m, const void *base, uint64_t inner, uint64_t outer, uint64_t ld,
-                            uint32_t box_inner, uint32_t box_outer, const char *what) {
+// 2-D tiled map over a row-major matrix of `esize`-byte elements: `inner` elements
+// per row (row stride `ld` elements), `outer` rows.
+static pact_status map_2d(CUtensorMap *m, CUtensorMapDataType dt, int esize, CUtensorMapSwizzle sw, const void *base,
+                          uint64_t inner, uint64_t outer, uint64_t ld, uint32_t box_inner, uint32_t box_outer,
+                          const char *what) {
     static EncodeTiled enc = nullptr;
     if (!enc) {
         void *fp = nullptr;
@@ -238,29 +376,63 @@ static pact_status map_bf16(CUtensorMap *m, const void *base, uint64_t inner, ui
     }
     if (!enc) return fail(PACT_ERR_CUDA, "%s: cuTensorMapEncodeTiled unavailable", what);
     const cuuint64_t dims[2] = {inner, outer};
-    const cuuint64_t strides[1] = {ld * 2};
+    const cuuint64_t strides[1] = {ld * (uint64_t)esize};
     const cuuint32_t box[2] = {box_inner, box_outer};
     const cuuint32_t es[2] = {1, 1};
-    CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box, es,
-                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    CUresult r = enc(m, dt, 2, const_cast<void *>(base), dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
+                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS) return fail(PACT_ERR_CUDA, "%s: cuTensorMapEncodeTiled failed (%d)", what, (int)r);
     return PACT_OK;
 }
 
-template <bool A_MN, bool B_MN>
+// BF16 row-major matrix, 128-byte swizzle (the MMA operand layout).
+static pact_status map_bf16(CUtensorMap *m, const void *base, uint64_t inner, uint64_t outer, uint64_t ld,
+                            uint32_t box_inner, uint32_t box_outer, const char *what) {
+    return map_2d(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, CU_TENSOR_MAP_SWIZZLE_128B, base, inner, outer, ld,
+                  box_inner, box_outer, what);
+}
+
+// The code bytes of an NVFP4 tensor ([rows x cols / 2] bytes), unswizzled boxes of
+// box_bytes x box_rows: the staging copies of an NVFP4 A operand.
+static pact_status map_codes(CUtensorMap *m, const pact_nvfp4_t &t, uint32_t box_bytes, uint32_t box_rows,
+                             const char *what) {
+    return map_2d(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, CU_TENSOR_MAP_SWIZZLE_NONE, t.codes, (uint64_t)t.cols / 2,
+                  (uint64_t)t.rows, (uint64_t)t.cols / 2, box_bytes, box_rows, what);
+}
+
+// Params of an NVFP4 A operand.
+static void set_fp4_a(Params &p, const pact_nvfp4_t &t) {
+    p.a_scales = static_cast<const uint8_t *>(t.scales);
+    p.a_rows = t.rows;
+    p.a_cols = t.cols;
+}
+
+template <bool A_MN, bool B_MN, bool A_FP4 = false>
 static pact_status launch_mma(const CUtensorMap &ta, const CUtensorMap &tb, const Params &p, int row_tiles,
                               cudaStream_t st, const char *what) {
     static bool done[64] = {false};
     const int d = current_device();
+    constexpr int smem = smem_bytes<A_FP4>();
     if (d >= 0 && d < 64 && !done[d]) {
         cudaError_t e =
-            cudaFuncSetAttribute(k_lora_mma<A_MN, B_MN>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+            cudaFuncSetAttribute(k_lora_mma<A_MN, B_MN, A_FP4>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
         if (e != cudaSuccess) return fail(PACT_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
         done[d] = true;
     }
     dim3 grid((unsigned)row_tiles, (unsigned)p.splits, (unsigned)p.nprob);
-    return launch_dep(k_lora_mma<A_MN, B_MN>, grid, dim3(THREADS), SMEM_BYTES, st, what, ta, tb, p);
+    return launch_dep(k_lora_mma<A_MN, B_MN, A_FP4>, grid, dim3(THREADS), smem, st, what, ta, tb, p);
+}
+
+static FinJob fin_job(const float *ws, const Params &p, int64_t rows, int64_t cols, float scale, int mode,
+                      void *out, int64_t ldo, int64_t lo_off) {
+    return FinJob{ws, p.splits, p.ws_split_stride, p.ws_ld, rows, cols, scale, mode,
+                  mode >= 3 ? nullptr : static_cast<pact_bf16 *>(out), ldo, lo_off,
+                  mode >= 3 ? static_cast<float *>(out) : nullptr};
+}
+
+static pact_status finalize(const FinJob &j0, const FinJob *j1, cudaStream_t st, const char *what) {
+    const int64_t n = j0.rows * j0.cols + (j1 ? j1->rows * j1->cols : 0);
+    return launch_dep(k_finalize, dim3(finalize_grid(n)), dim3(256), 0, st, what, j0, j1 ? *j1 : j0, j1 ? 2 : 1);
 }
 
 // Split a contraction of length `len` over CTAs so that `blocks` output blocks x
@@ -292,10 +464,12 @@ static size_t partial_bytes(int64_t rows, int64_t cols, int splits) {
     return round256((size_t)(rows * cols * 4) * (size_t)splits);
 }
 
-// scale * X . A^T for X [M x K] (map tx) and A [R x K], written hi/lo into out
-// (row stride ldo, lo at column R); ws holds the partials.
-static pact_status rows_times_a(const CUtensorMap &tx, int64_t M, int64_t K, const pact_bf16 *A, int R, float scale,
-                                pact_bf16 *out, int64_t ldo, float *ws, cudaStream_t st, const char *what) {
+// scale * X . A^T for X [M x K] (map tx: BF16 rows, or the codes of the NVFP4 X when
+// xq is given) and A [R x K], written hi/lo into out (row stride ldo, lo at column R);
+// ws holds the partials.
+static pact_status rows_times_a(const CUtensorMap &tx, const pact_nvfp4_t *xq, int64_t M, int64_t K,
+                                const pact_bf16 *A, int R, float scale, pact_bf16 *out, int64_t ldo, float *ws,
+                                cudaStream_t st, const char *what) {
     CUtensorMap tb;
     pact_status s = map_bf16(&tb, A, K, R, K, 64, R, what);
     if (s != PACT_OK) return s;
@@ -309,10 +483,14 @@ static pact_status rows_times_a(const CUtensorMap &tx, int64_t M, int64_t K, con
     p.ws = ws;
     p.ws_ld = R;
     p.ws_split_stride = M * R;
-    s = launch_mma<false, false>(tx, tb, p, tiles, st, what);
+    if (xq) {
+        set_fp4_a(p, *xq);
+        s = launch_mma<false, false, true>(tx, tb, p, tiles, st, what);
+    } else {
+        s = launch_mma<false, false>(tx, tb, p, tiles, st, what);
+    }
     if (s != PACT_OK) return s;
-    return launch_dep(k_finalize, dim3(finalize_grid(M * R)), dim3(256), 0, st, what, (const float *)ws, p.splits,
-                      (int64_t)(M * R), (int64_t)R, (int64_t)M, (int64_t)R, scale, 0, out, ldo, (int64_t)R);
+    return finalize(fin_job(ws, p, M, R, scale, 0, out, ldo, R), nullptr, st, what);
 }
 
 static pact_status check_segments(int64_t N, int nseg, const int64_t *seg_end, const char *what) {
@@ -358,7 +536,7 @@ pact_status pact_lora_fwd(const pact_bf16 *x, int64_t ldx, int64_t M, int64_t K,
     CUtensorMap tx;
     pact_status s = map_bf16(&tx, x, K, M, ldx, 64, BM, "pact_lora_fwd");
     if (s != PACT_OK) return s;
-    return rows_times_a(tx, M, K, A, R, scale, T, ldt, static_cast<float *>(workspace), (cudaStream_t)stream,
+    return rows_times_a(tx, nullptr, M, K, A, R, scale, T, ldt, static_cast<float *>(workspace), (cudaStream_t)stream,
                         "pact_lora_fwd");
 }
 
@@ -405,16 +583,14 @@ pact_status pact_lora_bwd_u(const pact_bf16 *dy, int64_t lddy, int64_t M, int64_
     p.ws_split_stride = M * R;
     s = launch_mma<false, true>(ta, tb, p, tiles, st, "pact_lora_bwd_u");
     if (s != PACT_OK) return s;
-    return launch_dep(k_finalize, dim3(finalize_grid(M * R)), dim3(256), 0, st, "pact_lora_bwd_u", (const float *)ws,
-                      p.splits, (int64_t)(M * R), (int64_t)R, (int64_t)M, (int64_t)R, scale, 0, U, ldu, (int64_t)R);
+    return finalize(fin_job(ws, p, M, R, scale, 0, U, ldu, R), nullptr, st, "pact_lora_bwd_u");
 }
 
 // Upper bound over segmentations: the dB output blocks number at least N / 128.
 size_t pact_lora_bwd_workspace_bytes(int64_t M, int64_t N, int64_t K, int r, int nseg) {
     const int64_t R = (int64_t)r * nseg;
-    return round256((size_t)(M * K * 2))                                     /* X~ as BF16 */
-           + partial_bytes(M, R, splits_of(K, (M + BM - 1) / BM))         /* T~ partials */
-           + round256((size_t)(M * 2 * R * 2))                               /* T~ hi/lo */
+    return partial_bytes(M, R, splits_of(K, (M + BM - 1) / BM))          /* T~ partials */
+           + round256((size_t)(M * 2 * R * 2))                             /* T~ hi/lo */
            + partial_bytes(N, r, splits_of(M, (N + BM - 1) / BM))         /* dB partials */
            + partial_bytes(K, R, splits_of(M, (K + BM - 1) / BM));        /* dA^T partials */
 }
@@ -430,6 +606,7 @@ pact_status pact_lora_bwd(const pact_lora_bwd_t *g, void *workspace, size_t ws_b
                    nseg * r <= 64,
                PACT_ERR_SHAPE, "pact_lora_bwd: bad shape");
     PACT_CHECK(g->u_gexp >= -100 && g->u_gexp <= 100, PACT_ERR_INVALID_ARG, "pact_lora_bwd: |u_gexp| <= 100 required");
+    PACT_CHECK(g->grads_fp32 == 0 || g->grads_fp32 == 1, PACT_ERR_INVALID_ARG, "pact_lora_bwd: grads_fp32 is 0 or 1");
     pact_status s = check_segments(N, nseg, g->seg_end, "pact_lora_bwd");
     if (s != PACT_OK) return s;
     const int R = nseg * r;
@@ -445,8 +622,6 @@ pact_status pact_lora_bwd(const pact_lora_bwd_t *g, void *workspace, size_t ws_b
     }
     cudaStream_t st = (cudaStream_t)stream;
     uint8_t *w8 = static_cast<uint8_t *>(workspace);
-    pact_bf16 *xt = reinterpret_cast<pact_bf16 *>(w8);
-    w8 += round256((size_t)(M * K * 2));
     float *ws_t = reinterpret_cast<float *>(w8);
     w8 += partial_bytes(M, R, splits_of(K, (M + BM - 1) / BM));
     pact_bf16 *tt = reinterpret_cast<pact_bf16 *>(w8);
@@ -455,55 +630,46 @@ pact_status pact_lora_bwd(const pact_lora_bwd_t *g, void *workspace, size_t ws_b
     w8 += partial_bytes(N, r, splits_of(M, (N + BM - 1) / BM));
     float *ws_da = reinterpret_cast<float *>(w8);
 
-    // X~ as BF16
-    const pact_bf16 *x = g->x;
-    int64_t ldx = g->ldx;
-    if (g->xq) {
-        s = launch_dep(k_dequantize, dim3(finalize_grid(M * K / 8)), dim3(256), 0, st, "pact_lora_bwd", *g->xq, xt);
-        if (s != PACT_OK) return s;
-        x = xt;
-        ldx = K;
-    }
+    // X~ is read where it lies: BF16 rows, or the saved NVFP4 copy decoded in shared
+    // memory by the MMA kernel (no BF16 copy of it is written)
     // T~ = X~ . A^T (unscaled), hi/lo
     CUtensorMap tx;
-    s = map_bf16(&tx, x, K, M, ldx, 64, BM, "pact_lora_bwd");
-    if (s == PACT_OK) s = rows_times_a(tx, M, K, g->A, R, 1.0f, tt, 2 * R, ws_t, st, "pact_lora_bwd");
+    s = g->xq ? map_codes(&tx, *g->xq, BK / 2, BM, "pact_lora_bwd")
+              : map_bf16(&tx, g->x, K, M, g->ldx, 64, BM, "pact_lora_bwd");
+    if (s == PACT_OK) s = rows_times_a(tx, g->xq, M, K, g->A, R, 1.0f, tt, 2 * R, ws_t, st, "pact_lora_bwd");
     if (s != PACT_OK) return s;
     // dB_i = scale * dY_i^T . T~_i: output rows are the outputs n of segment i,
     // contraction over the tokens
+    Params pb = {};
     {
         CUtensorMap ta, tb;
         s = map_bf16(&ta, g->dy, N, M, g->lddy, 64, 64, "pact_lora_bwd");                // dY^T, MN-major
         if (s == PACT_OK) s = map_bf16(&tb, tt, 2 * R, M, 2 * R, 64, 64, "pact_lora_bwd");  // T~^T, MN-major
         if (s != PACT_OK) return s;
-        Params p = {};
-        p.n_mma = 64;
-        p.n_valid = r;
-        p.nprob = nseg;
+        pb.n_mma = 64;
+        pb.n_valid = r;
+        pb.nprob = nseg;
         int64_t widest = 0, blocks = 0, prev = 0;
         for (int i = 0; i < nseg; ++i) {
-            p.prob[i] = Prob{(int)prev, (int)g->seg_end[i], 0, (int)M, i * r, 0};
+            pb.prob[i] = Prob{(int)prev, (int)g->seg_end[i], 0, (int)M, i * r, 0};
             const int64_t w = g->seg_end[i] - prev;
             if (w > widest) widest = w;
             blocks += (w + BM - 1) / BM;
             prev = g->seg_end[i];
         }
-        p.b_split = 1;
-        p.b_lo_off = R;
-        choose_split(M, blocks, &p.splits, &p.k_per_split);
-        p.ws = ws_db;
-        p.ws_ld = r;
-        p.ws_split_stride = N * r;
-        s = launch_mma<true, true>(ta, tb, p, (int)((widest + BM - 1) / BM), st, "pact_lora_bwd");
-        if (s != PACT_OK) return s;
-        s = launch_dep(k_finalize, dim3(finalize_grid(N * r)), dim3(256), 0, st, "pact_lora_bwd", (const float *)ws_db,
-                       p.splits, (int64_t)(N * r), (int64_t)r, (int64_t)N, (int64_t)r, g->scale, 1, g->dB, (int64_t)r,
-                       (int64_t)0);
+        pb.b_split = 1;
+        pb.b_lo_off = R;
+        choose_split(M, blocks, &pb.splits, &pb.k_per_split);
+        pb.ws = ws_db;
+        pb.ws_ld = r;
+        pb.ws_split_stride = N * r;
+        s = launch_mma<true, true>(ta, tb, pb, (int)((widest + BM - 1) / BM), st, "pact_lora_bwd");
         if (s != PACT_OK) return s;
     }
     // dA^T = X~^T . U  [K x R], U = hi + lo
     CUtensorMap ta, tb;
-    s = map_bf16(&ta, x, K, M, ldx, 64, 64, "pact_lora_bwd");                   // X~^T, MN-major
+    s = g->xq ? map_codes(&ta, *g->xq, BM / 2, BK, "pact_lora_bwd")
+              : map_bf16(&ta, g->x, K, M, g->ldx, 64, 64, "pact_lora_bwd");             // X~^T, MN-major
     if (s == PACT_OK) s = map_bf16(&tb, g->U, 2 * R, M, g->ldu, 64, 64, "pact_lora_bwd");  // U^T, MN-major
     if (s != PACT_OK) return s;
     Params p = {};
@@ -518,11 +684,18 @@ pact_status pact_lora_bwd(const pact_lora_bwd_t *g, void *workspace, size_t ws_b
     p.ws = ws_da;
     p.ws_ld = R;
     p.ws_split_stride = K * R;
-    s = launch_mma<true, true>(ta, tb, p, tiles, st, "pact_lora_bwd");
+    if (g->xq) {
+        set_fp4_a(p, *g->xq);
+        s = launch_mma<true, true, true>(ta, tb, p, tiles, st, "pact_lora_bwd");
+    } else {
+        s = launch_mma<true, true>(ta, tb, p, tiles, st, "pact_lora_bwd");
+    }
     if (s != PACT_OK) return s;
-    return launch_dep(k_finalize, dim3(finalize_grid(K * R)), dim3(256), 0, st, "pact_lora_bwd", (const float *)ws_da,
-                      p.splits, (int64_t)(K * R), (int64_t)R, (int64_t)K, (int64_t)R, std::ldexp(1.0f, g->u_gexp), 2,
-                      g->dA, K, (int64_t)0);
+    // one pass finalizes both gradients (BF16, or FP32 for a later reduction)
+    const int f32 = g->grads_fp32 ? 2 : 0;
+    const FinJob jb = fin_job(ws_db, pb, N, r, g->scale, 1 + f32, g->dB, r, 0);
+    const FinJob ja = fin_job(ws_da, p, K, R, std::ldexp(1.0f, g->u_gexp), 2 + f32, g->dA, K, 0);
+    return finalize(jb, &ja, st, "pact_lora_bwd");
 }
 
 }  // extern "C"
@@ -549,11 +722,14 @@ static __device__ __align__(256) unsigned char g_noalloc_scratch[NOALLOC_SCRATCH
 
 // Device address of g_noalloc_scratch for the current device.  The symbol's host
 // name is only a stand-in, so the address is looked up once per device (with that
-// device current) and kept.
+// device current) and kept; a mutex makes concurrent first calls from several host
+// threads safe, and a failed lookup is retried on the next call.
 static pact_status noalloc_scratch(void **out) {
+    static std::mutex lock;
     static void *addr[64] = {nullptr};
     const int d = current_device();
     if (d < 0 || d >= 64) return fail(PACT_ERR_UNSUPPORTED, "pact_lora_fwd_noalloc: device index %d unsupported", d);
+    std::lock_guard<std::mutex> guard(lock);
     if (!addr[d]) {
         void *p = nullptr;
         const cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
@@ -588,6 +764,6 @@ extern "C" pact_status pact_lora_fwd_noalloc(const pact_bf16 *x, int64_t ldx, in
     CUtensorMap tx;
     s = map_bf16(&tx, x, K, M, ldx, 64, BM, "pact_lora_fwd_noalloc");
     if (s != PACT_OK) return s;
-    return rows_times_a(tx, M, K, A, R, scale, T, ldt, static_cast<float *>(scratch), (cudaStream_t)stream,
+    return rows_times_a(tx, nullptr, M, K, A, R, scale, T, ldt, static_cast<float *>(scratch), (cudaStream_t)stream,
                         "pact_lora_fwd_noalloc");
 }

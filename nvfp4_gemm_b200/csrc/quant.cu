@@ -496,6 +496,13 @@ __global__ void __launch_bounds__(256) k_weight_bwd_layout(pact_nvfp4_t wf, pact
     }
 }
 
+// y = BF16_RNE(x), elementwise.
+__global__ void __launch_bounds__(256) k_round_bf16(const float *__restrict__ x, pact_bf16 *__restrict__ y, int64_t n) {
+    pdl_wait();
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x)
+        y[i] = __bfloat16_as_ushort(__float2bfloat16_rn(x[i]));
+}
+
 // Zero scale rows [rows, round_up(rows, 128)) of a tensor (the layout's padding).
 __global__ void k_zero_scale_pad(pact_nvfp4_t t) {
     pdl_wait();
@@ -525,6 +532,14 @@ static size_t up256(size_t b) { return (b + 255) & ~(size_t)255; }
 size_t pact_weight_cache_bytes(int64_t N, int64_t K) {
     return up256(pact_nvfp4_code_bytes(N, K)) + up256(pact_scale_bytes(N, K)) + up256(pact_nvfp4_code_bytes(K, N)) +
            up256(pact_scale_bytes(K, N));
+}
+
+pact_status pact_round_bf16(const float *x, pact_bf16 *y, int64_t n, pact_stream_t stream) {
+    PACT_CHECK(x && y, PACT_ERR_INVALID_ARG, "pact_round_bf16: NULL argument");
+    PACT_CHECK(n >= 1, PACT_ERR_SHAPE, "pact_round_bf16: n >= 1 required");
+    PACT_CHECK(aligned16(x) && aligned16(y), PACT_ERR_ALIGN, "pact_round_bf16: pointers must be 16-byte aligned");
+    return launch_dep(k_round_bf16, dim3(grid_for((n + 31) / 32, 256)), dim3(256), 0, (cudaStream_t)stream,
+                      "pact_round_bf16", x, y, n);
 }
 
 pact_status pact_quantize_nvfp4(const pact_bf16 *x, int64_t ldx, int64_t rows, int64_t cols, const pact_nvfp4_t *out,

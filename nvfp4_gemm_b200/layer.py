@@ -73,13 +73,19 @@ class PactLayer:
     w = {q, k, v, o, gate, up, down}; lora_a = {p: [r, in]}, lora_b = {p: [out, r]};
     gamma1, gamma2: [H].  Frozen weights are cached as NVFP4 forward/backward layouts
     at construction (once); two_level selects the variant with a power of two per
-    cached group (pact_weight_layout_cache_scaled)."""
+    cached group (pact_weight_layout_cache_scaled).  grad_fp32: the LoRA weight
+    gradients are written unrounded in FP32 into one flat buffer (grad_bucket, views
+    in grads32), to be summed over data-parallel replicas in one collective and then
+    rounded once to BF16 by round_grads() into `grads`."""
+
+    input_keys = ("h", "attn", "d_out", "d_qkv")
 
     def __init__(self, shape: LayerShape, w: Dict[str, torch.Tensor], lora_a: Dict[str, torch.Tensor],
                  lora_b: Dict[str, torch.Tensor], gamma1: torch.Tensor, gamma2: torch.Tensor,
-                 two_level: bool = False):
+                 two_level: bool = False, grad_fp32: bool = False):
         self.s = shape
         self.two_level = two_level
+        self.grad_fp32 = grad_fp32
         S = shape
         dev = gamma1.device
         cat = lambda names, d: torch.cat([d[n] for n in names], 0).contiguous()
@@ -120,13 +126,13 @@ class PactLayer:
         self.dh2, self.dh2q = bf(M, H), nv(M, H)
         self.u_o, self.dattn = bf(M, 2 * r), bf(M, H)
         self.u_qkv, self.dqkvq, self.dx1, self.dh = bf(M, 2 * 3 * r), nv(M, S.n_qkv), bf(M, H), bf(M, H)
-        # LoRA weight gradients (BF16, same stacking as the adapters)
-        self.grads = {
-            "a_qkv": torch.empty_like(self.a_qkv), "b_qkv": torch.empty_like(self.b_qkv),
-            "a_o": torch.empty_like(self.a_o), "b_o": torch.empty_like(self.b_o),
-            "a_gu": torch.empty_like(self.a_gu), "b_gu": torch.empty_like(self.b_gu),
-            "a_d": torch.empty_like(self.a_d), "b_d": torch.empty_like(self.b_d),
-        }
+        # LoRA weight gradients (BF16, same stacking as the adapters), views of one flat
+        # buffer; with grad_fp32 also an FP32 flat buffer the backward writes
+        shapes = {"a_qkv": self.a_qkv.shape, "b_qkv": self.b_qkv.shape, "a_o": self.a_o.shape,
+                  "b_o": self.b_o.shape, "a_gu": self.a_gu.shape, "b_gu": self.b_gu.shape,
+                  "a_d": self.a_d.shape, "b_d": self.b_d.shape}
+        self.grad_bucket_bf16, self.grads = flat_views(shapes, torch.bfloat16, dev)
+        self.grad_bucket, self.grads32 = (flat_views(shapes, torch.float32, dev) if grad_fp32 else (None, None))
         # one scratch buffer shared by the LoRA calls (they run in order on one stream)
         ws = max(P.pact_lora_bwd_workspace_bytes(M, S.n_qkv, H, r, 3),
                  P.pact_lora_bwd_workspace_bytes(M, 2 * I, H, r, 2),
@@ -212,7 +218,8 @@ class PactLayer:
         S, s, r = self.s, self.s.scale, self.s.r
         H, I = S.H, S.I
         _, attn, d_out, d_qkv = self.inputs
-        g = self.grads
+        g = self.grads32 if self.grad_fp32 else self.grads
+        f32 = self.grad_fp32
         M = S.M
         gemm = lambda M, N, K: 2.0 * M * N * K
         gbytes = lambda N, K, R: S.nv(M, K) + S.nv(N, K) + 2 * M * N + 2 * M * 2 * R + 2 * K * R
@@ -220,7 +227,7 @@ class PactLayer:
         lora_u = lambda N, R: 2 * M * N + 2 * N * R + 2 * M * 2 * R
         # dA, dB: dY [M x N], the saved input (x_bytes), U [M x 2R] and A [R x K] in; dA, dB out
         lora_bwd = lambda N, x_bytes, K, R: 2 * M * N + x_bytes + 2 * M * 2 * R + 2 * R * K + 2 * R * K + 2 * N * R
-        LB = 7  # kernels of one pact_lora_bwd call reading an NVFP4 copy (6 with BF16 input)
+        LB = 5  # kernels of one pact_lora_bwd call
         return [
             # down projection
             Op("lora_bwd_u_down", lambda: P.pact_lora_bwd_u(d_out, self.b_d, r, [H], self.sc["d"], self.u_d, self.ws), kernels=2,
@@ -233,8 +240,8 @@ class PactLayer:
                bytes=2 * M * I + 2 * S.nv(M, I) + 4 * M * I + S.nv(M, 2 * I) + 2 * M * I),
             Op("lora_bwd_down", lambda: P.pact_lora_bwd(d_out, self.a_d, self.u_d, r, [H], s, x=self.m_re,
                                                         dA=g["a_d"], dB=g["b_d"], workspace=self.ws_leaf["down"],
-                                                        u_gexp=self.gexp["d"]),
-               kernels=LB - 1, side=True,
+                                                        u_gexp=self.gexp["d"], grads_fp32=f32),
+               kernels=LB, side=True,
                bytes=lora_bwd(H, 2 * M * I, I, r)),
             # gate|up
             Op("lora_bwd_u_gu", lambda: P.pact_lora_bwd_u(self.dgu, self.b_gu, r, self.seg_gu, self.sc["gu"], self.u_gu, self.ws), kernels=2,
@@ -243,7 +250,7 @@ class PactLayer:
                "gemm", gemm(S.M, H, 2 * I), bytes=gbytes(H, 2 * I, 2 * r)),
             Op("lora_bwd_gu", lambda: P.pact_lora_bwd(self.dgu, self.a_gu, self.u_gu, r, self.seg_gu, s,
                                                       xq=self.xq2, dA=g["a_gu"], dB=g["b_gu"],
-                                                      workspace=self.ws_leaf["gu"], u_gexp=self.gexp["gu"]),
+                                                      workspace=self.ws_leaf["gu"], u_gexp=self.gexp["gu"], grads_fp32=f32),
                kernels=LB, side=True, bytes=lora_bwd(2 * I, S.nv(M, H), H, 2 * r)),
             Op("rmsnorm_bwd_2", lambda: P.pact_rmsnorm_bwd(self.dx2, self.xq2, self.rstd2, self.g2, dres=d_out,
                                                            dx=self.dh2, dxq=self.dh2q),
@@ -255,8 +262,8 @@ class PactLayer:
                "gemm", gemm(S.M, H, H), bytes=gbytes(H, H, r)),
             Op("lora_bwd_o", lambda: P.pact_lora_bwd(self.dh2, self.a_o, self.u_o, r, [H], s, x=attn,
                                                      dA=g["a_o"], dB=g["b_o"], workspace=self.ws_leaf["o"],
-                                                     u_gexp=self.gexp["o"]),
-               kernels=LB - 1, side=True,
+                                                     u_gexp=self.gexp["o"], grads_fp32=f32),
+               kernels=LB, side=True,
                bytes=lora_bwd(H, 2 * M * H, H, r)),
             # q|k|v (d_qkv stands in for the attention backward)
             Op("lora_bwd_u_qkv", lambda: P.pact_lora_bwd_u(d_qkv, self.b_qkv, r, self.seg_qkv, self.sc["qkv"], self.u_qkv, self.ws), kernels=2,
@@ -266,13 +273,17 @@ class PactLayer:
                "gemm", gemm(S.M, H, S.n_qkv), bytes=gbytes(H, S.n_qkv, 3 * r)),
             Op("lora_bwd_qkv", lambda: P.pact_lora_bwd(d_qkv, self.a_qkv, self.u_qkv, r, self.seg_qkv, s,
                                                        xq=self.xq1, dA=g["a_qkv"], dB=g["b_qkv"],
-                                                       workspace=self.ws_leaf["qkv"], u_gexp=self.gexp["qkv"]),
+                                                       workspace=self.ws_leaf["qkv"], u_gexp=self.gexp["qkv"], grads_fp32=f32),
                kernels=LB, side=True,
                bytes=lora_bwd(S.n_qkv, S.nv(M, H), H, 3 * r)),
             Op("rmsnorm_bwd_1", lambda: P.pact_rmsnorm_bwd(self.dx1, self.xq1, self.rstd1, self.g1, dres=self.dh2,
                                                            dx=self.dh),
                bytes=2 * M * H + S.nv(M, H) + 4 * M + 2 * H + 2 * M * H + 2 * M * H),
         ]
+
+    def round_grads(self):
+        """grads = BF16_RNE(grads32), one rounding of the (possibly summed) FP32 gradients."""
+        P.pact_round_bf16(self.grad_bucket, self.grad_bucket_bf16)
 
     def saved_for_backward(self) -> Dict[str, torch.Tensor]:
         """The device tensors the forward leaves for the backward, i.e. the activation
@@ -294,6 +305,10 @@ class PactLayer:
         """Device bytes of the four cached weight groups (both layouts each)."""
         return sum(c.buf.numel() for c in (self.c_qkv, self.c_o, self.c_gu, self.c_d))
 
+    def bf16_weight_bytes(self) -> int:
+        """Bytes of the seven frozen weights in BF16."""
+        return 2 * int(self.s.frozen_flops() / (4.0 * self.s.M))
+
     def step_ops(self) -> List[Op]:
         return self.forward_ops() + self.backward_ops()
 
@@ -306,16 +321,131 @@ class PactLayer:
         ordered after everything issued before it on the current stream; the current
         stream waits for `side` at the end.  Same results as step(); under CUDA graph
         capture the leaves become a parallel branch of the graph."""
-        main = torch.cuda.current_stream()
-        for op in self.step_ops():
-            if op.side:
-                ready = torch.cuda.Event()
-                ready.record(main)
-                side.wait_event(ready)
-                with torch.cuda.stream(side):
-                    op.fn()
-            else:
+        run_concurrent(self.step_ops(), side)
+
+
+def flat_views(shapes: Dict[str, tuple], dtype, dev):
+    """One flat device buffer and a view of each requested shape in it, every view
+    starting 16-byte aligned."""
+    esz = torch.empty(0, dtype=dtype).element_size()
+    step = 16 // esz
+    offs, n = {}, 0
+    for k, shp in shapes.items():
+        offs[k] = n
+        cnt = 1
+        for d in shp:
+            cnt *= d
+        n += (cnt + step - 1) // step * step
+    buf = torch.zeros(n, dtype=dtype, device=dev)
+    views = {}
+    for k, shp in shapes.items():
+        cnt = 1
+        for d in shp:
+            cnt *= d
+        views[k] = buf[offs[k]:offs[k] + cnt].view(shp)
+    return buf, views
+
+
+def run_concurrent(ops: List[Op], side: torch.cuda.Stream):
+    """Run `ops` in order on the current stream, except the leaves (op.side), which
+    run on `side` after everything issued before them; the current stream waits for
+    `side` at the end."""
+    main = torch.cuda.current_stream()
+    for op in ops:
+        if op.side:
+            ready = torch.cuda.Event()
+            ready.record(main)
+            side.wait_event(ready)
+            with torch.cuda.stream(side):
                 op.fn()
-        done = torch.cuda.Event()
-        done.record(side)
-        main.wait_event(done)
+        else:
+            op.fn()
+    done = torch.cuda.Event()
+    done.record(side)
+    main.wait_event(done)
+
+
+class PactProjection:
+    """One frozen projection with its BF16 LoRA branch, forward and backward: the
+    single-projection workload (X[M x K], W[N x K], LoRA r, alpha).
+
+      forward   xq = q(X);  T = s X A^T;  Y = deq(xq) deq(Wf)^T + T B^T
+      backward  U = s dY B;  dX = deq(q(dY)) deq(Wb)^T + U A
+                dA = U^T X~,  dB = s dY^T (X~ A^T)   with X~ = deq(xq), the saved copy
+
+    (PACT blog summary, section "方法", bullets 1, 2 and 4 and the paragraph after
+    them; PEFT explainer, section "LoRA").  Same interface as PactLayer: bind() the
+    step's inputs, then step() / step_ops() / step_concurrent()."""
+
+    input_keys = ("x", "dy")
+
+    def __init__(self, W: torch.Tensor, A: torch.Tensor, B: torch.Tensor, M: int, r: int = 16,
+                 alpha: float = 32.0):
+        N, K = W.shape
+        self.M, self.N, self.K, self.r = M, N, K, r
+        self.scale = alpha / r
+        dev = W.device
+        self.c_w = P.pact_weight_layout_cache(W)
+        self.A, self.B = A.contiguous(), B.contiguous()
+        bf = lambda *sh: torch.empty(sh, dtype=torch.bfloat16, device=dev)
+        self.xq, self.t, self.y = P.NVFP4Tensor.empty(M, K, dev), bf(M, 2 * r), bf(M, N)
+        self.u, self.dyq, self.dx = bf(M, 2 * r), P.NVFP4Tensor.empty(M, N, dev), bf(M, K)
+        self.grads = {"a": torch.empty_like(self.A), "b": torch.empty_like(self.B)}
+        ws = max(P.pact_lora_fwd_workspace_bytes(M, K, r), P.pact_lora_bwd_u_workspace_bytes(M, N, r, 1))
+        self.ws = PactLayer._scratch(ws, dev)
+        self.ws_leaf = PactLayer._scratch(P.pact_lora_bwd_workspace_bytes(M, N, K, r, 1), dev)
+        self.l_f = P.lora_struct(self.t, self.B, r, [N])
+        self.l_b = P.lora_struct(self.u, self.A, r, [K])
+        self.inputs = None
+
+    def bind(self, x: torch.Tensor, dy: torch.Tensor):
+        self.inputs = (x, dy)
+
+    def forward_ops(self) -> List[Op]:
+        M, N, K, r = self.M, self.N, self.K, self.r
+        x, _ = self.inputs
+        nv = lambda rows, cols: rows * cols / 2 + rows * cols / 16
+        return [
+            Op("quantize_x", lambda: P.pact_quantize_nvfp4(x, self.xq), bytes=2 * M * K + nv(M, K)),
+            Op("lora_fwd", lambda: P.pact_lora_fwd(x, self.A, self.scale, self.t, self.ws), kernels=2,
+               bytes=2 * M * K + 2 * r * K + 2 * M * 2 * r),
+            Op("gemm_fwd", lambda: P.pact_frozen_gemm_fwd(self.xq, self.c_w, self.l_f, y=self.y), "gemm",
+               2.0 * M * N * K, bytes=nv(M, K) + nv(N, K) + 2 * M * N + 2 * M * 2 * r + 2 * N * r),
+        ]
+
+    def backward_ops(self) -> List[Op]:
+        M, N, K, r = self.M, self.N, self.K, self.r
+        _, dy = self.inputs
+        g = self.grads
+        nv = lambda rows, cols: rows * cols / 2 + rows * cols / 16
+        return [
+            Op("lora_bwd_u", lambda: P.pact_lora_bwd_u(dy, self.B, r, [N], self.scale, self.u, self.ws), kernels=2,
+               bytes=2 * M * N + 2 * N * r + 2 * M * 2 * r),
+            Op("quantize_dy", lambda: P.pact_quantize_nvfp4(dy, self.dyq), bytes=2 * M * N + nv(M, N)),
+            Op("gemm_dgrad", lambda: P.pact_frozen_gemm_dgrad(self.dyq, self.c_w, self.l_b, dx=self.dx), "gemm",
+               2.0 * M * N * K, bytes=nv(M, N) + nv(N, K) + 2 * M * K + 2 * M * 2 * r + 2 * K * r),
+            Op("lora_bwd", lambda: P.pact_lora_bwd(dy, self.A, self.u, r, [N], self.scale, xq=self.xq, dA=g["a"],
+                                                   dB=g["b"], workspace=self.ws_leaf),
+               kernels=5, side=True, bytes=2 * M * N + nv(M, K) + 2 * M * 2 * r + 4 * r * K + 2 * N * r),
+        ]
+
+    def step_ops(self) -> List[Op]:
+        return self.forward_ops() + self.backward_ops()
+
+    def step(self):
+        for op in self.step_ops():
+            op.fn()
+
+    def step_concurrent(self, side: torch.cuda.Stream):
+        run_concurrent(self.step_ops(), side)
+
+    def saved_bytes(self) -> int:
+        """The forward leaves the NVFP4 copy of X (codes and padded scales) for the
+        backward."""
+        return self.xq.codes.numel() + self.xq.scales.numel()
+
+    def weight_cache_bytes(self) -> int:
+        return self.c_w.buf.numel()
+
+    def bf16_weight_bytes(self) -> int:
+        return 2 * self.N * self.K

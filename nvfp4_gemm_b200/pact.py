@@ -51,7 +51,7 @@ class c_lora_bwd(ctypes.Structure):
                 ("A", ctypes.c_void_p), ("U", ctypes.c_void_p), ("ldu", ctypes.c_int64),
                 ("r", ctypes.c_int), ("nseg", ctypes.c_int), ("seg_end", ctypes.c_int64 * 4),
                 ("scale", ctypes.c_float), ("u_gexp", ctypes.c_int), ("dA", ctypes.c_void_p),
-                ("dB", ctypes.c_void_p)]
+                ("dB", ctypes.c_void_p), ("grads_fp32", ctypes.c_int)]
 
 
 def _load() -> ctypes.CDLL:
@@ -89,6 +89,11 @@ def _load() -> ctypes.CDLL:
         "pact_status_string": (ctypes.c_char_p, [S]),
         "pact_get_device_status": (S, [P]),
         "pact_abi_version": (I, []),
+        "pact_selftest_wait_timeout": (S, [I64, P, P]),
+        "pact_round_bf16": (S, [P, P, I64, P]),
+        "pact_gptq_workspace_bytes": (ctypes.c_size_t, [I64, I64, I64]),
+        "pact_gptq_nvfp4": (S, [P, I64, I64, I64, P, I64, I64, ctypes.c_double, P, ctypes.c_size_t, NV, P, P]),
+        "pact_weight_layout_cache_from_nvfp4": (S, [NV, I, P, ctypes.c_size_t, ctypes.POINTER(c_weight_cache), P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -281,6 +286,47 @@ def pact_weight_layout_cache(W: torch.Tensor, stream=None, two_level: bool = Fal
     return WeightCache(buf, c, N, K)
 
 
+def pact_gptq_workspace_bytes(N: int, K: int, n: int) -> int:
+    return int(_lib.pact_gptq_workspace_bytes(N, K, n))
+
+
+def pact_gptq_nvfp4(W: torch.Tensor, X: torch.Tensor, damp: float = 0.01, out: Optional[NVFP4Tensor] = None,
+                    workspace: Optional[torch.Tensor] = None, pivot_error: Optional[torch.Tensor] = None,
+                    stream=None) -> NVFP4Tensor:
+    """NVFP4-adapted GPTQ calibration of W [N x K] on calibration inputs X [n x K]:
+    the calibrated forward NVFP4 layout of W."""
+    _bf16(W, "W")
+    _bf16(X, "X")
+    N, K = W.shape
+    n = X.shape[0]
+    out = out or NVFP4Tensor.empty(N, K, W.device)
+    need = pact_gptq_workspace_bytes(N, K, n)
+    if workspace is None:
+        raw = torch.empty(need + 256, dtype=torch.uint8, device=W.device)
+        off = (-raw.data_ptr()) % 256
+        workspace = raw[off:off + need]
+    s = out.c()
+    _check(_lib.pact_gptq_nvfp4(W.data_ptr(), _ld(W), N, K, X.data_ptr(), _ld(X), n, float(damp),
+                                workspace.data_ptr(), workspace.numel(), ctypes.byref(s), _ptr(pivot_error),
+                                _stream(stream)))
+    return out
+
+
+def pact_weight_layout_cache_from_nvfp4(wf: NVFP4Tensor, gexp: int = 0, stream=None) -> WeightCache:
+    """The cached layouts of a weight given by its forward NVFP4 layout (e.g. a
+    GPTQ-calibrated one)."""
+    N, K = wf.rows, wf.cols
+    nbytes = pact_weight_cache_bytes(N, K)
+    buf = torch.empty(nbytes + 256, dtype=torch.uint8, device=wf.codes.device)
+    off = (-buf.data_ptr()) % 256
+    buf = buf[off:off + nbytes]
+    c = c_weight_cache()
+    s = wf.c()
+    _check(_lib.pact_weight_layout_cache_from_nvfp4(ctypes.byref(s), int(gexp), buf.data_ptr(), nbytes,
+                                                    ctypes.byref(c), _stream(stream)))
+    return WeightCache(buf, c, N, K)
+
+
 def pact_frozen_gemm_fwd(xq: NVFP4Tensor, w: WeightCache, lora: Optional[c_lora] = None,
                          residual: Optional[torch.Tensor] = None, y: Optional[torch.Tensor] = None,
                          stream=None) -> torch.Tensor:
@@ -370,15 +416,19 @@ def pact_lora_bwd_workspace_bytes(M: int, N: int, K: int, r: int, nseg: int) -> 
 def pact_lora_bwd(dy: torch.Tensor, A: torch.Tensor, U: torch.Tensor, r: int, seg_end: Sequence[int], scale: float,
                   x: Optional[torch.Tensor] = None, xq: Optional[NVFP4Tensor] = None,
                   dA: Optional[torch.Tensor] = None, dB: Optional[torch.Tensor] = None,
-                  workspace: Optional[torch.Tensor] = None, stream=None, u_gexp: int = 0):
+                  workspace: Optional[torch.Tensor] = None, stream=None, u_gexp: int = 0, grads_fp32: bool = False):
+    """dA, dB (BF16, or FP32 when grads_fp32: unrounded, for a later sum over replicas)."""
     _bf16(dy, "dy")
     M, N = dy.shape
     K = A.shape[1]
     nseg = len(seg_end)
+    gdt = torch.float32 if grads_fp32 else torch.bfloat16
     if dA is None:
-        dA = torch.empty((nseg * r, K), dtype=torch.bfloat16, device=dy.device)
+        dA = torch.empty((nseg * r, K), dtype=gdt, device=dy.device)
     if dB is None:
-        dB = torch.empty((N, r), dtype=torch.bfloat16, device=dy.device)
+        dB = torch.empty((N, r), dtype=gdt, device=dy.device)
+    if dA.dtype != gdt or dB.dtype != gdt:
+        raise TypeError(f"dA and dB must be {gdt}")
     need = pact_lora_bwd_workspace_bytes(M, N, K, r, nseg)
     if workspace is None:
         workspace = torch.empty(need + 256, dtype=torch.uint8, device=dy.device)
@@ -397,8 +447,19 @@ def pact_lora_bwd(dy: torch.Tensor, A: torch.Tensor, U: torch.Tensor, r: int, se
     args.scale = float(scale)
     args.u_gexp = int(u_gexp)
     args.dA, args.dB = dA.data_ptr(), dB.data_ptr()
+    args.grads_fp32 = int(bool(grads_fp32))
     _check(_lib.pact_lora_bwd(ctypes.byref(args), workspace.data_ptr(), workspace.numel(), _stream(stream)))
     return dA, dB
+
+
+def pact_round_bf16(x: torch.Tensor, y: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """BF16 rounding of a contiguous FP32 device tensor (same shape)."""
+    if x.dtype != torch.float32 or not x.is_contiguous():
+        raise TypeError("x: expected a contiguous float32 tensor")
+    if y is None:
+        y = torch.empty(x.shape, dtype=torch.bfloat16, device=x.device)
+    _check(_lib.pact_round_bf16(x.data_ptr(), y.data_ptr(), x.numel(), _stream(stream)))
+    return y
 
 
 def pact_silu_mul_bwd_quant(dm: torch.Tensor, gq: NVFP4Tensor, uq: NVFP4Tensor, dgu: Optional[torch.Tensor] = None,
@@ -443,3 +504,9 @@ def pact_last_error() -> str:
 
 def pact_abi_version() -> int:
     return int(_lib.pact_abi_version())
+
+
+def pact_selftest_wait_timeout(limit_cycles: int, waited: Optional[torch.Tensor] = None, stream=None) -> None:
+    """Make one bounded device wait run out (see include/pact.h); `waited`, a one-element
+    int64 device tensor, receives the cycles the wait took."""
+    _check(_lib.pact_selftest_wait_timeout(int(limit_cycles), _ptr(waited), _stream(stream)))

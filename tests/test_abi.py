@@ -36,7 +36,7 @@ def test_every_declared_symbol_is_exported(P):
 
 
 def test_abi_version_and_status_names(P):
-    assert P.pact_abi_version() == 2
+    assert P.pact_abi_version() == 3
     lib = P.pact.lib
     assert lib.pact_status_string(0) == b"PACT_OK"
     assert lib.pact_status_string(5) == b"PACT_ERR_TIMEOUT"
@@ -140,6 +140,13 @@ def test_two_level_host_checks(P):
     wcache = pm.c_weight_cache(pm.c_nvfp4(0x1000, 0x2000, 512, 512), pm.c_nvfp4(0x3000, 0x4000, 512, 512), 200)
     xq = pm.c_nvfp4(0x5000, 0x6000, 256, 512)
     assert lib.pact_frozen_gemm_fwd(ctypes.byref(xq), ctypes.byref(wcache), None, None, 0, 0x7000, 512, None) == 1
+
+
+def test_wait_selftest_limit_is_checked_on_the_host(P):
+    lib = P.pact.lib
+    for bad in (0, 10, 5_000_000_000):
+        assert lib.pact_selftest_wait_timeout(bad, None, None) == 1
+    assert lib.pact_selftest_wait_timeout(10_000, 0x1004, None) == 3      # misaligned output
 
 
 def test_plain_c_program_links_and_calls_the_host_functions(P, tmp_path):

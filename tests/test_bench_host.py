@@ -11,11 +11,11 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
 def test_gemm_traffic_follows_the_source_hash():
     csrc = os.path.join(ROOT, "nvfp4_gemm_b200", "csrc")
-    same = all(hashlib.sha256(open(os.path.join(csrc, n), "rb").read()).hexdigest()[:16] == h
-               for n, h in bench.GEMM_TRAFFIC["sha256_16"].items())
-    got = bench.gemm_traffic("llama-3.2-1b")
-    assert got == (bench.GEMM_TRAFFIC["bytes_per_launch"] if same else None)
-    assert bench.gemm_traffic("qwen2.5-1.5b") is None      # captured on one workload only
+    for workload, rec in bench.GEMM_TRAFFIC.items():
+        same = all(hashlib.sha256(open(os.path.join(csrc, n), "rb").read()).hexdigest()[:16] == h
+                   for n, h in rec["sha256_16"].items())
+        assert bench.gemm_traffic(workload) == (rec["bytes_per_launch"] if same else None)
+    assert bench.gemm_traffic("no-such-workload") is None
 
 
 def test_bf16_lora_saved_bytes_hand_count():

@@ -237,12 +237,15 @@ def test_gemm_dgrad_lora(P, orc, M, N, K, R):
 
 
 # ------------------------------------------------------------------------- LoRA
-@pytest.mark.parametrize("M,parts,r", [(256, [512], 16), (300, [512, 256, 256], 16), (130, [256, 320], 32)])
-def test_lora_bwd(P, orc, M, parts, r):
+@pytest.mark.parametrize("M,parts,r,K", [(256, [512], 16, 384), (300, [512, 256, 256], 16, 576),
+                                         (130, [256, 320], 32, 320), (2048, [1024], 16, 2112)])
+def test_lora_bwd(P, orc, M, parts, r, K):
+    """dA and dB from BF16 X and from the NVFP4 copy of X (decoded inside the MMA
+    kernel); K values that end mid-way through a 128-feature tile and token counts
+    that end mid-way through a 128-token scale group cover the ragged edges."""
     N = sum(parts)
     seg_end = _segments(N, parts)
     nseg = len(parts)
-    K = 384
     dy = synth.gaussian_bf16(50, (M, N))
     x = synth.gaussian_bf16(1, (M, K))
     a = synth.gaussian_bf16(20, (nseg * r, K), std=0.02)
@@ -253,7 +256,12 @@ def test_lora_bwd(P, orc, M, parts, r):
     dA, dB = P.pact_lora_bwd(dyd, ad, U, r, seg_end, s, x=xd)
     xq = P.pact_quantize_nvfp4(xd)
     dA2, dB2 = P.pact_lora_bwd(dyd, ad, U, r, seg_end, s, xq=xq)
+    # FP32 gradients (for a sum over replicas) round to the BF16 ones bit for bit
+    dA3, dB3 = P.pact_lora_bwd(dyd, ad, U, r, seg_end, s, xq=xq, grads_fp32=True)
     sync()
+    assert dA3.dtype == torch.float32 and dB3.dtype == torch.float32
+    for g32, g16 in ((dA3, dA2), (dB3, dB2)):
+        assert torch.equal(P.pact_round_bf16(g32.contiguous()).view(torch.int16), g16.view(torch.int16))
     dyf, xf = synth.bf16_bits_to_f64(dy), synth.bf16_bits_to_f64(x)
     af, bf = synth.bf16_bits_to_f64(a), synth.bf16_bits_to_f64(b)
     R = nseg * r
