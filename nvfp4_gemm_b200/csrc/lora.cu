@@ -24,7 +24,7 @@ namespace lmma {
 
 constexpr int BM = 128;        // output rows per CTA (MMA M)
 constexpr int BK = 64;         // contraction elements per stage (128 bytes of BF16)
-constexpr int STAGES = 4;
+constexpr int STAGES = 3;      // with stages sized to the product, two CTAs fit on an SM
 constexpr int THREADS = 192;
 constexpr int A_BYTES = BM * BK * 2;     // 16384
 constexpr int B_BYTES = 64 * BK * 2;     // 8192 per B part
@@ -33,11 +33,13 @@ constexpr int B_BYTES = 64 * BK * 2;     // 8192 per B part
 // warps decode them into the BF16 operand buffer before the MMA reads it
 constexpr int RAW_CODE_BYTES = BM * BK / 2;                      // 4096
 constexpr int RAW_BYTES = RAW_CODE_BYTES + 1024;
-constexpr int OPER_BYTES = A_BYTES + 2 * B_BYTES;                // 32768
-template <bool A_FP4>
-__host__ __device__ constexpr int stage_bytes() { return OPER_BYTES + (A_FP4 ? RAW_BYTES : 0); }   // multiples of 1024
-template <bool A_FP4>
-__host__ __device__ constexpr int smem_bytes() { return 1024 + STAGES * stage_bytes<A_FP4>() + 256; }
+// A stage holds the A tile, one or two B parts (the hi and lo halves of T or U) and,
+// for an NVFP4 A, its staging area; all multiples of 1024 bytes.
+__host__ __device__ constexpr int oper_bytes(int nparts) { return A_BYTES + nparts * B_BYTES; }
+__host__ __device__ constexpr int stage_bytes(int nparts, bool fp4) { return oper_bytes(nparts) + (fp4 ? RAW_BYTES : 0); }
+__host__ __device__ constexpr int smem_bytes(int nparts, bool fp4) { return 1024 + STAGES * stage_bytes(nparts, fp4) + 256; }
+constexpr int SM_SMEM = 233472;   // shared memory per SM (228 KiB), 1 KiB of it reserved per CTA
+__host__ __device__ constexpr int ctas_per_sm(int nparts, bool fp4) { return SM_SMEM / (smem_bytes(nparts, fp4) + 1024); }
 constexpr uint32_t TMEM_COLS = 64;
 
 // One output block: rows [row_begin, row_end) of the output, contraction
@@ -128,7 +130,8 @@ __device__ __forceinline__ void decode_stage(const uint8_t *raw, uint8_t *oper, 
 template <bool A_MN, bool B_MN, bool A_FP4>
 __global__ void __launch_bounds__(THREADS, 1)
 k_lora_mma(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, const Params p) {
-    constexpr int STAGE_BYTES = stage_bytes<A_FP4>();
+    const int nparts = p.b_split ? 2 : 1;
+    const int STAGE_BYTES = stage_bytes(nparts, A_FP4), OPER_BYTES = oper_bytes(nparts);
     const Prob pr = p.prob[blockIdx.z];
     const int row0 = pr.row_begin + blockIdx.x * BM;
     if (row0 >= pr.row_end) return;  // block-uniform, before any shared state
@@ -176,7 +179,6 @@ k_lora_mma(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUte
     tc_fence_after();
     pdl_wait();   // inputs of the previous kernel are complete from here on
     const uint32_t tmem = *tmem_slot;
-    const int nparts = p.b_split ? 2 : 1;
     const uint32_t b_bytes = B_MN ? (uint32_t)B_BYTES : (uint32_t)p.n_mma * BK * 2;
 
     if (warp == 0) {
@@ -412,10 +414,10 @@ static pact_status launch_mma(const CUtensorMap &ta, const CUtensorMap &tb, cons
                               cudaStream_t st, const char *what) {
     static bool done[64] = {false};
     const int d = current_device();
-    constexpr int smem = smem_bytes<A_FP4>();
+    const int smem = smem_bytes(p.b_split ? 2 : 1, A_FP4);
     if (d >= 0 && d < 64 && !done[d]) {
-        cudaError_t e =
-            cudaFuncSetAttribute(k_lora_mma<A_MN, B_MN, A_FP4>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+        cudaError_t e = cudaFuncSetAttribute(k_lora_mma<A_MN, B_MN, A_FP4>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             smem_bytes(2, A_FP4));
         if (e != cudaSuccess) return fail(PACT_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
         done[d] = true;
     }
@@ -435,13 +437,12 @@ static pact_status finalize(const FinJob &j0, const FinJob *j1, cudaStream_t st,
     return launch_dep(k_finalize, dim3(finalize_grid(n)), dim3(256), 0, st, what, j0, j1 ? *j1 : j0, j1 ? 2 : 1);
 }
 
-// Split a contraction of length `len` over CTAs so that `blocks` output blocks x
-// splits covers the SMs, with at least 4 stages (256 elements) per split.
-// Splits of the contraction so that blocks x splits CTAs fill the SMs in ONE wave
-// (a CTA takes a whole SM: 132 KB of shared memory), each split at least 4 stages
-// long.  Rounding the split count up instead left a nearly empty second wave.
-static void choose_split(int64_t len, int64_t blocks, int *splits, int *kps) {
-    int64_t s = sm_count() / (blocks > 0 ? blocks : 1);
+// Splits of a contraction of length `len` so that `blocks` output blocks x splits
+// CTAs fill the SMs in ONE wave (`per_sm` CTAs of this kind fit on an SM), each split
+// at least 4 stages long.  Rounding the split count up instead left a nearly empty
+// second wave.
+static void choose_split(int64_t len, int64_t blocks, int per_sm, int *splits, int *kps) {
+    int64_t s = (int64_t)sm_count() * per_sm / (blocks > 0 ? blocks : 1);
     const int64_t max_s = (len + 4 * BK - 1) / (4 * BK);
     if (s > max_s) s = max_s;
     if (s < 1) s = 1;
@@ -479,7 +480,7 @@ static pact_status rows_times_a(const CUtensorMap &tx, const pact_nvfp4_t *xq, i
     p.nprob = 1;
     p.prob[0] = Prob{0, (int)M, 0, (int)K, 0, 0};
     const int tiles = (int)((M + BM - 1) / BM);
-    choose_split(K, tiles, &p.splits, &p.k_per_split);
+    choose_split(K, tiles, ctas_per_sm(1, xq != nullptr), &p.splits, &p.k_per_split);
     p.ws = ws;
     p.ws_ld = R;
     p.ws_split_stride = M * R;
@@ -511,14 +512,19 @@ using namespace pact::lmma;
 
 extern "C" {
 
-static int splits_of(int64_t len, int64_t blocks) {
+static int splits_of(int64_t len, int64_t blocks, int per_sm) {
     int s, k;
-    choose_split(len, blocks, &s, &k);
+    choose_split(len, blocks, per_sm, &s, &k);
     return s;
 }
 
+// Workspace bounds cover both the BF16 and the NVFP4 form of X~ (more CTAs per SM
+// give at least as many splits).
+constexpr int T_PER_SM = ctas_per_sm(1, false) > ctas_per_sm(1, true) ? ctas_per_sm(1, false) : ctas_per_sm(1, true);
+constexpr int DA_PER_SM = ctas_per_sm(2, false) > ctas_per_sm(2, true) ? ctas_per_sm(2, false) : ctas_per_sm(2, true);
+
 size_t pact_lora_fwd_workspace_bytes(int64_t M, int64_t K, int R) {
-    return partial_bytes(M, R, splits_of(K, (M + BM - 1) / BM));
+    return partial_bytes(M, R, splits_of(K, (M + BM - 1) / BM, ctas_per_sm(1, false)));
 }
 
 pact_status pact_lora_fwd(const pact_bf16 *x, int64_t ldx, int64_t M, int64_t K, const pact_bf16 *A, int R,
@@ -542,7 +548,7 @@ pact_status pact_lora_fwd(const pact_bf16 *x, int64_t ldx, int64_t M, int64_t K,
 
 // Upper bound over segmentations: one segment may span all N outputs.
 size_t pact_lora_bwd_u_workspace_bytes(int64_t M, int64_t N, int r, int nseg) {
-    return partial_bytes(M, (int64_t)r * nseg, splits_of(N, (M + BM - 1) / BM));
+    return partial_bytes(M, (int64_t)r * nseg, splits_of(N, (M + BM - 1) / BM, ctas_per_sm(1, false)));
 }
 
 pact_status pact_lora_bwd_u(const pact_bf16 *dy, int64_t lddy, int64_t M, int64_t N, const pact_bf16 *B, int r,
@@ -576,7 +582,7 @@ pact_status pact_lora_bwd_u(const pact_bf16 *dy, int64_t lddy, int64_t M, int64_
         prev = seg_end[i];
     }
     const int tiles = (int)((M + BM - 1) / BM);
-    choose_split(longest, (int64_t)tiles * nseg, &p.splits, &p.k_per_split);
+    choose_split(longest, (int64_t)tiles * nseg, ctas_per_sm(1, false), &p.splits, &p.k_per_split);
     float *ws = static_cast<float *>(workspace);
     p.ws = ws;
     p.ws_ld = R;
@@ -589,10 +595,10 @@ pact_status pact_lora_bwd_u(const pact_bf16 *dy, int64_t lddy, int64_t M, int64_
 // Upper bound over segmentations: the dB output blocks number at least N / 128.
 size_t pact_lora_bwd_workspace_bytes(int64_t M, int64_t N, int64_t K, int r, int nseg) {
     const int64_t R = (int64_t)r * nseg;
-    return partial_bytes(M, R, splits_of(K, (M + BM - 1) / BM))          /* T~ partials */
-           + round256((size_t)(M * 2 * R * 2))                             /* T~ hi/lo */
-           + partial_bytes(N, r, splits_of(M, (N + BM - 1) / BM))         /* dB partials */
-           + partial_bytes(K, R, splits_of(M, (K + BM - 1) / BM));        /* dA^T partials */
+    return partial_bytes(M, R, splits_of(K, (M + BM - 1) / BM, T_PER_SM))      /* T~ partials */
+           + round256((size_t)(M * 2 * R * 2))                                  /* T~ hi/lo */
+           + partial_bytes(N, r, splits_of(M, (N + BM - 1) / BM, ctas_per_sm(2, false)))  /* dB partials */
+           + partial_bytes(K, R, splits_of(M, (K + BM - 1) / BM, DA_PER_SM));  /* dA^T partials */
 }
 
 pact_status pact_lora_bwd(const pact_lora_bwd_t *g, void *workspace, size_t ws_bytes, pact_stream_t stream) {
@@ -623,11 +629,11 @@ pact_status pact_lora_bwd(const pact_lora_bwd_t *g, void *workspace, size_t ws_b
     cudaStream_t st = (cudaStream_t)stream;
     uint8_t *w8 = static_cast<uint8_t *>(workspace);
     float *ws_t = reinterpret_cast<float *>(w8);
-    w8 += partial_bytes(M, R, splits_of(K, (M + BM - 1) / BM));
+    w8 += partial_bytes(M, R, splits_of(K, (M + BM - 1) / BM, T_PER_SM));
     pact_bf16 *tt = reinterpret_cast<pact_bf16 *>(w8);
     w8 += round256((size_t)(M * 2 * R * 2));
     float *ws_db = reinterpret_cast<float *>(w8);
-    w8 += partial_bytes(N, r, splits_of(M, (N + BM - 1) / BM));
+    w8 += partial_bytes(N, r, splits_of(M, (N + BM - 1) / BM, ctas_per_sm(2, false)));
     float *ws_da = reinterpret_cast<float *>(w8);
 
     // X~ is read where it lies: BF16 rows, or the saved NVFP4 copy decoded in shared
@@ -659,7 +665,7 @@ pact_status pact_lora_bwd(const pact_lora_bwd_t *g, void *workspace, size_t ws_b
         }
         pb.b_split = 1;
         pb.b_lo_off = R;
-        choose_split(M, blocks, &pb.splits, &pb.k_per_split);
+        choose_split(M, blocks, ctas_per_sm(2, false), &pb.splits, &pb.k_per_split);
         pb.ws = ws_db;
         pb.ws_ld = r;
         pb.ws_split_stride = N * r;
@@ -680,7 +686,7 @@ pact_status pact_lora_bwd(const pact_lora_bwd_t *g, void *workspace, size_t ws_b
     p.b_split = 1;
     p.b_lo_off = R;
     const int tiles = (int)((K + BM - 1) / BM);
-    choose_split(M, tiles, &p.splits, &p.k_per_split);
+    choose_split(M, tiles, ctas_per_sm(2, g->xq != nullptr), &p.splits, &p.k_per_split);
     p.ws = ws_da;
     p.ws_ld = R;
     p.ws_split_stride = K * R;

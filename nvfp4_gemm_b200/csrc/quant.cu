@@ -103,24 +103,16 @@ static int grid_for(int64_t warp_tasks, int threads) {
 }
 
 // ------------------------------------------------------- A3: RMSNorm + quantize
-// A group of WPR warps owns a row (256 / 32 / WPR rows per 256-thread CTA); warp w of
-// the group holds chunks w, w + WPR, ... of the row as packed BF16 between the
-// reduction and the output pass.  One warp per row when H <= 2048, so the row's
-// loads are all in flight at once and the reduction needs no block barrier.
-constexpr int RMS_THREADS = 256;
-constexpr int RMS_WARPS = RMS_THREADS / 32;
-constexpr int RMS_MAX_CHUNKS = 8;  // H <= 8 warps x 8 chunks x 256 = 16384
-
-// Warps per row for H columns: the fewest (1, 2, 4 or 8) whose chunks fit in 8 each.
-static int rms_wpr(int64_t H) {
-    const int64_t chunks = (H + CHUNK - 1) / CHUNK;
-    return chunks <= 8 ? 1 : chunks <= 16 ? 2 : chunks <= 32 ? 4 : 8;
-}
-// Chunks each warp holds: 1, 2, 4 or 8.
-static int rms_nch(int64_t H) {
-    const int64_t per_warp = ((H + CHUNK - 1) / CHUNK + rms_wpr(H) - 1) / rms_wpr(H);
-    return per_warp <= 1 ? 1 : per_warp <= 2 ? 2 : per_warp <= 4 ? 4 : 8;
-}
+// A CTA of 4 warps works through rows blockIdx.x, blockIdx.x + gridDim.x, ... (and
+// the padding rows of the scale layout).  Whole rows stream into a ring of shared-
+// memory slots by bulk copies issued `stages` rows ahead, so the next rows are in
+// flight while the current one is reduced and written: the row's sum of squares
+// (warp w takes 256-column chunks w, w + 4, ...; FP64 partial sums, reduced across the
+// CTA), then y = BF16(x * rstd * gamma) and its NVFP4 copy, read again from shared
+// memory.
+constexpr int RING_THREADS = 128;
+constexpr int RING_WARPS = RING_THREADS / 32;
+constexpr int RMS_MAX_H = 16384;
 
 // BF16 rounding of y = (x * rstd) * gamma with one correct rounding of the double
 // expression: the FP32 evaluation decides unless it lies within 64 FP32 ulps of a
@@ -137,63 +129,111 @@ __device__ __forceinline__ float rms_out(float x, float g, float r32, double rst
     return __bfloat162float(__float2bfloat16_rn(y));
 }
 
-template <int NCH, int WPR>
-__global__ void __launch_bounds__(RMS_THREADS, 2) k_rmsnorm_quant(const pact_bf16 *__restrict__ x, int64_t ldx,
+// Ring geometry: slots of `slot_bytes`, as many (2 .. 4) as fit in ~48 KiB, and CTAs
+// per SM so that a few hundred KiB... of shared memory per SM are in use.
+struct Ring {
+    int stages;
+    size_t slot_bytes, smem;
+    int grid;
+};
+static Ring ring_for(int64_t rows, size_t slot_bytes) {
+    Ring r;
+    r.slot_bytes = (slot_bytes + 127) & ~(size_t)127;
+    r.stages = (int)(49152 / r.slot_bytes);
+    r.stages = r.stages < 2 ? 2 : (r.stages > 4 ? 4 : r.stages);
+    r.smem = r.stages * r.slot_bytes + 64;
+    int per_sm = (int)(200 * 1024 / r.smem);
+    per_sm = per_sm < 1 ? 1 : (per_sm > 8 ? 8 : per_sm);
+    const int64_t g = (int64_t)sm_count() * per_sm;
+    r.grid = (int)(rows < g ? rows : g);
+    return r;
+}
+
+__global__ void __launch_bounds__(RING_THREADS) k_rmsnorm_quant(const pact_bf16 *__restrict__ x, int64_t ldx,
                                                                const pact_bf16 *__restrict__ gamma, float eps,
                                                                int64_t M, int64_t H, pact_nvfp4_t yq,
-                                                               pact_bf16 *__restrict__ y, float *__restrict__ rstd_out) {
-    pdl_wait();
-    __shared__ double red[RMS_WARPS];
+                                                               pact_bf16 *__restrict__ y, float *__restrict__ rstd_out,
+                                                               int stages, int slot_bytes) {
+    extern __shared__ __align__(128) uint8_t ring[];
+    uint64_t *full = reinterpret_cast<uint64_t *>(ring + stages * slot_bytes);
+    __shared__ double red[RING_WARPS];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const int wr = warp % WPR;                                       // warp within the row group
-    const int64_t row = (int64_t)blockIdx.x * (RMS_WARPS / WPR) + warp / WPR;
-    const bool real = row < M;                                       // else a padding row of the scale layout
-    uint4 xv[NCH];
-    double ss = 0.0;
-#pragma unroll
-    for (int k = 0; k < NCH; ++k) {
-        const int64_t c = (wr + (int64_t)k * WPR) * CHUNK + 8 * lane;
-        xv[k] = make_uint4(0, 0, 0, 0);
-        if (real && c < H) xv[k] = *reinterpret_cast<const uint4 *>(x + row * ldx + c);
+    const int64_t rows_pad = (M + 127) & ~int64_t(127);
+    const int nchunk = (int)((H + CHUNK - 1) / CHUNK);
+    const uint32_t row_bytes = (uint32_t)(H * 2);
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < stages; ++i) mbar_init(&full[i], 1);
+        fence_barrier_init();
     }
-#pragma unroll
-    for (int k = 0; k < NCH; ++k) {
-        float v[8];
-        unpack8_bf16(xv[k], v);
-#pragma unroll
-        for (int i = 0; i < 8; ++i) ss = fma((double)v[i], (double)v[i], ss);
-    }
-#pragma unroll
-    for (int o = 16; o; o >>= 1) ss += __shfl_xor_sync(0xFFFFFFFFu, ss, o);
-    if (WPR > 1) {
-        if (lane == 0) red[warp] = ss;
-        __syncthreads();
-        ss = 0.0;
-#pragma unroll
-        for (int w = 0; w < WPR; ++w) ss += red[warp - wr + w];
-    }
-    const double rstd = 1.0 / sqrt(ss / (double)H + (double)eps);
-    const float r32 = (float)rstd;
-    if (real && wr == 0 && lane == 0 && rstd_out) rstd_out[row] = r32;
-#pragma unroll
-    for (int k = 0; k < NCH; ++k) {
-        const int64_t c0 = (wr + (int64_t)k * WPR) * CHUNK;
-        if (c0 >= H) break;  // warp-uniform
-        if (!real) {
-            zero_pad_scales(yq, row, c0);
+    __syncthreads();
+    pdl_wait();
+    auto issue = [&](int i) {   // thread 0: row i of this CTA into its slot
+        const int64_t r = blockIdx.x + (int64_t)i * gridDim.x;
+        if (r < M) {
+            mbar_arrive_expect_tx(&full[i % stages], row_bytes);
+            bulk_load(ring + (i % stages) * slot_bytes, x + r * ldx, row_bytes, &full[i % stages]);
+        }
+    };
+    if (threadIdx.x == 0)
+        for (int i = 0; i < stages; ++i) issue(i);
+    bool ok = true;
+    int i = 0;
+    for (int64_t row = blockIdx.x; row < rows_pad; row += gridDim.x, ++i) {
+        const int slot = i % stages;
+        if (row >= M) {   // a padding row of the scale layout: zero scales (block-uniform)
+            for (int k = warp; k < nchunk; k += RING_WARPS) zero_pad_scales(yq, row, (int64_t)k * CHUNK);
             continue;
         }
-        const int64_t c = c0 + 8 * lane;
-        const bool valid = c < H;
-        float v[8], g[8] = {0, 0, 0, 0, 0, 0, 0, 0}, o[8];
-        unpack8_bf16(xv[k], v);
-        if (valid) load8_bf16(gamma + c, g);
+        ok = __syncthreads_and(ok && mbar_wait(&full[slot], (uint32_t)(i / stages) & 1u));
+        if (!ok) break;
+        const uint8_t *rs = ring + slot * slot_bytes;
+        double s0 = 0.0, s1 = 0.0;
+        for (int k = warp; k < nchunk; k += RING_WARPS) {
+            const int c = k * CHUNK + 8 * lane;
+            if (c < H) {
+                float v[8];
+                load8_bf16(reinterpret_cast<const pact_bf16 *>(rs) + c, v);
 #pragma unroll
-        for (int i = 0; i < 8; ++i) o[i] = valid ? rms_out(v[i], g[i], r32, rstd) : 0.0f;
-        if (valid && y) store8_bf16(y + row * H + c, o);
-        uint32_t sb;
-        const uint32_t codes = quant8(o, &sb);
-        store_chunk(yq, row, c0, codes, sb, valid);
+                for (int j = 0; j < 8; j += 2) {
+                    s0 = fma((double)v[j], (double)v[j], s0);
+                    s1 = fma((double)v[j + 1], (double)v[j + 1], s1);
+                }
+            }
+        }
+        double ss = s0 + s1;
+#pragma unroll
+        for (int o = 16; o; o >>= 1) ss += __shfl_xor_sync(0xFFFFFFFFu, ss, o);
+        if (lane == 0) red[warp] = ss;
+        __syncthreads();
+        ss = (red[0] + red[1]) + (red[2] + red[3]);
+        const double rstd = 1.0 / sqrt(ss / (double)H + (double)eps);
+        const float r32 = (float)rstd;
+        if (threadIdx.x == 0 && rstd_out) rstd_out[row] = r32;
+        for (int k = warp; k < nchunk; k += RING_WARPS) {
+            const int64_t c0 = (int64_t)k * CHUNK;
+            const int64_t c = c0 + 8 * lane;
+            const bool valid = c < H;
+            float v[8] = {0, 0, 0, 0, 0, 0, 0, 0}, g[8] = {0, 0, 0, 0, 0, 0, 0, 0}, o[8];
+            if (valid) {
+                load8_bf16(reinterpret_cast<const pact_bf16 *>(rs) + c, v);
+                load8_bf16(gamma + c, g);
+            }
+#pragma unroll
+            for (int j = 0; j < 8; ++j) o[j] = valid ? rms_out(v[j], g[j], r32, rstd) : 0.0f;
+            if (valid && y) store8_bf16(y + row * H + c, o);
+            uint32_t sb;
+            const uint32_t codes = quant8(o, &sb);
+            store_chunk(yq, row, c0, codes, sb, valid);
+        }
+        __syncthreads();                      // every thread is done with the slot and with red
+        if (threadIdx.x == 0) issue(i + stages);
+    }
+    // copies still in flight land before the CTA leaves (bounded waits)
+    if (threadIdx.x == 0) {
+        for (int j = i; j < i + stages; ++j) {
+            const int64_t r = blockIdx.x + (int64_t)j * gridDim.x;
+            if (r < M) mbar_wait(&full[j % stages], (uint32_t)(j / stages) & 1u);
+        }
     }
 }
 
@@ -365,83 +405,117 @@ __global__ void __launch_bounds__(256) k_silu_mul_bwd_quant(const pact_bf16 *__r
 }
 
 // ------------------------------------------------------- A10: RMSNorm backward
-// Same row groups as the forward; dy stays packed BF16 and y^ stays NVFP4 (codes and
-// scale byte) in registers between the reduction and the output pass.
-template <int NCH, int WPR>
-__global__ void __launch_bounds__(RMS_THREADS, 2) k_rmsnorm_bwd(const pact_bf16 *__restrict__ dy, int64_t lddy,
+// The ring of the forward kernel, with a slot holding a row of dy, the row's NVFP4
+// codes of y^ and (when given) a row of the residual gradient dres.  Pass 1 forms
+// sum(dy * y^) (the row's scale bytes come from global memory, L1-resident after the
+// first pass); pass 2 writes dx and, when asked, its NVFP4 copy.
+struct BwdSlot {
+    int codes_off, dres_off;
+};
+__host__ __device__ inline BwdSlot bwd_slot(int64_t H) {
+    const int dy_bytes = (int)(H * 2), code_bytes = (int)(H / 2);
+    BwdSlot b;
+    b.codes_off = (dy_bytes + 127) & ~127;
+    b.dres_off = (b.codes_off + code_bytes + 127) & ~127;
+    return b;
+}
+
+__global__ void __launch_bounds__(RING_THREADS) k_rmsnorm_bwd(const pact_bf16 *__restrict__ dy, int64_t lddy,
                                                              pact_nvfp4_t yq, const float *__restrict__ rstd,
                                                              const pact_bf16 *__restrict__ gamma, int64_t M, int64_t H,
                                                              const pact_bf16 *__restrict__ dres,
-                                                             pact_bf16 *__restrict__ dx, pact_nvfp4_t dxq, int has_dxq) {
-    pdl_wait();
-    __shared__ float red[RMS_WARPS];
+                                                             pact_bf16 *__restrict__ dx, pact_nvfp4_t dxq, int has_dxq,
+                                                             int stages, int slot_bytes) {
+    extern __shared__ __align__(128) uint8_t ring[];
+    uint64_t *full = reinterpret_cast<uint64_t *>(ring + stages * slot_bytes);
+    __shared__ float red[RING_WARPS];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const int wr = warp % WPR;
-    const int64_t row = (int64_t)blockIdx.x * (RMS_WARPS / WPR) + warp / WPR;
-    const bool real = row < M;
-    uint4 dv[NCH];
-    uint32_t yc[NCH], ys[NCH];
-    float dot = 0.0f;
-#pragma unroll
-    for (int k = 0; k < NCH; ++k) {
-        const int64_t c = (wr + (int64_t)k * WPR) * CHUNK + 8 * lane;
-        dv[k] = make_uint4(0, 0, 0, 0);
-        yc[k] = 0;
-        ys[k] = 0;
-        if (real && c < H) {
-            dv[k] = *reinterpret_cast<const uint4 *>(dy + row * lddy + c);
-            yc[k] = *reinterpret_cast<const uint32_t *>(static_cast<const uint8_t *>(yq.codes) + row * (H >> 1) +
-                                                         (c >> 1));
-            ys[k] = static_cast<const uint8_t *>(yq.scales)[scale_offset(row, c >> 4, H)];
+    const int64_t rows = has_dxq ? (M + 127) & ~int64_t(127) : M;
+    const int nchunk = (int)((H + CHUNK - 1) / CHUNK);
+    const BwdSlot sl = bwd_slot(H);
+    const uint32_t dy_bytes = (uint32_t)(H * 2), code_bytes = (uint32_t)(H / 2);
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < stages; ++i) mbar_init(&full[i], 1);
+        fence_barrier_init();
+    }
+    __syncthreads();
+    pdl_wait();
+    auto issue = [&](int i) {   // thread 0: row i of this CTA into its slot
+        const int64_t r = blockIdx.x + (int64_t)i * gridDim.x;
+        if (r < M) {
+            uint8_t *slot = ring + (i % stages) * slot_bytes;
+            uint64_t *bar = &full[i % stages];
+            mbar_arrive_expect_tx(bar, dy_bytes + code_bytes + (dres ? dy_bytes : 0u));
+            bulk_load(slot, dy + r * lddy, dy_bytes, bar);
+            bulk_load(slot + sl.codes_off, static_cast<const uint8_t *>(yq.codes) + r * (H / 2), code_bytes, bar);
+            if (dres) bulk_load(slot + sl.dres_off, dres + r * H, dy_bytes, bar);
         }
-    }
-#pragma unroll
-    for (int k = 0; k < NCH; ++k) {
-        float d[8], yv[8];
-        unpack8_bf16(dv[k], d);
-        dequant8(yc[k], ys[k], yv);
-        // (gamma * dy) * (y^ / gamma) == dy * y^
-#pragma unroll
-        for (int i = 0; i < 8; ++i) dot = fmaf(d[i], yv[i], dot);
-    }
-#pragma unroll
-    for (int o = 16; o; o >>= 1) dot += __shfl_xor_sync(0xFFFFFFFFu, dot, o);
-    if (WPR > 1) {
-        if (lane == 0) red[warp] = dot;
-        __syncthreads();
-        dot = 0.0f;
-#pragma unroll
-        for (int w = 0; w < WPR; ++w) dot += red[warp - wr + w];
-    }
-    const float mean = dot / (float)H;
-    const float r = real ? rstd[row] : 0.0f;
-#pragma unroll
-    for (int k = 0; k < NCH; ++k) {
-        const int64_t c0 = (wr + (int64_t)k * WPR) * CHUNK;
-        if (c0 >= H) break;
-        if (!real) {
-            if (has_dxq) zero_pad_scales(dxq, row, c0);
+    };
+    if (threadIdx.x == 0)
+        for (int i = 0; i < stages; ++i) issue(i);
+    bool ok = true;
+    int i = 0;
+    for (int64_t row = blockIdx.x; row < rows; row += gridDim.x, ++i) {
+        const int slot = i % stages;
+        if (row >= M) {   // padding row of dxq's scale layout (block-uniform)
+            for (int k = warp; k < nchunk; k += RING_WARPS) zero_pad_scales(dxq, row, (int64_t)k * CHUNK);
             continue;
         }
-        const int64_t c = c0 + 8 * lane;
-        const bool valid = c < H;
-        float d[8], yv[8], g[8] = {1, 1, 1, 1, 1, 1, 1, 1}, res[8] = {0, 0, 0, 0, 0, 0, 0, 0}, o[8];
-        unpack8_bf16(dv[k], d);
-        dequant8(yc[k], ys[k], yv);
-        if (valid) {
-            load8_bf16(gamma + c, g);
-            if (dres) load8_bf16(dres + row * H + c, res);
+        ok = __syncthreads_and(ok && mbar_wait(&full[slot], (uint32_t)(i / stages) & 1u));
+        if (!ok) break;
+        const uint8_t *rs = ring + slot * slot_bytes;
+        const pact_bf16 *dys = reinterpret_cast<const pact_bf16 *>(rs);
+        const uint8_t *cs = rs + sl.codes_off;
+        const pact_bf16 *rrs = reinterpret_cast<const pact_bf16 *>(rs + sl.dres_off);
+        const uint8_t *ysc = static_cast<const uint8_t *>(yq.scales);
+        float dot = 0.0f;
+        for (int k = warp; k < nchunk; k += RING_WARPS) {
+            const int c = k * CHUNK + 8 * lane;
+            if (c < H) {
+                float d[8], yv[8];
+                load8_bf16(dys + c, d);
+                dequant8(*reinterpret_cast<const uint32_t *>(cs + c / 2), ysc[scale_offset(row, c >> 4, H)], yv);
+                // (gamma * dy) * (y^ / gamma) == dy * y^
+#pragma unroll
+                for (int j = 0; j < 8; ++j) dot = fmaf(d[j], yv[j], dot);
+            }
         }
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            const float val = r * (g[i] * d[i] - __fdividef(yv[i], g[i]) * mean) + res[i];
-            o[i] = valid ? __bfloat162float(__float2bfloat16_rn(val)) : 0.0f;
+        for (int o = 16; o; o >>= 1) dot += __shfl_xor_sync(0xFFFFFFFFu, dot, o);
+        if (lane == 0) red[warp] = dot;
+        __syncthreads();
+        const float mean = ((red[0] + red[1]) + (red[2] + red[3])) / (float)H;
+        const float r = rstd[row];
+        for (int k = warp; k < nchunk; k += RING_WARPS) {
+            const int64_t c0 = (int64_t)k * CHUNK;
+            const int64_t c = c0 + 8 * lane;
+            const bool valid = c < H;
+            float d[8], yv[8], g[8] = {1, 1, 1, 1, 1, 1, 1, 1}, res[8] = {0, 0, 0, 0, 0, 0, 0, 0}, o[8];
+            if (valid) {
+                load8_bf16(dys + c, d);
+                dequant8(*reinterpret_cast<const uint32_t *>(cs + c / 2), ysc[scale_offset(row, c >> 4, H)], yv);
+                load8_bf16(gamma + c, g);
+                if (dres) load8_bf16(rrs + c, res);
+            }
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                const float val = r * (g[j] * d[j] - __fdividef(yv[j], g[j]) * mean) + res[j];
+                o[j] = valid ? __bfloat162float(__float2bfloat16_rn(val)) : 0.0f;
+            }
+            if (valid) store8_bf16(dx + row * H + c, o);
+            if (has_dxq) {
+                uint32_t sb;
+                const uint32_t codes = quant8(o, &sb);
+                store_chunk(dxq, row, c0, codes, sb, valid);
+            }
         }
-        if (valid) store8_bf16(dx + row * H + c, o);
-        if (has_dxq) {
-            uint32_t sb;
-            const uint32_t codes = quant8(o, &sb);
-            store_chunk(dxq, row, c0, codes, sb, valid);
+        __syncthreads();
+        if (threadIdx.x == 0) issue(i + stages);
+    }
+    if (threadIdx.x == 0) {
+        for (int j = i; j < i + stages; ++j) {
+            const int64_t r = blockIdx.x + (int64_t)j * gridDim.x;
+            if (r < M) mbar_wait(&full[j % stages], (uint32_t)(j / stages) & 1u);
         }
     }
 }
@@ -586,7 +660,7 @@ int pact_two_level_exponent(float amax) {
 pact_status pact_rmsnorm_quant(const pact_bf16 *x, int64_t ldx, const pact_bf16 *gamma, float eps, int64_t M,
                                int64_t H, const pact_nvfp4_t *yq, pact_bf16 *y, float *rstd, pact_stream_t stream) {
     PACT_CHECK(x && gamma && yq, PACT_ERR_INVALID_ARG, "pact_rmsnorm_quant: NULL argument");
-    PACT_CHECK(M >= 1 && H >= 64 && H % 64 == 0 && H <= RMS_WARPS * RMS_MAX_CHUNKS * CHUNK, PACT_ERR_SHAPE,
+    PACT_CHECK(M >= 1 && H >= 64 && H % 64 == 0 && H <= RMS_MAX_H, PACT_ERR_SHAPE,
                "pact_rmsnorm_quant: M >= 1, H a multiple of 64 in [64, 16384] required (M=%lld H=%lld)",
                (long long)M, (long long)H);
     PACT_CHECK(!(eps < 0.0f) && isfinite(eps), PACT_ERR_INVALID_ARG, "pact_rmsnorm_quant: eps must be finite and >= 0");
@@ -596,28 +670,16 @@ pact_status pact_rmsnorm_quant(const pact_bf16 *x, int64_t ldx, const pact_bf16 
     if (s != PACT_OK) return s;
     const int64_t rows_pad = (M + 127) / 128 * 128;
     PACT_CHECK(rows_pad <= 0x7FFFFFFF, PACT_ERR_SHAPE, "pact_rmsnorm_quant: M too large");
-    cudaStream_t st = (cudaStream_t)stream;
-    const int wpr = rms_wpr(H), nch = rms_nch(H);
-    const unsigned grid = (unsigned)(rows_pad / (RMS_WARPS / wpr));
-#define PACT_RMS_FWD(NC, WP) \
-    s = launch_dep(k_rmsnorm_quant<NC, WP>, dim3(grid), dim3(RMS_THREADS), 0, st, "pact_rmsnorm_quant", x, ldx, gamma, eps, \
-                   M, H, *yq, y, rstd)
-    if (wpr == 1) {
-        switch (nch) {
-            case 1: PACT_RMS_FWD(1, 1); break;
-            case 2: PACT_RMS_FWD(2, 1); break;
-            case 4: PACT_RMS_FWD(4, 1); break;
-            default: PACT_RMS_FWD(8, 1); break;
-        }
-    } else if (wpr == 2) {
-        PACT_RMS_FWD(8, 2);
-    } else if (wpr == 4) {
-        PACT_RMS_FWD(8, 4);
-    } else {
-        PACT_RMS_FWD(8, 8);
+    const Ring r = ring_for(rows_pad, (size_t)H * 2);
+    static bool attr_done[64] = {false};
+    const int d = current_device();
+    if (d >= 0 && d < 64 && !attr_done[d]) {
+        const cudaError_t e = cudaFuncSetAttribute(k_rmsnorm_quant, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
+        if (e != cudaSuccess) return fail(PACT_ERR_CUDA, "pact_rmsnorm_quant: %s", cudaGetErrorString(e));
+        attr_done[d] = true;
     }
-#undef PACT_RMS_FWD
-    return s;
+    return launch_dep(k_rmsnorm_quant, dim3(r.grid), dim3(RING_THREADS), r.smem, (cudaStream_t)stream,
+                      "pact_rmsnorm_quant", x, ldx, gamma, eps, M, H, *yq, y, rstd, r.stages, (int)r.slot_bytes);
 }
 
 pact_status pact_silu_mul_quant(const pact_bf16 *g, const pact_bf16 *u, int64_t ld_gu, int64_t M, int64_t I,
@@ -661,7 +723,7 @@ pact_status pact_rmsnorm_bwd(const pact_bf16 *dy, int64_t lddy, const pact_nvfp4
                              const pact_bf16 *gamma, int64_t M, int64_t H, const pact_bf16 *dres, pact_bf16 *dx,
                              const pact_nvfp4_t *dxq, pact_stream_t stream) {
     PACT_CHECK(dy && yq && rstd && gamma && dx, PACT_ERR_INVALID_ARG, "pact_rmsnorm_bwd: NULL argument");
-    PACT_CHECK(M >= 1 && H >= 64 && H % 64 == 0 && H <= RMS_WARPS * RMS_MAX_CHUNKS * CHUNK, PACT_ERR_SHAPE,
+    PACT_CHECK(M >= 1 && H >= 64 && H % 64 == 0 && H <= RMS_MAX_H, PACT_ERR_SHAPE,
                "pact_rmsnorm_bwd: M >= 1, H a multiple of 64 in [64, 16384] required");
     PACT_CHECK(lddy >= H && lddy % 8 == 0 && aligned16(dy) && aligned16(gamma) && aligned16(dx) && aligned16(dres),
                PACT_ERR_ALIGN, "pact_rmsnorm_bwd: pointers must be 16-byte aligned, lddy %% 8 == 0");
@@ -670,31 +732,19 @@ pact_status pact_rmsnorm_bwd(const pact_bf16 *dy, int64_t lddy, const pact_nvfp4
     if (s != PACT_OK) return s;
     pact_nvfp4_t none = {nullptr, nullptr, M, H};
     const int64_t rows = dxq ? (M + 127) / 128 * 128 : M;
-    cudaStream_t st = (cudaStream_t)stream;
-    const pact_nvfp4_t q = dxq ? *dxq : none;
-    const int has = dxq != nullptr;
-    const int wpr = rms_wpr(H), nch = rms_nch(H);
-    const int64_t per_cta = RMS_WARPS / wpr;
-    const unsigned grid = (unsigned)((rows + per_cta - 1) / per_cta);
-#define PACT_RMS_BWD(NC, WP) \
-    s = launch_dep(k_rmsnorm_bwd<NC, WP>, dim3(grid), dim3(RMS_THREADS), 0, st, "pact_rmsnorm_bwd", dy, lddy, *yq, rstd, \
-                   gamma, M, H, dres, dx, q, has)
-    if (wpr == 1) {
-        switch (nch) {
-            case 1: PACT_RMS_BWD(1, 1); break;
-            case 2: PACT_RMS_BWD(2, 1); break;
-            case 4: PACT_RMS_BWD(4, 1); break;
-            default: PACT_RMS_BWD(8, 1); break;
-        }
-    } else if (wpr == 2) {
-        PACT_RMS_BWD(8, 2);
-    } else if (wpr == 4) {
-        PACT_RMS_BWD(8, 4);
-    } else {
-        PACT_RMS_BWD(8, 8);
+    PACT_CHECK(rows <= 0x7FFFFFFF, PACT_ERR_SHAPE, "pact_rmsnorm_bwd: M too large");
+    const BwdSlot sl = bwd_slot(H);
+    const Ring r = ring_for(rows, (size_t)(dres ? sl.dres_off + H * 2 : sl.codes_off + H / 2));
+    static bool attr_done[64] = {false};
+    const int d = current_device();
+    if (d >= 0 && d < 64 && !attr_done[d]) {
+        const cudaError_t e = cudaFuncSetAttribute(k_rmsnorm_bwd, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
+        if (e != cudaSuccess) return fail(PACT_ERR_CUDA, "pact_rmsnorm_bwd: %s", cudaGetErrorString(e));
+        attr_done[d] = true;
     }
-#undef PACT_RMS_BWD
-    return s;
+    return launch_dep(k_rmsnorm_bwd, dim3(r.grid), dim3(RING_THREADS), r.smem, (cudaStream_t)stream, "pact_rmsnorm_bwd",
+                      dy, lddy, *yq, rstd, gamma, M, H, dres, dx, dxq ? *dxq : none, (int)(dxq != nullptr), r.stages,
+                      (int)r.slot_bytes);
 }
 
 pact_status pact_weight_layout_cache(const pact_bf16 *W, int64_t ldw, int64_t N, int64_t K, void *buf, size_t bytes,

@@ -17,3 +17,12 @@ def orc():
     import oracle
     oracle.build()
     return oracle
+
+
+@pytest.fixture
+def guards():
+    """Output buffers with canary guard bands (tests.util.Guards), checked after the test."""
+    from tests.util import Guards
+    g = Guards()
+    yield g
+    g.check()

@@ -72,10 +72,10 @@ def test_quantize_all_elements(P, orc):
 
 @pytest.mark.parametrize("rows,cols,ld", [(1, 64, 64), (200, 320, 320), (300, 1024, 1088), (128, 256, 256),
                                           (2048, 2048, 2048)])
-def test_quantize_shapes(P, orc, rows, cols, ld):
+def test_quantize_shapes(P, orc, guards, rows, cols, ld):
     x = synth.gaussian_bf16(1, (rows, ld), std=2.0)
     xd = to_dev(x)[:, :cols]
-    dev = P.pact_quantize_nvfp4(xd)
+    dev = P.pact_quantize_nvfp4(xd, out=guards.nvfp4(rows, cols))
     sync()
     assert_nvfp4_equal(dev, orc.quantize(x[:, :cols]), orc, f"quantize {rows}x{cols}")
 
@@ -128,12 +128,12 @@ GEMM_SHAPES = [(256, 512, 512), (300, 640, 576), (128, 256, 64), (1, 320, 448), 
 
 
 @pytest.mark.parametrize("M,N,K", GEMM_SHAPES)
-def test_gemm_fwd(P, orc, M, N, K):
+def test_gemm_fwd(P, orc, guards, M, N, K):
     x = synth.gaussian_bf16(1, (M, K))
     w = synth.weight_bf16(0, (N, K))
     wc = P.pact_weight_layout_cache(to_dev(w))
     xq = P.pact_quantize_nvfp4(to_dev(x))
-    y = P.pact_frozen_gemm_fwd(xq, wc)
+    y = P.pact_frozen_gemm_fwd(xq, wc, y=guards.matrix(M, N, pad_cols=8))
     sync()
     status_ok(P)
     wf, _ = orc.weight_cache(w)
@@ -141,24 +141,25 @@ def test_gemm_fwd(P, orc, M, N, K):
 
 
 @pytest.mark.parametrize("M,N,K", GEMM_SHAPES)
-def test_gemm_dgrad(P, orc, M, N, K):
+def test_gemm_dgrad(P, orc, guards, M, N, K):
     dy = synth.gaussian_bf16(50, (M, N))
     w = synth.weight_bf16(0, (N, K))
     wc = P.pact_weight_layout_cache(to_dev(w))
     dyq = P.pact_quantize_nvfp4(to_dev(dy))
-    dx = P.pact_frozen_gemm_dgrad(dyq, wc)
+    dx = P.pact_frozen_gemm_dgrad(dyq, wc, dx=guards.matrix(M, K, pad_cols=16))
     sync()
     _, wb = orc.weight_cache(w)
     assert_close(to_f64(dx), orc.frozen_dgrad(dy, wb), "dgrad")
 
 
-def test_gemm_fwd_residual(P, orc):
+def test_gemm_fwd_residual(P, orc, guards):
     M, N, K = 300, 768, 512
     x = synth.gaussian_bf16(1, (M, K))
     res = synth.gaussian_bf16(2, (M, N))
     w = synth.weight_bf16(0, (N, K))
     wc = P.pact_weight_layout_cache(to_dev(w))
-    y = P.pact_frozen_gemm_fwd(P.pact_quantize_nvfp4(to_dev(x)), wc, residual=to_dev(res))
+    y = P.pact_frozen_gemm_fwd(P.pact_quantize_nvfp4(to_dev(x)), wc, residual=to_dev(res),
+                               y=guards.matrix(M, N, pad_cols=64))
     sync()
     wf, _ = orc.weight_cache(w)
     assert_close(to_f64(y), orc.nvfp4_gemm(orc.quantize(x), wf) + synth.bf16_bits_to_f64(res), "fwd + residual")
@@ -239,7 +240,7 @@ def test_gemm_dgrad_lora(P, orc, M, N, K, R):
 # ------------------------------------------------------------------------- LoRA
 @pytest.mark.parametrize("M,parts,r,K", [(256, [512], 16, 384), (300, [512, 256, 256], 16, 576),
                                          (130, [256, 320], 32, 320), (2048, [1024], 16, 2112)])
-def test_lora_bwd(P, orc, M, parts, r, K):
+def test_lora_bwd(P, orc, guards, M, parts, r, K):
     """dA and dB from BF16 X and from the NVFP4 copy of X (decoded inside the MMA
     kernel); K values that end mid-way through a 128-feature tile and token counts
     that end mid-way through a 128-token scale group cover the ragged edges."""
@@ -252,10 +253,11 @@ def test_lora_bwd(P, orc, M, parts, r, K):
     b = synth.gaussian_bf16(30, (N, r), std=0.02)
     s = 2.0
     dyd, xd, ad, bd = to_dev(dy), to_dev(x), to_dev(a), to_dev(b)
-    U = P.pact_lora_bwd_u(dyd, bd, r, seg_end, s)
-    dA, dB = P.pact_lora_bwd(dyd, ad, U, r, seg_end, s, x=xd)
+    U = P.pact_lora_bwd_u(dyd, bd, r, seg_end, s, U=guards.matrix(M, 2 * nseg * r, pad_cols=8))
+    dA, dB = P.pact_lora_bwd(dyd, ad, U, r, seg_end, s, x=xd, dA=guards.matrix(nseg * r, K), dB=guards.matrix(N, r))
     xq = P.pact_quantize_nvfp4(xd)
-    dA2, dB2 = P.pact_lora_bwd(dyd, ad, U, r, seg_end, s, xq=xq)
+    dA2, dB2 = P.pact_lora_bwd(dyd, ad, U, r, seg_end, s, xq=xq, dA=guards.matrix(nseg * r, K),
+                               dB=guards.matrix(N, r))
     # FP32 gradients (for a sum over replicas) round to the BF16 ones bit for bit
     dA3, dB3 = P.pact_lora_bwd(dyd, ad, U, r, seg_end, s, xq=xq, grads_fp32=True)
     sync()
@@ -286,10 +288,11 @@ def test_lora_bwd(P, orc, M, parts, r, K):
 
 # --------------------------------------------------------------- fused producers
 @pytest.mark.parametrize("M,H", [(64, 512), (257, 2048), (96, 3072), (33, 1536)])
-def test_rmsnorm_quant(P, orc, M, H):
+def test_rmsnorm_quant(P, orc, guards, M, H):
     x = synth.gaussian_bf16(1, (M, H))
     g = synth.gaussian_bf16(40, (H,), std=0.02, mean=1.0)
-    yq, y, rstd = P.pact_rmsnorm_quant(to_dev(x), to_dev(g), 1e-5)
+    yq, y, rstd = P.pact_rmsnorm_quant(to_dev(x), to_dev(g), 1e-5, yq=guards.nvfp4(M, H), y=guards.matrix(M, H),
+                                       rstd=guards.matrix(1, M, torch.float32)[0])
     sync()
     y_ref, yq_ref, rstd_ref = orc.rmsnorm_quant(x, g, 1e-5)
     yb = to_bits(y)
@@ -299,11 +302,12 @@ def test_rmsnorm_quant(P, orc, M, H):
 
 
 @pytest.mark.parametrize("M,I,std", [(64, 512, 2.0), (130, 8960, 2.0), (257, 2048, 2.0), (96, 2048, 9.0)])
-def test_silu_mul_quant(P, orc, M, I, std):
+def test_silu_mul_quant(P, orc, guards, M, I, std):
     # std 2 reaches both margins of the rounding check; std 9 also |g| > 16 (FP64 path)
     gu = synth.gaussian_bf16(4, (M, 2 * I), std=std)
     gud = to_dev(gu)
-    m, mq, gq, uq = P.pact_silu_mul_quant(gud[:, :I], gud[:, I:])
+    m, mq, gq, uq = P.pact_silu_mul_quant(gud[:, :I], gud[:, I:], m=guards.matrix(M, I), mq=guards.nvfp4(M, I),
+                                          gq=guards.nvfp4(M, I), uq=guards.nvfp4(M, I))
     sync()
     m_ref, mq_ref, gq_ref, uq_ref = orc.silu_mul_quant(gu[:, :I], gu[:, I:])
     mb = to_bits(m)
@@ -314,12 +318,13 @@ def test_silu_mul_quant(P, orc, M, I, std):
 
 
 @pytest.mark.parametrize("M,I,std", [(64, 512, 2.0), (130, 2048, 2.0), (96, 1024, 9.0)])
-def test_silu_mul_bwd_quant(P, orc, M, I, std):
+def test_silu_mul_bwd_quant(P, orc, guards, M, I, std):
     gu = synth.gaussian_bf16(4, (M, 2 * I), std=std)
     dm = synth.gaussian_bf16(56, (M, I))
     _, _, gq, uq = orc.silu_mul_quant(gu[:, :I], gu[:, I:])
     gqd, uqd = _nvfp4_from_oracle(P, gq, orc), _nvfp4_from_oracle(P, uq, orc)
-    dgu, dguq, m_re = P.pact_silu_mul_bwd_quant(to_dev(dm), gqd, uqd, want_m=True)
+    dgu, dguq, m_re = P.pact_silu_mul_bwd_quant(to_dev(dm), gqd, uqd, dgu=guards.matrix(M, 2 * I, pad_cols=64),
+                                                dguq=guards.nvfp4(M, 2 * I), m_re=guards.matrix(M, I))
     sync()
     dg_ref, du_ref = orc.silu_mul_bwd(synth.bf16_bits_to_f64(dm), gq, uq)
     dgu_dev = to_f64(dgu)
@@ -332,14 +337,14 @@ def test_silu_mul_bwd_quant(P, orc, M, I, std):
 
 
 @pytest.mark.parametrize("M,H,with_res", [(64, 512, False), (130, 2048, True), (33, 3072, True)])
-def test_rmsnorm_bwd(P, orc, M, H, with_res):
+def test_rmsnorm_bwd(P, orc, guards, M, H, with_res):
     x = synth.gaussian_bf16(1, (M, H))
     g = synth.gaussian_bf16(40, (H,), std=0.02, mean=1.0)
     dy = synth.gaussian_bf16(57, (M, H))
     res = synth.gaussian_bf16(58, (M, H))
     yq, _, rstd = P.pact_rmsnorm_quant(to_dev(x), to_dev(g), 1e-5)
     dx, dxq = P.pact_rmsnorm_bwd(to_dev(dy), yq, rstd, to_dev(g), dres=to_dev(res) if with_res else None,
-                                 want_q=True)
+                                 dx=guards.matrix(M, H), dxq=guards.nvfp4(M, H))
     sync()
     _, yq_ref, _ = orc.rmsnorm_quant(x, g, 1e-5)
     ref = orc.rmsnorm_bwd(synth.bf16_bits_to_f64(dy), yq_ref, rstd.cpu().numpy().astype(np.float64), g)
