@@ -210,6 +210,18 @@ PACT_API pact_status pact_frozen_gemm_fwd(const pact_nvfp4_t *xq, const pact_wei
                                           const pact_lora_t *lora, const pact_bf16 *residual, int64_t ldr,
                                           pact_bf16 *y, int64_t ldy, pact_stream_t stream);
 
+/* pact_frozen_gemm_fwd that also writes the NVFP4 copy of its output: y as above,
+ * and q(y) of the BF16-rounded y, split along the columns into nq (1 or 2) NVFP4
+ * tensors yq[0] (columns 0 .. yq[0].cols - 1) and yq[1] (the rest), each [M x cols_i],
+ * cols_i multiples of 64 adding up to N.  [METHOD] bullet 2: the gate and up
+ * projections' NVFP4 copies are what the backward keeps; quantizing them in the
+ * GEMM epilogue, where the output rows are in registers, saves the SiLU-multiply
+ * kernel two of its three quantizations. */
+PACT_API pact_status pact_frozen_gemm_fwd_quant(const pact_nvfp4_t *xq, const pact_weight_cache_t *w,
+                                                const pact_lora_t *lora, const pact_bf16 *residual, int64_t ldr,
+                                                pact_bf16 *y, int64_t ldy, const pact_nvfp4_t *yq, int nq,
+                                                pact_stream_t stream);
+
 /* ------------------------------------------------------ A6: dgrad GEMM */
 /* [METHOD] bullet 1 (input gradient) with [LORA]:
  *   dx[M x K] = BF16_RNE( residual + 2^g (deq(dyq) . deq(w->bwd)^T + U . A) )

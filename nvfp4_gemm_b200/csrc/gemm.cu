@@ -39,7 +39,7 @@
 //    shared-memory slab), rounds to BF16 into the slab and writes it with one TMA
 //    store, which also clips the ragged edges of the output.
 #include <cmath>
-#include "common.cuh"
+#include "quant.cuh"
 
 namespace pact {
 namespace gemm {
@@ -87,6 +87,12 @@ struct Params {
     int64_t seg_end[4];
     float out_scale;      // 2^gexp of the weight cache: scales the accumulator (exact)
     int n_fast;           // tile order: 1 = N tiles fastest (A streamed once), 0 = M tiles fastest
+    // optional NVFP4 copy of the BF16 output, split along N into nq (1 or 2) tensors:
+    // columns [0, q_split) into q[0], [q_split, N) into q[1]
+    int nq;
+    int q_split;
+    uint8_t *q_codes[2];
+    uint8_t *q_scales[2];
 };
 
 // Pair-tile coordinates of persistent tile index t.  Consecutive indices run at the
@@ -108,6 +114,27 @@ __device__ __forceinline__ int lora_segment(const Params &p, int n0) {
 #pragma unroll
     for (int i = 0; i < 3; ++i) s += (i + 1 < p.lora_nseg && n0 >= p.seg_end[i]) ? 1 : 0;
     return s;
+}
+
+// NVFP4 copy of one row's 64 output columns (the BF16-rounded values, 32 packed
+// words: columns 2j, 2j+1 in word j): four 16-value blocks quantized in this thread,
+// 32 code bytes and 4 scale bytes stored; rows past M in the 128-row padding of the
+// scale layout get zero scales.
+// Where a row's NVFP4 copy of 64 output columns goes: its codes (nullptr for rows
+// that get none) and its 4 scale bytes (nullptr past the 128-row padding).
+struct QDest {
+    uint8_t *codes, *scales;
+};
+__device__ __forceinline__ QDest qdest(const Params &p, int row, int col) {
+    QDest d = {nullptr, nullptr};
+    if (!p.nq || row >= ((p.M + 127) & ~127)) return d;
+    const int seg = (p.nq > 1 && col >= p.q_split) ? 1 : 0;
+    const int lc = col - (seg ? p.q_split : 0);
+    const int cols = seg ? p.N - p.q_split : (p.nq > 1 ? p.q_split : p.N);
+    // select, not index: a runtime index into the parameter arrays would copy them to local memory
+    d.scales = (seg ? p.q_scales[1] : p.q_scales[0]) + scale_offset(row, lc >> 4, cols);
+    if (row < p.M) d.codes = (seg ? p.q_codes[1] : p.q_codes[0]) + (int64_t)row * (cols >> 1) + (lc >> 1);
+    return d;
 }
 
 // Every stage of the ring is used in the same order by all roles: per tile, one LoRA
@@ -419,6 +446,11 @@ k_nvfp4_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CU
             __syncwarp();
             if (lane == 0) mbar_arrive_remote_relaxed(acc_empty_leader);  // the pair may reuse the accumulator
             acc_phase ^= 1;
+            if (p.nq && !inside(t) && block_x(t) < p.N) {
+                // a 32-row block wholly in the scale layout's padding rows: zero scales only
+                const QDest qd = qdest(p, block_y(t) + lane, block_x(t));
+                if (qd.scales) *reinterpret_cast<uint32_t *>(qd.scales) = 0u;
+            }
             if (inside(t)) {
                 if (p.has_res) {
                     if (lane == 0) got = mbar_wait_sleep(&res_full[ew], res_phase);
@@ -428,6 +460,10 @@ k_nvfp4_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CU
                     if (lane == 0) bulk_wait_read_all();  // the previous block's store has read the slab
                     __syncwarp();
                 }
+                // the NVFP4 copy of the block's rounded values: block b of this lane's row is
+                // quantized once its two 8-value pieces are rounded
+                const QDest qd = qdest(p, block_y(t) + lane, block_x(t));
+                uint32_t sbs = 0;
                 // row `lane` of the block: 8 pieces of 16 bytes, 128-byte swizzle
 #pragma unroll
                 for (int q = 0; q < 8; ++q) {
@@ -443,11 +479,22 @@ k_nvfp4_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CU
                         f[0] += bf16lo(o0); f[1] += bf16hi(o0); f[2] += bf16lo(o1); f[3] += bf16hi(o1);
                         f[4] += bf16lo(o2); f[5] += bf16hi(o2); f[6] += bf16lo(o3); f[7] += bf16hi(o3);
                     }
-                    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(a), "r"(pack_bf16x2(f[0], f[1])),
-                                 "r"(pack_bf16x2(f[2], f[3])), "r"(pack_bf16x2(f[4], f[5])),
-                                 "r"(pack_bf16x2(f[6], f[7]))
+                    const uint32_t w0 = pack_bf16x2(f[0], f[1]), w1 = pack_bf16x2(f[2], f[3]);
+                    const uint32_t w2 = pack_bf16x2(f[4], f[5]), w3 = pack_bf16x2(f[6], f[7]);
+                    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(a), "r"(w0), "r"(w1), "r"(w2),
+                                 "r"(w3)
                                  : "memory");
+                    // the rounded values, kept for the NVFP4 copy (r[] is free again)
+                    r[4 * q] = w0; r[4 * q + 1] = w1; r[4 * q + 2] = w2; r[4 * q + 3] = w3;
+                    if ((q & 1) && qd.codes) {
+                        uint32_t lo, hi, sb;
+                        quant16_bf16(make_uint4(r[4 * q - 4], r[4 * q - 3], r[4 * q - 2], r[4 * q - 1]),
+                                     make_uint4(w0, w1, w2, w3), &lo, &hi, &sb);
+                        *reinterpret_cast<uint2 *>(qd.codes + 4 * (q - 1)) = make_uint2(lo, hi);
+                        sbs |= sb << (4 * (q - 1));
+                    }
                 }
+                if (qd.scales) *reinterpret_cast<uint32_t *>(qd.scales) = sbs;
                 fence_proxy_async_smem();
                 __syncwarp();
                 if (lane == 0) {
@@ -549,8 +596,8 @@ static pact_status check_lora(const pact_lora_t *l, int64_t M, int64_t N, int64_
 
 // D[M x N] = deq(a) . deq(b)^T (+ LoRA); a [M x K], b [N x K].
 static pact_status run(const pact_nvfp4_t *a, const pact_nvfp4_t *b, int gexp, const pact_lora_t *lora, bool dgrad,
-                       const pact_bf16 *res, int64_t ldr, pact_bf16 *out, int64_t ldo, cudaStream_t stream,
-                       const char *what) {
+                       const pact_bf16 *res, int64_t ldr, pact_bf16 *out, int64_t ldo, const pact_nvfp4_t *yq, int nq,
+                       cudaStream_t stream, const char *what) {
     const int64_t M = a->rows, K = a->cols, N = b->rows;
     PACT_CHECK(gexp >= -100 && gexp <= 100, PACT_ERR_INVALID_ARG, "%s: w->gexp out of range (%d)", what, gexp);
     PACT_CHECK(M <= 0x7FFFFFFF && N <= 0x7FFFFFFF && K <= 0x7FFFFFFF, PACT_ERR_SHAPE, "%s: dimension too large", what);
@@ -594,6 +641,13 @@ static pact_status run(const pact_nvfp4_t *a, const pact_nvfp4_t *b, int gexp, c
     p.out_scale = std::ldexp(1.0f, gexp);
     // stream the larger operand once: A (M x K) when M > N, else B (N x K)
     p.n_fast = M > N ? 1 : 0;
+    p.nq = nq;
+    p.q_split = (int)N;
+    for (int i = 0; i < 2; ++i) {
+        p.q_codes[i] = i < nq ? static_cast<uint8_t *>(yq[i].codes) : nullptr;
+        p.q_scales[i] = i < nq ? static_cast<uint8_t *>(yq[i].scales) : nullptr;
+    }
+    if (nq == 2) p.q_split = (int)yq[0].cols;
     p.lora_mode = LORA_NONE;
     p.lora_steps = 0; p.lora_r = 0; p.lora_nseg = 1;
     for (int i = 0; i < 4; ++i) p.seg_end[i] = N;
@@ -642,7 +696,31 @@ pact_status pact_frozen_gemm_fwd(const pact_nvfp4_t *xq, const pact_weight_cache
     if (s == PACT_OK) s = check_nvfp4(xq, xq->rows, K, "xq");
     if (s != PACT_OK) return s;
     PACT_CHECK(xq->rows >= 1 && N % 64 == 0 && K % 64 == 0, PACT_ERR_SHAPE, "pact_frozen_gemm_fwd: bad shape");
-    return gemm::run(xq, &w->fwd, w->gexp, lora, false, residual, ldr, y, ldy, (cudaStream_t)stream, "pact_frozen_gemm_fwd");
+    return gemm::run(xq, &w->fwd, w->gexp, lora, false, residual, ldr, y, ldy, nullptr, 0, (cudaStream_t)stream,
+                     "pact_frozen_gemm_fwd");
+}
+
+pact_status pact_frozen_gemm_fwd_quant(const pact_nvfp4_t *xq, const pact_weight_cache_t *w, const pact_lora_t *lora,
+                                       const pact_bf16 *residual, int64_t ldr, pact_bf16 *y, int64_t ldy,
+                                       const pact_nvfp4_t *yq, int nq, pact_stream_t stream) {
+    const char *what = "pact_frozen_gemm_fwd_quant";
+    PACT_CHECK(xq && w && yq, PACT_ERR_INVALID_ARG, "%s: NULL argument", what);
+    PACT_CHECK(nq == 1 || nq == 2, PACT_ERR_INVALID_ARG, "%s: nq must be 1 or 2", what);
+    const int64_t N = w->fwd.rows, K = w->fwd.cols;
+    pact_status s = check_nvfp4(&w->fwd, N, K, "w->fwd");
+    if (s == PACT_OK) s = check_nvfp4(xq, xq->rows, K, "xq");
+    if (s != PACT_OK) return s;
+    PACT_CHECK(xq->rows >= 1 && N % 64 == 0 && K % 64 == 0, PACT_ERR_SHAPE, "%s: bad shape", what);
+    int64_t covered = 0;
+    for (int i = 0; i < nq; ++i) {
+        PACT_CHECK(yq[i].cols >= 64 && yq[i].cols % 64 == 0, PACT_ERR_SHAPE, "%s: yq[%d].cols must be a multiple of 64", what, i);
+        s = check_nvfp4(&yq[i], xq->rows, yq[i].cols, "yq");
+        if (s != PACT_OK) return s;
+        PACT_CHECK(aligned16(yq[i].codes) && aligned16(yq[i].scales), PACT_ERR_ALIGN, "%s: yq 16-byte aligned", what);
+        covered += yq[i].cols;
+    }
+    PACT_CHECK(covered == N, PACT_ERR_SHAPE, "%s: the yq tensors' columns must add up to N = %lld", what, (long long)N);
+    return gemm::run(xq, &w->fwd, w->gexp, lora, false, residual, ldr, y, ldy, yq, nq, (cudaStream_t)stream, what);
 }
 
 pact_status pact_frozen_gemm_dgrad(const pact_nvfp4_t *dyq, const pact_weight_cache_t *w, const pact_lora_t *lora,
@@ -654,7 +732,7 @@ pact_status pact_frozen_gemm_dgrad(const pact_nvfp4_t *dyq, const pact_weight_ca
     if (s == PACT_OK) s = check_nvfp4(dyq, dyq->rows, N, "dyq");
     if (s != PACT_OK) return s;
     PACT_CHECK(dyq->rows >= 1 && N % 64 == 0 && K % 64 == 0, PACT_ERR_SHAPE, "pact_frozen_gemm_dgrad: bad shape");
-    return gemm::run(dyq, &w->bwd, w->gexp, lora, true, residual, ldr, dx, lddx, (cudaStream_t)stream,
+    return gemm::run(dyq, &w->bwd, w->gexp, lora, true, residual, ldr, dx, lddx, nullptr, 0, (cudaStream_t)stream,
                      "pact_frozen_gemm_dgrad");
 }
 

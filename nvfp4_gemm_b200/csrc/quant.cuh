@@ -46,6 +46,28 @@ __device__ __forceinline__ float quotient(float a, float s, float r) {
     return __fmaf_rn(e, r, q0);
 }
 
+// The same quotient for a pair of values at once (packed FP32: each half is exactly
+// the scalar quotient above).  ns2 holds -s twice, r2 holds r twice.  Returns the two
+// quotients with the signs of the inputs (a -0 input keeps its sign).
+__device__ __forceinline__ void quotient2(float a0, float a1, uint64_t ns2, uint64_t r2, float &q0, float &q1) {
+    const uint64_t a = f2_pack(a0, a1);
+    const uint64_t p = f2_mul(a, r2);
+    const uint64_t e = f2_fma(p, ns2, a);
+    f2_unpack(f2_fma(e, r2, p), q0, q1);
+    q0 = copysignf(q0, a0);
+    q1 = copysignf(q1, a1);
+}
+
+// Two E2M1 codes (RNE, saturating, signs kept) of a pair of quotients as one byte:
+// element 0 in the low nibble.
+__device__ __forceinline__ uint32_t e2m1_pair(float q0, float q1) {
+    uint32_t byte;
+    asm("{\n\t.reg .b8 t;\n\tcvt.rn.satfinite.e2m1x2.f32 t, %2, %1;\n\tcvt.u32.u8 %0, t;\n\t}"
+        : "=r"(byte)
+        : "f"(q0), "f"(q1));
+    return byte;
+}
+
 // amax -> E4M3 scale byte: RNE(amax / 6) with saturation.  The product with the
 // correctly rounded FP32 value of 1/6 takes the same decision as the exact quotient
 // for every BF16 amax (checked over all of them by the tests).
@@ -69,9 +91,10 @@ __device__ __forceinline__ uint32_t quant8(const float (&v)[8], uint32_t *sb) {
     const uint32_t b = scale_byte(amax);
     const float s = e4m3_to_float(b);
     const float r = b ? __frcp_rn(s) : 0.0f;
+    const uint64_t r2 = f2_pack(r, r), ns2 = f2_pack(-s, -s);
     float q[8];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) q[i] = copysignf(quotient(v[i], s, r), v[i]);
+    for (int i = 0; i < 8; i += 2) quotient2(v[i], v[i + 1], ns2, r2, q[i], q[i + 1]);
     uint32_t out;
     asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
         "cvt.rn.satfinite.e2m1x2.f32 b0, %2, %1;\n\t"
@@ -83,6 +106,32 @@ __device__ __forceinline__ uint32_t quant8(const float (&v)[8], uint32_t *sb) {
         : "f"(q[0]), "f"(q[1]), "f"(q[2]), "f"(q[3]), "f"(q[4]), "f"(q[5]), "f"(q[6]), "f"(q[7]));
     *sb = b;
     return out;
+}
+
+// Quantize one NVFP4 block of 16 BF16 values held by one thread as 8 packed words
+// (values 2j, 2j+1 in the low and high half of word j of wa, wb): the 8 code bytes go to *lo
+// (elements 0..7, element 0 in the low nibble) and *hi (8..15), the scale byte to
+// *sb.  Same arithmetic as quant8 (without the shuffle), one pair at a time so that
+// little state is live.
+__device__ __forceinline__ void quant16_bf16(const uint4 wa, const uint4 wb, uint32_t *lo, uint32_t *hi, uint32_t *sb) {
+    const uint32_t w[8] = {wa.x, wa.y, wa.z, wa.w, wb.x, wb.y, wb.z, wb.w};
+    float amax = 0.0f;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) amax = fmaxf(amax, fmaxf(fabsf(bf16lo(w[j])), fabsf(bf16hi(w[j]))));
+    const uint32_t b = scale_byte(amax);
+    const float s = e4m3_to_float(b);
+    const float r = b ? __frcp_rn(s) : 0.0f;
+    const uint64_t r2 = f2_pack(r, r), ns2 = f2_pack(-s, -s);
+    uint32_t out[2] = {0u, 0u};
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+        float q0, q1;
+        quotient2(bf16lo(w[j]), bf16hi(w[j]), ns2, r2, q0, q1);
+        out[j >> 2] |= e2m1_pair(q0, q1) << (8 * (j & 3));
+    }
+    *lo = out[0];
+    *hi = out[1];
+    *sb = b;
 }
 
 // Gather the scales of blocks 4q..4q+3 (lanes 8q, 8q+2, 8q+4, 8q+6) into lane 8q

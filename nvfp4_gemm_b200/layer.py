@@ -8,7 +8,8 @@ Data flow (PACT blog summary, section "方法" (method); PACT abstract):
             h2   = h + NVFP4 GEMM(q(attn), W_o) + LoRA(attn)  residual fused in the epilogue
             xq2, x2, rstd2 = RMSNorm+quantize(h2)
             gu   = NVFP4 GEMM(xq2, W_gu) + LoRA(x2)           gate|up concatenated along N
-            m, mq, gq, uq = SiLU-multiply+quantize(gate, up)  gq, uq saved for backward
+            m, mq = SiLU-multiply+quantize(gate, up)           gq, uq (NVFP4 copies of gate, up,
+                                                                written by the GEMM) saved for backward
             out  = h2 + NVFP4 GEMM(mq, W_down) + LoRA(m)
   saved for backward: xq1, rstd1, xq2, rstd2, gq, uq (NVFP4) and attn.
   backward  the input gradients run the NVFP4 dgrad GEMMs on the cached transposed,
@@ -202,11 +203,13 @@ class PactLayer:
                bytes=2 * M * H + 2 * H + S.nv(M, H) + 2 * M * H + 4 * M),
             Op("lora_fwd_gu", lambda: P.pact_lora_fwd(self.x2, self.a_gu, self.sc["gu"], self.t_gu, self.ws), kernels=2,
                bytes=lora_fwd(H, 2 * r)),
-            Op("gemm_fwd_gu", lambda: P.pact_frozen_gemm_fwd(self.xq2, self.c_gu, self.l_gu_f, y=self.gu),
-               "gemm", gemm(S.M, 2 * I, S.H), bytes=gbytes(2 * I, H, 2 * r)),
+            # the gate|up GEMM also writes the NVFP4 copies gq, uq kept for the backward
+            Op("gemm_fwd_gu", lambda: P.pact_frozen_gemm_fwd_quant(self.xq2, self.c_gu, [self.gq, self.uq],
+                                                                   self.l_gu_f, y=self.gu),
+               "gemm", gemm(S.M, 2 * I, S.H), bytes=gbytes(2 * I, H, 2 * r) + 2 * S.nv(M, I)),
             Op("silu_mul_quant", lambda: P.pact_silu_mul_quant(self.gu[:, :I], self.gu[:, I:], self.m, self.mq,
-                                                               self.gq, self.uq),
-               bytes=4 * M * I + 2 * M * I + 3 * S.nv(M, I)),
+                                                               want_copies=False),
+               bytes=4 * M * I + 2 * M * I + S.nv(M, I)),
             Op("lora_fwd_down", lambda: P.pact_lora_fwd(self.m, self.a_d, self.sc["d"], self.t_d, self.ws), kernels=2,
                bytes=lora_fwd(I, r)),
             Op("gemm_fwd_down", lambda: P.pact_frozen_gemm_fwd(self.mq, self.c_d, self.l_d_f, residual=self.h2,

@@ -76,6 +76,8 @@ def _load() -> ctypes.CDLL:
         "pact_frozen_gemm_fwd": (S, [NV, ctypes.POINTER(c_weight_cache), ctypes.POINTER(c_lora), P, I64, P, I64, P]),
         "pact_frozen_gemm_dgrad": (S, [NV, ctypes.POINTER(c_weight_cache), ctypes.POINTER(c_lora), P, I64, P, I64,
                                        P]),
+        "pact_frozen_gemm_fwd_quant": (S, [NV, ctypes.POINTER(c_weight_cache), ctypes.POINTER(c_lora), P, I64, P,
+                                           I64, NV, I, P]),
         "pact_lora_fwd_workspace_bytes": (ctypes.c_size_t, [I64, I64, I]),
         "pact_lora_fwd": (S, [P, I64, I64, I64, P, I, F, P, I64, P, ctypes.c_size_t, P]),
         "pact_lora_fwd_noalloc": (S, [P, I64, I64, I64, P, I, F, P, I64, P]),
@@ -337,6 +339,22 @@ def pact_frozen_gemm_fwd(xq: NVFP4Tensor, w: WeightCache, lora: Optional[c_lora]
                                      ctypes.byref(lora) if lora is not None else None,
                                      _ptr(residual), _ld(residual) if residual is not None else 0,
                                      y.data_ptr(), _ld(y), _stream(stream)))
+    return y
+
+
+def pact_frozen_gemm_fwd_quant(xq: NVFP4Tensor, w: WeightCache, yq: Sequence[NVFP4Tensor],
+                               lora: Optional[c_lora] = None, residual: Optional[torch.Tensor] = None,
+                               y: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """pact_frozen_gemm_fwd that also writes the NVFP4 copy of y, split along the
+    columns into the tensors of yq (1 or 2, in column order)."""
+    if y is None:
+        y = torch.empty((xq.rows, w.N), dtype=torch.bfloat16, device=xq.codes.device)
+    s = xq.c()
+    arr = (c_nvfp4 * len(yq))(*[t.c() for t in yq])
+    _check(_lib.pact_frozen_gemm_fwd_quant(ctypes.byref(s), ctypes.byref(w.cstruct),
+                                           ctypes.byref(lora) if lora is not None else None,
+                                           _ptr(residual), _ld(residual) if residual is not None else 0,
+                                           y.data_ptr(), _ld(y), arr, len(yq), _stream(stream)))
     return y
 
 

@@ -237,6 +237,40 @@ def test_gemm_dgrad_lora(P, orc, M, N, K, R):
     assert_close(to_f64(dx), ref, "dgrad + LoRA")
 
 
+@pytest.mark.parametrize("M,parts,K,lora", [(300, [512, 256], 512, False), (130, [768], 320, True),
+                                             (2048, [1024, 1024], 256, True), (64, [256, 1280], 192, False)])
+def test_gemm_fwd_quant(P, orc, guards, M, parts, K, lora):
+    """The forward GEMM that also writes the NVFP4 copy of its BF16 output, split along
+    the columns: the copy equals the quantizer's on the device's own y (bit-exact,
+    padding scales included), y is as pact_frozen_gemm_fwd's."""
+    N = sum(parts)
+    x = synth.gaussian_bf16(1, (M, K))
+    w = synth.weight_bf16(0, (N, K), outliers=True)
+    wc = P.pact_weight_layout_cache(to_dev(w))
+    xq = P.pact_quantize_nvfp4(to_dev(x))
+    lo = None
+    if lora:
+        r = 16
+        a = synth.gaussian_bf16(20, (len(parts) * r, K), std=0.02)
+        b = synth.gaussian_bf16(30, (N, r), std=0.02)
+        T = P.pact_lora_fwd(to_dev(x), to_dev(a), 2.0)
+        lo = P.lora_struct(T, to_dev(b), r, _segments(N, parts))
+    yq = [guards.nvfp4(M, c) for c in parts]
+    y = P.pact_frozen_gemm_fwd_quant(xq, wc, yq, lora=lo, y=guards.matrix(M, N, pad_cols=8))
+    y_ref = P.pact_frozen_gemm_fwd(xq, wc, lora=lo)
+    sync()
+    status_ok(P)
+    assert torch.equal(y.contiguous().view(torch.int16), y_ref.view(torch.int16))
+    yb = to_bits(y)
+    c0 = 0
+    for t, c in zip(yq, parts):
+        assert_nvfp4_equal(t, orc.quantize(yb[:, c0:c0 + c]), orc, f"q(y) columns {c0}..{c0 + c}")
+        c0 += c
+    if not lora:
+        wf, _ = orc.weight_cache(w)
+        assert_close(to_f64(y), orc.nvfp4_gemm(orc.quantize(x), wf), "fwd")
+
+
 # ------------------------------------------------------------------------- LoRA
 @pytest.mark.parametrize("M,parts,r,K", [(256, [512], 16, 384), (300, [512, 256, 256], 16, 576),
                                          (130, [256, 320], 32, 320), (2048, [1024], 16, 2112)])
