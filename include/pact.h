@@ -222,6 +222,20 @@ PACT_API pact_status pact_frozen_gemm_fwd_quant(const pact_nvfp4_t *xq, const pa
                                                 pact_bf16 *y, int64_t ldy, const pact_nvfp4_t *yq, int nq,
                                                 pact_stream_t stream);
 
+/* The gate|up GEMM fused with the SiLU-multiply ([METHOD] bullet 2): for the
+ * concatenated gate|up weight (w->fwd [2I x K], gate rows first, I a multiple of
+ * 256) it computes g|u = BF16_RNE(2^g (deq(xq) . deq(w->fwd)^T + LoRA)) exactly as
+ * pact_frozen_gemm_fwd would, but writes, instead of g and u,
+ *   m = BF16_RNE(silu(g) u)   [M x I], row stride ldm (>= I, multiple of 8)
+ *   mq = q(m), gq = q(g), uq = q(u)   NVFP4 [M x I] each
+ * with the same values as pact_silu_mul_quant on those g, u.  The tiles of gate and
+ * up columns [256 j, 256 j + 256) run back to back on one CTA pair, so the gate block
+ * waits in shared memory for its up block.  No residual; lora may be NULL. */
+PACT_API pact_status pact_frozen_gemm_fwd_silu(const pact_nvfp4_t *xq, const pact_weight_cache_t *w,
+                                               const pact_lora_t *lora, pact_bf16 *m, int64_t ldm,
+                                               const pact_nvfp4_t *mq, const pact_nvfp4_t *gq,
+                                               const pact_nvfp4_t *uq, pact_stream_t stream);
+
 /* ------------------------------------------------------ A6: dgrad GEMM */
 /* [METHOD] bullet 1 (input gradient) with [LORA]:
  *   dx[M x K] = BF16_RNE( residual + 2^g (deq(dyq) . deq(w->bwd)^T + U . A) )

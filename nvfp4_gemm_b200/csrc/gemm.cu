@@ -93,6 +93,14 @@ struct Params {
     int q_split;
     uint8_t *q_codes[2];
     uint8_t *q_scales[2];
+    // gate|up mode: N = 2 I with the gate rows first; the tiles of gate columns
+    // [256 j, 256 j + 256) and up columns [I + 256 j, ...) run back to back on one CTA
+    // pair, and the epilogue writes m = BF16(silu(g) u) (map tmD over m [M x I]) and its
+    // NVFP4 copy instead of g and u
+    int silu;
+    int half_tiles;       // I / 256
+    uint8_t *m_codes;
+    uint8_t *m_scales;
 };
 
 // Pair-tile coordinates of persistent tile index t.  Consecutive indices run at the
@@ -100,13 +108,31 @@ struct Params {
 // L2 while the other one streams: with N fastest each row block of A is read once
 // and shared by the clusters working across N; with M fastest the same holds for B.
 __device__ __forceinline__ void tile_coords(const Params &p, int t, int mpairs, int ntiles, int &mp, int &nt) {
-    if (p.n_fast) {
+    if (p.silu) {   // t = 2 u + which: pair u of (gate, up) tiles
+        const int u = t >> 1, h = p.half_tiles;
+        int jn;
+        if (p.n_fast) {
+            jn = u % h;
+            mp = u / h;
+        } else {
+            mp = u % mpairs;
+            jn = u / mpairs;
+        }
+        nt = jn + (t & 1) * h;
+    } else if (p.n_fast) {
         nt = t % ntiles;
         mp = t / ntiles;
     } else {
         mp = t % mpairs;
         nt = t / mpairs;
     }
+}
+// The persistent tile sequence of a cluster (every role walks the same one): tiles
+// cluster, cluster + nclusters, ...; in gate|up mode the two tiles of each pair
+// 2 u, 2 u + 1 for u = cluster, cluster + nclusters, ...
+__device__ __forceinline__ int first_tile(const Params &p, int cluster) { return p.silu ? 2 * cluster : cluster; }
+__device__ __forceinline__ int next_tile(const Params &p, int t, int nclusters) {
+    return p.silu ? ((t & 1) ? t + 2 * nclusters - 1 : t + 1) : t + nclusters;
 }
 
 __device__ __forceinline__ int lora_segment(const Params &p, int n0) {
@@ -125,6 +151,15 @@ __device__ __forceinline__ int lora_segment(const Params &p, int n0) {
 struct QDest {
     uint8_t *codes, *scales;
 };
+// The same for m's NVFP4 copy in gate|up mode (col: the up block's column, I + c).
+__device__ __forceinline__ QDest mdest(const Params &p, int row, int col) {
+    QDest d = {nullptr, nullptr};
+    if (row >= ((p.M + 127) & ~127)) return d;
+    const int I = p.half_tiles * BN, lc = col - I;
+    d.scales = p.m_scales + scale_offset(row, lc >> 4, I);
+    if (row < p.M) d.codes = p.m_codes + (int64_t)row * (I >> 1) + (lc >> 1);
+    return d;
+}
 __device__ __forceinline__ QDest qdest(const Params &p, int row, int col) {
     QDest d = {nullptr, nullptr};
     if (!p.nq || row >= ((p.M + 127) & ~127)) return d;
@@ -146,6 +181,9 @@ struct Ring {
     }
 };
 
+// SILU: gate|up mode (p.silu set), instantiated apart so that the plain GEMM's
+// epilogue keeps its registers.
+template <bool SILU>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
 k_nvfp4_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
              const __grid_constant__ CUtensorMap tmSFA, const __grid_constant__ CUtensorMap tmSFB,
@@ -218,7 +256,7 @@ k_nvfp4_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CU
             const uint32_t full_leader = mapa_shared(smem_u32(full), 0);
             Ring rg;
             bool ok = true;
-            for (int t = cluster; ok && t < total; t += nclusters) {
+            for (int t = first_tile(p, cluster); ok && t < total; t = next_tile(p, t, nclusters)) {
                 int mp, nt;
                 tile_coords(p, t, mpairs, ntiles, mp, nt);
                 const int m0 = mp * 2 * BM + (int)rank * BM;     // this CTA's rows
@@ -269,14 +307,18 @@ k_nvfp4_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CU
             Ring rg;
             uint32_t acc_phase = 0;
             bool ok = true;
-            for (int t = cluster; ok && t < total; t += nclusters) {
+            for (int t = first_tile(p, cluster); ok && t < total; t = next_tile(p, t, nclusters)) {
                 ok = mbar_wait(acc_empty, acc_phase ^ 1);
                 tc_fence_after();
                 uint32_t accum = 0;
-                for (int i = 0; ok && i < nsteps; ++i) {
-                    if (!(ok = mbar_wait(&full[rg.stage], rg.phase))) break;
-                    tc_fence_after();
-                    const uint32_t st = smem_u32(smem + rg.stage * STAGE_BYTES);
+                // Per stage: its MMAs, the commit that frees the stage once they are done,
+                // then the next stage's barrier (a non-blocking test first: the producers
+                // run stages ahead).  The ring position lives in registers here.
+                uint32_t stage = rg.stage, phase = rg.phase;
+                bool ready = nsteps > 0 && (ok = mbar_wait(&full[stage], phase));
+                tc_fence_after();
+                for (int i = 0; ready && i < nsteps; ++i) {
+                    const uint32_t st = smem_u32(smem) + stage * STAGE_BYTES;
                     if (lora && i == 0) {
                         const int R = p.lora_nseg * p.lora_r;
                         for (int c = 0; c < p.lora_steps; ++c) {
@@ -292,9 +334,9 @@ k_nvfp4_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CU
                     } else {
                         const int kt = i - (lora ? 1 : 0);
                         const int nk = min(BK / KSTEP, (p.K - kt * BK) / KSTEP);
-                        const uint32_t sf = tmem + COL_SF + rg.stage * SF_COLS;
-                        const uint64_t ad = adesc0 + (uint64_t)((rg.stage * STAGE_BYTES) >> 4);
-                        const uint64_t bd = bdesc0 + (uint64_t)((rg.stage * STAGE_BYTES) >> 4);
+                        const uint32_t sf = tmem + COL_SF + stage * SF_COLS;
+                        const uint64_t ad = adesc0 + (uint64_t)((stage * STAGE_BYTES) >> 4);
+                        const uint64_t bd = bdesc0 + (uint64_t)((stage * STAGE_BYTES) >> 4);
                         if (nk == BK / KSTEP) {
 #pragma unroll
                             for (int s = 0; s < BK / KSTEP; ++s) {
@@ -310,9 +352,18 @@ k_nvfp4_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CU
                             }
                         }
                     }
-                    tc_commit_pair(&empty[rg.stage], 3);
-                    rg.next();
+                    tc_commit_pair(&empty[stage], 3);
+                    if (++stage == STAGES) {
+                        stage = 0;
+                        phase ^= 1;
+                    }
+                    if (i + 1 < nsteps) {
+                        if (!mbar_test_wait(&full[stage], phase)) ready = ok = mbar_wait(&full[stage], phase);
+                        tc_fence_after();
+                    }
                 }
+                rg.stage = stage;
+                rg.phase = phase;
                 if (!ok) break;
                 tc_commit_pair(acc_full, 3);
                 acc_phase ^= 1;
@@ -329,7 +380,7 @@ k_nvfp4_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CU
         const uint32_t lane_base = tmem + ((uint32_t)(sub * 32) << 16);
         Ring rg;
         bool ok = true;
-        for (int t = cluster; ok && t < total; t += nclusters) {
+        for (int t = first_tile(p, cluster); ok && t < total; t = next_tile(p, t, nclusters)) {
             for (int i = 0; i < nsteps; ++i) {
                 const bool lstep = lora && i == 0;   // a LoRA stage carries no scales
                 if (!(ok = warp_all(mbar_wait(&sf_full[rg.stage], rg.phase)))) break;
@@ -377,7 +428,7 @@ k_nvfp4_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CU
             Ring rg;
             uint32_t lora_prev = 0;   // bit s: the previous use of stage s was a LoRA stage
             bool ok = true;
-            for (int t = cluster; ok && t < total; t += nclusters) {
+            for (int t = first_tile(p, cluster); ok && t < total; t = next_tile(p, t, nclusters)) {
                 int mp, nt;
                 tile_coords(p, t, mpairs, ntiles, mp, nt);
                 const int ga = (mp * 2 * BM + (int)rank * BM) / 128, gb = (nt * BN) / 128;
@@ -431,11 +482,12 @@ k_nvfp4_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CU
             tma_load_2d(slab_p, &tmR, &res_full[ew], block_x(t), block_y(t));
         };
         uint32_t acc_phase = 0, res_phase = 0;
-        if (p.has_res && lane == 0 && cluster < total && inside(cluster)) load_residual(cluster);
+        if (p.has_res && lane == 0 && first_tile(p, cluster) < total && inside(first_tile(p, cluster)))
+            load_residual(first_tile(p, cluster));
         bool ok = true;
-        for (int t = cluster; ok && t < total; t += nclusters) {
+        for (int t = first_tile(p, cluster); ok && t < total; t = next_tile(p, t, nclusters)) {
             bool got = false;
-            if (lane == 0) got = mbar_wait_sleep(acc_full, acc_phase);
+            if (lane == 0) got = mbar_wait(acc_full, acc_phase);
             if (!(ok = __shfl_sync(0xffffffffu, got, 0))) break;
             tc_fence_after();
             uint32_t r[64];
@@ -450,6 +502,10 @@ k_nvfp4_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CU
                 // a 32-row block wholly in the scale layout's padding rows: zero scales only
                 const QDest qd = qdest(p, block_y(t) + lane, block_x(t));
                 if (qd.scales) *reinterpret_cast<uint32_t *>(qd.scales) = 0u;
+                if (SILU && (t & 1)) {
+                    const QDest md = mdest(p, block_y(t) + lane, block_x(t));
+                    if (md.scales) *reinterpret_cast<uint32_t *>(md.scales) = 0u;
+                }
             }
             if (inside(t)) {
                 if (p.has_res) {
@@ -463,6 +519,8 @@ k_nvfp4_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CU
                 // the NVFP4 copy of the block's rounded values: block b of this lane's row is
                 // quantized once its two 8-value pieces are rounded
                 const QDest qd = qdest(p, block_y(t) + lane, block_x(t));
+                // gate|up mode: the gate block stays in the slab for the up block that follows
+                const bool up = SILU && (t & 1);
                 uint32_t sbs = 0;
                 // row `lane` of the block: 8 pieces of 16 bytes, 128-byte swizzle
 #pragma unroll
@@ -481,9 +539,10 @@ k_nvfp4_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CU
                     }
                     const uint32_t w0 = pack_bf16x2(f[0], f[1]), w1 = pack_bf16x2(f[2], f[3]);
                     const uint32_t w2 = pack_bf16x2(f[4], f[5]), w3 = pack_bf16x2(f[6], f[7]);
-                    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(a), "r"(w0), "r"(w1), "r"(w2),
-                                 "r"(w3)
-                                 : "memory");
+                    if (!up)
+                        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(a), "r"(w0), "r"(w1), "r"(w2),
+                                     "r"(w3)
+                                     : "memory");
                     // the rounded values, kept for the NVFP4 copy (r[] is free again)
                     r[4 * q] = w0; r[4 * q + 1] = w1; r[4 * q + 2] = w2; r[4 * q + 3] = w3;
                     if ((q & 1) && qd.codes) {
@@ -495,16 +554,49 @@ k_nvfp4_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CU
                     }
                 }
                 if (qd.scales) *reinterpret_cast<uint32_t *>(qd.scales) = sbs;
-                fence_proxy_async_smem();
-                __syncwarp();
-                if (lane == 0) {
-                    tma_store_2d(&tmD, slab, block_x(t), block_y(t));
-                    bulk_commit_group();
+                if (up) {
+                    // m = BF16(silu(g) u) for the 64 columns of this row: g from the slab (the
+                    // gate block, same rows and columns), u from the packed words in r[0..31];
+                    // m replaces g in the slab and is quantized block by block
+                    const QDest md = mdest(p, block_y(t) + lane, block_x(t));
+                    uint32_t msbs = 0, n0 = 0, n1 = 0, n2 = 0, n3 = 0;
+#pragma unroll
+                    for (int q = 0; q < 8; ++q) {
+                        const uint32_t a = slab + lane * 128 + ((q ^ (lane & 7)) << 4);
+                        uint32_t g4[4], mw[4];
+                        asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                                     : "=r"(g4[0]), "=r"(g4[1]), "=r"(g4[2]), "=r"(g4[3])
+                                     : "r"(a));
+#pragma unroll
+                        for (int j = 0; j < 4; ++j)
+                            mw[j] = pack_bf16x2(silu_mul_out(bf16lo(g4[j]), bf16lo(r[4 * q + j])),
+                                                silu_mul_out(bf16hi(g4[j]), bf16hi(r[4 * q + j])));
+                        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(a), "r"(mw[0]), "r"(mw[1]),
+                                     "r"(mw[2]), "r"(mw[3])
+                                     : "memory");
+                        if ((q & 1) && md.codes) {
+                            uint32_t lo, hi, sb;
+                            quant16_bf16(make_uint4(n0, n1, n2, n3), make_uint4(mw[0], mw[1], mw[2], mw[3]), &lo, &hi,
+                                         &sb);
+                            *reinterpret_cast<uint2 *>(md.codes + 4 * (q - 1)) = make_uint2(lo, hi);
+                            msbs |= sb << (4 * (q - 1));
+                        }
+                        n0 = mw[0]; n1 = mw[1]; n2 = mw[2]; n3 = mw[3];
+                    }
+                    if (md.scales) *reinterpret_cast<uint32_t *>(md.scales) = msbs;
+                }
+                if (!SILU || up) {   // a gate block is not stored: its m follows with the up block
+                    fence_proxy_async_smem();
+                    __syncwarp();
+                    if (lane == 0) {
+                        tma_store_2d(&tmD, slab, up ? block_x(t) - p.half_tiles * BN : block_x(t), block_y(t));
+                        bulk_commit_group();
+                    }
                 }
             }
-            if (lane == 0 && p.has_res && t + nclusters < total && inside(t + nclusters)) {
+            if (lane == 0 && p.has_res && next_tile(p, t, nclusters) < total && inside(next_tile(p, t, nclusters))) {
                 bulk_wait_read_all();
-                load_residual(t + nclusters);
+                load_residual(next_tile(p, t, nclusters));
             }
             __syncwarp();
         }
@@ -562,7 +654,9 @@ static pact_status ensure_attrs() {
     const int d = current_device();
     if (d >= 0 && d < 64 && done[d]) return PACT_OK;
     cudaError_t e =
-        cudaFuncSetAttribute(k_nvfp4_gemm, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+        cudaFuncSetAttribute(k_nvfp4_gemm<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+    if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(k_nvfp4_gemm<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
     if (e != cudaSuccess) return fail(PACT_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));
     if (d >= 0 && d < 64) done[d] = true;
     return PACT_OK;
@@ -595,9 +689,18 @@ static pact_status check_lora(const pact_lora_t *l, int64_t M, int64_t N, int64_
 }
 
 // D[M x N] = deq(a) . deq(b)^T (+ LoRA); a [M x K], b [N x K].
+// Gate|up mode outputs: m [M x I] (BF16, row stride ldm) and the NVFP4 copies mq, gq, uq.
+struct SiluOut {
+    pact_bf16 *m;
+    int64_t ldm;
+    const pact_nvfp4_t *mq;
+};
+
+// D[M x N] = deq(a) . deq(b)^T (+ LoRA); a [M x K], b [N x K].  With so, gate|up mode:
+// D is not written; m, mq (and through yq, gq and uq) are.
 static pact_status run(const pact_nvfp4_t *a, const pact_nvfp4_t *b, int gexp, const pact_lora_t *lora, bool dgrad,
                        const pact_bf16 *res, int64_t ldr, pact_bf16 *out, int64_t ldo, const pact_nvfp4_t *yq, int nq,
-                       cudaStream_t stream, const char *what) {
+                       cudaStream_t stream, const char *what, const SiluOut *so = nullptr) {
     const int64_t M = a->rows, K = a->cols, N = b->rows;
     PACT_CHECK(gexp >= -100 && gexp <= 100, PACT_ERR_INVALID_ARG, "%s: w->gexp out of range (%d)", what, gexp);
     PACT_CHECK(M <= 0x7FFFFFFF && N <= 0x7FFFFFFF && K <= 0x7FFFFFFF, PACT_ERR_SHAPE, "%s: dimension too large", what);
@@ -626,10 +729,13 @@ static pact_status run(const pact_nvfp4_t *a, const pact_nvfp4_t *b, int gexp, c
     if (s == PACT_OK)
         s = make_map(&tmSFB, CU_TENSOR_MAP_DATA_TYPE_UINT8, b->scales, 256, 2 * chunks_b, 256, 256, 8,
                      CU_TENSOR_MAP_SWIZZLE_NONE, what);
-    // output (and residual) blocks: 32 rows x 64 BF16 columns, 128-byte swizzle
+    // output (and residual) blocks: 32 rows x 64 BF16 columns, 128-byte swizzle; in
+    // gate|up mode the output is m [M x N / 2]
     if (s == PACT_OK)
-        s = make_map(&tmD, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, out, N, M, ldo * 2, 64, 32, CU_TENSOR_MAP_SWIZZLE_128B,
-                     what);
+        s = so ? make_map(&tmD, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, so->m, N / 2, M, so->ldm * 2, 64, 32,
+                          CU_TENSOR_MAP_SWIZZLE_128B, what)
+               : make_map(&tmD, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, out, N, M, ldo * 2, 64, 32, CU_TENSOR_MAP_SWIZZLE_128B,
+                          what);
     tmR = tmD;
     if (s == PACT_OK && res)
         s = make_map(&tmR, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, res, N, M, ldr * 2, 64, 32, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -648,6 +754,10 @@ static pact_status run(const pact_nvfp4_t *a, const pact_nvfp4_t *b, int gexp, c
         p.q_scales[i] = i < nq ? static_cast<uint8_t *>(yq[i].scales) : nullptr;
     }
     if (nq == 2) p.q_split = (int)yq[0].cols;
+    p.silu = so ? 1 : 0;
+    p.half_tiles = so ? (int)(N / 2 / BN) : 0;
+    p.m_codes = so ? static_cast<uint8_t *>(so->mq->codes) : nullptr;
+    p.m_scales = so ? static_cast<uint8_t *>(so->mq->scales) : nullptr;
     p.lora_mode = LORA_NONE;
     p.lora_steps = 0; p.lora_r = 0; p.lora_nseg = 1;
     for (int i = 0; i < 4; ++i) p.seg_end[i] = N;
@@ -674,10 +784,11 @@ static pact_status run(const pact_nvfp4_t *a, const pact_nvfp4_t *b, int gexp, c
         }
         if (s != PACT_OK) return s;
     }
-    const int pairs = (int)(((M + 255) / 256) * ((N + 255) / 256));
-    const int clusters = pairs < sm_count() / 2 ? pairs : sm_count() / 2;
-    return launch_dep(k_nvfp4_gemm, dim3(2 * clusters), dim3(THREADS), SMEM_BYTES, stream, what, tmA, tmB, tmSFA, tmSFB,
-                      tmLa, tmLb, tmD, tmR, p);
+    // work units: output tiles, or (gate, up) tile pairs in gate|up mode
+    const int units = (int)(((M + 255) / 256) * ((N + 255) / 256)) / (so ? 2 : 1);
+    const int clusters = units < sm_count() / 2 ? units : sm_count() / 2;
+    return launch_dep(so ? k_nvfp4_gemm<true> : k_nvfp4_gemm<false>, dim3(2 * clusters), dim3(THREADS), SMEM_BYTES,
+                      stream, what, tmA, tmB, tmSFA, tmSFB, tmLa, tmLb, tmD, tmR, p);
 }
 
 }  // namespace gemm
@@ -721,6 +832,29 @@ pact_status pact_frozen_gemm_fwd_quant(const pact_nvfp4_t *xq, const pact_weight
     }
     PACT_CHECK(covered == N, PACT_ERR_SHAPE, "%s: the yq tensors' columns must add up to N = %lld", what, (long long)N);
     return gemm::run(xq, &w->fwd, w->gexp, lora, false, residual, ldr, y, ldy, yq, nq, (cudaStream_t)stream, what);
+}
+
+pact_status pact_frozen_gemm_fwd_silu(const pact_nvfp4_t *xq, const pact_weight_cache_t *w, const pact_lora_t *lora,
+                                      pact_bf16 *m, int64_t ldm, const pact_nvfp4_t *mq, const pact_nvfp4_t *gq,
+                                      const pact_nvfp4_t *uq, pact_stream_t stream) {
+    const char *what = "pact_frozen_gemm_fwd_silu";
+    PACT_CHECK(xq && w && m && mq && gq && uq, PACT_ERR_INVALID_ARG, "%s: NULL argument", what);
+    const int64_t N = w->fwd.rows, K = w->fwd.cols, I = N / 2, M = xq->rows;
+    pact_status s = check_nvfp4(&w->fwd, N, K, "w->fwd");
+    if (s == PACT_OK) s = check_nvfp4(xq, M, K, "xq");
+    if (s != PACT_OK) return s;
+    PACT_CHECK(M >= 1 && N % 512 == 0 && K % 64 == 0, PACT_ERR_SHAPE,
+               "%s: the gate|up weight needs I = N / 2 a multiple of 256 (N = %lld)", what, (long long)N);
+    PACT_CHECK(ldm >= I && ldm % 8 == 0 && aligned16(m), PACT_ERR_ALIGN, "%s: m 16-byte aligned with ldm >= I, %% 8 == 0",
+               what);
+    s = check_nvfp4(mq, M, I, "mq");
+    if (s == PACT_OK) s = check_nvfp4(gq, M, I, "gq");
+    if (s == PACT_OK) s = check_nvfp4(uq, M, I, "uq");
+    if (s != PACT_OK) return s;
+    const pact_nvfp4_t yq[2] = {*gq, *uq};
+    const gemm::SiluOut so = {m, ldm, mq};
+    // D itself is not written in this mode; out only has to satisfy the argument checks
+    return gemm::run(xq, &w->fwd, w->gexp, lora, false, nullptr, 0, m, N, yq, 2, (cudaStream_t)stream, what, &so);
 }
 
 pact_status pact_frozen_gemm_dgrad(const pact_nvfp4_t *dyq, const pact_weight_cache_t *w, const pact_lora_t *lora,

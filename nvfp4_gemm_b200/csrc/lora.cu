@@ -24,7 +24,7 @@ namespace lmma {
 
 constexpr int BM = 128;        // output rows per CTA (MMA M)
 constexpr int BK = 64;         // contraction elements per stage (128 bytes of BF16)
-constexpr int STAGES = 3;      // with stages sized to the product, two CTAs fit on an SM
+constexpr int MAX_STAGES = 6;  // ring depth: 6, or 3 where two CTAs should share an SM
 constexpr int THREADS = 192;
 constexpr int A_BYTES = BM * BK * 2;     // 16384
 constexpr int B_BYTES = 64 * BK * 2;     // 8192 per B part
@@ -37,9 +37,19 @@ constexpr int RAW_BYTES = RAW_CODE_BYTES + 1024;
 // for an NVFP4 A, its staging area; all multiples of 1024 bytes.
 __host__ __device__ constexpr int oper_bytes(int nparts) { return A_BYTES + nparts * B_BYTES; }
 __host__ __device__ constexpr int stage_bytes(int nparts, bool fp4) { return oper_bytes(nparts) + (fp4 ? RAW_BYTES : 0); }
-__host__ __device__ constexpr int smem_bytes(int nparts, bool fp4) { return 1024 + STAGES * stage_bytes(nparts, fp4) + 256; }
+__host__ __device__ constexpr int smem_bytes(int nparts, bool fp4, int stages) {
+    return 1024 + stages * stage_bytes(nparts, fp4) + 256;
+}
 constexpr int SM_SMEM = 233472;   // shared memory per SM (228 KiB), 1 KiB of it reserved per CTA
-__host__ __device__ constexpr int ctas_per_sm(int nparts, bool fp4) { return SM_SMEM / (smem_bytes(nparts, fp4) + 1024); }
+__host__ __device__ constexpr int ctas_per_sm(int nparts, bool fp4, int stages) {
+    return SM_SMEM / (smem_bytes(nparts, fp4, stages) + 1024);
+}
+// Ring depth per product: the weight-gradient products (contraction over the tokens,
+// two B parts) run 3 stages so that two CTAs share an SM; the forward and U products
+// (contraction over the features) run one CTA per SM with 6 stages in flight, where
+// more splits would cost more in FP32 partial-sum traffic than they gain.
+__host__ __device__ constexpr int stages_for(int nparts) { return nparts == 2 ? 3 : 6; }
+constexpr int FWD_PER_SM = 1;   // split residency of the one-part products
 constexpr uint32_t TMEM_COLS = 64;
 
 // One output block: rows [row_begin, row_end) of the output, contraction
@@ -153,10 +163,11 @@ k_lora_mma(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUte
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = smem_u32(smem_raw);
     uint8_t *smem = smem_raw + (((raw + 1023) & ~1023u) - raw);
+    const int STAGES = stages_for(nparts);
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + STAGES * STAGE_BYTES);
-    uint64_t *full = bars, *empty = bars + STAGES, *acc_full = bars + 2 * STAGES;
-    uint64_t *raw_full = bars + 2 * STAGES + 1;   // [STAGES], A_FP4 only
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 3 * STAGES + 1);
+    uint64_t *full = bars, *empty = bars + MAX_STAGES, *acc_full = bars + 2 * MAX_STAGES;
+    uint64_t *raw_full = bars + 2 * MAX_STAGES + 1;   // [stages], A_FP4 only
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 3 * MAX_STAGES + 1);
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
@@ -414,10 +425,12 @@ static pact_status launch_mma(const CUtensorMap &ta, const CUtensorMap &tb, cons
                               cudaStream_t st, const char *what) {
     static bool done[64] = {false};
     const int d = current_device();
-    const int smem = smem_bytes(p.b_split ? 2 : 1, A_FP4);
+    const int np = p.b_split ? 2 : 1;
+    const int smem = smem_bytes(np, A_FP4, stages_for(np));
     if (d >= 0 && d < 64 && !done[d]) {
-        cudaError_t e = cudaFuncSetAttribute(k_lora_mma<A_MN, B_MN, A_FP4>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             smem_bytes(2, A_FP4));
+        int mx = 0;
+        for (int n = 1; n <= 2; ++n) mx = mx > smem_bytes(n, A_FP4, stages_for(n)) ? mx : smem_bytes(n, A_FP4, stages_for(n));
+        cudaError_t e = cudaFuncSetAttribute(k_lora_mma<A_MN, B_MN, A_FP4>, cudaFuncAttributeMaxDynamicSharedMemorySize, mx);
         if (e != cudaSuccess) return fail(PACT_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
         done[d] = true;
     }
@@ -480,7 +493,7 @@ static pact_status rows_times_a(const CUtensorMap &tx, const pact_nvfp4_t *xq, i
     p.nprob = 1;
     p.prob[0] = Prob{0, (int)M, 0, (int)K, 0, 0};
     const int tiles = (int)((M + BM - 1) / BM);
-    choose_split(K, tiles, ctas_per_sm(1, xq != nullptr), &p.splits, &p.k_per_split);
+    choose_split(K, tiles, FWD_PER_SM, &p.splits, &p.k_per_split);
     p.ws = ws;
     p.ws_ld = R;
     p.ws_split_stride = M * R;
@@ -520,11 +533,11 @@ static int splits_of(int64_t len, int64_t blocks, int per_sm) {
 
 // Workspace bounds cover both the BF16 and the NVFP4 form of X~ (more CTAs per SM
 // give at least as many splits).
-constexpr int T_PER_SM = ctas_per_sm(1, false) > ctas_per_sm(1, true) ? ctas_per_sm(1, false) : ctas_per_sm(1, true);
-constexpr int DA_PER_SM = ctas_per_sm(2, false) > ctas_per_sm(2, true) ? ctas_per_sm(2, false) : ctas_per_sm(2, true);
+constexpr int T_PER_SM = FWD_PER_SM;
+constexpr int DA_PER_SM = ctas_per_sm(2, false, stages_for(2)) > ctas_per_sm(2, true, stages_for(2)) ? ctas_per_sm(2, false, stages_for(2)) : ctas_per_sm(2, true, stages_for(2));
 
 size_t pact_lora_fwd_workspace_bytes(int64_t M, int64_t K, int R) {
-    return partial_bytes(M, R, splits_of(K, (M + BM - 1) / BM, ctas_per_sm(1, false)));
+    return partial_bytes(M, R, splits_of(K, (M + BM - 1) / BM, FWD_PER_SM));
 }
 
 pact_status pact_lora_fwd(const pact_bf16 *x, int64_t ldx, int64_t M, int64_t K, const pact_bf16 *A, int R,
@@ -548,7 +561,7 @@ pact_status pact_lora_fwd(const pact_bf16 *x, int64_t ldx, int64_t M, int64_t K,
 
 // Upper bound over segmentations: one segment may span all N outputs.
 size_t pact_lora_bwd_u_workspace_bytes(int64_t M, int64_t N, int r, int nseg) {
-    return partial_bytes(M, (int64_t)r * nseg, splits_of(N, (M + BM - 1) / BM, ctas_per_sm(1, false)));
+    return partial_bytes(M, (int64_t)r * nseg, splits_of(N, (M + BM - 1) / BM, FWD_PER_SM));
 }
 
 pact_status pact_lora_bwd_u(const pact_bf16 *dy, int64_t lddy, int64_t M, int64_t N, const pact_bf16 *B, int r,
@@ -582,7 +595,7 @@ pact_status pact_lora_bwd_u(const pact_bf16 *dy, int64_t lddy, int64_t M, int64_
         prev = seg_end[i];
     }
     const int tiles = (int)((M + BM - 1) / BM);
-    choose_split(longest, (int64_t)tiles * nseg, ctas_per_sm(1, false), &p.splits, &p.k_per_split);
+    choose_split(longest, (int64_t)tiles * nseg, FWD_PER_SM, &p.splits, &p.k_per_split);
     float *ws = static_cast<float *>(workspace);
     p.ws = ws;
     p.ws_ld = R;
@@ -597,7 +610,7 @@ size_t pact_lora_bwd_workspace_bytes(int64_t M, int64_t N, int64_t K, int r, int
     const int64_t R = (int64_t)r * nseg;
     return partial_bytes(M, R, splits_of(K, (M + BM - 1) / BM, T_PER_SM))      /* T~ partials */
            + round256((size_t)(M * 2 * R * 2))                                  /* T~ hi/lo */
-           + partial_bytes(N, r, splits_of(M, (N + BM - 1) / BM, ctas_per_sm(2, false)))  /* dB partials */
+           + partial_bytes(N, r, splits_of(M, (N + BM - 1) / BM, ctas_per_sm(2, false, stages_for(2))))  /* dB partials */
            + partial_bytes(K, R, splits_of(M, (K + BM - 1) / BM, DA_PER_SM));  /* dA^T partials */
 }
 
@@ -633,7 +646,7 @@ pact_status pact_lora_bwd(const pact_lora_bwd_t *g, void *workspace, size_t ws_b
     pact_bf16 *tt = reinterpret_cast<pact_bf16 *>(w8);
     w8 += round256((size_t)(M * 2 * R * 2));
     float *ws_db = reinterpret_cast<float *>(w8);
-    w8 += partial_bytes(N, r, splits_of(M, (N + BM - 1) / BM, ctas_per_sm(2, false)));
+    w8 += partial_bytes(N, r, splits_of(M, (N + BM - 1) / BM, ctas_per_sm(2, false, stages_for(2))));
     float *ws_da = reinterpret_cast<float *>(w8);
 
     // X~ is read where it lies: BF16 rows, or the saved NVFP4 copy decoded in shared
@@ -665,7 +678,7 @@ pact_status pact_lora_bwd(const pact_lora_bwd_t *g, void *workspace, size_t ws_b
         }
         pb.b_split = 1;
         pb.b_lo_off = R;
-        choose_split(M, blocks, ctas_per_sm(2, false), &pb.splits, &pb.k_per_split);
+        choose_split(M, blocks, ctas_per_sm(2, false, stages_for(2)), &pb.splits, &pb.k_per_split);
         pb.ws = ws_db;
         pb.ws_ld = r;
         pb.ws_split_stride = N * r;
@@ -686,7 +699,7 @@ pact_status pact_lora_bwd(const pact_lora_bwd_t *g, void *workspace, size_t ws_b
     p.b_split = 1;
     p.b_lo_off = R;
     const int tiles = (int)((K + BM - 1) / BM);
-    choose_split(M, tiles, ctas_per_sm(2, g->xq != nullptr), &p.splits, &p.k_per_split);
+    choose_split(M, tiles, ctas_per_sm(2, g->xq != nullptr, stages_for(2)), &p.splits, &p.k_per_split);
     p.ws = ws_da;
     p.ws_ld = R;
     p.ws_split_stride = K * R;

@@ -21,12 +21,6 @@ __device__ __forceinline__ void zero_pad_scales(const pact_nvfp4_t &t, int64_t r
     }
 }
 
-// 8 packed BF16 values -> floats (element 0 in the low half of .x).
-__device__ __forceinline__ void unpack8_bf16(const uint4 &u, float (&v)[8]) {
-    v[0] = bf16lo(u.x); v[1] = bf16hi(u.x); v[2] = bf16lo(u.y); v[3] = bf16hi(u.y);
-    v[4] = bf16lo(u.z); v[5] = bf16hi(u.z); v[6] = bf16lo(u.w); v[7] = bf16hi(u.w);
-}
-
 // ------------------------------------------------------------------ A2: quantize
 // prescale: a power of two the values are multiplied by first (exact in FP32); 1
 // for every quantization on the step path, 2^-gexp for two-level weight layouts.
@@ -110,6 +104,16 @@ static int grid_for(int64_t warp_tasks, int threads) {
 // (warp w takes 256-column chunks w, w + 4, ...; FP64 partial sums, reduced across the
 // CTA), then y = BF16(x * rstd * gamma) and its NVFP4 copy, read again from shared
 // memory.
+// |x| for the BF16 value whose exponent and mantissa bits sit at bits 20..27 and
+// 13..19 of `field` (FP64's exponent and top mantissa positions): the exponent is
+// rebiased from 127 to 1023, so a normal value comes out exact without a conversion
+// instruction.  Zeros and subnormals come out below 2^-126: their squares (under
+// 2^-252) vanish from any FP64 sum that reaches 2^-200, and a row of them only is
+// governed by eps.  Exponent 255 (infinities, NaN) is left to the caller.
+__device__ __forceinline__ double f64_of_bf16(uint32_t field) {
+    return __hiloint2double((int)(field + 0x38000000u), 0);
+}
+
 constexpr int RING_THREADS = 128;
 constexpr int RING_WARPS = RING_THREADS / 32;
 constexpr int RMS_MAX_H = 16384;
@@ -119,6 +123,8 @@ constexpr int RMS_MAX_H = 16384;
 // BF16 midpoint (its error is below 4 ulps), in which case the double expression
 // is rounded directly (Ziv, "Fast evaluation of elementary mathematical functions
 // with correctly rounded last bit", ACM TOMS 17(3), 1991).
+// Returns the value whose round-to-nearest BF16 conversion is the result: the FP32
+// product where it decides, else the correctly rounded value itself.
 __device__ __forceinline__ float rms_out(float x, float g, float r32, double rstd) {
     const float y = __fmul_rn(__fmul_rn(x, r32), g);
     const uint32_t lo = __float_as_uint(y) & 0xFFFFu;
@@ -126,22 +132,23 @@ __device__ __forceinline__ float rms_out(float x, float g, float r32, double rst
         const double yd = ((double)x * rstd) * (double)g;
         return __bfloat162float(__double2bfloat16(yd));
     }
-    return __bfloat162float(__float2bfloat16_rn(y));
+    return y;
 }
 
-// Ring geometry: slots of `slot_bytes`, as many (2 .. 4) as fit in ~48 KiB, and CTAs
-// per SM so that a few hundred KiB... of shared memory per SM are in use.
+// Ring geometry: slots of `slot_bytes`, as many (2 .. 4) as fit in ~48 KiB, then the
+// slot barriers and `extra` bytes (a shared copy of gamma); as many CTAs per SM (up to
+// 8) as fit in 200 KiB.
 struct Ring {
     int stages;
     size_t slot_bytes, smem;
     int grid;
 };
-static Ring ring_for(int64_t rows, size_t slot_bytes) {
+static Ring ring_for(int64_t rows, size_t slot_bytes, size_t extra) {
     Ring r;
     r.slot_bytes = (slot_bytes + 127) & ~(size_t)127;
     r.stages = (int)(49152 / r.slot_bytes);
     r.stages = r.stages < 2 ? 2 : (r.stages > 4 ? 4 : r.stages);
-    r.smem = r.stages * r.slot_bytes + 64;
+    r.smem = r.stages * r.slot_bytes + 64 + extra;   // + the barriers, + a copy of gamma
     int per_sm = (int)(200 * 1024 / r.smem);
     per_sm = per_sm < 1 ? 1 : (per_sm > 8 ? 8 : per_sm);
     const int64_t g = (int64_t)sm_count() * per_sm;
@@ -156,7 +163,9 @@ __global__ void __launch_bounds__(RING_THREADS) k_rmsnorm_quant(const pact_bf16 
                                                                int stages, int slot_bytes) {
     extern __shared__ __align__(128) uint8_t ring[];
     uint64_t *full = reinterpret_cast<uint64_t *>(ring + stages * slot_bytes);
+    pact_bf16 *gs = reinterpret_cast<pact_bf16 *>(ring + stages * slot_bytes + 64);   // gamma [H]
     __shared__ double red[RING_WARPS];
+    __shared__ double rstd_s;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int64_t rows_pad = (M + 127) & ~int64_t(127);
     const int nchunk = (int)((H + CHUNK - 1) / CHUNK);
@@ -165,8 +174,10 @@ __global__ void __launch_bounds__(RING_THREADS) k_rmsnorm_quant(const pact_bf16 
         for (int i = 0; i < stages; ++i) mbar_init(&full[i], 1);
         fence_barrier_init();
     }
-    __syncthreads();
     pdl_wait();
+    for (int c = 8 * threadIdx.x; c < H; c += 8 * RING_THREADS)
+        *reinterpret_cast<uint4 *>(gs + c) = *reinterpret_cast<const uint4 *>(gamma + c);
+    __syncthreads();
     auto issue = [&](int i) {   // thread 0: row i of this CTA into its slot
         const int64_t r = blockIdx.x + (int64_t)i * gridDim.x;
         if (r < M) {
@@ -187,28 +198,55 @@ __global__ void __launch_bounds__(RING_THREADS) k_rmsnorm_quant(const pact_bf16 
         ok = __syncthreads_and(ok && mbar_wait(&full[slot], (uint32_t)(i / stages) & 1u));
         if (!ok) break;
         const uint8_t *rs = ring + slot * slot_bytes;
-        double s0 = 0.0, s1 = 0.0;
+        // sum of squares in FP64 from values widened by integer operations (f64_of_bf16)
+        double s0 = 0.0, s1 = 0.0, s2 = 0.0, s3 = 0.0;
+        uint32_t top = 0;   // the largest exponent|mantissa pattern of either half
         for (int k = warp; k < nchunk; k += RING_WARPS) {
             const int c = k * CHUNK + 8 * lane;
             if (c < H) {
-                float v[8];
-                load8_bf16(reinterpret_cast<const pact_bf16 *>(rs) + c, v);
+                const uint4 u = *reinterpret_cast<const uint4 *>(rs + 2 * c);
+                const uint32_t w[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
-                for (int j = 0; j < 8; j += 2) {
-                    s0 = fma((double)v[j], (double)v[j], s0);
-                    s1 = fma((double)v[j + 1], (double)v[j + 1], s1);
+                for (int j = 0; j < 4; ++j) {
+                    const uint32_t lo = (w[j] << 13) & 0x0FFFE000u, hi = (w[j] >> 3) & 0x0FFFE000u;
+                    top = max(top, max(lo, hi));
+                    const double a = f64_of_bf16(lo), b = f64_of_bf16(hi);
+                    if (j & 1) {
+                        s2 = fma(a, a, s2);
+                        s3 = fma(b, b, s3);
+                    } else {
+                        s0 = fma(a, a, s0);
+                        s1 = fma(b, b, s1);
+                    }
                 }
             }
         }
-        double ss = s0 + s1;
+        if (__any_sync(0xFFFFFFFFu, top >= (0xFFu << 20))) {
+            // an infinity or NaN in the row: the sum as plain conversions give it
+            s0 = s1 = s2 = s3 = 0.0;
+            for (int k = warp; k < nchunk; k += RING_WARPS) {
+                const int c = k * CHUNK + 8 * lane;
+                if (c < H) {
+                    float v[8];
+                    load8_bf16(reinterpret_cast<const pact_bf16 *>(rs) + c, v);
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) s0 = fma((double)v[j], (double)v[j], s0);
+                }
+            }
+        }
+        double ss = (s0 + s1) + (s2 + s3);
 #pragma unroll
         for (int o = 16; o; o >>= 1) ss += __shfl_xor_sync(0xFFFFFFFFu, ss, o);
         if (lane == 0) red[warp] = ss;
         __syncthreads();
-        ss = (red[0] + red[1]) + (red[2] + red[3]);
-        const double rstd = 1.0 / sqrt(ss / (double)H + (double)eps);
+        if (threadIdx.x == 0) {   // one thread evaluates rstd; the others read it
+            const double q = ((red[0] + red[1]) + (red[2] + red[3])) / (double)H + (double)eps;
+            rstd_s = 1.0 / sqrt(q);
+            if (rstd_out) rstd_out[row] = (float)rstd_s;
+        }
+        __syncthreads();
+        const double rstd = rstd_s;
         const float r32 = (float)rstd;
-        if (threadIdx.x == 0 && rstd_out) rstd_out[row] = r32;
         for (int k = warp; k < nchunk; k += RING_WARPS) {
             const int64_t c0 = (int64_t)k * CHUNK;
             const int64_t c = c0 + 8 * lane;
@@ -216,11 +254,13 @@ __global__ void __launch_bounds__(RING_THREADS) k_rmsnorm_quant(const pact_bf16 
             float v[8] = {0, 0, 0, 0, 0, 0, 0, 0}, g[8] = {0, 0, 0, 0, 0, 0, 0, 0}, o[8];
             if (valid) {
                 load8_bf16(reinterpret_cast<const pact_bf16 *>(rs) + c, v);
-                load8_bf16(gamma + c, g);
+                load8_bf16(gs + c, g);
             }
 #pragma unroll
-            for (int j = 0; j < 8; ++j) o[j] = valid ? rms_out(v[j], g[j], r32, rstd) : 0.0f;
-            if (valid && y) store8_bf16(y + row * H + c, o);
+            for (int j = 0; j < 8; ++j) o[j] = rms_out(v[j], g[j], r32, rstd);   // zeros past the row end
+            uint4 ow;
+            round8_bf16(o, ow, o);
+            if (valid && y) *reinterpret_cast<uint4 *>(y + row * H + c) = ow;
             uint32_t sb;
             const uint32_t codes = quant8(o, &sb);
             store_chunk(yq, row, c0, codes, sb, valid);
@@ -238,30 +278,7 @@ __global__ void __launch_bounds__(RING_THREADS) k_rmsnorm_quant(const pact_bf16 
 }
 
 // --------------------------------------------------- A4: SiLU-multiply + quantize
-// m = BF16_RNE(silu(g) * u), exactly rounded.  The FP32 evaluation with the fast
-// exponential and division has a relative error of at most (5 + 1.16 |g|) FP32
-// ulps (CUDA's documented bounds for __expf and __fdividef plus three roundings),
-// i.e. at most 2 (5 + 1.16 |g|) = 10 + 2.32 |g| ulps of the result: under 19.3 for
-// |g| <= 4 and under 47.2 for |g| <= 16.  It decides unless it lies within 24 (resp.
-// 48) ulps of a BF16 midpoint, and the double expression decides otherwise and for
-// |g| > 16 (Ziv's method, as above).  Two margins keep the double path rare both for
-// gate activations of unit scale and for the wider ones of outlier weights, without
-// a float-to-integer conversion per element.
-__device__ __forceinline__ float sigmoid_fast(float g) { return __fdividef(1.0f, 1.0f + __expf(-g)); }
 
-__device__ __forceinline__ float silu_mul_round(float g, float u, float s) {
-    const float m = __fmul_rn(__fmul_rn(g, s), u);
-    // |low 16 bits - 0x8000| <= margin, as one unsigned range test
-    const float ag = fabsf(g);
-    const uint32_t margin = ag <= 4.0f ? 24u : 48u;
-    if ((__float_as_uint(m) & 0xFFFFu) + margin - 0x8000u <= 2u * margin || !(ag <= 16.0f) || !isfinite(m)) {
-        const double gd = (double)g;
-        return __bfloat162float(__double2bfloat16((gd / (1.0 + exp(-gd))) * (double)u));
-    }
-    return __bfloat162float(__float2bfloat16_rn(m));
-}
-
-__device__ __forceinline__ float silu_mul_out(float g, float u) { return silu_mul_round(g, u, sigmoid_fast(g)); }
 
 // The task loops below are software-pipelined: a warp loads the next task's inputs
 // before it computes the current one, so two tasks' loads are in flight per warp.
@@ -304,8 +321,10 @@ __global__ void __launch_bounds__(256) k_silu_mul_quant(const pact_bf16 *__restr
             unpack8_bf16(gr, gv);
             unpack8_bf16(ur, uv);
 #pragma unroll
-            for (int i = 0; i < 8; ++i) mv[i] = valid ? silu_mul_out(gv[i], uv[i]) : 0.0f;
-            if (valid && m) store8_bf16(m + row * I + c, mv);
+            for (int i = 0; i < 8; ++i) mv[i] = silu_mul_out(gv[i], uv[i]);   // zeros past the row end
+            uint4 mw;
+            round8_bf16(mv, mw, mv);
+            if (valid && m) *reinterpret_cast<uint4 *>(m + row * I + c) = mw;
             const ChunkAt at = chunk_at(row, c0, I);   // mq, gq and uq share their shape
             uint32_t sb;
             uint32_t codes = quant8(mv, &sb);
@@ -376,18 +395,30 @@ __global__ void __launch_bounds__(256) k_silu_mul_bwd_quant(const pact_bf16 *__r
             unpack8_bf16(cur.d, d);
             dequant8(cur.gc, cur.gs, gh);
             dequant8(cur.uc, cur.us, uh);
+            // dg = dm u sigma(g) (1 + g (1 - sigma(g))), du = dm g sigma(g), two values
+            // per packed FP32 operation; m~ = BF16_RNE(silu(g^) u^) exactly
             float dg[8], du[8], mr[8];
+            const uint64_t one2 = f2_pack(1.0f, 1.0f), neg2 = f2_pack(-1.0f, -1.0f);
 #pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                const float sg = sigmoid_fast(gh[i]);
-                dg[i] = __bfloat162float(__float2bfloat16_rn(d[i] * uh[i] * sg * (1.0f + gh[i] * (1.0f - sg))));
-                du[i] = __bfloat162float(__float2bfloat16_rn(d[i] * gh[i] * sg));
-                mr[i] = valid ? silu_mul_round(gh[i], uh[i], sg) : 0.0f;
+            for (int i = 0; i < 8; i += 2) {
+                const float s0 = sigmoid_fast(gh[i]), s1 = sigmoid_fast(gh[i + 1]);
+                const uint64_t g2 = f2_pack(gh[i], gh[i + 1]), sg2 = f2_pack(s0, s1);
+                const uint64_t ds = f2_mul(f2_pack(d[i], d[i + 1]), sg2);
+                const uint64_t w = f2_fma(g2, f2_fma(sg2, neg2, one2), one2);
+                f2_unpack(f2_mul(f2_mul(ds, f2_pack(uh[i], uh[i + 1])), w), dg[i], dg[i + 1]);
+                f2_unpack(f2_mul(ds, g2), du[i], du[i + 1]);
+                mr[i] = silu_mul_value<true>(gh[i], uh[i], s0);
+                mr[i + 1] = silu_mul_value<true>(gh[i + 1], uh[i + 1], s1);
             }
+            uint4 wg, wu, wm;
+            round8_bf16(dg, wg, dg);
+            round8_bf16(du, wu, du);
+            wm.x = pack_bf16x2(mr[0], mr[1]); wm.y = pack_bf16x2(mr[2], mr[3]);
+            wm.z = pack_bf16x2(mr[4], mr[5]); wm.w = pack_bf16x2(mr[6], mr[7]);
             if (valid) {
-                store8_bf16(dgu + row * lddgu + c, dg);
-                store8_bf16(dgu + row * lddgu + I + c, du);
-                if (m_re) store8_bf16(m_re + row * I + c, mr);
+                *reinterpret_cast<uint4 *>(dgu + row * lddgu + c) = wg;
+                *reinterpret_cast<uint4 *>(dgu + row * lddgu + I + c) = wu;
+                if (m_re) *reinterpret_cast<uint4 *>(m_re + row * I + c) = wm;
             }
             // du's chunk sits I columns to the right: I / 2 code bytes, and I / 64 whole
             // scale tiles (I is a multiple of 64)
@@ -428,6 +459,7 @@ __global__ void __launch_bounds__(RING_THREADS) k_rmsnorm_bwd(const pact_bf16 *_
                                                              int stages, int slot_bytes) {
     extern __shared__ __align__(128) uint8_t ring[];
     uint64_t *full = reinterpret_cast<uint64_t *>(ring + stages * slot_bytes);
+    pact_bf16 *gs = reinterpret_cast<pact_bf16 *>(ring + stages * slot_bytes + 64);   // gamma [H]
     __shared__ float red[RING_WARPS];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int64_t rows = has_dxq ? (M + 127) & ~int64_t(127) : M;
@@ -438,8 +470,10 @@ __global__ void __launch_bounds__(RING_THREADS) k_rmsnorm_bwd(const pact_bf16 *_
         for (int i = 0; i < stages; ++i) mbar_init(&full[i], 1);
         fence_barrier_init();
     }
-    __syncthreads();
     pdl_wait();
+    for (int c = 8 * threadIdx.x; c < H; c += 8 * RING_THREADS)
+        *reinterpret_cast<uint4 *>(gs + c) = *reinterpret_cast<const uint4 *>(gamma + c);
+    __syncthreads();
     auto issue = [&](int i) {   // thread 0: row i of this CTA into its slot
         const int64_t r = blockIdx.x + (int64_t)i * gridDim.x;
         if (r < M) {
@@ -461,20 +495,34 @@ __global__ void __launch_bounds__(RING_THREADS) k_rmsnorm_bwd(const pact_bf16 *_
             for (int k = warp; k < nchunk; k += RING_WARPS) zero_pad_scales(dxq, row, (int64_t)k * CHUNK);
             continue;
         }
+        // the row's scale bytes of y^ (scattered over the tiled layout) and its rstd come
+        // from global memory: loaded before the wait, so their latency overlaps it
+        const uint8_t *ysc = static_cast<const uint8_t *>(yq.scales);
+        uint32_t sc[4];
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) {
+            const int c = (warp + kk * RING_WARPS) * CHUNK + 8 * lane;
+            sc[kk] = c < H ? ysc[scale_offset(row, c >> 4, H)] : 0u;
+        }
+        const float r = rstd[row];
         ok = __syncthreads_and(ok && mbar_wait(&full[slot], (uint32_t)(i / stages) & 1u));
         if (!ok) break;
         const uint8_t *rs = ring + slot * slot_bytes;
         const pact_bf16 *dys = reinterpret_cast<const pact_bf16 *>(rs);
         const uint8_t *cs = rs + sl.codes_off;
         const pact_bf16 *rrs = reinterpret_cast<const pact_bf16 *>(rs + sl.dres_off);
-        const uint8_t *ysc = static_cast<const uint8_t *>(yq.scales);
+        auto scale_of = [&](int k, int c) -> uint32_t {   // k = warp + kk * RING_WARPS; selects, not an index
+            const int kk = (k - warp) / RING_WARPS;
+            return kk == 0 ? sc[0] : kk == 1 ? sc[1] : kk == 2 ? sc[2] : kk == 3 ? sc[3]
+                                                                        : ysc[scale_offset(row, c >> 4, H)];
+        };
         float dot = 0.0f;
         for (int k = warp; k < nchunk; k += RING_WARPS) {
             const int c = k * CHUNK + 8 * lane;
             if (c < H) {
                 float d[8], yv[8];
                 load8_bf16(dys + c, d);
-                dequant8(*reinterpret_cast<const uint32_t *>(cs + c / 2), ysc[scale_offset(row, c >> 4, H)], yv);
+                dequant8(*reinterpret_cast<const uint32_t *>(cs + c / 2), scale_of(k, c), yv);
                 // (gamma * dy) * (y^ / gamma) == dy * y^
 #pragma unroll
                 for (int j = 0; j < 8; ++j) dot = fmaf(d[j], yv[j], dot);
@@ -485,24 +533,23 @@ __global__ void __launch_bounds__(RING_THREADS) k_rmsnorm_bwd(const pact_bf16 *_
         if (lane == 0) red[warp] = dot;
         __syncthreads();
         const float mean = ((red[0] + red[1]) + (red[2] + red[3])) / (float)H;
-        const float r = rstd[row];
         for (int k = warp; k < nchunk; k += RING_WARPS) {
             const int64_t c0 = (int64_t)k * CHUNK;
             const int64_t c = c0 + 8 * lane;
             const bool valid = c < H;
-            float d[8], yv[8], g[8] = {1, 1, 1, 1, 1, 1, 1, 1}, res[8] = {0, 0, 0, 0, 0, 0, 0, 0}, o[8];
+            float d[8] = {0, 0, 0, 0, 0, 0, 0, 0}, yv[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+            float g[8] = {1, 1, 1, 1, 1, 1, 1, 1}, res[8] = {0, 0, 0, 0, 0, 0, 0, 0}, o[8];
             if (valid) {
                 load8_bf16(dys + c, d);
-                dequant8(*reinterpret_cast<const uint32_t *>(cs + c / 2), ysc[scale_offset(row, c >> 4, H)], yv);
-                load8_bf16(gamma + c, g);
+                dequant8(*reinterpret_cast<const uint32_t *>(cs + c / 2), scale_of(k, (int)c), yv);
+                load8_bf16(gs + c, g);
                 if (dres) load8_bf16(rrs + c, res);
             }
 #pragma unroll
-            for (int j = 0; j < 8; ++j) {
-                const float val = r * (g[j] * d[j] - __fdividef(yv[j], g[j]) * mean) + res[j];
-                o[j] = valid ? __bfloat162float(__float2bfloat16_rn(val)) : 0.0f;
-            }
-            if (valid) store8_bf16(dx + row * H + c, o);
+            for (int j = 0; j < 8; ++j) o[j] = r * (g[j] * d[j] - __fdividef(yv[j], g[j]) * mean) + res[j];
+            uint4 ow;
+            round8_bf16(o, ow, o);   // zeros past the row end
+            if (valid) *reinterpret_cast<uint4 *>(dx + row * H + c) = ow;
             if (has_dxq) {
                 uint32_t sb;
                 const uint32_t codes = quant8(o, &sb);
@@ -670,7 +717,7 @@ pact_status pact_rmsnorm_quant(const pact_bf16 *x, int64_t ldx, const pact_bf16 
     if (s != PACT_OK) return s;
     const int64_t rows_pad = (M + 127) / 128 * 128;
     PACT_CHECK(rows_pad <= 0x7FFFFFFF, PACT_ERR_SHAPE, "pact_rmsnorm_quant: M too large");
-    const Ring r = ring_for(rows_pad, (size_t)H * 2);
+    const Ring r = ring_for(rows_pad, (size_t)H * 2, (size_t)H * 2);
     static bool attr_done[64] = {false};
     const int d = current_device();
     if (d >= 0 && d < 64 && !attr_done[d]) {
@@ -734,7 +781,7 @@ pact_status pact_rmsnorm_bwd(const pact_bf16 *dy, int64_t lddy, const pact_nvfp4
     const int64_t rows = dxq ? (M + 127) / 128 * 128 : M;
     PACT_CHECK(rows <= 0x7FFFFFFF, PACT_ERR_SHAPE, "pact_rmsnorm_bwd: M too large");
     const BwdSlot sl = bwd_slot(H);
-    const Ring r = ring_for(rows, (size_t)(dres ? sl.dres_off + H * 2 : sl.codes_off + H / 2));
+    const Ring r = ring_for(rows, (size_t)(dres ? sl.dres_off + H * 2 : sl.codes_off + H / 2), (size_t)H * 2);
     static bool attr_done[64] = {false};
     const int d = current_device();
     if (d >= 0 && d < 64 && !attr_done[d]) {

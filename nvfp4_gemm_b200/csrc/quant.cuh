@@ -46,17 +46,20 @@ __device__ __forceinline__ float quotient(float a, float s, float r) {
     return __fmaf_rn(e, r, q0);
 }
 
-// The same quotient for a pair of values at once (packed FP32: each half is exactly
-// the scalar quotient above).  ns2 holds -s twice, r2 holds r twice.  Returns the two
-// quotients with the signs of the inputs (a -0 input keeps its sign).
-__device__ __forceinline__ void quotient2(float a0, float a1, uint64_t ns2, uint64_t r2, float &q0, float &q1) {
+// The negated quotients -(a/s) of a pair of values at once (packed FP32), with
+// s2 = (s, s) and nr2 = (-r, -r).  Round-to-nearest is symmetric in sign, so each
+// step is the negation of the corresponding step above: t = RN(a (-r)) = -RN(a r),
+// e = RN(a + t s) is the same residual, and RN(t + e (-r)) = -quotient(a, s, r).
+// Zeros come out with the sign opposite to a's (a = -0 gives +0, a = +0 gives -0),
+// so flipping the sign bit of every code afterwards yields the codes of a / s with
+// a's sign, -0 included, without a per-value sign copy.
+__device__ __forceinline__ void neg_quotient2(float a0, float a1, uint64_t s2, uint64_t nr2, float &q0, float &q1) {
     const uint64_t a = f2_pack(a0, a1);
-    const uint64_t p = f2_mul(a, r2);
-    const uint64_t e = f2_fma(p, ns2, a);
-    f2_unpack(f2_fma(e, r2, p), q0, q1);
-    q0 = copysignf(q0, a0);
-    q1 = copysignf(q1, a1);
+    const uint64_t t = f2_mul(a, nr2);
+    const uint64_t e = f2_fma(t, s2, a);
+    f2_unpack(f2_fma(e, nr2, t), q0, q1);
 }
+constexpr uint32_t CODE_SIGNS = 0x88888888u;   // the sign bit of all 8 codes of a word
 
 // Two E2M1 codes (RNE, saturating, signs kept) of a pair of quotients as one byte:
 // element 0 in the low nibble.
@@ -81,7 +84,7 @@ __device__ __forceinline__ uint32_t scale_byte(float amax) {
 // (lane ^ 1) holds the other half of the block.  All 32 lanes must call this.
 // Returns the 4 code bytes (element 0 in the low nibble of byte 0); *sb gets the
 // block's scale byte (identical in both lanes of the pair).  The quotients keep the
-// sign of x (a -0 quotient of a -0 input included), and the hardware conversion
+// sign of x (a -0 input included: see neg_quotient2), and the hardware conversion
 // rounds the magnitude and keeps the sign bit.
 __device__ __forceinline__ uint32_t quant8(const float (&v)[8], uint32_t *sb) {
     float amax = 0.0f;
@@ -90,11 +93,11 @@ __device__ __forceinline__ uint32_t quant8(const float (&v)[8], uint32_t *sb) {
     amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, 1));
     const uint32_t b = scale_byte(amax);
     const float s = e4m3_to_float(b);
-    const float r = b ? __frcp_rn(s) : 0.0f;
-    const uint64_t r2 = f2_pack(r, r), ns2 = f2_pack(-s, -s);
+    const float nr = b ? -__frcp_rn(s) : -0.0f;
+    const uint64_t nr2 = f2_pack(nr, nr), s2 = f2_pack(s, s);
     float q[8];
 #pragma unroll
-    for (int i = 0; i < 8; i += 2) quotient2(v[i], v[i + 1], ns2, r2, q[i], q[i + 1]);
+    for (int i = 0; i < 8; i += 2) neg_quotient2(v[i], v[i + 1], s2, nr2, q[i], q[i + 1]);
     uint32_t out;
     asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
         "cvt.rn.satfinite.e2m1x2.f32 b0, %2, %1;\n\t"
@@ -105,7 +108,7 @@ __device__ __forceinline__ uint32_t quant8(const float (&v)[8], uint32_t *sb) {
         : "=r"(out)
         : "f"(q[0]), "f"(q[1]), "f"(q[2]), "f"(q[3]), "f"(q[4]), "f"(q[5]), "f"(q[6]), "f"(q[7]));
     *sb = b;
-    return out;
+    return out ^ CODE_SIGNS;
 }
 
 // Quantize one NVFP4 block of 16 BF16 values held by one thread as 8 packed words
@@ -120,17 +123,17 @@ __device__ __forceinline__ void quant16_bf16(const uint4 wa, const uint4 wb, uin
     for (int j = 0; j < 8; ++j) amax = fmaxf(amax, fmaxf(fabsf(bf16lo(w[j])), fabsf(bf16hi(w[j]))));
     const uint32_t b = scale_byte(amax);
     const float s = e4m3_to_float(b);
-    const float r = b ? __frcp_rn(s) : 0.0f;
-    const uint64_t r2 = f2_pack(r, r), ns2 = f2_pack(-s, -s);
+    const float nr = b ? -__frcp_rn(s) : -0.0f;
+    const uint64_t nr2 = f2_pack(nr, nr), s2 = f2_pack(s, s);
     uint32_t out[2] = {0u, 0u};
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
         float q0, q1;
-        quotient2(bf16lo(w[j]), bf16hi(w[j]), ns2, r2, q0, q1);
+        neg_quotient2(bf16lo(w[j]), bf16hi(w[j]), s2, nr2, q0, q1);
         out[j >> 2] |= e2m1_pair(q0, q1) << (8 * (j & 3));
     }
-    *lo = out[0];
-    *hi = out[1];
+    *lo = out[0] ^ CODE_SIGNS;
+    *hi = out[1] ^ CODE_SIGNS;
     *sb = b;
 }
 
@@ -205,6 +208,49 @@ __device__ __forceinline__ void load8_nvfp4(const pact_nvfp4_t &t, int64_t row, 
     const uint32_t codes =
         *reinterpret_cast<const uint32_t *>(static_cast<const uint8_t *>(t.codes) + row * (t.cols >> 1) + (c >> 1));
     dequant8(codes, static_cast<const uint8_t *>(t.scales)[scale_offset(row, c >> 4, t.cols)], v);
+}
+
+// m = BF16_RNE(silu(g) * u), exactly rounded.  The FP32 evaluation with the fast
+// exponential and division has a relative error of at most (5 + 1.16 |g|) FP32
+// ulps (CUDA's documented bounds for __expf and __fdividef plus three roundings),
+// i.e. at most 2 (5 + 1.16 |g|) = 10 + 2.32 |g| ulps of the result: under 19.3 for
+// |g| <= 4 and under 47.2 for |g| <= 16.  It decides unless it lies within 24 (resp.
+// 48) ulps of a BF16 midpoint, and the double expression decides otherwise and for
+// |g| > 16 (Ziv's method, as above).  Two margins keep the double path rare both for
+// gate activations of unit scale and for the wider ones of outlier weights, without
+// a float-to-integer conversion per element.
+__device__ __forceinline__ float sigmoid_fast(float g) { return __fdividef(1.0f, 1.0f + __expf(-g)); }
+
+// The value whose round-to-nearest BF16 conversion is BF16_RNE(silu(g) u): the FP32
+// product where it decides, else the exactly rounded value itself (a BF16 value, so
+// converting it again changes nothing).  s = sigmoid_fast(g).  BOUNDED: u is known
+// to be finite (dequantized NVFP4), so a finite g of at most 16 gives a finite m.
+template <bool BOUNDED = false>
+__device__ __forceinline__ float silu_mul_value(float g, float u, float s) {
+    const float m = __fmul_rn(__fmul_rn(g, s), u);
+    // |low 16 bits - 0x8000| <= margin, as one unsigned range test
+    const float ag = fabsf(g);
+    const uint32_t margin = ag <= 4.0f ? 24u : 48u;
+    if ((__float_as_uint(m) & 0xFFFFu) + margin - 0x8000u <= 2u * margin || !(ag <= 16.0f) ||
+        (!BOUNDED && !isfinite(m))) {
+        const double gd = (double)g;
+        return __bfloat162float(__double2bfloat16((gd / (1.0 + exp(-gd))) * (double)u));
+    }
+    return m;
+}
+__device__ __forceinline__ float silu_mul_out(float g, float u) { return silu_mul_value(g, u, sigmoid_fast(g)); }
+
+// 8 packed BF16 values -> floats (element 0 in the low half of .x).
+__device__ __forceinline__ void unpack8_bf16(const uint4 &u, float (&v)[8]) {
+    v[0] = bf16lo(u.x); v[1] = bf16hi(u.x); v[2] = bf16lo(u.y); v[3] = bf16hi(u.y);
+    v[4] = bf16lo(u.z); v[5] = bf16hi(u.z); v[6] = bf16lo(u.w); v[7] = bf16hi(u.w);
+}
+// Round 8 values to BF16 (round to nearest even, two per conversion): the packed
+// words w (values 2j, 2j+1 in word j) and the rounded values as floats in r.
+__device__ __forceinline__ void round8_bf16(const float (&v)[8], uint4 &w, float (&r)[8]) {
+    w.x = pack_bf16x2(v[0], v[1]); w.y = pack_bf16x2(v[2], v[3]);
+    w.z = pack_bf16x2(v[4], v[5]); w.w = pack_bf16x2(v[6], v[7]);
+    unpack8_bf16(w, r);
 }
 
 // Row-major (row, 256-column chunk) tasks visited by a grid-stride loop without a

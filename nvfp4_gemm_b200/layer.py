@@ -83,10 +83,15 @@ class PactLayer:
 
     def __init__(self, shape: LayerShape, w: Dict[str, torch.Tensor], lora_a: Dict[str, torch.Tensor],
                  lora_b: Dict[str, torch.Tensor], gamma1: torch.Tensor, gamma2: torch.Tensor,
-                 two_level: bool = False, grad_fp32: bool = False):
+                 two_level: bool = False, grad_fp32: bool = False, fuse_silu: bool = False):
         self.s = shape
         self.two_level = two_level
         self.grad_fp32 = grad_fp32
+        # fuse_silu: the SiLU-multiply in the gate|up GEMM's epilogue (needs I a multiple
+        # of 256).  Off by default: at K = H = 3072 the 16 epilogue warps, not the tensor
+        # pipe, bound that kernel, and it takes longer than the GEMM that writes g|u
+        # plus the separate SiLU kernel that reads it back.
+        self.fuse_silu = fuse_silu and shape.I % 256 == 0
         S = shape
         dev = gamma1.device
         cat = lambda names, d: torch.cat([d[n] for n in names], 0).contiguous()
@@ -117,7 +122,8 @@ class PactLayer:
         self.t_qkv, self.qkv = bf(M, 2 * 3 * r), bf(M, S.n_qkv)
         self.aq, self.t_o, self.h2 = nv(M, H), bf(M, 2 * r), bf(M, H)
         self.xq2, self.x2, self.rstd2 = nv(M, H), bf(M, H), torch.empty(M, dtype=torch.float32, device=dev)
-        self.t_gu, self.gu = bf(M, 2 * 2 * r), bf(M, 2 * I)
+        self.t_gu = bf(M, 2 * 2 * r)
+        self.gu = None if self.fuse_silu else bf(M, 2 * I)
         self.m, self.mq, self.gq, self.uq = bf(M, I), nv(M, I), nv(M, I), nv(M, I)
         self.t_d, self.out = bf(M, 2 * r), bf(M, H)
         # backward
@@ -203,19 +209,29 @@ class PactLayer:
                bytes=2 * M * H + 2 * H + S.nv(M, H) + 2 * M * H + 4 * M),
             Op("lora_fwd_gu", lambda: P.pact_lora_fwd(self.x2, self.a_gu, self.sc["gu"], self.t_gu, self.ws), kernels=2,
                bytes=lora_fwd(H, 2 * r)),
-            # the gate|up GEMM also writes the NVFP4 copies gq, uq kept for the backward
-            Op("gemm_fwd_gu", lambda: P.pact_frozen_gemm_fwd_quant(self.xq2, self.c_gu, [self.gq, self.uq],
-                                                                   self.l_gu_f, y=self.gu),
-               "gemm", gemm(S.M, 2 * I, S.H), bytes=gbytes(2 * I, H, 2 * r) + 2 * S.nv(M, I)),
-            Op("silu_mul_quant", lambda: P.pact_silu_mul_quant(self.gu[:, :I], self.gu[:, I:], self.m, self.mq,
-                                                               want_copies=False),
-               bytes=4 * M * I + 2 * M * I + S.nv(M, I)),
+            *self._gate_up_ops(gemm, gbytes),
             Op("lora_fwd_down", lambda: P.pact_lora_fwd(self.m, self.a_d, self.sc["d"], self.t_d, self.ws), kernels=2,
                bytes=lora_fwd(I, r)),
             Op("gemm_fwd_down", lambda: P.pact_frozen_gemm_fwd(self.mq, self.c_d, self.l_d_f, residual=self.h2,
                                                                y=self.out),
                "gemm", gemm(S.M, S.H, I), bytes=gbytes(H, I, r) + 2 * M * H),
         ]
+
+    def _gate_up_ops(self, gemm, gbytes) -> List[Op]:
+        S, M, H, I, r = self.s, self.s.M, self.s.H, self.s.I, self.s.r
+        if self.fuse_silu:
+            # one kernel: g|u stays on chip; m, mq and the saved copies gq, uq are written
+            return [Op("gemm_fwd_silu", lambda: P.pact_frozen_gemm_fwd_silu(self.xq2, self.c_gu, self.m, self.mq,
+                                                                            self.gq, self.uq, self.l_gu_f),
+                       "gemm", gemm(S.M, 2 * I, S.H),
+                       bytes=gbytes(2 * I, H, 2 * r) - 2 * M * 2 * I + 2 * M * I + 3 * S.nv(M, I))]
+        # the gate|up GEMM also writes the NVFP4 copies gq, uq kept for the backward
+        return [Op("gemm_fwd_gu", lambda: P.pact_frozen_gemm_fwd_quant(self.xq2, self.c_gu, [self.gq, self.uq],
+                                                                       self.l_gu_f, y=self.gu),
+                   "gemm", gemm(S.M, 2 * I, S.H), bytes=gbytes(2 * I, H, 2 * r) + 2 * S.nv(M, I)),
+                Op("silu_mul_quant", lambda: P.pact_silu_mul_quant(self.gu[:, :I], self.gu[:, I:], self.m, self.mq,
+                                                                   want_copies=False),
+                   bytes=4 * M * I + 2 * M * I + S.nv(M, I))]
 
     def backward_ops(self) -> List[Op]:
         S, s, r = self.s, self.s.scale, self.s.r

@@ -78,6 +78,8 @@ def _load() -> ctypes.CDLL:
                                        P]),
         "pact_frozen_gemm_fwd_quant": (S, [NV, ctypes.POINTER(c_weight_cache), ctypes.POINTER(c_lora), P, I64, P,
                                            I64, NV, I, P]),
+        "pact_frozen_gemm_fwd_silu": (S, [NV, ctypes.POINTER(c_weight_cache), ctypes.POINTER(c_lora), P, I64, NV,
+                                          NV, NV, P]),
         "pact_lora_fwd_workspace_bytes": (ctypes.c_size_t, [I64, I64, I]),
         "pact_lora_fwd": (S, [P, I64, I64, I64, P, I, F, P, I64, P, ctypes.c_size_t, P]),
         "pact_lora_fwd_noalloc": (S, [P, I64, I64, I64, P, I, F, P, I64, P]),
@@ -188,8 +190,12 @@ class WeightCache:
 
 
 def lora_struct(act: torch.Tensor, weight: torch.Tensor, r: int, seg_end: Sequence[int]) -> c_lora:
+    """The pact_lora_t of (act, weight).  The struct holds the two tensors, so their
+    memory stays allocated for as long as the struct can reach a launch."""
     se = (ctypes.c_int64 * 4)(*(list(seg_end) + [0] * (4 - len(seg_end))))
-    return c_lora(act.data_ptr(), _ld(act), weight.data_ptr(), _ld(weight), r, len(seg_end), se)
+    c = c_lora(act.data_ptr(), _ld(act), weight.data_ptr(), _ld(weight), r, len(seg_end), se)
+    c._tensors = (act, weight)
+    return c
 
 
 # ------------------------------------------------------------------- entry points
@@ -356,6 +362,17 @@ def pact_frozen_gemm_fwd_quant(xq: NVFP4Tensor, w: WeightCache, yq: Sequence[NVF
                                            _ptr(residual), _ld(residual) if residual is not None else 0,
                                            y.data_ptr(), _ld(y), arr, len(yq), _stream(stream)))
     return y
+
+
+def pact_frozen_gemm_fwd_silu(xq: NVFP4Tensor, w: WeightCache, m: torch.Tensor, mq: NVFP4Tensor, gq: NVFP4Tensor,
+                              uq: NVFP4Tensor, lora: Optional[c_lora] = None, stream=None) -> torch.Tensor:
+    """The gate|up GEMM with the SiLU-multiply in its epilogue: m = BF16(silu(g) u)
+    and the NVFP4 copies mq, gq, uq; g and u themselves are not written."""
+    s, a, b, c = xq.c(), mq.c(), gq.c(), uq.c()
+    _check(_lib.pact_frozen_gemm_fwd_silu(ctypes.byref(s), ctypes.byref(w.cstruct),
+                                          ctypes.byref(lora) if lora is not None else None, m.data_ptr(), _ld(m),
+                                          ctypes.byref(a), ctypes.byref(b), ctypes.byref(c), _stream(stream)))
+    return m
 
 
 def pact_frozen_gemm_dgrad(dyq: NVFP4Tensor, w: WeightCache, lora: Optional[c_lora] = None,

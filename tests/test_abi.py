@@ -175,3 +175,23 @@ int main(void) {
                            "-L", lib_dir, "-lpact", f"-Wl,-rpath,{lib_dir}", "-o", str(exe)])
     out = subprocess.run([str(exe)], capture_output=True, text=True)
     assert out.returncode == 0 and out.stdout.strip() == "ok", (out.returncode, out.stdout, out.stderr)
+
+
+def test_lora_struct_keeps_its_tensors_alive(P):
+    """The descriptor carries raw device pointers; the tensors behind them must live as
+    long as the descriptor, or a later allocation could reuse their memory while a
+    GEMM still reads it."""
+    import gc
+    import weakref
+
+    import torch
+    act, w = torch.zeros(64, 32, dtype=torch.bfloat16), torch.zeros(256, 16, dtype=torch.bfloat16)
+    refs = weakref.ref(act), weakref.ref(w)
+    lo = P.lora_struct(act, w, 16, [256])
+    del act, w
+    gc.collect()
+    assert all(r() is not None for r in refs)
+    assert lo.act == refs[0]().data_ptr() and lo.weight == refs[1]().data_ptr()
+    del lo
+    gc.collect()
+    assert all(r() is None for r in refs)

@@ -271,6 +271,61 @@ def test_gemm_fwd_quant(P, orc, guards, M, parts, K, lora):
         assert_close(to_f64(y), orc.nvfp4_gemm(orc.quantize(x), wf), "fwd")
 
 
+@pytest.mark.parametrize("M,I,K,lora,two_level", [(300, 256, 512, False, False), (130, 512, 320, True, False),
+                                                   (2048, 768, 256, True, True), (1, 256, 192, False, False),
+                                                   (4096, 1280, 640, True, False)])
+def test_gemm_fwd_silu(P, orc, guards, M, I, K, lora, two_level):
+    """The gate|up GEMM with the SiLU-multiply in its epilogue: m, mq, gq, uq equal the
+    oracle's SiLU-multiply of the plain GEMM's g|u (which the fused kernel computes with
+    the same instructions) bit for bit, padding scales included; nothing past m's row
+    ends or past the copies' buffers is written."""
+    N = 2 * I
+    x = synth.gaussian_bf16(1, (M, K))
+    w = synth.weight_bf16(0, (N, K), outliers=True)
+    wc = P.pact_weight_layout_cache(to_dev(w), two_level=two_level)
+    xq = P.pact_quantize_nvfp4(to_dev(x))
+    lo = None
+    if lora:
+        r = 16
+        a = synth.gaussian_bf16(20, (2 * r, K), std=0.02)
+        b = synth.gaussian_bf16(30, (N, r), std=0.02)
+        T = P.pact_lora_fwd(to_dev(x), to_dev(a), 2.0 * 2.0 ** -wc.gexp)
+        lo = P.lora_struct(T, to_dev(b), r, [I, N])
+    m = guards.matrix(M, I, pad_cols=8)
+    mq, gq, uq = guards.nvfp4(M, I), guards.nvfp4(M, I), guards.nvfp4(M, I)
+    P.pact_frozen_gemm_fwd_silu(xq, wc, m, mq, gq, uq, lora=lo)
+    gu = P.pact_frozen_gemm_fwd(xq, wc, lora=lo)
+    sync()
+    status_ok(P)
+    gub = to_bits(gu)
+    m_ref, mq_ref, gq_ref, uq_ref = orc.silu_mul_quant(gub[:, :I], gub[:, I:])
+    assert np.array_equal(to_bits(m), m_ref), "m"
+    assert_nvfp4_equal(mq, mq_ref, orc, "mq")
+    assert_nvfp4_equal(gq, gq_ref, orc, "gq")
+    assert_nvfp4_equal(uq, uq_ref, orc, "uq")
+    if not lora and not two_level:
+        wf, _ = orc.weight_cache(w)
+        assert_close(to_f64(gu), orc.nvfp4_gemm(orc.quantize(x), wf), "g|u")
+
+
+def test_gemm_fwd_silu_rejects_bad_shapes(P):
+    """I must be a multiple of 256 (the gate and up tiles pair up); the copies must
+    be [M x I]."""
+    x = torch.zeros((64, 128), dtype=torch.bfloat16, device="cuda")
+    xq = P.pact_quantize_nvfp4(x)
+    wc = P.pact_weight_layout_cache(torch.zeros((2 * 320, 128), dtype=torch.bfloat16, device="cuda"))
+    m = torch.empty((64, 320), dtype=torch.bfloat16, device="cuda")
+    q = [P.NVFP4Tensor.empty(64, 320, torch.device("cuda")) for _ in range(3)]
+    with pytest.raises(P.PactError):
+        P.pact_frozen_gemm_fwd_silu(xq, wc, m, *q)
+    wc = P.pact_weight_layout_cache(torch.zeros((512, 128), dtype=torch.bfloat16, device="cuda"))
+    q = [P.NVFP4Tensor.empty(64, 128, torch.device("cuda")) for _ in range(3)]
+    with pytest.raises(P.PactError):
+        P.pact_frozen_gemm_fwd_silu(xq, wc, torch.empty((64, 256), dtype=torch.bfloat16, device="cuda"), *q)
+    sync()
+    status_ok(P)
+
+
 # ------------------------------------------------------------------------- LoRA
 @pytest.mark.parametrize("M,parts,r,K", [(256, [512], 16, 384), (300, [512, 256, 256], 16, 576),
                                          (130, [256, 320], 32, 320), (2048, [1024], 16, 2112)])

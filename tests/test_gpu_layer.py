@@ -5,11 +5,16 @@ error downstream.  NVFP4 codes/scales and BF16 values the method rounds exactly
 (RMSNorm and SiLU-multiply outputs) must match bit for bit; GEMM and LoRA outputs
 must satisfy |gpu - oracle| <= 8e-3 |oracle| + 1e-3 rms(oracle).
 
-The full-size case runs the bench's workload (Llama-3.2-1B layer, 2048 tokens) in
+The full-size case runs the bench's workload (Llama-3.2-3B layer, 8192 tokens) in
 the launch configuration bench.py times (the same op list captured into one CUDA
 graph, the LoRA weight gradients on a parallel branch); the frozen GEMM outputs are
 checked on sampled rows the oracle computes one by one, everything else in full,
-and the graph's results must equal an eager sequential step bit for bit."""
+and the graph's results must equal an eager sequential step bit for bit.
+
+With the SiLU-multiply fused into the gate|up GEMM, g|u never reaches memory; the
+check recomputes it with the plain GEMM call on the layer's own xq2 and T, which
+issues the same tensor-core instructions per tile and so yields the same bits, and
+then holds m, mq, gq, uq to the oracle's SiLU-multiply of those bits."""
 import numpy as np
 import pytest
 import torch
@@ -28,7 +33,7 @@ def _bits(t):
     return to_bits(t)
 
 
-def run_layer(name, M, graphs, two_level=False):
+def run_layer(name, M, graphs, two_level=False, fuse_silu=False):
     import nvfp4_gemm_b200 as P
     from nvfp4_gemm_b200.layer import LayerShape, PactLayer
     c = synth.LAYERS[name]
@@ -38,7 +43,7 @@ def run_layer(name, M, graphs, two_level=False):
     shape = LayerShape(M=M, H=c["H"], I=c["I"], KV=c["KV"])
     L = PactLayer(shape, {k: d(v) for k, v in inp["w"].items()}, {k: d(v) for k, v in inp["lora_a"].items()},
                   {k: d(v) for k, v in inp["lora_b"].items()}, d(inp["gamma1"]), d(inp["gamma2"]),
-                  two_level=two_level)
+                  two_level=two_level, fuse_silu=fuse_silu)
     L.bind(d(inp["h"]), d(inp["attn"]), d(inp["d_out"]), d(inp["d_qkv"]))
     ops = L.step_ops()
     if graphs:
@@ -147,8 +152,15 @@ def check_layer(L, inp, orc, rows):
     nv_equal(L.xq2, xq2, "xq2")
     t_gu = hilo(L.t_gu)
     assert_close(t_gu, sc["gu"] * orc.gemm_nt(f(y2), A["gu"]), "T gu")
-    assert_close(to_f64(L.gu)[sel], p2["gu"] * (gemm_rows(xq2, wf["gu"]) + lora_rows(t_gu, "gu", True)), "gate|up")
-    gu = _bits(L.gu)
+    if L.gu is None:
+        import nvfp4_gemm_b200 as P
+        gu_dev = P.pact_frozen_gemm_fwd(L.xq2, L.c_gu, L.l_gu_f)
+        torch.cuda.synchronize()
+    else:
+        gu_dev = L.gu
+    assert_close(to_f64(gu_dev)[sel], p2["gu"] * (gemm_rows(xq2, wf["gu"]) + lora_rows(t_gu, "gu", True)),
+                 "gate|up")
+    gu = _bits(gu_dev)
     m, mq, gq, uq = orc.silu_mul_quant(gu[:, :I], gu[:, I:])
     assert np.array_equal(_bits(L.m), m), "m"
     nv_equal(L.mq, mq, "mq")
@@ -213,9 +225,10 @@ def small_layer(monkeypatch):
     return "tiny"
 
 
-@pytest.mark.parametrize("graphs", [False, True])
-def test_layer_small_all_rows(orc, small_layer, graphs):
-    L, inp = run_layer(small_layer, 300, graphs)
+@pytest.mark.parametrize("graphs,fuse", [(False, False), (False, True), (True, True)])
+def test_layer_small_all_rows(orc, small_layer, graphs, fuse):
+    L, inp = run_layer(small_layer, 300, graphs, fuse_silu=fuse)
+    assert L.fuse_silu == fuse
     check_layer(L, inp, orc, rows=None)
     assert L.saved_bytes() == orc.saved_bytes_pact(300, L.s.H, L.s.I)
 
@@ -228,20 +241,23 @@ def test_layer_small_two_level(orc, small_layer):
     check_layer(L, inp, orc, rows=None)
 
 
-@pytest.mark.parametrize("name", ["qwen2.5-1.5b", "llama-3.2-3b"])
-def test_layer_full_size(orc, name):
-    """The other two layer workloads (Qwen2.5-1.5B at 2048 tokens; Llama-3.2-3B at
-    8192 tokens with 1% x20 weight outliers) in the bench's launch configuration."""
-    L, inp = run_layer(name, synth.tokens(name), graphs=True)
+@pytest.mark.parametrize("name,fuse", [("qwen2.5-1.5b", True), ("llama-3.2-1b", False)])
+def test_layer_full_size(orc, name, fuse):
+    """The other two layer workloads (Qwen2.5-1.5B, I = 8960 = 35 x 256, with the
+    SiLU-multiply in the gate|up GEMM's epilogue, and Llama-3.2-1B, each at 2048
+    tokens) in the bench's launch configuration."""
+    L, inp = run_layer(name, synth.tokens(name), graphs=True, fuse_silu=fuse)
     assert L.saved_bytes() == orc.saved_bytes_pact(L.s.M, L.s.H, L.s.I)
     rows = np.sort(np.random.default_rng(12).choice(L.s.M, size=32, replace=False))
     rows[-1] = L.s.M - 1
     check_layer(L, inp, orc, rows=rows)
 
 
-def test_layer_llama1b_full_size(orc):
-    """The bench workload itself, in the bench's launch configuration."""
-    L, inp = run_layer("llama-3.2-1b", synth.tokens("llama-3.2-1b"), graphs=True)
+def test_layer_bench_workload_full_size(orc):
+    """The bench workload itself (Llama-3.2-3B at 8192 tokens, 1% x20 weight
+    outliers), in the bench's launch configuration."""
+    L, inp = run_layer("llama-3.2-3b", synth.tokens("llama-3.2-3b"), graphs=True, fuse_silu=False)
+    assert not L.fuse_silu and L.saved_bytes() == orc.saved_bytes_pact(L.s.M, L.s.H, L.s.I)
     # the concurrent graph step and an eager sequential step agree bit for bit
     snap = {k: v.clone() for k, v in L.grads.items()}
     outs = {"out": L.out.clone(), "dh": L.dh.clone(), "dattn": L.dattn.clone()}
