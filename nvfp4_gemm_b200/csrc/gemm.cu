@@ -296,8 +296,10 @@ k_nvfp4_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CU
             }
         }
     } else if (warp == 1) {
-        // ------------------------------------------------------------ MMA issuer (leader, one thread)
-        if (leader && lane == 0) {
+        // ------------------------------------------------------------ MMA issuer (leader)
+        // The whole warp runs this loop converged (waits, ring position, descriptors are
+        // warp-uniform); lane 0 alone issues the MMAs and commits (the _w forms).
+        if (leader) {
             const uint32_t idesc = idesc_nvf4(2 * BM, BN);
             const uint32_t idesc_lora = idesc_bf16(2 * BM, BN, false, p.lora_mode == LORA_DGRAD);
             // operand descriptors of stage 0, K step 0; a stage / K step adds its byte
@@ -308,16 +310,29 @@ k_nvfp4_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CU
             uint32_t acc_phase = 0;
             bool ok = true;
             for (int t = first_tile(p, cluster); ok && t < total; t = next_tile(p, t, nclusters)) {
-                ok = mbar_wait(acc_empty, acc_phase ^ 1);
+                ok = warp_all(mbar_wait(acc_empty, acc_phase ^ 1));
                 tc_fence_after();
                 uint32_t accum = 0;
-                // Per stage: its MMAs, the commit that frees the stage once they are done,
-                // then the next stage's barrier (a non-blocking test first: the producers
-                // run stages ahead).  The ring position lives in registers here.
+                // Per stage: its MMAs and the commit that frees the stage once they are
+                // done.  Stage barriers are observed in batches: when no observed stage is
+                // left, the thread waits for the next one and tests the two after it
+                // without blocking (the producers run stages ahead); one fence covers the
+                // batch, whose MMAs are then issued back to back.  The ring position lives
+                // in registers here.
                 uint32_t stage = rg.stage, phase = rg.phase;
-                bool ready = nsteps > 0 && (ok = mbar_wait(&full[stage], phase));
-                tc_fence_after();
-                for (int i = 0; ready && i < nsteps; ++i) {
+                int known = 0;   // observed, fenced stages from step i on
+                for (int i = 0; i < nsteps; ++i) {
+                    if (known == 0) {
+                        if (!(ok = warp_all(mbar_wait(&full[stage], phase)))) break;
+                        const uint32_t s1 = stage + 1 == STAGES ? 0 : stage + 1;
+                        const uint32_t p1 = stage + 1 == STAGES ? phase ^ 1 : phase;
+                        const uint32_t s2 = s1 + 1 == STAGES ? 0 : s1 + 1;
+                        const uint32_t p2 = s1 + 1 == STAGES ? p1 ^ 1 : p1;
+                        const bool r1 = i + 1 < nsteps && warp_all(mbar_test_wait(&full[s1], p1));
+                        const bool r2 = r1 && i + 2 < nsteps && warp_all(mbar_test_wait(&full[s2], p2));
+                        known = 1 + (r1 ? 1 + (r2 ? 1 : 0) : 0);
+                        tc_fence_after();
+                    }
                     const uint32_t st = smem_u32(smem) + stage * STAGE_BYTES;
                     if (lora && i == 0) {
                         const int R = p.lora_nseg * p.lora_r;
@@ -327,7 +342,7 @@ k_nvfp4_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CU
                                                     : smem_desc(st + OFF_LW + c * 2048, R * 128, 1024, SW_128);
                             for (int h = 0; h < 2; ++h) {  // hi part, then lo part
                                 const uint64_t ad = smem_desc(st + (h * p.lora_steps + c) * BM * 32, 16, 256, SW_32);
-                                mma_bf16_pair(tmem + COL_ACC, ad, bd, idesc_lora, accum);
+                                mma_bf16_pair_w(tmem + COL_ACC, ad, bd, idesc_lora, accum);
                                 accum = 1;
                             }
                         }
@@ -340,37 +355,34 @@ k_nvfp4_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CU
                         if (nk == BK / KSTEP) {
 #pragma unroll
                             for (int s = 0; s < BK / KSTEP; ++s) {
-                                mma_nvf4_pair(tmem + COL_ACC, ad + 2 * s, bd + 2 * s, idesc, sf + 4 * s, sf + 16 + 8 * s,
+                                mma_nvf4_pair_w(tmem + COL_ACC, ad + 2 * s, bd + 2 * s, idesc, sf + 4 * s, sf + 16 + 8 * s,
                                               accum);
                                 accum = 1;
                             }
                         } else {
                             for (int s = 0; s < nk; ++s) {
-                                mma_nvf4_pair(tmem + COL_ACC, ad + 2 * s, bd + 2 * s, idesc, sf + 4 * s, sf + 16 + 8 * s,
+                                mma_nvf4_pair_w(tmem + COL_ACC, ad + 2 * s, bd + 2 * s, idesc, sf + 4 * s, sf + 16 + 8 * s,
                                               accum);
                                 accum = 1;
                             }
                         }
                     }
-                    tc_commit_pair(&empty[stage], 3);
+                    tc_commit_pair_w(&empty[stage], 3);
+                    --known;
                     if (++stage == STAGES) {
                         stage = 0;
                         phase ^= 1;
-                    }
-                    if (i + 1 < nsteps) {
-                        if (!mbar_test_wait(&full[stage], phase)) ready = ok = mbar_wait(&full[stage], phase);
-                        tc_fence_after();
                     }
                 }
                 rg.stage = stage;
                 rg.phase = phase;
                 if (!ok) break;
-                tc_commit_pair(acc_full, 3);
+                tc_commit_pair_w(acc_full, 3);
                 acc_phase ^= 1;
             }
             // tensor memory is released below only after every MMA issued here has completed
-            tc_commit_pair(drained, 1);
-            mbar_wait(drained, 0);
+            tc_commit_pair_w(drained, 1);
+            warp_all(mbar_wait(drained, 0));
         }
         __syncwarp();
     } else if (warp < 2 + SCALE_WARPS) {
