@@ -16,23 +16,17 @@
 //    leader (rank 0) issues every MMA for the pair.  Each SM streams 38 KiB per
 //    K = 256 stage, 30% less than a single-CTA 128 x 256 tile needs, which keeps
 //    the L2 -> shared-memory stream below what the tensor core consumes.
-//  * warp 0 (both CTAs): TMA producer of the operand tiles into a 4-stage ring; they
-//    complete on the leader's `full` barrier (armed by the leader for both CTAs'
-//    bytes).
-//  * warp 22 (both CTAs): scale-tile producer.  It refills a stage's scale tiles
-//    (local `sf_full` barrier) as soon as the scale writers have read the previous
-//    ones (`sf_empty`), ahead of the operand tiles.
-//  * warps 2-5 (both CTAs): scale writers.  Each moves the stage's scale tiles from
-//    shared memory into a per-stage slot of its own sub-partition's tensor memory
-//    with tcgen05.st (once the slot's previous MMAs are done) and arrives on the
-//    leader's `full` barrier of the stage, which therefore completes only when
-//    operands and scales of both CTAs are in place.
-//    Writing scales from registers keeps them out of the tensor core's instruction
-//    stream; tcgen05.cp copies there serialise with the MMAs and cost more than
-//    the MMAs themselves.
-//  * warp 1, lane 0 (leader): one barrier wait per stage, then the LoRA MMAs
-//    (kind::f16) or 4 NVFP4 MMAs, committed to both CTAs' `empty` barriers.
-//  * warps 6-21 (both CTAs): epilogue, four warps per tensor-memory sub-partition,
+//  * warp 0 (both CTAs): TMA producer into a 4-stage ring: per stage the operand
+//    tiles and the stage's scale tiles, all completing on the leader's `full`
+//    barrier (armed by the leader for both CTAs' bytes).
+//  * warp 1 (leader; the whole warp runs the loop, lane 0 issues): barrier waits in
+//    batches, then per stage the LoRA MMAs (kind::f16), or per K = 64 step the three
+//    tcgen05.cp copies of that step's scale chunks from shared memory into the
+//    stage's tensor-memory scale slot (32 rows x 16 bytes each, replicated into the
+//    four sub-partitions) followed by the NVFP4 MMA; the stage is committed to both
+//    CTAs' `empty` barriers.  Copies and MMAs of one thread execute in issue order,
+//    so the scales need no synchronisation of their own.
+//  * warps 2-17 (both CTAs): epilogue, four warps per tensor-memory sub-partition,
 //    64 columns each.  A warp loads its 32 x 64 block of the accumulator into
 //    registers and releases the accumulator at once, so the pair's next tile starts
 //    while the warp adds the residual (prefetched by TMA into the warp's 4 KiB
@@ -58,14 +52,12 @@ constexpr int SF_BYTES = 2048 + 4096;
 constexpr int STAGE_BYTES = OFF_SFB + 4096;   // 38912 = 38 KiB
 constexpr int OFF_LW = 6 * BM * 32;           // LoRA weight chunks follow 6 activation chunks
 static_assert(OFF_LW + 3 * BM * 32 <= STAGE_BYTES && OFF_LW + 2 * 48 * 128 <= STAGE_BYTES, "LoRA stage");
-constexpr int SCALE_WARPS = 4;
 constexpr int EPI_WARPS = 16;
 constexpr int SLAB_BYTES = 32 * 128;          // 32 rows x 64 BF16 columns, 128-byte swizzle
 constexpr int OFF_SLABS = STAGES * STAGE_BYTES;
 constexpr int OFF_BARS = OFF_SLABS + EPI_WARPS * SLAB_BYTES;
 constexpr int SMEM_BYTES = 1024 + OFF_BARS + 512;
-constexpr int SF_WARP = 2 + SCALE_WARPS + EPI_WARPS;          // 22: scale-tile producer
-constexpr int THREADS = 32 * (SF_WARP + 1);                   // 736
+constexpr int THREADS = 32 * (2 + EPI_WARPS);                 // 576
 static_assert(SMEM_BYTES <= 232448, "shared memory");
 
 // tensor memory columns
@@ -194,10 +186,8 @@ k_nvfp4_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CU
     uint8_t *smem = smem_raw + (((raw + 1023) & ~1023u) - raw);
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + OFF_BARS);
     uint64_t *full = bars;                        // [STAGES] leader: operands and scales of both CTAs
-    uint64_t *sf_full = bars + STAGES;            // [STAGES] local: this CTA's scale tiles in shared memory
-    uint64_t *empty = bars + 2 * STAGES;          // [STAGES] local: the pair's MMAs are done with the stage
-    uint64_t *sf_empty = bars + 3 * STAGES;       // [STAGES] local: the scale writers have read the scale tiles
-    uint64_t *acc_full = bars + 4 * STAGES;       // local: accumulator complete
+    uint64_t *empty = bars + STAGES;              // [STAGES] local: the pair's MMAs are done with the stage
+    uint64_t *acc_full = bars + 2 * STAGES;       // local: accumulator complete
     uint64_t *acc_empty = acc_full + 1;           // leader: all epilogue warps of both CTAs have read it
     uint64_t *drained = acc_full + 2;             // leader: every tcgen05 operation has completed
     uint64_t *res_full = acc_full + 3;            // [EPI_WARPS] local: residual block in the warp's slab
@@ -216,10 +206,8 @@ k_nvfp4_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CU
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
-            mbar_init(&full[s], 1 + 2 * SCALE_WARPS);
-            mbar_init(&sf_full[s], 1);
+            mbar_init(&full[s], 1);
             mbar_init(&empty[s], 1);
-            mbar_init(&sf_empty[s], SCALE_WARPS);
         }
         mbar_init(acc_full, 1);
         mbar_init(acc_empty, 2 * EPI_WARPS);
@@ -284,13 +272,20 @@ k_nvfp4_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CU
                     }
                     rg.next();
                 }
+                // scale map rows: 2 per 512-byte chunk; this CTA's 128-row group of A,
+                // both 128-row groups of the B tile
+                const int ga = m0 / 128, gb = n0 / 128;
                 for (int kt = 0; kt < ktiles; ++kt) {
                     if (!(ok = mbar_wait(&empty[rg.stage], rg.phase ^ 1))) break;
                     const uint32_t st = smem_u32(smem + rg.stage * STAGE_BYTES);
                     const uint32_t fb = full_leader + 8 * rg.stage;
-                    if (leader) mbar_arrive_expect_tx(&full[rg.stage], 2 * (A_BYTES + B_BYTES));
+                    if (leader) mbar_arrive_expect_tx(&full[rg.stage], 2 * (A_BYTES + B_BYTES + SF_BYTES));
                     tma_load_2d_pair(st, &tmA, fb, kt * (BK / 2), m0);
                     tma_load_2d_pair(st + OFF_B, &tmB, fb, kt * (BK / 2), nb);
+                    // the stage's scale chunks (one box = the 4 chunks of this K stage)
+                    tma_load_2d_pair(st + OFF_SFA, &tmSFA, fb, 0, 2 * (ga * kgroups + kt * 4));
+                    tma_load_2d_pair(st + OFF_SFB, &tmSFB, fb, 0, 2 * (gb * kgroups + kt * 4));
+                    tma_load_2d_pair(st + OFF_SFB + 2048, &tmSFB, fb, 0, 2 * ((gb + 1) * kgroups + kt * 4));
                     rg.next();
                 }
             }
@@ -352,15 +347,25 @@ k_nvfp4_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CU
                         const uint32_t sf = tmem + COL_SF + stage * SF_COLS;
                         const uint64_t ad = adesc0 + (uint64_t)((stage * STAGE_BYTES) >> 4);
                         const uint64_t bd = bdesc0 + (uint64_t)((stage * STAGE_BYTES) >> 4);
+                        // K step s: scale chunks s of A (columns 4s..4s+3 of the slot) and of
+                        // the two 128-row groups of B (16 + 8s + 4g), then its MMA
+                        const uint32_t sc = st + OFF_SFA;
+                        auto copy_scales = [&](int s) {
+                            tmem_cp_pair_32x128b_x4_w(sf + 4 * s, smem_desc(sc + s * 512, 0, 128, SW_NONE));
+                            tmem_cp_pair_32x128b_x4_w(sf + 16 + 8 * s, smem_desc(sc + 2048 + s * 512, 0, 128, SW_NONE));
+                            tmem_cp_pair_32x128b_x4_w(sf + 20 + 8 * s, smem_desc(sc + 4096 + s * 512, 0, 128, SW_NONE));
+                        };
                         if (nk == BK / KSTEP) {
 #pragma unroll
                             for (int s = 0; s < BK / KSTEP; ++s) {
+                                copy_scales(s);
                                 mma_nvf4_pair_w(tmem + COL_ACC, ad + 2 * s, bd + 2 * s, idesc, sf + 4 * s, sf + 16 + 8 * s,
                                               accum);
                                 accum = 1;
                             }
                         } else {
                             for (int s = 0; s < nk; ++s) {
+                                copy_scales(s);
                                 mma_nvf4_pair_w(tmem + COL_ACC, ad + 2 * s, bd + 2 * s, idesc, sf + 4 * s, sf + 16 + 8 * s,
                                               accum);
                                 accum = 1;
@@ -385,92 +390,9 @@ k_nvfp4_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CU
             warp_all(mbar_wait(drained, 0));
         }
         __syncwarp();
-    } else if (warp < 2 + SCALE_WARPS) {
-        // ------------------------------------------------------------ scale writers (both CTAs)
-        const int sub = warp & 3;  // tensor-memory sub-partition this warp may access
-        const uint32_t full_leader = mapa_shared(smem_u32(full), 0);
-        const uint32_t lane_base = tmem + ((uint32_t)(sub * 32) << 16);
-        Ring rg;
-        bool ok = true;
-        for (int t = first_tile(p, cluster); ok && t < total; t = next_tile(p, t, nclusters)) {
-            for (int i = 0; i < nsteps; ++i) {
-                const bool lstep = lora && i == 0;   // a LoRA stage carries no scales
-                if (!(ok = warp_all(mbar_wait(&sf_full[rg.stage], rg.phase)))) break;
-                uint32_t v[48];
-                if (!lstep) {
-                    // Lane j takes the 16 bytes of row j of every 512-byte chunk: the
-                    // chunk's 4 scale columns for lanes j of each sub-partition, the
-                    // layout the block-scaled MMA reads.
-                    const uint8_t *src = smem + rg.stage * STAGE_BYTES + OFF_SFA + lane * 16;
-#pragma unroll
-                    for (int c = 0; c < 12; ++c) {  // A chunks 0-3, then B: step s, group g at 4 + 2s + g
-                        const int off = c < 4 ? c * 512 : 2048 + ((c - 4) & 1) * 2048 + ((c - 4) >> 1) * 512;
-                        const uint4 q = *reinterpret_cast<const uint4 *>(src + off);
-                        v[4 * c] = q.x; v[4 * c + 1] = q.y; v[4 * c + 2] = q.z; v[4 * c + 3] = q.w;
-                    }
-                }
-                // the tensor-memory slot is free once the pair's MMAs of its previous use
-                // are done
-                if (!(ok = warp_all(mbar_wait(&empty[rg.stage], rg.phase ^ 1)))) break;
-                if (!lstep) {
-                    const uint32_t col = lane_base + COL_SF + rg.stage * SF_COLS;
-                    tmem_st_32x32b_x32(col, v);
-                    tmem_st_32x32b_x16(col + 32, v + 32);
-                    tmem_st_wait();
-                }
-                // The scale tiles may be refilled now: their values have been consumed,
-                // and releasing them only after the previous use's MMAs are done keeps
-                // the producer within one phase of every barrier it waits on.
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&sf_empty[rg.stage]);
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive_remote_relaxed(full_leader + 8 * rg.stage);
-                rg.next();
-            }
-        }
-    } else if (warp == SF_WARP) {
-        // ------------------------------------------------------------ scale-tile producer (both CTAs)
-        // Refills a stage's scale tiles as soon as the scale writers have consumed the
-        // previous ones (one use earlier than the operand tiles, which wait for that
-        // use's MMAs): the TMA latency of the scales leaves the chain MMA done ->
-        // refill -> scales in tensor memory -> MMA.  After a LoRA stage (whose weight
-        // chunks overlap the scale region) it also waits for that stage's MMAs.
-        if (lane == 0) {
-            Ring rg;
-            uint32_t lora_prev = 0;   // bit s: the previous use of stage s was a LoRA stage
-            bool ok = true;
-            for (int t = first_tile(p, cluster); ok && t < total; t = next_tile(p, t, nclusters)) {
-                int mp, nt;
-                tile_coords(p, t, mpairs, ntiles, mp, nt);
-                const int ga = (mp * 2 * BM + (int)rank * BM) / 128, gb = (nt * BN) / 128;
-                for (int i = 0; ok && i < nsteps; ++i) {
-                    const uint32_t sb = 1u << rg.stage;
-                    if (!(ok = mbar_wait(&sf_empty[rg.stage], rg.phase ^ 1))) break;
-                    if ((lora_prev & sb) && !(ok = mbar_wait(&empty[rg.stage], rg.phase ^ 1))) break;
-                    if (lora && i == 0) {
-                        mbar_arrive(&sf_full[rg.stage]);
-                        lora_prev |= sb;
-                    } else {
-                        const int kt = i - (lora ? 1 : 0);
-                        uint8_t *stp = smem + rg.stage * STAGE_BYTES;
-                        // scale chunks: 512 bytes = two 256-byte rows of the scale map; one
-                        // box is the 4 chunks of this K stage
-                        mbar_arrive_expect_tx(&sf_full[rg.stage], SF_BYTES);
-                        tma_load_2d(stp + OFF_SFA, &tmSFA, &sf_full[rg.stage], 0, 2 * (ga * kgroups + kt * 4));
-                        tma_load_2d(stp + OFF_SFB, &tmSFB, &sf_full[rg.stage], 0, 2 * (gb * kgroups + kt * 4));
-                        tma_load_2d(stp + OFF_SFB + 2048, &tmSFB, &sf_full[rg.stage], 0,
-                                    2 * ((gb + 1) * kgroups + kt * 4));
-                        lora_prev &= ~sb;
-                    }
-                    rg.next();
-                }
-            }
-        }
-        __syncwarp();
     } else {
         // ------------------------------------------------------------ epilogue (both CTAs)
-        const int ew = warp - 2 - SCALE_WARPS;   // 0..15
+        const int ew = warp - 2;                 // 0..15
         const int sub = warp & 3;                // tensor-memory sub-partition this warp may read
         const int quarter = ew >> 2;             // columns 64*quarter .. 64*quarter+63 of the tile
         const uint32_t acc_empty_leader = mapa_shared(smem_u32(acc_empty), 0);

@@ -24,7 +24,7 @@ namespace lmma {
 
 constexpr int BM = 128;        // output rows per CTA (MMA M)
 constexpr int BK = 64;         // contraction elements per stage (128 bytes of BF16)
-constexpr int MAX_STAGES = 3;  // ring depth
+constexpr int MAX_STAGES = 6;  // ring depth: 6, or 3 where two CTAs should share an SM
 constexpr int THREADS = 192;
 constexpr int A_BYTES = BM * BK * 2;     // 16384
 constexpr int B_BYTES = 64 * BK * 2;     // 8192 per B part
@@ -36,24 +36,19 @@ constexpr int RAW_BYTES = RAW_CODE_BYTES + 1024;
 // A stage holds the A tile, one or two B parts (the hi and lo halves of T or U) and,
 // for an NVFP4 A, its staging area; all multiples of 1024 bytes.
 __host__ __device__ constexpr int oper_bytes(int nparts) { return A_BYTES + nparts * B_BYTES; }
-// one 64-wide slice of the contraction (a sub-tile): its operands and staging area
 __host__ __device__ constexpr int stage_bytes(int nparts, bool fp4) { return oper_bytes(nparts) + (fp4 ? RAW_BYTES : 0); }
-// Sub-tiles per ring stage: the one-part products move two per barrier round trip (the
-// per-stage wait, fence and commit of the MMA warp are paid once per 128 contraction
-// elements); the two-part products keep one so that two CTAs fit on an SM.
-__host__ __device__ constexpr int sub_for(int nparts) { return nparts == 2 ? 1 : 2; }
 __host__ __device__ constexpr int smem_bytes(int nparts, bool fp4, int stages) {
-    return 1024 + stages * sub_for(nparts) * stage_bytes(nparts, fp4) + 256;
+    return 1024 + stages * stage_bytes(nparts, fp4) + 256;
 }
 constexpr int SM_SMEM = 233472;   // shared memory per SM (228 KiB), 1 KiB of it reserved per CTA
 __host__ __device__ constexpr int ctas_per_sm(int nparts, bool fp4, int stages) {
     return SM_SMEM / (smem_bytes(nparts, fp4, stages) + 1024);
 }
-// Ring depth: 3 stages.  The weight-gradient products (contraction over the tokens, two
-// B parts) fit two CTAs on an SM; the forward and U products (contraction over the
-// features) run one CTA per SM with 3 x 2 sub-tiles in flight, where more splits would
-// cost more in FP32 partial-sum traffic than they gain.
-__host__ __device__ constexpr int stages_for(int nparts) { return 3; }
+// Ring depth per product: the weight-gradient products (contraction over the tokens,
+// two B parts) run 3 stages so that two CTAs share an SM; the forward and U products
+// (contraction over the features) run one CTA per SM with 6 stages in flight, where
+// more splits would cost more in FP32 partial-sum traffic than they gain.
+__host__ __device__ constexpr int stages_for(int nparts) { return nparts == 2 ? 3 : 6; }
 constexpr int FWD_PER_SM = 1;   // split residency of the one-part products
 constexpr uint32_t TMEM_COLS = 64;
 
@@ -146,16 +141,13 @@ template <bool A_MN, bool B_MN, bool A_FP4>
 __global__ void __launch_bounds__(THREADS, 1)
 k_lora_mma(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, const Params p) {
     const int nparts = p.b_split ? 2 : 1;
-    // a ring stage holds SUB sub-tiles of SUB_BYTES each
-    const int SUB = sub_for(nparts), SUB_BYTES = stage_bytes(nparts, A_FP4), OPER_BYTES = oper_bytes(nparts);
-    const int STAGE_BYTES = SUB * SUB_BYTES;
+    const int STAGE_BYTES = stage_bytes(nparts, A_FP4), OPER_BYTES = oper_bytes(nparts);
     const Prob pr = p.prob[blockIdx.z];
     const int row0 = pr.row_begin + blockIdx.x * BM;
     if (row0 >= pr.row_end) return;  // block-uniform, before any shared state
     const int kb = pr.k_begin + blockIdx.y * p.k_per_split;
     const int ke = min(pr.k_end, kb + p.k_per_split);
-    const int ktiles = ke > kb ? (ke - kb + BK - 1) / BK : 0;   // 64-wide sub-tiles
-    const int nstages = (ktiles + SUB - 1) / SUB;               // ring stages to run
+    const int ktiles = ke > kb ? (ke - kb + BK - 1) / BK : 0;
     float *part = p.ws + (size_t)blockIdx.y * p.ws_split_stride;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
@@ -203,49 +195,45 @@ k_lora_mma(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUte
     if (warp == 0) {
         if (lane == 0) {
             uint32_t stage = 0, phase = 0, pending = 0, pending_parity = 0, raw_pending = 0;
-            const int64_t chunks_per_group = p.a_cols / 64;
-            // the second half's scale chunk of an MN-major NVFP4 A exists only while its columns do
-            const uint32_t mn_sbytes = (A_MN && row0 / 64 + 1 < chunks_per_group) ? 1024u : 512u;
-            for (int ks = 0; ks < nstages; ++ks) {
+            for (int kt = 0; kt < ktiles; ++kt) {
                 if (!mbar_wait(&empty[stage], phase ^ 1)) break;
-                const int nsub = min(SUB, ktiles - ks * SUB);
-                // one arrival per barrier and stage, for all of the stage's sub-tiles
+                uint8_t *st = smem + stage * STAGE_BYTES;
+                const int k = kb + kt * BK;
                 if (A_FP4) {
-                    mbar_arrive_expect_tx(&raw_full[stage], nsub * (RAW_CODE_BYTES + (A_MN ? mn_sbytes : 512u)));
-                    mbar_arrive_expect_tx(&full[stage], nsub * nparts * b_bytes);
+                    // codes box and the scale chunk(s) of this stage's A tile
+                    uint8_t *rw = st + OPER_BYTES;
+                    const int64_t chunks_per_group = p.a_cols / 64;
+                    if (!A_MN) {
+                        mbar_arrive_expect_tx(&raw_full[stage], RAW_CODE_BYTES + 512);
+                        tma_load_2d(rw, &tmA, &raw_full[stage], k / 2, row0);
+                        bulk_load(rw + RAW_CODE_BYTES,
+                                  p.a_scales + ((int64_t)(row0 / 128) * chunks_per_group + k / 64) * 512, 512,
+                                  &raw_full[stage]);
+                    } else {
+                        // the second half's chunk exists only while its columns do
+                        const uint32_t sbytes = (row0 / 64 + 1 < chunks_per_group) ? 1024u : 512u;
+                        mbar_arrive_expect_tx(&raw_full[stage], RAW_CODE_BYTES + sbytes);
+                        tma_load_2d(rw, &tmA, &raw_full[stage], row0 / 2, k);
+                        bulk_load(rw + RAW_CODE_BYTES,
+                                  p.a_scales + ((int64_t)(k / 128) * chunks_per_group + row0 / 64) * 512, sbytes,
+                                  &raw_full[stage]);
+                    }
+                    raw_pending |= 1u << stage;
+                    mbar_arrive_expect_tx(&full[stage], nparts * b_bytes);
                 } else {
-                    mbar_arrive_expect_tx(&full[stage], nsub * (A_BYTES + nparts * b_bytes));
-                }
-                for (int j = 0; j < nsub; ++j) {
-                    uint8_t *st = smem + stage * STAGE_BYTES + j * SUB_BYTES;
-                    const int k = kb + (ks * SUB + j) * BK;
-                    if (A_FP4) {
-                        // codes box and the scale chunk(s) of this sub-tile's A tile
-                        uint8_t *rw = st + OPER_BYTES;
-                        if (!A_MN) {
-                            tma_load_2d(rw, &tmA, &raw_full[stage], k / 2, row0);
-                            bulk_load(rw + RAW_CODE_BYTES,
-                                      p.a_scales + ((int64_t)(row0 / 128) * chunks_per_group + k / 64) * 512, 512,
-                                      &raw_full[stage]);
-                        } else {
-                            tma_load_2d(rw, &tmA, &raw_full[stage], row0 / 2, k);
-                            bulk_load(rw + RAW_CODE_BYTES,
-                                      p.a_scales + ((int64_t)(k / 128) * chunks_per_group + row0 / 64) * 512,
-                                      mn_sbytes, &raw_full[stage]);
-                        }
-                    } else if (A_MN) {
+                    mbar_arrive_expect_tx(&full[stage], A_BYTES + nparts * b_bytes);
+                    if (A_MN) {
                         tma_load_2d(st, &tmA, &full[stage], row0, k);
                         tma_load_2d(st + A_BYTES / 2, &tmA, &full[stage], row0 + 64, k);
                     } else {
                         tma_load_2d(st, &tmA, &full[stage], k, row0);
                     }
-                    for (int h = 0; h < nparts; ++h) {
-                        uint8_t *bd = st + A_BYTES + h * B_BYTES;
-                        if (B_MN) tma_load_2d(bd, &tmB, &full[stage], pr.b_coord + h * p.b_lo_off, k);
-                        else tma_load_2d(bd, &tmB, &full[stage], k, pr.b_coord);
-                    }
                 }
-                if (A_FP4) raw_pending |= 1u << stage;
+                for (int h = 0; h < nparts; ++h) {
+                    uint8_t *bd = st + A_BYTES + h * B_BYTES;
+                    if (B_MN) tma_load_2d(bd, &tmB, &full[stage], pr.b_coord + h * p.b_lo_off, k);
+                    else tma_load_2d(bd, &tmB, &full[stage], k, pr.b_coord);
+                }
                 pending |= 1u << stage;
                 pending_parity = (pending_parity & ~(1u << stage)) | (phase << stage);
                 if (++stage == STAGES) { stage = 0; phase ^= 1; }
@@ -264,23 +252,20 @@ k_lora_mma(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUte
         const uint32_t idesc = idesc_bf16(BM, p.n_mma, A_MN, B_MN);
         uint32_t stage = 0, phase = 0, accum = 0;
         // the whole warp runs the loop converged; lane 0 alone issues (the _w forms)
-        for (int ks = 0; ks < nstages; ++ks) {
+        for (int kt = 0; kt < ktiles; ++kt) {
             const bool ok = warp_all(mbar_wait(&full[stage], phase));
             tc_fence_after();
             if (!ok) break;
-            const int nsub = min(SUB, ktiles - ks * SUB);
-            for (int j = 0; j < nsub; ++j) {
-                const uint32_t st = smem_u32(smem + stage * STAGE_BYTES + j * SUB_BYTES);
-                for (int s = 0; s < BK / 16; ++s) {
-                    const uint64_t ad = A_MN ? smem_desc(st + s * 2048, A_BYTES / 2, 1024, SW_128)
-                                             : smem_desc(st + s * 32, 16, 1024, SW_128);
-                    for (int h = 0; h < nparts; ++h) {
-                        const uint32_t b0 = st + A_BYTES + h * B_BYTES;
-                        const uint64_t bd = B_MN ? smem_desc(b0 + s * 2048, B_BYTES, 1024, SW_128)
-                                                 : smem_desc(b0 + s * 32, 16, 1024, SW_128);
-                        mma_bf16_w(tmem, ad, bd, idesc, accum);
-                        accum = 1;
-                    }
+            const uint32_t st = smem_u32(smem + stage * STAGE_BYTES);
+            for (int s = 0; s < BK / 16; ++s) {
+                const uint64_t ad = A_MN ? smem_desc(st + s * 2048, A_BYTES / 2, 1024, SW_128)
+                                         : smem_desc(st + s * 32, 16, 1024, SW_128);
+                for (int h = 0; h < nparts; ++h) {
+                    const uint32_t b0 = st + A_BYTES + h * B_BYTES;
+                    const uint64_t bd = B_MN ? smem_desc(b0 + s * 2048, B_BYTES, 1024, SW_128)
+                                             : smem_desc(b0 + s * 32, 16, 1024, SW_128);
+                    mma_bf16_w(tmem, ad, bd, idesc, accum);
+                    accum = 1;
                 }
             }
             tc_commit_w(&empty[stage]);
@@ -297,13 +282,10 @@ k_lora_mma(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUte
             // tensor core reads shared memory through the async proxy)
             const int tid = threadIdx.x - 64;
             uint32_t stage = 0, phase = 0;
-            for (int ks = 0; ks < nstages; ++ks) {
+            for (int kt = 0; kt < ktiles; ++kt) {
                 if (!(ok = warp_all(mbar_wait(&raw_full[stage], phase)))) break;
-                const int nsub = min(SUB, ktiles - ks * SUB);
-                for (int j = 0; j < nsub; ++j) {
-                    uint8_t *st = smem + stage * STAGE_BYTES + j * SUB_BYTES;
-                    decode_stage<A_MN>(st + OPER_BYTES, st, p, row0, kb + (ks * SUB + j) * BK, tid);
-                }
+                uint8_t *st = smem + stage * STAGE_BYTES;
+                decode_stage<A_MN>(st + OPER_BYTES, st, p, row0, kb + kt * BK, tid);
                 fence_proxy_async_smem();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&full[stage]);
