@@ -47,8 +47,10 @@ __host__ __device__ constexpr int ctas_per_sm(int nparts, bool fp4, int stages) 
 // Ring depth per product: the weight-gradient products (contraction over the tokens,
 // two B parts) run 3 stages so that two CTAs share an SM; the forward and U products
 // (contraction over the features) run one CTA per SM with 6 stages in flight, where
-// more splits would cost more in FP32 partial-sum traffic than they gain.
-__host__ __device__ constexpr int stages_for(int nparts) { return nparts == 2 ? 3 : 6; }
+// more splits would cost more in FP32 partial-sum traffic than they gain.  A product
+// whose A operand is decoded from NVFP4 in the kernel is bound by the decoding warps,
+// so it runs 3 stages and two CTAs per SM (twice the decoders).
+__host__ __device__ constexpr int stages_for(int nparts, bool fp4) { return nparts == 2 || fp4 ? 3 : 6; }
 constexpr int FWD_PER_SM = 1;   // split residency of the one-part products
 constexpr uint32_t TMEM_COLS = 64;
 
@@ -163,7 +165,7 @@ k_lora_mma(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUte
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = smem_u32(smem_raw);
     uint8_t *smem = smem_raw + (((raw + 1023) & ~1023u) - raw);
-    const int STAGES = stages_for(nparts);
+    const int STAGES = stages_for(nparts, A_FP4);
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + STAGES * STAGE_BYTES);
     uint64_t *full = bars, *empty = bars + MAX_STAGES, *acc_full = bars + 2 * MAX_STAGES;
     uint64_t *raw_full = bars + 2 * MAX_STAGES + 1;   // [stages], A_FP4 only
@@ -424,10 +426,11 @@ static pact_status launch_mma(const CUtensorMap &ta, const CUtensorMap &tb, cons
     static bool done[64] = {false};
     const int d = current_device();
     const int np = p.b_split ? 2 : 1;
-    const int smem = smem_bytes(np, A_FP4, stages_for(np));
+    const int smem = smem_bytes(np, A_FP4, stages_for(np, A_FP4));
     if (d >= 0 && d < 64 && !done[d]) {
         int mx = 0;
-        for (int n = 1; n <= 2; ++n) mx = mx > smem_bytes(n, A_FP4, stages_for(n)) ? mx : smem_bytes(n, A_FP4, stages_for(n));
+        for (int n = 1; n <= 2; ++n)
+            mx = mx > smem_bytes(n, A_FP4, stages_for(n, A_FP4)) ? mx : smem_bytes(n, A_FP4, stages_for(n, A_FP4));
         cudaError_t e = cudaFuncSetAttribute(k_lora_mma<A_MN, B_MN, A_FP4>, cudaFuncAttributeMaxDynamicSharedMemorySize, mx);
         if (e != cudaSuccess) return fail(PACT_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
         done[d] = true;
@@ -491,7 +494,7 @@ static pact_status rows_times_a(const CUtensorMap &tx, const pact_nvfp4_t *xq, i
     p.nprob = 1;
     p.prob[0] = Prob{0, (int)M, 0, (int)K, 0, 0};
     const int tiles = (int)((M + BM - 1) / BM);
-    choose_split(K, tiles, FWD_PER_SM, &p.splits, &p.k_per_split);
+    choose_split(K, tiles, xq ? ctas_per_sm(1, true, stages_for(1, true)) : FWD_PER_SM, &p.splits, &p.k_per_split);
     p.ws = ws;
     p.ws_ld = R;
     p.ws_split_stride = M * R;
@@ -531,8 +534,13 @@ static int splits_of(int64_t len, int64_t blocks, int per_sm) {
 
 // Workspace bounds cover both the BF16 and the NVFP4 form of X~ (more CTAs per SM
 // give at least as many splits).
-constexpr int T_PER_SM = FWD_PER_SM;
-constexpr int DA_PER_SM = ctas_per_sm(2, false, stages_for(2)) > ctas_per_sm(2, true, stages_for(2)) ? ctas_per_sm(2, false, stages_for(2)) : ctas_per_sm(2, true, stages_for(2));
+// residency of the T~ product: the NVFP4-decoding form fits more CTAs per SM (splits
+// and workspace are sized for the larger of the two)
+constexpr int T_PER_SM = ctas_per_sm(1, true, stages_for(1, true)) > FWD_PER_SM ? ctas_per_sm(1, true, stages_for(1, true))
+                                                                                 : FWD_PER_SM;
+constexpr int DA_PER_SM = ctas_per_sm(2, false, stages_for(2, false)) > ctas_per_sm(2, true, stages_for(2, true))
+                              ? ctas_per_sm(2, false, stages_for(2, false))
+                              : ctas_per_sm(2, true, stages_for(2, true));
 
 size_t pact_lora_fwd_workspace_bytes(int64_t M, int64_t K, int R) {
     return partial_bytes(M, R, splits_of(K, (M + BM - 1) / BM, FWD_PER_SM));
@@ -608,7 +616,7 @@ size_t pact_lora_bwd_workspace_bytes(int64_t M, int64_t N, int64_t K, int r, int
     const int64_t R = (int64_t)r * nseg;
     return partial_bytes(M, R, splits_of(K, (M + BM - 1) / BM, T_PER_SM))      /* T~ partials */
            + round256((size_t)(M * 2 * R * 2))                                  /* T~ hi/lo */
-           + partial_bytes(N, r, splits_of(M, (N + BM - 1) / BM, ctas_per_sm(2, false, stages_for(2))))  /* dB partials */
+           + partial_bytes(N, r, splits_of(M, (N + BM - 1) / BM, ctas_per_sm(2, false, stages_for(2, false))))  /* dB partials */
            + partial_bytes(K, R, splits_of(M, (K + BM - 1) / BM, DA_PER_SM));  /* dA^T partials */
 }
 
@@ -644,7 +652,7 @@ pact_status pact_lora_bwd(const pact_lora_bwd_t *g, void *workspace, size_t ws_b
     pact_bf16 *tt = reinterpret_cast<pact_bf16 *>(w8);
     w8 += round256((size_t)(M * 2 * R * 2));
     float *ws_db = reinterpret_cast<float *>(w8);
-    w8 += partial_bytes(N, r, splits_of(M, (N + BM - 1) / BM, ctas_per_sm(2, false, stages_for(2))));
+    w8 += partial_bytes(N, r, splits_of(M, (N + BM - 1) / BM, ctas_per_sm(2, false, stages_for(2, false))));
     float *ws_da = reinterpret_cast<float *>(w8);
 
     // X~ is read where it lies: BF16 rows, or the saved NVFP4 copy decoded in shared
@@ -676,7 +684,7 @@ pact_status pact_lora_bwd(const pact_lora_bwd_t *g, void *workspace, size_t ws_b
         }
         pb.b_split = 1;
         pb.b_lo_off = R;
-        choose_split(M, blocks, ctas_per_sm(2, false, stages_for(2)), &pb.splits, &pb.k_per_split);
+        choose_split(M, blocks, ctas_per_sm(2, false, stages_for(2, false)), &pb.splits, &pb.k_per_split);
         pb.ws = ws_db;
         pb.ws_ld = r;
         pb.ws_split_stride = N * r;
@@ -697,7 +705,7 @@ pact_status pact_lora_bwd(const pact_lora_bwd_t *g, void *workspace, size_t ws_b
     p.b_split = 1;
     p.b_lo_off = R;
     const int tiles = (int)((K + BM - 1) / BM);
-    choose_split(M, tiles, ctas_per_sm(2, g->xq != nullptr, stages_for(2)), &p.splits, &p.k_per_split);
+    choose_split(M, tiles, ctas_per_sm(2, g->xq != nullptr, stages_for(2, g->xq != nullptr)), &p.splits, &p.k_per_split);
     p.ws = ws_da;
     p.ws_ld = R;
     p.ws_split_stride = K * R;
