@@ -26,6 +26,9 @@ constexpr int BM = 128;        // output rows per CTA (MMA M)
 constexpr int BK = 64;         // contraction elements per stage (128 bytes of BF16)
 constexpr int MAX_STAGES = 6;  // ring depth: 6, or 3 where two CTAs should share an SM
 constexpr int THREADS = 192;
+// With an NVFP4 A operand, two groups of four decoding warps take alternate stages
+// (the decode, not the MMA or the copies, bounds those products).
+__host__ __device__ constexpr int threads_for(bool fp4) { return fp4 ? THREADS + 128 : THREADS; }
 constexpr int A_BYTES = BM * BK * 2;     // 16384
 constexpr int B_BYTES = 64 * BK * 2;     // 8192 per B part
 // NVFP4 A operand: per stage, the codes of the A tile (128 x 64 values, 4 KiB) and
@@ -140,7 +143,7 @@ __device__ __forceinline__ void decode_stage(const uint8_t *raw, uint8_t *oper, 
 }
 
 template <bool A_MN, bool B_MN, bool A_FP4>
-__global__ void __launch_bounds__(THREADS, 1)
+__global__ void __launch_bounds__(threads_for(A_FP4), 1)
 k_lora_mma(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, const Params p) {
     const int nparts = p.b_split ? 2 : 1;
     const int STAGE_BYTES = stage_bytes(nparts, A_FP4), OPER_BYTES = oper_bytes(nparts);
@@ -155,7 +158,7 @@ k_lora_mma(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUte
 
     if (ktiles == 0) {  // empty split: its partial is zero
         pdl_wait();
-        for (int i = threadIdx.x; i < BM * p.n_valid; i += THREADS) {
+        for (int i = threadIdx.x; i < BM * p.n_valid; i += blockDim.x) {
             const int r = row0 + i / p.n_valid;
             if (r < pr.row_end) part[(size_t)r * p.ws_ld + pr.out_col + i % p.n_valid] = 0.0f;
         }
@@ -170,6 +173,7 @@ k_lora_mma(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUte
     uint64_t *full = bars, *empty = bars + MAX_STAGES, *acc_full = bars + 2 * MAX_STAGES;
     uint64_t *raw_full = bars + 2 * MAX_STAGES + 1;   // [stages], A_FP4 only
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 3 * MAX_STAGES + 1);
+    __shared__ uint32_t aborted;   // a bounded wait gave up somewhere in the CTA
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
@@ -179,6 +183,7 @@ k_lora_mma(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUte
             mbar_init(&raw_full[s], 1);
         }
         mbar_init(acc_full, 1);
+        aborted = 0;
         fence_barrier_init();
         prefetch_tensormap(&tmA);
         prefetch_tensormap(&tmB);
@@ -198,7 +203,10 @@ k_lora_mma(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUte
         if (lane == 0) {
             uint32_t stage = 0, phase = 0, pending = 0, pending_parity = 0, raw_pending = 0;
             for (int kt = 0; kt < ktiles; ++kt) {
-                if (!mbar_wait(&empty[stage], phase ^ 1)) break;
+                if (!mbar_wait(&empty[stage], phase ^ 1)) {
+                    aborted = 1;
+                    break;
+                }
                 uint8_t *st = smem + stage * STAGE_BYTES;
                 const int k = kb + kt * BK;
                 if (A_FP4) {
@@ -257,7 +265,10 @@ k_lora_mma(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUte
         for (int kt = 0; kt < ktiles; ++kt) {
             const bool ok = warp_all(mbar_wait(&full[stage], phase));
             tc_fence_after();
-            if (!ok) break;
+            if (!ok) {
+                aborted = 1;
+                break;
+            }
             const uint32_t st = smem_u32(smem + stage * STAGE_BYTES);
             for (int s = 0; s < BK / 16; ++s) {
                 const uint64_t ad = A_MN ? smem_desc(st + s * 2048, A_BYTES / 2, 1024, SW_128)
@@ -282,18 +293,26 @@ k_lora_mma(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUte
             // decode each stage's NVFP4 A tile into the BF16 operand buffer, then
             // announce it on the stage's `full` barrier (after a proxy fence: the
             // tensor core reads shared memory through the async proxy)
-            const int tid = threadIdx.x - 64;
-            uint32_t stage = 0, phase = 0;
-            for (int kt = 0; kt < ktiles; ++kt) {
-                if (!(ok = warp_all(mbar_wait(&raw_full[stage], phase)))) break;
+            const int group = (warp - 2) >> 2;             // stages group, group + 2, ...
+            const int tid = threadIdx.x - 64 - 128 * group;
+            for (int kt = group; kt < ktiles; kt += 2) {
+                const int stage = kt % STAGES;
+                const uint32_t phase = (uint32_t)(kt / STAGES) & 1u;
+                if (!(ok = warp_all(mbar_wait(&raw_full[stage], phase)))) {
+                    aborted = 1;
+                    break;
+                }
                 uint8_t *st = smem + stage * STAGE_BYTES;
                 decode_stage<A_MN>(st + OPER_BYTES, st, p, row0, kb + kt * BK, tid);
                 fence_proxy_async_smem();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&full[stage]);
-                if (++stage == STAGES) { stage = 0; phase ^= 1; }
             }
         }
+    }
+    if (warp >= 2 && warp < 6) {
+        // the epilogue: warps 2-5, one tensor-memory sub-partition each
+        bool ok = true;
         const int sub = warp & 3;
         ok = mbar_wait(acc_full, 0) && ok;
         tc_fence_after();
@@ -317,6 +336,13 @@ k_lora_mma(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUte
     if (warp == 1) {
         tc_fence_after();
         tmem_dealloc(tmem, TMEM_COLS);
+    }
+    if (aborted && warp >= 2 && warp < 6) {
+        // some role of this CTA gave up a wait: its partial tile is NaN, whatever the
+        // accumulator held
+        const int r = row0 + (warp & 3) * 32 + lane;
+        if (r < pr.row_end)
+            for (int c = 0; c < p.n_valid; ++c) part[(size_t)r * p.ws_ld + pr.out_col + c] = __int_as_float(0x7fc00000);
     }
 }
 
@@ -436,7 +462,7 @@ static pact_status launch_mma(const CUtensorMap &ta, const CUtensorMap &tb, cons
         done[d] = true;
     }
     dim3 grid((unsigned)row_tiles, (unsigned)p.splits, (unsigned)p.nprob);
-    return launch_dep(k_lora_mma<A_MN, B_MN, A_FP4>, grid, dim3(THREADS), smem, st, what, ta, tb, p);
+    return launch_dep(k_lora_mma<A_MN, B_MN, A_FP4>, grid, dim3(threads_for(A_FP4)), smem, st, what, ta, tb, p);
 }
 
 static FinJob fin_job(const float *ws, const Params &p, int64_t rows, int64_t cols, float scale, int mode,
