@@ -22,46 +22,63 @@ __device__ __forceinline__ void zero_pad_scales(const pact_nvfp4_t &t, int64_t r
 }
 
 // ------------------------------------------------------------------ A2: quantize
-// prescale: a power of two the values are multiplied by first (exact in FP32); 1
-// for every quantization on the step path, 2^-gexp for two-level weight layouts.
+// A warp task is 512 columns of a row: lane j quantizes the 16-value block j on its
+// own (no block-maximum shuffle, one scale computation per block), writes its 8 code
+// bytes and its scale byte.  prescale: a power of two the values are multiplied by
+// first (exact in FP32); 1 for every quantization on the step path, 2^-gexp for
+// two-level weight layouts.
+constexpr int QCHUNK = 512;
 __global__ void __launch_bounds__(256) k_quantize(const pact_bf16 *__restrict__ x, int64_t ldx, int64_t rows,
                                                   pact_nvfp4_t out, float prescale) {
     pdl_wait();
     const int lane = threadIdx.x & 31;
-    const int64_t nchunk = (out.cols + CHUNK - 1) / CHUNK;
+    const int64_t nchunk = (out.cols + QCHUNK - 1) / QCHUNK;
     const int64_t rows_pad = (rows + 127) & ~int64_t(127);
     const int64_t warp0 = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
     const int64_t nwarps = (int64_t)gridDim.x * (blockDim.x >> 5);
-    auto load = [&](const TaskIter &t) {
-        const int64_t c = t.chunk * CHUNK + 8 * lane;
-        return (t.row < rows && c < out.cols) ? *reinterpret_cast<const uint4 *>(x + t.row * ldx + c)
-                                              : make_uint4(0, 0, 0, 0);
+    uint8_t *codes = static_cast<uint8_t *>(out.codes), *scales = static_cast<uint8_t *>(out.scales);
+    auto load = [&](const TaskIter &t, uint4 &a, uint4 &b) {
+        const int64_t c = t.chunk * QCHUNK + 16 * lane;
+        a = b = make_uint4(0, 0, 0, 0);
+        if (t.row < rows && c < out.cols) {
+            const uint4 *p = reinterpret_cast<const uint4 *>(x + t.row * ldx + c);
+            a = p[0];
+            b = p[1];
+        }
     };
     TaskIter it(warp0, nchunk, nwarps);
-    uint4 cur = make_uint4(0, 0, 0, 0);
-    if (it.row < rows_pad) cur = load(it);
-    while (it.row < rows_pad) {    // software-pipelined: the next task's load is in flight
+    uint4 ca, cb;
+    if (it.row < rows_pad) load(it, ca, cb);
+    while (it.row < rows_pad) {    // software-pipelined: the next task's loads are in flight
         TaskIter nx = it;
         nx.next();
-        const uint4 nxt = nx.row < rows_pad ? load(nx) : make_uint4(0, 0, 0, 0);
+        uint4 na = make_uint4(0, 0, 0, 0), nb = make_uint4(0, 0, 0, 0);
+        if (nx.row < rows_pad) load(nx, na, nb);
         const int64_t row = it.row;
-        const int64_t c0 = it.chunk * CHUNK;
-        if (row >= rows) {
-            zero_pad_scales(out, row, c0);
-        } else {
-            const bool valid = c0 + 8 * lane < out.cols;
-            float v[8];
-            unpack8_bf16(cur, v);
-            if (prescale != 1.0f) {   // uniform over the launch
+        const int64_t c = it.chunk * QCHUNK + 16 * lane;
+        if (c < out.cols) {
+            uint8_t *sp = scales + scale_offset(row, c >> 4, out.cols);
+            if (row >= rows) {
+                *sp = 0;   // a padding row of the scale layout
+            } else {
+                uint32_t lo, hi, sb;
+                if (prescale != 1.0f) {   // uniform over the launch; the FP32 products are exact
+                    float v[16];
+                    unpack8_bf16(ca, *reinterpret_cast<float(*)[8]>(v));
+                    unpack8_bf16(cb, *reinterpret_cast<float(*)[8]>(v + 8));
 #pragma unroll
-                for (int i = 0; i < 8; ++i) v[i] *= prescale;
+                    for (int i = 0; i < 16; ++i) v[i] *= prescale;
+                    quant16_f32(v, &lo, &hi, &sb);
+                } else {
+                    quant16_bf16(ca, cb, &lo, &hi, &sb);
+                }
+                *reinterpret_cast<uint2 *>(codes + row * (out.cols >> 1) + (c >> 1)) = make_uint2(lo, hi);
+                *sp = (uint8_t)sb;
             }
-            uint32_t sb;
-            const uint32_t codes = quant8(v, &sb);
-            store_chunk(out, row, c0, codes, sb, valid);
         }
         it = nx;
-        cur = nxt;
+        ca = na;
+        cb = nb;
     }
 }
 
@@ -86,14 +103,23 @@ __global__ void __launch_bounds__(256) k_absmax_bf16(const pact_bf16 *__restrict
     if ((threadIdx.x & 31) == 0) atomicMax(amax, __float_as_uint(m));
 }
 
-static int grid_for(int64_t warp_tasks, int threads) {
+static int grid_for(int64_t warp_tasks, int threads, int per_sm = 8) {
     const int sms = sm_count();
     const int64_t per_block = threads / 32;
     int64_t blocks = (warp_tasks + per_block - 1) / per_block;
-    const int64_t cap = (int64_t)sms * 8;
+    const int64_t cap = (int64_t)sms * per_sm;
     if (blocks > cap) blocks = cap;
     if (blocks < 1) blocks = 1;
     return (int)blocks;
+}
+
+// Blocks of `kernel` (256 threads, no dynamic shared memory) resident on one SM: the
+// grid-stride kernels launch one wave of them, so no block waits behind another.
+template <typename K>
+static int resident_per_sm(K kernel) {
+    int n = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kernel, 256, 0) != cudaSuccess || n < 1) n = 1;
+    return n;
 }
 
 // ------------------------------------------------------- A3: RMSNorm + quantize
@@ -282,95 +308,37 @@ __global__ void __launch_bounds__(RING_THREADS) k_rmsnorm_quant(const pact_bf16 
 
 // The task loops below are software-pipelined: a warp loads the next task's inputs
 // before it computes the current one, so two tasks' loads are in flight per warp.
+// A task is 512 columns of a row; lane j owns the 16-value block j of every tensor
+// (one scale computation per block, no block-maximum shuffle).
 __global__ void __launch_bounds__(256) k_silu_mul_quant(const pact_bf16 *__restrict__ g, const pact_bf16 *__restrict__ u,
                                                         int64_t ld_gu, int64_t M, int64_t I,
                                                         pact_bf16 *__restrict__ m, pact_nvfp4_t mq, pact_nvfp4_t gq,
                                                         pact_nvfp4_t uq, int has_gq, int has_uq) {
     pdl_wait();
     const int lane = threadIdx.x & 31;
-    const int64_t nchunk = (I + CHUNK - 1) / CHUNK;
-    const int64_t rows_pad = (M + 127) & ~int64_t(127);
-    const int64_t warp0 = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
-    const int64_t nwarps = (int64_t)gridDim.x * (blockDim.x >> 5);
-    auto load = [&](const TaskIter &t, uint4 &gr, uint4 &ur) {
-        const int64_t c = t.chunk * CHUNK + 8 * lane;
-        gr = ur = make_uint4(0, 0, 0, 0);
-        if (t.row < M && c < I) {
-            gr = *reinterpret_cast<const uint4 *>(g + t.row * ld_gu + c);
-            ur = *reinterpret_cast<const uint4 *>(u + t.row * ld_gu + c);
-        }
-    };
-    TaskIter it(warp0, nchunk, nwarps);
-    uint4 gr, ur;
-    if (it.row < rows_pad) load(it, gr, ur);
-    while (it.row < rows_pad) {
-        TaskIter nx = it;
-        nx.next();
-        uint4 gn = make_uint4(0, 0, 0, 0), un = make_uint4(0, 0, 0, 0);
-        if (nx.row < rows_pad) load(nx, gn, un);
-        const int64_t row = it.row;
-        const int64_t c0 = it.chunk * CHUNK;
-        if (row >= M) {
-            zero_pad_scales(mq, row, c0);
-            if (has_gq) zero_pad_scales(gq, row, c0);
-            if (has_uq) zero_pad_scales(uq, row, c0);
-        } else {
-            const int64_t c = c0 + 8 * lane;
-            const bool valid = c < I;
-            float gv[8], uv[8], mv[8];
-            unpack8_bf16(gr, gv);
-            unpack8_bf16(ur, uv);
-#pragma unroll
-            for (int i = 0; i < 8; ++i) mv[i] = silu_mul_out(gv[i], uv[i]);   // zeros past the row end
-            uint4 mw;
-            round8_bf16(mv, mw, mv);
-            if (valid && m) *reinterpret_cast<uint4 *>(m + row * I + c) = mw;
-            const ChunkAt at = chunk_at(row, c0, I);   // mq, gq and uq share their shape
-            uint32_t sb;
-            uint32_t codes = quant8(mv, &sb);
-            store_chunk_at(mq, at, codes, sb, valid);
-            if (has_gq) {
-                codes = quant8(gv, &sb);
-                store_chunk_at(gq, at, codes, sb, valid);
-            }
-            if (has_uq) {
-                codes = quant8(uv, &sb);
-                store_chunk_at(uq, at, codes, sb, valid);
-            }
-        }
-        it = nx;
-        gr = gn;
-        ur = un;
-    }
-}
-
-// ---------------------------------------------- A9: SiLU-multiply backward + quantize
-__global__ void __launch_bounds__(256) k_silu_mul_bwd_quant(const pact_bf16 *__restrict__ dm, int64_t lddm,
-                                                            pact_nvfp4_t gq, pact_nvfp4_t uq, int64_t M, int64_t I,
-                                                            pact_bf16 *__restrict__ dgu, int64_t lddgu,
-                                                            pact_nvfp4_t dguq, pact_bf16 *__restrict__ m_re) {
-    pdl_wait();
-    const int lane = threadIdx.x & 31;
-    const int64_t nchunk = (I + CHUNK - 1) / CHUNK;
+    const int64_t nchunk = (I + QCHUNK - 1) / QCHUNK;
     const int64_t rows_pad = (M + 127) & ~int64_t(127);
     const int64_t warp0 = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
     const int64_t nwarps = (int64_t)gridDim.x * (blockDim.x >> 5);
     struct In {
-        uint4 d;
-        uint32_t gc, uc, gs, us;
+        uint4 g0, g1, u0, u1;
     };
     auto load = [&](const TaskIter &t, In &v) {
-        const int64_t c = t.chunk * CHUNK + 8 * lane;
-        v.d = make_uint4(0, 0, 0, 0);
-        v.gc = v.uc = v.gs = v.us = 0;
+        const int64_t c = t.chunk * QCHUNK + 16 * lane;
+        v.g0 = v.g1 = v.u0 = v.u1 = make_uint4(0, 0, 0, 0);
         if (t.row < M && c < I) {
-            v.d = *reinterpret_cast<const uint4 *>(dm + t.row * lddm + c);
-            // gq and uq share their shape: one code offset, one scale offset
-            const int64_t co = t.row * (I >> 1) + (c >> 1), so = scale_offset(t.row, c >> 4, I);
-            v.gc = *reinterpret_cast<const uint32_t *>(static_cast<const uint8_t *>(gq.codes) + co);
-            v.uc = *reinterpret_cast<const uint32_t *>(static_cast<const uint8_t *>(uq.codes) + co);
-            v.gs = static_cast<const uint8_t *>(gq.scales)[so];
-            v.us = static_cast<const uint8_t *>(uq.scales)[so];
+            const uint4 *gp = reinterpret_cast<const uint4 *>(g + t.row * ld_gu + c);
+            const uint4 *up = reinterpret_cast<const uint4 *>(u + t.row * ld_gu + c);
+            v.g0 = gp[0]; v.g1 = gp[1]; v.u0 = up[0]; v.u1 = up[1];
+        }
+    };
+    // m for 8 values (one 16-byte piece of g and of u): the values to round, in mv
+    auto silu8 = [&](const uint4 &gw, const uint4 &uw, float (&mv)[8]) {
+        const uint32_t gs[4] = {gw.x, gw.y, gw.z, gw.w}, us[4] = {uw.x, uw.y, uw.z, uw.w};
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            mv[2 * j] = silu_mul_out(bf16lo(gs[j]), bf16lo(us[j]));
+            mv[2 * j + 1] = silu_mul_out(bf16hi(gs[j]), bf16hi(us[j]));
         }
     };
     TaskIter it(warp0, nchunk, nwarps);
@@ -380,55 +348,157 @@ __global__ void __launch_bounds__(256) k_silu_mul_bwd_quant(const pact_bf16 *__r
         TaskIter nx = it;
         nx.next();
         In nxt;
-        nxt.d = make_uint4(0, 0, 0, 0);
-        nxt.gc = nxt.uc = nxt.gs = nxt.us = 0;
         if (nx.row < rows_pad) load(nx, nxt);
+        else nxt.g0 = nxt.g1 = nxt.u0 = nxt.u1 = make_uint4(0, 0, 0, 0);
         const int64_t row = it.row;
-        const int64_t c0 = it.chunk * CHUNK;
-        if (row >= M) {
-            zero_pad_scales(dguq, row, c0);
-            zero_pad_scales(dguq, row, c0 + I);
-        } else {
-            const int64_t c = c0 + 8 * lane;
-            const bool valid = c < I;
-            float d[8], gh[8], uh[8];
-            unpack8_bf16(cur.d, d);
-            dequant8(cur.gc, cur.gs, gh);
-            dequant8(cur.uc, cur.us, uh);
-            // dg = dm u sigma(g) (1 + g (1 - sigma(g))), du = dm g sigma(g), two values
-            // per packed FP32 operation; m~ = BF16_RNE(silu(g^) u^) exactly
-            float dg[8], du[8], mr[8];
-            const uint64_t one2 = f2_pack(1.0f, 1.0f), neg2 = f2_pack(-1.0f, -1.0f);
+        const int64_t c = it.chunk * QCHUNK + 16 * lane;
+        if (c < I) {
+            // mq, gq and uq share their shape: one code offset, one scale offset
+            const int64_t so = scale_offset(row, c >> 4, I), co = row * (I >> 1) + (c >> 1);
+            if (row >= M) {   // a padding row of the scale layout
+                static_cast<uint8_t *>(mq.scales)[so] = 0;
+                if (has_gq) static_cast<uint8_t *>(gq.scales)[so] = 0;
+                if (has_uq) static_cast<uint8_t *>(uq.scales)[so] = 0;
+            } else {
+                float mv[8];
+                uint4 m0, m1;
+                silu8(cur.g0, cur.u0, mv);
+                round8_bf16(mv, m0, mv);
+                silu8(cur.g1, cur.u1, mv);
+                round8_bf16(mv, m1, mv);
+                if (m) {
+                    uint4 *mp = reinterpret_cast<uint4 *>(m + row * I + c);
+                    mp[0] = m0;
+                    mp[1] = m1;
+                }
+                uint32_t lo, hi, sb;
+                quant16_bf16(m0, m1, &lo, &hi, &sb);
+                *reinterpret_cast<uint2 *>(static_cast<uint8_t *>(mq.codes) + co) = make_uint2(lo, hi);
+                static_cast<uint8_t *>(mq.scales)[so] = (uint8_t)sb;
+                if (has_gq) {
+                    quant16_bf16(cur.g0, cur.g1, &lo, &hi, &sb);
+                    *reinterpret_cast<uint2 *>(static_cast<uint8_t *>(gq.codes) + co) = make_uint2(lo, hi);
+                    static_cast<uint8_t *>(gq.scales)[so] = (uint8_t)sb;
+                }
+                if (has_uq) {
+                    quant16_bf16(cur.u0, cur.u1, &lo, &hi, &sb);
+                    *reinterpret_cast<uint2 *>(static_cast<uint8_t *>(uq.codes) + co) = make_uint2(lo, hi);
+                    static_cast<uint8_t *>(uq.scales)[so] = (uint8_t)sb;
+                }
+            }
+        }
+        it = nx;
+        cur = nxt;
+    }
+}
+
+// ---------------------------------------------- A9: SiLU-multiply backward + quantize
+// A task is 512 columns of a row; lane j owns the 16-value block j: one scale byte of
+// g^ and of u^ to read, one block each of dg and du to quantize.
+__global__ void __launch_bounds__(256) k_silu_mul_bwd_quant(const pact_bf16 *__restrict__ dm, int64_t lddm,
+                                                            pact_nvfp4_t gq, pact_nvfp4_t uq, int64_t M, int64_t I,
+                                                            pact_bf16 *__restrict__ dgu, int64_t lddgu,
+                                                            pact_nvfp4_t dguq, pact_bf16 *__restrict__ m_re) {
+    pdl_wait();
+    const int lane = threadIdx.x & 31;
+    const int64_t nchunk = (I + QCHUNK - 1) / QCHUNK;
+    const int64_t rows_pad = (M + 127) & ~int64_t(127);
+    const int64_t warp0 = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+    const int64_t nwarps = (int64_t)gridDim.x * (blockDim.x >> 5);
+    struct In {
+        uint4 d0, d1;
+        uint2 gc, uc;
+        uint32_t gs, us;
+    };
+    auto load = [&](const TaskIter &t, In &v) {
+        const int64_t c = t.chunk * QCHUNK + 16 * lane;
+        v.d0 = v.d1 = make_uint4(0, 0, 0, 0);
+        v.gc = v.uc = make_uint2(0, 0);
+        v.gs = v.us = 0;
+        if (t.row < M && c < I) {
+            const uint4 *dp = reinterpret_cast<const uint4 *>(dm + t.row * lddm + c);
+            v.d0 = dp[0];
+            v.d1 = dp[1];
+            // gq and uq share their shape: one code offset, one scale offset
+            const int64_t co = t.row * (I >> 1) + (c >> 1), so = scale_offset(t.row, c >> 4, I);
+            v.gc = *reinterpret_cast<const uint2 *>(static_cast<const uint8_t *>(gq.codes) + co);
+            v.uc = *reinterpret_cast<const uint2 *>(static_cast<const uint8_t *>(uq.codes) + co);
+            v.gs = static_cast<const uint8_t *>(gq.scales)[so];
+            v.us = static_cast<const uint8_t *>(uq.scales)[so];
+        }
+    };
+    // dg = dm u sigma(g) (1 + g (1 - sigma(g))), du = dm g sigma(g), two values per packed
+    // FP32 operation, and m~ = BF16_RNE(silu(g^) u^) exactly, for 8 values: rounded to
+    // BF16 words (wg, wu, wm)
+    const uint64_t one2 = f2_pack(1.0f, 1.0f), neg2 = f2_pack(-1.0f, -1.0f);
+    auto half8 = [&](const uint4 &dw, uint32_t gc, uint32_t gsb, uint32_t uc, uint32_t usb, uint4 &wg, uint4 &wu,
+                     uint4 &wm) {
+        float d[8], gh[8], uh[8], dg[8], du[8], mr[8];
+        unpack8_bf16(dw, d);
+        dequant8(gc, gsb, gh);
+        dequant8(uc, usb, uh);
 #pragma unroll
-            for (int i = 0; i < 8; i += 2) {
-                const float s0 = sigmoid_fast(gh[i]), s1 = sigmoid_fast(gh[i + 1]);
-                const uint64_t g2 = f2_pack(gh[i], gh[i + 1]), sg2 = f2_pack(s0, s1);
-                const uint64_t ds = f2_mul(f2_pack(d[i], d[i + 1]), sg2);
-                const uint64_t w = f2_fma(g2, f2_fma(sg2, neg2, one2), one2);
-                f2_unpack(f2_mul(f2_mul(ds, f2_pack(uh[i], uh[i + 1])), w), dg[i], dg[i + 1]);
-                f2_unpack(f2_mul(ds, g2), du[i], du[i + 1]);
-                mr[i] = silu_mul_value<true>(gh[i], uh[i], s0);
-                mr[i + 1] = silu_mul_value<true>(gh[i + 1], uh[i + 1], s1);
+        for (int i = 0; i < 8; i += 2) {
+            const float s0 = sigmoid_fast(gh[i]), s1 = sigmoid_fast(gh[i + 1]);
+            const uint64_t g2 = f2_pack(gh[i], gh[i + 1]), sg2 = f2_pack(s0, s1);
+            const uint64_t ds = f2_mul(f2_pack(d[i], d[i + 1]), sg2);
+            const uint64_t w = f2_fma(g2, f2_fma(sg2, neg2, one2), one2);
+            f2_unpack(f2_mul(f2_mul(ds, f2_pack(uh[i], uh[i + 1])), w), dg[i], dg[i + 1]);
+            f2_unpack(f2_mul(ds, g2), du[i], du[i + 1]);
+            mr[i] = silu_mul_value<true>(gh[i], uh[i], s0);
+            mr[i + 1] = silu_mul_value<true>(gh[i + 1], uh[i + 1], s1);
+        }
+        wg.x = pack_bf16x2(dg[0], dg[1]); wg.y = pack_bf16x2(dg[2], dg[3]);
+        wg.z = pack_bf16x2(dg[4], dg[5]); wg.w = pack_bf16x2(dg[6], dg[7]);
+        wu.x = pack_bf16x2(du[0], du[1]); wu.y = pack_bf16x2(du[2], du[3]);
+        wu.z = pack_bf16x2(du[4], du[5]); wu.w = pack_bf16x2(du[6], du[7]);
+        wm.x = pack_bf16x2(mr[0], mr[1]); wm.y = pack_bf16x2(mr[2], mr[3]);
+        wm.z = pack_bf16x2(mr[4], mr[5]); wm.w = pack_bf16x2(mr[6], mr[7]);
+    };
+    TaskIter it(warp0, nchunk, nwarps);
+    In cur;
+    if (it.row < rows_pad) load(it, cur);
+    while (it.row < rows_pad) {
+        TaskIter nx = it;
+        nx.next();
+        In nxt;
+        if (nx.row < rows_pad) {
+            load(nx, nxt);
+        } else {
+            nxt.d0 = nxt.d1 = make_uint4(0, 0, 0, 0);
+            nxt.gc = nxt.uc = make_uint2(0, 0);
+            nxt.gs = nxt.us = 0;
+        }
+        const int64_t row = it.row;
+        const int64_t c = it.chunk * QCHUNK + 16 * lane;
+        if (c < I) {
+            // dg's block is block c / 16 of the [M x 2I] copy; du's lies I columns right
+            uint8_t *codes = static_cast<uint8_t *>(dguq.codes) + row * I + (c >> 1);
+            uint8_t *sg = static_cast<uint8_t *>(dguq.scales) + scale_offset(row, c >> 4, 2 * I);
+            uint8_t *su = static_cast<uint8_t *>(dguq.scales) + scale_offset(row, (I + c) >> 4, 2 * I);
+            if (row >= M) {   // a padding row of the scale layout
+                *sg = 0;
+                *su = 0;
+            } else {
+                uint4 wg0, wu0, wm0, wg1, wu1, wm1;
+                half8(cur.d0, cur.gc.x, cur.gs, cur.uc.x, cur.us, wg0, wu0, wm0);
+                half8(cur.d1, cur.gc.y, cur.gs, cur.uc.y, cur.us, wg1, wu1, wm1);
+                uint4 *gp = reinterpret_cast<uint4 *>(dgu + row * lddgu + c);
+                uint4 *upp = reinterpret_cast<uint4 *>(dgu + row * lddgu + I + c);
+                gp[0] = wg0; gp[1] = wg1;
+                upp[0] = wu0; upp[1] = wu1;
+                if (m_re) {
+                    uint4 *mp = reinterpret_cast<uint4 *>(m_re + row * I + c);
+                    mp[0] = wm0; mp[1] = wm1;
+                }
+                uint32_t lo, hi, sb;
+                quant16_bf16(wg0, wg1, &lo, &hi, &sb);
+                *reinterpret_cast<uint2 *>(codes) = make_uint2(lo, hi);
+                *sg = (uint8_t)sb;
+                quant16_bf16(wu0, wu1, &lo, &hi, &sb);
+                *reinterpret_cast<uint2 *>(codes + (I >> 1)) = make_uint2(lo, hi);
+                *su = (uint8_t)sb;
             }
-            uint4 wg, wu, wm;
-            round8_bf16(dg, wg, dg);
-            round8_bf16(du, wu, du);
-            wm.x = pack_bf16x2(mr[0], mr[1]); wm.y = pack_bf16x2(mr[2], mr[3]);
-            wm.z = pack_bf16x2(mr[4], mr[5]); wm.w = pack_bf16x2(mr[6], mr[7]);
-            if (valid) {
-                *reinterpret_cast<uint4 *>(dgu + row * lddgu + c) = wg;
-                *reinterpret_cast<uint4 *>(dgu + row * lddgu + I + c) = wu;
-                if (m_re) *reinterpret_cast<uint4 *>(m_re + row * I + c) = wm;
-            }
-            // du's chunk sits I columns to the right: I / 2 code bytes, and I / 64 whole
-            // scale tiles (I is a multiple of 64)
-            const ChunkAt at = chunk_at(row, c0, 2 * I);
-            const ChunkAt at_u = {at.code_off + (I >> 1), at.scale_off + (I >> 6) * 512};
-            uint32_t sb;
-            uint32_t codes = quant8(dg, &sb);
-            store_chunk_at(dguq, at, codes, sb, valid);
-            codes = quant8(du, &sb);
-            store_chunk_at(dguq, at_u, codes, sb, valid);
         }
         it = nx;
         cur = nxt;
@@ -673,7 +743,7 @@ pact_status pact_quantize_nvfp4(const pact_bf16 *x, int64_t ldx, int64_t rows, i
                "pact_quantize_nvfp4: x must be 16-byte aligned with ldx >= cols, ldx %% 8 == 0");
     pact_status s = check_nvfp4(out, rows, cols, "out");
     if (s != PACT_OK) return s;
-    const int64_t tasks = ((rows + 127) / 128 * 128) * ((cols + CHUNK - 1) / CHUNK);
+    const int64_t tasks = ((rows + 127) / 128 * 128) * ((cols + QCHUNK - 1) / QCHUNK);
     return launch_dep(k_quantize, dim3(grid_for(tasks, 256)), dim3(256), 0, (cudaStream_t)stream, "pact_quantize_nvfp4",
                       x, ldx, rows, *out, 1.0f);
 }
@@ -742,8 +812,9 @@ pact_status pact_silu_mul_quant(const pact_bf16 *g, const pact_bf16 *u, int64_t 
     if (s == PACT_OK && uq) s = check_nvfp4(uq, M, I, "uq");
     if (s != PACT_OK) return s;
     pact_nvfp4_t none = {nullptr, nullptr, M, I};
-    const int64_t tasks = ((M + 127) / 128 * 128) * ((I + CHUNK - 1) / CHUNK);
-    return launch_dep(k_silu_mul_quant, dim3(grid_for(tasks, 256)), dim3(256), 0, (cudaStream_t)stream,
+    const int64_t tasks = ((M + 127) / 128 * 128) * ((I + QCHUNK - 1) / QCHUNK);
+    static const int per_sm = resident_per_sm(k_silu_mul_quant);
+    return launch_dep(k_silu_mul_quant, dim3(grid_for(tasks, 256, per_sm)), dim3(256), 0, (cudaStream_t)stream,
                       "pact_silu_mul_quant", g, u, ld_gu, M, I, m, *mq, gq ? *gq : none, uq ? *uq : none,
                       (int)(gq != nullptr), (int)(uq != nullptr));
 }
@@ -761,8 +832,9 @@ pact_status pact_silu_mul_bwd_quant(const pact_bf16 *dm, int64_t lddm, const pac
     if (s == PACT_OK) s = check_nvfp4(uq, M, I, "uq");
     if (s == PACT_OK) s = check_nvfp4(dguq, M, 2 * I, "dguq");
     if (s != PACT_OK) return s;
-    const int64_t tasks = ((M + 127) / 128 * 128) * ((I + CHUNK - 1) / CHUNK);
-    return launch_dep(k_silu_mul_bwd_quant, dim3(grid_for(tasks, 256)), dim3(256), 0, (cudaStream_t)stream,
+    const int64_t tasks = ((M + 127) / 128 * 128) * ((I + QCHUNK - 1) / QCHUNK);
+    static const int per_sm = resident_per_sm(k_silu_mul_bwd_quant);
+    return launch_dep(k_silu_mul_bwd_quant, dim3(grid_for(tasks, 256, per_sm)), dim3(256), 0, (cudaStream_t)stream,
                       "pact_silu_mul_bwd_quant", dm, lddm, *gq, *uq, M, I, dgu, lddgu, *dguq, m_re);
 }
 
@@ -821,7 +893,7 @@ pact_status pact_weight_layout_cache_scaled(const pact_bf16 *W, int64_t ldw, int
     c.bwd.codes = p; p += up256(pact_nvfp4_code_bytes(K, N));
     c.bwd.scales = p;
     c.gexp = gexp;
-    const int64_t tasks = ((N + 127) / 128 * 128) * ((K + CHUNK - 1) / CHUNK);
+    const int64_t tasks = ((N + 127) / 128 * 128) * ((K + QCHUNK - 1) / QCHUNK);
     pact_status s = launch_dep(k_quantize, dim3(grid_for(tasks, 256)), dim3(256), 0, (cudaStream_t)stream,
                                "pact_weight_layout_cache", W, ldw, N, c.fwd, std::ldexp(1.0f, -gexp));
     if (s != PACT_OK) return s;

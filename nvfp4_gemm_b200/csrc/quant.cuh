@@ -137,6 +137,27 @@ __device__ __forceinline__ void quant16_bf16(const uint4 wa, const uint4 wb, uin
     *sb = b;
 }
 
+// quant16_bf16 for 16 FP32 values (the same decisions for values that are BF16).
+__device__ __forceinline__ void quant16_f32(const float (&v)[16], uint32_t *lo, uint32_t *hi, uint32_t *sb) {
+    float amax = 0.0f;
+#pragma unroll
+    for (int j = 0; j < 16; ++j) amax = fmaxf(amax, fabsf(v[j]));
+    const uint32_t b = scale_byte(amax);
+    const float s = e4m3_to_float(b);
+    const float nr = b ? -__frcp_rn(s) : -0.0f;
+    const uint64_t nr2 = f2_pack(nr, nr), s2 = f2_pack(s, s);
+    uint32_t out[2] = {0u, 0u};
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+        float q0, q1;
+        neg_quotient2(v[2 * j], v[2 * j + 1], s2, nr2, q0, q1);
+        out[j >> 2] |= e2m1_pair(q0, q1) << (8 * (j & 3));
+    }
+    *lo = out[0] ^ CODE_SIGNS;
+    *hi = out[1] ^ CODE_SIGNS;
+    *sb = b;
+}
+
 // Gather the scales of blocks 4q..4q+3 (lanes 8q, 8q+2, 8q+4, 8q+6) into lane 8q
 // as one little-endian word; meaningful in lanes with lane % 8 == 0.
 __device__ __forceinline__ uint32_t gather_scales4(uint32_t sb) {
