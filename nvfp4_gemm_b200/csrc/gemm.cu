@@ -719,8 +719,13 @@ static pact_status run(const pact_nvfp4_t *a, const pact_nvfp4_t *b, int gexp, c
         if (s != PACT_OK) return s;
     }
     // work units: output tiles, or (gate, up) tile pairs in gate|up mode
+    // As few pairs as finish the tiles in the same number of rounds as all of them
+    // would: the grid's last round is then full, and the pairs left over are free for
+    // kernels on other streams (384 tiles on 148 SMs: 6 rounds on 64 pairs, not 5.2 on 74).
     const int units = (int)(((M + 255) / 256) * ((N + 255) / 256)) / (so ? 2 : 1);
-    const int clusters = units < sm_count() / 2 ? units : sm_count() / 2;
+    const int max_clusters = sm_count() / 2;
+    const int rounds = (units + max_clusters - 1) / max_clusters;
+    const int clusters = (units + rounds - 1) / rounds;
     return launch_dep(so ? k_nvfp4_gemm<true> : k_nvfp4_gemm<false>, dim3(2 * clusters), dim3(THREADS), SMEM_BYTES,
                       stream, what, tmA, tmB, tmSFA, tmSFB, tmLa, tmLb, tmD, tmR, p);
 }

@@ -26,9 +26,6 @@ constexpr int BM = 128;        // output rows per CTA (MMA M)
 constexpr int BK = 64;         // contraction elements per stage (128 bytes of BF16)
 constexpr int MAX_STAGES = 6;  // ring depth: 6, or 3 where two CTAs should share an SM
 constexpr int THREADS = 192;
-// With an NVFP4 A operand, two groups of four decoding warps take alternate stages
-// (the decode, not the MMA or the copies, bounds those products).
-__host__ __device__ constexpr int threads_for(bool fp4) { return fp4 ? THREADS + 128 : THREADS; }
 constexpr int A_BYTES = BM * BK * 2;     // 16384
 constexpr int B_BYTES = 64 * BK * 2;     // 8192 per B part
 // NVFP4 A operand: per stage, the codes of the A tile (128 x 64 values, 4 KiB) and
@@ -143,7 +140,7 @@ __device__ __forceinline__ void decode_stage(const uint8_t *raw, uint8_t *oper, 
 }
 
 template <bool A_MN, bool B_MN, bool A_FP4>
-__global__ void __launch_bounds__(threads_for(A_FP4), 1)
+__global__ void __launch_bounds__(THREADS, 1)
 k_lora_mma(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, const Params p) {
     const int nparts = p.b_split ? 2 : 1;
     const int STAGE_BYTES = stage_bytes(nparts, A_FP4), OPER_BYTES = oper_bytes(nparts);
@@ -293,11 +290,10 @@ k_lora_mma(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUte
             // decode each stage's NVFP4 A tile into the BF16 operand buffer, then
             // announce it on the stage's `full` barrier (after a proxy fence: the
             // tensor core reads shared memory through the async proxy)
-            const int group = (warp - 2) >> 2;             // stages group, group + 2, ...
-            const int tid = threadIdx.x - 64 - 128 * group;
-            for (int kt = group; kt < ktiles; kt += 2) {
-                const int stage = kt % STAGES;
-                const uint32_t phase = (uint32_t)(kt / STAGES) & 1u;
+            // (one consumer per barrier: a parity wait may run at most one phase ahead)
+            const int tid = threadIdx.x - 64;
+            uint32_t stage = 0, phase = 0;
+            for (int kt = 0; kt < ktiles; ++kt) {
                 if (!(ok = warp_all(mbar_wait(&raw_full[stage], phase)))) {
                     aborted = 1;
                     break;
@@ -307,6 +303,7 @@ k_lora_mma(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUte
                 fence_proxy_async_smem();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&full[stage]);
+                if (++stage == STAGES) { stage = 0; phase ^= 1; }
             }
         }
     }
@@ -462,7 +459,7 @@ static pact_status launch_mma(const CUtensorMap &ta, const CUtensorMap &tb, cons
         done[d] = true;
     }
     dim3 grid((unsigned)row_tiles, (unsigned)p.splits, (unsigned)p.nprob);
-    return launch_dep(k_lora_mma<A_MN, B_MN, A_FP4>, grid, dim3(threads_for(A_FP4)), smem, st, what, ta, tb, p);
+    return launch_dep(k_lora_mma<A_MN, B_MN, A_FP4>, grid, dim3(THREADS), smem, st, what, ta, tb, p);
 }
 
 static FinJob fin_job(const float *ws, const Params &p, int64_t rows, int64_t cols, float scale, int mode,
