@@ -42,7 +42,6 @@ constexpr int BM = 128;               // rows per CTA; the pair tile has 256
 constexpr int BN = 256;               // columns of the pair tile; each CTA loads 128 rows of B
 constexpr int BK = 256;               // FP4 elements per stage = 128 bytes per row
 constexpr int KSTEP = 64;             // FP4 elements per MMA
-constexpr int STAGES = 4;
 constexpr int A_BYTES = BM * BK / 2;          // 16384
 constexpr int B_BYTES = (BN / 2) * BK / 2;    // 16384
 constexpr int OFF_B = A_BYTES;
@@ -53,19 +52,30 @@ constexpr int STAGE_BYTES = OFF_SFB + 4096;   // 38912 = 38 KiB
 constexpr int OFF_LW = 6 * BM * 32;           // LoRA weight chunks follow 6 activation chunks
 static_assert(OFF_LW + 3 * BM * 32 <= STAGE_BYTES && OFF_LW + 2 * 48 * 128 <= STAGE_BYTES, "LoRA stage");
 constexpr int EPI_WARPS = 16;
-constexpr int SLAB_BYTES = 32 * 128;          // 32 rows x 64 BF16 columns, 128-byte swizzle
-constexpr int OFF_SLABS = STAGES * STAGE_BYTES;
-constexpr int OFF_BARS = OFF_SLABS + EPI_WARPS * SLAB_BYTES;
-constexpr int SMEM_BYTES = 1024 + OFF_BARS + 512;
 constexpr int THREADS = 32 * (2 + EPI_WARPS);                 // 576
-static_assert(SMEM_BYTES <= 232448, "shared memory");
+// Shared memory: the ring, then one slab per epilogue warp, then the barriers.  The
+// plain GEMM writes a warp's 32 x 64 block through a 32 x 32 slab (two TMA stores,
+// 64-byte swizzle), which leaves room for a fifth ring stage; the gate|up mode keeps a
+// whole 32 x 64 gate block (128-byte swizzle) in the slab until the up block of the
+// same columns, so it runs four stages.
+template <bool SILU>
+struct Layout {
+    static constexpr int STAGES = SILU ? 4 : 5;
+    static constexpr int SLAB_COLS = SILU ? 64 : 32;
+    static constexpr int SLAB_BYTES = 32 * SLAB_COLS * 2;
+    static constexpr int OFF_SLABS = STAGES * STAGE_BYTES;
+    static constexpr int OFF_BARS = OFF_SLABS + EPI_WARPS * SLAB_BYTES;
+    static constexpr int SMEM_BYTES = 1024 + OFF_BARS + 512;
+    static_assert(SMEM_BYTES <= 232448, "shared memory");
+};
+constexpr int MAX_STAGES = Layout<false>::STAGES > Layout<true>::STAGES ? Layout<false>::STAGES : Layout<true>::STAGES;
 
 // tensor memory columns
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t COL_ACC = 0;        // 256 FP32 columns
 constexpr uint32_t COL_SF = 256;       // per stage: 16 columns of A scales, then 32 of B scales
 constexpr uint32_t SF_COLS = 48;
-static_assert(COL_SF + STAGES * SF_COLS <= TMEM_COLS, "tensor memory");
+static_assert(COL_SF + MAX_STAGES * SF_COLS <= TMEM_COLS, "tensor memory");
 
 enum LoraMode : int { LORA_NONE = 0, LORA_FWD = 1, LORA_DGRAD = 2 };
 
@@ -78,6 +88,8 @@ struct Params {
     int lora_nseg;
     int64_t seg_end[4];
     float out_scale;      // 2^gexp of the weight cache: scales the accumulator (exact)
+    const pact_bf16 *res; // the residual (its second 32-column half of a block is read directly)
+    int64_t ldr;
     int n_fast;           // tile order: 1 = N tiles fastest (A streamed once), 0 = M tiles fastest
     // optional NVFP4 copy of the BF16 output, split along N into nq (1 or 2) tensors:
     // columns [0, q_split) into q[0], [q_split, N) into q[1]
@@ -166,6 +178,7 @@ __device__ __forceinline__ QDest qdest(const Params &p, int row, int col) {
 
 // Every stage of the ring is used in the same order by all roles: per tile, one LoRA
 // stage (when the GEMM carries a LoRA term) and then ktiles K stages.
+template <int STAGES>
 struct Ring {
     uint32_t stage = 0, phase = 0;
     __device__ __forceinline__ void next() {
@@ -181,10 +194,13 @@ k_nvfp4_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CU
              const __grid_constant__ CUtensorMap tmSFA, const __grid_constant__ CUtensorMap tmSFB,
              const __grid_constant__ CUtensorMap tmLa, const __grid_constant__ CUtensorMap tmLb,
              const __grid_constant__ CUtensorMap tmD, const __grid_constant__ CUtensorMap tmR, const Params p) {
+    using L = Layout<SILU>;
+    constexpr int STAGES = L::STAGES;
+    using Ring = pact::gemm::Ring<STAGES>;
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = smem_u32(smem_raw);
     uint8_t *smem = smem_raw + (((raw + 1023) & ~1023u) - raw);
-    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + OFF_BARS);
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + L::OFF_BARS);
     uint64_t *full = bars;                        // [STAGES] leader: operands and scales of both CTAs
     uint64_t *empty = bars + STAGES;              // [STAGES] local: the pair's MMAs are done with the stage
     uint64_t *acc_full = bars + 2 * STAGES;       // local: accumulator complete
@@ -397,7 +413,7 @@ k_nvfp4_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CU
         const int quarter = ew >> 2;             // columns 64*quarter .. 64*quarter+63 of the tile
         const uint32_t acc_empty_leader = mapa_shared(smem_u32(acc_empty), 0);
         const uint32_t taddr = tmem + ((uint32_t)(sub * 32) << 16) + COL_ACC + quarter * 64;
-        uint8_t *slab_p = smem + OFF_SLABS + ew * SLAB_BYTES;
+        uint8_t *slab_p = smem + L::OFF_SLABS + ew * L::SLAB_BYTES;
         const uint32_t slab = smem_u32(slab_p);
         // this warp's 32 x 64 block of tile t: first row and column
         auto block_y = [&](int t) {
@@ -412,7 +428,7 @@ k_nvfp4_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CU
         };
         auto inside = [&](int t) { return block_y(t) < p.M && block_x(t) < p.N; };
         auto load_residual = [&](int t) {  // lane 0; the slab is free
-            mbar_arrive_expect_tx(&res_full[ew], SLAB_BYTES);
+            mbar_arrive_expect_tx(&res_full[ew], L::SLAB_BYTES);
             tma_load_2d(slab_p, &tmR, &res_full[ew], block_x(t), block_y(t));
         };
         uint32_t acc_phase = 0, res_phase = 0;
@@ -442,88 +458,161 @@ k_nvfp4_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CU
                 }
             }
             if (inside(t)) {
-                if (p.has_res) {
-                    if (lane == 0) got = mbar_wait_sleep(&res_full[ew], res_phase);
-                    if (!(ok = __shfl_sync(0xffffffffu, got, 0))) break;
-                    res_phase ^= 1;
-                } else {
-                    if (lane == 0) bulk_wait_read_all();  // the previous block's store has read the slab
-                    __syncwarp();
-                }
-                // the NVFP4 copy of the block's rounded values: block b of this lane's row is
-                // quantized once its two 8-value pieces are rounded
-                const QDest qd = qdest(p, block_y(t) + lane, block_x(t));
-                // gate|up mode: the gate block stays in the slab for the up block that follows
-                const bool up = SILU && (t & 1);
-                uint32_t sbs = 0;
-                // row `lane` of the block: 8 pieces of 16 bytes, 128-byte swizzle
-#pragma unroll
-                for (int q = 0; q < 8; ++q) {
-                    const uint32_t a = slab + lane * 128 + ((q ^ (lane & 7)) << 4);
-                    float f[8];
-#pragma unroll
-                    for (int i = 0; i < 8; ++i) f[i] = __uint_as_float(r[8 * q + i]) * p.out_scale;
+                if constexpr (SILU) {
                     if (p.has_res) {
-                        uint32_t o0, o1, o2, o3;
-                        asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
-                                     : "=r"(o0), "=r"(o1), "=r"(o2), "=r"(o3)
-                                     : "r"(a));
-                        f[0] += bf16lo(o0); f[1] += bf16hi(o0); f[2] += bf16lo(o1); f[3] += bf16hi(o1);
-                        f[4] += bf16lo(o2); f[5] += bf16hi(o2); f[6] += bf16lo(o3); f[7] += bf16hi(o3);
+                        if (lane == 0) got = mbar_wait_sleep(&res_full[ew], res_phase);
+                        if (!(ok = __shfl_sync(0xffffffffu, got, 0))) break;
+                        res_phase ^= 1;
+                    } else {
+                        if (lane == 0) bulk_wait_read_all();  // the previous block's store has read the slab
+                        __syncwarp();
                     }
-                    const uint32_t w0 = pack_bf16x2(f[0], f[1]), w1 = pack_bf16x2(f[2], f[3]);
-                    const uint32_t w2 = pack_bf16x2(f[4], f[5]), w3 = pack_bf16x2(f[6], f[7]);
-                    if (!up)
+                    // the NVFP4 copy of the block's rounded values: block b of this lane's row is
+                    // quantized once its two 8-value pieces are rounded
+                    const QDest qd = qdest(p, block_y(t) + lane, block_x(t));
+                    // gate|up mode: the gate block stays in the slab for the up block that follows
+                    const bool up = SILU && (t & 1);
+                    uint32_t sbs = 0;
+                    // row `lane` of the block: 8 pieces of 16 bytes, 128-byte swizzle
+    #pragma unroll
+                    for (int q = 0; q < 8; ++q) {
+                        const uint32_t a = slab + lane * 128 + ((q ^ (lane & 7)) << 4);
+                        float f[8];
+    #pragma unroll
+                        for (int i = 0; i < 8; ++i) f[i] = __uint_as_float(r[8 * q + i]) * p.out_scale;
+                        if (p.has_res) {
+                            uint32_t o0, o1, o2, o3;
+                            asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                                         : "=r"(o0), "=r"(o1), "=r"(o2), "=r"(o3)
+                                         : "r"(a));
+                            f[0] += bf16lo(o0); f[1] += bf16hi(o0); f[2] += bf16lo(o1); f[3] += bf16hi(o1);
+                            f[4] += bf16lo(o2); f[5] += bf16hi(o2); f[6] += bf16lo(o3); f[7] += bf16hi(o3);
+                        }
+                        const uint32_t w0 = pack_bf16x2(f[0], f[1]), w1 = pack_bf16x2(f[2], f[3]);
+                        const uint32_t w2 = pack_bf16x2(f[4], f[5]), w3 = pack_bf16x2(f[6], f[7]);
+                        if (!up)
+                            asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(a), "r"(w0), "r"(w1), "r"(w2),
+                                         "r"(w3)
+                                         : "memory");
+                        // the rounded values, kept for the NVFP4 copy (r[] is free again)
+                        r[4 * q] = w0; r[4 * q + 1] = w1; r[4 * q + 2] = w2; r[4 * q + 3] = w3;
+                        if ((q & 1) && qd.codes) {
+                            uint32_t lo, hi, sb;
+                            quant16_bf16(make_uint4(r[4 * q - 4], r[4 * q - 3], r[4 * q - 2], r[4 * q - 1]),
+                                         make_uint4(w0, w1, w2, w3), &lo, &hi, &sb);
+                            *reinterpret_cast<uint2 *>(qd.codes + 4 * (q - 1)) = make_uint2(lo, hi);
+                            sbs |= sb << (4 * (q - 1));
+                        }
+                    }
+                    if (qd.scales) *reinterpret_cast<uint32_t *>(qd.scales) = sbs;
+                    if (up) {
+                        // m = BF16(silu(g) u) for the 64 columns of this row: g from the slab (the
+                        // gate block, same rows and columns), u from the packed words in r[0..31];
+                        // m replaces g in the slab and is quantized block by block
+                        const QDest md = mdest(p, block_y(t) + lane, block_x(t));
+                        uint32_t msbs = 0, n0 = 0, n1 = 0, n2 = 0, n3 = 0;
+    #pragma unroll
+                        for (int q = 0; q < 8; ++q) {
+                            const uint32_t a = slab + lane * 128 + ((q ^ (lane & 7)) << 4);
+                            uint32_t g4[4], mw[4];
+                            asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                                         : "=r"(g4[0]), "=r"(g4[1]), "=r"(g4[2]), "=r"(g4[3])
+                                         : "r"(a));
+    #pragma unroll
+                            for (int j = 0; j < 4; ++j)
+                                mw[j] = pack_bf16x2(silu_mul_out(bf16lo(g4[j]), bf16lo(r[4 * q + j])),
+                                                    silu_mul_out(bf16hi(g4[j]), bf16hi(r[4 * q + j])));
+                            asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(a), "r"(mw[0]), "r"(mw[1]),
+                                         "r"(mw[2]), "r"(mw[3])
+                                         : "memory");
+                            if ((q & 1) && md.codes) {
+                                uint32_t lo, hi, sb;
+                                quant16_bf16(make_uint4(n0, n1, n2, n3), make_uint4(mw[0], mw[1], mw[2], mw[3]), &lo, &hi,
+                                             &sb);
+                                *reinterpret_cast<uint2 *>(md.codes + 4 * (q - 1)) = make_uint2(lo, hi);
+                                msbs |= sb << (4 * (q - 1));
+                            }
+                            n0 = mw[0]; n1 = mw[1]; n2 = mw[2]; n3 = mw[3];
+                        }
+                        if (md.scales) *reinterpret_cast<uint32_t *>(md.scales) = msbs;
+                    }
+                    if (!SILU || up) {   // a gate block is not stored: its m follows with the up block
+                        fence_proxy_async_smem();
+                        __syncwarp();
+                        if (lane == 0) {
+                            tma_store_2d(&tmD, slab, up ? block_x(t) - p.half_tiles * BN : block_x(t), block_y(t));
+                            bulk_commit_group();
+                        }
+                    }
+                } else {
+                    // two 32-column halves through the 32 x 32 slab (64-byte swizzle): the
+                    // first half's residual was prefetched into the slab by TMA, the second
+                    // half's is read directly while the first half is written
+                    const QDest qd = qdest(p, block_y(t) + lane, block_x(t));
+                    uint4 rh[4];
+                    if (p.has_res) {
+                        const int row = block_y(t) + lane, c1 = block_x(t) + 32;
+#pragma unroll
+                        for (int j = 0; j < 4; ++j)
+                            rh[j] = (row < p.M && c1 + 8 * j < p.N)
+                                        ? *reinterpret_cast<const uint4 *>(p.res + (int64_t)row * p.ldr + c1 + 8 * j)
+                                        : make_uint4(0, 0, 0, 0);
+                        if (lane == 0) got = mbar_wait_sleep(&res_full[ew], res_phase);
+                        if (!(ok = __shfl_sync(0xffffffffu, got, 0))) break;
+                        res_phase ^= 1;
+                    } else {
+                        if (lane == 0) bulk_wait_read_all();  // the previous block's stores have read the slab
+                        __syncwarp();
+                    }
+                    uint32_t sbs = 0;
+#pragma unroll
+                    for (int q = 0; q < 8; ++q) {
+                        if (q == 4) {   // the first half is in the slab: store it, then reuse the slab
+                            fence_proxy_async_smem();
+                            __syncwarp();
+                            if (lane == 0) {
+                                tma_store_2d(&tmD, slab, block_x(t), block_y(t));
+                                bulk_commit_group();
+                                bulk_wait_read_all();
+                            }
+                            __syncwarp();
+                        }
+                        const uint32_t a = slab + lane * 64 + (((q & 3) ^ ((lane >> 1) & 3)) << 4);
+                        float f[8];
+#pragma unroll
+                        for (int i = 0; i < 8; ++i) f[i] = __uint_as_float(r[8 * q + i]) * p.out_scale;
+                        if (p.has_res) {
+                            uint32_t o0, o1, o2, o3;
+                            if (q < 4) {
+                                asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                                             : "=r"(o0), "=r"(o1), "=r"(o2), "=r"(o3)
+                                             : "r"(a));
+                            } else {
+                                o0 = rh[q - 4].x; o1 = rh[q - 4].y; o2 = rh[q - 4].z; o3 = rh[q - 4].w;
+                            }
+                            f[0] += bf16lo(o0); f[1] += bf16hi(o0); f[2] += bf16lo(o1); f[3] += bf16hi(o1);
+                            f[4] += bf16lo(o2); f[5] += bf16hi(o2); f[6] += bf16lo(o3); f[7] += bf16hi(o3);
+                        }
+                        const uint32_t w0 = pack_bf16x2(f[0], f[1]), w1 = pack_bf16x2(f[2], f[3]);
+                        const uint32_t w2 = pack_bf16x2(f[4], f[5]), w3 = pack_bf16x2(f[6], f[7]);
                         asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(a), "r"(w0), "r"(w1), "r"(w2),
                                      "r"(w3)
                                      : "memory");
-                    // the rounded values, kept for the NVFP4 copy (r[] is free again)
-                    r[4 * q] = w0; r[4 * q + 1] = w1; r[4 * q + 2] = w2; r[4 * q + 3] = w3;
-                    if ((q & 1) && qd.codes) {
-                        uint32_t lo, hi, sb;
-                        quant16_bf16(make_uint4(r[4 * q - 4], r[4 * q - 3], r[4 * q - 2], r[4 * q - 1]),
-                                     make_uint4(w0, w1, w2, w3), &lo, &hi, &sb);
-                        *reinterpret_cast<uint2 *>(qd.codes + 4 * (q - 1)) = make_uint2(lo, hi);
-                        sbs |= sb << (4 * (q - 1));
-                    }
-                }
-                if (qd.scales) *reinterpret_cast<uint32_t *>(qd.scales) = sbs;
-                if (up) {
-                    // m = BF16(silu(g) u) for the 64 columns of this row: g from the slab (the
-                    // gate block, same rows and columns), u from the packed words in r[0..31];
-                    // m replaces g in the slab and is quantized block by block
-                    const QDest md = mdest(p, block_y(t) + lane, block_x(t));
-                    uint32_t msbs = 0, n0 = 0, n1 = 0, n2 = 0, n3 = 0;
-#pragma unroll
-                    for (int q = 0; q < 8; ++q) {
-                        const uint32_t a = slab + lane * 128 + ((q ^ (lane & 7)) << 4);
-                        uint32_t g4[4], mw[4];
-                        asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
-                                     : "=r"(g4[0]), "=r"(g4[1]), "=r"(g4[2]), "=r"(g4[3])
-                                     : "r"(a));
-#pragma unroll
-                        for (int j = 0; j < 4; ++j)
-                            mw[j] = pack_bf16x2(silu_mul_out(bf16lo(g4[j]), bf16lo(r[4 * q + j])),
-                                                silu_mul_out(bf16hi(g4[j]), bf16hi(r[4 * q + j])));
-                        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(a), "r"(mw[0]), "r"(mw[1]),
-                                     "r"(mw[2]), "r"(mw[3])
-                                     : "memory");
-                        if ((q & 1) && md.codes) {
+                        // the rounded values, kept for the NVFP4 copy (r[] is free again)
+                        r[4 * q] = w0; r[4 * q + 1] = w1; r[4 * q + 2] = w2; r[4 * q + 3] = w3;
+                        if ((q & 1) && qd.codes) {
                             uint32_t lo, hi, sb;
-                            quant16_bf16(make_uint4(n0, n1, n2, n3), make_uint4(mw[0], mw[1], mw[2], mw[3]), &lo, &hi,
-                                         &sb);
-                            *reinterpret_cast<uint2 *>(md.codes + 4 * (q - 1)) = make_uint2(lo, hi);
-                            msbs |= sb << (4 * (q - 1));
+                            quant16_bf16(make_uint4(r[4 * q - 4], r[4 * q - 3], r[4 * q - 2], r[4 * q - 1]),
+                                         make_uint4(w0, w1, w2, w3), &lo, &hi, &sb);
+                            *reinterpret_cast<uint2 *>(qd.codes + 4 * (q - 1)) = make_uint2(lo, hi);
+                            sbs |= sb << (4 * (q - 1));
                         }
-                        n0 = mw[0]; n1 = mw[1]; n2 = mw[2]; n3 = mw[3];
                     }
-                    if (md.scales) *reinterpret_cast<uint32_t *>(md.scales) = msbs;
-                }
-                if (!SILU || up) {   // a gate block is not stored: its m follows with the up block
+                    if (qd.scales) *reinterpret_cast<uint32_t *>(qd.scales) = sbs;
                     fence_proxy_async_smem();
                     __syncwarp();
                     if (lane == 0) {
-                        tma_store_2d(&tmD, slab, up ? block_x(t) - p.half_tiles * BN : block_x(t), block_y(t));
+                        tma_store_2d(&tmD, slab, block_x(t) + 32, block_y(t));
                         bulk_commit_group();
                     }
                 }
@@ -588,9 +677,9 @@ static pact_status ensure_attrs() {
     const int d = current_device();
     if (d >= 0 && d < 64 && done[d]) return PACT_OK;
     cudaError_t e =
-        cudaFuncSetAttribute(k_nvfp4_gemm<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+        cudaFuncSetAttribute(k_nvfp4_gemm<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, Layout<false>::SMEM_BYTES);
     if (e == cudaSuccess)
-        e = cudaFuncSetAttribute(k_nvfp4_gemm<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+        e = cudaFuncSetAttribute(k_nvfp4_gemm<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, Layout<true>::SMEM_BYTES);
     if (e != cudaSuccess) return fail(PACT_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));
     if (d >= 0 && d < 64) done[d] = true;
     return PACT_OK;
@@ -668,17 +757,19 @@ static pact_status run(const pact_nvfp4_t *a, const pact_nvfp4_t *b, int gexp, c
     if (s == PACT_OK)
         s = so ? make_map(&tmD, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, so->m, N / 2, M, so->ldm * 2, 64, 32,
                           CU_TENSOR_MAP_SWIZZLE_128B, what)
-               : make_map(&tmD, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, out, N, M, ldo * 2, 64, 32, CU_TENSOR_MAP_SWIZZLE_128B,
+               : make_map(&tmD, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, out, N, M, ldo * 2, 32, 32, CU_TENSOR_MAP_SWIZZLE_64B,
                           what);
     tmR = tmD;
-    if (s == PACT_OK && res)
-        s = make_map(&tmR, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, res, N, M, ldr * 2, 64, 32, CU_TENSOR_MAP_SWIZZLE_128B,
+    if (s == PACT_OK && res)   // the plain GEMM's residual: the first half of each 32 x 64 block
+        s = make_map(&tmR, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, res, N, M, ldr * 2, 32, 32, CU_TENSOR_MAP_SWIZZLE_64B,
                      what);
     if (s != PACT_OK) return s;
     Params p;
     p.M = (int)M; p.N = (int)N; p.K = (int)K;
     p.has_res = res != nullptr;
     p.out_scale = std::ldexp(1.0f, gexp);
+    p.res = res;
+    p.ldr = ldr;
     // stream the larger operand once: A (M x K) when M > N, else B (N x K)
     p.n_fast = M > N ? 1 : 0;
     p.nq = nq;
@@ -726,7 +817,8 @@ static pact_status run(const pact_nvfp4_t *a, const pact_nvfp4_t *b, int gexp, c
     const int max_clusters = sm_count() / 2;
     const int rounds = (units + max_clusters - 1) / max_clusters;
     const int clusters = (units + rounds - 1) / rounds;
-    return launch_dep(so ? k_nvfp4_gemm<true> : k_nvfp4_gemm<false>, dim3(2 * clusters), dim3(THREADS), SMEM_BYTES,
+    return launch_dep(so ? k_nvfp4_gemm<true> : k_nvfp4_gemm<false>, dim3(2 * clusters), dim3(THREADS),
+                      so ? Layout<true>::SMEM_BYTES : Layout<false>::SMEM_BYTES,
                       stream, what, tmA, tmB, tmSFA, tmSFB, tmLa, tmLb, tmD, tmR, p);
 }
 
