@@ -189,8 +189,8 @@ class Replicas:
 # Valid only for the GEMM source it was taken on: reported as null once csrc/gemm.cu
 # or csrc/common.cuh differ from the recorded hashes.
 GEMM_TRAFFIC = {
-    "llama-3.2-3b": {"bytes_per_launch": 114363072,
-                     "sha256_16": {"gemm.cu": "193d4d9c11bd5b22", "common.cuh": "abb370a5c89b6426"}},
+    "llama-3.2-3b": {"bytes_per_launch": 116853536,
+                     "sha256_16": {"gemm.cu": "8be81cf457ac1318", "common.cuh": "abb370a5c89b6426"}},
 }
 
 
