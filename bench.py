@@ -186,11 +186,13 @@ class Replicas:
 # ------------------------------------------------------------------ CPU oracle
 # DRAM bytes (read + write) per k_nvfp4_gemm launch, mean over the GEMMs of one layer
 # step, from one ncu capture of the step's first eager pass (cold L2), per workload.
-# Valid only for the GEMM source it was taken on: reported as null once csrc/gemm.cu
-# or csrc/common.cuh differ from the recorded hashes.
+# Valid only for the GEMM source it was taken on: reported as null once csrc/gemm.cu,
+# csrc/common.cuh or csrc/quant.cuh (the epilogue's quantizer) differ from the
+# recorded hashes.
 GEMM_TRAFFIC = {
     "llama-3.2-3b": {"bytes_per_launch": 116853536,
-                     "sha256_16": {"gemm.cu": "8be81cf457ac1318", "common.cuh": "abb370a5c89b6426"}},
+                     "sha256_16": {"gemm.cu": "8be81cf457ac1318", "common.cuh": "abb370a5c89b6426",
+                                   "quant.cuh": "ab1a0fd06f3ea89c"}},
 }
 
 

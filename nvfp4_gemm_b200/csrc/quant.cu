@@ -134,8 +134,9 @@ static int resident_per_sm(K kernel) {
 // 13..19 of `field` (FP64's exponent and top mantissa positions): the exponent is
 // rebiased from 127 to 1023, so a normal value comes out exact without a conversion
 // instruction.  Zeros and subnormals come out below 2^-126: their squares (under
-// 2^-252) vanish from any FP64 sum that reaches 2^-200, and a row of them only is
-// governed by eps.  Exponent 255 (infinities, NaN) is left to the caller.
+// 2^-252, at most 2^-238 for a whole row) are below half an ulp of any sum from
+// 2^-180 on, so the callers recompute a sum below that (and one that met exponent
+// 255, infinities and NaN) from plain conversions.
 __device__ __forceinline__ double f64_of_bf16(uint32_t field) {
     return __hiloint2double((int)(field + 0x38000000u), 0);
 }
@@ -150,17 +151,19 @@ constexpr int RMS_MAX_H = 16384;
 // is rounded directly (Ziv, "Fast evaluation of elementary mathematical functions
 // with correctly rounded last bit", ACM TOMS 17(3), 1991).
 // Returns the value whose round-to-nearest BF16 conversion is the result: the FP32
-// product where it decides, else the correctly rounded value itself.
+// product where it decides, else the correctly rounded value itself.  r32 = (float)rstd
+// must be finite: a row whose rstd lies beyond FP32's range (eps = 0 and a row of zeros
+// and subnormals only) is rounded by rms_exact throughout.
+__device__ __forceinline__ bool near_bf16_midpoint(float y) {   // within 64 FP32 ulps of one
+    return (__float_as_uint(y) & 0xFFFFu) - 0x7FC0u <= 0x80u;
+}
+__device__ __forceinline__ float rms_exact(float x, float g, double rstd) {
+    return __bfloat162float(__double2bfloat16(((double)x * rstd) * (double)g));
+}
 __device__ __forceinline__ float rms_out(float x, float g, float r32, double rstd) {
     const float y = __fmul_rn(__fmul_rn(x, r32), g);
-    const uint32_t lo = __float_as_uint(y) & 0xFFFFu;
-    if (lo - 0x7FC0u <= 0x80u) {
-        const double yd = ((double)x * rstd) * (double)g;
-        return __bfloat162float(__double2bfloat16(yd));
-    }
-    return y;
+    return near_bf16_midpoint(y) ? rms_exact(x, g, rstd) : y;
 }
-
 // Ring geometry: slots of `slot_bytes`, as many (2 .. 4) as fit in ~48 KiB, then the
 // slot barriers and `extra` bytes (a shared copy of gamma); as many CTAs per SM (up to
 // 8) as fit in 200 KiB.
@@ -247,22 +250,26 @@ __global__ void __launch_bounds__(RING_THREADS) k_rmsnorm_quant(const pact_bf16 
                 }
             }
         }
-        if (__any_sync(0xFFFFFFFFu, top >= (0xFFu << 20))) {
-            // an infinity or NaN in the row: the sum as plain conversions give it
-            s0 = s1 = s2 = s3 = 0.0;
+        double ss = (s0 + s1) + (s2 + s3);
+#pragma unroll
+        for (int o = 16; o; o >>= 1) ss += __shfl_xor_sync(0xFFFFFFFFu, ss, o);
+        if (__any_sync(0xFFFFFFFFu, top >= (0xFFu << 20)) || !(ss >= 0x1p-180)) {
+            // an infinity or NaN among the warp's values, or a partial sum so small that
+            // the widened zeros and subnormals (each square below 2^-252, at most 2^-238
+            // together) could count: the sum as plain conversions give it
+            ss = 0.0;
             for (int k = warp; k < nchunk; k += RING_WARPS) {
                 const int c = k * CHUNK + 8 * lane;
                 if (c < H) {
                     float v[8];
                     load8_bf16(reinterpret_cast<const pact_bf16 *>(rs) + c, v);
 #pragma unroll
-                    for (int j = 0; j < 8; ++j) s0 = fma((double)v[j], (double)v[j], s0);
+                    for (int j = 0; j < 8; ++j) ss = fma((double)v[j], (double)v[j], ss);
                 }
             }
-        }
-        double ss = (s0 + s1) + (s2 + s3);
 #pragma unroll
-        for (int o = 16; o; o >>= 1) ss += __shfl_xor_sync(0xFFFFFFFFu, ss, o);
+            for (int o = 16; o; o >>= 1) ss += __shfl_xor_sync(0xFFFFFFFFu, ss, o);
+        }
         if (lane == 0) red[warp] = ss;
         __syncthreads();
         if (threadIdx.x == 0) {   // one thread evaluates rstd; the others read it
@@ -273,6 +280,7 @@ __global__ void __launch_bounds__(RING_THREADS) k_rmsnorm_quant(const pact_bf16 
         __syncthreads();
         const double rstd = rstd_s;
         const float r32 = (float)rstd;
+        const bool wide = isinf(r32);
         for (int k = warp; k < nchunk; k += RING_WARPS) {
             const int64_t c0 = (int64_t)k * CHUNK;
             const int64_t c = c0 + 8 * lane;
@@ -282,8 +290,13 @@ __global__ void __launch_bounds__(RING_THREADS) k_rmsnorm_quant(const pact_bf16 
                 load8_bf16(reinterpret_cast<const pact_bf16 *>(rs) + c, v);
                 load8_bf16(gs + c, g);
             }
+            if (wide) {
 #pragma unroll
-            for (int j = 0; j < 8; ++j) o[j] = rms_out(v[j], g[j], r32, rstd);   // zeros past the row end
+                for (int j = 0; j < 8; ++j) o[j] = rms_exact(v[j], g[j], rstd);
+            } else {
+#pragma unroll
+                for (int j = 0; j < 8; ++j) o[j] = rms_out(v[j], g[j], r32, rstd);   // zeros past the row end
+            }
             uint4 ow;
             round8_bf16(o, ow, o);
             if (valid && y) *reinterpret_cast<uint4 *>(y + row * H + c) = ow;
@@ -303,14 +316,32 @@ __global__ void __launch_bounds__(RING_THREADS) k_rmsnorm_quant(const pact_bf16 
     }
 }
 
+// Register-resident RMSNorm backward (below): a warp per row, 128-thread CTAs.
+constexpr int ROWS_THREADS = 128;
+constexpr int ROWS_WARPS = ROWS_THREADS / 32;
+
+// Stage gamma [H] (NB 512-column chunks, zero past H) in shared memory, per 512-column
+// chunk the first halves of its 32 blocks and then the second halves: a lane's two
+// 16-byte reads of its block then hit distinct banks across the warp.
+template <int NB>
+__device__ __forceinline__ void stage_gamma(uint4 *gs, const pact_bf16 *__restrict__ gamma, int64_t H) {
+    for (int i = threadIdx.x; i < NB * 64; i += blockDim.x) {
+        const int c = 512 * (i >> 6) + 16 * (i & 31) + 8 * ((i >> 5) & 1);
+        gs[i] = c < H ? *reinterpret_cast<const uint4 *>(gamma + c) : make_uint4(0u, 0u, 0u, 0u);
+    }
+}
+
 // --------------------------------------------------- A4: SiLU-multiply + quantize
 
 
 // The task loops below are software-pipelined: a warp loads the next task's inputs
 // before it computes the current one, so two tasks' loads are in flight per warp.
 // A task is 512 columns of a row; lane j owns the 16-value block j of every tensor
-// (one scale computation per block, no block-maximum shuffle).
-__global__ void __launch_bounds__(256) k_silu_mul_quant(const pact_bf16 *__restrict__ g, const pact_bf16 *__restrict__ u,
+// (one scale computation per block, no block-maximum shuffle).  GU: the instance that
+// also quantizes g and u (the layer's gate|up GEMM writes those copies itself, so its
+// instance carries neither, and fits three CTAs per SM).
+template <bool GU>
+__global__ void __launch_bounds__(256, GU ? 2 : 3) k_silu_mul_quant(const pact_bf16 *__restrict__ g, const pact_bf16 *__restrict__ u,
                                                         int64_t ld_gu, int64_t M, int64_t I,
                                                         pact_bf16 *__restrict__ m, pact_nvfp4_t mq, pact_nvfp4_t gq,
                                                         pact_nvfp4_t uq, int has_gq, int has_uq) {
@@ -332,14 +363,18 @@ __global__ void __launch_bounds__(256) k_silu_mul_quant(const pact_bf16 *__restr
             v.g0 = gp[0]; v.g1 = gp[1]; v.u0 = up[0]; v.u1 = up[1];
         }
     };
-    // m for 8 values (one 16-byte piece of g and of u): the values to round, in mv
-    auto silu8 = [&](const uint4 &gw, const uint4 &uw, float (&mv)[8]) {
-        const uint32_t gs[4] = {gw.x, gw.y, gw.z, gw.w}, us[4] = {uw.x, uw.y, uw.z, uw.w};
+    // m for 8 values (one 16-byte piece of g and of u) as BF16 words
+    auto silu8 = [&](const uint4 &gw, const uint4 &uw) {
+        float gv[8], uv[8], sv[8], mv[8];
+        unpack8_bf16(gw, gv);
+        unpack8_bf16(uw, uv);
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            mv[2 * j] = silu_mul_out(bf16lo(gs[j]), bf16lo(us[j]));
-            mv[2 * j + 1] = silu_mul_out(bf16hi(gs[j]), bf16hi(us[j]));
-        }
+        for (int i = 0; i < 8; ++i) sv[i] = sigmoid_fast(gv[i]);
+        silu_mul8<false>(gv, uv, sv, mv);
+        uint4 mw;
+        mw.x = pack_bf16x2(mv[0], mv[1]); mw.y = pack_bf16x2(mv[2], mv[3]);
+        mw.z = pack_bf16x2(mv[4], mv[5]); mw.w = pack_bf16x2(mv[6], mv[7]);
+        return mw;
     };
     TaskIter it(warp0, nchunk, nwarps);
     In cur;
@@ -357,15 +392,10 @@ __global__ void __launch_bounds__(256) k_silu_mul_quant(const pact_bf16 *__restr
             const int64_t so = scale_offset(row, c >> 4, I), co = row * (I >> 1) + (c >> 1);
             if (row >= M) {   // a padding row of the scale layout
                 static_cast<uint8_t *>(mq.scales)[so] = 0;
-                if (has_gq) static_cast<uint8_t *>(gq.scales)[so] = 0;
-                if (has_uq) static_cast<uint8_t *>(uq.scales)[so] = 0;
+                if (GU && has_gq) static_cast<uint8_t *>(gq.scales)[so] = 0;
+                if (GU && has_uq) static_cast<uint8_t *>(uq.scales)[so] = 0;
             } else {
-                float mv[8];
-                uint4 m0, m1;
-                silu8(cur.g0, cur.u0, mv);
-                round8_bf16(mv, m0, mv);
-                silu8(cur.g1, cur.u1, mv);
-                round8_bf16(mv, m1, mv);
+                const uint4 m0 = silu8(cur.g0, cur.u0), m1 = silu8(cur.g1, cur.u1);
                 if (m) {
                     uint4 *mp = reinterpret_cast<uint4 *>(m + row * I + c);
                     mp[0] = m0;
@@ -375,12 +405,12 @@ __global__ void __launch_bounds__(256) k_silu_mul_quant(const pact_bf16 *__restr
                 quant16_bf16(m0, m1, &lo, &hi, &sb);
                 *reinterpret_cast<uint2 *>(static_cast<uint8_t *>(mq.codes) + co) = make_uint2(lo, hi);
                 static_cast<uint8_t *>(mq.scales)[so] = (uint8_t)sb;
-                if (has_gq) {
+                if (GU && has_gq) {
                     quant16_bf16(cur.g0, cur.g1, &lo, &hi, &sb);
                     *reinterpret_cast<uint2 *>(static_cast<uint8_t *>(gq.codes) + co) = make_uint2(lo, hi);
                     static_cast<uint8_t *>(gq.scales)[so] = (uint8_t)sb;
                 }
-                if (has_uq) {
+                if (GU && has_uq) {
                     quant16_bf16(cur.u0, cur.u1, &lo, &hi, &sb);
                     *reinterpret_cast<uint2 *>(static_cast<uint8_t *>(uq.codes) + co) = make_uint2(lo, hi);
                     static_cast<uint8_t *>(uq.scales)[so] = (uint8_t)sb;
@@ -437,17 +467,18 @@ __global__ void __launch_bounds__(256) k_silu_mul_bwd_quant(const pact_bf16 *__r
         unpack8_bf16(dw, d);
         dequant8(gc, gsb, gh);
         dequant8(uc, usb, uh);
+        float sg[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) sg[i] = sigmoid_fast(gh[i]);
 #pragma unroll
         for (int i = 0; i < 8; i += 2) {
-            const float s0 = sigmoid_fast(gh[i]), s1 = sigmoid_fast(gh[i + 1]);
-            const uint64_t g2 = f2_pack(gh[i], gh[i + 1]), sg2 = f2_pack(s0, s1);
+            const uint64_t g2 = f2_pack(gh[i], gh[i + 1]), sg2 = f2_pack(sg[i], sg[i + 1]);
             const uint64_t ds = f2_mul(f2_pack(d[i], d[i + 1]), sg2);
             const uint64_t w = f2_fma(g2, f2_fma(sg2, neg2, one2), one2);
             f2_unpack(f2_mul(f2_mul(ds, f2_pack(uh[i], uh[i + 1])), w), dg[i], dg[i + 1]);
             f2_unpack(f2_mul(ds, g2), du[i], du[i + 1]);
-            mr[i] = silu_mul_value<true>(gh[i], uh[i], s0);
-            mr[i + 1] = silu_mul_value<true>(gh[i + 1], uh[i + 1], s1);
         }
+        silu_mul8<true>(gh, uh, sg, mr);
         wg.x = pack_bf16x2(dg[0], dg[1]); wg.y = pack_bf16x2(dg[2], dg[3]);
         wg.z = pack_bf16x2(dg[4], dg[5]); wg.w = pack_bf16x2(dg[6], dg[7]);
         wu.x = pack_bf16x2(du[0], du[1]); wu.y = pack_bf16x2(du[2], du[3]);
@@ -637,6 +668,156 @@ __global__ void __launch_bounds__(RING_THREADS) k_rmsnorm_bwd(const pact_bf16 *_
     }
 }
 
+// ---------------------------------------- A10: RMSNorm backward, rows of up to 4096 columns
+// The layout of k_rmsnorm_quant_rows: a warp per row, lane l owning the blocks at
+// columns 512 j + 16 l.  When a warp starts a row it has the L2 prefetch the next
+// row's dy, codes and dres (one bulk prefetch each).  Pass 1 loads the row's dy and the
+// codes and scale bytes of y^ into registers and forms sum(dy * y^) as, per block, the
+// scale times the sum of dy times the E2M1 values; pass 2, a loop over the lane's
+// blocks, reads each block again (from L1) with its dres and writes
+//   dx = rstd (gamma dy - (y^ / gamma) mean) + dres
+// with 1/gamma from a table staged in shared memory (correctly rounded FP32), and,
+// when asked, the NVFP4 copy of dx.
+constexpr int ROWS_MAX_NB_BWD = 8;
+
+// The 16 values of one E2M1 block (8 code bytes, element 0 in the low nibble of the
+// first byte) as 8 packed FP32 pairs, exactly.
+__device__ __forceinline__ void e2m1_block_f32(uint32_t lo, uint32_t hi, uint64_t (&p)[8]) {
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+        const uint32_t h = e2m1x2_to_f16x2(((k < 4 ? lo : hi) >> (8 * (k & 3))) & 0xFFu);
+        const float2 f = __half22float2(*reinterpret_cast<const __half2 *>(&h));
+        p[k] = f2_pack(f.x, f.y);
+    }
+}
+
+template <int NB>
+__global__ void __launch_bounds__(ROWS_THREADS) k_rmsnorm_bwd_rows(const pact_bf16 *__restrict__ dy, int64_t lddy,
+                                                                  pact_nvfp4_t yq, const float *__restrict__ rstd,
+                                                                  const pact_bf16 *__restrict__ gamma, int64_t M,
+                                                                  int64_t H, const pact_bf16 *__restrict__ dres,
+                                                                  pact_bf16 *__restrict__ dx, pact_nvfp4_t dxq,
+                                                                  int has_dxq) {
+    __shared__ uint4 gs[NB * 64];          // gamma, in the order of stage_gamma
+    __shared__ float4 igs[NB * 128];       // 1 / gamma: per chunk, quarter k of lane l's block at 32 k + l
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int64_t rows = has_dxq ? (M + 127) & ~int64_t(127) : M;
+    const int64_t nw = (int64_t)gridDim.x * ROWS_WARPS;
+    const uint8_t *ycodes = static_cast<const uint8_t *>(yq.codes), *yscales = static_cast<const uint8_t *>(yq.scales);
+    uint8_t *codes = static_cast<uint8_t *>(dxq.codes), *scales = static_cast<uint8_t *>(dxq.scales);
+    pdl_wait();
+    stage_gamma<NB>(gs, gamma, H);
+    for (int i = threadIdx.x; i < NB * 128; i += blockDim.x) {
+        // float4 i: chunk j = i / 128, quarter k = (i / 32) % 4 of the block of lane l = i % 32
+        const int c = 512 * (i >> 7) + 16 * (i & 31) + 4 * ((i >> 5) & 3);
+        float4 f = make_float4(1.0f, 1.0f, 1.0f, 1.0f);
+        if (c < H) {
+            const uint2 g = *reinterpret_cast<const uint2 *>(gamma + c);
+            f = make_float4(1.0f / bf16lo(g.x), 1.0f / bf16hi(g.x), 1.0f / bf16lo(g.y), 1.0f / bf16hi(g.y));
+        }
+        igs[i] = f;
+    }
+    __syncthreads();
+    for (int64_t row = (int64_t)warp * gridDim.x + blockIdx.x; row < rows; row += nw) {   // as the forward
+        if (row >= M) {   // a padding row of dxq's scale layout: zero scales
+#pragma unroll 1
+            for (int c = 16 * lane; c < H; c += 512) scales[scale_offset(row, c >> 4, H)] = 0;
+            continue;
+        }
+        if (lane == 0 && row + nw < M) {
+            const int64_t n = row + nw;
+            bulk_prefetch_l2(dy + n * lddy, (uint32_t)(H * 2));
+            bulk_prefetch_l2(ycodes + n * (H >> 1), (uint32_t)(H >> 1));
+            if (dres) bulk_prefetch_l2(dres + n * H, (uint32_t)(H * 2));
+        }
+        const pact_bf16 *dyr = dy + row * lddy;
+        const uint8_t *ycr = ycodes + row * (H >> 1);
+        // pass 1: sum(dy * y^); lanes whose block lies past the row end hold zeros
+        uint4 d[2 * NB];
+        uint2 q[NB];
+        uint32_t sq[NB];
+#pragma unroll
+        for (int j = 0; j < NB; ++j) {
+            const int c = 512 * j + 16 * lane;
+            d[2 * j] = d[2 * j + 1] = make_uint4(0u, 0u, 0u, 0u);
+            q[j] = make_uint2(0u, 0u);
+            sq[j] = 0u;
+            if (c < H) {
+                const uint4 *p = reinterpret_cast<const uint4 *>(dyr + c);
+                d[2 * j] = p[0];
+                d[2 * j + 1] = p[1];
+                q[j] = *reinterpret_cast<const uint2 *>(ycr + (c >> 1));
+                sq[j] = yscales[scale_offset(row, c >> 4, H)];
+            }
+        }
+        const float r = rstd[row];
+        float dot = 0.0f;
+#pragma unroll
+        for (int j = 0; j < NB; ++j) {
+            const uint32_t dw[8] = {d[2 * j].x, d[2 * j].y, d[2 * j].z, d[2 * j].w,
+                                    d[2 * j + 1].x, d[2 * j + 1].y, d[2 * j + 1].z, d[2 * j + 1].w};
+            uint64_t e[8];
+            e2m1_block_f32(q[j].x, q[j].y, e);
+            uint64_t acc = f2_pack(0.0f, 0.0f);
+#pragma unroll
+            for (int k = 0; k < 8; ++k) acc = f2_fma(f2_pack(bf16lo(dw[k]), bf16hi(dw[k])), e[k], acc);
+            float a0, a1;
+            f2_unpack(acc, a0, a1);
+            dot = fmaf(e4m3_to_float(sq[j]), a0 + a1, dot);
+        }
+#pragma unroll
+        for (int o = 16; o; o >>= 1) dot += __shfl_xor_sync(0xFFFFFFFFu, dot, o);
+        const float mean = dot / (float)H;
+        const uint64_t r2 = f2_pack(r, r), nm2 = f2_pack(-mean, -mean);
+        // pass 2
+#pragma unroll 1
+        for (int c = 16 * lane; c < H; c += 512) {
+            const uint4 *p = reinterpret_cast<const uint4 *>(dyr + c);
+            const uint4 da = p[0], db = p[1];
+            uint4 ra = make_uint4(0u, 0u, 0u, 0u), rb = ra;
+            if (dres) {
+                const uint4 *pr = reinterpret_cast<const uint4 *>(dres + row * H + c);
+                ra = pr[0];
+                rb = pr[1];
+            }
+            const uint2 qc = *reinterpret_cast<const uint2 *>(ycr + (c >> 1));
+            const float sc = e4m3_to_float(yscales[scale_offset(row, c >> 4, H)]);
+            const uint32_t dw[8] = {da.x, da.y, da.z, da.w, db.x, db.y, db.z, db.w};
+            const uint32_t rw[8] = {ra.x, ra.y, ra.z, ra.w, rb.x, rb.y, rb.z, rb.w};
+            const int gi = (c >> 9) * 64 + lane;
+            const uint4 ga = gs[gi], gb = gs[gi + 32];
+            const uint32_t gw[8] = {ga.x, ga.y, ga.z, ga.w, gb.x, gb.y, gb.z, gb.w};
+            const float4 *ig = &igs[(c >> 9) * 128 + lane];
+            const uint64_t sc2 = f2_pack(sc, sc);
+            uint64_t e[8];
+            e2m1_block_f32(qc.x, qc.y, e);
+            uint32_t ow[8];
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {
+                const float4 i4 = ig[32 * (k >> 1)];
+                const uint64_t ig2 = (k & 1) ? f2_pack(i4.z, i4.w) : f2_pack(i4.x, i4.y);
+                const uint64_t yh = f2_mul(e[k], sc2);                                   // y^ (exact)
+                const uint64_t t = f2_mul(f2_pack(bf16lo(gw[k]), bf16hi(gw[k])),
+                                          f2_pack(bf16lo(dw[k]), bf16hi(dw[k])));       // gamma dy
+                const uint64_t u = f2_fma(f2_mul(yh, ig2), nm2, t);                       // - (y^ / gamma) mean
+                float o0, o1;
+                f2_unpack(f2_fma(r2, u, f2_pack(bf16lo(rw[k]), bf16hi(rw[k]))), o0, o1);
+                ow[k] = pack_bf16x2(o0, o1);
+            }
+            const uint4 xa = make_uint4(ow[0], ow[1], ow[2], ow[3]), xb = make_uint4(ow[4], ow[5], ow[6], ow[7]);
+            uint4 *xp = reinterpret_cast<uint4 *>(dx + row * H + c);
+            xp[0] = xa;
+            xp[1] = xb;
+            if (has_dxq) {
+                uint32_t lo, hi, sb;
+                quant16_bf16(xa, xb, &lo, &hi, &sb);
+                *reinterpret_cast<uint2 *>(codes + row * (H >> 1) + (c >> 1)) = make_uint2(lo, hi);
+                scales[scale_offset(row, c >> 4, H)] = (uint8_t)sb;
+            }
+        }
+    }
+}
+
 // ------------------------------------------------------- A1: backward weight layout
 // Wb = q(deq(Wf)^T): a CTA turns a 64 (n) x 64 (k) tile of the forward layout into
 // 64 rows (k) x 4 blocks (n) of the backward layout.  Runs once per frozen weight.
@@ -704,6 +885,28 @@ __global__ void k_zero_scale_pad(pact_nvfp4_t t) {
         const int64_t r = t.rows + i / nblk, c = i % nblk;
         static_cast<uint8_t *>(t.scales)[scale_offset(r, c, t.cols)] = 0;
     }
+}
+
+// Register-resident RMSNorm backward: one instance per number of 512-column chunks.
+using RmsRowsBwd = void (*)(const pact_bf16 *, int64_t, pact_nvfp4_t, const float *, const pact_bf16 *, int64_t,
+                            int64_t, const pact_bf16 *, pact_bf16 *, pact_nvfp4_t, int);
+static const RmsRowsBwd kRmsRowsBwd[ROWS_MAX_NB_BWD] = {
+    k_rmsnorm_bwd_rows<1>, k_rmsnorm_bwd_rows<2>, k_rmsnorm_bwd_rows<3>, k_rmsnorm_bwd_rows<4>,
+    k_rmsnorm_bwd_rows<5>, k_rmsnorm_bwd_rows<6>, k_rmsnorm_bwd_rows<7>, k_rmsnorm_bwd_rows<8>};
+
+// Grid of a register-resident kernel: one resident wave of CTAs (they are issue-bound:
+// every SM gets the same number of CTAs), or fewer when the rows do not need them all.
+// `per_sm` caches the kernel's residency (0 until the first call).
+template <typename K>
+static int rows_grid(K kernel, int &per_sm, int64_t rows, size_t smem = 0) {
+    if (per_sm == 0) {
+        int n = 0;
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kernel, ROWS_THREADS, smem) != cudaSuccess || n < 1)
+            n = 1;
+        per_sm = n;
+    }
+    const int64_t need = (rows + ROWS_WARPS - 1) / ROWS_WARPS, cap = (int64_t)sm_count() * per_sm;
+    return (int)(need < cap ? need : cap);
 }
 
 }  // namespace pact
@@ -813,10 +1016,15 @@ pact_status pact_silu_mul_quant(const pact_bf16 *g, const pact_bf16 *u, int64_t 
     if (s != PACT_OK) return s;
     pact_nvfp4_t none = {nullptr, nullptr, M, I};
     const int64_t tasks = ((M + 127) / 128 * 128) * ((I + QCHUNK - 1) / QCHUNK);
-    static const int per_sm = resident_per_sm(k_silu_mul_quant);
-    return launch_dep(k_silu_mul_quant, dim3(grid_for(tasks, 256, per_sm)), dim3(256), 0, (cudaStream_t)stream,
-                      "pact_silu_mul_quant", g, u, ld_gu, M, I, m, *mq, gq ? *gq : none, uq ? *uq : none,
-                      (int)(gq != nullptr), (int)(uq != nullptr));
+    if (gq || uq) {
+        static const int per_sm = resident_per_sm(k_silu_mul_quant<true>);
+        return launch_dep(k_silu_mul_quant<true>, dim3(grid_for(tasks, 256, per_sm)), dim3(256), 0,
+                          (cudaStream_t)stream, "pact_silu_mul_quant", g, u, ld_gu, M, I, m, *mq, gq ? *gq : none,
+                          uq ? *uq : none, (int)(gq != nullptr), (int)(uq != nullptr));
+    }
+    static const int per_sm = resident_per_sm(k_silu_mul_quant<false>);
+    return launch_dep(k_silu_mul_quant<false>, dim3(grid_for(tasks, 256, per_sm)), dim3(256), 0, (cudaStream_t)stream,
+                      "pact_silu_mul_quant", g, u, ld_gu, M, I, m, *mq, none, none, 0, 0);
 }
 
 pact_status pact_silu_mul_bwd_quant(const pact_bf16 *dm, int64_t lddm, const pact_nvfp4_t *gq, const pact_nvfp4_t *uq,
@@ -852,6 +1060,14 @@ pact_status pact_rmsnorm_bwd(const pact_bf16 *dy, int64_t lddy, const pact_nvfp4
     pact_nvfp4_t none = {nullptr, nullptr, M, H};
     const int64_t rows = dxq ? (M + 127) / 128 * 128 : M;
     PACT_CHECK(rows <= 0x7FFFFFFF, PACT_ERR_SHAPE, "pact_rmsnorm_bwd: M too large");
+    if (H <= 512 * ROWS_MAX_NB_BWD) {
+        static int per_sm[ROWS_MAX_NB_BWD] = {0};
+        const int nb = (int)((H + 511) / 512);
+        const int grid = rows_grid(kRmsRowsBwd[nb - 1], per_sm[nb - 1], rows);
+        return launch_dep(kRmsRowsBwd[nb - 1], dim3(grid), dim3(ROWS_THREADS), 0, (cudaStream_t)stream,
+                          "pact_rmsnorm_bwd", dy, lddy, *yq, rstd, gamma, M, H, dres, dx, dxq ? *dxq : none,
+                          (int)(dxq != nullptr));
+    }
     const BwdSlot sl = bwd_slot(H);
     const Ring r = ring_for(rows, (size_t)(dres ? sl.dres_off + H * 2 : sl.codes_off + H / 2), (size_t)H * 2);
     static bool attr_done[64] = {false};

@@ -12,6 +12,12 @@
 
 namespace pact {
 
+// Have the L2 prefetch `bytes` of global memory (source 16-byte aligned, bytes a
+// multiple of 16); no completion to wait for.
+__device__ __forceinline__ void bulk_prefetch_l2(const void *src, uint32_t bytes) {
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
+}
+
 // Byte offset of the scale of (row r, block c) in the tiled scale layout of a
 // tensor with `cols` columns (cols a multiple of 64).
 __host__ __device__ __forceinline__ int64_t scale_offset(int64_t r, int64_t c, int64_t cols) {
@@ -61,16 +67,6 @@ __device__ __forceinline__ void neg_quotient2(float a0, float a1, uint64_t s2, u
 }
 constexpr uint32_t CODE_SIGNS = 0x88888888u;   // the sign bit of all 8 codes of a word
 
-// Two E2M1 codes (RNE, saturating, signs kept) of a pair of quotients as one byte:
-// element 0 in the low nibble.
-__device__ __forceinline__ uint32_t e2m1_pair(float q0, float q1) {
-    uint32_t byte;
-    asm("{\n\t.reg .b8 t;\n\tcvt.rn.satfinite.e2m1x2.f32 t, %2, %1;\n\tcvt.u32.u8 %0, t;\n\t}"
-        : "=r"(byte)
-        : "f"(q0), "f"(q1));
-    return byte;
-}
-
 // amax -> E4M3 scale byte: RNE(amax / 6) with saturation.  The product with the
 // correctly rounded FP32 value of 1/6 takes the same decision as the exact quotient
 // for every BF16 amax (checked over all of them by the tests).
@@ -78,6 +74,29 @@ __device__ __forceinline__ uint32_t scale_byte(float amax) {
     uint16_t r;
     asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(0.0f), "f"(__fmul_rn(amax, 1.0f / 6.0f)));
     return r & 0xFFu;
+}
+
+// max(|a|, |b|) of each BF16 half of two packed words (the sign bits come out as their
+// XOR; a NaN half yields the other operand's half, as fmaxf does).
+__device__ __forceinline__ uint32_t bf16x2_absmax(uint32_t a, uint32_t b) {
+    uint32_t r;
+    asm("max.xorsign.abs.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+    return r;
+}
+
+// The E2M1 codes of 8 quotients (RNE, saturating, signs kept) as one word: element 0
+// in the low nibble.
+__device__ __forceinline__ uint32_t e2m1_word(const float *q) {
+    uint32_t out;
+    asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b0, %2, %1;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b1, %4, %3;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b2, %6, %5;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b3, %8, %7;\n\t"
+        "mov.b32 %0, {b0, b1, b2, b3};\n\t}"
+        : "=r"(out)
+        : "f"(q[0]), "f"(q[1]), "f"(q[2]), "f"(q[3]), "f"(q[4]), "f"(q[5]), "f"(q[6]), "f"(q[7]));
+    return out;
 }
 
 // Quantize the 8 values of this lane (v[0] is the lowest column); the partner lane
@@ -98,43 +117,42 @@ __device__ __forceinline__ uint32_t quant8(const float (&v)[8], uint32_t *sb) {
     float q[8];
 #pragma unroll
     for (int i = 0; i < 8; i += 2) neg_quotient2(v[i], v[i + 1], s2, nr2, q[i], q[i + 1]);
-    uint32_t out;
-    asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
-        "cvt.rn.satfinite.e2m1x2.f32 b0, %2, %1;\n\t"
-        "cvt.rn.satfinite.e2m1x2.f32 b1, %4, %3;\n\t"
-        "cvt.rn.satfinite.e2m1x2.f32 b2, %6, %5;\n\t"
-        "cvt.rn.satfinite.e2m1x2.f32 b3, %8, %7;\n\t"
-        "mov.b32 %0, {b0, b1, b2, b3};\n\t}"
-        : "=r"(out)
-        : "f"(q[0]), "f"(q[1]), "f"(q[2]), "f"(q[3]), "f"(q[4]), "f"(q[5]), "f"(q[6]), "f"(q[7]));
     *sb = b;
-    return out ^ CODE_SIGNS;
+    return e2m1_word(q) ^ CODE_SIGNS;
+}
+
+// Codes and scale byte of a block whose magnitude maximum is amax, from the 16 values
+// as 8 pairs (element 2j, 2j+1 in pair j).
+template <typename Pair>
+__device__ __forceinline__ void quant16_from(float amax, Pair pair, uint32_t *lo, uint32_t *hi, uint32_t *sb) {
+    const uint32_t b = scale_byte(amax);
+    const float s = e4m3_to_float(b);
+    const float nr = b ? -__frcp_rn(s) : -0.0f;
+    const uint64_t nr2 = f2_pack(nr, nr), s2 = f2_pack(s, s);
+    float q[16];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+        float a0, a1;
+        pair(j, a0, a1);
+        neg_quotient2(a0, a1, s2, nr2, q[2 * j], q[2 * j + 1]);
+    }
+    *lo = e2m1_word(q) ^ CODE_SIGNS;
+    *hi = e2m1_word(q + 8) ^ CODE_SIGNS;
+    *sb = b;
 }
 
 // Quantize one NVFP4 block of 16 BF16 values held by one thread as 8 packed words
 // (values 2j, 2j+1 in the low and high half of word j of wa, wb): the 8 code bytes go to *lo
 // (elements 0..7, element 0 in the low nibble) and *hi (8..15), the scale byte to
-// *sb.  Same arithmetic as quant8 (without the shuffle), one pair at a time so that
-// little state is live.
+// *sb.  Same arithmetic as quant8, without the shuffle; the block maximum is taken on
+// the packed words.
 __device__ __forceinline__ void quant16_bf16(const uint4 wa, const uint4 wb, uint32_t *lo, uint32_t *hi, uint32_t *sb) {
     const uint32_t w[8] = {wa.x, wa.y, wa.z, wa.w, wb.x, wb.y, wb.z, wb.w};
-    float amax = 0.0f;
-#pragma unroll
-    for (int j = 0; j < 8; ++j) amax = fmaxf(amax, fmaxf(fabsf(bf16lo(w[j])), fabsf(bf16hi(w[j]))));
-    const uint32_t b = scale_byte(amax);
-    const float s = e4m3_to_float(b);
-    const float nr = b ? -__frcp_rn(s) : -0.0f;
-    const uint64_t nr2 = f2_pack(nr, nr), s2 = f2_pack(s, s);
-    uint32_t out[2] = {0u, 0u};
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-        float q0, q1;
-        neg_quotient2(bf16lo(w[j]), bf16hi(w[j]), s2, nr2, q0, q1);
-        out[j >> 2] |= e2m1_pair(q0, q1) << (8 * (j & 3));
-    }
-    *lo = out[0] ^ CODE_SIGNS;
-    *hi = out[1] ^ CODE_SIGNS;
-    *sb = b;
+    const uint32_t m = bf16x2_absmax(bf16x2_absmax(bf16x2_absmax(w[0], w[1]), bf16x2_absmax(w[2], w[3])),
+                                     bf16x2_absmax(bf16x2_absmax(w[4], w[5]), bf16x2_absmax(w[6], w[7])));
+    // fmaxf with 0 first: a block of NaN only has amax 0, as a running fmaxf from 0 gives
+    const float amax = fmaxf(0.0f, fmaxf(fabsf(bf16lo(m)), fabsf(bf16hi(m))));
+    quant16_from(amax, [&](int j, float &a0, float &a1) { a0 = bf16lo(w[j]); a1 = bf16hi(w[j]); }, lo, hi, sb);
 }
 
 // quant16_bf16 for 16 FP32 values (the same decisions for values that are BF16).
@@ -142,20 +160,7 @@ __device__ __forceinline__ void quant16_f32(const float (&v)[16], uint32_t *lo, 
     float amax = 0.0f;
 #pragma unroll
     for (int j = 0; j < 16; ++j) amax = fmaxf(amax, fabsf(v[j]));
-    const uint32_t b = scale_byte(amax);
-    const float s = e4m3_to_float(b);
-    const float nr = b ? -__frcp_rn(s) : -0.0f;
-    const uint64_t nr2 = f2_pack(nr, nr), s2 = f2_pack(s, s);
-    uint32_t out[2] = {0u, 0u};
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-        float q0, q1;
-        neg_quotient2(v[2 * j], v[2 * j + 1], s2, nr2, q0, q1);
-        out[j >> 2] |= e2m1_pair(q0, q1) << (8 * (j & 3));
-    }
-    *lo = out[0] ^ CODE_SIGNS;
-    *hi = out[1] ^ CODE_SIGNS;
-    *sb = b;
+    quant16_from(amax, [&](int j, float &a0, float &a1) { a0 = v[2 * j]; a1 = v[2 * j + 1]; }, lo, hi, sb);
 }
 
 // Gather the scales of blocks 4q..4q+3 (lanes 8q, 8q+2, 8q+4, 8q+6) into lane 8q
@@ -232,34 +237,57 @@ __device__ __forceinline__ void load8_nvfp4(const pact_nvfp4_t &t, int64_t row, 
 }
 
 // m = BF16_RNE(silu(g) * u), exactly rounded.  The FP32 evaluation with the fast
-// exponential and division has a relative error of at most (5 + 1.16 |g|) FP32
-// ulps (CUDA's documented bounds for __expf and __fdividef plus three roundings),
-// i.e. at most 2 (5 + 1.16 |g|) = 10 + 2.32 |g| ulps of the result: under 19.3 for
-// |g| <= 4 and under 47.2 for |g| <= 16.  It decides unless it lies within 24 (resp.
-// 48) ulps of a BF16 midpoint, and the double expression decides otherwise and for
-// |g| > 16 (Ziv's method, as above).  Two margins keep the double path rare both for
-// gate activations of unit scale and for the wider ones of outlier weights, without
-// a float-to-integer conversion per element.
+// exponential and division has a relative error of at most (5 + 1.16 |g|) FP32 ulps
+// (CUDA's documented bounds for __expf and __fdividef plus three roundings), i.e. at
+// most 2 (5 + 1.16 |g|) = 10 + 2.32 |g| ulps of the result: under 47.2 for |g| <= 16.
+// It decides unless it lies within 48 ulps of a BF16 midpoint, and the double
+// expression decides otherwise and for |g| > 16 (Ziv's method, as above).  One margin
+// for every |g| keeps the test at three integer operations; the double path stays
+// rare (about 0.15 % of values).
 __device__ __forceinline__ float sigmoid_fast(float g) { return __fdividef(1.0f, 1.0f + __expf(-g)); }
 
+// True when m = (g s) u (FP32, s = sigmoid_fast(g)) does not decide BF16_RNE(silu(g) u):
+// m within 48 ulps of a BF16 midpoint, |g| > 16 or NaN, or (unless BOUNDED: u is known
+// to be finite, so a finite g of at most 16 gives a finite m) m not finite.
+template <bool BOUNDED>
+__device__ __forceinline__ bool silu_undecided(float g, float m) {
+    return ((__float_as_uint(m) + 0x8030u) & 0xFFFFu) <= 0x60u || !(fabsf(g) <= 16.0f) ||
+           (!BOUNDED && !isfinite(m));
+}
+// BF16_RNE(silu(g) u) from the double expression (a BF16 value, returned as a float).
+__device__ __forceinline__ float silu_exact(float g, float u) {
+    const double gd = (double)g;
+    return __bfloat162float(__double2bfloat16((gd / (1.0 + exp(-gd))) * (double)u));
+}
+
 // The value whose round-to-nearest BF16 conversion is BF16_RNE(silu(g) u): the FP32
-// product where it decides, else the exactly rounded value itself (a BF16 value, so
-// converting it again changes nothing).  s = sigmoid_fast(g).  BOUNDED: u is known
-// to be finite (dequantized NVFP4), so a finite g of at most 16 gives a finite m.
+// product where it decides, else the exactly rounded value itself.
 template <bool BOUNDED = false>
 __device__ __forceinline__ float silu_mul_value(float g, float u, float s) {
     const float m = __fmul_rn(__fmul_rn(g, s), u);
-    // |low 16 bits - 0x8000| <= margin, as one unsigned range test
-    const float ag = fabsf(g);
-    const uint32_t margin = ag <= 4.0f ? 24u : 48u;
-    if ((__float_as_uint(m) & 0xFFFFu) + margin - 0x8000u <= 2u * margin || !(ag <= 16.0f) ||
-        (!BOUNDED && !isfinite(m))) {
-        const double gd = (double)g;
-        return __bfloat162float(__double2bfloat16((gd / (1.0 + exp(-gd))) * (double)u));
-    }
-    return m;
+    return silu_undecided<BOUNDED>(g, m) ? silu_exact(g, u) : m;
 }
 __device__ __forceinline__ float silu_mul_out(float g, float u) { return silu_mul_value(g, u, sigmoid_fast(g)); }
+
+// silu_mul_value for 8 values, the products two at a time (packed FP32, the same
+// roundings) and the rounding test once for all 8: into mv.  The FP64 path stays
+// inline: moved out of line (a call per undecided group) the kernels got 10 % slower.
+template <bool BOUNDED>
+__device__ __forceinline__ void silu_mul8(const float (&g)[8], const float (&u)[8], const float (&s)[8],
+                                          float (&mv)[8]) {
+    bool slow = false;
+#pragma unroll
+    for (int i = 0; i < 8; i += 2) {
+        f2_unpack(f2_mul(f2_mul(f2_pack(g[i], g[i + 1]), f2_pack(s[i], s[i + 1])), f2_pack(u[i], u[i + 1])),
+                  mv[i], mv[i + 1]);
+        slow |= silu_undecided<BOUNDED>(g[i], mv[i]) | silu_undecided<BOUNDED>(g[i + 1], mv[i + 1]);
+    }
+    if (slow) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+            if (silu_undecided<BOUNDED>(g[i], mv[i])) mv[i] = silu_exact(g[i], u[i]);
+    }
+}
 
 // 8 packed BF16 values -> floats (element 0 in the low half of .x).
 __device__ __forceinline__ void unpack8_bf16(const uint4 &u, float (&v)[8]) {

@@ -376,7 +376,10 @@ def test_lora_bwd(P, orc, guards, M, parts, r, K):
 
 
 # --------------------------------------------------------------- fused producers
-@pytest.mark.parametrize("M,H", [(64, 512), (257, 2048), (96, 3072), (33, 1536)])
+# several rows per CTA ring (one row slot per row in flight), ragged row counts; 16384
+# is the widest row the entry point accepts
+@pytest.mark.parametrize("M,H", [(64, 512), (257, 2048), (96, 3072), (33, 1536), (40, 4096), (24, 8192),
+                                 (9, 16384)])
 def test_rmsnorm_quant(P, orc, guards, M, H):
     x = synth.gaussian_bf16(1, (M, H))
     g = synth.gaussian_bf16(40, (H,), std=0.02, mean=1.0)
@@ -388,6 +391,65 @@ def test_rmsnorm_quant(P, orc, guards, M, H):
     assert np.array_equal(yb, y_ref), f"y differs at {np.argwhere(yb != y_ref)[:3].tolist()}"
     assert_nvfp4_equal(yq, yq_ref, orc, "yq")
     np.testing.assert_allclose(rstd.cpu().numpy(), rstd_ref, rtol=1e-7)
+
+
+def _special_rows(H, eps):
+    """BF16 rows at the edges of RMSNorm's arithmetic: all zeros (eps > 0 only: with eps
+    = 0 the result is 0 * inf), subnormals only (with eps = 0 the rstd of the second
+    such row lies beyond FP32's range), tiny and huge normal values, a single non-zero
+    value, subnormals with one normal value, and two ordinary rows."""
+    g = synth.gaussian_bf16(3, (8, H)).astype(np.uint16)
+    u = synth.uniform(77, 2 * H)
+    sign = np.where(u[H:] < 0.5, 0x8000, 0)
+    sub = ((1 + np.floor(u[:H] * 127)).astype(np.uint16) | sign).astype(np.uint16)
+    sub_small = ((1 + np.floor(u[:H] * 7)).astype(np.uint16) | sign).astype(np.uint16)
+    f32 = lambda a: synth.f64_to_bf16_bits(np.asarray(a, dtype=np.float64))
+    rows = [np.zeros(H, np.uint16) if eps > 0 else g[0],
+            sub,
+            f32(synth.bf16_bits_to_f64(g[1]) * 2.0 ** -100),
+            f32(synth.bf16_bits_to_f64(g[2]) * 2.0 ** 60),
+            np.where(np.arange(H) == H // 3, g[3], 0).astype(np.uint16),
+            np.where(np.arange(H) == 5, g[4], sub).astype(np.uint16),
+            g[5], g[6], sub_small]
+    return np.stack(rows)
+
+
+@pytest.mark.parametrize("H", [3072, 8192])
+@pytest.mark.parametrize("eps", [1e-5, 0.0])
+def test_rmsnorm_quant_special_rows(P, orc, guards, H, eps):
+    x = _special_rows(H, eps)
+    M = x.shape[0]
+    g = synth.gaussian_bf16(40, (H,), std=0.02, mean=1.0)
+    yq, y, rstd = P.pact_rmsnorm_quant(to_dev(x), to_dev(g), eps, yq=guards.nvfp4(M, H), y=guards.matrix(M, H),
+                                       rstd=guards.matrix(1, M, torch.float32)[0])
+    sync()
+    # the entry point takes eps as FP32: the oracle gets that value (rows of zeros and
+    # subnormals have rstd = 1/sqrt(eps), which tells 1e-5 from FP32(1e-5))
+    y_ref, yq_ref, rstd_ref = orc.rmsnorm_quant(x, g, float(np.float32(eps)))
+    yb = to_bits(y)
+    assert np.array_equal(yb, y_ref), f"y differs at {np.argwhere(yb != y_ref)[:3].tolist()}"
+    assert_nvfp4_equal(yq, yq_ref, orc, "yq")
+    with np.errstate(over="ignore"):   # the kernel writes rstd as FP32: beyond its range, inf
+        np.testing.assert_array_equal(rstd.cpu().numpy(), rstd_ref.astype(np.float32))
+
+
+@pytest.mark.parametrize("H", [3072, 8192])
+def test_rmsnorm_quant_nonfinite_rows(P, orc, H):
+    """An infinity or a NaN in a row makes rstd 0 or NaN: y is then 0 where x is finite
+    and NaN elsewhere (compared as NaN, whatever its payload)."""
+    x = synth.gaussian_bf16(5, (4, H)).astype(np.uint16)
+    x[0, 7] = 0x7F80        # +inf
+    x[1, H - 1] = 0xFF80    # -inf
+    x[2, 100] = 0x7FC1      # NaN
+    g = synth.gaussian_bf16(40, (H,), std=0.02, mean=1.0)
+    _, y, rstd = P.pact_rmsnorm_quant(to_dev(x), to_dev(g), 1e-5)
+    sync()
+    y_ref, _, rstd_ref = orc.rmsnorm_quant(x, g, float(np.float32(1e-5)))
+    got, want = synth.bf16_bits_to_f64(to_bits(y)), synth.bf16_bits_to_f64(y_ref)
+    assert np.array_equal(np.isnan(got), np.isnan(want))
+    ok = ~np.isnan(want)
+    assert np.array_equal(to_bits(y)[ok], y_ref[ok])
+    np.testing.assert_array_equal(rstd.cpu().numpy(), rstd_ref.astype(np.float32))
 
 
 @pytest.mark.parametrize("M,I,std", [(64, 512, 2.0), (130, 8960, 2.0), (257, 2048, 2.0), (96, 2048, 9.0)])
@@ -425,7 +487,9 @@ def test_silu_mul_bwd_quant(P, orc, guards, M, I, std):
     assert np.array_equal(mr, want), f"m~ differs at {np.argwhere(mr != want)[:3].tolist()}"
 
 
-@pytest.mark.parametrize("M,H,with_res", [(64, 512, False), (130, 2048, True), (33, 3072, True)])
+# rows of up to 4096 columns take the register-resident kernel, wider ones the ring
+@pytest.mark.parametrize("M,H,with_res", [(64, 512, False), (130, 2048, True), (33, 3072, True), (40, 1536, False),
+                                          (24, 4096, True), (9, 8192, False)])
 def test_rmsnorm_bwd(P, orc, guards, M, H, with_res):
     x = synth.gaussian_bf16(1, (M, H))
     g = synth.gaussian_bf16(40, (H,), std=0.02, mean=1.0)
