@@ -151,19 +151,22 @@ constexpr int RMS_MAX_H = 16384;
 // is rounded directly (Ziv, "Fast evaluation of elementary mathematical functions
 // with correctly rounded last bit", ACM TOMS 17(3), 1991).
 // Returns the value whose round-to-nearest BF16 conversion is the result: the FP32
-// product where it decides, else the correctly rounded value itself.  r32 = (float)rstd
-// must be finite: a row whose rstd lies beyond FP32's range (eps = 0 and a row of zeros
-// and subnormals only) is rounded by rms_exact throughout.
-__device__ __forceinline__ bool near_bf16_midpoint(float y) {   // within 64 FP32 ulps of one
-    return (__float_as_uint(y) & 0xFFFFu) - 0x7FC0u <= 0x80u;
+// product where it decides, else the correctly rounded value itself.
+__device__ __forceinline__ float rms_out(float x, float g, float r32, double rstd) {
+    const float y = __fmul_rn(__fmul_rn(x, r32), g);
+    const uint32_t lo = __float_as_uint(y) & 0xFFFFu;
+    if (lo - 0x7FC0u <= 0x80u) {
+        const double yd = ((double)x * rstd) * (double)g;
+        return __bfloat162float(__double2bfloat16(yd));
+    }
+    return y;
 }
+// The same value from the double expression alone: for a row whose rstd lies beyond
+// FP32's range, which needs eps = 0 and a row of zeros and subnormals only.
 __device__ __forceinline__ float rms_exact(float x, float g, double rstd) {
     return __bfloat162float(__double2bfloat16(((double)x * rstd) * (double)g));
 }
-__device__ __forceinline__ float rms_out(float x, float g, float r32, double rstd) {
-    const float y = __fmul_rn(__fmul_rn(x, r32), g);
-    return near_bf16_midpoint(y) ? rms_exact(x, g, rstd) : y;
-}
+
 // Ring geometry: slots of `slot_bytes`, as many (2 .. 4) as fit in ~48 KiB, then the
 // slot barriers and `extra` bytes (a shared copy of gamma); as many CTAs per SM (up to
 // 8) as fit in 200 KiB.
@@ -185,6 +188,12 @@ static Ring ring_for(int64_t rows, size_t slot_bytes, size_t extra) {
     return r;
 }
 
+// EPS0: the instance for eps = 0, where a row of zeros and subnormals can have an rstd
+// beyond FP32's range (rounded by rms_exact throughout) and a sum of squares small
+// enough for the widened zeros and subnormals of f64_of_bf16 to count (summed again
+// from plain conversions).  With eps > 0 neither can change a result: rstd is at most
+// 2^74.5, and eps hides the widened values' 2^-238 at most.
+template <bool EPS0>
 __global__ void __launch_bounds__(RING_THREADS) k_rmsnorm_quant(const pact_bf16 *__restrict__ x, int64_t ldx,
                                                                const pact_bf16 *__restrict__ gamma, float eps,
                                                                int64_t M, int64_t H, pact_nvfp4_t yq,
@@ -250,26 +259,29 @@ __global__ void __launch_bounds__(RING_THREADS) k_rmsnorm_quant(const pact_bf16 
                 }
             }
         }
-        double ss = (s0 + s1) + (s2 + s3);
+        bool plain = __any_sync(0xFFFFFFFFu, top >= (0xFFu << 20));   // an infinity or NaN
+        if constexpr (EPS0) {   // or a warp sum below 2^-180
+            double t = (s0 + s1) + (s2 + s3);
 #pragma unroll
-        for (int o = 16; o; o >>= 1) ss += __shfl_xor_sync(0xFFFFFFFFu, ss, o);
-        if (__any_sync(0xFFFFFFFFu, top >= (0xFFu << 20)) || !(ss >= 0x1p-180)) {
-            // an infinity or NaN among the warp's values, or a partial sum so small that
-            // the widened zeros and subnormals (each square below 2^-252, at most 2^-238
-            // together) could count: the sum as plain conversions give it
-            ss = 0.0;
+            for (int o = 16; o; o >>= 1) t += __shfl_xor_sync(0xFFFFFFFFu, t, o);
+            plain |= !(t >= 0x1p-180);
+        }
+        if (plain) {
+            // the sum as plain conversions give it
+            s0 = s1 = s2 = s3 = 0.0;
             for (int k = warp; k < nchunk; k += RING_WARPS) {
                 const int c = k * CHUNK + 8 * lane;
                 if (c < H) {
                     float v[8];
                     load8_bf16(reinterpret_cast<const pact_bf16 *>(rs) + c, v);
 #pragma unroll
-                    for (int j = 0; j < 8; ++j) ss = fma((double)v[j], (double)v[j], ss);
+                    for (int j = 0; j < 8; ++j) s0 = fma((double)v[j], (double)v[j], s0);
                 }
             }
-#pragma unroll
-            for (int o = 16; o; o >>= 1) ss += __shfl_xor_sync(0xFFFFFFFFu, ss, o);
         }
+        double ss = (s0 + s1) + (s2 + s3);
+#pragma unroll
+        for (int o = 16; o; o >>= 1) ss += __shfl_xor_sync(0xFFFFFFFFu, ss, o);
         if (lane == 0) red[warp] = ss;
         __syncthreads();
         if (threadIdx.x == 0) {   // one thread evaluates rstd; the others read it
@@ -280,7 +292,7 @@ __global__ void __launch_bounds__(RING_THREADS) k_rmsnorm_quant(const pact_bf16 
         __syncthreads();
         const double rstd = rstd_s;
         const float r32 = (float)rstd;
-        const bool wide = isinf(r32);
+        const bool wide = EPS0 && isinf(r32);
         for (int k = warp; k < nchunk; k += RING_WARPS) {
             const int64_t c0 = (int64_t)k * CHUNK;
             const int64_t c = c0 + 8 * lane;
@@ -290,7 +302,7 @@ __global__ void __launch_bounds__(RING_THREADS) k_rmsnorm_quant(const pact_bf16 
                 load8_bf16(reinterpret_cast<const pact_bf16 *>(rs) + c, v);
                 load8_bf16(gs + c, g);
             }
-            if (wide) {
+            if (EPS0 && wide) {
 #pragma unroll
                 for (int j = 0; j < 8; ++j) o[j] = rms_exact(v[j], g[j], rstd);
             } else {
@@ -994,11 +1006,14 @@ pact_status pact_rmsnorm_quant(const pact_bf16 *x, int64_t ldx, const pact_bf16 
     static bool attr_done[64] = {false};
     const int d = current_device();
     if (d >= 0 && d < 64 && !attr_done[d]) {
-        const cudaError_t e = cudaFuncSetAttribute(k_rmsnorm_quant, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
+        cudaError_t e = cudaFuncSetAttribute(k_rmsnorm_quant<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
+        if (e == cudaSuccess)
+            e = cudaFuncSetAttribute(k_rmsnorm_quant<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
         if (e != cudaSuccess) return fail(PACT_ERR_CUDA, "pact_rmsnorm_quant: %s", cudaGetErrorString(e));
         attr_done[d] = true;
     }
-    return launch_dep(k_rmsnorm_quant, dim3(r.grid), dim3(RING_THREADS), r.smem, (cudaStream_t)stream,
+    return launch_dep(eps == 0.0f ? k_rmsnorm_quant<true> : k_rmsnorm_quant<false>, dim3(r.grid), dim3(RING_THREADS),
+                      r.smem, (cudaStream_t)stream,
                       "pact_rmsnorm_quant", x, ldx, gamma, eps, M, H, *yq, y, rstd, r.stages, (int)r.slot_bytes);
 }
 
