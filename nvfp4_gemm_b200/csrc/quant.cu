@@ -293,6 +293,7 @@ __global__ void __launch_bounds__(RING_THREADS) k_rmsnorm_quant(const pact_bf16 
         const double rstd = rstd_s;
         const float r32 = (float)rstd;
         const bool wide = EPS0 && isinf(r32);
+        const uint64_t r2 = f2_pack(r32, r32);
         for (int k = warp; k < nchunk; k += RING_WARPS) {
             const int64_t c0 = (int64_t)k * CHUNK;
             const int64_t c = c0 + 8 * lane;
@@ -302,12 +303,29 @@ __global__ void __launch_bounds__(RING_THREADS) k_rmsnorm_quant(const pact_bf16 
                 load8_bf16(reinterpret_cast<const pact_bf16 *>(rs) + c, v);
                 load8_bf16(gs + c, g);
             }
-            if (EPS0 && wide) {
+            if constexpr (EPS0) {
+                if (wide) {
 #pragma unroll
-                for (int j = 0; j < 8; ++j) o[j] = rms_exact(v[j], g[j], rstd);
+                    for (int j = 0; j < 8; ++j) o[j] = rms_exact(v[j], g[j], rstd);
+                } else {
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) o[j] = rms_out(v[j], g[j], r32, rstd);   // zeros past the row end
+                }
             } else {
+                // the FP32 products two at a time (the roundings of rms_out), the midpoint
+                // test once for the 8 values, the FP64 expression behind one branch
+                bool near = false;
 #pragma unroll
-                for (int j = 0; j < 8; ++j) o[j] = rms_out(v[j], g[j], r32, rstd);   // zeros past the row end
+                for (int j = 0; j < 8; j += 2) {
+                    f2_unpack(f2_mul(f2_mul(f2_pack(v[j], v[j + 1]), r2), f2_pack(g[j], g[j + 1])), o[j], o[j + 1]);
+                    near |= ((__float_as_uint(o[j]) & 0xFFFFu) - 0x7FC0u <= 0x80u) |
+                            ((__float_as_uint(o[j + 1]) & 0xFFFFu) - 0x7FC0u <= 0x80u);
+                }
+                if (near) {
+#pragma unroll
+                    for (int j = 0; j < 8; ++j)
+                        if ((__float_as_uint(o[j]) & 0xFFFFu) - 0x7FC0u <= 0x80u) o[j] = rms_exact(v[j], g[j], rstd);
+                }
             }
             uint4 ow;
             round8_bf16(o, ow, o);
