@@ -76,6 +76,12 @@ struct Params {
     // output rows])
     const uint8_t *a_scales;
     int64_t a_rows, a_cols;
+    // With one split, the epilogue writes out_scale * acc itself as hi + lo BF16 halves
+    // (hi at out[row * out_ld + col], lo at col + out_lo_off; k_finalize's mode 0) and no
+    // finalize runs; null otherwise.
+    pact_bf16 *out;
+    int64_t out_ld, out_lo_off;
+    float out_scale;
 };
 
 // 8 E2M1 codes (element 0 in the low nibble) times their E4M3 block scale, as 8
@@ -318,7 +324,26 @@ k_lora_mma(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUte
             uint32_t v[16];
             tmem_ld_32x32b_x16(tmem + ((uint32_t)(sub * 32) << 16) + c * 16, v);
             tmem_ld_wait();
-            if (r < pr.row_end) {
+            if (r < pr.row_end && p.out) {
+                if (c * 16 < p.n_valid) {   // whole 16-column chunks (n_valid is a multiple of 16)
+                    uint32_t hi[8], lo[8];
+#pragma unroll
+                    for (int j = 0; j < 16; j += 2) {
+                        // k_finalize's arithmetic for one split: (0 + acc) * scale, then hi, lo
+                        const float a0 = ok ? (0.0f + __uint_as_float(v[j])) * p.out_scale : __int_as_float(0x7fc00000);
+                        const float a1 =
+                            ok ? (0.0f + __uint_as_float(v[j + 1])) * p.out_scale : __int_as_float(0x7fc00000);
+                        hi[j / 2] = pack_bf16x2(a0, a1);
+                        lo[j / 2] = pack_bf16x2(a0 - bf16lo(hi[j / 2]), a1 - bf16hi(hi[j / 2]));
+                    }
+                    uint4 *oh = reinterpret_cast<uint4 *>(p.out + (size_t)r * p.out_ld + pr.out_col + c * 16);
+                    uint4 *ol = reinterpret_cast<uint4 *>(p.out + (size_t)r * p.out_ld + pr.out_col + c * 16 + p.out_lo_off);
+                    oh[0] = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+                    oh[1] = make_uint4(hi[4], hi[5], hi[6], hi[7]);
+                    ol[0] = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+                    ol[1] = make_uint4(lo[4], lo[5], lo[6], lo[7]);
+                }
+            } else if (r < pr.row_end) {
                 // a wait that gave up leaves NaN partials, so the result is NaN rather
                 // than whatever the scratch held before
                 float *dst = part + (size_t)r * p.ws_ld + pr.out_col + c * 16;
@@ -338,8 +363,14 @@ k_lora_mma(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUte
         // some role of this CTA gave up a wait: its partial tile is NaN, whatever the
         // accumulator held
         const int r = row0 + (warp & 3) * 32 + lane;
-        if (r < pr.row_end)
+        if (r < pr.row_end && p.out) {
+            for (int c = 0; c < p.n_valid; ++c) {
+                p.out[(size_t)r * p.out_ld + pr.out_col + c] = 0x7FC0u;   // BF16 NaN
+                p.out[(size_t)r * p.out_ld + pr.out_col + c + p.out_lo_off] = 0x7FC0u;
+            }
+        } else if (r < pr.row_end) {
             for (int c = 0; c < p.n_valid; ++c) part[(size_t)r * p.ws_ld + pr.out_col + c] = __int_as_float(0x7fc00000);
+        }
     }
 }
 
@@ -469,6 +500,16 @@ static FinJob fin_job(const float *ws, const Params &p, int64_t rows, int64_t co
                   mode >= 3 ? static_cast<float *>(out) : nullptr};
 }
 
+// A product with one split writes its hi + lo output from the epilogue (mode 0 of
+// k_finalize, with the same arithmetic) instead of partials and a finalize launch.
+static void set_direct_out(Params &p, pact_bf16 *out, int64_t ldo, int64_t lo_off, float scale) {
+    if (p.splits != 1) return;
+    p.out = out;
+    p.out_ld = ldo;
+    p.out_lo_off = lo_off;
+    p.out_scale = scale;
+}
+
 static pact_status finalize(const FinJob &j0, const FinJob *j1, cudaStream_t st, const char *what) {
     const int64_t n = j0.rows * j0.cols + (j1 ? j1->rows * j1->cols : 0);
     return launch_dep(k_finalize, dim3(finalize_grid(n)), dim3(256), 0, st, what, j0, j1 ? *j1 : j0, j1 ? 2 : 1);
@@ -521,13 +562,14 @@ static pact_status rows_times_a(const CUtensorMap &tx, const pact_nvfp4_t *xq, i
     p.ws = ws;
     p.ws_ld = R;
     p.ws_split_stride = M * R;
+    set_direct_out(p, out, ldo, R, scale);
     if (xq) {
         set_fp4_a(p, *xq);
         s = launch_mma<false, false, true>(tx, tb, p, tiles, st, what);
     } else {
         s = launch_mma<false, false>(tx, tb, p, tiles, st, what);
     }
-    if (s != PACT_OK) return s;
+    if (s != PACT_OK || p.out) return s;
     return finalize(fin_job(ws, p, M, R, scale, 0, out, ldo, R), nullptr, st, what);
 }
 
@@ -629,8 +671,9 @@ pact_status pact_lora_bwd_u(const pact_bf16 *dy, int64_t lddy, int64_t M, int64_
     p.ws = ws;
     p.ws_ld = R;
     p.ws_split_stride = M * R;
+    set_direct_out(p, U, ldu, R, scale);
     s = launch_mma<false, true>(ta, tb, p, tiles, st, "pact_lora_bwd_u");
-    if (s != PACT_OK) return s;
+    if (s != PACT_OK || p.out) return s;
     return finalize(fin_job(ws, p, M, R, scale, 0, U, ldu, R), nullptr, st, "pact_lora_bwd_u");
 }
 

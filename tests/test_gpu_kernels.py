@@ -327,6 +327,33 @@ def test_gemm_fwd_silu_rejects_bad_shapes(P):
 
 
 # ------------------------------------------------------------------------- LoRA
+def test_lora_products_with_one_split(P, orc, guards):
+    """T = s X A^T and U = s dY B with enough 128-row output blocks (150 >= the SM
+    count) that the contraction is not split: the MMA kernel then writes the hi + lo
+    output itself (no finalize launch).  Compared with the oracle through hi + lo."""
+    r, s = 16, 2.0
+    M, K, R = 19200, 128, 48
+    x = synth.gaussian_bf16(1, (M, K))
+    a = synth.gaussian_bf16(20, (R, K), std=0.02)
+    T = P.pact_lora_fwd(to_dev(x), to_dev(a), s, T=guards.matrix(M, 2 * R, pad_cols=8))
+    Mu, parts = 6400, [256, 256, 512]
+    N = sum(parts)
+    seg_end = _segments(N, parts)
+    dy = synth.gaussian_bf16(50, (Mu, N))
+    b = synth.gaussian_bf16(30, (N, r), std=0.02)
+    U = P.pact_lora_bwd_u(to_dev(dy), to_dev(b), r, seg_end, s, U=guards.matrix(Mu, 2 * 3 * r, pad_cols=8))
+    sync()
+    t_dev = to_f64(T[:, :R]) + to_f64(T[:, R:])
+    assert_close(t_dev, s * orc.gemm_nt(synth.bf16_bits_to_f64(x), synth.bf16_bits_to_f64(a)), "T")
+    dyf, bf = synth.bf16_bits_to_f64(dy), synth.bf16_bits_to_f64(b)
+    u_ref = np.zeros((Mu, 3 * r))
+    lo = 0
+    for i, hi in enumerate(seg_end):
+        u_ref[:, i * r:(i + 1) * r] = s * orc.gemm_nt(dyf[:, lo:hi], bf[lo:hi].T)
+        lo = hi
+    assert_close(to_f64(U[:, :3 * r]) + to_f64(U[:, 3 * r:]), u_ref, "U")
+
+
 @pytest.mark.parametrize("M,parts,r,K", [(256, [512], 16, 384), (300, [512, 256, 256], 16, 576),
                                          (130, [256, 320], 32, 320), (2048, [1024], 16, 2112)])
 def test_lora_bwd(P, orc, guards, M, parts, r, K):
