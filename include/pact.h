@@ -262,6 +262,20 @@ PACT_API pact_status pact_lora_fwd(const pact_bf16 *x, int64_t ldx, int64_t M, i
                                    const pact_bf16 *A, int R, float scale, pact_bf16 *T, int64_t ldt,
                                    void *workspace, size_t ws_bytes, pact_stream_t stream);
 
+/* pact_lora_fwd that also writes xq = q(x) ([M x K], the NVFP4 copy of x exactly as
+ * pact_quantize_nvfp4 writes it, padding rows' scales zeroed): the input of the
+ * frozen GEMM that follows.  The kernel quantizes the tiles of x it streams for the
+ * LoRA product, so x is read once for both.  xq must not overlap x, T or workspace. */
+PACT_API pact_status pact_lora_fwd_quant(const pact_bf16 *x, int64_t ldx, int64_t M, int64_t K,
+                                         const pact_bf16 *A, int R, float scale, pact_bf16 *T,
+                                         int64_t ldt, const pact_nvfp4_t *xq, void *workspace,
+                                         size_t ws_bytes, pact_stream_t stream);
+
+/* Kernels one pact_lora_fwd (or _quant) call launches for these sizes: 1 when the
+ * product runs unsplit (its kernel writes T itself), 2 when a finalize kernel sums
+ * the split contraction's partials. */
+PACT_API int pact_lora_fwd_launches(int64_t M, int64_t K, int R);
+
 /* pact_lora_fwd without a workspace argument.  The pages have no counterpart of
  * this call: it exists for callers that cannot allocate device memory where they
  * call the library (plain C callers without a device allocator, code that must not
@@ -295,6 +309,22 @@ PACT_API pact_status pact_lora_bwd_u(const pact_bf16 *dy, int64_t lddy, int64_t 
                                      const pact_bf16 *B, int r, int nseg, const int64_t *seg_end,
                                      float scale, pact_bf16 *U, int64_t ldu, void *workspace,
                                      size_t ws_bytes, pact_stream_t stream);
+
+/* pact_lora_bwd_u that also writes dyq = q(dY) ([M x N], as pact_quantize_nvfp4
+ * writes it): the input of the dgrad GEMM that follows, from the tiles of dY the
+ * kernel streams for U.  dyq must not overlap dy, U or workspace. */
+PACT_API pact_status pact_lora_bwd_u_quant(const pact_bf16 *dy, int64_t lddy, int64_t M, int64_t N,
+                                           const pact_bf16 *B, int r, int nseg, const int64_t *seg_end,
+                                           float scale, pact_bf16 *U, int64_t ldu, const pact_nvfp4_t *dyq,
+                                           void *workspace, size_t ws_bytes, pact_stream_t stream);
+
+/* Kernels one pact_lora_bwd_u (or _quant) call launches for these sizes (1 or 2, as
+ * pact_lora_fwd_launches). */
+PACT_API int pact_lora_bwd_u_launches(int64_t M, int64_t N, int r, int nseg, const int64_t *seg_end);
+
+/* Kernels one pact_lora_bwd call launches for these sizes (X~ [M x K], R = nseg*r;
+ * nvfp4_x non-zero when X~ is given as the saved NVFP4 copy): 4 or 5. */
+PACT_API int pact_lora_bwd_launches(int64_t M, int64_t K, int R, int nvfp4_x);
 
 /* The input X~ the adapter saw, as backward holds it: BF16 x, or the saved NVFP4
  * copy xq (dequantized on the fly); exactly one is non-NULL. */

@@ -82,6 +82,10 @@ struct Params {
     pact_bf16 *out;
     int64_t out_ld, out_lo_off;
     float out_scale;
+    // K-major BF16 A only: with aq.codes set, the epilogue warps (idle during the main
+    // loop) also quantize each stage's A tile as it passes through shared memory and
+    // write the NVFP4 copy aq of A ([rows x contraction]), padding rows' scales zeroed.
+    pact_nvfp4_t aq;
 };
 
 // 8 E2M1 codes (element 0 in the low nibble) times their E4M3 block scale, as 8
@@ -158,6 +162,7 @@ k_lora_mma(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUte
     const int ktiles = ke > kb ? (ke - kb + BK - 1) / BK : 0;
     float *part = p.ws + (size_t)blockIdx.y * p.ws_split_stride;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const bool quantize_a = !A_MN && !A_FP4 && p.aq.codes != nullptr;
 
     if (ktiles == 0) {  // empty split: its partial is zero
         pdl_wait();
@@ -182,7 +187,8 @@ k_lora_mma(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUte
         for (int s = 0; s < STAGES; ++s) {
             // A_FP4: the producer's arrival (B bytes) and the four decoding warps'
             mbar_init(&full[s], A_FP4 ? 5 : 1);
-            mbar_init(&empty[s], 1);
+            // the MMA warp's commit and, when they quantize A, the four epilogue warps'
+            mbar_init(&empty[s], quantize_a ? 5 : 1);
             mbar_init(&raw_full[s], 1);
         }
         mbar_init(acc_full, 1);
@@ -309,6 +315,49 @@ k_lora_mma(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUte
                 fence_proxy_async_smem();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&full[stage]);
+                if (++stage == STAGES) { stage = 0; phase ^= 1; }
+            }
+        } else if (quantize_a && warp < 6) {
+            // the NVFP4 copy of A: thread q quantizes operand row q of each stage (64
+            // values, four 16-value blocks) from the swizzled tile (16-byte chunk c of row
+            // q at (c ^ (q % 8)) * 16), then releases the stage with the MMA's commit
+            const int q = threadIdx.x - 64;
+            const int64_t row = row0 + q, rows_pad = ((int64_t)pr.row_end + 127) & ~int64_t(127);
+            const int64_t cols = p.aq.cols;
+            uint8_t *qcodes = static_cast<uint8_t *>(p.aq.codes), *qscales = static_cast<uint8_t *>(p.aq.scales);
+            uint32_t stage = 0, phase = 0;
+            for (int kt = 0; kt < ktiles; ++kt) {
+                if (!(ok = warp_all(mbar_wait(&full[stage], phase)))) {
+                    aborted = 1;
+                    break;
+                }
+                const int k = kb + kt * BK;
+                const uint32_t a = smem_u32(smem + stage * STAGE_BYTES) + q * 128;
+                if (row < pr.row_end) {
+                    uint32_t cw[8], sw = 0;
+#pragma unroll
+                    for (int b = 0; b < 4; ++b) {
+                        uint4 wa, wb;
+                        asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                                     : "=r"(wa.x), "=r"(wa.y), "=r"(wa.z), "=r"(wa.w)
+                                     : "r"(a + (((2 * b) ^ (q & 7)) << 4)));
+                        asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                                     : "=r"(wb.x), "=r"(wb.y), "=r"(wb.z), "=r"(wb.w)
+                                     : "r"(a + (((2 * b + 1) ^ (q & 7)) << 4)));
+                        uint32_t sb;
+                        quant16_bf16(wa, wb, &cw[2 * b], &cw[2 * b + 1], &sb);
+                        sw |= sb << (8 * b);
+                    }
+                    uint4 *cp = reinterpret_cast<uint4 *>(qcodes + row * (cols >> 1) + (k >> 1));
+                    cp[0] = make_uint4(cw[0], cw[1], cw[2], cw[3]);
+                    cp[1] = make_uint4(cw[4], cw[5], cw[6], cw[7]);
+                    // blocks k/16 .. k/16 + 3 (k a multiple of 64): one word of the layout
+                    *reinterpret_cast<uint32_t *>(qscales + scale_offset(row, k >> 4, cols)) = sw;
+                } else if (row < rows_pad) {
+                    *reinterpret_cast<uint32_t *>(qscales + scale_offset(row, k >> 4, cols)) = 0u;
+                }
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&empty[stage]);
                 if (++stage == STAGES) { stage = 0; phase ^= 1; }
             }
         }
@@ -548,7 +597,7 @@ static size_t partial_bytes(int64_t rows, int64_t cols, int splits) {
 // ws holds the partials.
 static pact_status rows_times_a(const CUtensorMap &tx, const pact_nvfp4_t *xq, int64_t M, int64_t K,
                                 const pact_bf16 *A, int R, float scale, pact_bf16 *out, int64_t ldo, float *ws,
-                                cudaStream_t st, const char *what) {
+                                cudaStream_t st, const char *what, const pact_nvfp4_t *aq = nullptr) {
     CUtensorMap tb;
     pact_status s = map_bf16(&tb, A, K, R, K, 64, R, what);
     if (s != PACT_OK) return s;
@@ -563,6 +612,7 @@ static pact_status rows_times_a(const CUtensorMap &tx, const pact_nvfp4_t *xq, i
     p.ws_ld = R;
     p.ws_split_stride = M * R;
     set_direct_out(p, out, ldo, R, scale);
+    if (aq) p.aq = *aq;   // BF16 x only (the kernel quantizes K-major BF16 A tiles)
     if (xq) {
         set_fp4_a(p, *xq);
         s = launch_mma<false, false, true>(tx, tb, p, tiles, st, what);
@@ -611,23 +661,43 @@ size_t pact_lora_fwd_workspace_bytes(int64_t M, int64_t K, int R) {
     return partial_bytes(M, R, splits_of(K, (M + BM - 1) / BM, FWD_PER_SM));
 }
 
+static pact_status lora_fwd(const pact_bf16 *x, int64_t ldx, int64_t M, int64_t K, const pact_bf16 *A, int R,
+                            float scale, pact_bf16 *T, int64_t ldt, const pact_nvfp4_t *xq, void *workspace,
+                            size_t ws_bytes, pact_stream_t stream, const char *what) {
+    PACT_CHECK(x && A && T && workspace, PACT_ERR_INVALID_ARG, "%s: NULL argument", what);
+    PACT_CHECK(M >= 1 && M <= 0x7FFFFFFF && K >= 64 && K % 64 == 0 && K <= 0x7FFFFFFF && R >= 16 && R <= 64 &&
+                   R % 16 == 0,
+               PACT_ERR_SHAPE, "%s: need M >= 1, K a multiple of 64, R in {16, 32, 48, 64}", what);
+    PACT_CHECK(ldx >= K && ldx % 8 == 0 && ldt >= 2 * R && ldt % 8 == 0 && aligned16(x) && aligned16(A) &&
+                   aligned16(T) && aligned16(workspace),
+               PACT_ERR_ALIGN, "%s: pointers 16-byte aligned, leading dims %% 8 == 0", what);
+    PACT_CHECK(ws_bytes >= pact_lora_fwd_workspace_bytes(M, K, R), PACT_ERR_INVALID_ARG,
+               "%s: workspace too small (%zu < %zu)", what, ws_bytes, pact_lora_fwd_workspace_bytes(M, K, R));
+    pact_status s = xq ? check_nvfp4(xq, M, K, "xq") : PACT_OK;
+    if (s != PACT_OK) return s;
+    CUtensorMap tx;
+    s = map_bf16(&tx, x, K, M, ldx, 64, BM, what);
+    if (s != PACT_OK) return s;
+    return rows_times_a(tx, nullptr, M, K, A, R, scale, T, ldt, static_cast<float *>(workspace), (cudaStream_t)stream,
+                        what, xq);
+}
+
 pact_status pact_lora_fwd(const pact_bf16 *x, int64_t ldx, int64_t M, int64_t K, const pact_bf16 *A, int R,
                           float scale, pact_bf16 *T, int64_t ldt, void *workspace, size_t ws_bytes,
                           pact_stream_t stream) {
-    PACT_CHECK(x && A && T && workspace, PACT_ERR_INVALID_ARG, "pact_lora_fwd: NULL argument");
-    PACT_CHECK(M >= 1 && M <= 0x7FFFFFFF && K >= 64 && K % 64 == 0 && K <= 0x7FFFFFFF && R >= 16 && R <= 64 &&
-                   R % 16 == 0,
-               PACT_ERR_SHAPE, "pact_lora_fwd: need M >= 1, K a multiple of 64, R in {16, 32, 48, 64}");
-    PACT_CHECK(ldx >= K && ldx % 8 == 0 && ldt >= 2 * R && ldt % 8 == 0 && aligned16(x) && aligned16(A) &&
-                   aligned16(T) && aligned16(workspace),
-               PACT_ERR_ALIGN, "pact_lora_fwd: pointers 16-byte aligned, leading dims %% 8 == 0");
-    PACT_CHECK(ws_bytes >= pact_lora_fwd_workspace_bytes(M, K, R), PACT_ERR_INVALID_ARG,
-               "pact_lora_fwd: workspace too small (%zu < %zu)", ws_bytes, pact_lora_fwd_workspace_bytes(M, K, R));
-    CUtensorMap tx;
-    pact_status s = map_bf16(&tx, x, K, M, ldx, 64, BM, "pact_lora_fwd");
-    if (s != PACT_OK) return s;
-    return rows_times_a(tx, nullptr, M, K, A, R, scale, T, ldt, static_cast<float *>(workspace), (cudaStream_t)stream,
-                        "pact_lora_fwd");
+    return lora_fwd(x, ldx, M, K, A, R, scale, T, ldt, nullptr, workspace, ws_bytes, stream, "pact_lora_fwd");
+}
+
+pact_status pact_lora_fwd_quant(const pact_bf16 *x, int64_t ldx, int64_t M, int64_t K, const pact_bf16 *A, int R,
+                                float scale, pact_bf16 *T, int64_t ldt, const pact_nvfp4_t *xq, void *workspace,
+                                size_t ws_bytes, pact_stream_t stream) {
+    PACT_CHECK(xq, PACT_ERR_INVALID_ARG, "pact_lora_fwd_quant: NULL argument");
+    return lora_fwd(x, ldx, M, K, A, R, scale, T, ldt, xq, workspace, ws_bytes, stream, "pact_lora_fwd_quant");
+}
+
+int pact_lora_fwd_launches(int64_t M, int64_t K, int R) {
+    (void)R;
+    return splits_of(K, (M + BM - 1) / BM, FWD_PER_SM) == 1 ? 1 : 2;
 }
 
 // Upper bound over segmentations: one segment may span all N outputs.
@@ -635,9 +705,9 @@ size_t pact_lora_bwd_u_workspace_bytes(int64_t M, int64_t N, int r, int nseg) {
     return partial_bytes(M, (int64_t)r * nseg, splits_of(N, (M + BM - 1) / BM, FWD_PER_SM));
 }
 
-pact_status pact_lora_bwd_u(const pact_bf16 *dy, int64_t lddy, int64_t M, int64_t N, const pact_bf16 *B, int r,
-                            int nseg, const int64_t *seg_end, float scale, pact_bf16 *U, int64_t ldu,
-                            void *workspace, size_t ws_bytes, pact_stream_t stream) {
+static pact_status lora_bwd_u(const pact_bf16 *dy, int64_t lddy, int64_t M, int64_t N, const pact_bf16 *B, int r,
+                              int nseg, const int64_t *seg_end, float scale, pact_bf16 *U, int64_t ldu,
+                              const pact_nvfp4_t *dyq, void *workspace, size_t ws_bytes, pact_stream_t stream) {
     PACT_CHECK(dy && B && U && seg_end && workspace, PACT_ERR_INVALID_ARG, "pact_lora_bwd_u: NULL argument");
     PACT_CHECK(M >= 1 && M <= 0x7FFFFFFF && N >= 64 && N % 64 == 0 && N <= 0x7FFFFFFF &&
                    (r == 16 || r == 32 || r == 48 || r == 64) && nseg >= 1 && nseg <= 3 && nseg * r <= 64,
@@ -650,6 +720,10 @@ pact_status pact_lora_bwd_u(const pact_bf16 *dy, int64_t lddy, int64_t M, int64_
                PACT_ERR_ALIGN, "pact_lora_bwd_u: pointers 16-byte aligned, leading dims %% 8 == 0");
     PACT_CHECK(ws_bytes >= pact_lora_bwd_u_workspace_bytes(M, N, r, nseg), PACT_ERR_INVALID_ARG,
                "pact_lora_bwd_u: workspace too small");
+    if (dyq) {
+        s = check_nvfp4(dyq, M, N, "dyq");
+        if (s != PACT_OK) return s;
+    }
     cudaStream_t st = (cudaStream_t)stream;
     CUtensorMap ta, tb;
     s = map_bf16(&ta, dy, N, M, lddy, 64, BM, "pact_lora_bwd_u");
@@ -672,9 +746,40 @@ pact_status pact_lora_bwd_u(const pact_bf16 *dy, int64_t lddy, int64_t M, int64_
     p.ws_ld = R;
     p.ws_split_stride = M * R;
     set_direct_out(p, U, ldu, R, scale);
+    if (dyq) p.aq = *dyq;
     s = launch_mma<false, true>(ta, tb, p, tiles, st, "pact_lora_bwd_u");
     if (s != PACT_OK || p.out) return s;
     return finalize(fin_job(ws, p, M, R, scale, 0, U, ldu, R), nullptr, st, "pact_lora_bwd_u");
+}
+
+pact_status pact_lora_bwd_u(const pact_bf16 *dy, int64_t lddy, int64_t M, int64_t N, const pact_bf16 *B, int r,
+                            int nseg, const int64_t *seg_end, float scale, pact_bf16 *U, int64_t ldu,
+                            void *workspace, size_t ws_bytes, pact_stream_t stream) {
+    return lora_bwd_u(dy, lddy, M, N, B, r, nseg, seg_end, scale, U, ldu, nullptr, workspace, ws_bytes, stream);
+}
+
+pact_status pact_lora_bwd_u_quant(const pact_bf16 *dy, int64_t lddy, int64_t M, int64_t N, const pact_bf16 *B,
+                                  int r, int nseg, const int64_t *seg_end, float scale, pact_bf16 *U, int64_t ldu,
+                                  const pact_nvfp4_t *dyq, void *workspace, size_t ws_bytes, pact_stream_t stream) {
+    PACT_CHECK(dyq, PACT_ERR_INVALID_ARG, "pact_lora_bwd_u_quant: NULL argument");
+    return lora_bwd_u(dy, lddy, M, N, B, r, nseg, seg_end, scale, U, ldu, dyq, workspace, ws_bytes, stream);
+}
+
+int pact_lora_bwd_launches(int64_t M, int64_t K, int R, int nvfp4_x) {
+    (void)R;
+    // T~ (a finalize unless unsplit), the dB and dA products, one finalize for both
+    const int t_splits = splits_of(K, (M + BM - 1) / BM, nvfp4_x ? ctas_per_sm(1, true, stages_for(1, true)) : FWD_PER_SM);
+    return (t_splits == 1 ? 1 : 2) + 3;
+}
+
+int pact_lora_bwd_u_launches(int64_t M, int64_t N, int r, int nseg, const int64_t *seg_end) {
+    (void)r;
+    int64_t longest = 0, prev = 0;
+    for (int i = 0; i < nseg; ++i) {
+        if (seg_end[i] - prev > longest) longest = seg_end[i] - prev;
+        prev = seg_end[i];
+    }
+    return splits_of(longest, ((M + BM - 1) / BM) * nseg, FWD_PER_SM) == 1 ? 1 : 2;
 }
 
 // Upper bound over segmentations: the dB output blocks number at least N / 128.

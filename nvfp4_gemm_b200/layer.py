@@ -192,26 +192,28 @@ class PactLayer:
         gbytes = lambda N, K, R: S.nv(M, K) + S.nv(N, K) + 2 * M * N + 2 * M * 2 * R + 2 * N * R
         # LoRA forward T = s x A^T as hi|lo: x [M x K] and A [R x K] in, T [M x 2R] out
         lora_fwd = lambda K, R: 2 * M * K + 2 * R * K + 2 * M * 2 * R
+        nk = lambda K, R: P.pact_lora_fwd_launches(M, K, R)   # 1 unsplit, 2 with a finalize
         return [
             Op("rmsnorm_quant_1", lambda: P.pact_rmsnorm_quant(h, self.g1, S.eps, self.xq1, self.x1, self.rstd1),
                bytes=2 * M * H + 2 * H + S.nv(M, H) + 2 * M * H + 4 * M),
-            Op("lora_fwd_qkv", lambda: P.pact_lora_fwd(self.x1, self.a_qkv, self.sc["qkv"], self.t_qkv, self.ws), kernels=2,
-               bytes=lora_fwd(H, 3 * r)),
+            Op("lora_fwd_qkv", lambda: P.pact_lora_fwd(self.x1, self.a_qkv, self.sc["qkv"], self.t_qkv, self.ws),
+               kernels=nk(H, 3 * r), bytes=lora_fwd(H, 3 * r)),
             Op("gemm_fwd_qkv", lambda: P.pact_frozen_gemm_fwd(self.xq1, self.c_qkv, self.l_qkv_f, y=self.qkv),
                "gemm", gemm(S.M, S.n_qkv, S.H), bytes=gbytes(S.n_qkv, H, 3 * r)),
-            Op("quantize_attn", lambda: P.pact_quantize_nvfp4(attn, self.aq), bytes=2 * M * H + S.nv(M, H)),
-            Op("lora_fwd_o", lambda: P.pact_lora_fwd(attn, self.a_o, self.sc["o"], self.t_o, self.ws), kernels=2,
-               bytes=lora_fwd(H, r)),
+            # the LoRA product streams attn and writes its NVFP4 copy aq (the GEMM's input)
+            Op("lora_fwd_o+q(attn)", lambda: P.pact_lora_fwd(attn, self.a_o, self.sc["o"], self.t_o, self.ws,
+                                                             xq=self.aq),
+               kernels=nk(H, r), bytes=lora_fwd(H, r) + S.nv(M, H)),
             Op("gemm_fwd_o", lambda: P.pact_frozen_gemm_fwd(self.aq, self.c_o, self.l_o_f, residual=h, y=self.h2),
                "gemm", gemm(S.M, S.H, S.H), bytes=gbytes(H, H, r) + 2 * M * H),
             Op("rmsnorm_quant_2", lambda: P.pact_rmsnorm_quant(self.h2, self.g2, S.eps, self.xq2, self.x2,
                                                                self.rstd2),
                bytes=2 * M * H + 2 * H + S.nv(M, H) + 2 * M * H + 4 * M),
-            Op("lora_fwd_gu", lambda: P.pact_lora_fwd(self.x2, self.a_gu, self.sc["gu"], self.t_gu, self.ws), kernels=2,
-               bytes=lora_fwd(H, 2 * r)),
+            Op("lora_fwd_gu", lambda: P.pact_lora_fwd(self.x2, self.a_gu, self.sc["gu"], self.t_gu, self.ws),
+               kernels=nk(H, 2 * r), bytes=lora_fwd(H, 2 * r)),
             *self._gate_up_ops(gemm, gbytes),
-            Op("lora_fwd_down", lambda: P.pact_lora_fwd(self.m, self.a_d, self.sc["d"], self.t_d, self.ws), kernels=2,
-               bytes=lora_fwd(I, r)),
+            Op("lora_fwd_down", lambda: P.pact_lora_fwd(self.m, self.a_d, self.sc["d"], self.t_d, self.ws),
+               kernels=nk(I, r), bytes=lora_fwd(I, r)),
             Op("gemm_fwd_down", lambda: P.pact_frozen_gemm_fwd(self.mq, self.c_d, self.l_d_f, residual=self.h2,
                                                                y=self.out),
                "gemm", gemm(S.M, S.H, I), bytes=gbytes(H, I, r) + 2 * M * H),
@@ -244,14 +246,16 @@ class PactLayer:
         gbytes = lambda N, K, R: S.nv(M, K) + S.nv(N, K) + 2 * M * N + 2 * M * 2 * R + 2 * K * R
         # U = s dY B as hi|lo: dY [M x N] and B [N x R] in, U [M x 2R] out
         lora_u = lambda N, R: 2 * M * N + 2 * N * R + 2 * M * 2 * R
+        nku = lambda N, seg: P.pact_lora_bwd_u_launches(M, N, r, seg)   # 1 unsplit, 2 with a finalize
         # dA, dB: dY [M x N], the saved input (x_bytes), U [M x 2R] and A [R x K] in; dA, dB out
         lora_bwd = lambda N, x_bytes, K, R: 2 * M * N + x_bytes + 2 * M * 2 * R + 2 * R * K + 2 * R * K + 2 * N * R
-        LB = 5  # kernels of one pact_lora_bwd call
+        LB = lambda K, R, nv: P.pact_lora_bwd_launches(M, K, R, nv)  # kernels of one pact_lora_bwd call
         return [
             # down projection
-            Op("lora_bwd_u_down", lambda: P.pact_lora_bwd_u(d_out, self.b_d, r, [H], self.sc["d"], self.u_d, self.ws), kernels=2,
-               bytes=lora_u(H, r)),
-            Op("quantize_dout", lambda: P.pact_quantize_nvfp4(d_out, self.doq), bytes=2 * M * H + S.nv(M, H)),
+            # U streams d_out and writes its NVFP4 copy doq (the dgrad GEMM's input)
+            Op("lora_bwd_u_down+q(dout)", lambda: P.pact_lora_bwd_u(d_out, self.b_d, r, [H], self.sc["d"], self.u_d,
+                                                                    self.ws, dyq=self.doq),
+               kernels=nku(H, [H]), bytes=lora_u(H, r) + S.nv(M, H)),
             Op("gemm_dgrad_down", lambda: P.pact_frozen_gemm_dgrad(self.doq, self.c_d, self.l_d_b, dx=self.dm),
                "gemm", gemm(S.M, I, H), bytes=gbytes(I, H, r)),
             Op("silu_mul_bwd_quant", lambda: P.pact_silu_mul_bwd_quant(self.dm, self.gq, self.uq, self.dgu,
@@ -260,40 +264,42 @@ class PactLayer:
             Op("lora_bwd_down", lambda: P.pact_lora_bwd(d_out, self.a_d, self.u_d, r, [H], s, x=self.m_re,
                                                         dA=g["a_d"], dB=g["b_d"], workspace=self.ws_leaf["down"],
                                                         u_gexp=self.gexp["d"], grads_fp32=f32),
-               kernels=LB, side=True,
+               kernels=LB(I, r, False), side=True,
                bytes=lora_bwd(H, 2 * M * I, I, r)),
             # gate|up
-            Op("lora_bwd_u_gu", lambda: P.pact_lora_bwd_u(self.dgu, self.b_gu, r, self.seg_gu, self.sc["gu"], self.u_gu, self.ws), kernels=2,
-               bytes=lora_u(2 * I, 2 * r)),
+            Op("lora_bwd_u_gu", lambda: P.pact_lora_bwd_u(self.dgu, self.b_gu, r, self.seg_gu, self.sc["gu"], self.u_gu,
+                                                          self.ws),
+               kernels=nku(2 * I, self.seg_gu), bytes=lora_u(2 * I, 2 * r)),
             Op("gemm_dgrad_gu", lambda: P.pact_frozen_gemm_dgrad(self.dguq, self.c_gu, self.l_gu_b, dx=self.dx2),
                "gemm", gemm(S.M, H, 2 * I), bytes=gbytes(H, 2 * I, 2 * r)),
             Op("lora_bwd_gu", lambda: P.pact_lora_bwd(self.dgu, self.a_gu, self.u_gu, r, self.seg_gu, s,
                                                       xq=self.xq2, dA=g["a_gu"], dB=g["b_gu"],
                                                       workspace=self.ws_leaf["gu"], u_gexp=self.gexp["gu"], grads_fp32=f32),
-               kernels=LB, side=True, bytes=lora_bwd(2 * I, S.nv(M, H), H, 2 * r)),
+               kernels=LB(H, 2 * r, True), side=True, bytes=lora_bwd(2 * I, S.nv(M, H), H, 2 * r)),
             Op("rmsnorm_bwd_2", lambda: P.pact_rmsnorm_bwd(self.dx2, self.xq2, self.rstd2, self.g2, dres=d_out,
                                                            dx=self.dh2, dxq=self.dh2q),
                bytes=2 * M * H + S.nv(M, H) + 4 * M + 2 * H + 2 * M * H + 2 * M * H + S.nv(M, H)),
             # o projection (its output joined the residual stream h2)
-            Op("lora_bwd_u_o", lambda: P.pact_lora_bwd_u(self.dh2, self.b_o, r, [H], self.sc["o"], self.u_o, self.ws), kernels=2,
-               bytes=lora_u(H, r)),
+            Op("lora_bwd_u_o", lambda: P.pact_lora_bwd_u(self.dh2, self.b_o, r, [H], self.sc["o"], self.u_o, self.ws),
+               kernels=nku(H, [H]), bytes=lora_u(H, r)),
             Op("gemm_dgrad_o", lambda: P.pact_frozen_gemm_dgrad(self.dh2q, self.c_o, self.l_o_b, dx=self.dattn),
                "gemm", gemm(S.M, H, H), bytes=gbytes(H, H, r)),
             Op("lora_bwd_o", lambda: P.pact_lora_bwd(self.dh2, self.a_o, self.u_o, r, [H], s, x=attn,
                                                      dA=g["a_o"], dB=g["b_o"], workspace=self.ws_leaf["o"],
                                                      u_gexp=self.gexp["o"], grads_fp32=f32),
-               kernels=LB, side=True,
+               kernels=LB(H, r, False), side=True,
                bytes=lora_bwd(H, 2 * M * H, H, r)),
             # q|k|v (d_qkv stands in for the attention backward)
-            Op("lora_bwd_u_qkv", lambda: P.pact_lora_bwd_u(d_qkv, self.b_qkv, r, self.seg_qkv, self.sc["qkv"], self.u_qkv, self.ws), kernels=2,
-               bytes=lora_u(S.n_qkv, 3 * r)),
-            Op("quantize_dqkv", lambda: P.pact_quantize_nvfp4(d_qkv, self.dqkvq), bytes=2 * M * S.n_qkv + S.nv(M, S.n_qkv)),
+            # U streams d_qkv and writes its NVFP4 copy dqkvq (the dgrad GEMM's input)
+            Op("lora_bwd_u_qkv+q(dqkv)", lambda: P.pact_lora_bwd_u(d_qkv, self.b_qkv, r, self.seg_qkv, self.sc["qkv"],
+                                                                   self.u_qkv, self.ws, dyq=self.dqkvq),
+               kernels=nku(S.n_qkv, self.seg_qkv), bytes=lora_u(S.n_qkv, 3 * r) + S.nv(M, S.n_qkv)),
             Op("gemm_dgrad_qkv", lambda: P.pact_frozen_gemm_dgrad(self.dqkvq, self.c_qkv, self.l_qkv_b, dx=self.dx1),
                "gemm", gemm(S.M, H, S.n_qkv), bytes=gbytes(H, S.n_qkv, 3 * r)),
             Op("lora_bwd_qkv", lambda: P.pact_lora_bwd(d_qkv, self.a_qkv, self.u_qkv, r, self.seg_qkv, s,
                                                        xq=self.xq1, dA=g["a_qkv"], dB=g["b_qkv"],
                                                        workspace=self.ws_leaf["qkv"], u_gexp=self.gexp["qkv"], grads_fp32=f32),
-               kernels=LB, side=True,
+               kernels=LB(H, 3 * r, True), side=True,
                bytes=lora_bwd(S.n_qkv, S.nv(M, H), H, 3 * r)),
             Op("rmsnorm_bwd_1", lambda: P.pact_rmsnorm_bwd(self.dx1, self.xq1, self.rstd1, self.g1, dres=self.dh2,
                                                            dx=self.dh),
@@ -425,9 +431,9 @@ class PactProjection:
         x, _ = self.inputs
         nv = lambda rows, cols: rows * cols / 2 + rows * cols / 16
         return [
-            Op("quantize_x", lambda: P.pact_quantize_nvfp4(x, self.xq), bytes=2 * M * K + nv(M, K)),
-            Op("lora_fwd", lambda: P.pact_lora_fwd(x, self.A, self.scale, self.t, self.ws), kernels=2,
-               bytes=2 * M * K + 2 * r * K + 2 * M * 2 * r),
+            # the LoRA product streams x and writes its NVFP4 copy xq (the GEMM's input)
+            Op("lora_fwd+q(x)", lambda: P.pact_lora_fwd(x, self.A, self.scale, self.t, self.ws, xq=self.xq),
+               kernels=P.pact_lora_fwd_launches(M, K, r), bytes=2 * M * K + 2 * r * K + 2 * M * 2 * r + nv(M, K)),
             Op("gemm_fwd", lambda: P.pact_frozen_gemm_fwd(self.xq, self.c_w, self.l_f, y=self.y), "gemm",
                2.0 * M * N * K, bytes=nv(M, K) + nv(N, K) + 2 * M * N + 2 * M * 2 * r + 2 * N * r),
         ]
@@ -438,14 +444,16 @@ class PactProjection:
         g = self.grads
         nv = lambda rows, cols: rows * cols / 2 + rows * cols / 16
         return [
-            Op("lora_bwd_u", lambda: P.pact_lora_bwd_u(dy, self.B, r, [N], self.scale, self.u, self.ws), kernels=2,
-               bytes=2 * M * N + 2 * N * r + 2 * M * 2 * r),
-            Op("quantize_dy", lambda: P.pact_quantize_nvfp4(dy, self.dyq), bytes=2 * M * N + nv(M, N)),
+            # U streams dy and writes its NVFP4 copy dyq (the dgrad GEMM's input)
+            Op("lora_bwd_u+q(dy)", lambda: P.pact_lora_bwd_u(dy, self.B, r, [N], self.scale, self.u, self.ws,
+                                                             dyq=self.dyq),
+               kernels=P.pact_lora_bwd_u_launches(M, N, r, [N]), bytes=2 * M * N + 2 * N * r + 2 * M * 2 * r + nv(M, N)),
             Op("gemm_dgrad", lambda: P.pact_frozen_gemm_dgrad(self.dyq, self.c_w, self.l_b, dx=self.dx), "gemm",
                2.0 * M * N * K, bytes=nv(M, N) + nv(N, K) + 2 * M * K + 2 * M * 2 * r + 2 * K * r),
             Op("lora_bwd", lambda: P.pact_lora_bwd(dy, self.A, self.u, r, [N], self.scale, xq=self.xq, dA=g["a"],
                                                    dB=g["b"], workspace=self.ws_leaf),
-               kernels=5, side=True, bytes=2 * M * N + nv(M, K) + 2 * M * 2 * r + 4 * r * K + 2 * N * r),
+               kernels=P.pact_lora_bwd_launches(M, K, r, True), side=True,
+               bytes=2 * M * N + nv(M, K) + 2 * M * 2 * r + 4 * r * K + 2 * N * r),
         ]
 
     def step_ops(self) -> List[Op]:

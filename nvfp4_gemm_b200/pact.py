@@ -82,9 +82,15 @@ def _load() -> ctypes.CDLL:
                                           NV, NV, P]),
         "pact_lora_fwd_workspace_bytes": (ctypes.c_size_t, [I64, I64, I]),
         "pact_lora_fwd": (S, [P, I64, I64, I64, P, I, F, P, I64, P, ctypes.c_size_t, P]),
+        "pact_lora_fwd_quant": (S, [P, I64, I64, I64, P, I, F, P, I64, NV, P, ctypes.c_size_t, P]),
+        "pact_lora_fwd_launches": (I, [I64, I64, I]),
         "pact_lora_fwd_noalloc": (S, [P, I64, I64, I64, P, I, F, P, I64, P]),
         "pact_lora_bwd_u_workspace_bytes": (ctypes.c_size_t, [I64, I64, I, I]),
         "pact_lora_bwd_u": (S, [P, I64, I64, I64, P, I, I, ctypes.POINTER(I64), F, P, I64, P, ctypes.c_size_t, P]),
+        "pact_lora_bwd_u_quant": (S, [P, I64, I64, I64, P, I, I, ctypes.POINTER(I64), F, P, I64, NV, P,
+                                      ctypes.c_size_t, P]),
+        "pact_lora_bwd_u_launches": (I, [I64, I64, I, I, ctypes.POINTER(I64)]),
+        "pact_lora_bwd_launches": (I, [I64, I64, I, I]),
         "pact_lora_bwd_workspace_bytes": (ctypes.c_size_t, [I64, I64, I64, I, I]),
         "pact_lora_bwd": (S, [ctypes.POINTER(c_lora_bwd), P, ctypes.c_size_t, P]),
         "pact_silu_mul_bwd_quant": (S, [P, I64, NV, NV, I64, I64, P, I64, NV, P, P]),
@@ -399,7 +405,10 @@ def pact_lora_fwd_workspace_bytes(M: int, K: int, R: int) -> int:
 
 
 def pact_lora_fwd(x: torch.Tensor, A: torch.Tensor, scale: float, T: Optional[torch.Tensor] = None,
-                  workspace: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+                  workspace: Optional[torch.Tensor] = None, xq: Optional[NVFP4Tensor] = None,
+                  stream=None) -> torch.Tensor:
+    """T = scale x A^T as hi|lo BF16; with xq given (pact_lora_fwd_quant) the kernel
+    also writes the NVFP4 copy of x into it."""
     _bf16(x, "x")
     _bf16(A, "A")
     M, K = x.shape
@@ -407,9 +416,19 @@ def pact_lora_fwd(x: torch.Tensor, A: torch.Tensor, scale: float, T: Optional[to
     if T is None:
         T = torch.empty((M, 2 * R), dtype=torch.bfloat16, device=x.device)
     ws = _workspace(workspace, pact_lora_fwd_workspace_bytes(M, K, R), x.device)
-    _check(_lib.pact_lora_fwd(x.data_ptr(), _ld(x), M, K, A.data_ptr(), R, float(scale), T.data_ptr(), _ld(T),
-                              ws.data_ptr(), ws.numel(), _stream(stream)))
+    if xq is None:
+        _check(_lib.pact_lora_fwd(x.data_ptr(), _ld(x), M, K, A.data_ptr(), R, float(scale), T.data_ptr(), _ld(T),
+                                  ws.data_ptr(), ws.numel(), _stream(stream)))
+    else:
+        sq = xq.c()
+        _check(_lib.pact_lora_fwd_quant(x.data_ptr(), _ld(x), M, K, A.data_ptr(), R, float(scale), T.data_ptr(),
+                                        _ld(T), ctypes.byref(sq), ws.data_ptr(), ws.numel(), _stream(stream)))
     return T
+
+
+def pact_lora_fwd_launches(M: int, K: int, R: int) -> int:
+    """Kernels one pact_lora_fwd call launches for these sizes (1 or 2)."""
+    return int(_lib.pact_lora_fwd_launches(M, K, R))
 
 
 def pact_lora_fwd_noalloc(x: torch.Tensor, A: torch.Tensor, scale: float, T: Optional[torch.Tensor] = None,
@@ -432,16 +451,35 @@ def pact_lora_bwd_u_workspace_bytes(M: int, N: int, r: int, nseg: int) -> int:
 
 def pact_lora_bwd_u(dy: torch.Tensor, B: torch.Tensor, r: int, seg_end: Sequence[int], scale: float,
                     U: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None,
-                    stream=None) -> torch.Tensor:
+                    dyq: Optional[NVFP4Tensor] = None, stream=None) -> torch.Tensor:
+    """U = scale dY B per segment as hi|lo BF16; with dyq given (pact_lora_bwd_u_quant)
+    the kernel also writes the NVFP4 copy of dY into it."""
     _bf16(dy, "dy")
     M, N = dy.shape
     if U is None:
         U = torch.empty((M, 2 * r * len(seg_end)), dtype=torch.bfloat16, device=dy.device)
     se = (ctypes.c_int64 * 4)(*(list(seg_end) + [0] * (4 - len(seg_end))))
     ws = _workspace(workspace, pact_lora_bwd_u_workspace_bytes(M, N, r, len(seg_end)), dy.device)
-    _check(_lib.pact_lora_bwd_u(dy.data_ptr(), _ld(dy), M, N, B.data_ptr(), r, len(seg_end), se, float(scale),
-                                U.data_ptr(), _ld(U), ws.data_ptr(), ws.numel(), _stream(stream)))
+    if dyq is None:
+        _check(_lib.pact_lora_bwd_u(dy.data_ptr(), _ld(dy), M, N, B.data_ptr(), r, len(seg_end), se, float(scale),
+                                    U.data_ptr(), _ld(U), ws.data_ptr(), ws.numel(), _stream(stream)))
+    else:
+        sq = dyq.c()
+        _check(_lib.pact_lora_bwd_u_quant(dy.data_ptr(), _ld(dy), M, N, B.data_ptr(), r, len(seg_end), se,
+                                          float(scale), U.data_ptr(), _ld(U), ctypes.byref(sq), ws.data_ptr(),
+                                          ws.numel(), _stream(stream)))
     return U
+
+
+def pact_lora_bwd_launches(M: int, K: int, R: int, nvfp4_x: bool) -> int:
+    """Kernels one pact_lora_bwd call launches for these sizes (4 or 5)."""
+    return int(_lib.pact_lora_bwd_launches(M, K, R, int(bool(nvfp4_x))))
+
+
+def pact_lora_bwd_u_launches(M: int, N: int, r: int, seg_end: Sequence[int]) -> int:
+    """Kernels one pact_lora_bwd_u call launches for these sizes (1 or 2)."""
+    se = (ctypes.c_int64 * 4)(*(list(seg_end) + [0] * (4 - len(seg_end))))
+    return int(_lib.pact_lora_bwd_u_launches(M, N, r, len(seg_end), se))
 
 
 def pact_lora_bwd_workspace_bytes(M: int, N: int, K: int, r: int, nseg: int) -> int:

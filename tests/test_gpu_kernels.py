@@ -354,6 +354,36 @@ def test_lora_products_with_one_split(P, orc, guards):
     assert_close(to_f64(U[:, :3 * r]) + to_f64(U[:, 3 * r:]), u_ref, "U")
 
 
+# the LoRA products that also write the NVFP4 copy of their streamed input: split
+# contractions (small M) and unsplit ones (M with >= 148 row blocks), ragged rows
+@pytest.mark.parametrize("M,K,R", [(300, 576, 48), (129, 128, 16), (19200, 192, 32)])
+def test_lora_fwd_quant(P, orc, guards, M, K, R):
+    x = synth.gaussian_bf16(1, (M, K))
+    a = synth.gaussian_bf16(20, (R, K), std=0.02)
+    xd, ad = to_dev(x), to_dev(a)
+    xq = guards.nvfp4(M, K)
+    T = P.pact_lora_fwd(xd, ad, 2.0, T=guards.matrix(M, 2 * R, pad_cols=8), xq=xq)
+    T_ref = P.pact_lora_fwd(xd, ad, 2.0)
+    sync()
+    assert torch.equal(T.contiguous().view(torch.int16), T_ref.view(torch.int16))
+    assert_nvfp4_equal(xq, orc.quantize(x), orc, "q(x)")
+
+
+@pytest.mark.parametrize("M,parts,r", [(300, [512, 256, 256], 16), (130, [320], 32), (6400, [256, 256, 512], 16)])
+def test_lora_bwd_u_quant(P, orc, guards, M, parts, r):
+    N = sum(parts)
+    seg_end = _segments(N, parts)
+    dy = synth.gaussian_bf16(50, (M, N))
+    b = synth.gaussian_bf16(30, (N, r), std=0.02)
+    dyd, bd = to_dev(dy), to_dev(b)
+    dyq = guards.nvfp4(M, N)
+    U = P.pact_lora_bwd_u(dyd, bd, r, seg_end, 2.0, U=guards.matrix(M, 2 * len(parts) * r, pad_cols=8), dyq=dyq)
+    U_ref = P.pact_lora_bwd_u(dyd, bd, r, seg_end, 2.0)
+    sync()
+    assert torch.equal(U.contiguous().view(torch.int16), U_ref.view(torch.int16))
+    assert_nvfp4_equal(dyq, orc.quantize(dy), orc, "q(dY)")
+
+
 @pytest.mark.parametrize("M,parts,r,K", [(256, [512], 16, 384), (300, [512, 256, 256], 16, 576),
                                          (130, [256, 320], 32, 320), (2048, [1024], 16, 2112)])
 def test_lora_bwd(P, orc, guards, M, parts, r, K):
