@@ -271,7 +271,20 @@ PACT_API pact_status pact_lora_fwd_quant(const pact_bf16 *x, int64_t ldx, int64_
                                          int64_t ldt, const pact_nvfp4_t *xq, void *workspace,
                                          size_t ws_bytes, pact_stream_t stream);
 
-/* Kernels one pact_lora_fwd (or _quant) call launches for these sizes: 1 when the
+/* [METHOD] + [LORA]: the down projection's LoRA input from the gate|up output, in
+ * one kernel: m = BF16_RNE(silu(g) * u) exactly as pact_silu_mul_quant rounds it, its
+ * NVFP4 copy mq = q(m) ([M x I], padding rows' scales zeroed), and T = scale * m .
+ * A^T (hi + lo halves as pact_lora_fwd, R as there).  g and u are [M x I] with one row
+ * stride ld_gu (the halves of the gate|up output).  m itself is written only when m
+ * is not NULL (row stride ldm): the data flow needs mq and T, and skipping m saves
+ * its write and its read by the LoRA product.  workspace as for pact_lora_fwd(M, I,
+ * R).  Outputs must not overlap the inputs or the workspace. */
+PACT_API pact_status pact_lora_fwd_silu(const pact_bf16 *g, const pact_bf16 *u, int64_t ld_gu, int64_t M,
+                                        int64_t I, const pact_bf16 *A, int R, float scale, pact_bf16 *T,
+                                        int64_t ldt, const pact_nvfp4_t *mq, pact_bf16 *m, int64_t ldm,
+                                        void *workspace, size_t ws_bytes, pact_stream_t stream);
+
+/* Kernels one pact_lora_fwd (or _quant, or _silu with K = I) call launches for these sizes: 1 when the
  * product runs unsplit (its kernel writes T itself), 2 when a finalize kernel sums
  * the split contraction's partials. */
 PACT_API int pact_lora_fwd_launches(int64_t M, int64_t K, int R);

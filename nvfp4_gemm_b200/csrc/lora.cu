@@ -26,6 +26,11 @@ constexpr int BM = 128;        // output rows per CTA (MMA M)
 constexpr int BK = 64;         // contraction elements per stage (128 bytes of BF16)
 constexpr int MAX_STAGES = 6;  // ring depth: 6, or 3 where two CTAs should share an SM
 constexpr int THREADS = 192;
+// SiLU A operand (A_SILU): per stage the g and u tiles (BF16, 128 x 64 each, the
+// 128-byte swizzle) land in a staging area, and 16 warps compute m = silu(g) u into
+// the operand buffer (writing q(m) on the way) before the MMA reads it.
+constexpr int SILU_WARPS = 16;
+__host__ __device__ constexpr int threads_of(bool silu) { return silu ? 64 + 32 * SILU_WARPS : THREADS; }
 constexpr int A_BYTES = BM * BK * 2;     // 16384
 constexpr int B_BYTES = 64 * BK * 2;     // 8192 per B part
 // NVFP4 A operand: per stage, the codes of the A tile (128 x 64 values, 4 KiB) and
@@ -36,9 +41,11 @@ constexpr int RAW_BYTES = RAW_CODE_BYTES + 1024;
 // A stage holds the A tile, one or two B parts (the hi and lo halves of T or U) and,
 // for an NVFP4 A, its staging area; all multiples of 1024 bytes.
 __host__ __device__ constexpr int oper_bytes(int nparts) { return A_BYTES + nparts * B_BYTES; }
-__host__ __device__ constexpr int stage_bytes(int nparts, bool fp4) { return oper_bytes(nparts) + (fp4 ? RAW_BYTES : 0); }
-__host__ __device__ constexpr int smem_bytes(int nparts, bool fp4, int stages) {
-    return 1024 + stages * stage_bytes(nparts, fp4) + 256;
+__host__ __device__ constexpr int stage_bytes(int nparts, bool fp4, bool silu = false) {
+    return oper_bytes(nparts) + (fp4 ? RAW_BYTES : 0) + (silu ? 2 * A_BYTES : 0);
+}
+__host__ __device__ constexpr int smem_bytes(int nparts, bool fp4, int stages, bool silu = false) {
+    return 1024 + stages * stage_bytes(nparts, fp4, silu) + 256;
 }
 constexpr int SM_SMEM = 233472;   // shared memory per SM (228 KiB), 1 KiB of it reserved per CTA
 __host__ __device__ constexpr int ctas_per_sm(int nparts, bool fp4, int stages) {
@@ -50,7 +57,9 @@ __host__ __device__ constexpr int ctas_per_sm(int nparts, bool fp4, int stages) 
 // more splits would cost more in FP32 partial-sum traffic than they gain.  A product
 // whose A operand is decoded from NVFP4 in the kernel is bound by the decoding warps,
 // so it runs 3 stages and two CTAs per SM (twice the decoders).
-__host__ __device__ constexpr int stages_for(int nparts, bool fp4) { return nparts == 2 || fp4 ? 3 : 6; }
+__host__ __device__ constexpr int stages_for(int nparts, bool fp4, bool silu = false) {
+    return nparts == 2 || fp4 || silu ? 3 : 6;
+}
 constexpr int FWD_PER_SM = 1;   // split residency of the one-part products
 constexpr uint32_t TMEM_COLS = 64;
 
@@ -85,7 +94,10 @@ struct Params {
     // K-major BF16 A only: with aq.codes set, the epilogue warps (idle during the main
     // loop) also quantize each stage's A tile as it passes through shared memory and
     // write the NVFP4 copy aq of A ([rows x contraction]), padding rows' scales zeroed.
+    // A_SILU: aq receives q(m) (always), m_out the BF16 m when not null.
     pact_nvfp4_t aq;
+    pact_bf16 *m_out;
+    int64_t m_ld;
 };
 
 // 8 E2M1 codes (element 0 in the low nibble) times their E4M3 block scale, as 8
@@ -149,11 +161,13 @@ __device__ __forceinline__ void decode_stage(const uint8_t *raw, uint8_t *oper, 
     }
 }
 
-template <bool A_MN, bool B_MN, bool A_FP4>
-__global__ void __launch_bounds__(THREADS, 1)
-k_lora_mma(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, const Params p) {
+template <bool A_MN, bool B_MN, bool A_FP4, bool A_SILU = false>
+__global__ void __launch_bounds__(threads_of(A_SILU), 1)
+k_lora_mma(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+           const __grid_constant__ CUtensorMap tmU, const Params p) {
+    // tmU: the u tiles of an A_SILU kernel (tmA then maps g); unused otherwise
     const int nparts = p.b_split ? 2 : 1;
-    const int STAGE_BYTES = stage_bytes(nparts, A_FP4), OPER_BYTES = oper_bytes(nparts);
+    const int STAGE_BYTES = stage_bytes(nparts, A_FP4, A_SILU), OPER_BYTES = oper_bytes(nparts);
     const Prob pr = p.prob[blockIdx.z];
     const int row0 = pr.row_begin + blockIdx.x * BM;
     if (row0 >= pr.row_end) return;  // block-uniform, before any shared state
@@ -162,7 +176,7 @@ k_lora_mma(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUte
     const int ktiles = ke > kb ? (ke - kb + BK - 1) / BK : 0;
     float *part = p.ws + (size_t)blockIdx.y * p.ws_split_stride;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const bool quantize_a = !A_MN && !A_FP4 && p.aq.codes != nullptr;
+    const bool quantize_a = !A_MN && !A_FP4 && !A_SILU && p.aq.codes != nullptr;
 
     if (ktiles == 0) {  // empty split: its partial is zero
         pdl_wait();
@@ -176,7 +190,7 @@ k_lora_mma(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUte
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = smem_u32(smem_raw);
     uint8_t *smem = smem_raw + (((raw + 1023) & ~1023u) - raw);
-    const int STAGES = stages_for(nparts, A_FP4);
+    const int STAGES = stages_for(nparts, A_FP4, A_SILU);
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + STAGES * STAGE_BYTES);
     uint64_t *full = bars, *empty = bars + MAX_STAGES, *acc_full = bars + 2 * MAX_STAGES;
     uint64_t *raw_full = bars + 2 * MAX_STAGES + 1;   // [stages], A_FP4 only
@@ -186,7 +200,7 @@ k_lora_mma(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUte
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
             // A_FP4: the producer's arrival (B bytes) and the four decoding warps'
-            mbar_init(&full[s], A_FP4 ? 5 : 1);
+            mbar_init(&full[s], A_SILU ? 1 + SILU_WARPS : A_FP4 ? 5 : 1);
             // the MMA warp's commit and, when they quantize A, the four epilogue warps'
             mbar_init(&empty[s], quantize_a ? 5 : 1);
             mbar_init(&raw_full[s], 1);
@@ -196,6 +210,7 @@ k_lora_mma(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUte
         fence_barrier_init();
         prefetch_tensormap(&tmA);
         prefetch_tensormap(&tmB);
+        if (A_SILU) prefetch_tensormap(&tmU);
     }
     if (warp == 1) {
         tmem_alloc(tmem_slot, TMEM_COLS);
@@ -218,7 +233,15 @@ k_lora_mma(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUte
                 }
                 uint8_t *st = smem + stage * STAGE_BYTES;
                 const int k = kb + kt * BK;
-                if (A_FP4) {
+                if (A_SILU) {
+                    // the g and u tiles into the staging area; the SiLU warps fill the operand
+                    uint8_t *rw = st + OPER_BYTES;
+                    mbar_arrive_expect_tx(&raw_full[stage], 2 * A_BYTES);
+                    tma_load_2d(rw, &tmA, &raw_full[stage], k, row0);
+                    tma_load_2d(rw + A_BYTES, &tmU, &raw_full[stage], k, row0);
+                    raw_pending |= 1u << stage;
+                    mbar_arrive_expect_tx(&full[stage], nparts * b_bytes);
+                } else if (A_FP4) {
                     // codes box and the scale chunk(s) of this stage's A tile
                     uint8_t *rw = st + OPER_BYTES;
                     const int64_t chunks_per_group = p.a_cols / 64;
@@ -263,7 +286,7 @@ k_lora_mma(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUte
             for (int s = 0; s < STAGES; ++s) {
                 if (!(pending & (1u << s))) continue;
                 const uint32_t par = (pending_parity >> s) & 1u;
-                if (A_FP4 && (raw_pending & (1u << s))) mbar_wait(&raw_full[s], par);
+                if ((A_FP4 || A_SILU) && (raw_pending & (1u << s))) mbar_wait(&raw_full[s], par);
                 mbar_wait(&full[s], par);
             }
         }
@@ -312,6 +335,73 @@ k_lora_mma(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUte
                 }
                 uint8_t *st = smem + stage * STAGE_BYTES;
                 decode_stage<A_MN>(st + OPER_BYTES, st, p, row0, kb + kt * BK, tid);
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&full[stage]);
+                if (++stage == STAGES) { stage = 0; phase ^= 1; }
+            }
+        } else if (A_SILU) {
+            // m = BF16_RNE(silu(g) u) for the stage's A tile: thread t computes the
+            // 16-value block b = t / 128 (columns 16 b .. 16 b + 15) of operand row q =
+            // t % 128 from the staged g and u tiles (16-byte chunk c of row q at
+            // (c ^ (q % 8)) * 16, as TMA's 128-byte swizzle lays them out), writes it to
+            // the operand buffer in the same layout and its NVFP4 block to aq (and m to
+            // m_out when set), then announces the stage (after a proxy fence: the tensor
+            // core reads shared memory through the async proxy)
+            const int t = threadIdx.x - 64, q = t & 127, b = t >> 7;
+            const int64_t row = row0 + q, rows_pad = ((int64_t)pr.row_end + 127) & ~int64_t(127);
+            const int64_t cols = p.aq.cols;
+            uint8_t *qcodes = static_cast<uint8_t *>(p.aq.codes), *qscales = static_cast<uint8_t *>(p.aq.scales);
+            auto silu8 = [](const uint4 &gw, const uint4 &uw) {
+                float gv[8], uv[8], sv[8], mv[8];
+                unpack8_bf16(gw, gv);
+                unpack8_bf16(uw, uv);
+#pragma unroll
+                for (int i = 0; i < 8; ++i) sv[i] = sigmoid_fast(gv[i]);
+                silu_mul8<false>(gv, uv, sv, mv);
+                return make_uint4(pack_bf16x2(mv[0], mv[1]), pack_bf16x2(mv[2], mv[3]), pack_bf16x2(mv[4], mv[5]),
+                                  pack_bf16x2(mv[6], mv[7]));
+            };
+            const uint32_t c0 = ((2 * b) ^ (q & 7)) << 4, c1 = ((2 * b + 1) ^ (q & 7)) << 4;
+            uint32_t stage = 0, phase = 0;
+            for (int kt = 0; kt < ktiles; ++kt) {
+                if (!(ok = warp_all(mbar_wait(&raw_full[stage], phase)))) {
+                    aborted = 1;
+                    break;
+                }
+                const int k = kb + kt * BK;
+                uint8_t *st = smem + stage * STAGE_BYTES;
+                const uint32_t ga = smem_u32(st + OPER_BYTES) + q * 128, ua = ga + A_BYTES, oa = smem_u32(st) + q * 128;
+                uint4 g0, g1, u0, u1;
+                asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                             : "=r"(g0.x), "=r"(g0.y), "=r"(g0.z), "=r"(g0.w) : "r"(ga + c0));
+                asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                             : "=r"(g1.x), "=r"(g1.y), "=r"(g1.z), "=r"(g1.w) : "r"(ga + c1));
+                asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                             : "=r"(u0.x), "=r"(u0.y), "=r"(u0.z), "=r"(u0.w) : "r"(ua + c0));
+                asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                             : "=r"(u1.x), "=r"(u1.y), "=r"(u1.z), "=r"(u1.w) : "r"(ua + c1));
+                const uint4 m0 = silu8(g0, u0), m1 = silu8(g1, u1);   // rows past the end: 0 (zero-filled g, u)
+                asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(oa + c0), "r"(m0.x), "r"(m0.y), "r"(m0.z),
+                             "r"(m0.w)
+                             : "memory");
+                asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(oa + c1), "r"(m1.x), "r"(m1.y), "r"(m1.z),
+                             "r"(m1.w)
+                             : "memory");
+                const int64_t c = k + 16 * b;
+                if (row < pr.row_end) {
+                    uint32_t lo, hi, sb;
+                    quant16_bf16(m0, m1, &lo, &hi, &sb);
+                    *reinterpret_cast<uint2 *>(qcodes + row * (cols >> 1) + (c >> 1)) = make_uint2(lo, hi);
+                    qscales[scale_offset(row, c >> 4, cols)] = (uint8_t)sb;
+                    if (p.m_out) {
+                        uint4 *mp = reinterpret_cast<uint4 *>(p.m_out + row * p.m_ld + c);
+                        mp[0] = m0;
+                        mp[1] = m1;
+                    }
+                } else if (row < rows_pad) {
+                    qscales[scale_offset(row, c >> 4, cols)] = 0;
+                }
                 fence_proxy_async_smem();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&full[stage]);
@@ -523,23 +613,27 @@ static void set_fp4_a(Params &p, const pact_nvfp4_t &t) {
     p.a_cols = t.cols;
 }
 
-template <bool A_MN, bool B_MN, bool A_FP4 = false>
+template <bool A_MN, bool B_MN, bool A_FP4 = false, bool A_SILU = false>
 static pact_status launch_mma(const CUtensorMap &ta, const CUtensorMap &tb, const Params &p, int row_tiles,
-                              cudaStream_t st, const char *what) {
+                              cudaStream_t st, const char *what, const CUtensorMap *tu = nullptr) {
     static bool done[64] = {false};
     const int d = current_device();
     const int np = p.b_split ? 2 : 1;
-    const int smem = smem_bytes(np, A_FP4, stages_for(np, A_FP4));
+    const int smem = smem_bytes(np, A_FP4, stages_for(np, A_FP4, A_SILU), A_SILU);
     if (d >= 0 && d < 64 && !done[d]) {
         int mx = 0;
-        for (int n = 1; n <= 2; ++n)
-            mx = mx > smem_bytes(n, A_FP4, stages_for(n, A_FP4)) ? mx : smem_bytes(n, A_FP4, stages_for(n, A_FP4));
-        cudaError_t e = cudaFuncSetAttribute(k_lora_mma<A_MN, B_MN, A_FP4>, cudaFuncAttributeMaxDynamicSharedMemorySize, mx);
+        for (int n = 1; n <= 2; ++n) {
+            const int b = smem_bytes(n, A_FP4, stages_for(n, A_FP4, A_SILU), A_SILU);
+            mx = mx > b ? mx : b;
+        }
+        cudaError_t e = cudaFuncSetAttribute(k_lora_mma<A_MN, B_MN, A_FP4, A_SILU>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, mx);
         if (e != cudaSuccess) return fail(PACT_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
         done[d] = true;
     }
     dim3 grid((unsigned)row_tiles, (unsigned)p.splits, (unsigned)p.nprob);
-    return launch_dep(k_lora_mma<A_MN, B_MN, A_FP4>, grid, dim3(THREADS), smem, st, what, ta, tb, p);
+    return launch_dep(k_lora_mma<A_MN, B_MN, A_FP4, A_SILU>, grid, dim3(threads_of(A_SILU)), smem, st, what, ta, tb,
+                      tu ? *tu : ta, p);
 }
 
 static FinJob fin_job(const float *ws, const Params &p, int64_t rows, int64_t cols, float scale, int mode,
@@ -693,6 +787,48 @@ pact_status pact_lora_fwd_quant(const pact_bf16 *x, int64_t ldx, int64_t M, int6
                                 size_t ws_bytes, pact_stream_t stream) {
     PACT_CHECK(xq, PACT_ERR_INVALID_ARG, "pact_lora_fwd_quant: NULL argument");
     return lora_fwd(x, ldx, M, K, A, R, scale, T, ldt, xq, workspace, ws_bytes, stream, "pact_lora_fwd_quant");
+}
+
+pact_status pact_lora_fwd_silu(const pact_bf16 *g, const pact_bf16 *u, int64_t ld_gu, int64_t M, int64_t I,
+                               const pact_bf16 *A, int R, float scale, pact_bf16 *T, int64_t ldt,
+                               const pact_nvfp4_t *mq, pact_bf16 *m, int64_t ldm, void *workspace, size_t ws_bytes,
+                               pact_stream_t stream) {
+    const char *what = "pact_lora_fwd_silu";
+    PACT_CHECK(g && u && A && T && mq && workspace, PACT_ERR_INVALID_ARG, "%s: NULL argument", what);
+    PACT_CHECK(M >= 1 && M <= 0x7FFFFFFF && I >= 64 && I % 64 == 0 && I <= 0x7FFFFFFF && R >= 16 && R <= 64 &&
+                   R % 16 == 0,
+               PACT_ERR_SHAPE, "%s: need M >= 1, I a multiple of 64, R in {16, 32, 48, 64}", what);
+    PACT_CHECK(ld_gu >= I && ld_gu % 8 == 0 && ldt >= 2 * R && ldt % 8 == 0 && (!m || (ldm >= I && ldm % 8 == 0)) &&
+                   aligned16(g) && aligned16(u) && aligned16(A) && aligned16(T) && aligned16(m) && aligned16(workspace),
+               PACT_ERR_ALIGN, "%s: pointers 16-byte aligned, leading dims %% 8 == 0", what);
+    PACT_CHECK(ws_bytes >= pact_lora_fwd_workspace_bytes(M, I, R), PACT_ERR_INVALID_ARG,
+               "%s: workspace too small (%zu < %zu)", what, ws_bytes, pact_lora_fwd_workspace_bytes(M, I, R));
+    pact_status s = check_nvfp4(mq, M, I, "mq");
+    if (s != PACT_OK) return s;
+    CUtensorMap tg, tu, tb;
+    s = map_bf16(&tg, g, I, M, ld_gu, 64, BM, what);
+    if (s == PACT_OK) s = map_bf16(&tu, u, I, M, ld_gu, 64, BM, what);
+    if (s == PACT_OK) s = map_bf16(&tb, A, I, R, I, 64, R, what);
+    if (s != PACT_OK) return s;
+    Params p = {};
+    p.n_mma = R;
+    p.n_valid = R;
+    p.nprob = 1;
+    p.prob[0] = Prob{0, (int)M, 0, (int)I, 0, 0};
+    const int tiles = (int)((M + BM - 1) / BM);
+    choose_split(I, tiles, FWD_PER_SM, &p.splits, &p.k_per_split);
+    float *ws = static_cast<float *>(workspace);
+    p.ws = ws;
+    p.ws_ld = R;
+    p.ws_split_stride = M * R;
+    set_direct_out(p, T, ldt, R, scale);
+    p.aq = *mq;
+    p.m_out = m;
+    p.m_ld = ldm;
+    cudaStream_t st = (cudaStream_t)stream;
+    s = launch_mma<false, false, false, true>(tg, tb, p, tiles, st, what, &tu);
+    if (s != PACT_OK || p.out) return s;
+    return finalize(fin_job(ws, p, M, R, scale, 0, T, ldt, R), nullptr, st, what);
 }
 
 int pact_lora_fwd_launches(int64_t M, int64_t K, int R) {

@@ -124,7 +124,10 @@ class PactLayer:
         self.xq2, self.x2, self.rstd2 = nv(M, H), bf(M, H), torch.empty(M, dtype=torch.float32, device=dev)
         self.t_gu = bf(M, 2 * 2 * r)
         self.gu = None if self.fuse_silu else bf(M, 2 * I)
-        self.m, self.mq, self.gq, self.uq = bf(M, I), nv(M, I), nv(M, I), nv(M, I)
+        # m itself (BF16) exists only with the fused SiLU GEMM; the default path takes
+        # mq and the down projection's T straight from gate|up (pact_lora_fwd_silu)
+        self.m = bf(M, I) if self.fuse_silu else None
+        self.mq, self.gq, self.uq = nv(M, I), nv(M, I), nv(M, I)
         self.t_d, self.out = bf(M, 2 * r), bf(M, H)
         # backward
         self.u_d, self.doq, self.dm = bf(M, 2 * r), nv(M, H), bf(M, I)
@@ -211,29 +214,33 @@ class PactLayer:
                bytes=2 * M * H + 2 * H + S.nv(M, H) + 2 * M * H + 4 * M),
             Op("lora_fwd_gu", lambda: P.pact_lora_fwd(self.x2, self.a_gu, self.sc["gu"], self.t_gu, self.ws),
                kernels=nk(H, 2 * r), bytes=lora_fwd(H, 2 * r)),
-            *self._gate_up_ops(gemm, gbytes),
-            Op("lora_fwd_down", lambda: P.pact_lora_fwd(self.m, self.a_d, self.sc["d"], self.t_d, self.ws),
-               kernels=nk(I, r), bytes=lora_fwd(I, r)),
+            *self._gate_up_ops(gemm, gbytes, nk),
             Op("gemm_fwd_down", lambda: P.pact_frozen_gemm_fwd(self.mq, self.c_d, self.l_d_f, residual=self.h2,
                                                                y=self.out),
                "gemm", gemm(S.M, S.H, I), bytes=gbytes(H, I, r) + 2 * M * H),
         ]
 
-    def _gate_up_ops(self, gemm, gbytes) -> List[Op]:
+    def _gate_up_ops(self, gemm, gbytes, nk) -> List[Op]:
         S, M, H, I, r = self.s, self.s.M, self.s.H, self.s.I, self.s.r
+        lora_fwd_d = 2 * r * I + 2 * M * 2 * r   # A_down in, T_down (hi|lo) out
         if self.fuse_silu:
             # one kernel: g|u stays on chip; m, mq and the saved copies gq, uq are written
             return [Op("gemm_fwd_silu", lambda: P.pact_frozen_gemm_fwd_silu(self.xq2, self.c_gu, self.m, self.mq,
                                                                             self.gq, self.uq, self.l_gu_f),
                        "gemm", gemm(S.M, 2 * I, S.H),
-                       bytes=gbytes(2 * I, H, 2 * r) - 2 * M * 2 * I + 2 * M * I + 3 * S.nv(M, I))]
-        # the gate|up GEMM also writes the NVFP4 copies gq, uq kept for the backward
+                       bytes=gbytes(2 * I, H, 2 * r) - 2 * M * 2 * I + 2 * M * I + 3 * S.nv(M, I)),
+                    Op("lora_fwd_down", lambda: P.pact_lora_fwd(self.m, self.a_d, self.sc["d"], self.t_d, self.ws),
+                       kernels=nk(I, r), bytes=2 * M * I + lora_fwd_d)]
+        # the gate|up GEMM also writes the NVFP4 copies gq, uq kept for the backward; one
+        # kernel then forms m = silu(g) u from gate|up, writes mq and the down
+        # projection's T (m itself never goes to memory)
         return [Op("gemm_fwd_gu", lambda: P.pact_frozen_gemm_fwd_quant(self.xq2, self.c_gu, [self.gq, self.uq],
                                                                        self.l_gu_f, y=self.gu),
                    "gemm", gemm(S.M, 2 * I, S.H), bytes=gbytes(2 * I, H, 2 * r) + 2 * S.nv(M, I)),
-                Op("silu_mul_quant", lambda: P.pact_silu_mul_quant(self.gu[:, :I], self.gu[:, I:], self.m, self.mq,
-                                                                   want_copies=False),
-                   bytes=4 * M * I + 2 * M * I + S.nv(M, I))]
+                Op("silu_mul_quant+lora_fwd_down", lambda: P.pact_lora_fwd_silu(self.gu[:, :I], self.gu[:, I:], self.a_d,
+                                                                                self.sc["d"], self.mq, self.t_d,
+                                                                                workspace=self.ws),
+                   kernels=nk(I, r), bytes=4 * M * I + S.nv(M, I) + lora_fwd_d)]
 
     def backward_ops(self) -> List[Op]:
         S, s, r = self.s, self.s.scale, self.s.r

@@ -84,6 +84,7 @@ def _load() -> ctypes.CDLL:
         "pact_lora_fwd": (S, [P, I64, I64, I64, P, I, F, P, I64, P, ctypes.c_size_t, P]),
         "pact_lora_fwd_quant": (S, [P, I64, I64, I64, P, I, F, P, I64, NV, P, ctypes.c_size_t, P]),
         "pact_lora_fwd_launches": (I, [I64, I64, I]),
+        "pact_lora_fwd_silu": (S, [P, P, I64, I64, I64, P, I, F, P, I64, NV, P, I64, P, ctypes.c_size_t, P]),
         "pact_lora_fwd_noalloc": (S, [P, I64, I64, I64, P, I, F, P, I64, P]),
         "pact_lora_bwd_u_workspace_bytes": (ctypes.c_size_t, [I64, I64, I, I]),
         "pact_lora_bwd_u": (S, [P, I64, I64, I64, P, I, I, ctypes.POINTER(I64), F, P, I64, P, ctypes.c_size_t, P]),
@@ -423,6 +424,28 @@ def pact_lora_fwd(x: torch.Tensor, A: torch.Tensor, scale: float, T: Optional[to
         sq = xq.c()
         _check(_lib.pact_lora_fwd_quant(x.data_ptr(), _ld(x), M, K, A.data_ptr(), R, float(scale), T.data_ptr(),
                                         _ld(T), ctypes.byref(sq), ws.data_ptr(), ws.numel(), _stream(stream)))
+    return T
+
+
+def pact_lora_fwd_silu(g: torch.Tensor, u: torch.Tensor, A: torch.Tensor, scale: float, mq: NVFP4Tensor,
+                       T: Optional[torch.Tensor] = None, m: Optional[torch.Tensor] = None,
+                       workspace: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """T = scale m A^T and mq = q(m) for m = silu(g) u, in one kernel; m itself is
+    written only into a given `m`."""
+    _bf16(g, "g")
+    _bf16(u, "u")
+    _bf16(A, "A")
+    if _ld(g) != _ld(u):
+        raise ValueError("g and u must share a row stride")
+    M, I = g.shape
+    R = A.shape[0]
+    if T is None:
+        T = torch.empty((M, 2 * R), dtype=torch.bfloat16, device=g.device)
+    ws = _workspace(workspace, pact_lora_fwd_workspace_bytes(M, I, R), g.device)
+    sq = mq.c()
+    _check(_lib.pact_lora_fwd_silu(g.data_ptr(), u.data_ptr(), _ld(g), M, I, A.data_ptr(), R, float(scale),
+                                   T.data_ptr(), _ld(T), ctypes.byref(sq), _ptr(m), _ld(m) if m is not None else 0,
+                                   ws.data_ptr(), ws.numel(), _stream(stream)))
     return T
 
 

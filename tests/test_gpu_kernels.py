@@ -525,6 +525,28 @@ def test_silu_mul_quant(P, orc, guards, M, I, std):
     assert_nvfp4_equal(uq, uq_ref, orc, "uq")
 
 
+# m = silu(g) u formed inside the down projection's LoRA kernel: m (when asked), q(m) and
+# T = s m A^T, split (small M) and unsplit (>= 148 row blocks), |g| > 16 included (std 9)
+@pytest.mark.parametrize("M,I,R,std", [(130, 512, 16, 2.0), (257, 1024, 32, 9.0), (19000, 128, 16, 2.0)])
+def test_lora_fwd_silu(P, orc, guards, M, I, R, std):
+    gu = synth.gaussian_bf16(4, (M, 2 * I), std=std)
+    a = synth.gaussian_bf16(20, (R, I), std=0.02)
+    gud, ad = to_dev(gu), to_dev(a)
+    mq, m = guards.nvfp4(M, I), guards.matrix(M, I)
+    T = P.pact_lora_fwd_silu(gud[:, :I], gud[:, I:], ad, 2.0, mq, T=guards.matrix(M, 2 * R, pad_cols=8), m=m)
+    mq2 = P.NVFP4Tensor.empty(M, I)
+    T2 = P.pact_lora_fwd_silu(gud[:, :I], gud[:, I:], ad, 2.0, mq2)   # without m: the same mq and T
+    sync()
+    m_ref, mq_ref, _, _ = orc.silu_mul_quant(gu[:, :I], gu[:, I:])
+    mb = to_bits(m)
+    assert np.array_equal(mb, m_ref), f"m differs at {np.argwhere(mb != m_ref)[:3].tolist()}"
+    assert_nvfp4_equal(mq, mq_ref, orc, "mq")
+    assert_nvfp4_equal(mq2, mq_ref, orc, "mq (no m)")
+    assert torch.equal(T.contiguous().view(torch.int16), T2.view(torch.int16))
+    t_dev = to_f64(T[:, :R]) + to_f64(T[:, R:])
+    assert_close(t_dev, 2.0 * orc.gemm_nt(synth.bf16_bits_to_f64(m_ref), synth.bf16_bits_to_f64(a)), "T")
+
+
 @pytest.mark.parametrize("M,I,std", [(64, 512, 2.0), (130, 2048, 2.0), (96, 1024, 9.0)])
 def test_silu_mul_bwd_quant(P, orc, guards, M, I, std):
     gu = synth.gaussian_bf16(4, (M, 2 * I), std=std)
