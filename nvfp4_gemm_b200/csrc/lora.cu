@@ -372,22 +372,27 @@ k_lora_mma(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUte
                 const int k = kb + kt * BK;
                 uint8_t *st = smem + stage * STAGE_BYTES;
                 const uint32_t ga = smem_u32(st + OPER_BYTES) + q * 128, ua = ga + A_BYTES, oa = smem_u32(st) + q * 128;
-                uint4 g0, g1, u0, u1;
+                // the two 8-value halves through one copy of the SiLU code (the kernel's
+                // roles compete for the instruction cache), then the block back from the
+                // operand buffer for its quantization
+#pragma unroll 1
+                for (int h = 0; h < 2; ++h) {
+                    const uint32_t c = h ? c1 : c0;
+                    uint4 gw, uw;
+                    asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                                 : "=r"(gw.x), "=r"(gw.y), "=r"(gw.z), "=r"(gw.w) : "r"(ga + c));
+                    asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                                 : "=r"(uw.x), "=r"(uw.y), "=r"(uw.z), "=r"(uw.w) : "r"(ua + c));
+                    const uint4 mw = silu8(gw, uw);   // rows past the end: 0 (zero-filled g, u)
+                    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(oa + c), "r"(mw.x), "r"(mw.y),
+                                 "r"(mw.z), "r"(mw.w)
+                                 : "memory");
+                }
+                uint4 m0, m1;
                 asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
-                             : "=r"(g0.x), "=r"(g0.y), "=r"(g0.z), "=r"(g0.w) : "r"(ga + c0));
+                             : "=r"(m0.x), "=r"(m0.y), "=r"(m0.z), "=r"(m0.w) : "r"(oa + c0) : "memory");
                 asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
-                             : "=r"(g1.x), "=r"(g1.y), "=r"(g1.z), "=r"(g1.w) : "r"(ga + c1));
-                asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
-                             : "=r"(u0.x), "=r"(u0.y), "=r"(u0.z), "=r"(u0.w) : "r"(ua + c0));
-                asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
-                             : "=r"(u1.x), "=r"(u1.y), "=r"(u1.z), "=r"(u1.w) : "r"(ua + c1));
-                const uint4 m0 = silu8(g0, u0), m1 = silu8(g1, u1);   // rows past the end: 0 (zero-filled g, u)
-                asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(oa + c0), "r"(m0.x), "r"(m0.y), "r"(m0.z),
-                             "r"(m0.w)
-                             : "memory");
-                asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(oa + c1), "r"(m1.x), "r"(m1.y), "r"(m1.z),
-                             "r"(m1.w)
-                             : "memory");
+                             : "=r"(m1.x), "=r"(m1.y), "=r"(m1.z), "=r"(m1.w) : "r"(oa + c1) : "memory");
                 const int64_t c = k + 16 * b;
                 if (row < pr.row_end) {
                     uint32_t lo, hi, sb;
