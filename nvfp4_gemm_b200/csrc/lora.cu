@@ -524,7 +524,11 @@ k_lora_mma(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUte
 //   mode 2: BF16 transposed (out[col * ldo + row])
 //   mode 3, 4: as modes 1, 2 in FP32 (out32)
 // The partials are summed in split order (deterministic).  One launch serves one or
-// two such jobs (the index space of the second follows the first's).
+// two such jobs (the index space of the second follows the first's).  A job with
+// `vec` set (modes 0, 1, 3; every stride a multiple of 4 elements, the pointers
+// aligned for it) takes 4 consecutive columns per thread: one 16-byte load per
+// partial, one 8-byte (BF16) or 16-byte (FP32) store per output; the sums are the
+// same, element by element.
 struct FinJob {
     const float *ws;
     int splits;
@@ -534,16 +538,44 @@ struct FinJob {
     pact_bf16 *out;
     int64_t ldo, lo_off;
     float *out32;
+    int vec;
 };
+
+__device__ __forceinline__ int64_t fin_items(const FinJob &j) { return j.rows * (j.vec ? j.cols / 4 : j.cols); }
 
 __global__ void k_finalize(const FinJob j0, const FinJob j1, int njobs) {
     pdl_wait();
-    const int64_t n0 = j0.rows * j0.cols;
-    const int64_t n = n0 + (njobs > 1 ? j1.rows * j1.cols : 0);
+    const int64_t n0 = fin_items(j0);
+    const int64_t n = n0 + (njobs > 1 ? fin_items(j1) : 0);
     for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x) {
         const bool second = i >= n0;
         const FinJob &j = second ? j1 : j0;
         const int64_t ii = second ? i - n0 : i;
+        if (j.vec) {
+            const int64_t c4 = j.cols / 4, r = ii / c4, c = (ii % c4) * 4;
+            float a[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+            for (int s = 0; s < j.splits; ++s) {
+                const float4 v = *reinterpret_cast<const float4 *>(j.ws + s * j.split_stride + r * j.ws_ld + c);
+                a[0] += v.x;
+                a[1] += v.y;
+                a[2] += v.z;
+                a[3] += v.w;
+            }
+#pragma unroll
+            for (int e = 0; e < 4; ++e) a[e] *= j.scale;
+            if (j.mode == 3) {
+                *reinterpret_cast<float4 *>(j.out32 + r * j.ldo + c) = make_float4(a[0], a[1], a[2], a[3]);
+                continue;
+            }
+            const uint32_t h0 = pack_bf16x2(a[0], a[1]), h1 = pack_bf16x2(a[2], a[3]);
+            *reinterpret_cast<uint2 *>(j.out + r * j.ldo + c) = make_uint2(h0, h1);
+            if (j.mode == 0) {
+                const uint32_t l0 = pack_bf16x2(a[0] - bf16lo(h0), a[1] - bf16hi(h0));
+                const uint32_t l1 = pack_bf16x2(a[2] - bf16lo(h1), a[3] - bf16hi(h1));
+                *reinterpret_cast<uint2 *>(j.out + r * j.ldo + c + j.lo_off) = make_uint2(l0, l1);
+            }
+            continue;
+        }
         const bool tr = j.mode == 2 || j.mode == 4;
         const int64_t r = tr ? ii % j.rows : ii / j.cols, c = tr ? ii / j.rows : ii % j.cols;
         float acc = 0.0f;
@@ -643,9 +675,16 @@ static pact_status launch_mma(const CUtensorMap &ta, const CUtensorMap &tb, cons
 
 static FinJob fin_job(const float *ws, const Params &p, int64_t rows, int64_t cols, float scale, int mode,
                       void *out, int64_t ldo, int64_t lo_off) {
+    // 4 columns per thread where every stride is a multiple of 4 elements and the
+    // pointers are aligned for 16-byte partial loads and 8-byte (BF16) or 16-byte
+    // (FP32) output stores
+    const uintptr_t oa = reinterpret_cast<uintptr_t>(out);
+    const int vec = (mode == 0 || mode == 1 || mode == 3) && cols % 4 == 0 && p.ws_ld % 4 == 0 &&
+                    p.ws_split_stride % 4 == 0 && ldo % 4 == 0 && lo_off % 4 == 0 &&
+                    (reinterpret_cast<uintptr_t>(ws) & 15) == 0 && (oa & (mode == 3 ? 15 : 7)) == 0;
     return FinJob{ws, p.splits, p.ws_split_stride, p.ws_ld, rows, cols, scale, mode,
                   mode >= 3 ? nullptr : static_cast<pact_bf16 *>(out), ldo, lo_off,
-                  mode >= 3 ? static_cast<float *>(out) : nullptr};
+                  mode >= 3 ? static_cast<float *>(out) : nullptr, vec};
 }
 
 // A product with one split writes its hi + lo output from the epilogue (mode 0 of
@@ -659,7 +698,8 @@ static void set_direct_out(Params &p, pact_bf16 *out, int64_t ldo, int64_t lo_of
 }
 
 static pact_status finalize(const FinJob &j0, const FinJob *j1, cudaStream_t st, const char *what) {
-    const int64_t n = j0.rows * j0.cols + (j1 ? j1->rows * j1->cols : 0);
+    auto items = [](const FinJob &j) { return j.rows * (j.vec ? j.cols / 4 : j.cols); };   // as fin_items
+    const int64_t n = items(j0) + (j1 ? items(*j1) : 0);
     return launch_dep(k_finalize, dim3(finalize_grid(n)), dim3(256), 0, st, what, j0, j1 ? *j1 : j0, j1 ? 2 : 1);
 }
 
