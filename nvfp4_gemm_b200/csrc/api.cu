@@ -39,15 +39,15 @@ int current_device() {
 }
 
 int sm_count() {
-    static int cache[64] = {0};
+    static std::atomic<int> cache[64];   // 0: not looked up yet (host threads may race to fill it)
     const int d = current_device();
     if (d < 0 || d >= 64) return 148;
-    if (cache[d] == 0) {
-        int n = 0;
+    int n = cache[d].load(std::memory_order_relaxed);
+    if (n == 0) {
         if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, d) != cudaSuccess || n <= 0) n = 148;
-        cache[d] = n;
+        cache[d].store(n, std::memory_order_relaxed);
     }
-    return cache[d];
+    return n;
 }
 
 pact_status check_nvfp4(const pact_nvfp4_t *t, int64_t rows, int64_t cols, const char *name) {

@@ -5,6 +5,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <atomic>
+
 #include "../../include/pact.h"
 
 #if defined(__CUDA_ARCH__) && (__CUDA_ARCH__ < 1000)

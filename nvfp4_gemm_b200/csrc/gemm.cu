@@ -643,15 +643,16 @@ typedef CUresult (*EncodeTiled)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, 
                                 CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 
 static EncodeTiled encode_fn() {
-    static EncodeTiled fn = nullptr;
-    if (!fn) {
+    // looked up once (a function-local static's initialisation is thread-safe)
+    static const EncodeTiled fn = [] {
         void *p = nullptr;
         cudaDriverEntryPointQueryResult q;
         if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault, &q) ==
                 cudaSuccess &&
             q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<EncodeTiled>(p);
-    }
+            return reinterpret_cast<EncodeTiled>(p);
+        return static_cast<EncodeTiled>(nullptr);
+    }();
     return fn;
 }
 
@@ -673,15 +674,15 @@ static pact_status make_map(CUtensorMap *m, CUtensorMapDataType dt, const void *
 }
 
 static pact_status ensure_attrs() {
-    static bool done[64] = {false};
+    static std::atomic<bool> done[64];   // per device; setting the attribute twice is harmless
     const int d = current_device();
-    if (d >= 0 && d < 64 && done[d]) return PACT_OK;
+    if (d >= 0 && d < 64 && done[d].load(std::memory_order_acquire)) return PACT_OK;
     cudaError_t e =
         cudaFuncSetAttribute(k_nvfp4_gemm<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, Layout<false>::SMEM_BYTES);
     if (e == cudaSuccess)
         e = cudaFuncSetAttribute(k_nvfp4_gemm<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, Layout<true>::SMEM_BYTES);
     if (e != cudaSuccess) return fail(PACT_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));
-    if (d >= 0 && d < 64) done[d] = true;
+    if (d >= 0 && d < 64) done[d].store(true, std::memory_order_release);
     return PACT_OK;
 }
 

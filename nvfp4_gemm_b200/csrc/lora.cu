@@ -608,15 +608,16 @@ typedef CUresult (*EncodeTiled)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, 
 static pact_status map_2d(CUtensorMap *m, CUtensorMapDataType dt, int esize, CUtensorMapSwizzle sw, const void *base,
                           uint64_t inner, uint64_t outer, uint64_t ld, uint32_t box_inner, uint32_t box_outer,
                           const char *what) {
-    static EncodeTiled enc = nullptr;
-    if (!enc) {
+    // looked up once (a function-local static's initialisation is thread-safe)
+    static const EncodeTiled enc = [] {
         void *fp = nullptr;
         cudaDriverEntryPointQueryResult q;
         if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &fp, 12000, cudaEnableDefault, &q) ==
                 cudaSuccess &&
             q == cudaDriverEntryPointSuccess)
-            enc = reinterpret_cast<EncodeTiled>(fp);
-    }
+            return reinterpret_cast<EncodeTiled>(fp);
+        return static_cast<EncodeTiled>(nullptr);
+    }();
     if (!enc) return fail(PACT_ERR_CUDA, "%s: cuTensorMapEncodeTiled unavailable", what);
     const cuuint64_t dims[2] = {inner, outer};
     const cuuint64_t strides[1] = {ld * (uint64_t)esize};
@@ -653,11 +654,11 @@ static void set_fp4_a(Params &p, const pact_nvfp4_t &t) {
 template <bool A_MN, bool B_MN, bool A_FP4 = false, bool A_SILU = false>
 static pact_status launch_mma(const CUtensorMap &ta, const CUtensorMap &tb, const Params &p, int row_tiles,
                               cudaStream_t st, const char *what, const CUtensorMap *tu = nullptr) {
-    static bool done[64] = {false};
+    static std::atomic<bool> done[64];   // per device; setting the attribute twice is harmless
     const int d = current_device();
     const int np = p.b_split ? 2 : 1;
     const int smem = smem_bytes(np, A_FP4, stages_for(np, A_FP4, A_SILU), A_SILU);
-    if (d >= 0 && d < 64 && !done[d]) {
+    if (d >= 0 && d < 64 && !done[d].load(std::memory_order_acquire)) {
         int mx = 0;
         for (int n = 1; n <= 2; ++n) {
             const int b = smem_bytes(n, A_FP4, stages_for(n, A_FP4, A_SILU), A_SILU);
@@ -666,7 +667,7 @@ static pact_status launch_mma(const CUtensorMap &ta, const CUtensorMap &tb, cons
         cudaError_t e = cudaFuncSetAttribute(k_lora_mma<A_MN, B_MN, A_FP4, A_SILU>,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize, mx);
         if (e != cudaSuccess) return fail(PACT_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
-        done[d] = true;
+        done[d].store(true, std::memory_order_release);
     }
     dim3 grid((unsigned)row_tiles, (unsigned)p.splits, (unsigned)p.nprob);
     return launch_dep(k_lora_mma<A_MN, B_MN, A_FP4, A_SILU>, grid, dim3(threads_of(A_SILU)), smem, st, what, ta, tb,

@@ -1021,14 +1021,14 @@ pact_status pact_rmsnorm_quant(const pact_bf16 *x, int64_t ldx, const pact_bf16 
     const int64_t rows_pad = (M + 127) / 128 * 128;
     PACT_CHECK(rows_pad <= 0x7FFFFFFF, PACT_ERR_SHAPE, "pact_rmsnorm_quant: M too large");
     const Ring r = ring_for(rows_pad, (size_t)H * 2, (size_t)H * 2);
-    static bool attr_done[64] = {false};
+    static std::atomic<bool> attr_done[64];   // per device; setting the attribute twice is harmless
     const int d = current_device();
-    if (d >= 0 && d < 64 && !attr_done[d]) {
+    if (d >= 0 && d < 64 && !attr_done[d].load(std::memory_order_acquire)) {
         cudaError_t e = cudaFuncSetAttribute(k_rmsnorm_quant<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
         if (e == cudaSuccess)
             e = cudaFuncSetAttribute(k_rmsnorm_quant<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
         if (e != cudaSuccess) return fail(PACT_ERR_CUDA, "pact_rmsnorm_quant: %s", cudaGetErrorString(e));
-        attr_done[d] = true;
+        attr_done[d].store(true, std::memory_order_release);
     }
     return launch_dep(eps == 0.0f ? k_rmsnorm_quant<true> : k_rmsnorm_quant<false>, dim3(r.grid), dim3(RING_THREADS),
                       r.smem, (cudaStream_t)stream,
@@ -1103,12 +1103,12 @@ pact_status pact_rmsnorm_bwd(const pact_bf16 *dy, int64_t lddy, const pact_nvfp4
     }
     const BwdSlot sl = bwd_slot(H);
     const Ring r = ring_for(rows, (size_t)(dres ? sl.dres_off + H * 2 : sl.codes_off + H / 2), (size_t)H * 2);
-    static bool attr_done[64] = {false};
+    static std::atomic<bool> attr_done[64];   // per device; setting the attribute twice is harmless
     const int d = current_device();
-    if (d >= 0 && d < 64 && !attr_done[d]) {
+    if (d >= 0 && d < 64 && !attr_done[d].load(std::memory_order_acquire)) {
         const cudaError_t e = cudaFuncSetAttribute(k_rmsnorm_bwd, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
         if (e != cudaSuccess) return fail(PACT_ERR_CUDA, "pact_rmsnorm_bwd: %s", cudaGetErrorString(e));
-        attr_done[d] = true;
+        attr_done[d].store(true, std::memory_order_release);
     }
     return launch_dep(k_rmsnorm_bwd, dim3(r.grid), dim3(RING_THREADS), r.smem, (cudaStream_t)stream, "pact_rmsnorm_bwd",
                       dy, lddy, *yq, rstd, gamma, M, H, dres, dx, dxq ? *dxq : none, (int)(dxq != nullptr), r.stages,
