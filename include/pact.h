@@ -278,7 +278,9 @@ PACT_API pact_status pact_lora_fwd_quant(const pact_bf16 *x, int64_t ldx, int64_
  * stride ld_gu (the halves of the gate|up output).  m itself is written only when m
  * is not NULL (row stride ldm): the data flow needs mq and T, and skipping m saves
  * its write and its read by the LoRA product.  workspace as for pact_lora_fwd(M, I,
- * R).  Outputs must not overlap the inputs or the workspace. */
+ * R).  Outputs must not overlap the inputs or the workspace.  PACT_ERR_SHAPE unless
+ * M >= 1, I is a multiple of 64 and R is 16, 32, 48 or 64; PACT_ERR_ALIGN unless the
+ * pointers are 16-byte aligned and the row strides multiples of 8 elements. */
 PACT_API pact_status pact_lora_fwd_silu(const pact_bf16 *g, const pact_bf16 *u, int64_t ld_gu, int64_t M,
                                         int64_t I, const pact_bf16 *A, int R, float scale, pact_bf16 *T,
                                         int64_t ldt, const pact_nvfp4_t *mq, pact_bf16 *m, int64_t ldm,
