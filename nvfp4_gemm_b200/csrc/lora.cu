@@ -31,6 +31,11 @@ constexpr int THREADS = 192;
 // the operand buffer (writing q(m) on the way) before the MMA reads it.
 constexpr int SILU_WARPS = 16;
 __host__ __device__ constexpr int threads_of(bool silu) { return silu ? 64 + 32 * SILU_WARPS : THREADS; }
+// K-major BF16 A with its NVFP4 copy written (Params::aq): eight quantizing warps
+// (2-9), two of each operand row's four 16-value blocks per thread
+constexpr int QUANT_WARPS = 8;
+constexpr int QUANT_THREADS = 64 + 32 * QUANT_WARPS;
+__host__ __device__ constexpr int max_threads_of(bool silu) { return silu ? threads_of(true) : QUANT_THREADS; }
 constexpr int A_BYTES = BM * BK * 2;     // 16384
 constexpr int B_BYTES = 64 * BK * 2;     // 8192 per B part
 // NVFP4 A operand: per stage, the codes of the A tile (128 x 64 values, 4 KiB) and
@@ -162,7 +167,7 @@ __device__ __forceinline__ void decode_stage(const uint8_t *raw, uint8_t *oper, 
 }
 
 template <bool A_MN, bool B_MN, bool A_FP4, bool A_SILU = false>
-__global__ void __launch_bounds__(threads_of(A_SILU), 1)
+__global__ void __launch_bounds__(max_threads_of(A_SILU), 1)
 k_lora_mma(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
            const __grid_constant__ CUtensorMap tmU, const Params p) {
     // tmU: the u tiles of an A_SILU kernel (tmA then maps g); unused otherwise
@@ -202,7 +207,7 @@ k_lora_mma(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUte
             // A_FP4: the producer's arrival (B bytes) and the four decoding warps'
             mbar_init(&full[s], A_SILU ? 1 + SILU_WARPS : A_FP4 ? 5 : 1);
             // the MMA warp's commit and, when they quantize A, the four epilogue warps'
-            mbar_init(&empty[s], quantize_a ? 5 : 1);
+            mbar_init(&empty[s], quantize_a ? 1 + QUANT_WARPS : 1);
             mbar_init(&raw_full[s], 1);
         }
         mbar_init(acc_full, 1);
@@ -412,11 +417,12 @@ k_lora_mma(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUte
                 if (lane == 0) mbar_arrive(&full[stage]);
                 if (++stage == STAGES) { stage = 0; phase ^= 1; }
             }
-        } else if (quantize_a && warp < 6) {
-            // the NVFP4 copy of A: thread q quantizes operand row q of each stage (64
-            // values, four 16-value blocks) from the swizzled tile (16-byte chunk c of row
-            // q at (c ^ (q % 8)) * 16), then releases the stage with the MMA's commit
-            const int q = threadIdx.x - 64;
+        } else if (quantize_a && warp < 2 + QUANT_WARPS) {
+            // the NVFP4 copy of A: thread t quantizes blocks 2h, 2h + 1 (h = t / 128) of
+            // operand row q = t % 128 of each stage (32 of its 64 values) from the
+            // swizzled tile (16-byte chunk c of row q at (c ^ (q % 8)) * 16), then releases
+            // the stage with the MMA's commit
+            const int t = threadIdx.x - 64, q = t & 127, h = t >> 7;
             const int64_t row = row0 + q, rows_pad = ((int64_t)pr.row_end + 127) & ~int64_t(127);
             const int64_t cols = p.aq.cols;
             uint8_t *qcodes = static_cast<uint8_t *>(p.aq.codes), *qscales = static_cast<uint8_t *>(p.aq.scales);
@@ -428,10 +434,14 @@ k_lora_mma(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUte
                 }
                 const int k = kb + kt * BK;
                 const uint32_t a = smem_u32(smem + stage * STAGE_BYTES) + q * 128;
+                // blocks k/16 .. k/16 + 3 (k a multiple of 64) are one word of the scale
+                // layout: this thread's two are its half h
+                uint16_t *sp = reinterpret_cast<uint16_t *>(qscales + scale_offset(row, k >> 4, cols)) + h;
                 if (row < pr.row_end) {
-                    uint32_t cw[8], sw = 0;
+                    uint32_t cw[4], sw = 0;
 #pragma unroll
-                    for (int b = 0; b < 4; ++b) {
+                    for (int bb = 0; bb < 2; ++bb) {
+                        const int b = 2 * h + bb;
                         uint4 wa, wb;
                         asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
                                      : "=r"(wa.x), "=r"(wa.y), "=r"(wa.z), "=r"(wa.w)
@@ -440,16 +450,14 @@ k_lora_mma(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUte
                                      : "=r"(wb.x), "=r"(wb.y), "=r"(wb.z), "=r"(wb.w)
                                      : "r"(a + (((2 * b + 1) ^ (q & 7)) << 4)));
                         uint32_t sb;
-                        quant16_bf16(wa, wb, &cw[2 * b], &cw[2 * b + 1], &sb);
-                        sw |= sb << (8 * b);
+                        quant16_bf16(wa, wb, &cw[2 * bb], &cw[2 * bb + 1], &sb);
+                        sw |= sb << (8 * bb);
                     }
-                    uint4 *cp = reinterpret_cast<uint4 *>(qcodes + row * (cols >> 1) + (k >> 1));
-                    cp[0] = make_uint4(cw[0], cw[1], cw[2], cw[3]);
-                    cp[1] = make_uint4(cw[4], cw[5], cw[6], cw[7]);
-                    // blocks k/16 .. k/16 + 3 (k a multiple of 64): one word of the layout
-                    *reinterpret_cast<uint32_t *>(qscales + scale_offset(row, k >> 4, cols)) = sw;
+                    *reinterpret_cast<uint4 *>(qcodes + row * (cols >> 1) + (k >> 1) + 16 * h) =
+                        make_uint4(cw[0], cw[1], cw[2], cw[3]);
+                    *sp = (uint16_t)sw;
                 } else if (row < rows_pad) {
-                    *reinterpret_cast<uint32_t *>(qscales + scale_offset(row, k >> 4, cols)) = 0u;
+                    *sp = 0;
                 }
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&empty[stage]);
@@ -670,7 +678,9 @@ static pact_status launch_mma(const CUtensorMap &ta, const CUtensorMap &tb, cons
         done[d].store(true, std::memory_order_release);
     }
     dim3 grid((unsigned)row_tiles, (unsigned)p.splits, (unsigned)p.nprob);
-    return launch_dep(k_lora_mma<A_MN, B_MN, A_FP4, A_SILU>, grid, dim3(threads_of(A_SILU)), smem, st, what, ta, tb,
+    const bool quant = !A_MN && !A_FP4 && !A_SILU && p.aq.codes != nullptr;   // the kernel's quantize_a
+    return launch_dep(k_lora_mma<A_MN, B_MN, A_FP4, A_SILU>, grid, dim3(quant ? QUANT_THREADS : threads_of(A_SILU)), smem,
+                      st, what, ta, tb,
                       tu ? *tu : ta, p);
 }
 
